@@ -1,0 +1,458 @@
+"""Benchmark: decoded bf16 weight throughput of the entropy-coded weight decoder on B200.
+
+Default workload (N = 1): the streamed 80-layer 70B-shape model -- every
+layer's seven matrices (q, o 8192x8192; k, v 1024x8192; gate, up 28672x8192;
+down 8192x28672) as Int8 symbols at ~2.1 bits/symbol, rANS-coded in 64 KiB
+chunks and resident in HBM (~17 GB), decoded block by block into a bf16
+ping-pong buffer pair (EntQuant technical summary, gist.science 2601.22787,
+section 2 "inference-time decoding").  Eight distinct seeded layers are
+encoded once and placed ten times at distinct HBM addresses; every layer is
+far larger than L2, so nothing is served from cache across layers.
+
+One "step" = one pass over all 80 blocks (decode + dequant + ping-pong
+events, no-op consumer).  The line also reports the same loop with the
+batch-1 bf16 GEMV consumer overlapped, the dominant kernel's roofline, the
+CPU oracle on the host cores, and an end-to-end number through the public
+API with the compressed weights copied from pinned host memory every step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {eqw,reference}]
+
+Multi-GPU (torchrun, one process per GPU): independent replicas, no
+collective on the data path (the decode does not shard any exchange);
+``value`` is the sum over ranks of decoded bytes divided by the slowest
+rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decoded bf16 weight GB/s per B200 (and Gsym/s); % of HBM roofline"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------
+# ranks (plumbing only: NCCL broadcast of the encoded blob, barrier, max/sum)
+# ---------------------------------------------------------------------------
+
+class Dist:
+    def __init__(self, backend: str | None = None):
+        import torch
+        import torch.distributed as dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.dist = dist if self.world > 1 else None
+        if self.dist is not None and not dist.is_initialized():
+            import datetime
+            backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+            if backend == "nccl":
+                torch.cuda.set_device(self.local_rank)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+        self.backend = dist.get_backend() if self.dist is not None else None
+
+    def _dev(self):
+        import torch
+        return torch.device("cuda", torch.cuda.current_device()) if self.backend == "nccl" else torch.device("cpu")
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def reduce(self, values: list[float], op: str) -> list[float]:
+        if self.dist is None:
+            return list(values)
+        import torch
+        t = torch.tensor(values, dtype=torch.float64, device=self._dev())
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX if op == "max" else self.dist.ReduceOp.SUM)
+        return t.cpu().tolist()
+
+    def broadcast_bytes(self, arr: np.ndarray | None) -> np.ndarray:
+        """Rank 0's uint8 array on every rank."""
+        if self.dist is None:
+            return arr
+        import torch
+        n = torch.tensor([arr.size if self.rank == 0 else 0], dtype=torch.int64, device=self._dev())
+        self.dist.broadcast(n, 0)
+        if self.rank == 0:
+            t = torch.from_numpy(arr).to(self._dev())
+        else:
+            t = torch.empty(int(n.item()), dtype=torch.uint8, device=self._dev())
+        self.dist.broadcast(t, 0)
+        return arr if self.rank == 0 else t.cpu().numpy()
+
+    def close(self):
+        if self.dist is not None and self.dist.is_initialized():
+            self.dist.destroy_process_group()
+
+
+def combine(local_ms: float, local_units: float, d: Dist) -> tuple[float, float]:
+    """(max over ranks of the timed milliseconds, sum over ranks of units)."""
+    ms = d.reduce([local_ms], "max")[0]
+    units = d.reduce([local_units], "sum")[0]
+    return ms, units
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        import torch
+        self.proc = None
+        self.lines: list[str] = []
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", uuid], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
+
+
+def measured_hbm_peak() -> tuple[float, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            return float(json.load(fh)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# workload: streamed 80-layer 70B-shape model
+# ---------------------------------------------------------------------------
+
+N_LAYERS = 80
+
+
+def build_blob(distinct: int, threads: int) -> tuple[np.ndarray, int, float]:
+    """Generate `distinct` seeded 70B-shape Int8 layers and encode them (host)."""
+    import entropy_coded_weight_b200 as E
+    import workloads as W
+    t0 = time.time()
+    mats = []
+    for layer in range(distinct):
+        mats += W.llama70b_int8_layer(layer, 2.1, threads=threads)
+    t1 = time.time()
+    blob = E.encode_host(mats, n_threads=threads)
+    n_syms = sum(m.n for m in mats)
+    del mats
+    print(f"[bench] generated {distinct} layers in {t1 - t0:.1f}s, encoded in {time.time() - t1:.1f}s "
+          f"({8.0 * blob.size / n_syms:.3f} bits/sym incl. metadata)", file=sys.stderr, flush=True)
+    return blob, n_syms, time.time() - t0
+
+
+class ResidentStack:
+    """`copies` device copies of an encoded `distinct`-layer blob = `n_layers` resident blocks."""
+
+    def __init__(self, blob: np.ndarray, distinct: int, device, n_layers: int = N_LAYERS):
+        import torch
+
+        import entropy_coded_weight_b200 as E
+        from entropy_coded_weight_b200.streamer import Step
+        self.copies = (n_layers + distinct - 1) // distinct
+        self.d_blobs = [E.upload(blob, device) for _ in range(self.copies)]
+        self.models = [E.Model(d, blob) for d in self.d_blobs]
+        self.steps = [Step(self.models[i // distinct], i % distinct) for i in range(n_layers)]
+        torch.cuda.synchronize(device)
+
+    def layer_bytes(self, step) -> dict:
+        """Algorithmic bytes of one block decode (read compressed + index + scales, write bf16)."""
+        m = step.model
+        comp = idx = sc = n = 0
+        for i in m.layer_matrices(step.layer):
+            inf = m.info(i)
+            comp += inf.compressed_bytes
+            idx += 8 * (inf.n_chunks + 1)
+            sc += 4 * inf.rows
+            n += inf.rows * inf.cols
+        return {"read": comp + idx + sc, "write": 2 * n, "symbols": n}
+
+    def close(self):
+        for m in self.models:
+            m.close()
+
+
+def run_pass(streamer, consumer=None, decode_events=None):
+    streamer.run(consumer, decode_events)
+
+
+def timed_passes(streamer, k: int, consumer=None, with_kernel_events: bool = True):
+    """Time k passes on the device: (elapsed ms, [per-launch decode ms])."""
+    import torch
+    dec_events = [] if with_kernel_events else None
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(streamer.consumer_stream)
+    streamer.decode_stream.wait_event(start)
+    for _ in range(k):
+        run_pass(streamer, consumer, dec_events)
+    streamer.consumer_stream.wait_stream(streamer.decode_stream)
+    end.record(streamer.consumer_stream)
+    torch.cuda.synchronize()
+    per = [a.elapsed_time(b) for a, b in dec_events] if dec_events is not None else []
+    return start.elapsed_time(end), per
+
+
+def cpu_oracle_sample(blob: np.ndarray, target_s: float = 12.0) -> dict:
+    """The CPU oracle (scalar rANS decode + dequant) on a bounded sample of chunks, all host cores."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    cores = len(os.sched_getaffinity(0))
+    parsed = oracle.parse_container(blob)
+    chunks = []
+    for mi, m in enumerate(parsed["matrices"]):
+        if m["layer"] != 0:
+            continue
+        for k in range(m["n_chunks"]):
+            chunks.append((mi, k))
+
+    def one(job):
+        mi, k = job
+        m = parsed["matrices"][mi]
+        n = m["rows"] * m["cols"]
+        cnt = min(oracle.CHUNK_SYMS, n - k * oracle.CHUNK_SYMS)
+        sym = oracle._decode_record(parsed["blob"], int(m["chunk_offsets"][k]), int(m["chunk_offsets"][k + 1]), cnt)
+        first = k * oracle.CHUNK_SYMS
+        rows = np.arange(first, first + cnt) // m["cols"]
+        oracle.dequant_pairs(m["dtype"], sym, m["scales"][rows])
+        return cnt
+
+    # calibrate on one chunk per core, then size the sample to ~target_s
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(cores) as ex:
+        done = sum(ex.map(one, chunks[:cores]))
+    dt = time.perf_counter() - t0
+    n_chunks = int(max(cores, cores * target_s / max(dt, 1e-3)))
+    sample = [chunks[(cores + i) % len(chunks)] for i in range(n_chunks)]
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(cores) as ex:
+        done = sum(ex.map(one, sample))
+    dt = time.perf_counter() - t0
+    return {"value": round(2.0 * done / dt / 1e9, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{len(sample)} chunks ({done} symbols) of layer 0, scalar rANS decode + dequant, "
+                      f"{cores} threads, {dt:.1f}s", "gsym_s": round(done / dt / 1e9, 5)}
+
+
+def bench_eqw(args, d: Dist) -> dict | None:
+    import torch
+
+    from entropy_coded_weight_b200.streamer import GemvConsumer, PingPongStreamer
+    import workloads as W
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    threads = len(os.sched_getaffinity(0))
+    blob = None
+    if d.rank == 0:
+        blob, _, _ = build_blob(args.distinct_layers, threads)
+    blob = d.broadcast_bytes(blob)
+    stack = ResidentStack(blob, args.distinct_layers, dev, args.layers)
+    streamer = PingPongStreamer(stack.steps, dev)
+    layer_bytes = [stack.layer_bytes(s) for s in stack.steps]
+    n_syms_pass = sum(b["symbols"] for b in layer_bytes)
+    dec_bytes_pass = 2.0 * n_syms_pass
+    alg_bytes_pass = sum(b["read"] + b["write"] for b in layer_bytes)
+
+    # ---- A: no-op consumer ----
+    for _ in range(args.warmup):
+        run_pass(streamer)
+    torch.cuda.synchronize()
+    if int(streamer.status.item()) != 0:
+        raise RuntimeError(f"decode status {int(streamer.status.item())}")
+    d.barrier()
+    clocks = ClockSampler(dev.index)
+    ms, per_launch = timed_passes(streamer, args.steps)
+    clk = clocks.stop()
+    d.barrier()
+    ms_max, dec_bytes_all = combine(ms, dec_bytes_pass * args.steps, d)
+    value = dec_bytes_all / (ms_max / 1e3) / 1e9
+    gsym = value / 2.0
+
+    # dominant kernel: one layer decode launch
+    launch_ms = statistics.mean(per_launch)
+    alg_per_launch = alg_bytes_pass / len(stack.steps)
+    peak, peak_kind = measured_hbm_peak()
+    achieved = alg_per_launch / (launch_ms / 1e3) / 1e9
+
+    # ---- B: GEMV consumer overlapped ----
+    xs, ys = [], []
+    for j, (rows, cols) in enumerate(W.LLAMA70B_BLOCK):
+        xs.append(W.gemv_activation(0, j, cols).to(dev))
+        ys.append(torch.empty(rows, dtype=torch.float32, device=dev))
+    gemv = GemvConsumer(xs, ys)
+    for _ in range(max(1, args.warmup)):
+        run_pass(streamer, gemv)
+    ms_b, _ = timed_passes(streamer, args.steps, gemv, with_kernel_events=False)
+    ms_b_max, _ = combine(ms_b, 0.0, d)
+    value_b = dec_bytes_all / (ms_b_max / 1e3) / 1e9
+
+    # ---- e2e: compressed weights copied from pinned host memory every step ----
+    pinned = torch.from_numpy(blob).pin_memory()
+    copy_stream = streamer.decode_stream
+    status_host = torch.zeros(1, dtype=torch.int32).pin_memory()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(copy_stream)
+    for _ in range(args.steps):
+        with torch.cuda.stream(copy_stream):
+            for db in stack.d_blobs:
+                db.copy_(pinned, non_blocking=True)
+        streamer.consumer_stream.wait_stream(copy_stream)
+        run_pass(streamer)
+        with torch.cuda.stream(streamer.consumer_stream):
+            status_host.copy_(streamer.status, non_blocking=True)
+        copy_stream.wait_stream(streamer.consumer_stream)
+    e1.record(copy_stream)
+    torch.cuda.synchronize()
+    ms_e = e0.elapsed_time(e1)
+    ms_e_max, _ = combine(ms_e, 0.0, d)
+    value_e = dec_bytes_all / (ms_e_max / 1e3) / 1e9
+    if int(status_host.item()) != 0 or int(streamer.status.item()) != 0:
+        raise RuntimeError("decode status nonzero after the e2e loop")
+
+    cpu = cpu_oracle_sample(blob) if (d.rank == 0 and d.world == 1 and not args.no_cpu_baseline) else None
+    stack.close()
+    if d.rank != 0:
+        return None
+    launches = len(stack.steps) * args.steps
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": d.world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u32 rANS state, f32 dequant -> bf16",
+        "data": "synthetic (seeded Laplace Int8 symbols at 2.1 bits; no checkpoint)",
+        "config": {"workload": f"streamed {args.layers}-layer Llama-70B-shape model, Int8 ~2.1 bits/sym, "
+                               f"{args.distinct_layers} distinct layers x {stack.copies} HBM copies, "
+                               "ping-pong bf16 buffers, no-op consumer",
+                   "layers": args.layers, "symbols_per_step": n_syms_pass,
+                   "l2": "inputs larger than L2 (each layer ~0.23 GB compressed, 1.7 GB decoded)",
+                   "parallelism": f"replicas x{d.world}"},
+        "gsym_s": round(gsym, 2),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "eq_rans_decode_dequant_kernel",
+                     "alg_bytes_per_launch": int(alg_per_launch), "launch_ms": round(launch_ms, 4)},
+        "with_gemv_consumer": {"value": round(value_b, 2), "unit": UNIT, "ms_per_step": round(ms_b_max / args.steps, 3),
+                               "loop_bytes_frac": round((alg_bytes_pass + dec_bytes_pass) * args.steps
+                                                        / (ms_b_max / 1e3) / 1e9 / peak, 4)},
+        "e2e": {"value": round(value_e, 2), "unit": UNIT, "h2d_bytes_per_step": int(blob.size * stack.copies),
+                "d2h_bytes_per_step": 4, "ms_per_step": round(ms_e_max / args.steps, 3)},
+        "cpu_baseline": cpu,
+        "clocks": clk,
+        "gpu_launches": launches,
+    }
+
+
+def bench_reference(args) -> dict:
+    """The CPU oracle, as it stands, on host cores: same metric and unit, bounded samples."""
+    import oracle
+    import workloads as W
+    mats = [W._int8_matrix(5, 0, 0, W.LLAMA70B_BLOCK[0], 2.1)]  # layer 0, q: 1024 chunks
+    blob = oracle.encode_container(mats)
+    res = []
+    for _ in range(args.warmup + args.steps):
+        res.append(cpu_oracle_sample(blob, target_s=max(2.0, 60.0 / max(1, args.warmup + args.steps))))
+    timed = res[args.warmup:]
+    v = statistics.mean(r["value"] for r in timed)
+    cpu = dict(timed[-1])
+    cpu["value"] = round(v, 4)
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": UNIT, "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "u32 rANS state, f32 dequant -> bf16",
+            "data": "synthetic (seeded Laplace Int8 symbols at 2.1 bits)",
+            "config": {"workload": "streamed 80-layer Llama-70B-shape model (sampled chunks of layer 0)"},
+            "cpu_baseline": cpu, "e2e": {"value": round(v, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                                         "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["eqw", "reference"], default="eqw")
+    ap.add_argument("--distinct-layers", type=int, default=8)
+    ap.add_argument("--layers", type=int, default=N_LAYERS, help="blocks per pass (80 = the 70B model)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return 0
+        print(json.dumps(bench_reference(args)), flush=True)
+        return 0
+
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    d = Dist()
+    if d.world == 1:
+        torch.cuda.set_device(0)
+    try:
+        line = bench_eqw(args, d)
+    finally:
+        d.close()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

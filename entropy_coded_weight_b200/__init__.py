@@ -1,0 +1,188 @@
+"""entropy_coded_weight_b200 -- B200 decoder for entropy-coded LLM weights.
+
+Thin Python layer over libeqw.so (C ABI in include/eqw.h).  Every function
+marshals arguments and calls the C entry point of the same name; all decoding
+runs in the library's CUDA kernels.  PyTorch provides device memory, streams
+and events.
+
+Typical use (EntQuant technical summary, gist.science 2601.22787, section 2:
+weights stored as a compressed bitstream in GPU memory and expanded block by
+block just before each block's forward pass)::
+
+    blob = encode_host(matrices)                 # host, threads over chunks
+    d_blob = upload(blob)                        # one copy into HBM
+    model = Model(d_blob, blob)                  # parse + validate
+    out = torch.empty(model.block_bytes(layer), dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    model.decode_block(layer, out, status)       # rANS decode + dequant + scatter
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import _lib
+from ._lib import (EQ_DEV_BAD_END, EQ_DEV_BAD_HEADER, EQ_DEV_BAD_OUTLIER, EQ_DEV_BAD_STATE, EQ_DEV_BAD_TABLE,
+                   EQ_DEV_TIMEOUT, EQ_E4M3, EQ_INT8, EqError, check, eq_matrix_in, eq_matrix_info, load)
+
+__all__ = [
+    "EQ_INT8", "EQ_E4M3", "EqError", "Model", "encode_host", "upload", "gemv_bf16", "eq_status_string",
+    "eq_format_version", "EQ_DEV_BAD_HEADER", "EQ_DEV_BAD_TABLE", "EQ_DEV_BAD_STATE", "EQ_DEV_BAD_END",
+    "EQ_DEV_TIMEOUT", "EQ_DEV_BAD_OUTLIER",
+]
+
+
+def _ptr(a) -> int | None:
+    if a is None:
+        return None
+    if isinstance(a, np.ndarray):
+        return a.ctypes.data
+    return a.data_ptr()
+
+
+def _stream_handle(stream) -> int | None:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def eq_status_string(code: int) -> str:
+    return load().eq_status_string(code).decode()
+
+
+def eq_format_version() -> int:
+    return load().eq_format_version()
+
+
+def _matrix_in_array(matrices):
+    """eq_matrix_in[] for objects with layer, dtype, symbols, scales, out_row/out_col/out_val."""
+    keep = []
+    arr = (eq_matrix_in * max(1, len(matrices)))()
+    for i, m in enumerate(matrices):
+        sym = np.ascontiguousarray(m.symbols, dtype=np.uint8)
+        if sym.ndim != 2:
+            raise ValueError("symbols must be [rows, cols]")
+        sc = np.ascontiguousarray(m.scales, dtype=np.float32)
+        orow = np.ascontiguousarray(getattr(m, "out_row", np.zeros(0)), dtype=np.uint32)
+        ocol = np.ascontiguousarray(getattr(m, "out_col", np.zeros(0)), dtype=np.uint32)
+        oval = np.ascontiguousarray(getattr(m, "out_val", np.zeros(0)), dtype=np.float32)
+        keep += [sym, sc, orow, ocol, oval]
+        e = arr[i]
+        e.layer = int(m.layer)
+        e.dtype = int(m.dtype)
+        e.rows, e.cols = sym.shape
+        e.symbols = sym.ctypes.data if sym.size else None
+        e.scales = sc.ctypes.data if sc.size else None
+        e.n_out = orow.size
+        e.out_row = orow.ctypes.data if orow.size else None
+        e.out_col = ocol.ctypes.data if ocol.size else None
+        e.out_val = oval.ctypes.data if oval.size else None
+    return arr, keep
+
+
+def encode_host(matrices, n_threads: int = 0) -> np.ndarray:
+    """Encode matrices into a container v1 blob (uint8 numpy array) with eq_encoder_run."""
+    L = load()
+    arr, keep = _matrix_in_array(matrices)
+    h = ctypes.c_void_p()
+    size = ctypes.c_size_t()
+    check(L.eq_encoder_run(arr, len(matrices), n_threads, ctypes.byref(h), ctypes.byref(size)), "eq_encoder_run")
+    try:
+        out = np.empty(size.value, np.uint8)
+        check(L.eq_encoded_write(h, out.ctypes.data, out.size), "eq_encoded_write")
+    finally:
+        L.eq_encoded_free(h)
+    del keep
+    return out
+
+
+def upload(blob: np.ndarray, device=None):
+    """Copy a host container into a fresh device tensor (uint8; the allocator aligns it to >= 256 B)."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(blob, dtype=np.uint8))
+    return t.to(device or "cuda", non_blocking=False)
+
+
+class Model:
+    """A container resident in device memory (eq_model_open / eq_model_close)."""
+
+    def __init__(self, d_blob, h_blob):
+        self._L = load()
+        self.d_blob = d_blob  # keep the device bytes alive
+        self._h = np.ascontiguousarray(h_blob, dtype=np.uint8)
+        if d_blob.numel() != self._h.size:
+            raise ValueError("device and host copies differ in length")
+        handle = ctypes.c_void_p()
+        check(self._L.eq_model_open(d_blob.data_ptr(), self._h.size, self._h.ctypes.data, ctypes.byref(handle)),
+              "eq_model_open")
+        self._m = handle
+        nl, nm = ctypes.c_uint32(), ctypes.c_uint32()
+        check(self._L.eq_model_counts(self._m, ctypes.byref(nl), ctypes.byref(nm)), "eq_model_counts")
+        self.n_layers, self.n_matrices = nl.value, nm.value
+        self._h = None  # only needed while opening
+
+    def close(self) -> None:
+        if getattr(self, "_m", None):
+            self._L.eq_model_close(self._m)
+            self._m = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def handle(self) -> int:
+        return self._m.value
+
+    def info(self, matrix: int) -> eq_matrix_info:
+        inf = eq_matrix_info()
+        check(self._L.eq_matrix_get_info(self._m, matrix, ctypes.byref(inf)), "eq_matrix_get_info")
+        return inf
+
+    def layer_matrices(self, layer: int) -> range:
+        f, c = ctypes.c_uint32(), ctypes.c_uint32()
+        check(self._L.eq_layer_matrices(self._m, layer, ctypes.byref(f), ctypes.byref(c)), "eq_layer_matrices")
+        return range(f.value, f.value + c.value)
+
+    def block_layout(self, layer: int) -> tuple[list[int], int]:
+        n = len(self.layer_matrices(layer))
+        offs = (ctypes.c_size_t * max(1, n))()
+        total = ctypes.c_size_t()
+        check(self._L.eq_block_layout(self._m, layer, offs, n, ctypes.byref(total)), "eq_block_layout")
+        return [offs[i] for i in range(n)], total.value
+
+    def block_bytes(self, layer: int) -> int:
+        return self.block_layout(layer)[1]
+
+    def decode_matrix(self, matrix: int, out, status, stream=None) -> None:
+        """eq_decode_matrix into ``out`` (device tensor, >= 2*rows*cols bytes)."""
+        nbytes = out.numel() * out.element_size()
+        check(self._L.eq_decode_matrix(self._m, matrix, out.data_ptr(), nbytes, status.data_ptr(),
+                                       _stream_handle(stream)), "eq_decode_matrix")
+
+    def decode_block(self, layer: int, out, status, stream=None) -> None:
+        """eq_decode_block into ``out`` (device tensor, >= block_bytes(layer) bytes)."""
+        nbytes = out.numel() * out.element_size()
+        check(self._L.eq_decode_block(self._m, layer, out.data_ptr(), nbytes, status.data_ptr(),
+                                      _stream_handle(stream)), "eq_decode_block")
+
+    def decode_model_stream(self, layer: int, bufs, status, decode_stream, ev_free, ev_ready) -> None:
+        """eq_decode_model_stream: wait ev_free[b], decode into bufs[b], record ev_ready[b] (b = layer & 1)."""
+        nbytes = min(b.numel() * b.element_size() for b in bufs)
+        pbuf = (ctypes.c_void_p * 2)(bufs[0].data_ptr(), bufs[1].data_ptr())
+        pfree = (ctypes.c_void_p * 2)(*(e.cuda_event if e is not None else None for e in ev_free))
+        pready = (ctypes.c_void_p * 2)(*(e.cuda_event for e in ev_ready))
+        check(self._L.eq_decode_model_stream(self._m, layer, pbuf, nbytes, status.data_ptr(),
+                                             _stream_handle(decode_stream), pfree, pready),
+              "eq_decode_model_stream")
+
+
+def gemv_bf16(w, x, y, stream=None) -> None:
+    """eq_gemv_bf16: y[r] = sum_c w[r, c] * x[c] (w bf16 [rows, cols], x bf16 [cols], y fp32 [rows])."""
+    rows, cols = w.shape
+    check(load().eq_gemv_bf16(w.data_ptr(), x.data_ptr(), y.data_ptr(), rows, cols, _stream_handle(stream)),
+          "eq_gemv_bf16")

@@ -1,0 +1,335 @@
+// Host encoder for container v1 (eq_encoder_run / eq_encoded_write /
+// eq_encode_host).
+//
+// EntQuant technical summary (gist.science 2601.22787), section 2 "weight
+// encoding": the (already quantised, low-entropy) weights are flattened into a
+// symbol stream and compressed losslessly with an ANS coder; storage is the
+// bitstream, the scales and metadata.  Here the stream of every matrix is cut
+// into independent 65536-symbol chunks (EntroLLM technical overview,
+// "parallel decoding strategy": chunks that keep the tensor structure and
+// decode independently); each chunk gets its own 12-bit frequency table and
+// 32 interleaved rANS states.  Chunks are encoded in parallel on host threads.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <memory>
+#include <new>
+#include <thread>
+#include <vector>
+
+#include "eqw_internal.h"
+
+using namespace eqw;
+
+namespace {
+
+// ---- frequency table ---------------------------------------------------------
+// Start from the proportional share rounded to nearest (at least 1 for every
+// present symbol), then move single units greedily where they cost the fewest
+// expected bits: adding one unit to s saves cnt_s * log2((f+1)/f) bits,
+// removing one costs cnt_s * log2(f/(f-1)).
+void quantize_table(const uint32_t cnt[256], uint32_t n, uint32_t f[256]) {
+    int present[256];
+    int np = 0;
+    int64_t sum = 0;
+    for (int s = 0; s < 256; ++s) {
+        f[s] = 0;
+        if (!cnt[s]) continue;
+        present[np++] = s;
+        uint64_t q = ((uint64_t)cnt[s] * kProbTotal + n / 2) / n;
+        f[s] = q ? (uint32_t)q : 1u;
+        sum += f[s];
+    }
+    while (sum < (int64_t)kProbTotal) {
+        int best = -1;
+        double gain = -1.0;
+        for (int i = 0; i < np; ++i) {
+            int s = present[i];
+            double g = cnt[s] * std::log2((f[s] + 1.0) / f[s]);
+            if (g > gain) { gain = g; best = s; }
+        }
+        f[best] += 1;
+        ++sum;
+    }
+    while (sum > (int64_t)kProbTotal) {
+        int best = -1;
+        double loss = 0.0;
+        for (int i = 0; i < np; ++i) {
+            int s = present[i];
+            if (f[s] <= 1) continue;
+            double l = cnt[s] * std::log2((double)f[s] / (f[s] - 1.0));
+            if (best < 0 || l < loss) { loss = l; best = s; }
+        }
+        f[best] -= 1;
+        --sum;
+    }
+}
+
+// ---- one chunk record ----------------------------------------------------------
+// Symbol j of the chunk belongs to lane (j % 256) / 8 at step 8 * (j / 256) + j % 8.
+// The decoder walks steps upward and lanes upward inside a step, so the encoder
+// walks both downward and writes each renormalisation word in front of the
+// previous one.
+void encode_record(const uint8_t *sym, uint32_t n, std::vector<uint8_t> &rec, std::vector<uint16_t> &scratch) {
+    uint32_t cnt[256] = {0};
+    for (uint32_t j = 0; j < n; ++j) ++cnt[sym[j]];
+    uint32_t f[256], cum[256];
+    quantize_table(cnt, n, f);
+    uint32_t c = 0;
+    uint32_t n_present = 0;
+    for (int s = 0; s < 256; ++s) {
+        cum[s] = c;
+        c += f[s];
+        n_present += f[s] != 0;
+    }
+
+    // x >= limit[s] means the state must shed 16 bits before coding s
+    uint64_t limit[256];
+    for (int s = 0; s < 256; ++s) limit[s] = (uint64_t)f[s] << (32 - kProbBits);
+
+    if (scratch.size() < n) scratch.resize(n);
+    uint16_t *wend = scratch.data() + n;
+    uint16_t *w = wend;
+    uint32_t x[kLanes];
+    for (uint32_t l = 0; l < kLanes; ++l) x[l] = kStateLow;
+
+    const uint32_t groups = (n + kGroupSyms - 1) / kGroupSyms;
+    for (uint32_t g = groups; g-- > 0;) {
+        const uint32_t base = g * kGroupSyms;
+        const bool full = base + kGroupSyms <= n;
+        for (uint32_t r = kGroup; r-- > 0;) {
+            for (uint32_t l = kLanes; l-- > 0;) {
+                const uint32_t j = base + l * kGroup + r;
+                if (!full && j >= n) continue;
+                const uint32_t s = sym[j];
+                uint32_t xv = x[l];
+                if (xv >= limit[s]) {
+                    *--w = (uint16_t)xv;
+                    xv >>= 16;
+                }
+                const uint32_t q = xv / f[s];
+                x[l] = q * kProbTotal + (xv - q * f[s]) + cum[s];
+            }
+        }
+    }
+    const uint32_t n_words = (uint32_t)(wend - w);
+
+    const size_t table_end = align_up(kRecordHeadBytes + 4 * (size_t)n_present, 16);
+    const size_t total = table_end + align_up(2 * (size_t)n_words, 16);
+    rec.assign(total, 0);
+    uint8_t *p = rec.data();
+    const uint32_t head[4] = {n, n_words, n_present, 0};
+    std::memcpy(p, head, 16);
+    std::memcpy(p + 16, x, 4 * kLanes);
+    uint32_t *tab = reinterpret_cast<uint32_t *>(p + kRecordHeadBytes);
+    for (int s = 0, k = 0; s < 256; ++s)
+        if (f[s]) tab[k++] = (uint32_t)s | (f[s] << 16);
+    std::memcpy(p + table_end, w, 2 * (size_t)n_words);
+}
+
+struct Job {
+    uint32_t mat;
+    uint32_t chunk;
+};
+
+int validate(const eq_matrix_in *mats, uint32_t n_mats, uint32_t *n_layers) {
+    if (!mats && n_mats) return EQ_ERR_INVALID_ARG;
+    uint32_t max_layer = 0;
+    for (uint32_t i = 0; i < n_mats; ++i) {
+        const eq_matrix_in &m = mats[i];
+        if (m.dtype != EQ_INT8 && m.dtype != EQ_E4M3) return EQ_ERR_INVALID_ARG;
+        const uint64_t n = (uint64_t)m.rows * m.cols;
+        if (n && (!m.symbols || !m.scales)) return EQ_ERR_INVALID_ARG;
+        if ((n + kChunkSyms - 1) / kChunkSyms > 0xFFFFFFFFull) return EQ_ERR_INVALID_ARG;
+        if (m.dtype == EQ_E4M3)
+            for (uint64_t k = 0; k < n; ++k)
+                if ((m.symbols[k] & 0x7F) == 0x7F) return EQ_ERR_INVALID_ARG;
+        if (m.n_out && (!m.out_row || !m.out_col || !m.out_val)) return EQ_ERR_INVALID_ARG;
+        uint64_t prev = 0;
+        for (uint32_t k = 0; k < m.n_out; ++k) {
+            if (m.out_row[k] >= m.rows || m.out_col[k] >= m.cols) return EQ_ERR_INVALID_ARG;
+            const uint64_t lin = (uint64_t)m.out_row[k] * m.cols + m.out_col[k];
+            if (k && lin <= prev) return EQ_ERR_INVALID_ARG;
+            prev = lin;
+        }
+        max_layer = std::max(max_layer, m.layer);
+    }
+    if (n_mats) {
+        std::vector<char> seen(max_layer + 1, 0);
+        for (uint32_t i = 0; i < n_mats; ++i) seen[mats[i].layer] = 1;
+        for (char s : seen)
+            if (!s) return EQ_ERR_INVALID_ARG;  // layers must be 0..n-1
+        *n_layers = max_layer + 1;
+    } else {
+        *n_layers = 0;
+    }
+    return EQ_OK;
+}
+
+}  // namespace
+
+struct eq_encoded {
+    std::vector<uint8_t> bytes;
+};
+
+extern "C" EQW_API int eq_encoder_run(const eq_matrix_in *mats, uint32_t n_mats, int n_threads,
+                                      eq_encoded **h, size_t *size) {
+    if (!h || !size) return EQ_ERR_INVALID_ARG;
+    *h = nullptr;
+    uint32_t n_layers = 0;
+    int rc = validate(mats, n_mats, &n_layers);
+    if (rc) return rc;
+
+    // directory order: by layer, input order inside a layer
+    std::vector<uint32_t> order(n_mats);
+    for (uint32_t i = 0; i < n_mats; ++i) order[i] = i;
+    std::stable_sort(order.begin(), order.end(),
+                     [&](uint32_t a, uint32_t b) { return mats[a].layer < mats[b].layer; });
+
+    std::vector<uint32_t> n_chunks(n_mats);
+    std::vector<Job> jobs;
+    for (uint32_t d = 0; d < n_mats; ++d) {
+        const eq_matrix_in &m = mats[order[d]];
+        const uint64_t n = (uint64_t)m.rows * m.cols;
+        n_chunks[d] = (uint32_t)((n + kChunkSyms - 1) / kChunkSyms);
+        for (uint32_t k = 0; k < n_chunks[d]; ++k) jobs.push_back({d, k});
+    }
+
+    std::vector<std::vector<uint8_t>> records(jobs.size());
+    std::atomic<size_t> next{0};
+    auto worker = [&]() {
+        std::vector<uint16_t> scratch;
+        std::vector<uint8_t> patched;
+        for (;;) {
+            const size_t i = next.fetch_add(1);
+            if (i >= jobs.size()) break;
+            const eq_matrix_in &m = mats[order[jobs[i].mat]];
+            const uint64_t n = (uint64_t)m.rows * m.cols;
+            const uint64_t first = (uint64_t)jobs[i].chunk * kChunkSyms;
+            const uint32_t len = (uint32_t)std::min<uint64_t>(kChunkSyms, n - first);
+            const uint8_t *src = m.symbols + first;
+            if (m.n_out) {
+                // super weights travel outside the stream: code the placeholder 0
+                patched.assign(src, src + len);
+                for (uint32_t k = 0; k < m.n_out; ++k) {
+                    const uint64_t lin = (uint64_t)m.out_row[k] * m.cols + m.out_col[k];
+                    if (lin >= first && lin < first + len) patched[lin - first] = 0;
+                }
+                src = patched.data();
+            }
+            encode_record(src, len, records[i], scratch);
+        }
+    };
+    unsigned nt = n_threads > 0 ? (unsigned)n_threads : std::max(1u, std::thread::hardware_concurrency());
+    nt = (unsigned)std::min<size_t>(nt, std::max<size_t>(1, jobs.size()));
+    std::vector<std::thread> pool;
+    for (unsigned t = 1; t < nt; ++t) pool.emplace_back(worker);
+    worker();
+    for (auto &t : pool) t.join();
+
+    // layout: header | directory | per matrix: chunk index, scales, outliers, records
+    uint64_t pos = align_up(kHeaderBytes + (uint64_t)kDirEntryBytes * n_mats, kSectionAlign);
+    struct Place { uint64_t ci, so, oo, rec0; };
+    std::vector<Place> place(n_mats);
+    std::vector<uint64_t> rec_off(jobs.size() + 1);
+    size_t j = 0;
+    for (uint32_t d = 0; d < n_mats; ++d) {
+        const eq_matrix_in &m = mats[order[d]];
+        Place &pl = place[d];
+        pl.ci = pos;
+        pos = align_up(pos + 8ull * (n_chunks[d] + 1), kSectionAlign);
+        pl.so = pos;
+        pos = align_up(pos + 4ull * m.rows, kSectionAlign);
+        pl.oo = 0;
+        if (m.n_out) {
+            pl.oo = pos;
+            pos = align_up(pos + 12ull * m.n_out, kSectionAlign);
+        }
+        pl.rec0 = pos;
+        for (uint32_t k = 0; k < n_chunks[d]; ++k, ++j) {
+            rec_off[j] = pos;
+            pos += records[j].size();
+        }
+        pos = align_up(pos, kSectionAlign);
+    }
+    const uint64_t total = pos;
+
+    auto *enc = new (std::nothrow) eq_encoded;
+    if (!enc) return EQ_ERR_NOSPACE;
+    try {
+        enc->bytes.assign(total, 0);
+    } catch (...) {
+        delete enc;
+        return EQ_ERR_NOSPACE;
+    }
+    uint8_t *b = enc->bytes.data();
+    auto put32 = [](uint8_t *p, uint32_t v) { std::memcpy(p, &v, 4); };
+    auto put64 = [](uint8_t *p, uint64_t v) { std::memcpy(p, &v, 8); };
+    std::memcpy(b, "EQW1", 4);
+    put32(b + 4, kVersion);
+    put32(b + 8, kHeaderBytes);
+    put32(b + 12, kProbBits);
+    put32(b + 16, kLanes);
+    put32(b + 20, kGroup);
+    put32(b + 24, kChunkSyms);
+    put32(b + 28, n_layers);
+    put32(b + 32, n_mats);
+    put64(b + 40, kHeaderBytes);
+    put64(b + 48, total);
+
+    std::vector<uint32_t> index_in_layer(n_layers, 0);
+    j = 0;
+    for (uint32_t d = 0; d < n_mats; ++d) {
+        const eq_matrix_in &m = mats[order[d]];
+        const Place &pl = place[d];
+        uint8_t *e = b + kHeaderBytes + (uint64_t)kDirEntryBytes * d;
+        put32(e + 0, m.layer);
+        put32(e + 4, index_in_layer[m.layer]++);
+        put32(e + 8, m.dtype);
+        put32(e + 12, n_chunks[d]);
+        put32(e + 16, m.rows);
+        put32(e + 20, m.cols);
+        put32(e + 24, m.n_out);
+        put64(e + 32, pl.ci);
+        put64(e + 40, pl.so);
+        put64(e + 48, pl.oo);
+        for (uint32_t k = 0; k < n_chunks[d]; ++k) put64(b + pl.ci + 8ull * k, rec_off[j + k]);
+        const uint64_t rec_end =
+            n_chunks[d] ? rec_off[j + n_chunks[d] - 1] + records[j + n_chunks[d] - 1].size() : pl.rec0;
+        put64(b + pl.ci + 8ull * n_chunks[d], rec_end);
+        if (m.rows) std::memcpy(b + pl.so, m.scales, 4ull * m.rows);
+        for (uint32_t k = 0; k < m.n_out; ++k) {
+            put32(b + pl.oo + 12ull * k, m.out_row[k]);
+            put32(b + pl.oo + 12ull * k + 4, m.out_col[k]);
+            std::memcpy(b + pl.oo + 12ull * k + 8, &m.out_val[k], 4);
+        }
+        for (uint32_t k = 0; k < n_chunks[d]; ++k, ++j)
+            std::memcpy(b + rec_off[j], records[j].data(), records[j].size());
+    }
+    *h = enc;
+    *size = total;
+    return EQ_OK;
+}
+
+extern "C" EQW_API int eq_encoded_write(const eq_encoded *h, void *out, size_t out_cap) {
+    if (!h || (!out && !h->bytes.empty())) return EQ_ERR_INVALID_ARG;
+    if (out_cap < h->bytes.size()) return EQ_ERR_NOSPACE;
+    std::memcpy(out, h->bytes.data(), h->bytes.size());
+    return EQ_OK;
+}
+
+extern "C" EQW_API void eq_encoded_free(eq_encoded *h) { delete h; }
+
+extern "C" EQW_API int eq_encode_host(const eq_matrix_in *mats, uint32_t n_mats, int n_threads, void *out,
+                                      size_t out_cap, size_t *out_len) {
+    if (!out_len) return EQ_ERR_INVALID_ARG;
+    eq_encoded *h = nullptr;
+    size_t size = 0;
+    int rc = eq_encoder_run(mats, n_mats, n_threads, &h, &size);
+    if (rc) return rc;
+    *out_len = size;
+    rc = eq_encoded_write(h, out, out_cap);
+    eq_encoded_free(h);
+    return rc;
+}

@@ -1,0 +1,47 @@
+// Internal definitions shared by the libeqw translation units (host side).
+// Format constants follow container v1 (magic "EQW1"): 12-bit frequencies,
+// 32 lanes, 8 consecutive symbols per lane per 256-symbol group, 65536-symbol
+// chunks, 256-byte section alignment, 16-byte chunk records.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <vector>
+
+#include "../../include/eqw.h"
+
+namespace eqw {
+
+constexpr uint32_t kVersion = 1;
+constexpr uint32_t kHeaderBytes = 64;
+constexpr uint32_t kDirEntryBytes = 64;
+constexpr uint32_t kProbBits = 12;
+constexpr uint32_t kProbTotal = 1u << kProbBits;
+constexpr uint32_t kLanes = 32;
+constexpr uint32_t kGroup = 8;
+constexpr uint32_t kGroupSyms = kLanes * kGroup;
+constexpr uint32_t kChunkSyms = 65536;
+constexpr uint32_t kStateLow = 1u << 16;
+constexpr uint32_t kRecordHeadBytes = 16 + 4 * kLanes;  // counts + 32 states
+constexpr uint64_t kSectionAlign = 256;
+constexpr uint32_t kMaxMatsPerLaunch = 16;
+
+inline uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+struct MatrixDesc {
+    eq_matrix_info info;
+    uint64_t chunk_index_off;
+    uint64_t scales_off;
+    uint64_t outliers_off;
+};
+
+}  // namespace eqw
+
+struct eq_model {
+    const uint8_t *d_blob;
+    size_t len;
+    uint32_t n_layers;
+    std::vector<eqw::MatrixDesc> mats;
+    std::vector<uint32_t> layer_first;
+    std::vector<uint32_t> layer_count;
+};

@@ -1,0 +1,211 @@
+/*
+ * eqw.h -- C ABI of libeqw, B200 (sm_100a) decoder for entropy-coded weights.
+ *
+ * The method (EntQuant technical summary, gist.science paper 2601.22787,
+ * section 2 "weight encoding" and "inference-time decoding"): weights keep an
+ * Int8 or Float8 base format, are flattened into a symbol stream and
+ * compressed losslessly with an ANS coder; storage is the bitstream plus the
+ * per-channel scales plus metadata.  The bitstream stays resident in GPU
+ * memory and, just before a transformer block runs, a parallel ANS decoder
+ * expands that block's weights into a buffer; decoding and the forward
+ * kernels are interleaved.  Super weights (extreme Int8 outliers, section 2
+ * "super weights") are kept outside the entropy-coded stream.  Chunks are
+ * independent so that they decode in parallel (EntroLLM technical overview,
+ * "parallel decoding strategy").
+ *
+ * Coding used here: rANS, 12-bit frequencies (M = 4096), 32-bit states in
+ * [2^16, 2^32), 16-bit renormalisation words, 32 interleaved states per chunk
+ * of up to 65536 symbols, per-chunk frequency tables, fp32 per-row scales,
+ * fp32 COO outliers.  The byte layout ("container v1", magic "EQW1") is
+ * specified in DESIGN.md of this repository, section "Container format v1".
+ *
+ * Conventions for every function below:
+ *   - Return value: EQ_OK (0) or one of the EQ_ERR_* codes; nothing throws.
+ *   - The caller owns all memory, streams and events.  The library never
+ *     allocates device memory, never frees caller memory and never
+ *     synchronises a stream or the device.  The only allocations it makes
+ *     are host-side descriptors (eq_model, eq_encoded).
+ *   - Device pointers are plain addresses in the current CUDA device's
+ *     memory (from PyTorch: tensor.data_ptr()); streams/events are raw
+ *     cudaStream_t / cudaEvent_t handles (torch.cuda.Stream().cuda_stream).
+ *     Every decode call launches on the stream it is given, in the device
+ *     that is current when it is called.
+ *   - Problems found by a kernel are OR-ed asynchronously into *d_status, a
+ *     caller-provided device int32 the caller zeroes beforehand and reads
+ *     after its own synchronisation (EQ_DEV_* bits below).  A chunk with a
+ *     problem leaves its output range unspecified; all others are exact.
+ *   - Decoded values are bit-exact: out = bf16_rne(fp32_rn(value * scale))
+ *     with round-to-nearest-even in both steps, no FMA, no flush-to-zero;
+ *     outliers are written as bf16_rne(value).
+ */
+#ifndef EQW_H
+#define EQW_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define EQW_API __attribute__((visibility("default")))
+
+/* ---- status codes --------------------------------------------------------- */
+enum {
+    EQ_OK = 0,
+    EQ_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad dtype, unsorted outliers ... */
+    EQ_ERR_CORRUPT = 2,      /* container fails validation */
+    EQ_ERR_UNSUPPORTED = 3,  /* format constant or version this build does not decode */
+    EQ_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, event, attribute) */
+    EQ_ERR_TIMEOUT = 5,      /* reserved for host-side bounded waits */
+    EQ_ERR_NOSPACE = 6       /* output buffer too small; required size is reported */
+};
+
+/* bits OR-ed into *d_status by the kernels */
+enum {
+    EQ_DEV_BAD_HEADER = 1,   /* chunk record header inconsistent with the directory */
+    EQ_DEV_BAD_TABLE = 2,    /* frequency table not ascending / f = 0 / sum != 4096 */
+    EQ_DEV_BAD_STATE = 4,    /* an initial state outside [2^16, 2^32) */
+    EQ_DEV_BAD_END = 8,      /* final states != 2^16 or words consumed != n_words */
+    EQ_DEV_TIMEOUT = 16,     /* a bounded wait for a staged copy gave up */
+    EQ_DEV_BAD_OUTLIER = 32  /* outlier position outside its matrix */
+};
+
+/* symbol formats */
+enum { EQ_INT8 = 1, EQ_E4M3 = 2 };
+
+/* ---- host encoder ------------------------------------------------------------
+ * One weight matrix to encode.  `symbols` is row-major [rows, cols] (Int8 as
+ * two's-complement bytes, or E4M3 bytes; the E4M3 NaN codes 0x7F / 0xFF are
+ * rejected).  `scales` holds one fp32 scale per row.  Outliers (super
+ * weights) are given as parallel arrays, sorted by row * cols + col, unique
+ * and in range; their positions are coded as symbol 0 in the stream and
+ * overwritten by the scatter after decoding.  `layer` groups matrices into
+ * blocks: layers must be 0..n_layers-1; matrices of one layer keep their
+ * order in the input array (that order is their index within the layer).
+ * All pointers are host pointers and are only read.
+ */
+typedef struct eq_matrix_in {
+    uint32_t layer;
+    uint32_t dtype;          /* EQ_INT8 or EQ_E4M3 */
+    uint32_t rows;
+    uint32_t cols;
+    const uint8_t *symbols;  /* rows * cols bytes */
+    const float *scales;     /* rows floats */
+    uint32_t n_out;
+    const uint32_t *out_row; /* n_out entries (may be NULL if n_out == 0) */
+    const uint32_t *out_col;
+    const float *out_val;
+} eq_matrix_in;
+
+typedef struct eq_encoded eq_encoded;  /* host-side result of eq_encoder_run */
+
+/*
+ * Encode `n_mats` matrices into a container with `n_threads` host threads
+ * (<= 0: all online cores).  On success *h holds the encoded container in
+ * library-owned host memory and *size its exact byte length.  Errors:
+ * EQ_ERR_INVALID_ARG for bad inputs.
+ */
+EQW_API int eq_encoder_run(const eq_matrix_in *mats, uint32_t n_mats, int n_threads,
+                           eq_encoded **h, size_t *size);
+
+/* Copy the encoded container to `out` (host, >= size bytes). EQ_ERR_NOSPACE if out_cap < size. */
+EQW_API int eq_encoded_write(const eq_encoded *h, void *out, size_t out_cap);
+
+/* Release the result of eq_encoder_run (NULL is ignored). */
+EQW_API void eq_encoded_free(eq_encoded *h);
+
+/*
+ * One-call encoder: eq_encoder_run + eq_encoded_write + eq_encoded_free.
+ * *out_len receives the container size; if out_cap is smaller the call
+ * returns EQ_ERR_NOSPACE and leaves `out` untouched.
+ */
+EQW_API int eq_encode_host(const eq_matrix_in *mats, uint32_t n_mats, int n_threads,
+                           void *out, size_t out_cap, size_t *out_len);
+
+/* ---- model (a container resident in device memory) ---------------------------- */
+typedef struct eq_model eq_model;
+
+typedef struct eq_matrix_info {
+    uint32_t layer, index, dtype, rows, cols, n_chunks, n_outliers, reserved;
+    uint64_t compressed_bytes;  /* bytes of its chunk records (tables, states, words) */
+    uint64_t payload_words;     /* total 16-bit renormalisation words */
+} eq_matrix_info;
+
+/*
+ * Open a container that the caller has copied to device memory at `d_blob`
+ * (`len` bytes, 256-byte aligned).  `h_blob` must point to a host copy of the
+ * same `len` bytes; it is read only during this call, to parse and validate
+ * the header, the directory, every chunk index entry and every chunk
+ * record's header and frequency table.  The model keeps `d_blob` (not a
+ * copy): the device bytes must outlive the model and must not change.
+ * Errors: EQ_ERR_INVALID_ARG, EQ_ERR_CORRUPT, EQ_ERR_UNSUPPORTED.
+ */
+EQW_API int eq_model_open(const void *d_blob, size_t len, const void *h_blob, eq_model **m);
+
+/* Free the host descriptor (NULL is ignored).  Device memory is the caller's. */
+EQW_API void eq_model_close(eq_model *m);
+
+EQW_API int eq_model_counts(const eq_model *m, uint32_t *n_layers, uint32_t *n_matrices);
+EQW_API int eq_matrix_get_info(const eq_model *m, uint32_t matrix, eq_matrix_info *info);
+
+/* Matrices of `layer` are [*first, *first + *count) in directory order. */
+EQW_API int eq_layer_matrices(const eq_model *m, uint32_t layer, uint32_t *first, uint32_t *count);
+
+/*
+ * Where eq_decode_block puts each matrix of `layer`: the bf16 matrices are
+ * packed in index order, each starting at a 256-byte-aligned byte offset.
+ * `offsets` (host, `cap` entries, may be NULL when cap == 0) receives the
+ * byte offsets; *total_bytes the buffer size a block decode needs.
+ */
+EQW_API int eq_block_layout(const eq_model *m, uint32_t layer, size_t *offsets, uint32_t cap,
+                            size_t *total_bytes);
+
+/* ---- decode (hot path) ------------------------------------------------------
+ * Decode one matrix into `d_out` (device, 16-byte aligned, >= 2*rows*cols
+ * bytes, row-major bf16): rANS decode + dequant of every chunk (one warp per
+ * chunk), then the outlier scatter, both enqueued on `s`.
+ */
+EQW_API int eq_decode_matrix(const eq_model *m, uint32_t matrix, void *d_out, size_t out_bytes,
+                             int32_t *d_status, cudaStream_t s);
+
+/*
+ * Decode every matrix of `layer` into `d_out` (device, 256-byte aligned,
+ * >= eq_block_layout total) in one decode launch plus one scatter launch
+ * when the layer has outliers.  EQ_ERR_NOSPACE if out_bytes is too small.
+ */
+EQW_API int eq_decode_block(const eq_model *m, uint32_t layer, void *d_out, size_t out_bytes,
+                            int32_t *d_status, cudaStream_t s);
+
+/*
+ * Ping-pong streaming step for block-wise decode interleaved with a consumer
+ * (EntQuant section 2 "inference-time decoding").  With b = layer & 1 it
+ * enqueues on `decode_stream`: wait for ev_free[b] (skipped if NULL), decode
+ * the block into d_buf[b] (eq_decode_block), record ev_ready[b].  The
+ * consumer, on its own stream, waits for ev_ready[b], reads d_buf[b] and
+ * records ev_free[b] when done.  Both buffers hold `buf_bytes` bytes.
+ */
+EQW_API int eq_decode_model_stream(const eq_model *m, uint32_t layer, void *const d_buf[2],
+                                   size_t buf_bytes, int32_t *d_status, cudaStream_t decode_stream,
+                                   cudaEvent_t const ev_free[2], cudaEvent_t const ev_ready[2]);
+
+/*
+ * Batch-1 consumer: y[r] = sum_c W[r, c] * x[c] with W bf16 [rows, cols]
+ * row-major (16-byte aligned rows: cols % 8 == 0), x bf16 [cols], y fp32
+ * [rows]; products and sums in fp32.  Enqueued on `s`.
+ */
+EQW_API int eq_gemv_bf16(const void *d_w, const void *d_x, float *d_y, uint32_t rows, uint32_t cols,
+                         cudaStream_t s);
+
+/* ---- misc ----------------------------------------------------------------------- */
+EQW_API const char *eq_status_string(int status);
+
+/* Container version this build decodes (1). */
+EQW_API int eq_format_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EQW_H */
