@@ -17,6 +17,7 @@ EQ_ERR_CUDA, EQ_ERR_TIMEOUT, EQ_ERR_NOSPACE = 4, 5, 6
 EQ_DEV_BAD_HEADER, EQ_DEV_BAD_TABLE, EQ_DEV_BAD_STATE = 1, 2, 4
 EQ_DEV_BAD_END, EQ_DEV_TIMEOUT, EQ_DEV_BAD_OUTLIER = 8, 16, 32
 EQ_INT8, EQ_E4M3 = 1, 2
+EQ_TABLE_PER_CHUNK = 1
 
 
 class EqError(RuntimeError):
@@ -38,12 +39,13 @@ class eq_matrix_in(ctypes.Structure):
         ("out_row", ctypes.c_void_p),
         ("out_col", ctypes.c_void_p),
         ("out_val", ctypes.c_void_p),
+        ("flags", ctypes.c_uint32),
     ]
 
 
 class eq_matrix_info(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint32) for n in
-                ("layer", "index", "dtype", "rows", "cols", "n_chunks", "n_outliers", "reserved")] + [
+                ("layer", "index", "dtype", "rows", "cols", "n_chunks", "n_outliers", "uniform_table")] + [
         ("compressed_bytes", ctypes.c_uint64),
         ("payload_words", ctypes.c_uint64),
     ]

@@ -40,11 +40,15 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, defines: dict | None = None, out: str | None = None) -> str:
+    """Compile and link libeqw.so.  ``defines`` (-D NAME=VALUE for the CUDA
+    sources, e.g. EQ_SHARED_WARPS) and ``out`` build a tuning variant elsewhere."""
+    target = out or LIB
+    if not force and out is None and not _stale():
         return LIB
     nvcc = _nvcc()
-    objdir = os.path.join(HERE, "_build")
+    objdir = os.path.join(os.path.dirname(target), "_build", os.path.basename(target)) if out else \
+        os.path.join(HERE, "_build")
     os.makedirs(objdir, exist_ok=True)
     objs = []
     for src in sources():
@@ -52,6 +56,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         if src.endswith(".cu"):
             cmd = [nvcc, GENCODE, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",
                    "-ftz=false", "-prec-div=true", "-prec-sqrt=true", "-I", INCLUDE, "-c", src, "-o", obj]
+            cmd += [f"-D{k}={v}" for k, v in (defines or {}).items()]
             if verbose:
                 cmd[1:1] = ["-Xptxas", "-v"]
         else:
@@ -60,10 +65,10 @@ def build(force: bool = False, verbose: bool = False) -> str:
                    "-Wall", "-Wextra", "-I", INCLUDE, "-I", cuda_inc, "-c", src, "-o", obj]
         subprocess.check_call(cmd)
         objs.append(obj)
-    tmp = LIB + f".{os.getpid()}.tmp"
+    tmp = target + f".{os.getpid()}.tmp"
     subprocess.check_call([nvcc, GENCODE, "-shared", "-Xcompiler", "-pthread", "-o", tmp] + objs)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

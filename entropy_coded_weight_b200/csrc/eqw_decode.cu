@@ -9,32 +9,40 @@
 // entropy-coded stream.  EntroLLM technical overview, "parallel decoding
 // strategy": independent chunks decode concurrently.
 //
-// Kernel KB2, eq_rans_decode_dequant_kernel (persistent, one warp per chunk):
-//   prologue  load the chunk's frequency list, check it, expand it into a
-//             4096-slot table in shared memory: slot -> (f, slot - cum, sym)
-//             packed in one u32, so every decoded symbol costs one LDS;
-//   staging   the chunk's 16-bit renormalisation words stream into a 2 KB
-//             shared-memory ring in 512-byte segments with TMA bulk copies
-//             (cp.async.bulk, mbarrier completion, no multicast), issued up
-//             to four segments ahead by lane 0;
-//   decode    each lane owns one of the 32 interleaved rANS states; a step is
-//             slot = x & 4095; x = f * (x >> 12) + (slot - cum); if x < 2^16
-//             the lane takes the next word, its position found from a warp
-//             ballot and a popcount of the lower lanes;
-//   dequant   lane l decodes symbols 8l .. 8l+7 of every 256-symbol group, so
-//             after 8 steps it holds 8 consecutive outputs: value * row scale
-//             (fp32, round to nearest even), packed to bf16 (round to nearest
-//             even) and written with one 16-byte store; the warp's 32 stores
-//             cover 512 contiguous bytes.
-// Kernel KB3, eq_outlier_scatter_kernel: out[r * cols + c] = bf16(v) for the
-// super weights, launched after KB2 on the same stream.
+// KB2, eq_decode_kernel<WARPS, SHARED> -- one warp per 64 KiB chunk:
+//   slot table  4096 entries (f << 20 | (slot - cum) << 8 | sym) in shared
+//               memory, so a decoded symbol costs one LDS.  SHARED = true:
+//               every chunk of the matrix carries the same frequency table
+//               (checked by eq_model_open and again per chunk), so one table
+//               per thread block serves all its warps, which work on tiles of
+//               WARPS consecutive chunks; SHARED = false: one table per warp,
+//               rebuilt for every chunk.
+//   staging     each warp streams its chunk's 16-bit renormalisation words
+//               into a private 2 KB shared-memory ring in 512-byte segments
+//               with TMA bulk copies (cp.async.bulk, mbarrier completion, no
+//               multicast), up to four segments ahead, issued by lane 0.
+//   decode      lane l owns interleaved state l; one step of all lanes is
+//               slot = x & 4095; x = f * (x >> 12) + (slot - cum);
+//               if x < 2^16: x = x << 16 | next word, where the word's position
+//               is the warp-wide count of lower lanes that also renormalise
+//               (ballot + popcount).
+//   dequant     lane l decodes symbols 8l..8l+7 of each 256-symbol group, so
+//               every 8 steps it holds 8 consecutive outputs: value * row scale
+//               in fp32 (round to nearest even, packed f32x2 multiplies),
+//               packed to bf16 (round to nearest even) and stored as one
+//               16-byte vector; a warp's 32 stores cover 512 contiguous bytes.
+// KB3, eq_outlier_scatter_kernel -- out[r * cols + c] = bf16(v) for the super
+// weights, after KB2 on the same stream.
 //
-// No tensor cores: nothing here is a dense contraction.
+// Every wait on a staged copy is bounded (~1 s of SM clock); on expiry the
+// warp records EQ_DEV_TIMEOUT, waits (bounded) for its copies in flight and
+// stops decoding.  No tensor cores: nothing here is a dense contraction.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
 #include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "eqw_internal.h"
 
@@ -42,23 +50,25 @@ using namespace eqw;
 
 namespace {
 
-constexpr int kWarpsPerCta = 4;
-constexpr int kThreads = kWarpsPerCta * 32;
-constexpr uint32_t kSegWords = 256;  // one staging segment: 512 bytes
-constexpr uint32_t kSegBytes = 2 * kSegWords;
-constexpr uint32_t kRingSegs = 4;
-constexpr uint32_t kRingWords = kSegWords * kRingSegs;
 constexpr uint32_t kFull = 0xFFFFFFFFu;
-// Bounded wait for a staged copy: about one second of SM clocks, after which
-// the warp records EQ_DEV_TIMEOUT and stops instead of spinning forever.
+constexpr uint32_t kRingBytes = 2048;  // per warp
+constexpr uint32_t kSegBytes = 512;    // one TMA segment = 256 words
+constexpr uint32_t kRingSegs = kRingBytes / kSegBytes;
+constexpr uint32_t kLutBytes = 4 * kProbTotal;
 constexpr long long kWaitCycles = 2000000000LL;
+constexpr uint32_t kNoLimit = 0xFFFFFFFFu;
 
-struct __align__(16) WarpSmem {
-    uint32_t lut[kProbTotal];     // 16 KB: (f << 20) | ((slot - cum) << 8) | sym
-    uint16_t ring[kRingWords];    // 2 KB of staged renormalisation words
-    uint64_t mbar[kRingSegs];     // one mbarrier per ring segment
-};
-constexpr size_t kSmemBytes = sizeof(WarpSmem) * kWarpsPerCta;
+#ifndef EQ_SHARED_WARPS
+#define EQ_SHARED_WARPS 16
+#endif
+#ifndef EQ_SHARED_MIN_CTAS
+#define EQ_SHARED_MIN_CTAS 3
+#endif
+constexpr int kSharedWarps = EQ_SHARED_WARPS;      // warps per block, shared-table kernel
+constexpr int kSharedMinCtas = EQ_SHARED_MIN_CTAS; // register budget: blocks of kSharedWarps per SM
+constexpr int kPrivateWarps = 4;                   // warps per block, per-warp-table kernel
+
+enum : uint32_t { kRowUniform = 0, kLaneRows = 1, kGeneric = 2 };
 
 struct MatJob {
     const uint64_t *chunk_index;  // absolute record offsets, n_chunks + 1 entries
@@ -67,10 +77,10 @@ struct MatJob {
     uint64_t n_elems;
     uint32_t cols;
     uint32_t n_chunks;
-    uint32_t chunk_begin;         // first launch-wide chunk id of this matrix
+    uint32_t begin;               // first launch-wide work unit (tile or chunk) of this matrix
     uint32_t dtype;
-    uint32_t aligned;             // cols % 8 == 0 and out 16-byte aligned
-    uint32_t pad;
+    uint32_t layout;              // kRowUniform: cols % 256 == 0; kLaneRows: cols % 8 == 0; else kGeneric
+    uint32_t small_scales;        // all |scale| < 2^8: E4M3 dequant in one multiply
 };
 
 struct DecodeParams {
@@ -78,7 +88,7 @@ struct DecodeParams {
     uint64_t blob_len;
     int32_t *status;
     uint32_t n_mats;
-    uint32_t total_chunks;
+    uint32_t total_units;
     MatJob mats[kMaxMatsPerLaunch];
 };
 
@@ -95,13 +105,13 @@ struct ScatterParams {
     ScatterJob jobs[kMaxMatsPerLaunch];
 };
 
-// ---- PTX helpers: mbarrier + bulk copy (TMA, 1-D, no multicast) -------------
+// ---- PTX helpers: mbarrier + bulk copy (TMA, 1-D, no multicast) ---------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ void fence_mbar_init() {
@@ -112,32 +122,29 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
 }
 
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(bar), "r"(parity)
         : "memory");
     return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
@@ -146,28 +153,37 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     }
 }
 
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return v;
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
 }
 
-// ---- number formats -------------------------------------------------------------
-// Int8: two's complement.  E4M3 (OCP E4M3FN, bias 7): placing the 7 exponent
-// and mantissa bits at bit 20 of an fp32 gives value * 2^-120 exactly
-// (subnormal inputs included), and multiplying by 2^120 is exact.
-template <int DT>
-__device__ __forceinline__ float symbol_value(uint32_t s) {
-    if constexpr (DT == EQ_INT8) {
-        return static_cast<float>(static_cast<int8_t>(s & 0xFFu));
-    } else {
-        const uint32_t b = ((s & 0x80u) << 24) | ((s & 0x7Fu) << 20);
-        return __fmul_rn(__uint_as_float(b), 0x1p120f);
-    }
+__device__ __forceinline__ void st_global_v4(uint16_t *p, uint4 v) {
+    asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+// ---- number formats ----------------------------------------------------------------
+// Two fp32 products, each rounded to nearest even (Blackwell packed multiply).
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+    unsigned long long A, B, C;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(B) : "f"(b.x), "f"(b.y));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(C) : "l"(A), "l"(B));
+    float2 c;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(c.x), "=f"(c.y) : "l"(C));
+    return c;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float2 v) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
@@ -176,177 +192,375 @@ __device__ __forceinline__ uint16_t to_bf16(float v) {
     return *reinterpret_cast<uint16_t *>(&h);
 }
 
-__device__ __forceinline__ void flag(int32_t *status, int32_t bits) {
-    if ((threadIdx.x & 31) == 0) atomicOr(status, bits);
+// Int8: two's complement.  E4M3 (OCP E4M3FN, bias 7): the 7 exponent and
+// mantissa bits placed at bit 20 of an fp32 give exactly value * 2^-120
+// (subnormal codes included); the factor 2^120 is applied exactly, either on
+// its own or folded into a scale below 2^8 (same real product, one rounding).
+template <int DT>
+__device__ __forceinline__ float raw_value(uint32_t e) {
+    if constexpr (DT == EQ_INT8) {
+        return static_cast<float>(static_cast<int8_t>(e & 0xFFu));
+    } else {
+        return __uint_as_float(((e & 0x80u) << 24) | ((e & 0x7Fu) << 20));
+    }
 }
 
-// Staging ring for one chunk's words (warp-uniform bookkeeping).
-struct Ring {
+template <int DT>
+__device__ __forceinline__ float dequant1(uint32_t e, float scale) {
+    float v = raw_value<DT>(e);
+    if constexpr (DT == EQ_E4M3) v = __fmul_rn(v, 0x1p120f);
+    return __fmul_rn(v, scale);
+}
+
+// 8 symbols (low bytes of e[]) -> 8 bf16 in one 16-byte vector.  For E4M3
+// with `folded` the scale already carries the factor 2^120.
+template <int DT>
+__device__ __forceinline__ uint4 dequant8(const uint32_t (&e)[8], float s, bool folded) {
+    const float2 s2 = make_float2(s, s);
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 v = make_float2(raw_value<DT>(e[2 * i]), raw_value<DT>(e[2 * i + 1]));
+        if constexpr (DT == EQ_E4M3) {
+            if (!folded) v = mul2_rn(v, make_float2(0x1p120f, 0x1p120f));
+        }
+        o[i] = pack_bf16x2(mul2_rn(v, s2));
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ void flag(int32_t *status, int32_t bits) {
+    if ((threadIdx.x & 31u) == 0) atomicOr(status, bits);
+}
+
+// ---- word staging ring ------------------------------------------------------------
+// Per-warp bookkeeping lives in shared memory so that the decode loop keeps a
+// single register for it: `limit`, the consumed-byte count at which the next
+// group needs service (refill free slots or wait for a segment).
+struct RingCtl {
     const uint8_t *payload;
-    uint32_t pbytes;   // payload bytes padded to 16
+    uint32_t pbytes;   // payload bytes rounded up to 16
     uint32_t n_segs;
     uint32_t issued;
     uint32_t ready;
     uint32_t phase;    // bit k: parity of the next completion of mbar[k]
+    uint32_t dead;     // a bounded wait gave up
 };
 
-__device__ __forceinline__ void ring_issue(WarpSmem &S, Ring &R, uint32_t lane) {
-    const uint32_t s = R.issued++;
-    if (lane == 0) {
-        const uint32_t bytes = min(kSegBytes, R.pbytes - s * kSegBytes);
-        uint64_t *bar = &S.mbar[s % kRingSegs];
-        mbar_expect_tx(bar, bytes);
-        bulk_load(&S.ring[(s % kRingSegs) * kSegWords], R.payload + (size_t)s * kSegBytes, bytes, bar);
+__device__ __forceinline__ uint32_t ring_limit(uint32_t n_segs, uint32_t issued, uint32_t ready) {
+    // safe while bytes [pw, pw + 512) are resident and no free slot can take a segment
+    uint32_t lim = kNoLimit;
+    if (ready < n_segs) lim = ready * kSegBytes >= kSegBytes - 1 ? ready * kSegBytes - (kSegBytes - 1) : 0u;
+    if (issued < n_segs) {
+        const uint32_t t = issued >= kRingSegs - 1 ? (issued - (kRingSegs - 1)) * kSegBytes : 0u;
+        lim = min(lim, t);
     }
+    return lim;
 }
 
-// Keep up to four segments in flight and make sure words [p, p + 256) are
-// resident.  Returns false if a wait gave up.
-__device__ __forceinline__ bool ring_prepare(WarpSmem &S, Ring &R, uint32_t p, uint32_t lane) {
-    if (R.n_segs == 0) return true;
-    const uint32_t horizon = (p / kSegWords) + kRingSegs;
-    if (R.issued < R.n_segs && R.issued < horizon) {
-        // the slots being refilled were read through the generic proxy
+// Refill free slots, then make payload bytes [pw, pw + 512) resident.  Returns
+// the new limit; on a wait that gave up sets ctl->dead and returns kNoLimit.
+__device__ __noinline__ uint32_t ring_service(RingCtl *ctl, uint32_t ring, uint32_t mbar, uint32_t pw) {
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t n_segs = ctl->n_segs, pbytes = ctl->pbytes;
+    uint32_t issued = ctl->issued, ready = ctl->ready, phase = ctl->phase;
+    const uint32_t horizon = pw / kSegBytes + kRingSegs;
+    if (issued < n_segs && issued < horizon) {
         __syncwarp();
-        fence_proxy_async_smem();
+        fence_proxy_async_smem();  // the slots being refilled were read through the generic proxy
         do {
-            ring_issue(S, R, lane);
-        } while (R.issued < R.n_segs && R.issued < horizon);
+            if (lane == 0) {
+                const uint32_t bytes = min(kSegBytes, pbytes - issued * kSegBytes);
+                const uint32_t slot = issued % kRingSegs;
+                mbar_expect_tx(mbar + 8 * slot, bytes);
+                bulk_load(ring + slot * kSegBytes, ctl->payload + (size_t)issued * kSegBytes, bytes, mbar + 8 * slot);
+            }
+            ++issued;
+        } while (issued < n_segs && issued < horizon);
     }
-    uint32_t need = (p + kSegWords - 1) / kSegWords;
-    if (need >= R.n_segs) need = R.n_segs - 1;
-    while (R.ready <= need && R.ready < R.issued) {
-        const uint32_t slot = R.ready % kRingSegs;
-        const bool ok = mbar_wait_bounded(&S.mbar[slot], (R.phase >> slot) & 1u);
-        R.phase ^= 1u << slot;
-        ++R.ready;
-        if (!__all_sync(kFull, ok)) return false;
-    }
-    return true;
-}
-
-// Wait for every copy still in flight (bounded) so the ring can be reused.
-__device__ __forceinline__ bool ring_drain(WarpSmem &S, Ring &R) {
-    bool all_ok = true;
-    while (R.ready < R.issued) {
-        const uint32_t slot = R.ready % kRingSegs;
-        const bool ok = mbar_wait_bounded(&S.mbar[slot], (R.phase >> slot) & 1u);
-        R.phase ^= 1u << slot;
-        ++R.ready;
-        all_ok = __all_sync(kFull, ok) && all_ok;
-    }
-    return all_ok;
-}
-
-// Row and column of this lane's next 8 outputs (aligned layouts only).
-struct RowCursor {
-    uint32_t row;
-    uint32_t col;
-};
-
-template <int DT>
-__device__ __forceinline__ void store8_aligned(const MatJob &M, uint64_t idx, const RowCursor &rc,
-                                               const uint32_t (&sy)[8]) {
-    const float sc = __ldg(M.scales + rc.row);
-    uint4 o;
-    o.x = pack_bf16x2(__fmul_rn(symbol_value<DT>(sy[0]), sc), __fmul_rn(symbol_value<DT>(sy[1]), sc));
-    o.y = pack_bf16x2(__fmul_rn(symbol_value<DT>(sy[2]), sc), __fmul_rn(symbol_value<DT>(sy[3]), sc));
-    o.z = pack_bf16x2(__fmul_rn(symbol_value<DT>(sy[4]), sc), __fmul_rn(symbol_value<DT>(sy[5]), sc));
-    o.w = pack_bf16x2(__fmul_rn(symbol_value<DT>(sy[6]), sc), __fmul_rn(symbol_value<DT>(sy[7]), sc));
-    *reinterpret_cast<uint4 *>(M.out + idx) = o;
-}
-
-// Element-wise store of up to 8 outputs starting at idx (ragged shapes and tails).
-template <int DT>
-__device__ __forceinline__ void store8_generic(const MatJob &M, uint64_t idx, uint32_t count,
-                                               const uint32_t (&sy)[8]) {
-#pragma unroll
-    for (uint32_t r = 0; r < 8; ++r) {
-        if (r < count) {
-            const uint64_t i = idx + r;
-            const float sc = __ldg(M.scales + i / M.cols);
-            M.out[i] = to_bf16(__fmul_rn(symbol_value<DT>(sy[r]), sc));
+    uint32_t need = (pw + kSegBytes - 1) / kSegBytes;  // last segment touched by bytes [pw, pw + 512)
+    if (need >= n_segs) need = n_segs - 1;
+    bool ok = true;
+    while (ready <= need && ready < issued) {
+        const uint32_t slot = ready % kRingSegs;
+        const bool got = mbar_wait_bounded(mbar + 8 * slot, (phase >> slot) & 1u);
+        phase ^= 1u << slot;
+        ++ready;
+        if (!__all_sync(kFull, got)) {
+            ok = false;
+            break;
         }
     }
-}
-
-__device__ __forceinline__ void advance(RowCursor &rc, uint32_t cols) {
-    rc.col += kGroupSyms;
-    while (rc.col >= cols) {
-        rc.col -= cols;
-        ++rc.row;
+    __syncwarp();
+    if (lane == 0) {
+        ctl->issued = issued;
+        ctl->ready = ready;
+        ctl->phase = phase;
+        if (!ok) ctl->dead = 1;
     }
+    __syncwarp();
+    return ok ? ring_limit(n_segs, issued, ready) : kNoLimit;
 }
 
-// One full 256-symbol group: 8 steps of all 32 lanes.
-__device__ __forceinline__ void decode_group(const WarpSmem &S, uint32_t &x, uint32_t &p, uint32_t lt,
-                                             uint32_t (&sy)[8]) {
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const uint32_t e = S.lut[x & (kProbTotal - 1)];
-        x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xFFFu);
-        sy[r] = e & 0xFFu;
-        const bool need = x < kStateLow;
-        const uint32_t b = __ballot_sync(kFull, need);
-        if (need) x = (x << 16) | S.ring[(p + __popc(b & lt)) & (kRingWords - 1)];
-        p += __popc(b);
+// Wait (bounded) for every copy still in flight so the ring can be reused.
+__device__ __noinline__ bool ring_drain(RingCtl *ctl, uint32_t mbar) {
+    const uint32_t lane = threadIdx.x & 31u;
+    uint32_t ready = ctl->ready, phase = ctl->phase;
+    const uint32_t issued = ctl->issued;
+    bool all_ok = true;
+    while (ready < issued) {
+        const uint32_t slot = ready % kRingSegs;
+        const bool got = mbar_wait_bounded(mbar + 8 * slot, (phase >> slot) & 1u);
+        phase ^= 1u << slot;
+        ++ready;
+        all_ok = __all_sync(kFull, got) && all_ok;
     }
+    __syncwarp();
+    if (lane == 0) {
+        ctl->ready = ready;
+        ctl->phase = phase;
+        if (!all_ok) ctl->dead = 1;
+    }
+    __syncwarp();
+    return all_ok && !ctl->dead;
 }
 
-// The last, partial group: lane l is active at step r while 8l + r < rem.
-__device__ __forceinline__ void decode_tail(const WarpSmem &S, uint32_t &x, uint32_t &p, uint32_t lt,
-                                            uint32_t lane, uint32_t rem, uint32_t (&sy)[8]) {
+// ---- the rANS step ---------------------------------------------------------------
+// One step of all 32 lanes.  `ring` is the warp's 2 KB-aligned shared ring;
+// `pw` counts payload bytes consumed (2 per word).  Returns the slot entry
+// (its low byte is the decoded symbol).
+__device__ __forceinline__ uint32_t rans_step(const uint32_t *lut, uint32_t ring, uint32_t &x, uint32_t &pw,
+                                              uint32_t lt) {
+    const uint32_t e = lut[x & (kProbTotal - 1)];
+    x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xFFFu);
+    const bool need = x < kStateLow;
+    const uint32_t b = __ballot_sync(kFull, need);
+    const uint32_t w = lds_u16(ring | ((pw + 2u * __popc(b & lt)) & (kRingBytes - 1)));
+    x = need ? ((x << 16) | w) : x;
+    pw += 2u * __popc(b);
+    return e;
+}
+
+// Last, partial group: lane l is active at step r while 8l + r < rem.
+__device__ __forceinline__ void rans_tail(const uint32_t *lut, uint32_t ring, uint32_t &x, uint32_t &pw, uint32_t lt,
+                                          uint32_t lane, uint32_t rem, uint32_t (&e8)[8]) {
 #pragma unroll
     for (uint32_t r = 0; r < 8; ++r) {
         const bool active = lane * kGroup + r < rem;
         bool need = false;
         if (active) {
-            const uint32_t e = S.lut[x & (kProbTotal - 1)];
+            const uint32_t e = lut[x & (kProbTotal - 1)];
             x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xFFFu);
-            sy[r] = e & 0xFFu;
+            e8[r] = e;
             need = x < kStateLow;
         }
         const uint32_t b = __ballot_sync(kFull, need);
-        if (need) x = (x << 16) | S.ring[(p + __popc(b & lt)) & (kRingWords - 1)];
-        p += __popc(b);
+        const uint32_t w = lds_u16(ring | ((pw + 2u * __popc(b & lt)) & (kRingBytes - 1)));
+        if (need) x = (x << 16) | w;
+        pw += 2u * __popc(b);
     }
 }
 
-// Returns false only if a bounded wait for staged words gave up: the warp's
-// ring state is then unknown and it must not take further chunks.
-template <int DT, bool ALIGNED>
-__device__ __forceinline__ bool decode_chunk(const DecodeParams &P, const MatJob &M, uint32_t k, WarpSmem &S, uint32_t &phase,
-                             uint32_t lane, uint32_t lt) {
+// Element-wise store of `count` outputs starting at linear index idx.
+template <int DT>
+__device__ __forceinline__ void store_elems(const MatJob &M, uint64_t idx, uint32_t count, const uint32_t (&e8)[8]) {
+#pragma unroll
+    for (uint32_t r = 0; r < 8; ++r) {
+        if (r < count) {
+            const uint64_t i = idx + r;
+            M.out[i] = to_bf16(dequant1<DT>(e8[r], __ldg(M.scales + i / M.cols)));
+        }
+    }
+}
+
+// Output bookkeeping for one chunk.  kRowUniform keeps the (warp-uniform) row
+// of the current 256-symbol group; kLaneRows keeps each lane's own row/col.
+struct Cursor {
+    uint32_t row, col;
+    float scale;
+};
+
+template <int DT, uint32_t LAYOUT>
+__device__ __forceinline__ void cursor_init(const MatJob &M, uint64_t first, uint32_t lane, Cursor &c) {
+    if constexpr (LAYOUT == kRowUniform) {
+        c.row = (uint32_t)(first / M.cols);
+        c.col = (uint32_t)(first - (uint64_t)c.row * M.cols);
+    } else if constexpr (LAYOUT == kLaneRows) {
+        const uint64_t e0 = first + kGroup * lane;
+        c.row = (uint32_t)(e0 / M.cols);
+        c.col = (uint32_t)(e0 - (uint64_t)c.row * M.cols);
+    }
+    if constexpr (LAYOUT != kGeneric) {
+        float s = __ldg(M.scales + c.row);
+        if (DT == EQ_E4M3 && M.small_scales) s *= 0x1p120f;
+        c.scale = s;
+    }
+}
+
+// Move the cursor to the next 256-symbol group (idx: this lane's current first output).
+template <int DT, uint32_t LAYOUT>
+__device__ __forceinline__ void cursor_advance(const MatJob &M, uint64_t idx, Cursor &c) {
+    bool moved = false;
+    c.col += kGroupSyms;
+    while (c.col >= M.cols) {
+        c.col -= M.cols;
+        ++c.row;
+        moved = true;
+    }
+    if (moved && idx + kGroupSyms < M.n_elems) {
+        float s = __ldg(M.scales + c.row);
+        if (DT == EQ_E4M3 && M.small_scales) s *= 0x1p120f;
+        c.scale = s;
+    }
+}
+
+template <int DT, uint32_t LAYOUT>
+__device__ __forceinline__ void group_store(const MatJob &M, uint16_t *dst, uint64_t idx, Cursor &c,
+                                            const uint32_t (&e8)[8]) {
+    if constexpr (LAYOUT == kGeneric) {
+        store_elems<DT>(M, idx, 8, e8);
+    } else {
+        st_global_v4(dst, dequant8<DT>(e8, c.scale, M.small_scales != 0));
+        cursor_advance<DT, LAYOUT>(M, idx, c);
+    }
+}
+
+// Decode one chunk whose slot table is ready in `lut` (n_present >= 2) or
+// whose single symbol is `single` (n_present == 1).  Returns false if a
+// bounded wait gave up (the warp must stop).
+template <int DT, uint32_t LAYOUT>
+__device__ __forceinline__ bool decode_body(const DecodeParams &P, const MatJob &M, uint64_t first, uint32_t n,
+                                            uint32_t n_words, const uint8_t *payload, bool single_sym,
+                                            uint32_t single, uint32_t x, const uint32_t *lut, uint32_t ring,
+                                            uint32_t mbar, RingCtl *ctl, uint32_t lane, uint32_t lt) {
+    const uint32_t n_full = n / kGroupSyms;
+    const uint32_t tail = n % kGroupSyms;
+    Cursor cur{0, 0, 0.f};
+    cursor_init<DT, LAYOUT>(M, first, lane, cur);
+    uint16_t *dst = M.out + first + kGroup * lane;
+
+    if (single_sym) {
+        // f = 4096: the states never change and there are no words
+        if (n_words != 0 || !__all_sync(kFull, x == kStateLow)) {
+            flag(P.status, EQ_DEV_BAD_END);
+            return true;
+        }
+        uint32_t e8[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) e8[r] = single;
+        for (uint32_t g = 0; g < n_full; ++g, dst += kGroupSyms)
+            group_store<DT, LAYOUT>(M, dst, first + (uint64_t)g * kGroupSyms + kGroup * lane, cur, e8);
+        if (tail) {
+            const uint32_t mine = tail > kGroup * lane ? min(8u, tail - kGroup * lane) : 0u;
+            store_elems<DT>(M, first + (uint64_t)n_full * kGroupSyms + kGroup * lane, mine, e8);
+        }
+        return true;
+    }
+
+    const uint32_t pbytes = (2u * n_words + 15u) & ~15u;
+    if (lane == 0) {
+        ctl->payload = payload;
+        ctl->pbytes = pbytes;
+        ctl->n_segs = (pbytes + kSegBytes - 1) / kSegBytes;
+        ctl->issued = 0;
+        ctl->ready = 0;
+    }
+    __syncwarp();
+    uint32_t limit = pbytes ? 0u : kNoLimit;
+    uint32_t pw = 0;
+    for (uint32_t g = 0; g < n_full; ++g, dst += kGroupSyms) {
+        if (pw >= limit) {
+            limit = ring_service(ctl, ring, mbar, pw);
+            if (ctl->dead) break;
+        }
+        if constexpr (LAYOUT == kGeneric) {
+            uint32_t e8[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) e8[r] = rans_step(lut, ring, x, pw, lt);
+            store_elems<DT>(M, first + (uint64_t)g * kGroupSyms + kGroup * lane, 8, e8);
+        } else {
+            // dequantise pairs as they are decoded: 4 packed registers instead of 8 entries
+            const float2 s2 = make_float2(cur.scale, cur.scale);
+            uint32_t o[4];
+#pragma unroll
+            for (int r = 0; r < 8; r += 2) {
+                const uint32_t e0 = rans_step(lut, ring, x, pw, lt);
+                const uint32_t e1 = rans_step(lut, ring, x, pw, lt);
+                float2 v = make_float2(raw_value<DT>(e0), raw_value<DT>(e1));
+                if constexpr (DT == EQ_E4M3) {
+                    if (!M.small_scales) v = mul2_rn(v, make_float2(0x1p120f, 0x1p120f));
+                }
+                o[r / 2] = pack_bf16x2(mul2_rn(v, s2));
+            }
+            st_global_v4(dst, make_uint4(o[0], o[1], o[2], o[3]));
+            cursor_advance<DT, LAYOUT>(M, first + (uint64_t)g * kGroupSyms + kGroup * lane, cur);
+        }
+    }
+    if (tail && !ctl->dead) {
+        if (pw >= limit) limit = ring_service(ctl, ring, mbar, pw);
+        if (!ctl->dead) {
+            uint32_t e8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            rans_tail(lut, ring, x, pw, lt, lane, tail, e8);
+            const uint32_t mine = tail > kGroup * lane ? min(8u, tail - kGroup * lane) : 0u;
+            store_elems<DT>(M, first + (uint64_t)n_full * kGroupSyms + kGroup * lane, mine, e8);
+        }
+    }
+    if (!ring_drain(ctl, mbar)) {
+        flag(P.status, EQ_DEV_TIMEOUT);
+        return false;
+    }
+    // a valid stream returns every state to 2^16 and consumes exactly n_words
+    if (!__all_sync(kFull, x == kStateLow) || pw != 2u * n_words) flag(P.status, EQ_DEV_BAD_END);
+    return true;
+}
+
+// Header of chunk k: checks it against the directory; on success fills the
+// record pointer, counts and this lane's initial state.
+struct ChunkHead {
+    const uint8_t *rec;
+    uint32_t n, n_words, n_present, table_bytes;
+    uint32_t x;
+};
+
+__device__ __forceinline__ bool load_head(const DecodeParams &P, const MatJob &M, uint32_t k, uint32_t lane,
+                                          ChunkHead &h) {
     const uint64_t first = (uint64_t)k * kChunkSyms;
-    const uint64_t rem_all = M.n_elems - first;
-    const uint32_t n_expect = rem_all < kChunkSyms ? (uint32_t)rem_all : kChunkSyms;
+    const uint64_t rem = M.n_elems - first;
+    const uint32_t n_expect = rem < kChunkSyms ? (uint32_t)rem : kChunkSyms;
     const uint64_t off = M.chunk_index[k];
     const uint64_t end = M.chunk_index[k + 1];
     if ((off & 15) || end > P.blob_len || end < off + kRecordHeadBytes + 16) {
         flag(P.status, EQ_DEV_BAD_HEADER);
-        return true;
+        return false;
     }
-    const uint8_t *rec = P.blob + off;
-    const uint4 head = *reinterpret_cast<const uint4 *>(rec);
-    const uint32_t n = head.x, n_words = head.y, n_present = head.z;
-    const uint32_t table_bytes = (kRecordHeadBytes + 4 * n_present + 15) & ~15u;
-    if (n != n_expect || n_present < 1 || n_present > 256 ||
-        off + table_bytes + ((2ull * n_words + 15) & ~15ull) != end) {
+    h.rec = P.blob + off;
+    const uint4 head = *reinterpret_cast<const uint4 *>(h.rec);
+    h.n = head.x;
+    h.n_words = head.y;
+    h.n_present = head.z;
+    h.table_bytes = (kRecordHeadBytes + 4 * h.n_present + 15) & ~15u;
+    if (h.n != n_expect || h.n_present < 1 || h.n_present > 256 ||
+        off + h.table_bytes + ((2ull * h.n_words + 15) & ~15ull) != end) {
         flag(P.status, EQ_DEV_BAD_HEADER);
-        return true;
+        return false;
     }
-    uint32_t x = reinterpret_cast<const uint32_t *>(rec + 16)[lane];
-    if (!__all_sync(kFull, x >= kStateLow)) {
+    h.x = reinterpret_cast<const uint32_t *>(h.rec + 16)[lane];
+    if (!__all_sync(kFull, h.x >= kStateLow)) {
         flag(P.status, EQ_DEV_BAD_STATE);
-        return true;
+        return false;
     }
+    return true;
+}
 
-    // ---- table: check it and expand it into the slot table ----
-    const uint32_t *tab = reinterpret_cast<const uint32_t *>(rec + kRecordHeadBytes);
+// Check a frequency list (n_present entries at `tab`): ascending symbols,
+// reserved bits zero, f >= 1, sum 4096.  Optionally copies the entries and
+// their cumulative frequencies to shared memory, and/or expands the list into
+// a warp's slot table.  Returns validity (warp-uniform).
+__device__ __forceinline__ bool warp_table(const uint32_t *tab, uint32_t n_present, uint32_t lane,
+                                           uint32_t *entries_out, uint32_t *cum_out, uint32_t *lut) {
     uint32_t run = 0;
     int prev_sym = -1;
     bool ok = true;
-    uint32_t single_sym = 0;
     for (uint32_t base = 0; base < n_present; base += 32) {
         const uint32_t i = base + lane;
         const bool have = i < n_present;
@@ -362,139 +576,142 @@ __device__ __forceinline__ bool decode_chunk(const DecodeParams &P, const MatJob
             if (lane >= (uint32_t)d) inc += t;
         }
         const uint32_t cum = run + inc - f;
+        if (have) {
+            if (entries_out) entries_out[i] = e;
+            if (cum_out) cum_out[i] = cum;
+        }
         ok = __all_sync(kFull, good) && ok;
         const uint32_t cnt = min(32u, n_present - base);
-        if (n_present > 1) {
+        if (lut && n_present > 1) {
             for (uint32_t q = 0; q < cnt; ++q) {
                 const uint32_t fq = __shfl_sync(kFull, f, q);
                 const uint32_t cq = __shfl_sync(kFull, cum, q);
                 const uint32_t sq = __shfl_sync(kFull, sym, q);
                 for (uint32_t t = lane; t < fq; t += 32) {
                     const uint32_t slot = cq + t;
-                    if (slot < kProbTotal && fq < kProbTotal) S.lut[slot] = (fq << 20) | (t << 8) | sq;
+                    if (slot < kProbTotal && fq < kProbTotal) lut[slot] = (fq << 20) | (t << 8) | sq;
                 }
             }
-        } else {
-            single_sym = __shfl_sync(kFull, sym, 0);
         }
         prev_sym = __shfl_sync(kFull, (int)sym, cnt - 1);
         run += __shfl_sync(kFull, inc, 31);
     }
-    if (!ok || run != kProbTotal) {
-        flag(P.status, EQ_DEV_BAD_TABLE);
-        return true;
-    }
-
-    const uint32_t n_full = n / kGroupSyms;
-    const uint32_t tail = n % kGroupSyms;
-    RowCursor rc{0, 0};
-    if (ALIGNED) {
-        const uint64_t e0 = first + kGroup * lane;
-        rc.row = (uint32_t)(e0 / M.cols);
-        rc.col = (uint32_t)(e0 - (uint64_t)rc.row * M.cols);
-    }
-
-    // ---- single-symbol chunk: no payload, every state stays at 2^16 ----
-    if (n_present == 1) {
-        if (n_words != 0 || !__all_sync(kFull, x == kStateLow)) {
-            flag(P.status, EQ_DEV_BAD_END);
-            return true;
-        }
-        uint32_t sy[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) sy[r] = single_sym;
-        for (uint32_t g = 0; g < n_full; ++g) {
-            const uint64_t idx = first + (uint64_t)g * kGroupSyms + kGroup * lane;
-            if (ALIGNED) {
-                store8_aligned<DT>(M, idx, rc, sy);
-                advance(rc, M.cols);
-            } else {
-                store8_generic<DT>(M, idx, 8, sy);
-            }
-        }
-        if (tail) {
-            const uint32_t mine = tail > kGroup * lane ? min(8u, tail - kGroup * lane) : 0u;
-            store8_generic<DT>(M, first + (uint64_t)n_full * kGroupSyms + kGroup * lane, mine, sy);
-        }
-        return true;
-    }
-
-    // ---- stream the words and decode ----
-    __syncwarp();
-    Ring R;
-    R.payload = rec + table_bytes;
-    R.pbytes = (2u * n_words + 15u) & ~15u;
-    R.n_segs = (R.pbytes + kSegBytes - 1) / kSegBytes;
-    R.issued = 0;
-    R.ready = 0;
-    R.phase = phase;
-
-    uint32_t p = 0;
-    bool alive = true;
-    for (uint32_t g = 0; g < n_full; ++g) {
-        if (!ring_prepare(S, R, p, lane)) {
-            alive = false;
-            break;
-        }
-        uint32_t sy[8];
-        decode_group(S, x, p, lt, sy);
-        const uint64_t idx = first + (uint64_t)g * kGroupSyms + kGroup * lane;
-        if (ALIGNED) {
-            store8_aligned<DT>(M, idx, rc, sy);
-            advance(rc, M.cols);
-        } else {
-            store8_generic<DT>(M, idx, 8, sy);
-        }
-    }
-    if (alive && tail) {
-        if (!ring_prepare(S, R, p, lane)) {
-            alive = false;
-        } else {
-            uint32_t sy[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            decode_tail(S, x, p, lt, lane, tail, sy);
-            const uint32_t mine = tail > kGroup * lane ? min(8u, tail - kGroup * lane) : 0u;
-            store8_generic<DT>(M, first + (uint64_t)n_full * kGroupSyms + kGroup * lane, mine, sy);
-        }
-    }
-    const bool drained = ring_drain(S, R);
-    phase = R.phase;
-    if (!alive || !drained) {
-        flag(P.status, EQ_DEV_TIMEOUT);
-        return false;
-    }
-    // a valid stream returns every state to 2^16 and consumes exactly n_words
-    if (!__all_sync(kFull, x == kStateLow) || p != n_words) flag(P.status, EQ_DEV_BAD_END);
-    return true;
+    return ok && run == kProbTotal;
 }
 
-__global__ void __launch_bounds__(kThreads) eq_rans_decode_dequant_kernel(const __grid_constant__ DecodeParams P) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
+// Shared memory of one block.  Rings start on a 2 KB boundary so a ring
+// address is (ring base | byte offset).
+template <int WARPS, bool SHARED>
+struct Smem {
+    static constexpr uint32_t kLuts = SHARED ? 1 : WARPS;
+    static constexpr uint32_t kRingOff = kLuts * kLutBytes;             // + runtime pad to 2 KB
+    static constexpr uint32_t kMbarOff = kRingOff + WARPS * kRingBytes; // all offsets below include the pad
+    static constexpr uint32_t kCtlOff = kMbarOff + WARPS * kRingSegs * 8;
+    static constexpr uint32_t kRefOff = kCtlOff + WARPS * 32;           // 32 bytes of RingCtl per warp
+    static constexpr uint32_t kBlockOff = kRefOff + (SHARED ? 2 * 256 * 4 : 0);
+    static constexpr uint32_t kBytes = kBlockOff + 16 + kRingBytes;     // + worst-case alignment pad
+};
+static_assert(sizeof(RingCtl) <= 32, "RingCtl slot");
+
+template <int WARPS, bool SHARED, int DT, uint32_t LAYOUT>
+__global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
+    eq_decode_kernel(const __grid_constant__ DecodeParams P) {
+    using L = Smem<WARPS, SHARED>;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = threadIdx.x >> 5;
-    WarpSmem &S = reinterpret_cast<WarpSmem *>(smem_raw)[warp];
+    const uint32_t base = smem_u32(smem_raw);
+    const uint32_t pad = (kRingBytes - ((base + L::kRingOff) & (kRingBytes - 1))) & (kRingBytes - 1);
+    unsigned char *padded = smem_raw + pad;  // offsets from kRingOff on are relative to this
+    const uint32_t ring = base + pad + L::kRingOff + warp * kRingBytes;
+    const uint32_t mbar = base + pad + L::kMbarOff + warp * kRingSegs * 8;
+    RingCtl *ctl = reinterpret_cast<RingCtl *>(padded + L::kCtlOff + warp * 32);
+    uint32_t *lut = reinterpret_cast<uint32_t *>(smem_raw) + (SHARED ? 0u : warp * kProbTotal);
     if (lane == 0) {
-        for (uint32_t i = 0; i < kRingSegs; ++i) mbar_init(&S.mbar[i], 1);
+        for (uint32_t i = 0; i < kRingSegs; ++i) mbar_init(mbar + 8 * i, 1);
         fence_mbar_init();
+        ctl->phase = 0;
+        ctl->dead = 0;
+        ctl->issued = ctl->ready = 0;
     }
     __syncwarp();
     const uint32_t lt = lanemask_lt();
-    uint32_t phase = 0;
-    const uint32_t stride = gridDim.x * kWarpsPerCta;
-    for (uint32_t c = blockIdx.x * kWarpsPerCta + warp; c < P.total_chunks; c += stride) {
-        uint32_t mi = 0;
-        while (mi + 1 < P.n_mats && c >= P.mats[mi + 1].chunk_begin) ++mi;
-        const MatJob &M = P.mats[mi];
-        const uint32_t k = c - M.chunk_begin;
-        bool go;
-        if (M.dtype == EQ_INT8) {
-            go = M.aligned ? decode_chunk<EQ_INT8, true>(P, M, k, S, phase, lane, lt)
-                           : decode_chunk<EQ_INT8, false>(P, M, k, S, phase, lane, lt);
-        } else {
-            go = M.aligned ? decode_chunk<EQ_E4M3, true>(P, M, k, S, phase, lane, lt)
-                           : decode_chunk<EQ_E4M3, false>(P, M, k, S, phase, lane, lt);
+
+    if constexpr (SHARED) {
+        uint32_t *ref_entries = reinterpret_cast<uint32_t *>(padded + L::kRefOff);
+        uint32_t *ref_cum = ref_entries + 256;
+        volatile uint32_t *blk = reinterpret_cast<uint32_t *>(padded + L::kBlockOff);  // [0] n_present, [1] valid
+        uint32_t cur_mat = kNoLimit;
+        for (uint32_t unit = blockIdx.x; unit < P.total_units; unit += gridDim.x) {
+            uint32_t mi = 0;
+            while (mi + 1 < P.n_mats && unit >= P.mats[mi + 1].begin) ++mi;
+            const MatJob &M = P.mats[mi];
+            const uint32_t k0 = (unit - M.begin) * WARPS;
+            if (mi != cur_mat) {
+                // rebuild the block's slot table from the tile's first chunk
+                __syncthreads();
+                if (warp == 0) {
+                    ChunkHead h;
+                    bool ok = load_head(P, M, k0, lane, h);
+                    if (ok) ok = warp_table(reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes), h.n_present,
+                                            lane, ref_entries, ref_cum, nullptr);
+                    if (lane == 0) {
+                        blk[0] = ok ? h.n_present : 0u;
+                        blk[1] = ok;
+                    }
+                }
+                __syncthreads();
+                const uint32_t np = blk[0];
+                if (blk[1] && np > 1) {
+                    for (uint32_t i = 0; i < np; ++i) {
+                        const uint32_t e = ref_entries[i], c = ref_cum[i];
+                        const uint32_t f = e >> 16, sy = e & 0xFFu;
+                        for (uint32_t t = threadIdx.x; t < f; t += WARPS * 32)
+                            if (c + t < kProbTotal && f < kProbTotal) lut[c + t] = (f << 20) | (t << 8) | sy;
+                    }
+                }
+                __syncthreads();
+                cur_mat = mi;
+            }
+            const uint32_t k = k0 + warp;
+            if (k >= M.n_chunks || ctl->dead) continue;
+            ChunkHead h;
+            if (!load_head(P, M, k, lane, h)) continue;
+            const uint32_t np = blk[0];
+            bool same = blk[1] && h.n_present == np;
+            if (same) {
+                const uint32_t *tab = reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes);
+                for (uint32_t i = lane; i < np; i += 32) same = same && tab[i] == ref_entries[i];
+            }
+            if (!__all_sync(kFull, same)) {
+                flag(P.status, EQ_DEV_BAD_TABLE);
+                continue;
+            }
+            decode_body<DT, LAYOUT>(P, M, (uint64_t)k * kChunkSyms, h.n, h.n_words, h.rec + h.table_bytes, np == 1,
+                                    ref_entries[0] & 0xFFu, h.x, lut, ring, mbar, ctl, lane, lt);
+            __syncwarp();
         }
-        __syncwarp();
-        if (!go) break;
+    } else {
+        const uint32_t stride = gridDim.x * WARPS;
+        for (uint32_t c = blockIdx.x * WARPS + warp; c < P.total_units && !ctl->dead; c += stride) {
+            uint32_t mi = 0;
+            while (mi + 1 < P.n_mats && c >= P.mats[mi + 1].begin) ++mi;
+            const MatJob &M = P.mats[mi];
+            const uint32_t k = c - M.begin;
+            ChunkHead h;
+            if (!load_head(P, M, k, lane, h)) continue;
+            const uint32_t *tab = reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes);
+            __syncwarp();  // the previous chunk's reads of the slot table are done
+            const bool ok = warp_table(tab, h.n_present, lane, nullptr, nullptr, lut);
+            if (!ok) {
+                flag(P.status, EQ_DEV_BAD_TABLE);
+                continue;
+            }
+            __syncwarp();
+            decode_body<DT, LAYOUT>(P, M, (uint64_t)k * kChunkSyms, h.n, h.n_words, h.rec + h.table_bytes,
+                                    h.n_present == 1, tab[0] & 0xFFu, h.x, lut, ring, mbar, ctl, lane, lt);
+            __syncwarp();
+        }
     }
 }
 
@@ -516,13 +733,47 @@ __global__ void eq_outlier_scatter_kernel(const __grid_constant__ ScatterParams 
 
 // ---- host side ---------------------------------------------------------------------
 
+using KernelFn = void (*)(DecodeParams);
+
+struct KernelSetup {
+    KernelFn fn = nullptr;
+    int warps = 0;
+    size_t smem = 0;
+    int ctas_per_sm = 0;
+    uint32_t units_per_cta = 0;  // work units (tiles or chunks) a block takes per round
+};
+
+// variants: [shared][dtype - 1][layout]
 struct DeviceSetup {
     bool ready = false;
     int sms = 0;
-    int ctas_per_sm = 0;
+    KernelSetup k[2][2][3];
 };
 std::mutex g_setup_mu;
 DeviceSetup g_setup[128];
+
+int setup_kernel(KernelSetup &k, KernelFn fn, int warps, size_t smem, uint32_t units_per_cta) {
+    k.fn = fn;
+    k.warps = warps;
+    k.smem = smem;
+    k.units_per_cta = units_per_cta;
+    if (cudaFuncSetAttribute(reinterpret_cast<const void *>(fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return EQ_ERR_CUDA;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&k.ctas_per_sm, fn, warps * 32, smem) != cudaSuccess ||
+        k.ctas_per_sm < 1)
+        return EQ_ERR_CUDA;
+    return EQ_OK;
+}
+
+template <int DT, uint32_t LAYOUT>
+int setup_pair(DeviceSetup &d) {
+    int rc = setup_kernel(d.k[1][DT - 1][LAYOUT], eq_decode_kernel<kSharedWarps, true, DT, LAYOUT>, kSharedWarps,
+                          Smem<kSharedWarps, true>::kBytes, 1);
+    if (rc) return rc;
+    return setup_kernel(d.k[0][DT - 1][LAYOUT], eq_decode_kernel<kPrivateWarps, false, DT, LAYOUT>, kPrivateWarps,
+                        Smem<kPrivateWarps, false>::kBytes, kPrivateWarps);
+}
 
 int device_setup(DeviceSetup **out) {
     int dev = 0;
@@ -531,20 +782,36 @@ int device_setup(DeviceSetup **out) {
     DeviceSetup &d = g_setup[dev];
     if (!d.ready) {
         if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return EQ_ERR_CUDA;
-        if (cudaFuncSetAttribute(eq_rans_decode_dequant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kSmemBytes) != cudaSuccess)
-            return EQ_ERR_CUDA;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.ctas_per_sm, eq_rans_decode_dequant_kernel, kThreads,
-                                                          kSmemBytes) != cudaSuccess ||
-            d.ctas_per_sm < 1)
-            return EQ_ERR_CUDA;
+        int rc;
+        if ((rc = setup_pair<EQ_INT8, kRowUniform>(d)) || (rc = setup_pair<EQ_INT8, kLaneRows>(d)) ||
+            (rc = setup_pair<EQ_INT8, kGeneric>(d)) || (rc = setup_pair<EQ_E4M3, kRowUniform>(d)) ||
+            (rc = setup_pair<EQ_E4M3, kLaneRows>(d)) || (rc = setup_pair<EQ_E4M3, kGeneric>(d)))
+            return rc;
         d.ready = true;
     }
     *out = &d;
     return EQ_OK;
 }
 
-// Decode matrices [first, first + count) of the model into outs[i].
+uint32_t layout_of(const eq_matrix_info &in, const uint16_t *out) {
+    const bool aligned = reinterpret_cast<uintptr_t>(out) % 16 == 0;
+    if (aligned && in.cols % kGroupSyms == 0) return kRowUniform;
+    if (aligned && in.cols % kGroup == 0) return kLaneRows;
+    return kGeneric;
+}
+
+int launch(const KernelSetup &k, int sms, const DecodeParams &P, cudaStream_t s) {
+    if (!P.total_units) return EQ_OK;
+    const uint32_t resident = (uint32_t)(sms * k.ctas_per_sm);
+    const uint32_t want = (P.total_units + k.units_per_cta - 1) / k.units_per_cta;
+    const uint32_t grid = std::min(want, resident);
+    k.fn<<<grid, k.warps * 32, k.smem, s>>>(P);
+    return cudaGetLastError() == cudaSuccess ? EQ_OK : EQ_ERR_CUDA;
+}
+
+// Decode matrices [first, first + count) of the model into outs[i]: one
+// launch per kernel variant (table scope x dtype x layout) present, then one
+// scatter launch for the super weights.
 int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *const *outs, int32_t *d_status,
                   cudaStream_t s) {
     DeviceSetup *dev = nullptr;
@@ -552,27 +819,36 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
     if (rc) return rc;
     for (uint32_t base = 0; base < count; base += kMaxMatsPerLaunch) {
         const uint32_t cnt = std::min<uint32_t>(kMaxMatsPerLaunch, count - base);
-        DecodeParams P{};
-        P.blob = m->d_blob;
-        P.blob_len = m->len;
-        P.status = d_status;
+        DecodeParams P[2][2][3];
+        for (auto &a : P)
+            for (auto &b : a)
+                for (auto &c : b) {
+                    c = DecodeParams{};
+                    c.blob = m->d_blob;
+                    c.blob_len = m->len;
+                    c.status = d_status;
+                }
         ScatterParams Q{};
         Q.status = d_status;
-        uint32_t chunks = 0, n_out = 0;
+        uint32_t n_out = 0;
         for (uint32_t i = 0; i < cnt; ++i) {
             const MatrixDesc &d = m->mats[first + base + i];
             if (d.info.n_chunks == 0) continue;
-            MatJob &J = P.mats[P.n_mats++];
+            const int sh = d.info.uniform_table ? 1 : 0;
+            const uint32_t lay = layout_of(d.info, outs[base + i]);
+            DecodeParams &Pv = P[sh][d.info.dtype - 1][lay];
+            MatJob &J = Pv.mats[Pv.n_mats++];
             J.chunk_index = reinterpret_cast<const uint64_t *>(m->d_blob + d.chunk_index_off);
             J.scales = reinterpret_cast<const float *>(m->d_blob + d.scales_off);
             J.out = outs[base + i];
             J.n_elems = (uint64_t)d.info.rows * d.info.cols;
             J.cols = d.info.cols;
             J.n_chunks = d.info.n_chunks;
-            J.chunk_begin = chunks;
+            J.begin = Pv.total_units;
             J.dtype = d.info.dtype;
-            J.aligned = (d.info.cols % kGroup == 0) && (reinterpret_cast<uintptr_t>(J.out) % 16 == 0);
-            chunks += d.info.n_chunks;
+            J.layout = lay;
+            J.small_scales = d.small_scales ? 1u : 0u;
+            Pv.total_units += sh ? (d.info.n_chunks + kSharedWarps - 1) / kSharedWarps : d.info.n_chunks;
             if (d.info.n_outliers) {
                 ScatterJob &O = Q.jobs[Q.n_jobs++];
                 O.rec = reinterpret_cast<const uint32_t *>(m->d_blob + d.outliers_off);
@@ -584,14 +860,11 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
                 n_out += d.info.n_outliers;
             }
         }
-        P.total_chunks = chunks;
         Q.total = n_out;
-        if (chunks) {
-            const uint32_t want = (chunks + kWarpsPerCta - 1) / kWarpsPerCta;
-            const uint32_t grid = std::min<uint32_t>(want, (uint32_t)(dev->sms * dev->ctas_per_sm));
-            eq_rans_decode_dequant_kernel<<<grid, kThreads, kSmemBytes, s>>>(P);
-            if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
-        }
+        for (int sh = 0; sh < 2; ++sh)
+            for (int dt = 0; dt < 2; ++dt)
+                for (int lay = 0; lay < 3; ++lay)
+                    if ((rc = launch(dev->k[sh][dt][lay], dev->sms, P[sh][dt][lay], s))) return rc;
         if (n_out) {
             eq_outlier_scatter_kernel<<<(n_out + 127) / 128, 128, 0, s>>>(Q);
             if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
@@ -617,21 +890,15 @@ extern "C" EQW_API int eq_decode_block(const eq_model *m, uint32_t layer, void *
                                        int32_t *d_status, cudaStream_t s) {
     if (!m || !d_status || layer >= m->n_layers) return EQ_ERR_INVALID_ARG;
     const uint32_t first = m->layer_first[layer], count = m->layer_count[layer];
-    size_t offs[256];
-    std::vector<size_t> big;
-    size_t *o = offs;
-    if (count > 256) {
-        big.resize(count);
-        o = big.data();
-    }
+    std::vector<size_t> offs(count);
     size_t total = 0;
-    int rc = eq_block_layout(m, layer, o, count, &total);
+    int rc = eq_block_layout(m, layer, offs.data(), count, &total);
     if (rc) return rc;
     if (total && (!d_out || reinterpret_cast<uintptr_t>(d_out) % 16)) return EQ_ERR_INVALID_ARG;
     if (out_bytes < total) return EQ_ERR_NOSPACE;
     std::vector<uint16_t *> outs(count);
     for (uint32_t i = 0; i < count; ++i)
-        outs[i] = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(d_out) + o[i]);
+        outs[i] = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(d_out) + offs[i]);
     return launch_decode(m, first, count, outs.data(), d_status, s);
 }
 

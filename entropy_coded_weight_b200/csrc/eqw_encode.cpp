@@ -10,6 +10,7 @@
 // decode independently); each chunk gets its own 12-bit frequency table and
 // 32 interleaved rANS states.  Chunks are encoded in parallel on host threads.
 #include <algorithm>
+#include <array>
 #include <atomic>
 #include <cmath>
 #include <cstring>
@@ -29,7 +30,7 @@ namespace {
 // present symbol), then move single units greedily where they cost the fewest
 // expected bits: adding one unit to s saves cnt_s * log2((f+1)/f) bits,
 // removing one costs cnt_s * log2(f/(f-1)).
-void quantize_table(const uint32_t cnt[256], uint32_t n, uint32_t f[256]) {
+void quantize_table(const uint64_t cnt[256], uint64_t n, uint32_t f[256]) {
     int present[256];
     int np = 0;
     int64_t sum = 0;
@@ -71,11 +72,17 @@ void quantize_table(const uint32_t cnt[256], uint32_t n, uint32_t f[256]) {
 // The decoder walks steps upward and lanes upward inside a step, so the encoder
 // walks both downward and writes each renormalisation word in front of the
 // previous one.
-void encode_record(const uint8_t *sym, uint32_t n, std::vector<uint8_t> &rec, std::vector<uint16_t> &scratch) {
-    uint32_t cnt[256] = {0};
-    for (uint32_t j = 0; j < n; ++j) ++cnt[sym[j]];
+// `table` is the matrix-wide frequency table, or null to quantise this chunk's own histogram.
+void encode_record(const uint8_t *sym, uint32_t n, const uint32_t *table, std::vector<uint8_t> &rec,
+                   std::vector<uint16_t> &scratch) {
     uint32_t f[256], cum[256];
-    quantize_table(cnt, n, f);
+    if (table) {
+        std::memcpy(f, table, sizeof f);
+    } else {
+        uint64_t cnt[256] = {0};
+        for (uint32_t j = 0; j < n; ++j) ++cnt[sym[j]];
+        quantize_table(cnt, n, f);
+    }
     uint32_t c = 0;
     uint32_t n_present = 0;
     for (int s = 0; s < 256; ++s) {
@@ -139,6 +146,7 @@ int validate(const eq_matrix_in *mats, uint32_t n_mats, uint32_t *n_layers) {
     for (uint32_t i = 0; i < n_mats; ++i) {
         const eq_matrix_in &m = mats[i];
         if (m.dtype != EQ_INT8 && m.dtype != EQ_E4M3) return EQ_ERR_INVALID_ARG;
+        if (m.flags & ~EQ_TABLE_PER_CHUNK) return EQ_ERR_INVALID_ARG;
         const uint64_t n = (uint64_t)m.rows * m.cols;
         if (n && (!m.symbols || !m.scales)) return EQ_ERR_INVALID_ARG;
         if ((n + kChunkSyms - 1) / kChunkSyms > 0xFFFFFFFFull) return EQ_ERR_INVALID_ARG;
@@ -196,37 +204,77 @@ extern "C" EQW_API int eq_encoder_run(const eq_matrix_in *mats, uint32_t n_mats,
         for (uint32_t k = 0; k < n_chunks[d]; ++k) jobs.push_back({d, k});
     }
 
-    std::vector<std::vector<uint8_t>> records(jobs.size());
-    std::atomic<size_t> next{0};
-    auto worker = [&]() {
-        std::vector<uint16_t> scratch;
-        std::vector<uint8_t> patched;
-        for (;;) {
-            const size_t i = next.fetch_add(1);
-            if (i >= jobs.size()) break;
-            const eq_matrix_in &m = mats[order[jobs[i].mat]];
-            const uint64_t n = (uint64_t)m.rows * m.cols;
-            const uint64_t first = (uint64_t)jobs[i].chunk * kChunkSyms;
-            const uint32_t len = (uint32_t)std::min<uint64_t>(kChunkSyms, n - first);
-            const uint8_t *src = m.symbols + first;
-            if (m.n_out) {
-                // super weights travel outside the stream: code the placeholder 0
-                patched.assign(src, src + len);
-                for (uint32_t k = 0; k < m.n_out; ++k) {
-                    const uint64_t lin = (uint64_t)m.out_row[k] * m.cols + m.out_col[k];
-                    if (lin >= first && lin < first + len) patched[lin - first] = 0;
-                }
-                src = patched.data();
-            }
-            encode_record(src, len, records[i], scratch);
+    // the symbols of chunk i, with super weights replaced by the placeholder 0
+    auto chunk_symbols = [&](size_t i, std::vector<uint8_t> &patched, uint32_t *len_out) -> const uint8_t * {
+        const eq_matrix_in &m = mats[order[jobs[i].mat]];
+        const uint64_t n = (uint64_t)m.rows * m.cols;
+        const uint64_t first = (uint64_t)jobs[i].chunk * kChunkSyms;
+        const uint32_t len = (uint32_t)std::min<uint64_t>(kChunkSyms, n - first);
+        *len_out = len;
+        const uint8_t *src = m.symbols + first;
+        if (!m.n_out) return src;
+        patched.assign(src, src + len);
+        for (uint32_t k = 0; k < m.n_out; ++k) {
+            const uint64_t lin = (uint64_t)m.out_row[k] * m.cols + m.out_col[k];
+            if (lin >= first && lin < first + len) patched[lin - first] = 0;
         }
+        return patched.data();
     };
-    unsigned nt = n_threads > 0 ? (unsigned)n_threads : std::max(1u, std::thread::hardware_concurrency());
-    nt = (unsigned)std::min<size_t>(nt, std::max<size_t>(1, jobs.size()));
-    std::vector<std::thread> pool;
-    for (unsigned t = 1; t < nt; ++t) pool.emplace_back(worker);
-    worker();
-    for (auto &t : pool) t.join();
+    auto run_parallel = [&](auto &&body) {
+        std::atomic<size_t> next{0};
+        auto worker = [&]() {
+            for (;;) {
+                const size_t i = next.fetch_add(1);
+                if (i >= jobs.size()) break;
+                body(i);
+            }
+        };
+        unsigned nt = n_threads > 0 ? (unsigned)n_threads : std::max(1u, std::thread::hardware_concurrency());
+        nt = (unsigned)std::min<size_t>(nt, std::max<size_t>(1, jobs.size()));
+        std::vector<std::thread> pool;
+        for (unsigned t = 1; t < nt; ++t) pool.emplace_back(worker);
+        worker();
+        for (auto &t : pool) t.join();
+    };
+
+    // pass 1 (matrices with one table): histogram of every chunk, summed per matrix
+    std::vector<std::array<uint64_t, 256>> hist(jobs.size());
+    bool any_matrix_table = false;
+    for (uint32_t d = 0; d < n_mats; ++d) any_matrix_table |= !(mats[order[d]].flags & EQ_TABLE_PER_CHUNK);
+    std::vector<std::array<uint32_t, 256>> mat_table(n_mats);
+    if (any_matrix_table) {
+        run_parallel([&](size_t i) {
+            if (mats[order[jobs[i].mat]].flags & EQ_TABLE_PER_CHUNK) return;
+            thread_local std::vector<uint8_t> patched;
+            uint32_t len = 0;
+            const uint8_t *src = chunk_symbols(i, patched, &len);
+            hist[i].fill(0);
+            for (uint32_t j = 0; j < len; ++j) ++hist[i][src[j]];
+        });
+        std::vector<std::array<uint64_t, 256>> total(n_mats);
+        for (auto &t : total) t.fill(0);
+        for (size_t i = 0; i < jobs.size(); ++i)
+            if (!(mats[order[jobs[i].mat]].flags & EQ_TABLE_PER_CHUNK))
+                for (int s = 0; s < 256; ++s) total[jobs[i].mat][s] += hist[i][s];
+        for (uint32_t d = 0; d < n_mats; ++d) {
+            uint64_t n = 0;
+            for (int s = 0; s < 256; ++s) n += total[d][s];
+            if (n) quantize_table(total[d].data(), n, mat_table[d].data());
+        }
+    }
+    hist.clear();
+    hist.shrink_to_fit();
+
+    // pass 2: encode every chunk
+    std::vector<std::vector<uint8_t>> records(jobs.size());
+    run_parallel([&](size_t i) {
+        thread_local std::vector<uint16_t> scratch;
+        thread_local std::vector<uint8_t> patched;
+        uint32_t len = 0;
+        const uint8_t *src = chunk_symbols(i, patched, &len);
+        const bool per_chunk = mats[order[jobs[i].mat]].flags & EQ_TABLE_PER_CHUNK;
+        encode_record(src, len, per_chunk ? nullptr : mat_table[jobs[i].mat].data(), records[i], scratch);
+    });
 
     // layout: header | directory | per matrix: chunk index, scales, outliers, records
     uint64_t pos = align_up(kHeaderBytes + (uint64_t)kDirEntryBytes * n_mats, kSectionAlign);

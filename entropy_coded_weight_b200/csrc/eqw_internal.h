@@ -33,6 +33,7 @@ struct MatrixDesc {
     uint64_t chunk_index_off;
     uint64_t scales_off;
     uint64_t outliers_off;
+    bool small_scales;    // every scale finite with |scale| < 2^8 (E4M3 single-multiply dequant is exact)
 };
 
 }  // namespace eqw

@@ -117,6 +117,8 @@ int parse(const uint8_t *b, size_t len, eq_model *m) {
         }
         uint64_t words = 0;
         const uint64_t first = rd<uint64_t>(b + d.chunk_index_off);
+        in.uniform_table = in.n_chunks > 0;
+        uint32_t np0 = 0;
         for (uint32_t k = 0; k < in.n_chunks; ++k) {
             const uint64_t off = rd<uint64_t>(b + d.chunk_index_off + 8ull * k);
             const uint64_t end = rd<uint64_t>(b + d.chunk_index_off + 8ull * (k + 1));
@@ -127,6 +129,20 @@ int parse(const uint8_t *b, size_t len, eq_model *m) {
             int rc = check_record(b, off, end, n_expect, &nw);
             if (rc) return rc;
             words += nw;
+            // does every chunk carry the first chunk's table?
+            const uint32_t np = rd<uint32_t>(b + off + 8);
+            if (k == 0) {
+                np0 = np;
+            } else if (in.uniform_table) {
+                const uint64_t off0 = rd<uint64_t>(b + d.chunk_index_off);
+                if (np != np0 || std::memcmp(b + off + kRecordHeadBytes, b + off0 + kRecordHeadBytes, 4ull * np) != 0)
+                    in.uniform_table = 0;
+            }
+        }
+        d.small_scales = true;
+        for (uint32_t r = 0; r < in.rows; ++r) {
+            const float v = rd<float>(b + d.scales_off + 4ull * r);
+            if (!(v > -256.f && v < 256.f)) d.small_scales = false;  // also false for NaN
         }
         in.payload_words = words;
         in.compressed_bytes = rd<uint64_t>(b + d.chunk_index_off + 8ull * in.n_chunks) - first;

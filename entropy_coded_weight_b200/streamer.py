@@ -34,12 +34,18 @@ class PingPongStreamer:
     correct either way: the events serialise them).
     """
 
-    def __init__(self, steps: list[Step], device=None, decode_priority: int = 0):
+    def __init__(self, steps: list[Step], device=None, decode_priority: int = 0, overlap_decodes: bool = True):
         self.steps = steps
         self.device = torch.device(device or "cuda")
         self.buf_bytes = max(s.model.block_bytes(s.layer) for s in steps)
         self.bufs = [torch.empty(self.buf_bytes, dtype=torch.uint8, device=self.device) for _ in range(2)]
-        self.decode_stream = torch.cuda.Stream(device=self.device, priority=decode_priority)
+        # One decode stream per buffer lets the decode of block i+1 start while
+        # the last chunks of block i are still decoding; the per-buffer events
+        # keep each buffer's writer and reader ordered.
+        first = torch.cuda.Stream(device=self.device, priority=decode_priority)
+        second = torch.cuda.Stream(device=self.device, priority=decode_priority) if overlap_decodes else first
+        self.decode_streams = [first, second]
+        self.decode_stream = first
         self.consumer_stream = torch.cuda.Stream(device=self.device)
         self.ev_free = [torch.cuda.Event(), torch.cuda.Event()]
         self.ev_ready = [torch.cuda.Event(), torch.cuda.Event()]
@@ -64,6 +70,16 @@ class PingPongStreamer:
             out.append(buf[off:off + 2 * rows * cols].view(torch.bfloat16).view(rows, cols))
         return out
 
+    def begin(self, event) -> None:
+        """Make both decode streams wait for ``event`` (e.g. the start of a timed region)."""
+        for ds in set(self.decode_streams):
+            ds.wait_event(event)
+
+    def join(self) -> None:
+        """Make the consumer stream wait for all decode work enqueued so far."""
+        for ds in set(self.decode_streams):
+            self.consumer_stream.wait_stream(ds)
+
     def run(self, consumer=None, decode_events: list | None = None) -> None:
         """Enqueue one pass over all steps.
 
@@ -74,17 +90,17 @@ class PingPongStreamer:
         """
         for i, step in enumerate(self.steps):
             b = step.layer & 1
+            ds = self.decode_streams[b]
             ev0 = ev1 = None
             if decode_events is not None:
                 # start after the buffer is free so the pair brackets the kernels only
-                self.decode_stream.wait_event(self.ev_free[b])
+                ds.wait_event(self.ev_free[b])
                 ev0 = torch.cuda.Event(enable_timing=True)
-                ev0.record(self.decode_stream)
-            step.model.decode_model_stream(step.layer, self.bufs, self.status, self.decode_stream,
-                                           self.ev_free, self.ev_ready)
+                ev0.record(ds)
+            step.model.decode_model_stream(step.layer, self.bufs, self.status, ds, self.ev_free, self.ev_ready)
             if decode_events is not None:
                 ev1 = torch.cuda.Event(enable_timing=True)
-                ev1.record(self.decode_stream)
+                ev1.record(ds)
                 decode_events.append((ev0, ev1))
             self.consumer_stream.wait_event(self.ev_ready[b])
             if consumer is not None:

@@ -97,7 +97,18 @@ typedef struct eq_matrix_in {
     const uint32_t *out_row; /* n_out entries (may be NULL if n_out == 0) */
     const uint32_t *out_col;
     const float *out_val;
+    uint32_t flags;          /* EQ_TABLE_* below; 0 = default */
 } eq_matrix_in;
+
+/*
+ * Frequency-table scope (eq_matrix_in.flags).  Every chunk record always
+ * carries its own 12-bit table.  By default the encoder quantises one table
+ * from the whole matrix's histogram and writes it into every chunk, which
+ * lets the decoder keep a single slot table per thread block for the matrix;
+ * EQ_TABLE_PER_CHUNK quantises each chunk's own histogram instead (adapts to
+ * local statistics; the decoder then builds one slot table per warp).
+ */
+#define EQ_TABLE_PER_CHUNK 1u
 
 typedef struct eq_encoded eq_encoded;  /* host-side result of eq_encoder_run */
 
@@ -128,7 +139,8 @@ EQW_API int eq_encode_host(const eq_matrix_in *mats, uint32_t n_mats, int n_thre
 typedef struct eq_model eq_model;
 
 typedef struct eq_matrix_info {
-    uint32_t layer, index, dtype, rows, cols, n_chunks, n_outliers, reserved;
+    uint32_t layer, index, dtype, rows, cols, n_chunks, n_outliers;
+    uint32_t uniform_table;     /* 1 if every chunk carries the same frequency table */
     uint64_t compressed_bytes;  /* bytes of its chunk records (tables, states, words) */
     uint64_t payload_words;     /* total 16-bit renormalisation words */
 } eq_matrix_info;

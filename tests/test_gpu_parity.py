@@ -83,11 +83,14 @@ def _ragged():
     return mats
 
 
-@pytest.mark.parametrize("encoder", ["product", "oracle"])
+@pytest.mark.parametrize("encoder", ["product", "product-chunk-tables", "oracle"])
 @pytest.mark.parametrize("per_matrix", [True, False])
 def test_ragged_shapes_bit_exact(eqw, orc, encoder, per_matrix):
     mats = _ragged()
-    blob = eqw.encode_host(mats) if encoder == "product" else orc.encode_container(mats)
+    if encoder == "oracle":
+        blob = orc.encode_container(mats)
+    else:
+        blob = eqw.encode_host(mats, table_scope="chunk" if encoder.endswith("tables") else "matrix")
     got, st = _decode_matrices(eqw, blob, per_matrix)
     assert st == 0
     _assert_parity(got, mats, orc)
@@ -116,6 +119,22 @@ def test_e4m3_all_codes_and_signed_zero(eqw, orc):
     _assert_parity(got, [m], orc)
 
 
+@pytest.mark.parametrize("cols", [4096, 1000, 1001])
+def test_e4m3_large_scales_each_layout(eqw, orc, cols):
+    """Scales >= 2^8 take the two-multiply E4M3 path; cols picks the output layout
+    (multiple of 256: warp-uniform rows; of 8: per-lane rows; else element-wise)."""
+    rng = np.random.default_rng(cols)
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    sym = rng.choice(codes, size=(40, cols)).astype(np.uint8)
+    sc = np.exp(rng.uniform(-20, 70, size=40)).astype(np.float32)
+    sc[0] = np.float32(300.0)
+    m = W.Matrix(0, 0, "big", W.E4M3, sym, sc)
+    for scope in ("matrix", "chunk"):
+        got, st = _decode_matrices(eqw, eqw.encode_host([m], table_scope=scope))
+        assert st == 0
+        _assert_parity(got, [m], orc)
+
+
 def test_int8_all_codes_extreme_scales(eqw, orc):
     rng = np.random.default_rng(6)
     sym = rng.integers(0, 256, size=(32, 2048)).astype(np.uint8)
@@ -135,19 +154,20 @@ def test_workload1_single_matrix(eqw, orc):
         _assert_parity(got, mats, orc)
 
 
-@pytest.mark.parametrize("h", [2.1, 3.0])
-def test_workload2_llama7b_block(eqw, orc, h):
+@pytest.mark.parametrize("h,scope", [(2.1, "matrix"), (3.0, "matrix"), (2.1, "chunk")])
+def test_workload2_llama7b_block(eqw, orc, h, scope):
     mats = W.llama7b_int8_block(h)
-    got, st = _decode_matrices(eqw, eqw.encode_host(mats), per_matrix=False)
+    got, st = _decode_matrices(eqw, eqw.encode_host(mats, table_scope=scope), per_matrix=False)
     assert st == 0
     _assert_parity(got, mats, orc)
 
 
-def test_workload3_llama70b_e4m3_block(eqw, orc):
+@pytest.mark.parametrize("scope", ["matrix", "chunk"])
+def test_workload3_llama70b_e4m3_block(eqw, orc, scope):
     mats = W.llama70b_e4m3_block(2.1)
     for m in mats:
         assert abs(W.empirical_entropy_bits(m.symbols) - 2.1) < 0.02
-    got, st = _decode_matrices(eqw, eqw.encode_host(mats), per_matrix=False)
+    got, st = _decode_matrices(eqw, eqw.encode_host(mats, table_scope=scope), per_matrix=False)
     assert st == 0
     _assert_parity(got, mats, orc)
 
