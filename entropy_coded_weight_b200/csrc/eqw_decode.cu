@@ -51,18 +51,22 @@ using namespace eqw;
 namespace {
 
 constexpr uint32_t kFull = 0xFFFFFFFFu;
-constexpr uint32_t kRingBytes = 2048;  // per warp
+constexpr uint32_t kRingBytes = 2048;  // per warp: four 512-byte segments ...
 constexpr uint32_t kSegBytes = 512;    // one TMA segment = 256 words
 constexpr uint32_t kRingSegs = kRingBytes / kSegBytes;
+// ... followed by a 512-byte mirror of segment slot 0, so the up to 512 bytes
+// one 256-symbol group reads from any starting offset are contiguous and the
+// per-step word address needs no wrap-around mask.
+constexpr uint32_t kRingStride = kRingBytes + kSegBytes;
 constexpr uint32_t kLutBytes = 4 * kProbTotal;
 constexpr long long kWaitCycles = 2000000000LL;
 constexpr uint32_t kNoLimit = 0xFFFFFFFFu;
 
 #ifndef EQ_SHARED_WARPS
-#define EQ_SHARED_WARPS 16
+#define EQ_SHARED_WARPS 32
 #endif
 #ifndef EQ_SHARED_MIN_CTAS
-#define EQ_SHARED_MIN_CTAS 3
+#define EQ_SHARED_MIN_CTAS 1
 #endif
 constexpr int kSharedWarps = EQ_SHARED_WARPS;      // warps per block, shared-table kernel
 constexpr int kSharedMinCtas = EQ_SHARED_MIN_CTAS; // register budget: blocks of kSharedWarps per SM
@@ -83,12 +87,20 @@ struct MatJob {
     uint32_t small_scales;        // all |scale| < 2^8: E4M3 dequant in one multiply
 };
 
+// Multipliers of the step's IMAD forms.  They arrive as kernel parameters so
+// that the compiler keeps them as multiplications on the FMA pipe rather than
+// rewriting them into shifts on the busier integer ALU pipe.
+struct StepK {
+    uint32_t two, k2e20, k2e14, k2e12, k2e24, kneg4096, k2e16, pad;
+};
+
 struct DecodeParams {
     const uint8_t *blob;
     uint64_t blob_len;
     int32_t *status;
     uint32_t n_mats;
     uint32_t total_units;
+    StepK k;
     MatJob mats[kMaxMatsPerLaunch];
 };
 
@@ -182,6 +194,19 @@ __device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
     return c;
 }
 
+#ifndef EQ_F32X2
+#define EQ_F32X2 0
+#endif
+
+// Two fp32 products rounded to nearest even, packed or as two multiplies.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+#if EQ_F32X2
+    return mul2_rn(a, b);
+#else
+    return make_float2(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y));
+#endif
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float2 v) {
     __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
     return *reinterpret_cast<uint32_t *>(&h);
@@ -196,10 +221,33 @@ __device__ __forceinline__ uint16_t to_bf16(float v) {
 // mantissa bits placed at bit 20 of an fp32 give exactly value * 2^-120
 // (subnormal codes included); the factor 2^120 is applied exactly, either on
 // its own or folded into a scale below 2^8 (same real product, one rounding).
+#ifndef EQ_INT8_MAGIC
+#define EQ_INT8_MAGIC 0
+#endif
+
+// Byte the slot table stores for a symbol.  With EQ_INT8_MAGIC, Int8 symbols
+// are stored with the sign bit flipped: then the float with bits
+// 0x4B000000 | byte is exactly 2^23 + 128 + value, and one exact subtraction
+// (FMA pipe) replaces an int-to-float conversion (conversion pipe).
+template <int DT>
+__host__ __device__ constexpr uint32_t stored_byte(uint32_t sym) {
+    return (DT == EQ_INT8 && EQ_INT8_MAGIC) ? (sym ^ 0x80u) : sym;
+}
+constexpr float kInt8Magic = 8388736.0f;  // 2^23 + 128
+
+// Value of the symbol whose stored byte is the low byte of e.  Int8: two's
+// complement.  E4M3 (OCP E4M3FN, bias 7): the 7 exponent and mantissa bits
+// placed at bit 20 of an fp32 give exactly value * 2^-120 (subnormal codes
+// included); the factor 2^120 is applied exactly, on its own or folded into
+// a scale below 2^8 (same real product, one rounding).
 template <int DT>
 __device__ __forceinline__ float raw_value(uint32_t e) {
     if constexpr (DT == EQ_INT8) {
+#if EQ_INT8_MAGIC
+        return __fadd_rn(__uint_as_float((e & 0xFFu) | 0x4B000000u), -kInt8Magic);
+#else
         return static_cast<float>(static_cast<int8_t>(e & 0xFFu));
+#endif
     } else {
         return __uint_as_float(((e & 0x80u) << 24) | ((e & 0x7Fu) << 20));
     }
@@ -222,9 +270,9 @@ __device__ __forceinline__ uint4 dequant8(const uint32_t (&e)[8], float s, bool 
     for (int i = 0; i < 4; ++i) {
         float2 v = make_float2(raw_value<DT>(e[2 * i]), raw_value<DT>(e[2 * i + 1]));
         if constexpr (DT == EQ_E4M3) {
-            if (!folded) v = mul2_rn(v, make_float2(0x1p120f, 0x1p120f));
+            if (!folded) v = mul2(v, make_float2(0x1p120f, 0x1p120f));
         }
-        o[i] = pack_bf16x2(mul2_rn(v, s2));
+        o[i] = pack_bf16x2(mul2(v, s2));
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -272,8 +320,10 @@ __device__ __noinline__ uint32_t ring_service(RingCtl *ctl, uint32_t ring, uint3
             if (lane == 0) {
                 const uint32_t bytes = min(kSegBytes, pbytes - issued * kSegBytes);
                 const uint32_t slot = issued % kRingSegs;
-                mbar_expect_tx(mbar + 8 * slot, bytes);
-                bulk_load(ring + slot * kSegBytes, ctl->payload + (size_t)issued * kSegBytes, bytes, mbar + 8 * slot);
+                const uint8_t *src = ctl->payload + (size_t)issued * kSegBytes;
+                mbar_expect_tx(mbar + 8 * slot, slot == 0 ? 2 * bytes : bytes);
+                bulk_load(ring + slot * kSegBytes, src, bytes, mbar + 8 * slot);
+                if (slot == 0) bulk_load(ring + kRingBytes, src, bytes, mbar);  // the mirror
             }
             ++issued;
         } while (issued < n_segs && issued < horizon);
@@ -326,133 +376,240 @@ __device__ __noinline__ bool ring_drain(RingCtl *ctl, uint32_t mbar) {
 }
 
 // ---- the rANS step ---------------------------------------------------------------
-// One step of all 32 lanes.  `ring` is the warp's 2 KB-aligned shared ring;
-// `pw` counts payload bytes consumed (2 per word).  Returns the slot entry
-// (its low byte is the decoded symbol).
-__device__ __forceinline__ uint32_t rans_step(const uint32_t *lut, uint32_t ring, uint32_t &x, uint32_t &pw,
-                                              uint32_t lt) {
-    const uint32_t e = lut[x & (kProbTotal - 1)];
-    x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xFFFu);
+// Integer helpers that run on the IMAD (FMA) pipe, keeping the ALU pipe free:
+// mad.hi gives hi32(a * b) + c, so shifts right and field extraction cost one
+// IMAD each.
+__device__ __forceinline__ uint32_t mad_hi(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t mad_lo(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+#ifndef EQ_TOTAL_SHFL
+#define EQ_TOTAL_SHFL 0
+#endif
+
+#ifndef EQ_TOTAL_MODE
+#define EQ_TOTAL_MODE 0  // 0: popcount of the ballot, 1: warp reduction, 2: shuffle from lane 31
+#endif
+
+// One step of all 32 lanes.  `lut` is the shared-memory address of the slot
+// table; `rp` the shared-memory address of the next unread word (inside the
+// ring or its mirror), advanced past the words this step consumes.  Returns
+// the slot entry (low byte: the stored symbol byte).
+//   slot = x & 4095, e = lut[slot] = f << 20 | (slot - cum) << 8 | byte
+//   x' = f * (x >> 12) + (slot - cum) = f * ((x >> 12) - 4096) + (e >> 8)
+// Every lane reads a word (the ring always holds valid memory) and keeps it
+// only if it renormalises, so the step has no branch.
+#ifndef EQ_PARAM_K
+#define EQ_PARAM_K 0
+#endif
+#ifndef EQ_SEL_MERGE
+#define EQ_SEL_MERGE 1
+#endif
+
+__device__ __forceinline__ uint32_t rans_step(uint32_t lut, uint32_t &rp, uint32_t &x, uint32_t lt, const StepK &Kp) {
+#if EQ_PARAM_K
+    const StepK &K = Kp;
+#else
+    (void)Kp;
+    constexpr StepK K{2u, 1u << 20, 1u << 14, 1u << 12, 1u << 24, 0u - kProbTotal, 1u << 16, 0u};
+#endif
+    const uint32_t addr = mad_hi(mad_lo(x, K.k2e20, 0u), K.k2e14, lut);  // lut + 4 * (x & 4095)
+    const uint32_t e = lds_u32(addr);
+    const uint32_t t = mad_hi(x, K.k2e20, K.kneg4096);                    // (x >> 12) - 4096
+    x = mad_lo(mad_hi(e, K.k2e12, 0u), t, mad_hi(e, K.k2e24, 0u));
     const bool need = x < kStateLow;
+    const uint32_t x_before_merge = x;
+    (void)x_before_merge;
     const uint32_t b = __ballot_sync(kFull, need);
-    const uint32_t w = lds_u16(ring | ((pw + 2u * __popc(b & lt)) & (kRingBytes - 1)));
-    x = need ? ((x << 16) | w) : x;
-    pw += 2u * __popc(b);
+    const uint32_t pre = __popc(b & lt);
+    const uint32_t w = lds_u16(mad_lo(pre, K.two, rp));
+#if EQ_SEL_MERGE
+    const uint32_t xr = mad_lo(x, K.k2e16, w);
+    x = need ? xr : x;
+#else
+    if (need) x = mad_lo(x, K.k2e16, w);
+#endif
+#if EQ_TOTAL_MODE == 3
+    // a second ballot whose only use is warp-uniform, so the count can live on
+    // the uniform datapath instead of the vector popcount (conversion) pipe
+    uint32_t bu;
+    asm volatile("{\n\t.reg .pred q;\n\tsetp.lt.u32 q, %1, 65536;\n\tvote.sync.ballot.b32 %0, q, 0xffffffff;\n\t}"
+                 : "=r"(bu) : "r"(x_before_merge));
+    rp = mad_lo(__popc(bu), K.two, rp);
+#elif EQ_TOTAL_MODE == 1
+    rp = mad_lo(__reduce_add_sync(kFull, need ? 1u : 0u), K.two, rp);
+#elif EQ_TOTAL_MODE == 2
+    rp = mad_lo(__shfl_sync(kFull, pre + (need ? 1u : 0u), 31), K.two, rp);
+#else
+    rp = mad_lo(__popc(b), K.two, rp);
+#endif
     return e;
 }
 
 // Last, partial group: lane l is active at step r while 8l + r < rem.
-__device__ __forceinline__ void rans_tail(const uint32_t *lut, uint32_t ring, uint32_t &x, uint32_t &pw, uint32_t lt,
+__device__ __forceinline__ void rans_tail(uint32_t lut, uint32_t ring, uint32_t &x, uint32_t &pw, uint32_t lt,
                                           uint32_t lane, uint32_t rem, uint32_t (&e8)[8]) {
 #pragma unroll
     for (uint32_t r = 0; r < 8; ++r) {
         const bool active = lane * kGroup + r < rem;
         bool need = false;
         if (active) {
-            const uint32_t e = lut[x & (kProbTotal - 1)];
+            const uint32_t e = lds_u32(lut + 4 * (x & (kProbTotal - 1)));
             x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xFFFu);
             e8[r] = e;
             need = x < kStateLow;
         }
         const uint32_t b = __ballot_sync(kFull, need);
-        const uint32_t w = lds_u16(ring | ((pw + 2u * __popc(b & lt)) & (kRingBytes - 1)));
+        const uint32_t w = lds_u16(ring + ((pw + 2u * __popc(b & lt)) & (kRingBytes - 1)));
         if (need) x = (x << 16) | w;
         pw += 2u * __popc(b);
     }
 }
 
+// Per-chunk copy of the output-side fields of a matrix, kept in registers.
+struct OutCtx {
+    uint16_t *out;
+    const float *scales;
+    uint64_t n_elems;
+    uint32_t cols;
+    uint32_t rows;
+    bool small_scales;
+};
+
+__device__ __forceinline__ OutCtx out_ctx(const MatJob &M) {
+    return OutCtx{M.out, M.scales, M.n_elems, M.cols, (uint32_t)(M.n_elems / M.cols), M.small_scales != 0};
+}
+
+#ifndef EQ_BRANCHLESS_CURSOR
+#define EQ_BRANCHLESS_CURSOR 0
+#endif
+#ifndef EQ_VOTE_SERVICE
+#define EQ_VOTE_SERVICE 0
+#endif
+
 // Element-wise store of `count` outputs starting at linear index idx.
 template <int DT>
-__device__ __forceinline__ void store_elems(const MatJob &M, uint64_t idx, uint32_t count, const uint32_t (&e8)[8]) {
+__device__ __forceinline__ void store_elems(const OutCtx &O, uint64_t idx, uint32_t count, const uint32_t (&e8)[8]) {
 #pragma unroll
     for (uint32_t r = 0; r < 8; ++r) {
         if (r < count) {
             const uint64_t i = idx + r;
-            M.out[i] = to_bf16(dequant1<DT>(e8[r], __ldg(M.scales + i / M.cols)));
+            O.out[i] = to_bf16(dequant1<DT>(e8[r], __ldg(O.scales + i / O.cols)));
         }
     }
 }
 
-// Output bookkeeping for one chunk.  kRowUniform keeps the (warp-uniform) row
-// of the current 256-symbol group; kLaneRows keeps each lane's own row/col.
+// Output bookkeeping for one chunk.  kRowUniform (cols % 256 == 0) keeps the
+// warp-uniform row of the current 256-symbol group; kLaneRows keeps each
+// lane's own row and column.
 struct Cursor {
     uint32_t row, col;
     float scale;
 };
 
+template <int DT>
+__device__ __forceinline__ float row_scale(const OutCtx &O, uint32_t row) {
+    float s = __ldg(O.scales + row);
+    if (DT == EQ_E4M3 && O.small_scales) s *= 0x1p120f;  // exact: |s| < 2^8
+    return s;
+}
+
 template <int DT, uint32_t LAYOUT>
-__device__ __forceinline__ void cursor_init(const MatJob &M, uint64_t first, uint32_t lane, Cursor &c) {
-    if constexpr (LAYOUT == kRowUniform) {
-        c.row = (uint32_t)(first / M.cols);
-        c.col = (uint32_t)(first - (uint64_t)c.row * M.cols);
-    } else if constexpr (LAYOUT == kLaneRows) {
-        const uint64_t e0 = first + kGroup * lane;
-        c.row = (uint32_t)(e0 / M.cols);
-        c.col = (uint32_t)(e0 - (uint64_t)c.row * M.cols);
-    }
+__device__ __forceinline__ void cursor_init(const OutCtx &O, uint64_t first, uint32_t lane, Cursor &c) {
     if constexpr (LAYOUT != kGeneric) {
-        float s = __ldg(M.scales + c.row);
-        if (DT == EQ_E4M3 && M.small_scales) s *= 0x1p120f;
-        c.scale = s;
+        const uint64_t e0 = LAYOUT == kRowUniform ? first : first + kGroup * lane;
+        c.row = (uint32_t)(e0 / O.cols);
+        c.col = (uint32_t)(e0 - (uint64_t)c.row * O.cols);
+        c.scale = row_scale<DT>(O, c.row);
     }
 }
 
-// Move the cursor to the next 256-symbol group (idx: this lane's current first output).
+// Move to the next 256-symbol group (idx: this lane's first output of the
+// group just stored).
 template <int DT, uint32_t LAYOUT>
-__device__ __forceinline__ void cursor_advance(const MatJob &M, uint64_t idx, Cursor &c) {
-    bool moved = false;
-    c.col += kGroupSyms;
-    while (c.col >= M.cols) {
-        c.col -= M.cols;
-        ++c.row;
-        moved = true;
-    }
-    if (moved && idx + kGroupSyms < M.n_elems) {
-        float s = __ldg(M.scales + c.row);
-        if (DT == EQ_E4M3 && M.small_scales) s *= 0x1p120f;
-        c.scale = s;
+__device__ __forceinline__ void cursor_advance(const OutCtx &O, uint64_t idx, Cursor &c) {
+    if constexpr (LAYOUT == kRowUniform) {
+#if EQ_BRANCHLESS_CURSOR
+        // cols % 256 == 0: the group's row is warp-uniform; reload its scale
+        // every group (an L1 hit) instead of branching on the row change
+        c.col += kGroupSyms;
+        const bool wrap = c.col == O.cols;
+        c.col = wrap ? 0u : c.col;
+        c.row += wrap ? 1u : 0u;
+        c.scale = row_scale<DT>(O, min(c.row, O.rows - 1));
+#else
+        c.col += kGroupSyms;
+        if (c.col == O.cols) {
+            c.col = 0;
+            ++c.row;
+            if (idx + kGroupSyms < O.n_elems) c.scale = row_scale<DT>(O, c.row);
+        }
+#endif
+    } else if constexpr (LAYOUT == kLaneRows) {
+        bool moved = false;
+        c.col += kGroupSyms;
+        while (c.col >= O.cols) {
+            c.col -= O.cols;
+            ++c.row;
+            moved = true;
+        }
+        if (moved && idx + kGroupSyms < O.n_elems) c.scale = row_scale<DT>(O, c.row);
     }
 }
 
 template <int DT, uint32_t LAYOUT>
-__device__ __forceinline__ void group_store(const MatJob &M, uint16_t *dst, uint64_t idx, Cursor &c,
+__device__ __forceinline__ void group_store(const OutCtx &O, uint16_t *dst, uint64_t idx, Cursor &c,
                                             const uint32_t (&e8)[8]) {
     if constexpr (LAYOUT == kGeneric) {
-        store_elems<DT>(M, idx, 8, e8);
+        store_elems<DT>(O, idx, 8, e8);
     } else {
-        st_global_v4(dst, dequant8<DT>(e8, c.scale, M.small_scales != 0));
-        cursor_advance<DT, LAYOUT>(M, idx, c);
+        st_global_v4(dst, dequant8<DT>(e8, c.scale, O.small_scales));
+        cursor_advance<DT, LAYOUT>(O, idx, c);
     }
 }
 
-// Decode one chunk whose slot table is ready in `lut` (n_present >= 2) or
-// whose single symbol is `single` (n_present == 1).  Returns false if a
-// bounded wait gave up (the warp must stop).
+// Decode one chunk whose slot table is ready at `lut` (n_present >= 2) or
+// whose single symbol's stored byte is `single` (n_present == 1).  Returns
+// false if a bounded wait gave up (the warp must stop).
 template <int DT, uint32_t LAYOUT>
-__device__ __forceinline__ bool decode_body(const DecodeParams &P, const MatJob &M, uint64_t first, uint32_t n,
-                                            uint32_t n_words, const uint8_t *payload, bool single_sym,
-                                            uint32_t single, uint32_t x, const uint32_t *lut, uint32_t ring,
-                                            uint32_t mbar, RingCtl *ctl, uint32_t lane, uint32_t lt) {
+__device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, const StepK &K, uint64_t first,
+                                            uint32_t n, uint32_t n_words, const uint8_t *payload, bool single_sym,
+                                            uint32_t single, uint32_t x, uint32_t lut, uint32_t ring, uint32_t mbar,
+                                            RingCtl *ctl, uint32_t lane, uint32_t lt) {
     const uint32_t n_full = n / kGroupSyms;
     const uint32_t tail = n % kGroupSyms;
     Cursor cur{0, 0, 0.f};
-    cursor_init<DT, LAYOUT>(M, first, lane, cur);
-    uint16_t *dst = M.out + first + kGroup * lane;
+    cursor_init<DT, LAYOUT>(O, first, lane, cur);
+    uint16_t *dst = O.out + first + kGroup * lane;
 
     if (single_sym) {
         // f = 4096: the states never change and there are no words
         if (n_words != 0 || !__all_sync(kFull, x == kStateLow)) {
-            flag(P.status, EQ_DEV_BAD_END);
+            flag(status, EQ_DEV_BAD_END);
             return true;
         }
         uint32_t e8[8];
 #pragma unroll
         for (int r = 0; r < 8; ++r) e8[r] = single;
         for (uint32_t g = 0; g < n_full; ++g, dst += kGroupSyms)
-            group_store<DT, LAYOUT>(M, dst, first + (uint64_t)g * kGroupSyms + kGroup * lane, cur, e8);
+            group_store<DT, LAYOUT>(O, dst, first + (uint64_t)g * kGroupSyms + kGroup * lane, cur, e8);
         if (tail) {
             const uint32_t mine = tail > kGroup * lane ? min(8u, tail - kGroup * lane) : 0u;
-            store_elems<DT>(M, first + (uint64_t)n_full * kGroupSyms + kGroup * lane, mine, e8);
+            store_elems<DT>(O, first + (uint64_t)n_full * kGroupSyms + kGroup * lane, mine, e8);
         }
         return true;
     }
@@ -469,32 +626,39 @@ __device__ __forceinline__ bool decode_body(const DecodeParams &P, const MatJob 
     uint32_t limit = pbytes ? 0u : kNoLimit;
     uint32_t pw = 0;
     for (uint32_t g = 0; g < n_full; ++g, dst += kGroupSyms) {
+#if EQ_VOTE_SERVICE
+        if (__any_sync(kFull, pw >= limit)) {  // warp-uniform by construction
+#else
         if (pw >= limit) {
+#endif
             limit = ring_service(ctl, ring, mbar, pw);
             if (ctl->dead) break;
         }
+        const uint32_t rp0 = ring + (pw & (kRingBytes - 1));
+        uint32_t rp = rp0;
         if constexpr (LAYOUT == kGeneric) {
             uint32_t e8[8];
 #pragma unroll
-            for (int r = 0; r < 8; ++r) e8[r] = rans_step(lut, ring, x, pw, lt);
-            store_elems<DT>(M, first + (uint64_t)g * kGroupSyms + kGroup * lane, 8, e8);
+            for (int r = 0; r < 8; ++r) e8[r] = rans_step(lut, rp, x, lt, K);
+            store_elems<DT>(O, first + (uint64_t)g * kGroupSyms + kGroup * lane, 8, e8);
         } else {
             // dequantise pairs as they are decoded: 4 packed registers instead of 8 entries
             const float2 s2 = make_float2(cur.scale, cur.scale);
             uint32_t o[4];
 #pragma unroll
             for (int r = 0; r < 8; r += 2) {
-                const uint32_t e0 = rans_step(lut, ring, x, pw, lt);
-                const uint32_t e1 = rans_step(lut, ring, x, pw, lt);
+                const uint32_t e0 = rans_step(lut, rp, x, lt, K);
+                const uint32_t e1 = rans_step(lut, rp, x, lt, K);
                 float2 v = make_float2(raw_value<DT>(e0), raw_value<DT>(e1));
                 if constexpr (DT == EQ_E4M3) {
-                    if (!M.small_scales) v = mul2_rn(v, make_float2(0x1p120f, 0x1p120f));
+                    if (!O.small_scales) v = mul2(v, make_float2(0x1p120f, 0x1p120f));
                 }
-                o[r / 2] = pack_bf16x2(mul2_rn(v, s2));
+                o[r / 2] = pack_bf16x2(mul2(v, s2));
             }
             st_global_v4(dst, make_uint4(o[0], o[1], o[2], o[3]));
-            cursor_advance<DT, LAYOUT>(M, first + (uint64_t)g * kGroupSyms + kGroup * lane, cur);
+            cursor_advance<DT, LAYOUT>(O, first + (uint64_t)g * kGroupSyms + kGroup * lane, cur);
         }
+        pw += rp - rp0;
     }
     if (tail && !ctl->dead) {
         if (pw >= limit) limit = ring_service(ctl, ring, mbar, pw);
@@ -502,15 +666,15 @@ __device__ __forceinline__ bool decode_body(const DecodeParams &P, const MatJob 
             uint32_t e8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
             rans_tail(lut, ring, x, pw, lt, lane, tail, e8);
             const uint32_t mine = tail > kGroup * lane ? min(8u, tail - kGroup * lane) : 0u;
-            store_elems<DT>(M, first + (uint64_t)n_full * kGroupSyms + kGroup * lane, mine, e8);
+            store_elems<DT>(O, first + (uint64_t)n_full * kGroupSyms + kGroup * lane, mine, e8);
         }
     }
     if (!ring_drain(ctl, mbar)) {
-        flag(P.status, EQ_DEV_TIMEOUT);
+        flag(status, EQ_DEV_TIMEOUT);
         return false;
     }
     // a valid stream returns every state to 2^16 and consumes exactly n_words
-    if (!__all_sync(kFull, x == kStateLow) || pw != 2u * n_words) flag(P.status, EQ_DEV_BAD_END);
+    if (!__all_sync(kFull, x == kStateLow) || pw != 2u * n_words) flag(status, EQ_DEV_BAD_END);
     return true;
 }
 
@@ -557,7 +721,8 @@ __device__ __forceinline__ bool load_head(const DecodeParams &P, const MatJob &M
 // their cumulative frequencies to shared memory, and/or expands the list into
 // a warp's slot table.  Returns validity (warp-uniform).
 __device__ __forceinline__ bool warp_table(const uint32_t *tab, uint32_t n_present, uint32_t lane,
-                                           uint32_t *entries_out, uint32_t *cum_out, uint32_t *lut) {
+                                           uint32_t *entries_out, uint32_t *cum_out, uint32_t *lut,
+                                           uint32_t sym_xor) {
     uint32_t run = 0;
     int prev_sym = -1;
     bool ok = true;
@@ -589,7 +754,7 @@ __device__ __forceinline__ bool warp_table(const uint32_t *tab, uint32_t n_prese
                 const uint32_t sq = __shfl_sync(kFull, sym, q);
                 for (uint32_t t = lane; t < fq; t += 32) {
                     const uint32_t slot = cq + t;
-                    if (slot < kProbTotal && fq < kProbTotal) lut[slot] = (fq << 20) | (t << 8) | sq;
+                    if (slot < kProbTotal && fq < kProbTotal) lut[slot] = (fq << 20) | (t << 8) | (sq ^ sym_xor);
                 }
             }
         }
@@ -599,17 +764,18 @@ __device__ __forceinline__ bool warp_table(const uint32_t *tab, uint32_t n_prese
     return ok && run == kProbTotal;
 }
 
-// Shared memory of one block.  Rings start on a 2 KB boundary so a ring
-// address is (ring base | byte offset).
+// Shared memory of one block: slot table(s), then per warp a 2.5 KB word ring
+// (with its mirror), the ring's mbarriers and bookkeeping, then the block's
+// reference frequency list (shared-table kernel only).
 template <int WARPS, bool SHARED>
 struct Smem {
     static constexpr uint32_t kLuts = SHARED ? 1 : WARPS;
-    static constexpr uint32_t kRingOff = kLuts * kLutBytes;             // + runtime pad to 2 KB
-    static constexpr uint32_t kMbarOff = kRingOff + WARPS * kRingBytes; // all offsets below include the pad
+    static constexpr uint32_t kRingOff = kLuts * kLutBytes;             // + runtime pad to 128 B
+    static constexpr uint32_t kMbarOff = kRingOff + WARPS * kRingStride; // all offsets below include the pad
     static constexpr uint32_t kCtlOff = kMbarOff + WARPS * kRingSegs * 8;
     static constexpr uint32_t kRefOff = kCtlOff + WARPS * 32;           // 32 bytes of RingCtl per warp
     static constexpr uint32_t kBlockOff = kRefOff + (SHARED ? 2 * 256 * 4 : 0);
-    static constexpr uint32_t kBytes = kBlockOff + 16 + kRingBytes;     // + worst-case alignment pad
+    static constexpr uint32_t kBytes = kBlockOff + 16 + 128;            // + worst-case alignment pad
 };
 static_assert(sizeof(RingCtl) <= 32, "RingCtl slot");
 
@@ -621,12 +787,14 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = threadIdx.x >> 5;
     const uint32_t base = smem_u32(smem_raw);
-    const uint32_t pad = (kRingBytes - ((base + L::kRingOff) & (kRingBytes - 1))) & (kRingBytes - 1);
+    const uint32_t pad = (128u - ((base + L::kRingOff) & 127u)) & 127u;
     unsigned char *padded = smem_raw + pad;  // offsets from kRingOff on are relative to this
-    const uint32_t ring = base + pad + L::kRingOff + warp * kRingBytes;
+    const uint32_t ring = base + pad + L::kRingOff + warp * kRingStride;
     const uint32_t mbar = base + pad + L::kMbarOff + warp * kRingSegs * 8;
     RingCtl *ctl = reinterpret_cast<RingCtl *>(padded + L::kCtlOff + warp * 32);
     uint32_t *lut = reinterpret_cast<uint32_t *>(smem_raw) + (SHARED ? 0u : warp * kProbTotal);
+    const uint32_t lut_addr = smem_u32(lut);
+    const StepK K = P.k;
     if (lane == 0) {
         for (uint32_t i = 0; i < kRingSegs; ++i) mbar_init(mbar + 8 * i, 1);
         fence_mbar_init();
@@ -654,7 +822,7 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
                     ChunkHead h;
                     bool ok = load_head(P, M, k0, lane, h);
                     if (ok) ok = warp_table(reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes), h.n_present,
-                                            lane, ref_entries, ref_cum, nullptr);
+                                            lane, ref_entries, ref_cum, nullptr, 0u);
                     if (lane == 0) {
                         blk[0] = ok ? h.n_present : 0u;
                         blk[1] = ok;
@@ -667,7 +835,8 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
                         const uint32_t e = ref_entries[i], c = ref_cum[i];
                         const uint32_t f = e >> 16, sy = e & 0xFFu;
                         for (uint32_t t = threadIdx.x; t < f; t += WARPS * 32)
-                            if (c + t < kProbTotal && f < kProbTotal) lut[c + t] = (f << 20) | (t << 8) | sy;
+                            if (c + t < kProbTotal && f < kProbTotal)
+                                lut[c + t] = (f << 20) | (t << 8) | stored_byte<DT>(sy);
                     }
                 }
                 __syncthreads();
@@ -687,8 +856,9 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
                 flag(P.status, EQ_DEV_BAD_TABLE);
                 continue;
             }
-            decode_body<DT, LAYOUT>(P, M, (uint64_t)k * kChunkSyms, h.n, h.n_words, h.rec + h.table_bytes, np == 1,
-                                    ref_entries[0] & 0xFFu, h.x, lut, ring, mbar, ctl, lane, lt);
+            decode_body<DT, LAYOUT>(P.status, out_ctx(M), K, (uint64_t)k * kChunkSyms, h.n, h.n_words,
+                                    h.rec + h.table_bytes, np == 1, stored_byte<DT>(ref_entries[0] & 0xFFu), h.x,
+                                    lut_addr, ring, mbar, ctl, lane, lt);
             __syncwarp();
         }
     } else {
@@ -702,14 +872,15 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
             if (!load_head(P, M, k, lane, h)) continue;
             const uint32_t *tab = reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes);
             __syncwarp();  // the previous chunk's reads of the slot table are done
-            const bool ok = warp_table(tab, h.n_present, lane, nullptr, nullptr, lut);
+            const bool ok = warp_table(tab, h.n_present, lane, nullptr, nullptr, lut, stored_byte<DT>(0u));
             if (!ok) {
                 flag(P.status, EQ_DEV_BAD_TABLE);
                 continue;
             }
             __syncwarp();
-            decode_body<DT, LAYOUT>(P, M, (uint64_t)k * kChunkSyms, h.n, h.n_words, h.rec + h.table_bytes,
-                                    h.n_present == 1, tab[0] & 0xFFu, h.x, lut, ring, mbar, ctl, lane, lt);
+            decode_body<DT, LAYOUT>(P.status, out_ctx(M), K, (uint64_t)k * kChunkSyms, h.n, h.n_words,
+                                    h.rec + h.table_bytes, h.n_present == 1, stored_byte<DT>(tab[0] & 0xFFu), h.x,
+                                    lut_addr, ring, mbar, ctl, lane, lt);
             __syncwarp();
         }
     }
@@ -824,6 +995,7 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
             for (auto &b : a)
                 for (auto &c : b) {
                     c = DecodeParams{};
+                    c.k = StepK{2u, 1u << 20, 1u << 14, 1u << 12, 1u << 24, 0u - kProbTotal, 1u << 16, 0u};
                     c.blob = m->d_blob;
                     c.blob_len = m->len;
                     c.status = d_status;
