@@ -51,13 +51,15 @@ using namespace eqw;
 namespace {
 
 constexpr uint32_t kFull = 0xFFFFFFFFu;
-constexpr uint32_t kRingBytes = 2048;  // per warp: four 512-byte segments ...
+constexpr uint32_t kRingBytes = 4096;  // per warp: eight 512-byte segments ...
 constexpr uint32_t kSegBytes = 512;    // one TMA segment = 256 words
 constexpr uint32_t kRingSegs = kRingBytes / kSegBytes;
 // ... followed by a 512-byte mirror of segment slot 0, so the up to 512 bytes
 // one 256-symbol group reads from any starting offset are contiguous and the
 // per-step word address needs no wrap-around mask.
 constexpr uint32_t kRingStride = kRingBytes + kSegBytes;
+// Words the ring guarantees resident at each service check: two groups.
+constexpr uint32_t kSpan = 2 * kSegBytes;
 constexpr uint32_t kLutBytes = 4 * kProbTotal;
 constexpr long long kWaitCycles = 2000000000LL;
 constexpr uint32_t kNoLimit = 0xFFFFFFFFu;
@@ -296,9 +298,9 @@ struct RingCtl {
 };
 
 __device__ __forceinline__ uint32_t ring_limit(uint32_t n_segs, uint32_t issued, uint32_t ready) {
-    // safe while bytes [pw, pw + 512) are resident and no free slot can take a segment
+    // safe while bytes [pw, pw + kSpan) are resident and no free slot can take a segment
     uint32_t lim = kNoLimit;
-    if (ready < n_segs) lim = ready * kSegBytes >= kSegBytes - 1 ? ready * kSegBytes - (kSegBytes - 1) : 0u;
+    if (ready < n_segs) lim = ready * kSegBytes >= kSpan - 1 ? ready * kSegBytes - (kSpan - 1) : 0u;
     if (issued < n_segs) {
         const uint32_t t = issued >= kRingSegs - 1 ? (issued - (kRingSegs - 1)) * kSegBytes : 0u;
         lim = min(lim, t);
@@ -306,7 +308,7 @@ __device__ __forceinline__ uint32_t ring_limit(uint32_t n_segs, uint32_t issued,
     return lim;
 }
 
-// Refill free slots, then make payload bytes [pw, pw + 512) resident.  Returns
+// Refill free slots, then make payload bytes [pw, pw + kSpan) resident.  Returns
 // the new limit; on a wait that gave up sets ctl->dead and returns kNoLimit.
 __device__ __noinline__ uint32_t ring_service(RingCtl *ctl, uint32_t ring, uint32_t mbar, uint32_t pw) {
     const uint32_t lane = threadIdx.x & 31u;
@@ -328,7 +330,7 @@ __device__ __noinline__ uint32_t ring_service(RingCtl *ctl, uint32_t ring, uint3
             ++issued;
         } while (issued < n_segs && issued < horizon);
     }
-    uint32_t need = (pw + kSegBytes - 1) / kSegBytes;  // last segment touched by bytes [pw, pw + 512)
+    uint32_t need = (pw + kSpan - 1) / kSegBytes;  // last segment touched by bytes [pw, pw + kSpan)
     if (need >= n_segs) need = n_segs - 1;
     bool ok = true;
     while (ready <= need && ready < issued) {
@@ -582,6 +584,29 @@ __device__ __forceinline__ void group_store(const OutCtx &O, uint16_t *dst, uint
     }
 }
 
+// One 256-symbol group in a row-uniform layout: 8 steps, dequantised in pairs
+// as they are decoded (4 packed registers), one 16-byte store.
+template <int DT>
+__device__ __forceinline__ void group_row(uint32_t lut, uint32_t ring, uint32_t &pw, uint32_t &x, uint32_t lt,
+                                          float2 s2, bool small_scales, uint16_t *dst) {
+    const uint32_t rp0 = ring + (pw & (kRingBytes - 1));
+    uint32_t rp = rp0;
+    const StepK K{};
+    uint32_t o[4];
+#pragma unroll
+    for (int r = 0; r < 8; r += 2) {
+        const uint32_t e0 = rans_step(lut, rp, x, lt, K);
+        const uint32_t e1 = rans_step(lut, rp, x, lt, K);
+        float2 v = make_float2(raw_value<DT>(e0), raw_value<DT>(e1));
+        if constexpr (DT == EQ_E4M3) {
+            if (!small_scales) v = mul2(v, make_float2(0x1p120f, 0x1p120f));
+        }
+        o[r / 2] = pack_bf16x2(mul2(v, s2));
+    }
+    st_global_v4(dst, make_uint4(o[0], o[1], o[2], o[3]));
+    pw += rp - rp0;
+}
+
 // Decode one chunk whose slot table is ready at `lut` (n_present >= 2) or
 // whose single symbol's stored byte is `single` (n_present == 1).  Returns
 // false if a bounded wait gave up (the warp must stop).
@@ -625,6 +650,37 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, co
     __syncwarp();
     uint32_t limit = pbytes ? 0u : kNoLimit;
     uint32_t pw = 0;
+    if constexpr (LAYOUT == kRowUniform) {
+        // runs of groups within one row (scale fixed), two groups per ring check
+        uint32_t g = 0;
+        while (g < n_full && !ctl->dead) {
+            const uint32_t run = min((O.cols - cur.col) / kGroupSyms, n_full - g);
+            const float2 s2 = make_float2(cur.scale, cur.scale);
+            uint32_t i = 0;
+            for (; i + 1 < run; i += 2, dst += 2 * kGroupSyms) {
+                if (pw >= limit) {
+                    limit = ring_service(ctl, ring, mbar, pw);
+                    if (ctl->dead) break;
+                }
+                group_row<DT>(lut, ring, pw, x, lt, s2, O.small_scales, dst);
+                group_row<DT>(lut, ring, pw, x, lt, s2, O.small_scales, dst + kGroupSyms);
+            }
+            if (i < run && !ctl->dead) {
+                if (pw >= limit) limit = ring_service(ctl, ring, mbar, pw);
+                if (!ctl->dead) {
+                    group_row<DT>(lut, ring, pw, x, lt, s2, O.small_scales, dst);
+                    dst += kGroupSyms;
+                }
+            }
+            g += run;
+            cur.col += run * kGroupSyms;
+            if (cur.col == O.cols) {
+                cur.col = 0;
+                ++cur.row;
+                if (g < n_full) cur.scale = row_scale<DT>(O, cur.row);
+            }
+        }
+    } else {
     for (uint32_t g = 0; g < n_full; ++g, dst += kGroupSyms) {
 #if EQ_VOTE_SERVICE
         if (__any_sync(kFull, pw >= limit)) {  // warp-uniform by construction
@@ -659,6 +715,7 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, co
             cursor_advance<DT, LAYOUT>(O, first + (uint64_t)g * kGroupSyms + kGroup * lane, cur);
         }
         pw += rp - rp0;
+    }
     }
     if (tail && !ctl->dead) {
         if (pw >= limit) limit = ring_service(ctl, ring, mbar, pw);
