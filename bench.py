@@ -410,7 +410,7 @@ def bench_eqw(args, d: Dist) -> dict | None:
         "gsym_s": round(gsym, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": None,
-                     "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "eq_rans_decode_dequant_kernel",
+                     "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "eq_decode_kernel",
                      "alg_bytes_per_launch": int(alg_per_launch), "launch_ms": round(launch_ms, 4)},
         "with_gemv_consumer": {"value": round(value_b, 2), "unit": UNIT, "ms_per_step": round(ms_b_max / args.steps, 3),
                                "loop_bytes_frac": round((alg_bytes_pass + dec_bytes_pass) * args.steps

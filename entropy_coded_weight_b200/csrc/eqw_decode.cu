@@ -607,6 +607,47 @@ __device__ __forceinline__ void group_row(uint32_t lut, uint32_t ring, uint32_t 
     pw += rp - rp0;
 }
 
+#ifndef EQ_RANK_DEQUANT
+#define EQ_RANK_DEQUANT 1
+#endif
+
+// Rank mode: with 2..32 distinct symbols and a warp-uniform row per group, the
+// slot table's low byte holds the symbol's rank (index in the ascending
+// frequency list) and lane r keeps fp32_rn(value(symbol of rank r) * row
+// scale).  A decoded symbol's dequantised value is then one shuffle from the
+// lane named by its rank (shfl uses only the low 5 bits of the entry).
+template <uint32_t LAYOUT>
+__device__ __forceinline__ bool rank_mode(uint32_t n_present) {
+    return EQ_RANK_DEQUANT && LAYOUT == kRowUniform && n_present >= 2 && n_present <= 32;
+}
+
+// Exact fp32 value of a symbol byte (Int8 or E4M3).
+template <int DT>
+__device__ __forceinline__ float symbol_value(uint32_t sym) {
+    if constexpr (DT == EQ_INT8) {
+        return static_cast<float>(static_cast<int8_t>(sym & 0xFFu));
+    } else {
+        return __fmul_rn(__uint_as_float(((sym & 0x80u) << 24) | ((sym & 0x7Fu) << 20)), 0x1p120f);
+    }
+}
+
+// One 256-symbol group in rank mode: 8 steps, 8 shuffles, one 16-byte store.
+__device__ __forceinline__ void group_rank(uint32_t lut, uint32_t ring, uint32_t &pw, uint32_t &x, uint32_t lt,
+                                           float vr, uint16_t *dst) {
+    const uint32_t rp0 = ring + (pw & (kRingBytes - 1));
+    uint32_t rp = rp0;
+    const StepK K{};
+    uint32_t o[4];
+#pragma unroll
+    for (int r = 0; r < 8; r += 2) {
+        const uint32_t e0 = rans_step(lut, rp, x, lt, K);
+        const uint32_t e1 = rans_step(lut, rp, x, lt, K);
+        o[r / 2] = pack_bf16x2(make_float2(__shfl_sync(kFull, vr, e0), __shfl_sync(kFull, vr, e1)));
+    }
+    st_global_v4(dst, make_uint4(o[0], o[1], o[2], o[3]));
+    pw += rp - rp0;
+}
+
 // Decode one chunk whose slot table is ready at `lut` (n_present >= 2) or
 // whose single symbol's stored byte is `single` (n_present == 1).  Returns
 // false if a bounded wait gave up (the warp must stop).
@@ -614,7 +655,8 @@ template <int DT, uint32_t LAYOUT>
 __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, const StepK &K, uint64_t first,
                                             uint32_t n, uint32_t n_words, const uint8_t *payload, bool single_sym,
                                             uint32_t single, uint32_t x, uint32_t lut, uint32_t ring, uint32_t mbar,
-                                            RingCtl *ctl, uint32_t lane, uint32_t lt) {
+                                            RingCtl *ctl, uint32_t lane, uint32_t lt, bool by_rank,
+                                            uint32_t lane_sym) {
     const uint32_t n_full = n / kGroupSyms;
     const uint32_t tail = n % kGroupSyms;
     Cursor cur{0, 0, 0.f};
@@ -650,7 +692,56 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, co
     __syncwarp();
     uint32_t limit = pbytes ? 0u : kNoLimit;
     uint32_t pw = 0;
+    bool tail_done = false;
     if constexpr (LAYOUT == kRowUniform) {
+      if (by_rank) {
+        // runs of groups within one row, two groups per ring check; lane r holds
+        // the dequantised value of rank r for the current row
+        const float vraw = symbol_value<DT>(lane_sym);
+        uint32_t g = 0;
+        while (g < n_full && !ctl->dead) {
+            const uint32_t run = min((O.cols - cur.col) / kGroupSyms, n_full - g);
+            const float vr = __fmul_rn(vraw, __ldg(O.scales + cur.row));
+            uint32_t i = 0;
+            for (; i + 1 < run; i += 2, dst += 2 * kGroupSyms) {
+                if (pw >= limit) {
+                    limit = ring_service(ctl, ring, mbar, pw);
+                    if (ctl->dead) break;
+                }
+                group_rank(lut, ring, pw, x, lt, vr, dst);
+                group_rank(lut, ring, pw, x, lt, vr, dst + kGroupSyms);
+            }
+            if (i < run && !ctl->dead) {
+                if (pw >= limit) limit = ring_service(ctl, ring, mbar, pw);
+                if (!ctl->dead) {
+                    group_rank(lut, ring, pw, x, lt, vr, dst);
+                    dst += kGroupSyms;
+                }
+            }
+            g += run;
+            cur.col += run * kGroupSyms;
+            if (cur.col == O.cols) {
+                cur.col = 0;
+                ++cur.row;
+            }
+        }
+        if (tail && !ctl->dead) {
+            if (pw >= limit) limit = ring_service(ctl, ring, mbar, pw);
+            if (!ctl->dead) {
+                uint32_t e8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                rans_tail(lut, ring, x, pw, lt, lane, tail, e8);
+                const float vr = __fmul_rn(vraw, __ldg(O.scales + cur.row));
+                const uint32_t mine = tail > kGroup * lane ? min(8u, tail - kGroup * lane) : 0u;
+                const uint64_t idx = first + (uint64_t)n_full * kGroupSyms + kGroup * lane;
+#pragma unroll
+                for (uint32_t r = 0; r < 8; ++r) {
+                    const float v = __shfl_sync(kFull, vr, e8[r]);
+                    if (r < mine) O.out[idx + r] = to_bf16(v);
+                }
+            }
+        }
+        tail_done = true;
+      } else {
         // runs of groups within one row (scale fixed), two groups per ring check
         uint32_t g = 0;
         while (g < n_full && !ctl->dead) {
@@ -680,6 +771,7 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, co
                 if (g < n_full) cur.scale = row_scale<DT>(O, cur.row);
             }
         }
+      }
     } else {
     for (uint32_t g = 0; g < n_full; ++g, dst += kGroupSyms) {
 #if EQ_VOTE_SERVICE
@@ -717,7 +809,7 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, co
         pw += rp - rp0;
     }
     }
-    if (tail && !ctl->dead) {
+    if (tail && !tail_done && !ctl->dead) {
         if (pw >= limit) limit = ring_service(ctl, ring, mbar, pw);
         if (!ctl->dead) {
             uint32_t e8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -779,7 +871,7 @@ __device__ __forceinline__ bool load_head(const DecodeParams &P, const MatJob &M
 // a warp's slot table.  Returns validity (warp-uniform).
 __device__ __forceinline__ bool warp_table(const uint32_t *tab, uint32_t n_present, uint32_t lane,
                                            uint32_t *entries_out, uint32_t *cum_out, uint32_t *lut,
-                                           uint32_t sym_xor) {
+                                           uint32_t sym_xor, bool by_rank) {
     uint32_t run = 0;
     int prev_sym = -1;
     bool ok = true;
@@ -811,7 +903,8 @@ __device__ __forceinline__ bool warp_table(const uint32_t *tab, uint32_t n_prese
                 const uint32_t sq = __shfl_sync(kFull, sym, q);
                 for (uint32_t t = lane; t < fq; t += 32) {
                     const uint32_t slot = cq + t;
-                    if (slot < kProbTotal && fq < kProbTotal) lut[slot] = (fq << 20) | (t << 8) | (sq ^ sym_xor);
+                    if (slot < kProbTotal && fq < kProbTotal)
+                        lut[slot] = (fq << 20) | (t << 8) | (by_rank ? base + q : (sq ^ sym_xor));
                 }
             }
         }
@@ -879,7 +972,7 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
                     ChunkHead h;
                     bool ok = load_head(P, M, k0, lane, h);
                     if (ok) ok = warp_table(reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes), h.n_present,
-                                            lane, ref_entries, ref_cum, nullptr, 0u);
+                                            lane, ref_entries, ref_cum, nullptr, 0u, false);
                     if (lane == 0) {
                         blk[0] = ok ? h.n_present : 0u;
                         blk[1] = ok;
@@ -888,12 +981,13 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
                 __syncthreads();
                 const uint32_t np = blk[0];
                 if (blk[1] && np > 1) {
+                    const bool by_rank = rank_mode<LAYOUT>(np);
                     for (uint32_t i = 0; i < np; ++i) {
                         const uint32_t e = ref_entries[i], c = ref_cum[i];
                         const uint32_t f = e >> 16, sy = e & 0xFFu;
+                        const uint32_t low = by_rank ? i : stored_byte<DT>(sy);
                         for (uint32_t t = threadIdx.x; t < f; t += WARPS * 32)
-                            if (c + t < kProbTotal && f < kProbTotal)
-                                lut[c + t] = (f << 20) | (t << 8) | stored_byte<DT>(sy);
+                            if (c + t < kProbTotal && f < kProbTotal) lut[c + t] = (f << 20) | (t << 8) | low;
                     }
                 }
                 __syncthreads();
@@ -915,7 +1009,8 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
             }
             decode_body<DT, LAYOUT>(P.status, out_ctx(M), K, (uint64_t)k * kChunkSyms, h.n, h.n_words,
                                     h.rec + h.table_bytes, np == 1, stored_byte<DT>(ref_entries[0] & 0xFFu), h.x,
-                                    lut_addr, ring, mbar, ctl, lane, lt);
+                                    lut_addr, ring, mbar, ctl, lane, lt, rank_mode<LAYOUT>(np),
+                                    ref_entries[lane < np ? lane : 0] & 0xFFu);
             __syncwarp();
         }
     } else {
@@ -929,7 +1024,8 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
             if (!load_head(P, M, k, lane, h)) continue;
             const uint32_t *tab = reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes);
             __syncwarp();  // the previous chunk's reads of the slot table are done
-            const bool ok = warp_table(tab, h.n_present, lane, nullptr, nullptr, lut, stored_byte<DT>(0u));
+            const bool by_rank = rank_mode<LAYOUT>(h.n_present);
+            const bool ok = warp_table(tab, h.n_present, lane, nullptr, nullptr, lut, stored_byte<DT>(0u), by_rank);
             if (!ok) {
                 flag(P.status, EQ_DEV_BAD_TABLE);
                 continue;
@@ -937,7 +1033,8 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
             __syncwarp();
             decode_body<DT, LAYOUT>(P.status, out_ctx(M), K, (uint64_t)k * kChunkSyms, h.n, h.n_words,
                                     h.rec + h.table_bytes, h.n_present == 1, stored_byte<DT>(tab[0] & 0xFFu), h.x,
-                                    lut_addr, ring, mbar, ctl, lane, lt);
+                                    lut_addr, ring, mbar, ctl, lane, lt, by_rank,
+                                    tab[lane < h.n_present ? lane : 0] & 0xFFu);
             __syncwarp();
         }
     }
