@@ -51,7 +51,13 @@ using namespace eqw;
 namespace {
 
 constexpr uint32_t kFull = 0xFFFFFFFFu;
-constexpr uint32_t kRingBytes = 4096;  // per warp: eight 512-byte segments ...
+#ifndef EQ_RING_BYTES
+#define EQ_RING_BYTES 2048
+#endif
+#ifndef EQ_CHAINS
+#define EQ_CHAINS 2
+#endif
+constexpr uint32_t kRingBytes = EQ_RING_BYTES;  // per chain: 512-byte segments ...
 constexpr uint32_t kSegBytes = 512;    // one TMA segment = 256 words
 constexpr uint32_t kRingSegs = kRingBytes / kSegBytes;
 // ... followed by a 512-byte mirror of segment slot 0, so the up to 512 bytes
@@ -65,7 +71,7 @@ constexpr long long kWaitCycles = 2000000000LL;
 constexpr uint32_t kNoLimit = 0xFFFFFFFFu;
 
 #ifndef EQ_SHARED_WARPS
-#define EQ_SHARED_WARPS 32
+#define EQ_SHARED_WARPS 24
 #endif
 #ifndef EQ_SHARED_MIN_CTAS
 #define EQ_SHARED_MIN_CTAS 1
@@ -648,6 +654,116 @@ __device__ __forceinline__ void group_rank(uint32_t lut, uint32_t ring, uint32_t
     pw += rp - rp0;
 }
 
+// A chunk record's header fields and this lane's initial state.
+struct ChunkHead {
+    const uint8_t *rec;
+    uint32_t n, n_words, n_present, table_bytes;
+    uint32_t x;
+};
+
+// Two chunks per warp in lockstep (rank mode, row-uniform layout, both
+// chunks 65536 symbols, cols a multiple of 512): every step of chunk A is
+// followed by the same step of chunk B, giving each warp two independent
+// state chains whose latencies overlap.  Row changes fall on 512-symbol
+// boundaries, i.e. between pairs of groups.
+struct Chain {
+    uint32_t x, pw, limit, row, col;
+    float vr;
+    uint16_t *dst;
+};
+
+__device__ __forceinline__ void group2_rank(uint32_t lut, uint32_t ringA, uint32_t ringB, Chain &A, Chain &B,
+                                            uint32_t lt) {
+    const uint32_t a0 = ringA + (A.pw & (kRingBytes - 1));
+    const uint32_t b0 = ringB + (B.pw & (kRingBytes - 1));
+    uint32_t ra = a0, rb = b0;
+    const StepK K{};
+    uint32_t oa[4], ob[4];
+#pragma unroll
+    for (int r = 0; r < 8; r += 2) {
+        const uint32_t ea0 = rans_step(lut, ra, A.x, lt, K);
+        const uint32_t eb0 = rans_step(lut, rb, B.x, lt, K);
+        const uint32_t ea1 = rans_step(lut, ra, A.x, lt, K);
+        const uint32_t eb1 = rans_step(lut, rb, B.x, lt, K);
+        oa[r / 2] = pack_bf16x2(make_float2(__shfl_sync(kFull, A.vr, ea0), __shfl_sync(kFull, A.vr, ea1)));
+        ob[r / 2] = pack_bf16x2(make_float2(__shfl_sync(kFull, B.vr, eb0), __shfl_sync(kFull, B.vr, eb1)));
+    }
+    st_global_v4(A.dst, make_uint4(oa[0], oa[1], oa[2], oa[3]));
+    st_global_v4(B.dst, make_uint4(ob[0], ob[1], ob[2], ob[3]));
+    A.pw += ra - a0;
+    B.pw += rb - b0;
+    A.dst += kGroupSyms;
+    B.dst += kGroupSyms;
+}
+
+// Returns false if a bounded wait gave up (the warp must stop).
+__device__ __forceinline__ bool pair_start(RingCtl *ctl, const ChunkHead &h) {
+    if ((threadIdx.x & 31u) == 0) {
+        const uint32_t pbytes = (2u * h.n_words + 15u) & ~15u;
+        ctl->payload = h.rec + h.table_bytes;
+        ctl->pbytes = pbytes;
+        ctl->n_segs = (pbytes + kSegBytes - 1) / kSegBytes;
+        ctl->issued = 0;
+        ctl->ready = 0;
+    }
+    return true;
+}
+
+template <int DT>
+__device__ __forceinline__ bool decode_pair(int32_t *status, const OutCtx &O, const ChunkHead &hA,
+                                            const ChunkHead &hB, uint64_t firstA, uint64_t firstB, uint32_t lut,
+                                            uint32_t ringA, uint32_t ringB, uint32_t mbarA, uint32_t mbarB,
+                                            RingCtl *ctlA, RingCtl *ctlB, uint32_t lane, uint32_t lt,
+                                            uint32_t lane_sym) {
+    pair_start(ctlA, hA);
+    pair_start(ctlB, hB);
+    __syncwarp();
+    const float vraw = symbol_value<DT>(lane_sym);
+    Chain A, B;
+    A.x = hA.x;
+    B.x = hB.x;
+    A.pw = B.pw = 0;
+    A.limit = hA.n_words ? 0u : kNoLimit;
+    B.limit = hB.n_words ? 0u : kNoLimit;
+    A.row = (uint32_t)(firstA / O.cols);
+    A.col = (uint32_t)(firstA - (uint64_t)A.row * O.cols);
+    B.row = (uint32_t)(firstB / O.cols);
+    B.col = (uint32_t)(firstB - (uint64_t)B.row * O.cols);
+    A.vr = __fmul_rn(vraw, __ldg(O.scales + A.row));
+    B.vr = __fmul_rn(vraw, __ldg(O.scales + B.row));
+    A.dst = O.out + firstA + kGroup * lane;
+    B.dst = O.out + firstB + kGroup * lane;
+    constexpr uint32_t kPairs = kChunkSyms / (2 * kGroupSyms);
+    for (uint32_t q = 0; q < kPairs; ++q) {
+        if (A.pw >= A.limit) A.limit = ring_service(ctlA, ringA, mbarA, A.pw);
+        if (B.pw >= B.limit) B.limit = ring_service(ctlB, ringB, mbarB, B.pw);
+        if (ctlA->dead || ctlB->dead) break;
+        group2_rank(lut, ringA, ringB, A, B, lt);
+        group2_rank(lut, ringA, ringB, A, B, lt);
+        A.col += 2 * kGroupSyms;
+        if (A.col == O.cols) {
+            A.col = 0;
+            ++A.row;
+            if (A.row < O.rows) A.vr = __fmul_rn(vraw, __ldg(O.scales + A.row));
+        }
+        B.col += 2 * kGroupSyms;
+        if (B.col == O.cols) {
+            B.col = 0;
+            ++B.row;
+            if (B.row < O.rows) B.vr = __fmul_rn(vraw, __ldg(O.scales + B.row));
+        }
+    }
+    const bool okA = ring_drain(ctlA, mbarA);
+    const bool okB = ring_drain(ctlB, mbarB);
+    if (!okA || !okB) {
+        flag(status, EQ_DEV_TIMEOUT);
+        return false;
+    }
+    if (!__all_sync(kFull, A.x == kStateLow) || A.pw != 2u * hA.n_words) flag(status, EQ_DEV_BAD_END);
+    if (!__all_sync(kFull, B.x == kStateLow) || B.pw != 2u * hB.n_words) flag(status, EQ_DEV_BAD_END);
+    return true;
+}
+
 // Decode one chunk whose slot table is ready at `lut` (n_present >= 2) or
 // whose single symbol's stored byte is `single` (n_present == 1).  Returns
 // false if a bounded wait gave up (the warp must stop).
@@ -703,18 +819,22 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, co
             const uint32_t run = min((O.cols - cur.col) / kGroupSyms, n_full - g);
             const float vr = __fmul_rn(vraw, __ldg(O.scales + cur.row));
             uint32_t i = 0;
-            for (; i + 1 < run; i += 2, dst += 2 * kGroupSyms) {
+            while (i < run) {
                 if (pw >= limit) {
                     limit = ring_service(ctl, ring, mbar, pw);
                     if (ctl->dead) break;
                 }
-                group_rank(lut, ring, pw, x, lt, vr, dst);
-                group_rank(lut, ring, pw, x, lt, vr, dst + kGroupSyms);
-            }
-            if (i < run && !ctl->dead) {
-                if (pw >= limit) limit = ring_service(ctl, ring, mbar, pw);
-                if (!ctl->dead) {
+                if (i + 1 < run) {
+                    // hot loop: no calls, pairs of groups while the ring guarantees residency
+                    do {
+                        group_rank(lut, ring, pw, x, lt, vr, dst);
+                        group_rank(lut, ring, pw, x, lt, vr, dst + kGroupSyms);
+                        i += 2;
+                        dst += 2 * kGroupSyms;
+                    } while (i + 1 < run && pw < limit);
+                } else {
                     group_rank(lut, ring, pw, x, lt, vr, dst);
+                    i += 1;
                     dst += kGroupSyms;
                 }
             }
@@ -829,11 +949,6 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, co
 
 // Header of chunk k: checks it against the directory; on success fills the
 // record pointer, counts and this lane's initial state.
-struct ChunkHead {
-    const uint8_t *rec;
-    uint32_t n, n_words, n_present, table_bytes;
-    uint32_t x;
-};
 
 __device__ __forceinline__ bool load_head(const DecodeParams &P, const MatJob &M, uint32_t k, uint32_t lane,
                                           ChunkHead &h) {
@@ -919,11 +1034,12 @@ __device__ __forceinline__ bool warp_table(const uint32_t *tab, uint32_t n_prese
 // reference frequency list (shared-table kernel only).
 template <int WARPS, bool SHARED>
 struct Smem {
+    static constexpr uint32_t kChains = SHARED ? EQ_CHAINS : 1;          // chunks decoded at once per warp
     static constexpr uint32_t kLuts = SHARED ? 1 : WARPS;
     static constexpr uint32_t kRingOff = kLuts * kLutBytes;             // + runtime pad to 128 B
-    static constexpr uint32_t kMbarOff = kRingOff + WARPS * kRingStride; // all offsets below include the pad
-    static constexpr uint32_t kCtlOff = kMbarOff + WARPS * kRingSegs * 8;
-    static constexpr uint32_t kRefOff = kCtlOff + WARPS * 32;           // 32 bytes of RingCtl per warp
+    static constexpr uint32_t kMbarOff = kRingOff + WARPS * kChains * kRingStride;  // offsets below include the pad
+    static constexpr uint32_t kCtlOff = kMbarOff + WARPS * kChains * kRingSegs * 8;
+    static constexpr uint32_t kRefOff = kCtlOff + WARPS * kChains * 32;  // 32 bytes of RingCtl per chain
     static constexpr uint32_t kBlockOff = kRefOff + (SHARED ? 2 * 256 * 4 : 0);
     static constexpr uint32_t kBytes = kBlockOff + 16 + 128;            // + worst-case alignment pad
 };
@@ -939,18 +1055,21 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
     const uint32_t base = smem_u32(smem_raw);
     const uint32_t pad = (128u - ((base + L::kRingOff) & 127u)) & 127u;
     unsigned char *padded = smem_raw + pad;  // offsets from kRingOff on are relative to this
-    const uint32_t ring = base + pad + L::kRingOff + warp * kRingStride;
-    const uint32_t mbar = base + pad + L::kMbarOff + warp * kRingSegs * 8;
-    RingCtl *ctl = reinterpret_cast<RingCtl *>(padded + L::kCtlOff + warp * 32);
+    constexpr uint32_t C = L::kChains;
+    const uint32_t ring = base + pad + L::kRingOff + warp * C * kRingStride;
+    const uint32_t mbar = base + pad + L::kMbarOff + warp * C * kRingSegs * 8;
+    RingCtl *ctl = reinterpret_cast<RingCtl *>(padded + L::kCtlOff + warp * C * 32);
     uint32_t *lut = reinterpret_cast<uint32_t *>(smem_raw) + (SHARED ? 0u : warp * kProbTotal);
     const uint32_t lut_addr = smem_u32(lut);
     const StepK K = P.k;
     if (lane == 0) {
-        for (uint32_t i = 0; i < kRingSegs; ++i) mbar_init(mbar + 8 * i, 1);
+        for (uint32_t i = 0; i < C * kRingSegs; ++i) mbar_init(mbar + 8 * i, 1);
         fence_mbar_init();
-        ctl->phase = 0;
-        ctl->dead = 0;
-        ctl->issued = ctl->ready = 0;
+        for (uint32_t c = 0; c < C; ++c) {
+            ctl[c].phase = 0;
+            ctl[c].dead = 0;
+            ctl[c].issued = ctl[c].ready = 0;
+        }
     }
     __syncwarp();
     const uint32_t lt = lanemask_lt();
@@ -964,7 +1083,7 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
             uint32_t mi = 0;
             while (mi + 1 < P.n_mats && unit >= P.mats[mi + 1].begin) ++mi;
             const MatJob &M = P.mats[mi];
-            const uint32_t k0 = (unit - M.begin) * WARPS;
+            const uint32_t k0 = (unit - M.begin) * WARPS * C;
             if (mi != cur_mat) {
                 // rebuild the block's slot table from the tile's first chunk
                 __syncthreads();
@@ -993,25 +1112,46 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
                 __syncthreads();
                 cur_mat = mi;
             }
-            const uint32_t k = k0 + warp;
-            if (k >= M.n_chunks || ctl->dead) continue;
-            ChunkHead h;
-            if (!load_head(P, M, k, lane, h)) continue;
             const uint32_t np = blk[0];
-            bool same = blk[1] && h.n_present == np;
-            if (same) {
-                const uint32_t *tab = reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes);
-                for (uint32_t i = lane; i < np; i += 32) same = same && tab[i] == ref_entries[i];
+            const uint32_t lane_sym = ref_entries[lane < np ? lane : 0] & 0xFFu;
+            // this warp's chunks: k0 + warp (+ WARPS for the second chain)
+            ChunkHead hc[C];
+            bool have[C];
+            for (uint32_t c = 0; c < C; ++c) {
+                const uint32_t k = k0 + warp + c * WARPS;
+                have[c] = k < M.n_chunks && !ctl[0].dead && !ctl[C - 1].dead;
+                if (have[c]) have[c] = load_head(P, M, k, lane, hc[c]);
+                if (have[c]) {
+                    bool same = blk[1] && hc[c].n_present == np;
+                    if (same) {
+                        const uint32_t *tab = reinterpret_cast<const uint32_t *>(hc[c].rec + kRecordHeadBytes);
+                        for (uint32_t i = lane; i < np; i += 32) same = same && tab[i] == ref_entries[i];
+                    }
+                    if (!__all_sync(kFull, same)) {
+                        flag(P.status, EQ_DEV_BAD_TABLE);
+                        have[c] = false;
+                    }
+                }
             }
-            if (!__all_sync(kFull, same)) {
-                flag(P.status, EQ_DEV_BAD_TABLE);
-                continue;
+            const OutCtx O = out_ctx(M);
+            if constexpr (C == 2 && LAYOUT == kRowUniform) {
+                if (have[0] && have[1] && rank_mode<LAYOUT>(np) && hc[0].n == kChunkSyms &&
+                    hc[1].n == kChunkSyms && O.cols % (2 * kGroupSyms) == 0) {
+                    decode_pair<DT>(P.status, O, hc[0], hc[1], (uint64_t)(k0 + warp) * kChunkSyms,
+                                    (uint64_t)(k0 + warp + WARPS) * kChunkSyms, lut_addr, ring, ring + kRingStride,
+                                    mbar, mbar + 8 * kRingSegs, ctl, ctl + 1, lane, lt, lane_sym);
+                    __syncwarp();
+                    continue;
+                }
             }
-            decode_body<DT, LAYOUT>(P.status, out_ctx(M), K, (uint64_t)k * kChunkSyms, h.n, h.n_words,
-                                    h.rec + h.table_bytes, np == 1, stored_byte<DT>(ref_entries[0] & 0xFFu), h.x,
-                                    lut_addr, ring, mbar, ctl, lane, lt, rank_mode<LAYOUT>(np),
-                                    ref_entries[lane < np ? lane : 0] & 0xFFu);
-            __syncwarp();
+            for (uint32_t c = 0; c < C; ++c) {
+                if (!have[c] || ctl->dead) continue;
+                decode_body<DT, LAYOUT>(P.status, O, K, (uint64_t)(k0 + warp + c * WARPS) * kChunkSyms, hc[c].n,
+                                        hc[c].n_words, hc[c].rec + hc[c].table_bytes, np == 1,
+                                        stored_byte<DT>(ref_entries[0] & 0xFFu), hc[c].x, lut_addr, ring, mbar, ctl,
+                                        lane, lt, rank_mode<LAYOUT>(np), lane_sym);
+                __syncwarp();
+            }
         }
     } else {
         const uint32_t stride = gridDim.x * WARPS;
@@ -1174,7 +1314,8 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
             J.dtype = d.info.dtype;
             J.layout = lay;
             J.small_scales = d.small_scales ? 1u : 0u;
-            Pv.total_units += sh ? (d.info.n_chunks + kSharedWarps - 1) / kSharedWarps : d.info.n_chunks;
+            const uint32_t per_tile = kSharedWarps * EQ_CHAINS;
+            Pv.total_units += sh ? (d.info.n_chunks + per_tile - 1) / per_tile : d.info.n_chunks;
             if (d.info.n_outliers) {
                 ScatterJob &O = Q.jobs[Q.n_jobs++];
                 O.rec = reinterpret_cast<const uint32_t *>(m->d_blob + d.outliers_off);
