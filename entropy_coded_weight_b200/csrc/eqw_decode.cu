@@ -28,9 +28,16 @@
 //               (ballot + popcount).
 //   dequant     lane l decodes symbols 8l..8l+7 of each 256-symbol group, so
 //               every 8 steps it holds 8 consecutive outputs: value * row scale
-//               in fp32 (round to nearest even, packed f32x2 multiplies),
-//               packed to bf16 (round to nearest even) and stored as one
-//               16-byte vector; a warp's 32 stores cover 512 contiguous bytes.
+//               in fp32 (round to nearest even), packed to bf16 (round to
+//               nearest even) and stored as one 16-byte vector; a warp's 32
+//               stores cover 512 contiguous bytes.  Rank mode (2..32 distinct
+//               symbols, cols % 256 == 0): the slot table's low byte is the
+//               symbol's rank and lane r holds the fp32 product for rank r of
+//               the current row, so a symbol's product is one shuffle.
+//   chains      in rank mode with full chunks and cols % 512 == 0 each warp of
+//               the shared-table kernel decodes two chunks step by step in
+//               lockstep, so two independent state chains hide each other's
+//               latency.
 // KB3, eq_outlier_scatter_kernel -- out[r * cols + c] = bf16(v) for the super
 // weights, after KB2 on the same stream.
 //
@@ -95,20 +102,12 @@ struct MatJob {
     uint32_t small_scales;        // all |scale| < 2^8: E4M3 dequant in one multiply
 };
 
-// Multipliers of the step's IMAD forms.  They arrive as kernel parameters so
-// that the compiler keeps them as multiplications on the FMA pipe rather than
-// rewriting them into shifts on the busier integer ALU pipe.
-struct StepK {
-    uint32_t two, k2e20, k2e14, k2e12, k2e24, kneg4096, k2e16, pad;
-};
-
 struct DecodeParams {
     const uint8_t *blob;
     uint64_t blob_len;
     int32_t *status;
     uint32_t n_mats;
     uint32_t total_units;
-    StepK k;
     MatJob mats[kMaxMatsPerLaunch];
 };
 
@@ -191,28 +190,9 @@ __device__ __forceinline__ void st_global_v4(uint16_t *p, uint4 v) {
 }
 
 // ---- number formats ----------------------------------------------------------------
-// Two fp32 products, each rounded to nearest even (Blackwell packed multiply).
-__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
-    unsigned long long A, B, C;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a.x), "f"(a.y));
-    asm("mov.b64 %0, {%1, %2};" : "=l"(B) : "f"(b.x), "f"(b.y));
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(C) : "l"(A), "l"(B));
-    float2 c;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(c.x), "=f"(c.y) : "l"(C));
-    return c;
-}
-
-#ifndef EQ_F32X2
-#define EQ_F32X2 0
-#endif
-
-// Two fp32 products rounded to nearest even, packed or as two multiplies.
+// Two fp32 products, each rounded to nearest even.
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-#if EQ_F32X2
-    return mul2_rn(a, b);
-#else
     return make_float2(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y));
-#endif
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float2 v) {
@@ -225,25 +205,7 @@ __device__ __forceinline__ uint16_t to_bf16(float v) {
     return *reinterpret_cast<uint16_t *>(&h);
 }
 
-// Int8: two's complement.  E4M3 (OCP E4M3FN, bias 7): the 7 exponent and
-// mantissa bits placed at bit 20 of an fp32 give exactly value * 2^-120
-// (subnormal codes included); the factor 2^120 is applied exactly, either on
-// its own or folded into a scale below 2^8 (same real product, one rounding).
-#ifndef EQ_INT8_MAGIC
-#define EQ_INT8_MAGIC 0
-#endif
-
-// Byte the slot table stores for a symbol.  With EQ_INT8_MAGIC, Int8 symbols
-// are stored with the sign bit flipped: then the float with bits
-// 0x4B000000 | byte is exactly 2^23 + 128 + value, and one exact subtraction
-// (FMA pipe) replaces an int-to-float conversion (conversion pipe).
-template <int DT>
-__host__ __device__ constexpr uint32_t stored_byte(uint32_t sym) {
-    return (DT == EQ_INT8 && EQ_INT8_MAGIC) ? (sym ^ 0x80u) : sym;
-}
-constexpr float kInt8Magic = 8388736.0f;  // 2^23 + 128
-
-// Value of the symbol whose stored byte is the low byte of e.  Int8: two's
+// Value of the symbol in the low byte of e.  Int8: two's
 // complement.  E4M3 (OCP E4M3FN, bias 7): the 7 exponent and mantissa bits
 // placed at bit 20 of an fp32 give exactly value * 2^-120 (subnormal codes
 // included); the factor 2^120 is applied exactly, on its own or folded into
@@ -251,11 +213,7 @@ constexpr float kInt8Magic = 8388736.0f;  // 2^23 + 128
 template <int DT>
 __device__ __forceinline__ float raw_value(uint32_t e) {
     if constexpr (DT == EQ_INT8) {
-#if EQ_INT8_MAGIC
-        return __fadd_rn(__uint_as_float((e & 0xFFu) | 0x4B000000u), -kInt8Magic);
-#else
         return static_cast<float>(static_cast<int8_t>(e & 0xFFu));
-#endif
     } else {
         return __uint_as_float(((e & 0x80u) << 24) | ((e & 0x7Fu) << 20));
     }
@@ -405,14 +363,6 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
     return v;
 }
 
-#ifndef EQ_TOTAL_SHFL
-#define EQ_TOTAL_SHFL 0
-#endif
-
-#ifndef EQ_TOTAL_MODE
-#define EQ_TOTAL_MODE 0  // 0: popcount of the ballot, 1: warp reduction, 2: shuffle from lane 31
-#endif
-
 // One step of all 32 lanes.  `lut` is the shared-memory address of the slot
 // table; `rp` the shared-memory address of the next unread word (inside the
 // ring or its mirror), advanced past the words this step consumes.  Returns
@@ -420,51 +370,20 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
 //   slot = x & 4095, e = lut[slot] = f << 20 | (slot - cum) << 8 | byte
 //   x' = f * (x >> 12) + (slot - cum) = f * ((x >> 12) - 4096) + (e >> 8)
 // Every lane reads a word (the ring always holds valid memory) and keeps it
-// only if it renormalises, so the step has no branch.
-#ifndef EQ_PARAM_K
-#define EQ_PARAM_K 0
-#endif
-#ifndef EQ_SEL_MERGE
-#define EQ_SEL_MERGE 1
-#endif
-
-__device__ __forceinline__ uint32_t rans_step(uint32_t lut, uint32_t &rp, uint32_t &x, uint32_t lt, const StepK &Kp) {
-#if EQ_PARAM_K
-    const StepK &K = Kp;
-#else
-    (void)Kp;
-    constexpr StepK K{2u, 1u << 20, 1u << 14, 1u << 12, 1u << 24, 0u - kProbTotal, 1u << 16, 0u};
-#endif
-    const uint32_t addr = mad_hi(mad_lo(x, K.k2e20, 0u), K.k2e14, lut);  // lut + 4 * (x & 4095)
+// only if it renormalises (a select, not a branch).  Shifts and field
+// extractions are written as IMADs (mad.hi by a power of two) so that they
+// run on the FMA pipe next to the busier integer ALU pipe.
+__device__ __forceinline__ uint32_t rans_step(uint32_t lut, uint32_t &rp, uint32_t &x, uint32_t lt) {
+    const uint32_t addr = mad_hi(mad_lo(x, 1u << 20, 0u), 1u << 14, lut);  // lut + 4 * (x & 4095)
     const uint32_t e = lds_u32(addr);
-    const uint32_t t = mad_hi(x, K.k2e20, K.kneg4096);                    // (x >> 12) - 4096
-    x = mad_lo(mad_hi(e, K.k2e12, 0u), t, mad_hi(e, K.k2e24, 0u));
+    const uint32_t t = mad_hi(x, 1u << 20, 0u - kProbTotal);               // (x >> 12) - 4096
+    x = mad_lo(mad_hi(e, 1u << 12, 0u), t, mad_hi(e, 1u << 24, 0u));
     const bool need = x < kStateLow;
-    const uint32_t x_before_merge = x;
-    (void)x_before_merge;
     const uint32_t b = __ballot_sync(kFull, need);
-    const uint32_t pre = __popc(b & lt);
-    const uint32_t w = lds_u16(mad_lo(pre, K.two, rp));
-#if EQ_SEL_MERGE
-    const uint32_t xr = mad_lo(x, K.k2e16, w);
+    const uint32_t w = lds_u16(mad_lo(__popc(b & lt), 2u, rp));
+    const uint32_t xr = mad_lo(x, 1u << 16, w);
     x = need ? xr : x;
-#else
-    if (need) x = mad_lo(x, K.k2e16, w);
-#endif
-#if EQ_TOTAL_MODE == 3
-    // a second ballot whose only use is warp-uniform, so the count can live on
-    // the uniform datapath instead of the vector popcount (conversion) pipe
-    uint32_t bu;
-    asm volatile("{\n\t.reg .pred q;\n\tsetp.lt.u32 q, %1, 65536;\n\tvote.sync.ballot.b32 %0, q, 0xffffffff;\n\t}"
-                 : "=r"(bu) : "r"(x_before_merge));
-    rp = mad_lo(__popc(bu), K.two, rp);
-#elif EQ_TOTAL_MODE == 1
-    rp = mad_lo(__reduce_add_sync(kFull, need ? 1u : 0u), K.two, rp);
-#elif EQ_TOTAL_MODE == 2
-    rp = mad_lo(__shfl_sync(kFull, pre + (need ? 1u : 0u), 31), K.two, rp);
-#else
-    rp = mad_lo(__popc(b), K.two, rp);
-#endif
+    rp = mad_lo(__popc(b), 2u, rp);
     return e;
 }
 
@@ -501,13 +420,6 @@ struct OutCtx {
 __device__ __forceinline__ OutCtx out_ctx(const MatJob &M) {
     return OutCtx{M.out, M.scales, M.n_elems, M.cols, (uint32_t)(M.n_elems / M.cols), M.small_scales != 0};
 }
-
-#ifndef EQ_BRANCHLESS_CURSOR
-#define EQ_BRANCHLESS_CURSOR 0
-#endif
-#ifndef EQ_VOTE_SERVICE
-#define EQ_VOTE_SERVICE 0
-#endif
 
 // Element-wise store of `count` outputs starting at linear index idx.
 template <int DT>
@@ -551,22 +463,12 @@ __device__ __forceinline__ void cursor_init(const OutCtx &O, uint64_t first, uin
 template <int DT, uint32_t LAYOUT>
 __device__ __forceinline__ void cursor_advance(const OutCtx &O, uint64_t idx, Cursor &c) {
     if constexpr (LAYOUT == kRowUniform) {
-#if EQ_BRANCHLESS_CURSOR
-        // cols % 256 == 0: the group's row is warp-uniform; reload its scale
-        // every group (an L1 hit) instead of branching on the row change
-        c.col += kGroupSyms;
-        const bool wrap = c.col == O.cols;
-        c.col = wrap ? 0u : c.col;
-        c.row += wrap ? 1u : 0u;
-        c.scale = row_scale<DT>(O, min(c.row, O.rows - 1));
-#else
         c.col += kGroupSyms;
         if (c.col == O.cols) {
             c.col = 0;
             ++c.row;
             if (idx + kGroupSyms < O.n_elems) c.scale = row_scale<DT>(O, c.row);
         }
-#endif
     } else if constexpr (LAYOUT == kLaneRows) {
         bool moved = false;
         c.col += kGroupSyms;
@@ -597,12 +499,11 @@ __device__ __forceinline__ void group_row(uint32_t lut, uint32_t ring, uint32_t 
                                           float2 s2, bool small_scales, uint16_t *dst) {
     const uint32_t rp0 = ring + (pw & (kRingBytes - 1));
     uint32_t rp = rp0;
-    const StepK K{};
     uint32_t o[4];
 #pragma unroll
     for (int r = 0; r < 8; r += 2) {
-        const uint32_t e0 = rans_step(lut, rp, x, lt, K);
-        const uint32_t e1 = rans_step(lut, rp, x, lt, K);
+        const uint32_t e0 = rans_step(lut, rp, x, lt);
+        const uint32_t e1 = rans_step(lut, rp, x, lt);
         float2 v = make_float2(raw_value<DT>(e0), raw_value<DT>(e1));
         if constexpr (DT == EQ_E4M3) {
             if (!small_scales) v = mul2(v, make_float2(0x1p120f, 0x1p120f));
@@ -613,10 +514,6 @@ __device__ __forceinline__ void group_row(uint32_t lut, uint32_t ring, uint32_t 
     pw += rp - rp0;
 }
 
-#ifndef EQ_RANK_DEQUANT
-#define EQ_RANK_DEQUANT 1
-#endif
-
 // Rank mode: with 2..32 distinct symbols and a warp-uniform row per group, the
 // slot table's low byte holds the symbol's rank (index in the ascending
 // frequency list) and lane r keeps fp32_rn(value(symbol of rank r) * row
@@ -624,7 +521,13 @@ __device__ __forceinline__ void group_row(uint32_t lut, uint32_t ring, uint32_t 
 // lane named by its rank (shfl uses only the low 5 bits of the entry).
 template <uint32_t LAYOUT>
 __device__ __forceinline__ bool rank_mode(uint32_t n_present) {
-    return EQ_RANK_DEQUANT && LAYOUT == kRowUniform && n_present >= 2 && n_present <= 32;
+    return LAYOUT == kRowUniform && n_present >= 2 && n_present <= 32;
+}
+
+// The byte the shared table stores for list entry i (rank mode: the rank).
+template <uint32_t LAYOUT>
+__device__ __forceinline__ uint32_t table_low_byte(uint32_t n_present, uint32_t i, uint32_t sym) {
+    return rank_mode<LAYOUT>(n_present) ? i : sym;
 }
 
 // Exact fp32 value of a symbol byte (Int8 or E4M3).
@@ -642,12 +545,11 @@ __device__ __forceinline__ void group_rank(uint32_t lut, uint32_t ring, uint32_t
                                            float vr, uint16_t *dst) {
     const uint32_t rp0 = ring + (pw & (kRingBytes - 1));
     uint32_t rp = rp0;
-    const StepK K{};
     uint32_t o[4];
 #pragma unroll
     for (int r = 0; r < 8; r += 2) {
-        const uint32_t e0 = rans_step(lut, rp, x, lt, K);
-        const uint32_t e1 = rans_step(lut, rp, x, lt, K);
+        const uint32_t e0 = rans_step(lut, rp, x, lt);
+        const uint32_t e1 = rans_step(lut, rp, x, lt);
         o[r / 2] = pack_bf16x2(make_float2(__shfl_sync(kFull, vr, e0), __shfl_sync(kFull, vr, e1)));
     }
     st_global_v4(dst, make_uint4(o[0], o[1], o[2], o[3]));
@@ -672,19 +574,19 @@ struct Chain {
     uint16_t *dst;
 };
 
+// Two 256-symbol groups in rank mode, one per chain, interleaved step by step.
 __device__ __forceinline__ void group2_rank(uint32_t lut, uint32_t ringA, uint32_t ringB, Chain &A, Chain &B,
                                             uint32_t lt) {
     const uint32_t a0 = ringA + (A.pw & (kRingBytes - 1));
     const uint32_t b0 = ringB + (B.pw & (kRingBytes - 1));
     uint32_t ra = a0, rb = b0;
-    const StepK K{};
     uint32_t oa[4], ob[4];
 #pragma unroll
     for (int r = 0; r < 8; r += 2) {
-        const uint32_t ea0 = rans_step(lut, ra, A.x, lt, K);
-        const uint32_t eb0 = rans_step(lut, rb, B.x, lt, K);
-        const uint32_t ea1 = rans_step(lut, ra, A.x, lt, K);
-        const uint32_t eb1 = rans_step(lut, rb, B.x, lt, K);
+        const uint32_t ea0 = rans_step(lut, ra, A.x, lt);
+        const uint32_t eb0 = rans_step(lut, rb, B.x, lt);
+        const uint32_t ea1 = rans_step(lut, ra, A.x, lt);
+        const uint32_t eb1 = rans_step(lut, rb, B.x, lt);
         oa[r / 2] = pack_bf16x2(make_float2(__shfl_sync(kFull, A.vr, ea0), __shfl_sync(kFull, A.vr, ea1)));
         ob[r / 2] = pack_bf16x2(make_float2(__shfl_sync(kFull, B.vr, eb0), __shfl_sync(kFull, B.vr, eb1)));
     }
@@ -768,7 +670,7 @@ __device__ __forceinline__ bool decode_pair(int32_t *status, const OutCtx &O, co
 // whose single symbol's stored byte is `single` (n_present == 1).  Returns
 // false if a bounded wait gave up (the warp must stop).
 template <int DT, uint32_t LAYOUT>
-__device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, const StepK &K, uint64_t first,
+__device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, uint64_t first,
                                             uint32_t n, uint32_t n_words, const uint8_t *payload, bool single_sym,
                                             uint32_t single, uint32_t x, uint32_t lut, uint32_t ring, uint32_t mbar,
                                             RingCtl *ctl, uint32_t lane, uint32_t lt, bool by_rank,
@@ -894,11 +796,7 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, co
       }
     } else {
     for (uint32_t g = 0; g < n_full; ++g, dst += kGroupSyms) {
-#if EQ_VOTE_SERVICE
-        if (__any_sync(kFull, pw >= limit)) {  // warp-uniform by construction
-#else
         if (pw >= limit) {
-#endif
             limit = ring_service(ctl, ring, mbar, pw);
             if (ctl->dead) break;
         }
@@ -907,7 +805,7 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, co
         if constexpr (LAYOUT == kGeneric) {
             uint32_t e8[8];
 #pragma unroll
-            for (int r = 0; r < 8; ++r) e8[r] = rans_step(lut, rp, x, lt, K);
+            for (int r = 0; r < 8; ++r) e8[r] = rans_step(lut, rp, x, lt);
             store_elems<DT>(O, first + (uint64_t)g * kGroupSyms + kGroup * lane, 8, e8);
         } else {
             // dequantise pairs as they are decoded: 4 packed registers instead of 8 entries
@@ -915,8 +813,8 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, co
             uint32_t o[4];
 #pragma unroll
             for (int r = 0; r < 8; r += 2) {
-                const uint32_t e0 = rans_step(lut, rp, x, lt, K);
-                const uint32_t e1 = rans_step(lut, rp, x, lt, K);
+                const uint32_t e0 = rans_step(lut, rp, x, lt);
+                const uint32_t e1 = rans_step(lut, rp, x, lt);
                 float2 v = make_float2(raw_value<DT>(e0), raw_value<DT>(e1));
                 if constexpr (DT == EQ_E4M3) {
                     if (!O.small_scales) v = mul2(v, make_float2(0x1p120f, 0x1p120f));
@@ -986,7 +884,7 @@ __device__ __forceinline__ bool load_head(const DecodeParams &P, const MatJob &M
 // a warp's slot table.  Returns validity (warp-uniform).
 __device__ __forceinline__ bool warp_table(const uint32_t *tab, uint32_t n_present, uint32_t lane,
                                            uint32_t *entries_out, uint32_t *cum_out, uint32_t *lut,
-                                           uint32_t sym_xor, bool by_rank) {
+                                           bool by_rank) {
     uint32_t run = 0;
     int prev_sym = -1;
     bool ok = true;
@@ -1019,7 +917,7 @@ __device__ __forceinline__ bool warp_table(const uint32_t *tab, uint32_t n_prese
                 for (uint32_t t = lane; t < fq; t += 32) {
                     const uint32_t slot = cq + t;
                     if (slot < kProbTotal && fq < kProbTotal)
-                        lut[slot] = (fq << 20) | (t << 8) | (by_rank ? base + q : (sq ^ sym_xor));
+                        lut[slot] = (fq << 20) | (t << 8) | (by_rank ? base + q : sq);
                 }
             }
         }
@@ -1061,7 +959,6 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
     RingCtl *ctl = reinterpret_cast<RingCtl *>(padded + L::kCtlOff + warp * C * 32);
     uint32_t *lut = reinterpret_cast<uint32_t *>(smem_raw) + (SHARED ? 0u : warp * kProbTotal);
     const uint32_t lut_addr = smem_u32(lut);
-    const StepK K = P.k;
     if (lane == 0) {
         for (uint32_t i = 0; i < C * kRingSegs; ++i) mbar_init(mbar + 8 * i, 1);
         fence_mbar_init();
@@ -1091,7 +988,7 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
                     ChunkHead h;
                     bool ok = load_head(P, M, k0, lane, h);
                     if (ok) ok = warp_table(reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes), h.n_present,
-                                            lane, ref_entries, ref_cum, nullptr, 0u, false);
+                                            lane, ref_entries, ref_cum, nullptr, false);
                     if (lane == 0) {
                         blk[0] = ok ? h.n_present : 0u;
                         blk[1] = ok;
@@ -1100,11 +997,10 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
                 __syncthreads();
                 const uint32_t np = blk[0];
                 if (blk[1] && np > 1) {
-                    const bool by_rank = rank_mode<LAYOUT>(np);
                     for (uint32_t i = 0; i < np; ++i) {
                         const uint32_t e = ref_entries[i], c = ref_cum[i];
                         const uint32_t f = e >> 16, sy = e & 0xFFu;
-                        const uint32_t low = by_rank ? i : stored_byte<DT>(sy);
+                        const uint32_t low = table_low_byte<LAYOUT>(np, i, sy);
                         for (uint32_t t = threadIdx.x; t < f; t += WARPS * 32)
                             if (c + t < kProbTotal && f < kProbTotal) lut[c + t] = (f << 20) | (t << 8) | low;
                     }
@@ -1146,10 +1042,10 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
             }
             for (uint32_t c = 0; c < C; ++c) {
                 if (!have[c] || ctl->dead) continue;
-                decode_body<DT, LAYOUT>(P.status, O, K, (uint64_t)(k0 + warp + c * WARPS) * kChunkSyms, hc[c].n,
+                decode_body<DT, LAYOUT>(P.status, O, (uint64_t)(k0 + warp + c * WARPS) * kChunkSyms, hc[c].n,
                                         hc[c].n_words, hc[c].rec + hc[c].table_bytes, np == 1,
-                                        stored_byte<DT>(ref_entries[0] & 0xFFu), hc[c].x, lut_addr, ring, mbar, ctl,
-                                        lane, lt, rank_mode<LAYOUT>(np), lane_sym);
+                                        ref_entries[0] & 0xFFu, hc[c].x, lut_addr, ring, mbar, ctl, lane, lt,
+                                        rank_mode<LAYOUT>(np), lane_sym);
                 __syncwarp();
             }
         }
@@ -1165,14 +1061,14 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
             const uint32_t *tab = reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes);
             __syncwarp();  // the previous chunk's reads of the slot table are done
             const bool by_rank = rank_mode<LAYOUT>(h.n_present);
-            const bool ok = warp_table(tab, h.n_present, lane, nullptr, nullptr, lut, stored_byte<DT>(0u), by_rank);
+            const bool ok = warp_table(tab, h.n_present, lane, nullptr, nullptr, lut, by_rank);
             if (!ok) {
                 flag(P.status, EQ_DEV_BAD_TABLE);
                 continue;
             }
             __syncwarp();
-            decode_body<DT, LAYOUT>(P.status, out_ctx(M), K, (uint64_t)k * kChunkSyms, h.n, h.n_words,
-                                    h.rec + h.table_bytes, h.n_present == 1, stored_byte<DT>(tab[0] & 0xFFu), h.x,
+            decode_body<DT, LAYOUT>(P.status, out_ctx(M), (uint64_t)k * kChunkSyms, h.n, h.n_words,
+                                    h.rec + h.table_bytes, h.n_present == 1, tab[0] & 0xFFu, h.x,
                                     lut_addr, ring, mbar, ctl, lane, lt, by_rank,
                                     tab[lane < h.n_present ? lane : 0] & 0xFFu);
             __syncwarp();
@@ -1289,7 +1185,6 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
             for (auto &b : a)
                 for (auto &c : b) {
                     c = DecodeParams{};
-                    c.k = StepK{2u, 1u << 20, 1u << 14, 1u << 12, 1u << 24, 0u - kProbTotal, 1u << 16, 0u};
                     c.blob = m->d_blob;
                     c.blob_len = m->len;
                     c.status = d_status;
