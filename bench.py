@@ -294,19 +294,23 @@ def cpu_oracle_sample(blob: np.ndarray, target_s: float = 12.0) -> dict:
         oracle.dequant_pairs(m["dtype"], sym, m["scales"][rows])
         return cnt
 
-    # calibrate on one chunk per core, then size the sample to ~target_s
-    t0 = time.perf_counter()
+    # batches of 4 chunks per core until at least target_s of wall time has passed
+    batch = 4 * cores
+    done, n_sample, pos = 0, 0, 0
     with ThreadPoolExecutor(cores) as ex:
-        done = sum(ex.map(one, chunks[:cores]))
-    dt = time.perf_counter() - t0
-    n_chunks = int(max(cores, cores * target_s / max(dt, 1e-3)))
-    sample = [chunks[(cores + i) % len(chunks)] for i in range(n_chunks)]
-    t0 = time.perf_counter()
-    with ThreadPoolExecutor(cores) as ex:
-        done = sum(ex.map(one, sample))
-    dt = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        while True:
+            sample = [chunks[(pos + i) % len(chunks)] for i in range(batch)]
+            pos += batch
+            done += sum(ex.map(one, sample))
+            n_sample += batch
+            dt = time.perf_counter() - t0
+            if dt >= target_s:
+                break
+    sample = range(n_sample)
     return {"value": round(2.0 * done / dt / 1e9, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{len(sample)} chunks ({done} symbols) of layer 0, scalar rANS decode + dequant, "
+            "sample": f"{len(sample)} chunks ({done} symbols, cycling over the {len(chunks)} chunks of layer 0), "
+                      f"scalar rANS decode + dequant, "
                       f"{cores} threads, {dt:.1f}s", "gsym_s": round(done / dt / 1e9, 5)}
 
 
@@ -363,6 +367,31 @@ def bench_eqw(args, d: Dist) -> dict | None:
     ms_b_max, _ = combine(ms_b, 0.0, d)
     value_b = dec_bytes_all / (ms_b_max / 1e3) / 1e9
 
+    # ---- C: fused decode + GEMV, no bf16 buffers; blocks in sequence on one stream ----
+    fstream = torch.cuda.Stream(device=dev)
+    fys = [torch.empty_like(y) for y in ys]
+
+    def fused_pass():
+        for st in stack.steps:
+            st.model.decode_gemv_block(st.layer, xs, fys, streamer.status, fstream)
+
+    for _ in range(args.warmup):
+        fused_pass()
+    torch.cuda.synchronize()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(fstream)
+    for _ in range(args.steps):
+        fused_pass()
+    f1.record(fstream)
+    torch.cuda.synchronize()
+    if int(streamer.status.item()) != 0:
+        raise RuntimeError(f"fused decode status {int(streamer.status.item())}")
+    ms_c_max, _ = combine(f0.elapsed_time(f1), 0.0, d)
+    value_c = dec_bytes_all / (ms_c_max / 1e3) / 1e9
+    fused_read = statistics.mean(b["read"] for b in layer_bytes) + \
+        sum(2 * c + 4 * r for r, c in W.LLAMA70B_BLOCK)
+
     # ---- e2e: compressed weights copied from pinned host memory every step ----
     pinned = torch.from_numpy(blob).pin_memory()
     copy_stream = torch.cuda.Stream(device=dev)
@@ -415,6 +444,14 @@ def bench_eqw(args, d: Dist) -> dict | None:
         "with_gemv_consumer": {"value": round(value_b, 2), "unit": UNIT, "ms_per_step": round(ms_b_max / args.steps, 3),
                                "loop_bytes_frac": round((alg_bytes_pass + dec_bytes_pass) * args.steps
                                                         / (ms_b_max / 1e3) / 1e9 / peak, 4)},
+        "with_fused_gemv": {"value": round(value_c, 2), "unit": UNIT,
+                            "ms_per_step": round(ms_c_max / args.steps, 3),
+                            "ms_per_layer": round(ms_c_max / args.steps / len(stack.steps), 4),
+                            "hbm_frac": round(fused_read * len(stack.steps) * args.steps
+                                              / (ms_c_max / 1e3) / 1e9 / peak, 4),
+                            "kernel": "eq_decode_gemv_kernel",
+                            "note": "y = W x per matrix with W decoded in registers; value = bf16 weight bytes "
+                                    "consumed per second (2 x symbols / time), one block after another"},
         "e2e": {"value": round(value_e, 2), "unit": UNIT, "h2d_bytes_per_step": int(blob.size * stack.copies),
                 "d2h_bytes_per_step": 4, "ms_per_step": round(ms_e_max / args.steps, 3)},
         "cpu_baseline": cpu,
@@ -448,7 +485,7 @@ def bench_reference(args) -> dict:
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["eqw", "reference"], default="eqw")
     ap.add_argument("--distinct-layers", type=int, default=8)

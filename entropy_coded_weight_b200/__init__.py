@@ -188,9 +188,28 @@ class Model:
                                              _stream_handle(decode_stream), pfree, pready),
               "eq_decode_model_stream")
 
+    def decode_gemv_matrix(self, matrix: int, x, y, status, stream=None) -> None:
+        """eq_decode_gemv_matrix: y = W x without materialising W (x bf16 [cols], y fp32 [rows], device)."""
+        check(self._L.eq_decode_gemv_matrix(self._m, matrix, x.data_ptr(), y.data_ptr(), status.data_ptr(),
+                                            _stream_handle(stream)), "eq_decode_gemv_matrix")
+
+    def decode_gemv_block(self, layer: int, xs, ys, status, stream=None) -> None:
+        """eq_decode_gemv_block: ys[i] = W_i xs[i] for matrix i of ``layer`` (directory order)."""
+        n = len(xs)
+        px = (ctypes.c_void_p * max(1, n))(*(x.data_ptr() for x in xs))
+        py = (ctypes.c_void_p * max(1, n))(*(y.data_ptr() for y in ys))
+        check(self._L.eq_decode_gemv_block(self._m, layer, px, py, n, status.data_ptr(), _stream_handle(stream)),
+              "eq_decode_gemv_block")
+
 
 def gemv_bf16(w, x, y, stream=None) -> None:
     """eq_gemv_bf16: y[r] = sum_c w[r, c] * x[c] (w bf16 [rows, cols], x bf16 [cols], y fp32 [rows])."""
     rows, cols = w.shape
     check(load().eq_gemv_bf16(w.data_ptr(), x.data_ptr(), y.data_ptr(), rows, cols, _stream_handle(stream)),
           "eq_gemv_bf16")
+
+
+def selftest_wait_timeout(status, stream=None) -> None:
+    """eq_selftest_wait_timeout: make one bounded staging wait run out (about a
+    second); the kernel ORs EQ_DEV_TIMEOUT into ``status`` (device int32)."""
+    check(load().eq_selftest_wait_timeout(status.data_ptr(), _stream_handle(stream)), "eq_selftest_wait_timeout")

@@ -39,7 +39,8 @@
 //               lockstep, so two independent state chains hide each other's
 //               latency.
 // KB3, eq_outlier_scatter_kernel -- out[r * cols + c] = bf16(v) for the super
-// weights, after KB2 on the same stream.
+// weights, after KB2 on the same stream; it also checks that the stream held a
+// zero-valued placeholder there (the fused decode + GEMV relies on it).
 //
 // Every wait on a staged copy is bounded (~1 s of SM clock); on expiry the
 // warp records EQ_DEV_TIMEOUT, waits (bounded) for its copies in flight and
@@ -51,43 +52,9 @@
 #include <mutex>
 #include <vector>
 
-#include "eqw_internal.h"
-
-using namespace eqw;
+#include "eqw_device.cuh"
 
 namespace {
-
-constexpr uint32_t kFull = 0xFFFFFFFFu;
-#ifndef EQ_RING_BYTES
-#define EQ_RING_BYTES 2048
-#endif
-#ifndef EQ_CHAINS
-#define EQ_CHAINS 2
-#endif
-constexpr uint32_t kRingBytes = EQ_RING_BYTES;  // per chain: 512-byte segments ...
-constexpr uint32_t kSegBytes = 512;    // one TMA segment = 256 words
-constexpr uint32_t kRingSegs = kRingBytes / kSegBytes;
-// ... followed by a 512-byte mirror of segment slot 0, so the up to 512 bytes
-// one 256-symbol group reads from any starting offset are contiguous and the
-// per-step word address needs no wrap-around mask.
-constexpr uint32_t kRingStride = kRingBytes + kSegBytes;
-// Words the ring guarantees resident at each service check: two groups.
-constexpr uint32_t kSpan = 2 * kSegBytes;
-constexpr uint32_t kLutBytes = 4 * kProbTotal;
-constexpr long long kWaitCycles = 2000000000LL;
-constexpr uint32_t kNoLimit = 0xFFFFFFFFu;
-
-#ifndef EQ_SHARED_WARPS
-#define EQ_SHARED_WARPS 24
-#endif
-#ifndef EQ_SHARED_MIN_CTAS
-#define EQ_SHARED_MIN_CTAS 1
-#endif
-constexpr int kSharedWarps = EQ_SHARED_WARPS;      // warps per block, shared-table kernel
-constexpr int kSharedMinCtas = EQ_SHARED_MIN_CTAS; // register budget: blocks of kSharedWarps per SM
-constexpr int kPrivateWarps = 4;                   // warps per block, per-warp-table kernel
-
-enum : uint32_t { kRowUniform = 0, kLaneRows = 1, kGeneric = 2 };
 
 struct MatJob {
     const uint64_t *chunk_index;  // absolute record offsets, n_chunks + 1 entries
@@ -123,289 +90,6 @@ struct ScatterParams {
     uint32_t total;
     ScatterJob jobs[kMaxMatsPerLaunch];
 };
-
-// ---- PTX helpers: mbarrier + bulk copy (TMA, 1-D, no multicast) ---------------
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void fence_mbar_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(src), "r"(bytes), "r"(bar)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (clock64() - t0 > kWaitCycles) return false;
-    }
-}
-
-__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
-    uint16_t v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-    return v;
-}
-
-__device__ __forceinline__ uint32_t lanemask_lt() {
-    uint32_t m;
-    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-    return m;
-}
-
-__device__ __forceinline__ void st_global_v4(uint16_t *p, uint4 v) {
-    asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                 : "memory");
-}
-
-// ---- number formats ----------------------------------------------------------------
-// Two fp32 products, each rounded to nearest even.
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-    return make_float2(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y));
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float2 v) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
-    return *reinterpret_cast<uint32_t *>(&h);
-}
-
-__device__ __forceinline__ uint16_t to_bf16(float v) {
-    __nv_bfloat16 h = __float2bfloat16_rn(v);
-    return *reinterpret_cast<uint16_t *>(&h);
-}
-
-// Value of the symbol in the low byte of e.  Int8: two's
-// complement.  E4M3 (OCP E4M3FN, bias 7): the 7 exponent and mantissa bits
-// placed at bit 20 of an fp32 give exactly value * 2^-120 (subnormal codes
-// included); the factor 2^120 is applied exactly, on its own or folded into
-// a scale below 2^8 (same real product, one rounding).
-template <int DT>
-__device__ __forceinline__ float raw_value(uint32_t e) {
-    if constexpr (DT == EQ_INT8) {
-        return static_cast<float>(static_cast<int8_t>(e & 0xFFu));
-    } else {
-        return __uint_as_float(((e & 0x80u) << 24) | ((e & 0x7Fu) << 20));
-    }
-}
-
-template <int DT>
-__device__ __forceinline__ float dequant1(uint32_t e, float scale) {
-    float v = raw_value<DT>(e);
-    if constexpr (DT == EQ_E4M3) v = __fmul_rn(v, 0x1p120f);
-    return __fmul_rn(v, scale);
-}
-
-// 8 symbols (low bytes of e[]) -> 8 bf16 in one 16-byte vector.  For E4M3
-// with `folded` the scale already carries the factor 2^120.
-template <int DT>
-__device__ __forceinline__ uint4 dequant8(const uint32_t (&e)[8], float s, bool folded) {
-    const float2 s2 = make_float2(s, s);
-    uint32_t o[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float2 v = make_float2(raw_value<DT>(e[2 * i]), raw_value<DT>(e[2 * i + 1]));
-        if constexpr (DT == EQ_E4M3) {
-            if (!folded) v = mul2(v, make_float2(0x1p120f, 0x1p120f));
-        }
-        o[i] = pack_bf16x2(mul2(v, s2));
-    }
-    return make_uint4(o[0], o[1], o[2], o[3]);
-}
-
-__device__ __forceinline__ void flag(int32_t *status, int32_t bits) {
-    if ((threadIdx.x & 31u) == 0) atomicOr(status, bits);
-}
-
-// ---- word staging ring ------------------------------------------------------------
-// Per-warp bookkeeping lives in shared memory so that the decode loop keeps a
-// single register for it: `limit`, the consumed-byte count at which the next
-// group needs service (refill free slots or wait for a segment).
-struct RingCtl {
-    const uint8_t *payload;
-    uint32_t pbytes;   // payload bytes rounded up to 16
-    uint32_t n_segs;
-    uint32_t issued;
-    uint32_t ready;
-    uint32_t phase;    // bit k: parity of the next completion of mbar[k]
-    uint32_t dead;     // a bounded wait gave up
-};
-
-__device__ __forceinline__ uint32_t ring_limit(uint32_t n_segs, uint32_t issued, uint32_t ready) {
-    // safe while bytes [pw, pw + kSpan) are resident and no free slot can take a segment
-    uint32_t lim = kNoLimit;
-    if (ready < n_segs) lim = ready * kSegBytes >= kSpan - 1 ? ready * kSegBytes - (kSpan - 1) : 0u;
-    if (issued < n_segs) {
-        const uint32_t t = issued >= kRingSegs - 1 ? (issued - (kRingSegs - 1)) * kSegBytes : 0u;
-        lim = min(lim, t);
-    }
-    return lim;
-}
-
-// Refill free slots, then make payload bytes [pw, pw + kSpan) resident.  Returns
-// the new limit; on a wait that gave up sets ctl->dead and returns kNoLimit.
-__device__ __noinline__ uint32_t ring_service(RingCtl *ctl, uint32_t ring, uint32_t mbar, uint32_t pw) {
-    const uint32_t lane = threadIdx.x & 31u;
-    const uint32_t n_segs = ctl->n_segs, pbytes = ctl->pbytes;
-    uint32_t issued = ctl->issued, ready = ctl->ready, phase = ctl->phase;
-    const uint32_t horizon = pw / kSegBytes + kRingSegs;
-    if (issued < n_segs && issued < horizon) {
-        __syncwarp();
-        fence_proxy_async_smem();  // the slots being refilled were read through the generic proxy
-        do {
-            if (lane == 0) {
-                const uint32_t bytes = min(kSegBytes, pbytes - issued * kSegBytes);
-                const uint32_t slot = issued % kRingSegs;
-                const uint8_t *src = ctl->payload + (size_t)issued * kSegBytes;
-                mbar_expect_tx(mbar + 8 * slot, slot == 0 ? 2 * bytes : bytes);
-                bulk_load(ring + slot * kSegBytes, src, bytes, mbar + 8 * slot);
-                if (slot == 0) bulk_load(ring + kRingBytes, src, bytes, mbar);  // the mirror
-            }
-            ++issued;
-        } while (issued < n_segs && issued < horizon);
-    }
-    uint32_t need = (pw + kSpan - 1) / kSegBytes;  // last segment touched by bytes [pw, pw + kSpan)
-    if (need >= n_segs) need = n_segs - 1;
-    bool ok = true;
-    while (ready <= need && ready < issued) {
-        const uint32_t slot = ready % kRingSegs;
-        const bool got = mbar_wait_bounded(mbar + 8 * slot, (phase >> slot) & 1u);
-        phase ^= 1u << slot;
-        ++ready;
-        if (!__all_sync(kFull, got)) {
-            ok = false;
-            break;
-        }
-    }
-    __syncwarp();
-    if (lane == 0) {
-        ctl->issued = issued;
-        ctl->ready = ready;
-        ctl->phase = phase;
-        if (!ok) ctl->dead = 1;
-    }
-    __syncwarp();
-    return ok ? ring_limit(n_segs, issued, ready) : kNoLimit;
-}
-
-// Wait (bounded) for every copy still in flight so the ring can be reused.
-__device__ __noinline__ bool ring_drain(RingCtl *ctl, uint32_t mbar) {
-    const uint32_t lane = threadIdx.x & 31u;
-    uint32_t ready = ctl->ready, phase = ctl->phase;
-    const uint32_t issued = ctl->issued;
-    bool all_ok = true;
-    while (ready < issued) {
-        const uint32_t slot = ready % kRingSegs;
-        const bool got = mbar_wait_bounded(mbar + 8 * slot, (phase >> slot) & 1u);
-        phase ^= 1u << slot;
-        ++ready;
-        all_ok = __all_sync(kFull, got) && all_ok;
-    }
-    __syncwarp();
-    if (lane == 0) {
-        ctl->ready = ready;
-        ctl->phase = phase;
-        if (!all_ok) ctl->dead = 1;
-    }
-    __syncwarp();
-    return all_ok && !ctl->dead;
-}
-
-// ---- the rANS step ---------------------------------------------------------------
-// Integer helpers that run on the IMAD (FMA) pipe, keeping the ALU pipe free:
-// mad.hi gives hi32(a * b) + c, so shifts right and field extraction cost one
-// IMAD each.
-__device__ __forceinline__ uint32_t mad_hi(uint32_t a, uint32_t b, uint32_t c) {
-    uint32_t d;
-    asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-
-__device__ __forceinline__ uint32_t mad_lo(uint32_t a, uint32_t b, uint32_t c) {
-    uint32_t d;
-    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-
-__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
-}
-
-// One step of all 32 lanes.  `lut` is the shared-memory address of the slot
-// table; `rp` the shared-memory address of the next unread word (inside the
-// ring or its mirror), advanced past the words this step consumes.  Returns
-// the slot entry (low byte: the stored symbol byte).
-//   slot = x & 4095, e = lut[slot] = f << 20 | (slot - cum) << 8 | byte
-//   x' = f * (x >> 12) + (slot - cum) = f * ((x >> 12) - 4096) + (e >> 8)
-// Every lane reads a word (the ring always holds valid memory) and keeps it
-// only if it renormalises (a select, not a branch).  Shifts and field
-// extractions are written as IMADs (mad.hi by a power of two) so that they
-// run on the FMA pipe next to the busier integer ALU pipe.
-__device__ __forceinline__ uint32_t rans_step(uint32_t lut, uint32_t &rp, uint32_t &x, uint32_t lt) {
-    const uint32_t addr = mad_hi(mad_lo(x, 1u << 20, 0u), 1u << 14, lut);  // lut + 4 * (x & 4095)
-    const uint32_t e = lds_u32(addr);
-    const uint32_t t = mad_hi(x, 1u << 20, 0u - kProbTotal);               // (x >> 12) - 4096
-    x = mad_lo(mad_hi(e, 1u << 12, 0u), t, mad_hi(e, 1u << 24, 0u));
-    const bool need = x < kStateLow;
-    const uint32_t b = __ballot_sync(kFull, need);
-    const uint32_t w = lds_u16(mad_lo(__popc(b & lt), 2u, rp));
-    const uint32_t xr = mad_lo(x, 1u << 16, w);
-    x = need ? xr : x;
-    rp = mad_lo(__popc(b), 2u, rp);
-    return e;
-}
-
-// Last, partial group: lane l is active at step r while 8l + r < rem.
-__device__ __forceinline__ void rans_tail(uint32_t lut, uint32_t ring, uint32_t &x, uint32_t &pw, uint32_t lt,
-                                          uint32_t lane, uint32_t rem, uint32_t (&e8)[8]) {
-#pragma unroll
-    for (uint32_t r = 0; r < 8; ++r) {
-        const bool active = lane * kGroup + r < rem;
-        bool need = false;
-        if (active) {
-            const uint32_t e = lds_u32(lut + 4 * (x & (kProbTotal - 1)));
-            x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xFFFu);
-            e8[r] = e;
-            need = x < kStateLow;
-        }
-        const uint32_t b = __ballot_sync(kFull, need);
-        const uint32_t w = lds_u16(ring + ((pw + 2u * __popc(b & lt)) & (kRingBytes - 1)));
-        if (need) x = (x << 16) | w;
-        pw += 2u * __popc(b);
-    }
-}
 
 // Per-chunk copy of the output-side fields of a matrix, kept in registers.
 struct OutCtx {
@@ -514,32 +198,6 @@ __device__ __forceinline__ void group_row(uint32_t lut, uint32_t ring, uint32_t 
     pw += rp - rp0;
 }
 
-// Rank mode: with 2..32 distinct symbols and a warp-uniform row per group, the
-// slot table's low byte holds the symbol's rank (index in the ascending
-// frequency list) and lane r keeps fp32_rn(value(symbol of rank r) * row
-// scale).  A decoded symbol's dequantised value is then one shuffle from the
-// lane named by its rank (shfl uses only the low 5 bits of the entry).
-template <uint32_t LAYOUT>
-__device__ __forceinline__ bool rank_mode(uint32_t n_present) {
-    return LAYOUT == kRowUniform && n_present >= 2 && n_present <= 32;
-}
-
-// The byte the shared table stores for list entry i (rank mode: the rank).
-template <uint32_t LAYOUT>
-__device__ __forceinline__ uint32_t table_low_byte(uint32_t n_present, uint32_t i, uint32_t sym) {
-    return rank_mode<LAYOUT>(n_present) ? i : sym;
-}
-
-// Exact fp32 value of a symbol byte (Int8 or E4M3).
-template <int DT>
-__device__ __forceinline__ float symbol_value(uint32_t sym) {
-    if constexpr (DT == EQ_INT8) {
-        return static_cast<float>(static_cast<int8_t>(sym & 0xFFu));
-    } else {
-        return __fmul_rn(__uint_as_float(((sym & 0x80u) << 24) | ((sym & 0x7Fu) << 20)), 0x1p120f);
-    }
-}
-
 // One 256-symbol group in rank mode: 8 steps, 8 shuffles, one 16-byte store.
 __device__ __forceinline__ void group_rank(uint32_t lut, uint32_t ring, uint32_t &pw, uint32_t &x, uint32_t lt,
                                            float vr, uint16_t *dst) {
@@ -555,13 +213,6 @@ __device__ __forceinline__ void group_rank(uint32_t lut, uint32_t ring, uint32_t
     st_global_v4(dst, make_uint4(o[0], o[1], o[2], o[3]));
     pw += rp - rp0;
 }
-
-// A chunk record's header fields and this lane's initial state.
-struct ChunkHead {
-    const uint8_t *rec;
-    uint32_t n, n_words, n_present, table_bytes;
-    uint32_t x;
-};
 
 // Two chunks per warp in lockstep (rank mode, row-uniform layout, both
 // chunks 65536 symbols, cols a multiple of 512): every step of chunk A is
@@ -598,27 +249,14 @@ __device__ __forceinline__ void group2_rank(uint32_t lut, uint32_t ringA, uint32
     B.dst += kGroupSyms;
 }
 
-// Returns false if a bounded wait gave up (the warp must stop).
-__device__ __forceinline__ bool pair_start(RingCtl *ctl, const ChunkHead &h) {
-    if ((threadIdx.x & 31u) == 0) {
-        const uint32_t pbytes = (2u * h.n_words + 15u) & ~15u;
-        ctl->payload = h.rec + h.table_bytes;
-        ctl->pbytes = pbytes;
-        ctl->n_segs = (pbytes + kSegBytes - 1) / kSegBytes;
-        ctl->issued = 0;
-        ctl->ready = 0;
-    }
-    return true;
-}
-
 template <int DT>
 __device__ __forceinline__ bool decode_pair(int32_t *status, const OutCtx &O, const ChunkHead &hA,
                                             const ChunkHead &hB, uint64_t firstA, uint64_t firstB, uint32_t lut,
                                             uint32_t ringA, uint32_t ringB, uint32_t mbarA, uint32_t mbarB,
                                             RingCtl *ctlA, RingCtl *ctlB, uint32_t lane, uint32_t lt,
                                             uint32_t lane_sym) {
-    pair_start(ctlA, hA);
-    pair_start(ctlB, hB);
+    ring_start(ctlA, hA);
+    ring_start(ctlB, hB);
     __syncwarp();
     const float vraw = symbol_value<DT>(lane_sym);
     Chain A, B;
@@ -845,197 +483,45 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, ui
     return true;
 }
 
-// Header of chunk k: checks it against the directory; on success fills the
-// record pointer, counts and this lane's initial state.
-
-__device__ __forceinline__ bool load_head(const DecodeParams &P, const MatJob &M, uint32_t k, uint32_t lane,
-                                          ChunkHead &h) {
-    const uint64_t first = (uint64_t)k * kChunkSyms;
-    const uint64_t rem = M.n_elems - first;
-    const uint32_t n_expect = rem < kChunkSyms ? (uint32_t)rem : kChunkSyms;
-    const uint64_t off = M.chunk_index[k];
-    const uint64_t end = M.chunk_index[k + 1];
-    if ((off & 15) || end > P.blob_len || end < off + kRecordHeadBytes + 16) {
-        flag(P.status, EQ_DEV_BAD_HEADER);
-        return false;
-    }
-    h.rec = P.blob + off;
-    const uint4 head = *reinterpret_cast<const uint4 *>(h.rec);
-    h.n = head.x;
-    h.n_words = head.y;
-    h.n_present = head.z;
-    h.table_bytes = (kRecordHeadBytes + 4 * h.n_present + 15) & ~15u;
-    if (h.n != n_expect || h.n_present < 1 || h.n_present > 256 ||
-        off + h.table_bytes + ((2ull * h.n_words + 15) & ~15ull) != end) {
-        flag(P.status, EQ_DEV_BAD_HEADER);
-        return false;
-    }
-    h.x = reinterpret_cast<const uint32_t *>(h.rec + 16)[lane];
-    if (!__all_sync(kFull, h.x >= kStateLow)) {
-        flag(P.status, EQ_DEV_BAD_STATE);
-        return false;
-    }
-    return true;
-}
-
-// Check a frequency list (n_present entries at `tab`): ascending symbols,
-// reserved bits zero, f >= 1, sum 4096.  Optionally copies the entries and
-// their cumulative frequencies to shared memory, and/or expands the list into
-// a warp's slot table.  Returns validity (warp-uniform).
-__device__ __forceinline__ bool warp_table(const uint32_t *tab, uint32_t n_present, uint32_t lane,
-                                           uint32_t *entries_out, uint32_t *cum_out, uint32_t *lut,
-                                           bool by_rank) {
-    uint32_t run = 0;
-    int prev_sym = -1;
-    bool ok = true;
-    for (uint32_t base = 0; base < n_present; base += 32) {
-        const uint32_t i = base + lane;
-        const bool have = i < n_present;
-        const uint32_t e = have ? tab[i] : 0u;
-        const uint32_t f = e >> 16, sym = e & 0xFFu;
-        bool good = !have || ((e & 0xFF00u) == 0 && f >= 1 && f <= kProbTotal);
-        const int left = __shfl_up_sync(kFull, (int)sym, 1);
-        if (have && (int)sym <= (lane == 0 ? prev_sym : left)) good = false;
-        uint32_t inc = f;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const uint32_t t = __shfl_up_sync(kFull, inc, d);
-            if (lane >= (uint32_t)d) inc += t;
-        }
-        const uint32_t cum = run + inc - f;
-        if (have) {
-            if (entries_out) entries_out[i] = e;
-            if (cum_out) cum_out[i] = cum;
-        }
-        ok = __all_sync(kFull, good) && ok;
-        const uint32_t cnt = min(32u, n_present - base);
-        if (lut && n_present > 1) {
-            for (uint32_t q = 0; q < cnt; ++q) {
-                const uint32_t fq = __shfl_sync(kFull, f, q);
-                const uint32_t cq = __shfl_sync(kFull, cum, q);
-                const uint32_t sq = __shfl_sync(kFull, sym, q);
-                for (uint32_t t = lane; t < fq; t += 32) {
-                    const uint32_t slot = cq + t;
-                    if (slot < kProbTotal && fq < kProbTotal)
-                        lut[slot] = (fq << 20) | (t << 8) | (by_rank ? base + q : sq);
-                }
-            }
-        }
-        prev_sym = __shfl_sync(kFull, (int)sym, cnt - 1);
-        run += __shfl_sync(kFull, inc, 31);
-    }
-    return ok && run == kProbTotal;
-}
-
-// Shared memory of one block: slot table(s), then per warp a 2.5 KB word ring
-// (with its mirror), the ring's mbarriers and bookkeeping, then the block's
-// reference frequency list (shared-table kernel only).
-template <int WARPS, bool SHARED>
-struct Smem {
-    static constexpr uint32_t kChains = SHARED ? EQ_CHAINS : 1;          // chunks decoded at once per warp
-    static constexpr uint32_t kLuts = SHARED ? 1 : WARPS;
-    static constexpr uint32_t kRingOff = kLuts * kLutBytes;             // + runtime pad to 128 B
-    static constexpr uint32_t kMbarOff = kRingOff + WARPS * kChains * kRingStride;  // offsets below include the pad
-    static constexpr uint32_t kCtlOff = kMbarOff + WARPS * kChains * kRingSegs * 8;
-    static constexpr uint32_t kRefOff = kCtlOff + WARPS * kChains * 32;  // 32 bytes of RingCtl per chain
-    static constexpr uint32_t kBlockOff = kRefOff + (SHARED ? 2 * 256 * 4 : 0);
-    static constexpr uint32_t kBytes = kBlockOff + 16 + 128;            // + worst-case alignment pad
-};
-static_assert(sizeof(RingCtl) <= 32, "RingCtl slot");
-
 template <int WARPS, bool SHARED, int DT, uint32_t LAYOUT>
 __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
     eq_decode_kernel(const __grid_constant__ DecodeParams P) {
-    using L = Smem<WARPS, SHARED>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = threadIdx.x >> 5;
-    const uint32_t base = smem_u32(smem_raw);
-    const uint32_t pad = (128u - ((base + L::kRingOff) & 127u)) & 127u;
-    unsigned char *padded = smem_raw + pad;  // offsets from kRingOff on are relative to this
-    constexpr uint32_t C = L::kChains;
-    const uint32_t ring = base + pad + L::kRingOff + warp * C * kRingStride;
-    const uint32_t mbar = base + pad + L::kMbarOff + warp * C * kRingSegs * 8;
-    RingCtl *ctl = reinterpret_cast<RingCtl *>(padded + L::kCtlOff + warp * C * 32);
-    uint32_t *lut = reinterpret_cast<uint32_t *>(smem_raw) + (SHARED ? 0u : warp * kProbTotal);
-    const uint32_t lut_addr = smem_u32(lut);
-    if (lane == 0) {
-        for (uint32_t i = 0; i < C * kRingSegs; ++i) mbar_init(mbar + 8 * i, 1);
-        fence_mbar_init();
-        for (uint32_t c = 0; c < C; ++c) {
-            ctl[c].phase = 0;
-            ctl[c].dead = 0;
-            ctl[c].issued = ctl[c].ready = 0;
-        }
-    }
-    __syncwarp();
+    const WarpSmem<WARPS, SHARED> S(smem_raw, warp, lane);
+    constexpr uint32_t C = WarpSmem<WARPS, SHARED>::C;
+    RingCtl *ctl = S.ctl;
     const uint32_t lt = lanemask_lt();
 
     if constexpr (SHARED) {
-        uint32_t *ref_entries = reinterpret_cast<uint32_t *>(padded + L::kRefOff);
-        uint32_t *ref_cum = ref_entries + 256;
-        volatile uint32_t *blk = reinterpret_cast<uint32_t *>(padded + L::kBlockOff);  // [0] n_present, [1] valid
         uint32_t cur_mat = kNoLimit;
         for (uint32_t unit = blockIdx.x; unit < P.total_units; unit += gridDim.x) {
-            uint32_t mi = 0;
-            while (mi + 1 < P.n_mats && unit >= P.mats[mi + 1].begin) ++mi;
+            const uint32_t mi = job_of(P, unit);
             const MatJob &M = P.mats[mi];
             const uint32_t k0 = (unit - M.begin) * WARPS * C;
             if (mi != cur_mat) {
-                // rebuild the block's slot table from the tile's first chunk
-                __syncthreads();
-                if (warp == 0) {
-                    ChunkHead h;
-                    bool ok = load_head(P, M, k0, lane, h);
-                    if (ok) ok = warp_table(reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes), h.n_present,
-                                            lane, ref_entries, ref_cum, nullptr, false);
-                    if (lane == 0) {
-                        blk[0] = ok ? h.n_present : 0u;
-                        blk[1] = ok;
-                    }
-                }
-                __syncthreads();
-                const uint32_t np = blk[0];
-                if (blk[1] && np > 1) {
-                    for (uint32_t i = 0; i < np; ++i) {
-                        const uint32_t e = ref_entries[i], c = ref_cum[i];
-                        const uint32_t f = e >> 16, sy = e & 0xFFu;
-                        const uint32_t low = table_low_byte<LAYOUT>(np, i, sy);
-                        for (uint32_t t = threadIdx.x; t < f; t += WARPS * 32)
-                            if (c + t < kProbTotal && f < kProbTotal) lut[c + t] = (f << 20) | (t << 8) | low;
-                    }
-                }
-                __syncthreads();
+                shared_table_rebuild<WARPS, LAYOUT>(P, M, k0, lane, warp, S);
                 cur_mat = mi;
             }
-            const uint32_t np = blk[0];
-            const uint32_t lane_sym = ref_entries[lane < np ? lane : 0] & 0xFFu;
+            const uint32_t np = S.blk[0];
+            const uint32_t lane_sym = S.ref_entries[lane < np ? lane : 0] & 0xFFu;
             // this warp's chunks: k0 + warp (+ WARPS for the second chain)
             ChunkHead hc[C];
             bool have[C];
             for (uint32_t c = 0; c < C; ++c) {
                 const uint32_t k = k0 + warp + c * WARPS;
                 have[c] = k < M.n_chunks && !ctl[0].dead && !ctl[C - 1].dead;
-                if (have[c]) have[c] = load_head(P, M, k, lane, hc[c]);
-                if (have[c]) {
-                    bool same = blk[1] && hc[c].n_present == np;
-                    if (same) {
-                        const uint32_t *tab = reinterpret_cast<const uint32_t *>(hc[c].rec + kRecordHeadBytes);
-                        for (uint32_t i = lane; i < np; i += 32) same = same && tab[i] == ref_entries[i];
-                    }
-                    if (!__all_sync(kFull, same)) {
-                        flag(P.status, EQ_DEV_BAD_TABLE);
-                        have[c] = false;
-                    }
-                }
+                if (have[c]) have[c] = shared_chunk_head(P, M, k, lane, np, S, hc[c]);
             }
             const OutCtx O = out_ctx(M);
             if constexpr (C == 2 && LAYOUT == kRowUniform) {
                 if (have[0] && have[1] && rank_mode<LAYOUT>(np) && hc[0].n == kChunkSyms &&
                     hc[1].n == kChunkSyms && O.cols % (2 * kGroupSyms) == 0) {
                     decode_pair<DT>(P.status, O, hc[0], hc[1], (uint64_t)(k0 + warp) * kChunkSyms,
-                                    (uint64_t)(k0 + warp + WARPS) * kChunkSyms, lut_addr, ring, ring + kRingStride,
-                                    mbar, mbar + 8 * kRingSegs, ctl, ctl + 1, lane, lt, lane_sym);
+                                    (uint64_t)(k0 + warp + WARPS) * kChunkSyms, S.lut_addr, S.ring,
+                                    S.ring + kRingStride, S.mbar, S.mbar + 8 * kRingSegs, ctl, ctl + 1, lane, lt,
+                                    lane_sym);
                     __syncwarp();
                     continue;
                 }
@@ -1044,24 +530,22 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
                 if (!have[c] || ctl->dead) continue;
                 decode_body<DT, LAYOUT>(P.status, O, (uint64_t)(k0 + warp + c * WARPS) * kChunkSyms, hc[c].n,
                                         hc[c].n_words, hc[c].rec + hc[c].table_bytes, np == 1,
-                                        ref_entries[0] & 0xFFu, hc[c].x, lut_addr, ring, mbar, ctl, lane, lt,
-                                        rank_mode<LAYOUT>(np), lane_sym);
+                                        S.ref_entries[0] & 0xFFu, hc[c].x, S.lut_addr, S.ring, S.mbar, ctl, lane,
+                                        lt, rank_mode<LAYOUT>(np), lane_sym);
                 __syncwarp();
             }
         }
     } else {
         const uint32_t stride = gridDim.x * WARPS;
         for (uint32_t c = blockIdx.x * WARPS + warp; c < P.total_units && !ctl->dead; c += stride) {
-            uint32_t mi = 0;
-            while (mi + 1 < P.n_mats && c >= P.mats[mi + 1].begin) ++mi;
-            const MatJob &M = P.mats[mi];
+            const MatJob &M = P.mats[job_of(P, c)];
             const uint32_t k = c - M.begin;
             ChunkHead h;
             if (!load_head(P, M, k, lane, h)) continue;
             const uint32_t *tab = reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes);
             __syncwarp();  // the previous chunk's reads of the slot table are done
             const bool by_rank = rank_mode<LAYOUT>(h.n_present);
-            const bool ok = warp_table(tab, h.n_present, lane, nullptr, nullptr, lut, by_rank);
+            const bool ok = warp_table(tab, h.n_present, lane, nullptr, nullptr, S.lut, by_rank);
             if (!ok) {
                 flag(P.status, EQ_DEV_BAD_TABLE);
                 continue;
@@ -1069,7 +553,7 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
             __syncwarp();
             decode_body<DT, LAYOUT>(P.status, out_ctx(M), (uint64_t)k * kChunkSyms, h.n, h.n_words,
                                     h.rec + h.table_bytes, h.n_present == 1, tab[0] & 0xFFu, h.x,
-                                    lut_addr, ring, mbar, ctl, lane, lt, by_rank,
+                                    S.lut_addr, S.ring, S.mbar, ctl, lane, lt, by_rank,
                                     tab[lane < h.n_present ? lane : 0] & 0xFFu);
             __syncwarp();
         }
@@ -1089,43 +573,43 @@ __global__ void eq_outlier_scatter_kernel(const __grid_constant__ ScatterParams 
         atomicOr(P.status, EQ_DEV_BAD_OUTLIER);
         return;
     }
-    J.out[(uint64_t)row * J.cols + col] = to_bf16(v);
+    uint16_t *o = J.out + (uint64_t)row * J.cols + col;
+    // the stream carries a zero-valued placeholder symbol under every super weight
+    if (*o & 0x7FFFu) atomicOr(P.status, EQ_DEV_BAD_OUTLIER);
+    *o = to_bf16(v);
+}
+
+// Timeout path check: a ring whose only segment counts as issued but was never
+// copied, so ring_drain's bounded wait on its mbarrier must give up.
+__global__ void eq_wait_timeout_kernel(int32_t *status) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ RingCtl ctl;
+    const uint32_t mbar = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(mbar, 1);
+        fence_mbar_init();
+        ctl.payload = nullptr;
+        ctl.pbytes = kSegBytes;
+        ctl.n_segs = 1;
+        ctl.issued = 1;
+        ctl.ready = 0;
+        ctl.phase = 0;
+        ctl.dead = 0;
+    }
+    __syncwarp();
+    if (!ring_drain(&ctl, mbar)) flag(status, EQ_DEV_TIMEOUT);
 }
 
 // ---- host side ---------------------------------------------------------------------
-
-using KernelFn = void (*)(DecodeParams);
-
-struct KernelSetup {
-    KernelFn fn = nullptr;
-    int warps = 0;
-    size_t smem = 0;
-    int ctas_per_sm = 0;
-    uint32_t units_per_cta = 0;  // work units (tiles or chunks) a block takes per round
-};
 
 // variants: [shared][dtype - 1][layout]
 struct DeviceSetup {
     bool ready = false;
     int sms = 0;
-    KernelSetup k[2][2][3];
+    KernelSetup<DecodeParams> k[2][2][3];
 };
 std::mutex g_setup_mu;
 DeviceSetup g_setup[128];
-
-int setup_kernel(KernelSetup &k, KernelFn fn, int warps, size_t smem, uint32_t units_per_cta) {
-    k.fn = fn;
-    k.warps = warps;
-    k.smem = smem;
-    k.units_per_cta = units_per_cta;
-    if (cudaFuncSetAttribute(reinterpret_cast<const void *>(fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-        return EQ_ERR_CUDA;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&k.ctas_per_sm, fn, warps * 32, smem) != cudaSuccess ||
-        k.ctas_per_sm < 1)
-        return EQ_ERR_CUDA;
-    return EQ_OK;
-}
 
 template <int DT, uint32_t LAYOUT>
 int setup_pair(DeviceSetup &d) {
@@ -1159,15 +643,6 @@ uint32_t layout_of(const eq_matrix_info &in, const uint16_t *out) {
     if (aligned && in.cols % kGroupSyms == 0) return kRowUniform;
     if (aligned && in.cols % kGroup == 0) return kLaneRows;
     return kGeneric;
-}
-
-int launch(const KernelSetup &k, int sms, const DecodeParams &P, cudaStream_t s) {
-    if (!P.total_units) return EQ_OK;
-    const uint32_t resident = (uint32_t)(sms * k.ctas_per_sm);
-    const uint32_t want = (P.total_units + k.units_per_cta - 1) / k.units_per_cta;
-    const uint32_t grid = std::min(want, resident);
-    k.fn<<<grid, k.warps * 32, k.smem, s>>>(P);
-    return cudaGetLastError() == cudaSuccess ? EQ_OK : EQ_ERR_CUDA;
 }
 
 // Decode matrices [first, first + count) of the model into outs[i]: one
@@ -1275,4 +750,10 @@ extern "C" EQW_API int eq_decode_model_stream(const eq_model *m, uint32_t layer,
     if (rc) return rc;
     if (cudaEventRecord(ev_ready[b], decode_stream) != cudaSuccess) return EQ_ERR_CUDA;
     return EQ_OK;
+}
+
+extern "C" EQW_API int eq_selftest_wait_timeout(int32_t *d_status, cudaStream_t s) {
+    if (!d_status) return EQ_ERR_INVALID_ARG;
+    eq_wait_timeout_kernel<<<1, 32, 0, s>>>(d_status);
+    return cudaGetLastError() == cudaSuccess ? EQ_OK : EQ_ERR_CUDA;
 }

@@ -16,8 +16,20 @@
  * Coding used here: rANS, 12-bit frequencies (M = 4096), 32-bit states in
  * [2^16, 2^32), 16-bit renormalisation words, 32 interleaved states per chunk
  * of up to 65536 symbols, per-chunk frequency tables, fp32 per-row scales,
- * fp32 COO outliers.  The byte layout ("container v1", magic "EQW1") is
- * specified in DESIGN.md of this repository, section "Container format v1".
+ * fp32 COO outliers.  Byte layout ("container v1", little-endian, sections
+ * 256-byte aligned):
+ *   header (64 B): "EQW1", version 1, format constants, counts, total length;
+ *   directory (64 B per matrix): layer, index, dtype, rows, cols, chunk
+ *     count, outlier count, offsets of the chunk index, scales, outliers;
+ *   per matrix: chunk index u64[n_chunks + 1] (record offsets, the last one
+ *     the end), scales f32[rows], outliers {u32 row, u32 col, f32 value}
+ *     sorted by linear index (the symbol stream holds symbol 0 under each);
+ *   chunk records (16-byte aligned): u32 n_syms, n_words, n_present, 0;
+ *     u32 states[32]; u32 table[n_present] = symbol | f << 16 in ascending
+ *     symbol order; padding to 16 B; u16 words[n_words]; padding to 16 B.
+ *   Symbol j of a chunk belongs to lane (j mod 256) div 8 at step
+ *   8 (j div 256) + j mod 8; words are consumed step by step, lanes in
+ *   ascending order within a step.
  *
  * Conventions for every function below:
  *   - Return value: EQ_OK (0) or one of the EQ_ERR_* codes; nothing throws.
@@ -69,7 +81,7 @@ enum {
     EQ_DEV_BAD_STATE = 4,    /* an initial state outside [2^16, 2^32) */
     EQ_DEV_BAD_END = 8,      /* final states != 2^16 or words consumed != n_words */
     EQ_DEV_TIMEOUT = 16,     /* a bounded wait for a staged copy gave up */
-    EQ_DEV_BAD_OUTLIER = 32  /* outlier position outside its matrix */
+    EQ_DEV_BAD_OUTLIER = 32  /* outlier position outside its matrix, or a non-zero stream value under it */
 };
 
 /* symbol formats */
@@ -209,6 +221,50 @@ EQW_API int eq_decode_model_stream(const eq_model *m, uint32_t layer, void *cons
  */
 EQW_API int eq_gemv_bf16(const void *d_w, const void *d_x, float *d_y, uint32_t rows, uint32_t cols,
                          cudaStream_t s);
+
+/* ---- fused decode + batch-1 GEMV --------------------------------------------------
+ * y = W x for an entropy-coded matrix W without materialising W: each chunk
+ * is decoded in registers (same decoder as eq_decode_block) and multiplied by
+ * x as it is decoded (EntQuant section 2 "inference-time decoding"; fused
+ * decode kernels are the next step its section 4 names).
+ *   W[r, c] = bf16(fp32(value(sym) * scale[r])) with both roundings to nearest
+ *             even, and bf16(v) at the super weights -- exactly the matrix
+ *             eq_decode_block writes;
+ *   y[r]    = sum_c W[r, c] * x[c], products exact in fp32, sums in fp32 in
+ *             an order fixed by the chunk and lane layout (per lane, then a
+ *             warp butterfly, then at most two chunk partials per row when
+ *             cols <= 65536, so the result is deterministic).  Error bound:
+ *             |y - exact| <= gamma_h * sum_c |W[r, c] x[c]| with
+ *             h = cols / 64 + 8 + (super weights in the row), gamma_h =
+ *             h u / (1 - h u), u = 2^-24.
+ * The stream must hold a zero-valued symbol at every super-weight position
+ * (both encoders write symbol 0 there; eq_decode_* check it, see
+ * EQ_DEV_BAD_OUTLIER).
+ * Arguments: x (device, bf16 [cols], 16-byte aligned), y (device, fp32 [rows],
+ * overwritten: zeroed on `s` first, then accumulated by the kernel), d_status
+ * as for the decoders.  Every matrix with rows * cols > 0 needs
+ * cols % 256 == 0 (EQ_ERR_UNSUPPORTED otherwise).  Enqueued on `s`.
+ */
+EQW_API int eq_decode_gemv_matrix(const eq_model *m, uint32_t matrix, const void *d_x, float *d_y,
+                                  int32_t *d_status, cudaStream_t s);
+
+/*
+ * The same for every matrix of `layer`: d_x[i], d_y[i] (host arrays of
+ * `count` device pointers, count = the layer's matrix count) belong to
+ * matrix i of the layer in directory order.  One launch per kernel variant.
+ */
+EQW_API int eq_decode_gemv_block(const eq_model *m, uint32_t layer, const void *const *d_x, float *const *d_y,
+                                 uint32_t count, int32_t *d_status, cudaStream_t s);
+
+/* ---- failure detection ----------------------------------------------------------
+ * Check of the decode kernels' timeout path: one warp runs the decoder's own
+ * staging-ring drain on a ring slot marked as issued whose copy was never
+ * started (its mbarrier is never completed), so the bounded wait gives up
+ * after its limit (~2e9 SM cycles, about one second) and the warp ORs
+ * EQ_DEV_TIMEOUT into *d_status and returns; nothing faults or hangs and
+ * the context stays usable.  Enqueued on `s`; d_status as for the decoders.
+ */
+EQW_API int eq_selftest_wait_timeout(int32_t *d_status, cudaStream_t s);
 
 /* ---- misc ----------------------------------------------------------------------- */
 EQW_API const char *eq_status_string(int status);

@@ -16,8 +16,9 @@ Two ways to obtain the decoded bf16 weights of a matrix:
   decode of a container, followed by the same dequantiser and scatter.
 
 The scalar coder lives in ``rans_oracle.c`` (plain C, built by :func:`build`);
-this module holds the container format (written from its definition in
-DESIGN.md, "Container format v1") and thin ctypes wrappers.
+this module holds the container format v1 (magic "EQW1": header, matrix
+directory, chunk index, scales, outliers, 16-byte aligned chunk records) and
+thin ctypes wrappers.
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py``
 (round trip, brute force over tiny alphabets, the rANS ideal-code-length
@@ -270,6 +271,28 @@ def dequant_direct(m, threads: int | None = None) -> np.ndarray:
     out = dequant(m.dtype, m.symbols, m.scales, threads)
     scatter(out, m.out_row, m.out_col, m.out_val)
     return out
+
+
+def bf16_to_f64(bits) -> np.ndarray:
+    """bf16 bit patterns -> their exact values as float64 (bf16 is the top half of an fp32)."""
+    b = np.ascontiguousarray(bits, np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def gemv_exact(w_bits: np.ndarray, x_bits: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Batch-1 forward of a decoded matrix: y[r] = sum_c W[r, c] * x[c], and sum_c |W[r, c] * x[c]|.
+
+    EntQuant technical summary, section 2 "inference-time decoding": the
+    decoded block's weights feed its forward pass, which at batch 1 is a
+    matrix-vector product per linear layer.  W (bf16 bits, [rows, cols]) and
+    x (bf16 bits, [cols]) are widened exactly to float64; every product of two
+    bf16 values is exact there (at most 16 significant bits), and the float64
+    sums are within cols * 2^-53 of exact relative to the second result,
+    far below any fp32 bound a test applies.
+    """
+    w = bf16_to_f64(w_bits).reshape(np.shape(w_bits))
+    x = bf16_to_f64(x_bits).reshape(-1)
+    return w @ x, np.abs(w) @ np.abs(x)
 
 
 # ---------------------------------------------------------------------------
