@@ -41,6 +41,30 @@ if ROOT not in sys.path:
 
 METRIC = "decoded bf16 weight GB/s per B200 (and Gsym/s); % of HBM roofline"
 UNIT = "GB/s"
+
+# DRAM bytes (read + write) of one eq_decode_kernel launch on a 70B-shape
+# block, from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of
+# the same launch configuration, and the SHA-256 of the decode sources it was
+# taken on: the figure is reported only while the sources are unchanged.
+DECODE_TRAFFIC_BYTES = 1_897_507_936
+DECODE_TRAFFIC_SOURCES_SHA256 = "dd6fd885e04a84efc15272c5534d75a880bd670005d7c9fb030788120f21c1db"
+DECODE_SOURCES = ("entropy_coded_weight_b200/csrc/eqw_decode.cu", "entropy_coded_weight_b200/csrc/eqw_device.cuh")
+
+
+def decode_sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    root = os.path.dirname(os.path.abspath(__file__))
+    for rel in DECODE_SOURCES:
+        with open(os.path.join(root, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def decode_traffic() -> int | None:
+    if DECODE_TRAFFIC_BYTES is None or decode_sources_sha256() != DECODE_TRAFFIC_SOURCES_SHA256:
+        return None
+    return DECODE_TRAFFIC_BYTES
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -438,7 +462,7 @@ def bench_eqw(args, d: Dist) -> dict | None:
                    "parallelism": f"replicas x{d.world}"},
         "gsym_s": round(gsym, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": decode_traffic(),
                      "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "eq_decode_kernel",
                      "alg_bytes_per_launch": int(alg_per_launch), "launch_ms": round(launch_ms, 4)},
         "with_gemv_consumer": {"value": round(value_b, 2), "unit": UNIT, "ms_per_step": round(ms_b_max / args.steps, 3),

@@ -4,7 +4,8 @@
 // EntQuant technical summary (gist.science 2601.22787), section 2
 // "inference-time decoding": a block's weights are expanded into a buffer just
 // before its forward kernels read them, and at batch 1 a linear layer's
-// forward is y = W x; section 4 names fused decode kernels as the next speed-up.
+// forward is y = W x; section 5 expects large speed-ups from dedicated fused
+// kernels.
 // Here the buffer disappears: each warp decodes its chunk exactly as
 // eq_decode_kernel does (staging ring, interleaved rANS step, shared slot
 // table, rank-mode dequant) and, after every 8 steps, multiplies the 8 weights
@@ -32,12 +33,25 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <mutex>
 #include <vector>
 
 #include "eqw_device.cuh"
 
 namespace {
+
+#ifndef EQ_GEMV_WARPS
+#define EQ_GEMV_WARPS EQ_SHARED_WARPS
+#endif
+#ifndef EQ_GEMV_MIN_CTAS
+#define EQ_GEMV_MIN_CTAS 1
+#endif
+#ifndef EQ_GEMV_FMA2
+#define EQ_GEMV_FMA2 1
+#endif
+constexpr int kGemvWarps = EQ_GEMV_WARPS;       // warps per block, shared-table kernel
+constexpr int kGemvMinCtas = EQ_GEMV_MIN_CTAS;  // register budget: blocks of kGemvWarps per SM
 
 struct GemvJob {
     const uint64_t *chunk_index;  // absolute record offsets, n_chunks + 1 entries
@@ -68,6 +82,21 @@ __device__ __forceinline__ float bf16_round(float v) { return __bfloat162float(_
 // The two bf16 of a 32-bit word as fp32 (exact).
 __device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+// a0 += w0 * x0, a1 += w1 * x1, each a fused multiply-add rounded to nearest even.
+__device__ __forceinline__ void fma_pair(float &a0, float &a1, float w0, float w1, float x0, float x1) {
+#if EQ_GEMV_FMA2
+    unsigned long long A, Wp, X;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a0), "f"(a1));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(Wp) : "f"(w0), "f"(w1));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(X) : "f"(x0), "f"(x1));
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(A) : "l"(Wp), "l"(X));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(A));
+#else
+    a0 = fmaf(w0, x0, a0);
+    a1 = fmaf(w1, x1, a1);
+#endif
+}
 
 __device__ __forceinline__ uint32_t vec_word(const uint4 &v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
@@ -131,8 +160,7 @@ __device__ __forceinline__ void group_dot(uint32_t lut, uint32_t ring, uint32_t 
             w1 = bf16_round(dequant1<DT>(e1, w));
         }
         const uint32_t u = vec_word(xv, r / 2);
-        a0 = fmaf(w0, bf_lo(u), a0);
-        a1 = fmaf(w1, bf_hi(u), a1);
+        fma_pair(a0, a1, w0, w1, bf_lo(u), bf_hi(u));
     }
     pw += rp - rp0;
 }
@@ -257,10 +285,8 @@ __device__ __forceinline__ void group2_dot(uint32_t lut, uint32_t ringA, uint32_
         const uint32_t ea1 = rans_step(lut, ra, A.x, lt);
         const uint32_t eb1 = rans_step(lut, rb, B.x, lt);
         const uint32_t ua = vec_word(xa, r / 2), ub = vec_word(xb, r / 2);
-        A.a0 = fmaf(__shfl_sync(kFull, A.w, ea0), bf_lo(ua), A.a0);
-        A.a1 = fmaf(__shfl_sync(kFull, A.w, ea1), bf_hi(ua), A.a1);
-        B.a0 = fmaf(__shfl_sync(kFull, B.w, eb0), bf_lo(ub), B.a0);
-        B.a1 = fmaf(__shfl_sync(kFull, B.w, eb1), bf_hi(ub), B.a1);
+        fma_pair(A.a0, A.a1, __shfl_sync(kFull, A.w, ea0), __shfl_sync(kFull, A.w, ea1), bf_lo(ua), bf_hi(ua));
+        fma_pair(B.a0, B.a1, __shfl_sync(kFull, B.w, eb0), __shfl_sync(kFull, B.w, eb1), bf_lo(ub), bf_hi(ub));
     }
     A.pw += ra - a0;
     B.pw += rb - b0;
@@ -342,7 +368,7 @@ __device__ __forceinline__ bool gemv_pair(int32_t *status, const GemvJob &M, con
 // SHARED = one slot table per block over tiles of WARPS x chains chunks,
 // otherwise one table per warp and chunk.
 template <int WARPS, bool SHARED, int DT>
-__global__ void __launch_bounds__(WARPS * 32, 1) eq_decode_gemv_kernel(const __grid_constant__ GemvParams P) {
+__global__ void __launch_bounds__(WARPS * 32, SHARED ? kGemvMinCtas : 1) eq_decode_gemv_kernel(const __grid_constant__ GemvParams P) {
     constexpr uint32_t LAYOUT = kRowUniform;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t lane = threadIdx.x & 31u;
@@ -412,6 +438,19 @@ __global__ void __launch_bounds__(WARPS * 32, 1) eq_decode_gemv_kernel(const __g
     }
 }
 
+// y_i = 0 for every matrix of a launch (the fused kernel only adds).
+struct ZeroParams {
+    float *y[kMaxMatsPerLaunch];
+    uint32_t rows[kMaxMatsPerLaunch];
+    uint32_t n;
+};
+
+__global__ void eq_zero_rows_kernel(const __grid_constant__ ZeroParams Z) {
+    for (uint32_t j = 0; j < Z.n; ++j)
+        for (uint32_t r = blockIdx.x * blockDim.x + threadIdx.x; r < Z.rows[j]; r += gridDim.x * blockDim.x)
+            Z.y[j][r] = 0.f;
+}
+
 // ---- host side ---------------------------------------------------------------------
 
 // variants: [shared][dtype - 1]
@@ -425,8 +464,8 @@ GemvSetup g_gemv_setup[128];
 
 template <int DT>
 int setup_dtype(GemvSetup &d) {
-    int rc = setup_kernel(d.k[1][DT - 1], eq_decode_gemv_kernel<kSharedWarps, true, DT>, kSharedWarps,
-                          Smem<kSharedWarps, true>::kBytes, 1);
+    int rc = setup_kernel(d.k[1][DT - 1], eq_decode_gemv_kernel<kGemvWarps, true, DT>, kGemvWarps,
+                          Smem<kGemvWarps, true>::kBytes, 1);
     if (rc) return rc;
     return setup_kernel(d.k[0][DT - 1], eq_decode_gemv_kernel<kPrivateWarps, false, DT>, kPrivateWarps,
                         Smem<kPrivateWarps, false>::kBytes, kPrivateWarps);
@@ -462,20 +501,30 @@ int check_gemv_args(const eq_model *m, uint32_t first, uint32_t count, const voi
     return EQ_OK;
 }
 
-// y_i = W_i x_i for matrices [first, first + count): zero every y, then one
-// launch per kernel variant (table scope x dtype) present.
+// y_i = W_i x_i for matrices [first, first + count): per group of up to 16
+// matrices one launch zeroing their y, then one launch per kernel variant
+// (table scope x dtype) present.
 int launch_gemv(const eq_model *m, uint32_t first, uint32_t count, const void *const *xs, float *const *ys,
                 int32_t *d_status, cudaStream_t s) {
     int rc = check_gemv_args(m, first, count, xs, ys);
     if (rc) return rc;
     GemvSetup *dev = nullptr;
     if ((rc = gemv_setup(&dev))) return rc;
-    for (uint32_t i = 0; i < count; ++i) {
-        const eq_matrix_info &in = m->mats[first + i].info;
-        if (in.rows && cudaMemsetAsync(ys[i], 0, sizeof(float) * in.rows, s) != cudaSuccess) return EQ_ERR_CUDA;
-    }
     for (uint32_t base = 0; base < count; base += kMaxMatsPerLaunch) {
         const uint32_t cnt = std::min<uint32_t>(kMaxMatsPerLaunch, count - base);
+        ZeroParams Z{};
+        uint32_t max_rows = 0;
+        for (uint32_t i = 0; i < cnt; ++i) {
+            const uint32_t rows = m->mats[first + base + i].info.rows;
+            if (!rows) continue;
+            Z.y[Z.n] = ys[base + i];
+            Z.rows[Z.n++] = rows;
+            max_rows = std::max(max_rows, rows);
+        }
+        if (Z.n) {
+            eq_zero_rows_kernel<<<std::min<uint32_t>((max_rows + 255) / 256, 4u * dev->sms), 256, 0, s>>>(Z);
+            if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
+        }
         GemvParams P[2][2];
         for (auto &a : P)
             for (auto &c : a) {
@@ -501,7 +550,7 @@ int launch_gemv(const eq_model *m, uint32_t first, uint32_t count, const void *c
             J.n_chunks = d.info.n_chunks;
             J.begin = Pv.total_units;
             J.n_out = d.info.n_outliers;
-            const uint32_t per_tile = kSharedWarps * EQ_CHAINS;
+            const uint32_t per_tile = kGemvWarps * EQ_CHAINS;
             Pv.total_units += sh ? (d.info.n_chunks + per_tile - 1) / per_tile : d.info.n_chunks;
         }
         for (int sh = 0; sh < 2; ++sh)

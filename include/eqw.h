@@ -225,8 +225,8 @@ EQW_API int eq_gemv_bf16(const void *d_w, const void *d_x, float *d_y, uint32_t 
 /* ---- fused decode + batch-1 GEMV --------------------------------------------------
  * y = W x for an entropy-coded matrix W without materialising W: each chunk
  * is decoded in registers (same decoder as eq_decode_block) and multiplied by
- * x as it is decoded (EntQuant section 2 "inference-time decoding"; fused
- * decode kernels are the next step its section 4 names).
+ * x as it is decoded (EntQuant section 2 "inference-time decoding"; its
+ * section 5 expects large speed-ups from dedicated fused kernels).
  *   W[r, c] = bf16(fp32(value(sym) * scale[r])) with both roundings to nearest
  *             even, and bf16(v) at the super weights -- exactly the matrix
  *             eq_decode_block writes;
