@@ -11,9 +11,12 @@ far larger than L2, so nothing is served from cache across layers.
 
 One "step" = one pass over all 80 blocks (decode + dequant + ping-pong
 events, no-op consumer).  The line also reports the same loop with the
-batch-1 bf16 GEMV consumer overlapped, the dominant kernel's roofline, the
-CPU oracle on the host cores, and an end-to-end number through the public
-API with the compressed weights copied from pinned host memory every step.
+batch-1 bf16 GEMV consumer overlapped, the fused decode + GEMV kernel over
+the same blocks, the dominant kernel's roofline, the CPU oracle on the host
+cores, an end-to-end number through the public API with the compressed
+weights copied from pinned host memory every step, and the GPU encoder's
+throughput (it builds the resident model; one layer is cross-checked against
+the host encoder byte for byte).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {eqw,reference}]
 
@@ -65,6 +68,8 @@ def decode_traffic() -> int | None:
     if DECODE_TRAFFIC_BYTES is None or decode_sources_sha256() != DECODE_TRAFFIC_SOURCES_SHA256:
         return None
     return DECODE_TRAFFIC_BYTES
+
+
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -203,8 +208,23 @@ def measured_hbm_peak() -> tuple[float, str]:
 N_LAYERS = 80
 
 
-def build_blob(distinct: int, threads: int) -> tuple[np.ndarray, int, float]:
-    """Generate `distinct` seeded 70B-shape Int8 layers and encode them (host)."""
+class DeviceMatrix:
+    """A matrix whose symbols and scales live on the GPU (input of eq_encode_device)."""
+
+    def __init__(self, m, device):
+        import torch
+        self.layer, self.dtype = m.layer, m.dtype
+        self.symbols = torch.from_numpy(np.ascontiguousarray(m.symbols)).to(device)
+        self.scales = torch.from_numpy(np.ascontiguousarray(m.scales)).to(device)
+        self.out_row = self.out_col = self.out_val = None
+
+
+def build_blob(distinct: int, threads: int, device) -> tuple[np.ndarray, dict]:
+    """Generate `distinct` seeded 70B-shape Int8 layers (host) and encode them on
+    the GPU with eq_encode_device; layer 0 is also encoded on the host, timed,
+    and must give the same bytes."""
+    import torch
+
     import entropy_coded_weight_b200 as E
     import workloads as W
     t0 = time.time()
@@ -212,12 +232,33 @@ def build_blob(distinct: int, threads: int) -> tuple[np.ndarray, int, float]:
     for layer in range(distinct):
         mats += W.llama70b_int8_layer(layer, 2.1, threads=threads)
     t1 = time.time()
-    blob = E.encode_host(mats, n_threads=threads)
+    dmats = [DeviceMatrix(m, device) for m in mats]
+    torch.cuda.synchronize(device)
+    t2 = time.time()
+    d_blob = E.encode_device(dmats)
+    t3 = time.time()
+    blob = d_blob.cpu().numpy()
+    del d_blob, dmats
     n_syms = sum(m.n for m in mats)
-    del mats
-    print(f"[bench] generated {distinct} layers in {t1 - t0:.1f}s, encoded in {time.time() - t1:.1f}s "
-          f"({8.0 * blob.size / n_syms:.3f} bits/sym incl. metadata)", file=sys.stderr, flush=True)
-    return blob, n_syms, time.time() - t0
+    layer0 = [m for m in mats if m.layer == 0]
+    t4 = time.time()
+    host0 = E.encode_host(layer0, n_threads=threads)
+    t5 = time.time()
+    same = bool(np.array_equal(host0, E.encode_device([DeviceMatrix(m, device) for m in layer0]).cpu().numpy()))
+    n0 = sum(m.n for m in layer0)
+    del mats, layer0
+    torch.cuda.empty_cache()
+    print(f"[bench] generated {distinct} layers in {t1 - t0:.1f}s, device-encoded in {t3 - t2:.1f}s "
+          f"({8.0 * blob.size / n_syms:.3f} bits/sym incl. metadata); host encode of one layer {t5 - t4:.1f}s",
+          file=sys.stderr, flush=True)
+    enc = {"device_gsym_s": round(n_syms / (t3 - t2) / 1e9, 3), "device_s": round(t3 - t2, 2),
+           "symbols": n_syms, "host_gsym_s": round(n0 / (t5 - t4) / 1e9, 3), "host_threads": threads,
+           "bytes_equal_host": same,
+           "note": "eq_encode_device on symbols already in HBM (wall clock, it synchronises); host = eq_encode_host "
+                   "of layer 0 on all cores"}
+    if not same:
+        raise RuntimeError("device and host encoders disagree")
+    return blob, enc
 
 
 class ResidentStack:
@@ -346,9 +387,9 @@ def bench_eqw(args, d: Dist) -> dict | None:
 
     dev = torch.device("cuda", torch.cuda.current_device())
     threads = len(os.sched_getaffinity(0))
-    blob = None
+    blob, enc = None, None
     if d.rank == 0:
-        blob, _, _ = build_blob(args.distinct_layers, threads)
+        blob, enc = build_blob(args.distinct_layers, threads, dev)
     blob = d.broadcast_bytes(blob)
     stack = ResidentStack(blob, args.distinct_layers, dev, args.layers)
     streamer = PingPongStreamer(stack.steps, dev)
@@ -479,6 +520,7 @@ def bench_eqw(args, d: Dist) -> dict | None:
         "e2e": {"value": round(value_e, 2), "unit": UNIT, "h2d_bytes_per_step": int(blob.size * stack.copies),
                 "d2h_bytes_per_step": 4, "ms_per_step": round(ms_e_max / args.steps, 3)},
         "cpu_baseline": cpu,
+        "encode": enc,
         "clocks": clk,
         "gpu_launches": launches,
     }

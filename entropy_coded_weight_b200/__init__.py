@@ -106,6 +106,60 @@ def encode_host(matrices, n_threads: int = 0, table_scope: str = "matrix") -> np
     return out
 
 
+def _device_matrix_in_array(matrices, table_scope: str):
+    """eq_matrix_in[] whose pointers are device addresses (CUDA tensors on one device)."""
+    import torch
+    keep = []
+    arr = (eq_matrix_in * max(1, len(matrices)))()
+    for i, m in enumerate(matrices):
+        sym = m.symbols
+        if not (isinstance(sym, torch.Tensor) and sym.is_cuda and sym.dtype == torch.uint8 and sym.dim() == 2):
+            raise ValueError("symbols must be a uint8 CUDA tensor [rows, cols]")
+        sym = sym.contiguous()
+        sc = m.scales.to(torch.float32).contiguous()
+        n_out = 0 if getattr(m, "out_row", None) is None else int(m.out_row.numel())
+        orow = ocol = oval = None
+        if n_out:
+            orow = m.out_row.to(torch.int32).contiguous()  # the library reads them as uint32
+            ocol = m.out_col.to(torch.int32).contiguous()
+            oval = m.out_val.to(torch.float32).contiguous()
+        keep += [sym, sc, orow, ocol, oval]
+        e = arr[i]
+        e.layer = int(m.layer)
+        e.dtype = int(m.dtype)
+        e.rows, e.cols = sym.shape
+        e.symbols = sym.data_ptr() if sym.numel() else None
+        e.scales = sc.data_ptr() if sc.numel() else None
+        e.n_out = n_out
+        e.out_row = orow.data_ptr() if n_out else None
+        e.out_col = ocol.data_ptr() if n_out else None
+        e.out_val = oval.data_ptr() if n_out else None
+        e.flags = int(getattr(m, "flags", 0)) | (EQ_TABLE_PER_CHUNK if table_scope == "chunk" else 0)
+    return arr, keep
+
+
+def encode_device(matrices, table_scope: str = "matrix", stream=None):
+    """eq_encode_device: encode matrices whose symbols, scales and super weights
+    are CUDA tensors; returns the container as a uint8 CUDA tensor (the same
+    bytes eq_encode_host writes).  Each matrix needs ``layer``, ``dtype``,
+    ``symbols`` (uint8 [rows, cols]), ``scales`` (float32 [rows]) and optionally
+    ``out_row``, ``out_col`` (integer), ``out_val`` (float32).  Synchronises
+    the stream."""
+    import torch
+    arr, keep = _device_matrix_in_array(matrices, table_scope)
+    n = len(matrices)
+    L = load()
+    wb, ob, ln = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    check(L.eq_encode_device_workspace(arr, n, ctypes.byref(wb)), "eq_encode_device_workspace")
+    check(L.eq_encode_bound(arr, n, ctypes.byref(ob)), "eq_encode_bound")
+    dev = keep[0].device if keep else torch.device("cuda")
+    work = torch.empty(max(1, wb.value), dtype=torch.uint8, device=dev)
+    out = torch.empty(max(1, ob.value), dtype=torch.uint8, device=dev)
+    check(L.eq_encode_device(arr, n, out.data_ptr(), ob.value, ctypes.byref(ln), work.data_ptr(), wb.value,
+                             _stream_handle(stream)), "eq_encode_device")
+    return out[:ln.value]
+
+
 def upload(blob: np.ndarray, device=None):
     """Copy a host container into a fresh device tensor (uint8; the allocator aligns it to >= 256 B)."""
     import torch

@@ -19,53 +19,11 @@
 #include <thread>
 #include <vector>
 
-#include "eqw_internal.h"
+#include "eqw_encode_common.h"
 
 using namespace eqw;
 
 namespace {
-
-// ---- frequency table ---------------------------------------------------------
-// Start from the proportional share rounded to nearest (at least 1 for every
-// present symbol), then move single units greedily where they cost the fewest
-// expected bits: adding one unit to s saves cnt_s * log2((f+1)/f) bits,
-// removing one costs cnt_s * log2(f/(f-1)).
-void quantize_table(const uint64_t cnt[256], uint64_t n, uint32_t f[256]) {
-    int present[256];
-    int np = 0;
-    int64_t sum = 0;
-    for (int s = 0; s < 256; ++s) {
-        f[s] = 0;
-        if (!cnt[s]) continue;
-        present[np++] = s;
-        uint64_t q = ((uint64_t)cnt[s] * kProbTotal + n / 2) / n;
-        f[s] = q ? (uint32_t)q : 1u;
-        sum += f[s];
-    }
-    while (sum < (int64_t)kProbTotal) {
-        int best = -1;
-        double gain = -1.0;
-        for (int i = 0; i < np; ++i) {
-            int s = present[i];
-            double g = cnt[s] * std::log2((f[s] + 1.0) / f[s]);
-            if (g > gain) { gain = g; best = s; }
-        }
-        f[best] += 1;
-        ++sum;
-    }
-    while (sum > (int64_t)kProbTotal) {
-        int best = -1;
-        double loss = 0.0;
-        for (int i = 0; i < np; ++i) {
-            int s = present[i];
-            if (f[s] <= 1) continue;
-            double l = cnt[s] * std::log2((double)f[s] / (f[s] - 1.0));
-            if (best < 0 || l < loss) { loss = l; best = s; }
-        }
-        f[best] -= 1;
-        --sum;
-    }
-}
 
 // ---- one chunk record ----------------------------------------------------------
 // Symbol j of the chunk belongs to lane (j % 256) / 8 at step 8 * (j / 256) + j % 8.
@@ -140,37 +98,17 @@ struct Job {
     uint32_t chunk;
 };
 
+// Shape checks plus the checks that read host data: no E4M3 NaN code, outliers in range and ascending.
 int validate(const eq_matrix_in *mats, uint32_t n_mats, uint32_t *n_layers) {
-    if (!mats && n_mats) return EQ_ERR_INVALID_ARG;
-    uint32_t max_layer = 0;
+    int rc = validate_shapes(mats, n_mats, n_layers);
+    if (rc) return rc;
     for (uint32_t i = 0; i < n_mats; ++i) {
         const eq_matrix_in &m = mats[i];
-        if (m.dtype != EQ_INT8 && m.dtype != EQ_E4M3) return EQ_ERR_INVALID_ARG;
-        if (m.flags & ~EQ_TABLE_PER_CHUNK) return EQ_ERR_INVALID_ARG;
         const uint64_t n = (uint64_t)m.rows * m.cols;
-        if (n && (!m.symbols || !m.scales)) return EQ_ERR_INVALID_ARG;
-        if ((n + kChunkSyms - 1) / kChunkSyms > 0xFFFFFFFFull) return EQ_ERR_INVALID_ARG;
         if (m.dtype == EQ_E4M3)
             for (uint64_t k = 0; k < n; ++k)
                 if ((m.symbols[k] & 0x7F) == 0x7F) return EQ_ERR_INVALID_ARG;
-        if (m.n_out && (!m.out_row || !m.out_col || !m.out_val)) return EQ_ERR_INVALID_ARG;
-        uint64_t prev = 0;
-        for (uint32_t k = 0; k < m.n_out; ++k) {
-            if (m.out_row[k] >= m.rows || m.out_col[k] >= m.cols) return EQ_ERR_INVALID_ARG;
-            const uint64_t lin = (uint64_t)m.out_row[k] * m.cols + m.out_col[k];
-            if (k && lin <= prev) return EQ_ERR_INVALID_ARG;
-            prev = lin;
-        }
-        max_layer = std::max(max_layer, m.layer);
-    }
-    if (n_mats) {
-        std::vector<char> seen(max_layer + 1, 0);
-        for (uint32_t i = 0; i < n_mats; ++i) seen[mats[i].layer] = 1;
-        for (char s : seen)
-            if (!s) return EQ_ERR_INVALID_ARG;  // layers must be 0..n-1
-        *n_layers = max_layer + 1;
-    } else {
-        *n_layers = 0;
+        if (!outliers_valid(m.rows, m.cols, m.n_out, m.out_row, m.out_col)) return EQ_ERR_INVALID_ARG;
     }
     return EQ_OK;
 }
@@ -189,20 +127,13 @@ extern "C" EQW_API int eq_encoder_run(const eq_matrix_in *mats, uint32_t n_mats,
     int rc = validate(mats, n_mats, &n_layers);
     if (rc) return rc;
 
-    // directory order: by layer, input order inside a layer
-    std::vector<uint32_t> order(n_mats);
-    for (uint32_t i = 0; i < n_mats; ++i) order[i] = i;
-    std::stable_sort(order.begin(), order.end(),
-                     [&](uint32_t a, uint32_t b) { return mats[a].layer < mats[b].layer; });
-
-    std::vector<uint32_t> n_chunks(n_mats);
+    ContainerPlan P;
+    plan_order(mats, n_mats, n_layers, P);
+    const std::vector<uint32_t> &order = P.order;
     std::vector<Job> jobs;
-    for (uint32_t d = 0; d < n_mats; ++d) {
-        const eq_matrix_in &m = mats[order[d]];
-        const uint64_t n = (uint64_t)m.rows * m.cols;
-        n_chunks[d] = (uint32_t)((n + kChunkSyms - 1) / kChunkSyms);
-        for (uint32_t k = 0; k < n_chunks[d]; ++k) jobs.push_back({d, k});
-    }
+    jobs.reserve(P.n_jobs);
+    for (uint32_t d = 0; d < n_mats; ++d)
+        for (uint32_t k = 0; k < P.n_chunks[d]; ++k) jobs.push_back({d, k});
 
     // the symbols of chunk i, with super weights replaced by the placeholder 0
     auto chunk_symbols = [&](size_t i, std::vector<uint8_t> &patched, uint32_t *len_out) -> const uint8_t * {
@@ -276,32 +207,10 @@ extern "C" EQW_API int eq_encoder_run(const eq_matrix_in *mats, uint32_t n_mats,
         encode_record(src, len, per_chunk ? nullptr : mat_table[jobs[i].mat].data(), records[i], scratch);
     });
 
-    // layout: header | directory | per matrix: chunk index, scales, outliers, records
-    uint64_t pos = align_up(kHeaderBytes + (uint64_t)kDirEntryBytes * n_mats, kSectionAlign);
-    struct Place { uint64_t ci, so, oo, rec0; };
-    std::vector<Place> place(n_mats);
-    std::vector<uint64_t> rec_off(jobs.size() + 1);
-    size_t j = 0;
-    for (uint32_t d = 0; d < n_mats; ++d) {
-        const eq_matrix_in &m = mats[order[d]];
-        Place &pl = place[d];
-        pl.ci = pos;
-        pos = align_up(pos + 8ull * (n_chunks[d] + 1), kSectionAlign);
-        pl.so = pos;
-        pos = align_up(pos + 4ull * m.rows, kSectionAlign);
-        pl.oo = 0;
-        if (m.n_out) {
-            pl.oo = pos;
-            pos = align_up(pos + 12ull * m.n_out, kSectionAlign);
-        }
-        pl.rec0 = pos;
-        for (uint32_t k = 0; k < n_chunks[d]; ++k, ++j) {
-            rec_off[j] = pos;
-            pos += records[j].size();
-        }
-        pos = align_up(pos, kSectionAlign);
-    }
-    const uint64_t total = pos;
+    std::vector<uint64_t> rec_size(jobs.size());
+    for (size_t i = 0; i < jobs.size(); ++i) rec_size[i] = records[i].size();
+    plan_offsets(mats, rec_size, P);
+    const uint64_t total = P.total;
 
     auto *enc = new (std::nothrow) eq_encoded;
     if (!enc) return EQ_ERR_NOSPACE;
@@ -312,48 +221,17 @@ extern "C" EQW_API int eq_encoder_run(const eq_matrix_in *mats, uint32_t n_mats,
         return EQ_ERR_NOSPACE;
     }
     uint8_t *b = enc->bytes.data();
-    auto put32 = [](uint8_t *p, uint32_t v) { std::memcpy(p, &v, 4); };
-    auto put64 = [](uint8_t *p, uint64_t v) { std::memcpy(p, &v, 8); };
-    std::memcpy(b, "EQW1", 4);
-    put32(b + 4, kVersion);
-    put32(b + 8, kHeaderBytes);
-    put32(b + 12, kProbBits);
-    put32(b + 16, kLanes);
-    put32(b + 20, kGroup);
-    put32(b + 24, kChunkSyms);
-    put32(b + 28, n_layers);
-    put32(b + 32, n_mats);
-    put64(b + 40, kHeaderBytes);
-    put64(b + 48, total);
-
-    std::vector<uint32_t> index_in_layer(n_layers, 0);
-    j = 0;
+    write_header_directory(b, mats, P);
     for (uint32_t d = 0; d < n_mats; ++d) {
         const eq_matrix_in &m = mats[order[d]];
-        const Place &pl = place[d];
-        uint8_t *e = b + kHeaderBytes + (uint64_t)kDirEntryBytes * d;
-        put32(e + 0, m.layer);
-        put32(e + 4, index_in_layer[m.layer]++);
-        put32(e + 8, m.dtype);
-        put32(e + 12, n_chunks[d]);
-        put32(e + 16, m.rows);
-        put32(e + 20, m.cols);
-        put32(e + 24, m.n_out);
-        put64(e + 32, pl.ci);
-        put64(e + 40, pl.so);
-        put64(e + 48, pl.oo);
-        for (uint32_t k = 0; k < n_chunks[d]; ++k) put64(b + pl.ci + 8ull * k, rec_off[j + k]);
-        const uint64_t rec_end =
-            n_chunks[d] ? rec_off[j + n_chunks[d] - 1] + records[j + n_chunks[d] - 1].size() : pl.rec0;
-        put64(b + pl.ci + 8ull * n_chunks[d], rec_end);
+        const ContainerPlan::Place &pl = P.place[d];
+        write_chunk_index(b + pl.ci, P, d);
         if (m.rows) std::memcpy(b + pl.so, m.scales, 4ull * m.rows);
-        for (uint32_t k = 0; k < m.n_out; ++k) {
-            put32(b + pl.oo + 12ull * k, m.out_row[k]);
-            put32(b + pl.oo + 12ull * k + 4, m.out_col[k]);
-            std::memcpy(b + pl.oo + 12ull * k + 8, &m.out_val[k], 4);
+        write_outliers(b + pl.oo, m.n_out, m.out_row, m.out_col, m.out_val);
+        for (uint32_t k = 0; k < P.n_chunks[d]; ++k) {
+            const uint32_t j = P.first_job[d] + k;
+            std::memcpy(b + P.rec_off[j], records[j].data(), records[j].size());
         }
-        for (uint32_t k = 0; k < n_chunks[d]; ++k, ++j)
-            std::memcpy(b + rec_off[j], records[j].data(), records[j].size());
     }
     *h = enc;
     *size = total;

@@ -35,8 +35,9 @@
  *   - Return value: EQ_OK (0) or one of the EQ_ERR_* codes; nothing throws.
  *   - The caller owns all memory, streams and events.  The library never
  *     allocates device memory, never frees caller memory and never
- *     synchronises a stream or the device.  The only allocations it makes
- *     are host-side descriptors (eq_model, eq_encoded).
+ *     synchronises a stream or the device, except eq_encode_device, which
+ *     synchronises its stream.  The only allocations it makes are host-side
+ *     descriptors and staging (eq_model, eq_encoded, encoder plans).
  *   - Device pointers are plain addresses in the current CUDA device's
  *     memory (from PyTorch: tensor.data_ptr()); streams/events are raw
  *     cudaStream_t / cudaEvent_t handles (torch.cuda.Stream().cuda_stream).
@@ -146,6 +147,37 @@ EQW_API void eq_encoded_free(eq_encoded *h);
  */
 EQW_API int eq_encode_host(const eq_matrix_in *mats, uint32_t n_mats, int n_threads,
                            void *out, size_t out_cap, size_t *out_len);
+
+/* ---- device encoder ----------------------------------------------------------------
+ * eq_encode_device writes the same container bytes as eq_encode_host for the
+ * same inputs (same tables, same layout), with the per-symbol work on the GPU
+ * (EntQuant section 2 "weight encoding": a GPU ANS coder).  Here every
+ * pointer inside eq_matrix_in is a DEVICE address: symbols (8-byte aligned),
+ * scales, out_row, out_col, out_val.  Steps, all on stream `s`: per-chunk
+ * histograms on the GPU (super-weight positions count as symbol 0; an E4M3
+ * NaN code is an error), frequency tables on the host with the host
+ * encoder's routine, a GPU pass that counts each chunk's renormalisation
+ * words, the container plan on the host, and a GPU pass that writes the
+ * records.  Unlike every other entry point it synchronises `s` (the plan
+ * needs the counts on the host).
+ *   d_out    device, out_cap bytes (eq_encode_bound gives a sufficient size);
+ *            *out_len receives the exact container size; EQ_ERR_NOSPACE
+ *            (d_out untouched) if out_cap is smaller.
+ *   d_work   device workspace of eq_encode_device_workspace() bytes,
+ *            caller-owned; contents undefined afterwards.
+ * Errors: EQ_ERR_INVALID_ARG (shapes, flags, alignment, layers not 0..n-1,
+ * an E4M3 NaN code, super weights out of range or not ascending),
+ * EQ_ERR_NOSPACE, EQ_ERR_CUDA.
+ */
+EQW_API int eq_encode_device(const eq_matrix_in *mats, uint32_t n_mats, void *d_out, size_t out_cap,
+                             size_t *out_len, void *d_work, size_t work_bytes, cudaStream_t s);
+
+/* Workspace bytes eq_encode_device needs for these matrices (shapes only). */
+EQW_API int eq_encode_device_workspace(const eq_matrix_in *mats, uint32_t n_mats, size_t *work_bytes);
+
+/* An upper bound of the container size for these matrices (shapes only):
+ * every chunk with a 256-entry table and one word per symbol. */
+EQW_API int eq_encode_bound(const eq_matrix_in *mats, uint32_t n_mats, size_t *out_bytes);
 
 /* ---- model (a container resident in device memory) ---------------------------- */
 typedef struct eq_model eq_model;
