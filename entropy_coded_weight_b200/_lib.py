@@ -71,6 +71,7 @@ SIGNATURES = {
     "eq_gemv_bf16": (_i32, [_vp, _vp, _vp, _u32, _u32, _vp]),
     "eq_encode_device": (_i32, [_vp, _u32, _vp, _sz, _vp, _vp, _sz, _vp]),
     "eq_encode_device_workspace": (_i32, [_vp, _u32, _vp]),
+    "eq_encode_device_noalloc": (_i32, [_vp, _u32, _vp, _sz, _vp, _vp]),
     "eq_encode_bound": (_i32, [_vp, _u32, _vp]),
     "eq_decode_gemv_matrix": (_i32, [_vp, _u32, _vp, _vp, _vp, _vp]),
     "eq_decode_gemv_block": (_i32, [_vp, _u32, _vp, _vp, _u32, _vp, _vp]),

@@ -27,6 +27,7 @@
 
 #include <algorithm>
 #include <array>
+#include <mutex>
 #include <vector>
 
 #include "eqw_encode_common.h"
@@ -322,8 +323,10 @@ extern "C" EQW_API int eq_encode_device_workspace(const eq_matrix_in *mats, uint
     return EQ_OK;
 }
 
-extern "C" EQW_API int eq_encode_device(const eq_matrix_in *mats, uint32_t n_mats, void *d_out, size_t out_cap,
-                                        size_t *out_len, void *d_work, size_t work_bytes, cudaStream_t s) {
+namespace {
+
+int encode_device(const eq_matrix_in *mats, uint32_t n_mats, void *d_out, size_t out_cap, size_t *out_len,
+                  void *d_work, size_t work_bytes, cudaStream_t s) {
     if (!out_len) return EQ_ERR_INVALID_ARG;
     uint32_t n_layers = 0;
     int rc = validate_shapes(mats, n_mats, &n_layers);
@@ -497,4 +500,35 @@ extern "C" EQW_API int eq_encode_device(const eq_matrix_in *mats, uint32_t n_mat
         if ((rc = cuda_ok(cudaGetLastError()))) return rc;
     }
     return cuda_ok(cudaStreamSynchronize(s));
+}
+
+}  // namespace
+
+extern "C" EQW_API int eq_encode_device(const eq_matrix_in *mats, uint32_t n_mats, void *d_out, size_t out_cap,
+                                        size_t *out_len, void *d_work, size_t work_bytes, cudaStream_t s) {
+    return encode_device(mats, n_mats, d_out, out_cap, out_len, d_work, work_bytes, s);
+}
+
+namespace {
+
+// Workspace of eq_encode_device_noalloc: a file-scope device array (one per
+// device context, reserved when the library's module loads), so that entry
+// point allocates nothing; a host mutex serialises its users.
+constexpr size_t kStaticScratchBytes = 16u << 20;
+__device__ __align__(256) uint8_t g_encode_scratch[kStaticScratchBytes];
+std::mutex g_encode_scratch_mu;
+
+}  // namespace
+
+extern "C" EQW_API int eq_encode_device_noalloc(const eq_matrix_in *mats, uint32_t n_mats, void *d_out,
+                                                size_t out_cap, size_t *out_len, cudaStream_t s) {
+    if (!out_len) return EQ_ERR_INVALID_ARG;
+    size_t need = 0;
+    int rc = eq_encode_device_workspace(mats, n_mats, &need);
+    if (rc) return rc;
+    if (need > kStaticScratchBytes) return EQ_ERR_NOSPACE;
+    void *scratch = nullptr;
+    if (cudaGetSymbolAddress(&scratch, g_encode_scratch) != cudaSuccess) return EQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_encode_scratch_mu);
+    return encode_device(mats, n_mats, d_out, out_cap, out_len, scratch, kStaticScratchBytes, s);
 }

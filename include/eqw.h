@@ -172,6 +172,14 @@ EQW_API int eq_encode_host(const eq_matrix_in *mats, uint32_t n_mats, int n_thre
 EQW_API int eq_encode_device(const eq_matrix_in *mats, uint32_t n_mats, void *d_out, size_t out_cap,
                              size_t *out_len, void *d_work, size_t work_bytes, cudaStream_t s);
 
+/* eq_encode_device with a workspace the library keeps in a file-scope device
+ * array (16 MiB per device, reserved when the library loads): no device
+ * memory is allocated and no workspace is passed.  Calls are serialised by a
+ * host lock.  EQ_ERR_NOSPACE if the matrices need more workspace than that
+ * (eq_encode_device_workspace tells). */
+EQW_API int eq_encode_device_noalloc(const eq_matrix_in *mats, uint32_t n_mats, void *d_out, size_t out_cap,
+                                     size_t *out_len, cudaStream_t s);
+
 /* Workspace bytes eq_encode_device needs for these matrices (shapes only). */
 EQW_API int eq_encode_device_workspace(const eq_matrix_in *mats, uint32_t n_mats, size_t *work_bytes);
 
