@@ -37,11 +37,13 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "rans_oracle.c")
+_SRC_HUFF = os.path.join(_HERE, "huffman_oracle.c")
 _LIB = os.path.join(_HERE, "_oracle.so")
 
 OK, ERR_ARG, ERR_CORRUPT, ERR_SPACE = 0, 1, 2, 3
 
 INT8, E4M3 = 1, 2
+CODEC_RANS, CODEC_HUFFMAN = 0, 1  # directory entry word 7
 PROB_TOTAL = 4096
 STATE_LOW = 1 << 16
 LANES = 32
@@ -65,12 +67,13 @@ class OracleError(RuntimeError):
 # ---------------------------------------------------------------------------
 
 def build(force: bool = False) -> str:
-    """Compile rans_oracle.c into _oracle.so (gcc -O2, IEEE arithmetic, no contraction)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    """Compile rans_oracle.c and huffman_oracle.c into _oracle.so (gcc -O2, IEEE arithmetic, no contraction)."""
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_SRC_HUFF))
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
         tmp = _LIB + f".{os.getpid()}.tmp"
         subprocess.check_call([
             "gcc", "-O2", "-std=c11", "-Wall", "-Wextra", "-fno-fast-math", "-ffp-contract=off",
-            "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+            "-shared", "-fPIC", "-o", tmp, _SRC, _SRC_HUFF, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -104,6 +107,10 @@ def lib() -> ctypes.CDLL:
         L.orc_scatter.argtypes = [u64, u64, u32, vp, vp, vp, vp]
         L.orc_bf16_rne_n.argtypes = [vp, u64, vp]
         L.orc_bf16_rne_n.restype = None
+        L.orc_huff_lengths.argtypes = [vp, vp]
+        L.orc_huff_canonical.argtypes = [vp, vp]
+        L.orc_huff_encode_chunk.argtypes = [vp, u32, vp, i32, vp, u32, vp]
+        L.orc_huff_decode_chunk.argtypes = [vp, u32, vp, i32, ctypes.c_uint8, u32, vp]
         _lib = L
     return _lib
 
@@ -182,6 +189,61 @@ def decode_chunk(states: np.ndarray, words: np.ndarray, f: np.ndarray, n: int,
         return rc, out[:n], fin
     if rc:
         raise OracleError(rc, "decode_chunk")
+    return out[:n]
+
+
+# ---------------------------------------------------------------------------
+# one chunk, Huffman codec (EntroLLM technical overview, "Huffman weight
+# encoding"; readings in huffman_oracle.c)
+# ---------------------------------------------------------------------------
+
+HUFF_MAX_LEN = 12
+
+
+def huff_lengths(symbols=None, counts=None) -> np.ndarray:
+    """Optimal code lengths (uint8[256], <= 12 bits; all 0 for a single distinct symbol)."""
+    if counts is None:
+        counts = np.bincount(np.asarray(symbols, np.uint8).reshape(-1), minlength=256)
+    counts = np.ascontiguousarray(counts, np.uint64)
+    ln = np.zeros(256, np.uint8)
+    rc = lib().orc_huff_lengths(_p(counts), _p(ln))
+    if rc:
+        raise OracleError(rc, "huff_lengths")
+    return ln
+
+
+def huff_canonical(lengths) -> np.ndarray | None:
+    """Canonical codes (uint16[256]) for the lengths, or None if they are not a complete code."""
+    ln = np.ascontiguousarray(lengths, np.uint8)
+    code = np.zeros(256, np.uint16)
+    return code if lib().orc_huff_canonical(_p(ln), _p(code)) else None
+
+
+def huff_encode_chunk(symbols: np.ndarray, lengths: np.ndarray | None = None):
+    """Huffman-encode one chunk.  Returns (words uint16[W], lengths uint8[256], single)."""
+    sym = np.ascontiguousarray(symbols, dtype=np.uint8).reshape(-1)
+    if lengths is None:
+        lengths = huff_lengths(sym)
+    ln = np.ascontiguousarray(lengths, np.uint8)
+    single = int(sym.size > 0 and not ln.any())
+    cap = max(1, sym.size)
+    words = np.zeros(cap, np.uint16)
+    nw = np.zeros(1, np.uint32)
+    rc = lib().orc_huff_encode_chunk(_p(sym), sym.size, _p(ln), single, _p(words), cap, _p(nw))
+    if rc:
+        raise OracleError(rc, "huff_encode_chunk")
+    return words[: int(nw[0])].copy(), ln, bool(single)
+
+
+def huff_decode_chunk(words: np.ndarray, lengths: np.ndarray, n: int, single_symbol: int | None = None):
+    """Huffman-decode one chunk of ``n`` symbols (``single_symbol``: the symbol of an empty code)."""
+    words = np.ascontiguousarray(words, dtype=np.uint16)
+    ln = np.ascontiguousarray(lengths, np.uint8)
+    out = np.zeros(max(n, 1), np.uint8)
+    rc = lib().orc_huff_decode_chunk(_p(words) if words.size else None, words.size, _p(ln),
+                                     int(single_symbol is not None), single_symbol or 0, n, _p(out))
+    if rc:
+        raise OracleError(rc, "huff_decode_chunk")
     return out[:n]
 
 
@@ -303,7 +365,26 @@ def _align(x: int, a: int) -> int:
     return (x + a - 1) // a * a
 
 
-def _chunk_record(sym: np.ndarray) -> bytes:
+def _huffman_record(sym: np.ndarray) -> bytes:
+    """Huffman chunk record: n_syms, n_words, n_present, 0; entries symbol | length << 16
+    sorted by (length, symbol) (one entry of length 0 for a single-symbol chunk); words."""
+    words, ln, single = huff_encode_chunk(sym)
+    if single:
+        table = np.array([int(sym[0])], np.uint32)
+    else:
+        present = np.nonzero(ln)[0]
+        present = present[np.lexsort((present, ln[present]))]
+        table = (present.astype(np.uint32) | (ln[present].astype(np.uint32) << 16)).astype(np.uint32)
+    body = struct.pack("<4I", sym.size, words.size, table.size, 0) + table.astype("<u4").tobytes()
+    body += b"\0" * (_align(len(body), 16) - len(body))
+    wb = words.astype("<u2").tobytes()
+    wb += b"\0" * (_align(len(wb), 16) - len(wb))
+    return body + wb
+
+
+def _chunk_record(sym: np.ndarray, codec: int = CODEC_RANS) -> bytes:
+    if codec == CODEC_HUFFMAN:
+        return _huffman_record(sym)
     states, words, f = encode_chunk(sym)
     present = np.nonzero(f)[0]
     table = (present.astype(np.uint32) | (f[present].astype(np.uint32) << 16)).astype(np.uint32)
@@ -330,12 +411,14 @@ def _check_matrix(m) -> None:
             raise OracleError(ERR_ARG, "outliers not sorted/unique")
 
 
-def encode_container(mats, threads: int | None = None) -> np.ndarray:
+def encode_container(mats, threads: int | None = None, codec: str = "rans") -> np.ndarray:
     """Write matrices (objects with layer, index, dtype, symbols, scales, out_*) into a v1 blob.
 
     Layers must be numbered 0..n_layers-1; within a layer the matrices are
     ordered by ``index``.  The symbol at each outlier position is replaced by
     the placeholder 0 before encoding (its value is overwritten by the scatter).
+    ``codec``: "rans" or "huffman" for every matrix (a matrix's own ``codec``
+    attribute, if present, wins).
     """
     mats = sorted(mats, key=lambda m: (m.layer, m.index))
     layers = sorted({m.layer for m in mats})
@@ -344,6 +427,7 @@ def encode_container(mats, threads: int | None = None) -> np.ndarray:
     for m in mats:
         _check_matrix(m)
 
+    codecs = [{"rans": CODEC_RANS, "huffman": CODEC_HUFFMAN}[getattr(m, "codec", codec)] for m in mats]
     jobs = []
     for mi, m in enumerate(mats):
         flat = np.ascontiguousarray(m.symbols, np.uint8).reshape(-1)
@@ -353,7 +437,7 @@ def encode_container(mats, threads: int | None = None) -> np.ndarray:
         for k in range(0, m.n, CHUNK_SYMS):
             jobs.append((mi, flat[k:k + CHUNK_SYMS]))
     with ThreadPoolExecutor(_threads(threads)) as ex:
-        records = list(ex.map(lambda j: _chunk_record(j[1]), jobs))
+        records = list(ex.map(lambda j: _chunk_record(j[1], codecs[j[0]]), jobs))
     per_mat: list[list[bytes]] = [[] for _ in mats]
     for (mi, _), rec in zip(jobs, records):
         per_mat[mi].append(rec)
@@ -389,7 +473,7 @@ def encode_container(mats, threads: int | None = None) -> np.ndarray:
         nch = len(per_mat[mi])
         e = dir_off + DIR_ENTRY_BYTES * mi
         mv[e:e + DIR_ENTRY_BYTES] = struct.pack("<8I4Q", m.layer, m.index, m.dtype, nch, m.rows, m.cols,
-                                                len(m.out_row), 0, ci, so, oo, 0)
+                                                len(m.out_row), codecs[mi], ci, so, oo, 0)
         mv[ci:ci + 8 * (nch + 1)] = np.asarray(offs, "<u8").tobytes()
         mv[so:so + 4 * m.rows] = np.ascontiguousarray(m.scales, "<f4").tobytes()
         if len(m.out_row):
@@ -423,17 +507,18 @@ def parse_container(blob) -> dict:
     mats = []
     for mi in range(n_mats):
         e = dir_off + DIR_ENTRY_BYTES * mi
-        (layer, index, dtype, nch, rows, cols, n_out, _r, ci, so, oo, _q) = struct.unpack(
+        (layer, index, dtype, nch, rows, cols, n_out, codec, ci, so, oo, _q) = struct.unpack(
             "<8I4Q", bytes(b[e:e + DIR_ENTRY_BYTES]))
         n = rows * cols
-        if dtype not in (INT8, E4M3) or layer >= n_layers:
+        if dtype not in (INT8, E4M3) or layer >= n_layers or codec not in (CODEC_RANS, CODEC_HUFFMAN):
             raise OracleError(ERR_CORRUPT, "bad directory entry")
         if nch != (n + CHUNK_SYMS - 1) // CHUNK_SYMS:
             raise OracleError(ERR_CORRUPT, "chunk count")
         if ci + 8 * (nch + 1) > total or so + 4 * rows > total or (n_out and oo + 12 * n_out > total):
             raise OracleError(ERR_CORRUPT, "section out of range")
         offs = np.frombuffer(bytes(b[ci:ci + 8 * (nch + 1)]), "<u8").astype(np.int64)
-        if np.any(np.diff(offs) < 144) or offs[-1] > total or np.any(offs % 16):
+        min_rec = 144 if codec == CODEC_RANS else 32
+        if np.any(np.diff(offs) < min_rec) or offs[-1] > total or np.any(offs % 16):
             raise OracleError(ERR_CORRUPT, "chunk index")
         scales = np.frombuffer(bytes(b[so:so + 4 * rows]), "<f4").copy()
         if n_out:
@@ -442,16 +527,39 @@ def parse_container(blob) -> dict:
         else:
             orow = ocol = np.zeros(0, np.uint32)
             oval = np.zeros(0, np.float32)
-        mats.append(dict(layer=layer, index=index, dtype=dtype, rows=rows, cols=cols, n_chunks=nch,
+        mats.append(dict(layer=layer, index=index, dtype=dtype, codec=codec, rows=rows, cols=cols, n_chunks=nch,
                          chunk_offsets=offs, scales=scales, out_row=orow, out_col=ocol, out_val=oval))
     return dict(n_layers=n_layers, matrices=mats, blob=b)
 
 
-def _decode_record(b: np.ndarray, off: int, end: int, n_expected: int) -> np.ndarray:
+def _decode_huffman_record(b: np.ndarray, off: int, end: int, n: int, nw: int, npres: int) -> np.ndarray:
+    table = np.frombuffer(bytes(b[off + 16:off + 16 + 4 * npres]), "<u4")
+    wo = off + _align(16 + 4 * npres, 16)
+    if wo + 2 * nw > end:
+        raise OracleError(ERR_CORRUPT, "chunk record overflows")
+    words = np.frombuffer(bytes(b[wo:wo + 2 * nw]), "<u2")
+    syms, lens = (table & 0xFF).astype(np.int64), (table >> 16).astype(np.int64)
+    if np.any((table >> 8) & 0xFF):
+        raise OracleError(ERR_CORRUPT, "table entry")
+    if npres == 1:
+        if lens[0] != 0:
+            raise OracleError(ERR_CORRUPT, "single-symbol code")
+        return huff_decode_chunk(words, np.zeros(256, np.uint8), n, single_symbol=int(syms[0]))
+    key = lens * 256 + syms
+    if np.any(np.diff(key) <= 0) or np.any(lens < 1) or np.any(lens > HUFF_MAX_LEN):
+        raise OracleError(ERR_CORRUPT, "table order")
+    ln = np.zeros(256, np.uint8)
+    ln[syms] = lens
+    return huff_decode_chunk(words, ln, n)
+
+
+def _decode_record(b: np.ndarray, off: int, end: int, n_expected: int, codec: int = CODEC_RANS) -> np.ndarray:
     head = np.frombuffer(bytes(b[off:off + 16]), "<u4")
     n, nw, npres = int(head[0]), int(head[1]), int(head[2])
     if n != n_expected or not (1 <= npres <= 256):
         raise OracleError(ERR_CORRUPT, "chunk header")
+    if codec == CODEC_HUFFMAN:
+        return _decode_huffman_record(b, off, end, n, nw, npres)
     states = np.frombuffer(bytes(b[off + 16:off + 144]), "<u4")
     table = np.frombuffer(bytes(b[off + 144:off + 144 + 4 * npres]), "<u4")
     wo = off + _align(144 + 4 * npres, 16)
@@ -477,7 +585,7 @@ def decode_matrix_symbols(parsed: dict, mi: int, threads: int | None = None) -> 
     def one(k):
         lo = k * CHUNK_SYMS
         cnt = min(CHUNK_SYMS, n - lo)
-        out[lo:lo + cnt] = _decode_record(b, int(offs[k]), int(offs[k + 1]), cnt)
+        out[lo:lo + cnt] = _decode_record(b, int(offs[k]), int(offs[k + 1]), cnt, m["codec"])
 
     with ThreadPoolExecutor(_threads(threads)) as ex:
         list(ex.map(one, range(m["n_chunks"])))

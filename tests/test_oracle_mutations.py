@@ -13,9 +13,11 @@ import subprocess
 import pytest
 
 import test_oracle_formats as F
+import test_oracle_huffman as H
 import test_oracle_rans as R
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "rans_oracle.c")
+HUFF_SRC = os.path.join(os.path.dirname(SRC), "huffman_oracle.c")
 
 MUTATIONS = {
     # symbol j -> lane j mod 32 instead of 8-symbol groups per lane
@@ -72,6 +74,60 @@ MUTATIONS = {
 }
 
 
+# the same, planted in a copy of oracle/huffman_oracle.c
+HUFF_MUTATIONS = {
+    # canonical codes: no shift when the length grows
+    "canonical_no_shift": ("if (prev_len) c = (c + 1) << (L - prev_len);", "if (prev_len) c = c + 1;",
+                           [H.test_rfc1951_canonical_codes]),
+    # bits stored least significant first
+    "bit_order": ("bits[l][nbits[l]++] = (uint8_t)((code[sym[j]] >> (L - 1 - b)) & 1u);",
+                  "bits[l][nbits[l]++] = (uint8_t)((code[sym[j]] >> b) & 1u);",
+                  [H.test_hand_derived_interleaving, H.test_hand_derived_interleaving_multibit_codes]),
+    # refill threshold 11 bits instead of 12 (in the encoder's schedule)
+    "refill_threshold": ("            if (held[l] < HUF_MAX_LEN) {\n                uint32_t w = 0;",
+                         "            if (held[l] < HUF_MAX_LEN - 1) {\n                uint32_t w = 0;",
+                         [H.test_hand_derived_interleaving, H.test_exhaustive_round_trip_tiny]),
+    # package-merge keeps one item too few (suboptimal or invalid lengths)
+    "package_merge_count": ("for (int i = 0; i < 2 * n - 2; ++i)", "for (int i = 0; i < 2 * n - 3; ++i)",
+                            [H.test_textbook_lengths, H.test_lengths_optimal_against_dynamic_program]),
+    # merge prefers packages on equal weights (still optimal, different lengths on ties)
+    # is not a mistake; a merge that ignores package weights is:
+    "merge_order": ("if (b >= p || (a < n && leaves[a].w <= next[b].w)) merged[k++] = leaves[a++];",
+                    "if (b >= p || a < n) merged[k++] = leaves[a++];",
+                    [H.test_textbook_lengths, H.test_lengths_optimal_against_dynamic_program]),
+    # decoder skips the end check of the padding bits
+    "no_padding_check": ("            if (q[l][(head[l] + b) % 64]) return HUF_ERR_CORRUPT;", "            ;",
+                         [H.test_corruption_detected]),
+}
+
+
+@pytest.mark.parametrize("name", sorted(HUFF_MUTATIONS))
+def test_huffman_pins_catch_planted_mistake(orc, tmp_path, name):
+    old, new, pins = HUFF_MUTATIONS[name]
+    src = open(HUFF_SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    mutant = tmp_path / "mutant_huffman.c"
+    mutant.write_text(src.replace(old, new))
+    so = tmp_path / "mutant.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-shared",
+                           "-fPIC", "-o", str(so), SRC, str(mutant), "-lm"])
+    orc._use_library(str(so))
+    try:
+        caught = 0
+        for pin in pins:
+            try:
+                if pin is H.test_lengths_optimal_against_dynamic_program:
+                    for seed in range(6):
+                        pin(orc, seed)
+                else:
+                    pin(orc)
+            except (AssertionError, orc.OracleError, pytest.fail.Exception):
+                caught += 1
+        assert caught >= 1, f"planted mistake {name} passed every pin"
+    finally:
+        orc._use_library(None)
+
+
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_pins_catch_planted_mistake(orc, tmp_path, name):
     old, new, pins = MUTATIONS[name]
@@ -81,7 +137,7 @@ def test_pins_catch_planted_mistake(orc, tmp_path, name):
     mutant.write_text(src.replace(old, new))
     so = tmp_path / "mutant.so"
     subprocess.check_call(["gcc", "-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-shared",
-                           "-fPIC", "-o", str(so), str(mutant), "-lm"])
+                           "-fPIC", "-o", str(so), str(mutant), HUFF_SRC, "-lm"])
     orc._use_library(str(so))
     try:
         caught = 0
