@@ -24,7 +24,7 @@ import numpy as np
 
 from . import _lib
 from ._lib import (EQ_DEV_BAD_END, EQ_DEV_BAD_HEADER, EQ_DEV_BAD_OUTLIER, EQ_DEV_BAD_STATE, EQ_DEV_BAD_TABLE,
-                   EQ_DEV_TIMEOUT, EQ_E4M3, EQ_INT8, EQ_TABLE_PER_CHUNK, EqError, check, eq_matrix_in,
+                   EQ_CODEC_HUFFMAN, EQ_DEV_TIMEOUT, EQ_E4M3, EQ_INT8, EQ_TABLE_PER_CHUNK, EqError, check, eq_matrix_in,
                    eq_matrix_info, load)
 
 __all__ = [
@@ -57,7 +57,7 @@ def eq_format_version() -> int:
     return load().eq_format_version()
 
 
-def _matrix_in_array(matrices, table_scope: str = "matrix"):
+def _matrix_in_array(matrices, table_scope: str = "matrix", codec: str = "rans"):
     """eq_matrix_in[] for objects with layer, dtype, symbols, scales, out_row/out_col/out_val."""
     keep = []
     arr = (eq_matrix_in * max(1, len(matrices)))()
@@ -80,20 +80,27 @@ def _matrix_in_array(matrices, table_scope: str = "matrix"):
         e.out_row = orow.ctypes.data if orow.size else None
         e.out_col = ocol.ctypes.data if ocol.size else None
         e.out_val = oval.ctypes.data if oval.size else None
-        e.flags = int(getattr(m, "flags", 0)) | (EQ_TABLE_PER_CHUNK if table_scope == "chunk" else 0)
+        e.flags = _flags(m, table_scope, codec)
     return arr, keep
 
 
-def encode_host(matrices, n_threads: int = 0, table_scope: str = "matrix") -> np.ndarray:
+def _flags(m, table_scope: str, codec: str) -> int:
+    if table_scope not in ("matrix", "chunk") or codec not in ("rans", "huffman"):
+        raise ValueError("table_scope must be 'matrix' or 'chunk', codec 'rans' or 'huffman'")
+    return (int(getattr(m, "flags", 0)) | (EQ_TABLE_PER_CHUNK if table_scope == "chunk" else 0)
+            | (EQ_CODEC_HUFFMAN if getattr(m, "codec", codec) == "huffman" else 0))
+
+
+def encode_host(matrices, n_threads: int = 0, table_scope: str = "matrix", codec: str = "rans") -> np.ndarray:
     """Encode matrices into a container v1 blob (uint8 numpy array) with eq_encoder_run.
 
-    ``table_scope``: "matrix" (one 12-bit table quantised from the whole
-    matrix, written into every chunk) or "chunk" (each chunk's own histogram).
+    ``table_scope``: "matrix" (one table from the whole matrix's histogram,
+    written into every chunk) or "chunk" (each chunk's own histogram).
+    ``codec``: "rans" (12-bit rANS) or "huffman" (canonical Huffman codes of
+    at most 12 bits); a matrix's own ``codec`` attribute wins.
     """
-    if table_scope not in ("matrix", "chunk"):
-        raise ValueError("table_scope must be 'matrix' or 'chunk'")
     L = load()
-    arr, keep = _matrix_in_array(matrices, table_scope)
+    arr, keep = _matrix_in_array(matrices, table_scope, codec)
     h = ctypes.c_void_p()
     size = ctypes.c_size_t()
     check(L.eq_encoder_run(arr, len(matrices), n_threads, ctypes.byref(h), ctypes.byref(size)), "eq_encoder_run")
@@ -134,7 +141,7 @@ def _device_matrix_in_array(matrices, table_scope: str):
         e.out_row = orow.data_ptr() if n_out else None
         e.out_col = ocol.data_ptr() if n_out else None
         e.out_val = oval.data_ptr() if n_out else None
-        e.flags = int(getattr(m, "flags", 0)) | (EQ_TABLE_PER_CHUNK if table_scope == "chunk" else 0)
+        e.flags = _flags(m, table_scope, "rans")
     return arr, keep
 
 

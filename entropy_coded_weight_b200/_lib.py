@@ -18,6 +18,7 @@ EQ_DEV_BAD_HEADER, EQ_DEV_BAD_TABLE, EQ_DEV_BAD_STATE = 1, 2, 4
 EQ_DEV_BAD_END, EQ_DEV_TIMEOUT, EQ_DEV_BAD_OUTLIER = 8, 16, 32
 EQ_INT8, EQ_E4M3 = 1, 2
 EQ_TABLE_PER_CHUNK = 1
+EQ_CODEC_HUFFMAN = 2
 
 
 class EqError(RuntimeError):
@@ -45,7 +46,8 @@ class eq_matrix_in(ctypes.Structure):
 
 class eq_matrix_info(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint32) for n in
-                ("layer", "index", "dtype", "rows", "cols", "n_chunks", "n_outliers", "uniform_table")] + [
+                ("layer", "index", "dtype", "rows", "cols", "n_chunks", "n_outliers", "uniform_table",
+                 "codec", "reserved")] + [
         ("compressed_bytes", ctypes.c_uint64),
         ("payload_words", ctypes.c_uint64),
     ]

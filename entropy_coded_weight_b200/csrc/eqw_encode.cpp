@@ -93,6 +93,156 @@ void encode_record(const uint8_t *sym, uint32_t n, const uint32_t *table, std::v
     std::memcpy(p + table_end, w, 2 * (size_t)n_words);
 }
 
+// ---- Huffman codec (EntroLLM technical overview, "Huffman weight encoding") -----
+// Code lengths: Huffman's construction (repeatedly merge the two lightest
+// nodes; ties by creation order, leaves in symbol order first), then, if a
+// code exceeds 12 bits, the length adjustment of the JPEG standard (ITU-T
+// T.81 Annex K.3, "Adjust_BITS"): two codes of the longest length i give way
+// to one code of length i-1, and one code of the deepest shorter length j
+// becomes two codes of length j+1, which keeps the Kraft sum at 1.  The
+// lengths are then handed out shortest first to the most frequent symbols.
+// One distinct symbol: the empty code (all lengths 0).
+void huffman_lengths(const uint64_t cnt[256], uint8_t len[256]) {
+    std::memset(len, 0, 256);
+    struct Node {
+        uint64_t w;
+        int left, right;
+    };
+    std::vector<Node> nodes;
+    std::vector<int> sym_node(256, -1);
+    for (int s = 0; s < 256; ++s)
+        if (cnt[s]) {
+            sym_node[s] = (int)nodes.size();
+            nodes.push_back({cnt[s], -1, -1});
+        }
+    const int n = (int)nodes.size();
+    if (n < 2) return;
+    // min-heap on (weight, node index)
+    auto heavier = [&](int a, int b) { return nodes[a].w != nodes[b].w ? nodes[a].w > nodes[b].w : a > b; };
+    std::vector<int> heap;
+    for (int i = 0; i < n; ++i) heap.push_back(i);
+    std::make_heap(heap.begin(), heap.end(), heavier);
+    while (heap.size() > 1) {
+        std::pop_heap(heap.begin(), heap.end(), heavier);
+        const int a = heap.back();
+        heap.pop_back();
+        std::pop_heap(heap.begin(), heap.end(), heavier);
+        const int b = heap.back();
+        heap.pop_back();
+        nodes.push_back({nodes[a].w + nodes[b].w, a, b});
+        heap.push_back((int)nodes.size() - 1);
+        std::push_heap(heap.begin(), heap.end(), heavier);
+    }
+    // depth of every leaf
+    std::vector<int> depth(nodes.size(), 0);
+    for (int i = (int)nodes.size() - 1; i >= n; --i) {
+        depth[nodes[i].left] = depth[i] + 1;
+        depth[nodes[i].right] = depth[i] + 1;
+    }
+    std::vector<uint32_t> bits(258, 0);  // bits[l] = number of codes of length l
+    int max_len = 0;
+    for (int i = 0; i < n; ++i) {
+        ++bits[depth[i]];
+        max_len = std::max(max_len, depth[i]);
+    }
+    for (int i = max_len; i > (int)kHuffMaxLen; --i) {
+        while (bits[i] > 0) {
+            int j = i - 2;
+            while (bits[j] == 0) --j;
+            bits[i] -= 2;
+            bits[i - 1] += 1;
+            bits[j + 1] += 2;
+            bits[j] -= 1;
+        }
+    }
+    // shortest codes to the most frequent symbols (ties: smaller symbol first)
+    std::vector<int> order;
+    for (int s = 0; s < 256; ++s)
+        if (cnt[s]) order.push_back(s);
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cnt[a] > cnt[b]; });
+    size_t k = 0;
+    for (uint32_t l = 1; l <= kHuffMaxLen; ++l)
+        for (uint32_t c = 0; c < bits[l]; ++c) len[order[k++]] = (uint8_t)l;
+}
+
+// One Huffman chunk record.  `table_len` holds the matrix-wide lengths, or
+// null to build this chunk's own code.  Lane l's bit stream is its symbols'
+// canonical codes in step order, most significant bit first, cut into 16-bit
+// words; before each of its symbols a lane holding fewer than 12 unread bits
+// takes its next word, and the record stores those words in the order they
+// are taken (step by step, lanes ascending).
+void encode_record_huffman(const uint8_t *sym, uint32_t n, const uint32_t *table_len, std::vector<uint8_t> &rec) {
+    uint8_t len[256];
+    uint64_t cnt[256] = {0};
+    for (uint32_t j = 0; j < n; ++j) ++cnt[sym[j]];
+    if (table_len) {
+        for (int s = 0; s < 256; ++s) len[s] = (uint8_t)table_len[s];
+    } else {
+        huffman_lengths(cnt, len);
+    }
+    // canonical codes in (length, symbol) order
+    std::vector<uint32_t> entries;
+    uint16_t code[256] = {0};
+    uint32_t c = 0, prev_len = 0;
+    for (uint32_t l = 1; l <= kHuffMaxLen; ++l)
+        for (int s = 0; s < 256; ++s) {
+            if (len[s] != l) continue;
+            c = prev_len ? (c + 1) << (l - prev_len) : 0u;
+            prev_len = l;
+            code[s] = (uint16_t)c;
+            entries.push_back((uint32_t)s | (l << 16));
+        }
+    const bool single = entries.empty();
+    std::vector<uint16_t> out;
+    if (single) {
+        int s0 = 0;
+        while (s0 < 255 && !cnt[s0]) ++s0;
+        entries.push_back((uint32_t)s0);
+    } else {
+        // each lane's stream as 16-bit words
+        std::vector<uint16_t> stream[kLanes];
+        uint32_t acc[kLanes] = {0}, nacc[kLanes] = {0};
+        const uint32_t steps = kGroup * ((n + kGroupSyms - 1) / kGroupSyms);
+        auto index_of = [](uint32_t t, uint32_t l) { return kGroupSyms * (t / kGroup) + kGroup * l + t % kGroup; };
+        for (uint32_t t = 0; t < steps; ++t)
+            for (uint32_t l = 0; l < kLanes; ++l) {
+                const uint32_t j = index_of(t, l);
+                if (j >= n) continue;
+                const uint32_t L = len[sym[j]];
+                acc[l] = (acc[l] << L) | code[sym[j]];
+                nacc[l] += L;
+                if (nacc[l] >= 16) {
+                    stream[l].push_back((uint16_t)(acc[l] >> (nacc[l] - 16)));
+                    nacc[l] -= 16;
+                    acc[l] &= (1u << nacc[l]) - 1u;
+                }
+            }
+        for (uint32_t l = 0; l < kLanes; ++l)
+            if (nacc[l]) stream[l].push_back((uint16_t)(acc[l] << (16 - nacc[l])));
+        // the decoder's refill schedule
+        uint32_t held[kLanes] = {0}, taken[kLanes] = {0};
+        for (uint32_t t = 0; t < steps; ++t)
+            for (uint32_t l = 0; l < kLanes; ++l) {
+                const uint32_t j = index_of(t, l);
+                if (j >= n) continue;
+                if (held[l] < kHuffMaxLen) {
+                    out.push_back(taken[l] < stream[l].size() ? stream[l][taken[l]] : (uint16_t)0);
+                    ++taken[l];
+                    held[l] += 16;
+                }
+                held[l] -= len[sym[j]];
+            }
+    }
+    const uint32_t n_present = (uint32_t)entries.size();
+    const size_t table_end = align_up(kHuffRecordHeadBytes + 4 * (size_t)n_present, 16);
+    rec.assign(table_end + align_up(2 * out.size(), 16), 0);
+    uint8_t *p = rec.data();
+    const uint32_t head[4] = {n, (uint32_t)out.size(), n_present, 0};
+    std::memcpy(p, head, 16);
+    std::memcpy(p + kHuffRecordHeadBytes, entries.data(), 4 * entries.size());
+    if (!out.empty()) std::memcpy(p + table_end, out.data(), 2 * out.size());
+}
+
 struct Job {
     uint32_t mat;
     uint32_t chunk;
@@ -190,7 +340,14 @@ extern "C" EQW_API int eq_encoder_run(const eq_matrix_in *mats, uint32_t n_mats,
         for (uint32_t d = 0; d < n_mats; ++d) {
             uint64_t n = 0;
             for (int s = 0; s < 256; ++s) n += total[d][s];
-            if (n) quantize_table(total[d].data(), n, mat_table[d].data());
+            if (!n) continue;
+            if (mats[order[d]].flags & EQ_CODEC_HUFFMAN) {
+                uint8_t len[256];
+                huffman_lengths(total[d].data(), len);
+                for (int s = 0; s < 256; ++s) mat_table[d][s] = len[s];
+            } else {
+                quantize_table(total[d].data(), n, mat_table[d].data());
+            }
         }
     }
     hist.clear();
@@ -203,8 +360,10 @@ extern "C" EQW_API int eq_encoder_run(const eq_matrix_in *mats, uint32_t n_mats,
         thread_local std::vector<uint8_t> patched;
         uint32_t len = 0;
         const uint8_t *src = chunk_symbols(i, patched, &len);
-        const bool per_chunk = mats[order[jobs[i].mat]].flags & EQ_TABLE_PER_CHUNK;
-        encode_record(src, len, per_chunk ? nullptr : mat_table[jobs[i].mat].data(), records[i], scratch);
+        const uint32_t flags = mats[order[jobs[i].mat]].flags;
+        const uint32_t *table = (flags & EQ_TABLE_PER_CHUNK) ? nullptr : mat_table[jobs[i].mat].data();
+        if (flags & EQ_CODEC_HUFFMAN) encode_record_huffman(src, len, table, records[i]);
+        else encode_record(src, len, table, records[i], scratch);
     });
 
     std::vector<uint64_t> rec_size(jobs.size());

@@ -160,6 +160,7 @@ inline void write_header_directory(uint8_t *b, const eq_matrix_in *mats, const C
         put32(e + 16, m.rows);
         put32(e + 20, m.cols);
         put32(e + 24, m.n_out);
+        put32(e + 28, (m.flags & EQ_CODEC_HUFFMAN) ? kCodecHuffman : kCodecRans);
         put64(e + 32, pl.ci);
         put64(e + 40, pl.so);
         put64(e + 48, pl.oo);
@@ -202,7 +203,7 @@ inline int validate_shapes(const eq_matrix_in *mats, uint32_t n_mats, uint32_t *
     for (uint32_t i = 0; i < n_mats; ++i) {
         const eq_matrix_in &m = mats[i];
         if (m.dtype != EQ_INT8 && m.dtype != EQ_E4M3) return EQ_ERR_INVALID_ARG;
-        if (m.flags & ~EQ_TABLE_PER_CHUNK) return EQ_ERR_INVALID_ARG;
+        if (m.flags & ~(EQ_TABLE_PER_CHUNK | EQ_CODEC_HUFFMAN)) return EQ_ERR_INVALID_ARG;
         const uint64_t n = (uint64_t)m.rows * m.cols;
         if (n && (!m.symbols || !m.scales)) return EQ_ERR_INVALID_ARG;
         if ((n + kChunkSyms - 1) / kChunkSyms > 0xFFFFFFFFull) return EQ_ERR_INVALID_ARG;

@@ -333,6 +333,7 @@ int encode_device(const eq_matrix_in *mats, uint32_t n_mats, void *d_out, size_t
     if (rc) return rc;
     for (uint32_t i = 0; i < n_mats; ++i) {
         const eq_matrix_in &m = mats[i];
+        if (m.flags & EQ_CODEC_HUFFMAN) return EQ_ERR_UNSUPPORTED;
         if ((uint64_t)m.rows * m.cols && reinterpret_cast<uintptr_t>(m.symbols) % 8) return EQ_ERR_INVALID_ARG;
     }
     ContainerPlan P;

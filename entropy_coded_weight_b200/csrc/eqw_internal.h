@@ -25,6 +25,14 @@ constexpr uint32_t kStateLow = 1u << 16;
 constexpr uint32_t kRecordHeadBytes = 16 + 4 * kLanes;  // counts + 32 states
 constexpr uint64_t kSectionAlign = 256;
 constexpr uint32_t kMaxMatsPerLaunch = 16;
+constexpr uint32_t kCodecRans = 0;
+constexpr uint32_t kCodecHuffman = 1;
+constexpr uint32_t kHuffMaxLen = 12;          // longest Huffman code; refill below this many held bits
+constexpr uint32_t kHuffRecordHeadBytes = 16; // counts only (no states)
+
+inline uint32_t record_head_bytes(uint32_t codec) {
+    return codec == kCodecHuffman ? kHuffRecordHeadBytes : kRecordHeadBytes;
+}
 
 inline uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 
@@ -34,6 +42,7 @@ struct MatrixDesc {
     uint64_t scales_off;
     uint64_t outliers_off;
     bool small_scales;    // every scale finite with |scale| < 2^8 (E4M3 single-multiply dequant is exact)
+    uint32_t codec;       // kCodecRans or kCodecHuffman
 };
 
 }  // namespace eqw

@@ -57,6 +57,36 @@ int check_record(const uint8_t *b, uint64_t off, uint64_t end, uint32_t n_expect
     return EQ_OK;
 }
 
+// Validate one Huffman chunk record [off, end) holding n_expect symbols: table
+// sorted by (length, symbol), lengths 1..12 forming a complete prefix code
+// (Kraft sum exactly 1), or a single symbol with the empty code and no words.
+int check_huffman_record(const uint8_t *b, uint64_t off, uint64_t end, uint32_t n_expect, uint64_t *n_words_out) {
+    if (off % 16 || end % 16 || end < off + kHuffRecordHeadBytes + 16) return EQ_ERR_CORRUPT;
+    const uint32_t n = rd<uint32_t>(b + off);
+    const uint32_t n_words = rd<uint32_t>(b + off + 4);
+    const uint32_t n_present = rd<uint32_t>(b + off + 8);
+    if (n != n_expect || n_present < 1 || n_present > 256) return EQ_ERR_CORRUPT;
+    const uint64_t table_end = align_up(kHuffRecordHeadBytes + 4ull * n_present, 16);
+    if (off + table_end + align_up(2ull * n_words, 16) != end) return EQ_ERR_CORRUPT;
+    uint32_t kraft = 0;
+    uint32_t prev_key = 0;
+    for (uint32_t k = 0; k < n_present; ++k) {
+        const uint32_t e = rd<uint32_t>(b + off + kHuffRecordHeadBytes + 4 * k);
+        const uint32_t len = e >> 16, key = (len << 8) | (e & 0xFFu);
+        if (e & 0xFF00u) return EQ_ERR_CORRUPT;
+        if (n_present == 1) {
+            if (len != 0 || n_words != 0) return EQ_ERR_CORRUPT;
+            continue;
+        }
+        if (len < 1 || len > kHuffMaxLen || (k && key <= prev_key)) return EQ_ERR_CORRUPT;
+        prev_key = key;
+        kraft += 1u << (kHuffMaxLen - len);
+    }
+    if (n_present > 1 && kraft != (1u << kHuffMaxLen)) return EQ_ERR_CORRUPT;
+    *n_words_out = n_words;
+    return EQ_OK;
+}
+
 int parse(const uint8_t *b, size_t len, eq_model *m) {
     if (len < kHeaderBytes || std::memcmp(b, "EQW1", 4) != 0) return EQ_ERR_CORRUPT;
     if (rd<uint32_t>(b + 4) != kVersion) return EQ_ERR_UNSUPPORTED;
@@ -91,6 +121,9 @@ int parse(const uint8_t *b, size_t len, eq_model *m) {
         d.chunk_index_off = rd<uint64_t>(e + 32);
         d.scales_off = rd<uint64_t>(e + 40);
         d.outliers_off = rd<uint64_t>(e + 48);
+        d.codec = rd<uint32_t>(e + 28);
+        in.codec = d.codec;
+        if (d.codec != kCodecRans && d.codec != kCodecHuffman) return EQ_ERR_UNSUPPORTED;
         if (in.dtype != EQ_INT8 && in.dtype != EQ_E4M3) return EQ_ERR_CORRUPT;
         if (in.layer >= n_layers || in.layer < prev_layer) return EQ_ERR_CORRUPT;
         if (in.layer != prev_layer || i == 0) next_index = 0;
@@ -126,7 +159,8 @@ int parse(const uint8_t *b, size_t len, eq_model *m) {
             const uint64_t rem = n - (uint64_t)k * kChunkSyms;
             const uint32_t n_expect = (uint32_t)(rem < kChunkSyms ? rem : kChunkSyms);
             uint64_t nw = 0;
-            int rc = check_record(b, off, end, n_expect, &nw);
+            int rc = d.codec == kCodecHuffman ? check_huffman_record(b, off, end, n_expect, &nw)
+                                              : check_record(b, off, end, n_expect, &nw);
             if (rc) return rc;
             words += nw;
             // does every chunk carry the first chunk's table?
@@ -135,7 +169,8 @@ int parse(const uint8_t *b, size_t len, eq_model *m) {
                 np0 = np;
             } else if (in.uniform_table) {
                 const uint64_t off0 = rd<uint64_t>(b + d.chunk_index_off);
-                if (np != np0 || std::memcmp(b + off + kRecordHeadBytes, b + off0 + kRecordHeadBytes, 4ull * np) != 0)
+                const uint32_t hb = record_head_bytes(d.codec);
+                if (np != np0 || std::memcmp(b + off + hb, b + off0 + hb, 4ull * np) != 0)
                     in.uniform_table = 0;
             }
         }

@@ -123,6 +123,21 @@ typedef struct eq_matrix_in {
  */
 #define EQ_TABLE_PER_CHUNK 1u
 
+/*
+ * Codec (eq_matrix_in.flags; directory entry word 7 = 0 rANS, 1 Huffman).
+ * Default rANS.  EQ_CODEC_HUFFMAN codes the matrix with canonical Huffman
+ * codes of at most 12 bits (EntroLLM technical overview, "Huffman weight
+ * encoding"), on the same chunk and lane layout: a lane's bit stream is its
+ * symbols' codes in step order, most significant bit first; before decoding a
+ * symbol a lane holding fewer than 12 unread bits takes the next 16-bit word
+ * (words ordered by step, then lane); a chunk with one distinct symbol has
+ * the empty code.  Huffman chunk record: u32 n_syms, n_words, n_present, 0;
+ * u32 table[n_present] = symbol | length << 16 sorted by (length, symbol);
+ * padding to 16 B; u16 words; padding to 16 B (no states).  Host encoder
+ * only (eq_encode_device returns EQ_ERR_UNSUPPORTED).
+ */
+#define EQ_CODEC_HUFFMAN 2u
+
 typedef struct eq_encoded eq_encoded;  /* host-side result of eq_encoder_run */
 
 /*
@@ -193,6 +208,8 @@ typedef struct eq_model eq_model;
 typedef struct eq_matrix_info {
     uint32_t layer, index, dtype, rows, cols, n_chunks, n_outliers;
     uint32_t uniform_table;     /* 1 if every chunk carries the same frequency table */
+    uint32_t codec;             /* 0 rANS, 1 Huffman */
+    uint32_t reserved;
     uint64_t compressed_bytes;  /* bytes of its chunk records (tables, states, words) */
     uint64_t payload_words;     /* total 16-bit renormalisation words */
 } eq_matrix_info;

@@ -229,3 +229,96 @@ def test_matrix_table_costs_little(eqw):
     a = eqw.encode_host([m], table_scope="matrix").size
     b = eqw.encode_host([m], table_scope="chunk").size
     assert a <= b * 1.005
+
+
+# ---- Huffman codec (EntroLLM technical overview, "Huffman weight encoding") ----
+
+def _ragged_consistent(seed=0):
+    mats = [
+        W.random_int8_matrix(seed + 1, 300, 229, layer=0, index=0),
+        W.random_int8_matrix(seed + 2, 1, 1, layer=0, index=1),
+        W.random_e4m3_matrix(seed + 3, 77, 1000, alpha=1.0, layer=0, index=2),
+        W.random_int8_matrix(seed + 4, 512, 256, n_out=16, layer=1, index=0),
+        W.random_int8_matrix(seed + 5, 0, 64, layer=1, index=1),
+        W.random_int8_matrix(seed + 6, 700, 1300, h_bits=3.0, n_out=5, layer=1, index=2),
+    ]
+    single = W.random_int8_matrix(seed + 7, 64, 1100, layer=1, index=3)
+    single.symbols[:] = 0x03
+    mats.append(single)
+    return mats
+
+
+@pytest.mark.parametrize("scope", ["matrix", "chunk"])
+def test_product_huffman_encoder_decodes_with_oracle(eqw, orc, scope):
+    mats = _ragged_consistent(100)
+    blob = eqw.encode_host(mats, table_scope=scope, codec="huffman")
+    for m, got in zip(mats, orc.decode_container(blob)):
+        assert np.array_equal(got, orc.dequant_direct(m))
+    rc, h = _open(eqw, blob)
+    assert rc == 0
+    info = eqw.eq_matrix_info()
+    assert eqw.load().eq_matrix_get_info(h, 0, ctypes.byref(info)) == 0 and info.codec == 1
+    eqw.load().eq_model_close(h)
+
+
+def test_parser_accepts_oracle_huffman_containers(eqw, orc):
+    blob = orc.encode_container(_ragged_consistent(200), codec="huffman")
+    rc, h = _open(eqw, blob)
+    assert rc == 0
+    eqw.load().eq_model_close(h)
+
+
+def test_mixed_codecs_in_one_container(eqw, orc):
+    mats = _ragged_consistent(300)
+    for i, m in enumerate(mats):
+        m.codec = "huffman" if i % 2 else "rans"
+    blob = eqw.encode_host(mats)
+    parsed = orc.parse_container(blob)
+    assert [pm["codec"] for pm in parsed["matrices"]] == [i % 2 for i in range(len(mats))]
+    for m, got in zip(mats, orc.decode_container(blob)):
+        assert np.array_equal(got, orc.dequant_direct(m))
+
+
+@pytest.mark.parametrize("what", ["kraft", "order", "long_code", "single_with_words", "codec"])
+def test_parser_rejects_huffman_corruption(eqw, orc, what):
+    m = W.random_int8_matrix(400, 256, 600)
+    blob = eqw.encode_host([m], codec="huffman").copy()
+    off0 = int(orc.parse_container(blob)["matrices"][0]["chunk_offsets"][0])
+    t0 = off0 + 16
+    if what == "kraft":
+        blob[t0 + 2] += 1  # first (shortest) code one bit longer: Kraft sum < 1
+    elif what == "order":
+        a, b = bytes(blob[t0:t0 + 4]), bytes(blob[t0 + 4:t0 + 8])
+        blob[t0:t0 + 4] = np.frombuffer(b, np.uint8)
+        blob[t0 + 4:t0 + 8] = np.frombuffer(a, np.uint8)
+    elif what == "long_code":
+        npres = int(np.frombuffer(bytes(blob[off0 + 8:off0 + 12]), "<u4")[0])
+        blob[t0 + 4 * (npres - 1) + 2] = 13
+    elif what == "single_with_words":
+        s = W.random_int8_matrix(401, 64, 64)
+        s.symbols[:] = 1
+        blob = eqw.encode_host([s], codec="huffman").copy()
+        o = int(orc.parse_container(blob)["matrices"][0]["chunk_offsets"][0])
+        blob[o + 4] = 1  # claims a word it does not have
+    elif what == "codec":
+        blob[64 + 28] = 7
+    rc, _ = _open(eqw, blob)
+    assert rc in (2, 3)
+
+
+def test_huffman_size_near_entropy(eqw, orc):
+    """Huffman payload within one bit per symbol of the per-chunk Shannon bound
+    (integer code lengths) and never below it."""
+    m = W.random_int8_matrix(402, 1024, 1024, h_bits=2.1)
+    blob = eqw.encode_host([m], codec="huffman", table_scope="chunk")
+    pm = orc.parse_container(blob)["matrices"][0]
+    flat = m.symbols.reshape(-1)
+    payload, shannon = 0, 0.0
+    for k in range(pm["n_chunks"]):
+        off = int(pm["chunk_offsets"][k])
+        n_k, nw = struct.unpack("<2I", bytes(blob[off:off + 8]))
+        payload += 2 * nw
+        c = np.bincount(flat[k * 65536:k * 65536 + n_k], minlength=256).astype(np.float64)
+        p = c[c > 0] / n_k
+        shannon += n_k * float(-(p * np.log2(p)).sum()) / 8
+    assert shannon <= payload <= shannon + flat.size / 8
