@@ -432,6 +432,28 @@ def bench_eqw(args, d: Dist) -> dict | None:
     ms_b_max, _ = combine(ms_b, 0.0, d)
     value_b = dec_bytes_all / (ms_b_max / 1e3) / 1e9
 
+    # ---- D: the Huffman codec on layer 0 (host-encoded), one block decode at a time ----
+    huff = None
+    if d.rank == 0:
+        import entropy_coded_weight_b200 as E
+        layer0 = W.llama70b_int8_layer(0, 2.1, threads=threads)
+        hblob = E.encode_host(layer0, n_threads=threads, codec="huffman")
+        n0 = sum(m.n for m in layer0)
+        del layer0
+        hstack = ResidentStack(hblob, 1, dev, 12)
+        hb = hstack.layer_bytes(hstack.steps[0])
+        per_h = isolated_launches(hstack, 36, dev)
+        h_ms = statistics.mean(per_h[len(per_h) // 4:])
+        rstep = stack.steps[0]
+        r_read = stack.layer_bytes(rstep)["read"]
+        huff = {"value": round(2.0 * n0 / (h_ms / 1e3) / 1e9, 2), "unit": UNIT, "launch_ms": round(h_ms, 4),
+                "bits_per_sym": round(8.0 * hb["read"] / n0, 4), "rans_bits_per_sym": round(8.0 * r_read / n0, 4),
+                "rans_launch_ms": round(launch_ms, 4),
+                "note": "layer 0 Huffman-coded (canonical codes <= 12 bits) and decoded by eq_decode_kernel's "
+                        "Huffman instance, launches timed alone; bits/sym incl. tables and chunk index"}
+        hstack.close()
+        del hblob
+
     # ---- C: fused decode + GEMV, no bf16 buffers; blocks in sequence on one stream ----
     fstream = torch.cuda.Stream(device=dev)
     fys = [torch.empty_like(y) for y in ys]
@@ -517,6 +539,7 @@ def bench_eqw(args, d: Dist) -> dict | None:
                             "kernel": "eq_decode_gemv_kernel",
                             "note": "y = W x per matrix with W decoded in registers; value = bf16 weight bytes "
                                     "consumed per second (2 x symbols / time), one block after another"},
+        "huffman": huff,
         "e2e": {"value": round(value_e, 2), "unit": UNIT, "h2d_bytes_per_step": int(blob.size * stack.copies),
                 "d2h_bytes_per_step": 4, "ms_per_step": round(ms_e_max / args.steps, 3)},
         "cpu_baseline": cpu,

@@ -178,16 +178,16 @@ __device__ __forceinline__ void group_store(const OutCtx &O, uint16_t *dst, uint
 
 // One 256-symbol group in a row-uniform layout: 8 steps, dequantised in pairs
 // as they are decoded (4 packed registers), one 16-byte store.
-template <int DT>
-__device__ __forceinline__ void group_row(uint32_t lut, uint32_t ring, uint32_t &pw, uint32_t &x, uint32_t lt,
+template <int DT, uint32_t CODEC>
+__device__ __forceinline__ void group_row(uint32_t lut, uint32_t ring, uint32_t &pw, CodecState<CODEC> &x, uint32_t lt,
                                           float2 s2, bool small_scales, uint16_t *dst) {
     const uint32_t rp0 = ring + (pw & (kRingBytes - 1));
     uint32_t rp = rp0;
     uint32_t o[4];
 #pragma unroll
     for (int r = 0; r < 8; r += 2) {
-        const uint32_t e0 = rans_step(lut, rp, x, lt);
-        const uint32_t e1 = rans_step(lut, rp, x, lt);
+        const uint32_t e0 = codec_step<CODEC>(lut, rp, x, lt);
+        const uint32_t e1 = codec_step<CODEC>(lut, rp, x, lt);
         float2 v = make_float2(raw_value<DT>(e0), raw_value<DT>(e1));
         if constexpr (DT == EQ_E4M3) {
             if (!small_scales) v = mul2(v, make_float2(0x1p120f, 0x1p120f));
@@ -199,15 +199,16 @@ __device__ __forceinline__ void group_row(uint32_t lut, uint32_t ring, uint32_t 
 }
 
 // One 256-symbol group in rank mode: 8 steps, 8 shuffles, one 16-byte store.
-__device__ __forceinline__ void group_rank(uint32_t lut, uint32_t ring, uint32_t &pw, uint32_t &x, uint32_t lt,
+template <uint32_t CODEC>
+__device__ __forceinline__ void group_rank(uint32_t lut, uint32_t ring, uint32_t &pw, CodecState<CODEC> &x, uint32_t lt,
                                            float vr, uint16_t *dst) {
     const uint32_t rp0 = ring + (pw & (kRingBytes - 1));
     uint32_t rp = rp0;
     uint32_t o[4];
 #pragma unroll
     for (int r = 0; r < 8; r += 2) {
-        const uint32_t e0 = rans_step(lut, rp, x, lt);
-        const uint32_t e1 = rans_step(lut, rp, x, lt);
+        const uint32_t e0 = codec_step<CODEC>(lut, rp, x, lt);
+        const uint32_t e1 = codec_step<CODEC>(lut, rp, x, lt);
         o[r / 2] = pack_bf16x2(make_float2(__shfl_sync(kFull, vr, e0), __shfl_sync(kFull, vr, e1)));
     }
     st_global_v4(dst, make_uint4(o[0], o[1], o[2], o[3]));
@@ -219,14 +220,17 @@ __device__ __forceinline__ void group_rank(uint32_t lut, uint32_t ring, uint32_t
 // followed by the same step of chunk B, giving each warp two independent
 // state chains whose latencies overlap.  Row changes fall on 512-symbol
 // boundaries, i.e. between pairs of groups.
+template <uint32_t CODEC>
 struct Chain {
-    uint32_t x, pw, limit, row, col;
+    CodecState<CODEC> x;
+    uint32_t pw, limit, row, col;
     float vr;
     uint16_t *dst;
 };
 
 // Two 256-symbol groups in rank mode, one per chain, interleaved step by step.
-__device__ __forceinline__ void group2_rank(uint32_t lut, uint32_t ringA, uint32_t ringB, Chain &A, Chain &B,
+template <uint32_t CODEC>
+__device__ __forceinline__ void group2_rank(uint32_t lut, uint32_t ringA, uint32_t ringB, Chain<CODEC> &A, Chain<CODEC> &B,
                                             uint32_t lt) {
     const uint32_t a0 = ringA + (A.pw & (kRingBytes - 1));
     const uint32_t b0 = ringB + (B.pw & (kRingBytes - 1));
@@ -234,10 +238,10 @@ __device__ __forceinline__ void group2_rank(uint32_t lut, uint32_t ringA, uint32
     uint32_t oa[4], ob[4];
 #pragma unroll
     for (int r = 0; r < 8; r += 2) {
-        const uint32_t ea0 = rans_step(lut, ra, A.x, lt);
-        const uint32_t eb0 = rans_step(lut, rb, B.x, lt);
-        const uint32_t ea1 = rans_step(lut, ra, A.x, lt);
-        const uint32_t eb1 = rans_step(lut, rb, B.x, lt);
+        const uint32_t ea0 = codec_step<CODEC>(lut, ra, A.x, lt);
+        const uint32_t eb0 = codec_step<CODEC>(lut, rb, B.x, lt);
+        const uint32_t ea1 = codec_step<CODEC>(lut, ra, A.x, lt);
+        const uint32_t eb1 = codec_step<CODEC>(lut, rb, B.x, lt);
         oa[r / 2] = pack_bf16x2(make_float2(__shfl_sync(kFull, A.vr, ea0), __shfl_sync(kFull, A.vr, ea1)));
         ob[r / 2] = pack_bf16x2(make_float2(__shfl_sync(kFull, B.vr, eb0), __shfl_sync(kFull, B.vr, eb1)));
     }
@@ -249,7 +253,7 @@ __device__ __forceinline__ void group2_rank(uint32_t lut, uint32_t ringA, uint32
     B.dst += kGroupSyms;
 }
 
-template <int DT>
+template <int DT, uint32_t CODEC>
 __device__ __forceinline__ bool decode_pair(int32_t *status, const OutCtx &O, const ChunkHead &hA,
                                             const ChunkHead &hB, uint64_t firstA, uint64_t firstB, uint32_t lut,
                                             uint32_t ringA, uint32_t ringB, uint32_t mbarA, uint32_t mbarB,
@@ -259,9 +263,9 @@ __device__ __forceinline__ bool decode_pair(int32_t *status, const OutCtx &O, co
     ring_start(ctlB, hB);
     __syncwarp();
     const float vraw = symbol_value<DT>(lane_sym);
-    Chain A, B;
-    A.x = hA.x;
-    B.x = hB.x;
+    Chain<CODEC> A, B;
+    A.x = codec_start<CODEC>(hA.x);
+    B.x = codec_start<CODEC>(hB.x);
     A.pw = B.pw = 0;
     A.limit = hA.n_words ? 0u : kNoLimit;
     B.limit = hB.n_words ? 0u : kNoLimit;
@@ -299,18 +303,18 @@ __device__ __forceinline__ bool decode_pair(int32_t *status, const OutCtx &O, co
         flag(status, EQ_DEV_TIMEOUT);
         return false;
     }
-    if (!__all_sync(kFull, A.x == kStateLow) || A.pw != 2u * hA.n_words) flag(status, EQ_DEV_BAD_END);
-    if (!__all_sync(kFull, B.x == kStateLow) || B.pw != 2u * hB.n_words) flag(status, EQ_DEV_BAD_END);
+    if (!__all_sync(kFull, codec_done(A.x)) || A.pw != 2u * hA.n_words) flag(status, EQ_DEV_BAD_END);
+    if (!__all_sync(kFull, codec_done(B.x)) || B.pw != 2u * hB.n_words) flag(status, EQ_DEV_BAD_END);
     return true;
 }
 
 // Decode one chunk whose slot table is ready at `lut` (n_present >= 2) or
 // whose single symbol's stored byte is `single` (n_present == 1).  Returns
 // false if a bounded wait gave up (the warp must stop).
-template <int DT, uint32_t LAYOUT>
+template <int DT, uint32_t LAYOUT, uint32_t CODEC>
 __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, uint64_t first,
                                             uint32_t n, uint32_t n_words, const uint8_t *payload, bool single_sym,
-                                            uint32_t single, uint32_t x, uint32_t lut, uint32_t ring, uint32_t mbar,
+                                            uint32_t single, uint32_t x0, uint32_t lut, uint32_t ring, uint32_t mbar,
                                             RingCtl *ctl, uint32_t lane, uint32_t lt, bool by_rank,
                                             uint32_t lane_sym) {
     const uint32_t n_full = n / kGroupSyms;
@@ -321,7 +325,7 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, ui
 
     if (single_sym) {
         // f = 4096: the states never change and there are no words
-        if (n_words != 0 || !__all_sync(kFull, x == kStateLow)) {
+        if (n_words != 0 || !__all_sync(kFull, CODEC == kCodecHuffman || x0 == kStateLow)) {
             flag(status, EQ_DEV_BAD_END);
             return true;
         }
@@ -348,6 +352,7 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, ui
     __syncwarp();
     uint32_t limit = pbytes ? 0u : kNoLimit;
     uint32_t pw = 0;
+    CodecState<CODEC> x = codec_start<CODEC>(x0);
     bool tail_done = false;
     if constexpr (LAYOUT == kRowUniform) {
       if (by_rank) {
@@ -389,7 +394,7 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, ui
             if (pw >= limit) limit = ring_service(ctl, ring, mbar, pw);
             if (!ctl->dead) {
                 uint32_t e8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-                rans_tail(lut, ring, x, pw, lt, lane, tail, e8);
+                codec_tail<CODEC>(lut, ring, x, pw, lt, lane, tail, e8);
                 const float vr = __fmul_rn(vraw, __ldg(O.scales + cur.row));
                 const uint32_t mine = tail > kGroup * lane ? min(8u, tail - kGroup * lane) : 0u;
                 const uint64_t idx = first + (uint64_t)n_full * kGroupSyms + kGroup * lane;
@@ -413,13 +418,13 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, ui
                     limit = ring_service(ctl, ring, mbar, pw);
                     if (ctl->dead) break;
                 }
-                group_row<DT>(lut, ring, pw, x, lt, s2, O.small_scales, dst);
-                group_row<DT>(lut, ring, pw, x, lt, s2, O.small_scales, dst + kGroupSyms);
+                group_row<DT, CODEC>(lut, ring, pw, x, lt, s2, O.small_scales, dst);
+                group_row<DT, CODEC>(lut, ring, pw, x, lt, s2, O.small_scales, dst + kGroupSyms);
             }
             if (i < run && !ctl->dead) {
                 if (pw >= limit) limit = ring_service(ctl, ring, mbar, pw);
                 if (!ctl->dead) {
-                    group_row<DT>(lut, ring, pw, x, lt, s2, O.small_scales, dst);
+                    group_row<DT, CODEC>(lut, ring, pw, x, lt, s2, O.small_scales, dst);
                     dst += kGroupSyms;
                 }
             }
@@ -443,7 +448,7 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, ui
         if constexpr (LAYOUT == kGeneric) {
             uint32_t e8[8];
 #pragma unroll
-            for (int r = 0; r < 8; ++r) e8[r] = rans_step(lut, rp, x, lt);
+            for (int r = 0; r < 8; ++r) e8[r] = codec_step<CODEC>(lut, rp, x, lt);
             store_elems<DT>(O, first + (uint64_t)g * kGroupSyms + kGroup * lane, 8, e8);
         } else {
             // dequantise pairs as they are decoded: 4 packed registers instead of 8 entries
@@ -451,8 +456,8 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, ui
             uint32_t o[4];
 #pragma unroll
             for (int r = 0; r < 8; r += 2) {
-                const uint32_t e0 = rans_step(lut, rp, x, lt);
-                const uint32_t e1 = rans_step(lut, rp, x, lt);
+                const uint32_t e0 = codec_step<CODEC>(lut, rp, x, lt);
+                const uint32_t e1 = codec_step<CODEC>(lut, rp, x, lt);
                 float2 v = make_float2(raw_value<DT>(e0), raw_value<DT>(e1));
                 if constexpr (DT == EQ_E4M3) {
                     if (!O.small_scales) v = mul2(v, make_float2(0x1p120f, 0x1p120f));
@@ -469,7 +474,7 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, ui
         if (pw >= limit) limit = ring_service(ctl, ring, mbar, pw);
         if (!ctl->dead) {
             uint32_t e8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            rans_tail(lut, ring, x, pw, lt, lane, tail, e8);
+            codec_tail<CODEC>(lut, ring, x, pw, lt, lane, tail, e8);
             const uint32_t mine = tail > kGroup * lane ? min(8u, tail - kGroup * lane) : 0u;
             store_elems<DT>(O, first + (uint64_t)n_full * kGroupSyms + kGroup * lane, mine, e8);
         }
@@ -479,11 +484,11 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, ui
         return false;
     }
     // a valid stream returns every state to 2^16 and consumes exactly n_words
-    if (!__all_sync(kFull, x == kStateLow) || pw != 2u * n_words) flag(status, EQ_DEV_BAD_END);
+    if (!__all_sync(kFull, codec_done(x)) || pw != 2u * n_words) flag(status, EQ_DEV_BAD_END);
     return true;
 }
 
-template <int WARPS, bool SHARED, int DT, uint32_t LAYOUT>
+template <int WARPS, bool SHARED, int DT, uint32_t LAYOUT, uint32_t CODEC>
 __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
     eq_decode_kernel(const __grid_constant__ DecodeParams P) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -501,7 +506,7 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
             const MatJob &M = P.mats[mi];
             const uint32_t k0 = (unit - M.begin) * WARPS * C;
             if (mi != cur_mat) {
-                shared_table_rebuild<WARPS, LAYOUT>(P, M, k0, lane, warp, S);
+                shared_table_rebuild<WARPS, LAYOUT, CODEC>(P, M, k0, lane, warp, S);
                 cur_mat = mi;
             }
             const uint32_t np = S.blk[0];
@@ -512,13 +517,13 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
             for (uint32_t c = 0; c < C; ++c) {
                 const uint32_t k = k0 + warp + c * WARPS;
                 have[c] = k < M.n_chunks && !ctl[0].dead && !ctl[C - 1].dead;
-                if (have[c]) have[c] = shared_chunk_head(P, M, k, lane, np, S, hc[c]);
+                if (have[c]) have[c] = shared_chunk_head<CODEC>(P, M, k, lane, np, S, hc[c]);
             }
             const OutCtx O = out_ctx(M);
             if constexpr (C == 2 && LAYOUT == kRowUniform) {
                 if (have[0] && have[1] && rank_mode<LAYOUT>(np) && hc[0].n == kChunkSyms &&
                     hc[1].n == kChunkSyms && O.cols % (2 * kGroupSyms) == 0) {
-                    decode_pair<DT>(P.status, O, hc[0], hc[1], (uint64_t)(k0 + warp) * kChunkSyms,
+                    decode_pair<DT, CODEC>(P.status, O, hc[0], hc[1], (uint64_t)(k0 + warp) * kChunkSyms,
                                     (uint64_t)(k0 + warp + WARPS) * kChunkSyms, S.lut_addr, S.ring,
                                     S.ring + kRingStride, S.mbar, S.mbar + 8 * kRingSegs, ctl, ctl + 1, lane, lt,
                                     lane_sym);
@@ -528,7 +533,7 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
             }
             for (uint32_t c = 0; c < C; ++c) {
                 if (!have[c] || ctl->dead) continue;
-                decode_body<DT, LAYOUT>(P.status, O, (uint64_t)(k0 + warp + c * WARPS) * kChunkSyms, hc[c].n,
+                decode_body<DT, LAYOUT, CODEC>(P.status, O, (uint64_t)(k0 + warp + c * WARPS) * kChunkSyms, hc[c].n,
                                         hc[c].n_words, hc[c].rec + hc[c].table_bytes, np == 1,
                                         S.ref_entries[0] & 0xFFu, hc[c].x, S.lut_addr, S.ring, S.mbar, ctl, lane,
                                         lt, rank_mode<LAYOUT>(np), lane_sym);
@@ -541,17 +546,17 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
             const MatJob &M = P.mats[job_of(P, c)];
             const uint32_t k = c - M.begin;
             ChunkHead h;
-            if (!load_head(P, M, k, lane, h)) continue;
-            const uint32_t *tab = reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes);
+            if (!load_head<CODEC>(P, M, k, lane, h)) continue;
+            const uint32_t *tab = reinterpret_cast<const uint32_t *>(h.rec + kHeadBytes<CODEC>);
             __syncwarp();  // the previous chunk's reads of the slot table are done
             const bool by_rank = rank_mode<LAYOUT>(h.n_present);
-            const bool ok = warp_table(tab, h.n_present, lane, nullptr, nullptr, S.lut, by_rank);
+            const bool ok = warp_table<CODEC>(tab, h.n_present, lane, nullptr, nullptr, S.lut, by_rank);
             if (!ok) {
                 flag(P.status, EQ_DEV_BAD_TABLE);
                 continue;
             }
             __syncwarp();
-            decode_body<DT, LAYOUT>(P.status, out_ctx(M), (uint64_t)k * kChunkSyms, h.n, h.n_words,
+            decode_body<DT, LAYOUT, CODEC>(P.status, out_ctx(M), (uint64_t)k * kChunkSyms, h.n, h.n_words,
                                     h.rec + h.table_bytes, h.n_present == 1, tab[0] & 0xFFu, h.x,
                                     S.lut_addr, S.ring, S.mbar, ctl, lane, lt, by_rank,
                                     tab[lane < h.n_present ? lane : 0] & 0xFFu);
@@ -602,22 +607,28 @@ __global__ void eq_wait_timeout_kernel(int32_t *status) {
 
 // ---- host side ---------------------------------------------------------------------
 
-// variants: [shared][dtype - 1][layout]
+// variants: [codec][shared][dtype - 1][layout]
 struct DeviceSetup {
     bool ready = false;
     int sms = 0;
-    KernelSetup<DecodeParams> k[2][2][3];
+    KernelSetup<DecodeParams> k[2][2][2][3];
 };
 std::mutex g_setup_mu;
 DeviceSetup g_setup[128];
 
+template <int DT, uint32_t LAYOUT, uint32_t CODEC>
+int setup_variant(DeviceSetup &d) {
+    int rc = setup_kernel(d.k[CODEC][1][DT - 1][LAYOUT], eq_decode_kernel<kSharedWarps, true, DT, LAYOUT, CODEC>,
+                          kSharedWarps, Smem<kSharedWarps, true>::kBytes, 1);
+    if (rc) return rc;
+    return setup_kernel(d.k[CODEC][0][DT - 1][LAYOUT], eq_decode_kernel<kPrivateWarps, false, DT, LAYOUT, CODEC>,
+                        kPrivateWarps, Smem<kPrivateWarps, false>::kBytes, kPrivateWarps);
+}
+
 template <int DT, uint32_t LAYOUT>
 int setup_pair(DeviceSetup &d) {
-    int rc = setup_kernel(d.k[1][DT - 1][LAYOUT], eq_decode_kernel<kSharedWarps, true, DT, LAYOUT>, kSharedWarps,
-                          Smem<kSharedWarps, true>::kBytes, 1);
-    if (rc) return rc;
-    return setup_kernel(d.k[0][DT - 1][LAYOUT], eq_decode_kernel<kPrivateWarps, false, DT, LAYOUT>, kPrivateWarps,
-                        Smem<kPrivateWarps, false>::kBytes, kPrivateWarps);
+    int rc = setup_variant<DT, LAYOUT, kCodecRans>(d);
+    return rc ? rc : setup_variant<DT, LAYOUT, kCodecHuffman>(d);
 }
 
 int device_setup(DeviceSetup **out) {
@@ -646,7 +657,7 @@ uint32_t layout_of(const eq_matrix_info &in, const uint16_t *out) {
 }
 
 // Decode matrices [first, first + count) of the model into outs[i]: one
-// launch per kernel variant (table scope x dtype x layout) present, then one
+// launch per kernel variant (codec x table scope x dtype x layout) present, then one
 // scatter launch for the super weights.
 int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *const *outs, int32_t *d_status,
                   cudaStream_t s) {
@@ -655,15 +666,16 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
     if (rc) return rc;
     for (uint32_t base = 0; base < count; base += kMaxMatsPerLaunch) {
         const uint32_t cnt = std::min<uint32_t>(kMaxMatsPerLaunch, count - base);
-        DecodeParams P[2][2][3];
+        DecodeParams P[2][2][2][3];
         for (auto &a : P)
             for (auto &b : a)
-                for (auto &c : b) {
-                    c = DecodeParams{};
-                    c.blob = m->d_blob;
-                    c.blob_len = m->len;
-                    c.status = d_status;
-                }
+                for (auto &c : b)
+                    for (auto &v : c) {
+                        v = DecodeParams{};
+                        v.blob = m->d_blob;
+                        v.blob_len = m->len;
+                        v.status = d_status;
+                    }
         ScatterParams Q{};
         Q.status = d_status;
         uint32_t n_out = 0;
@@ -672,7 +684,7 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
             if (d.info.n_chunks == 0) continue;
             const int sh = d.info.uniform_table ? 1 : 0;
             const uint32_t lay = layout_of(d.info, outs[base + i]);
-            DecodeParams &Pv = P[sh][d.info.dtype - 1][lay];
+            DecodeParams &Pv = P[d.codec][sh][d.info.dtype - 1][lay];
             MatJob &J = Pv.mats[Pv.n_mats++];
             J.chunk_index = reinterpret_cast<const uint64_t *>(m->d_blob + d.chunk_index_off);
             J.scales = reinterpret_cast<const float *>(m->d_blob + d.scales_off);
@@ -698,10 +710,11 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
             }
         }
         Q.total = n_out;
-        for (int sh = 0; sh < 2; ++sh)
-            for (int dt = 0; dt < 2; ++dt)
-                for (int lay = 0; lay < 3; ++lay)
-                    if ((rc = launch(dev->k[sh][dt][lay], dev->sms, P[sh][dt][lay], s))) return rc;
+        for (int co = 0; co < 2; ++co)
+            for (int sh = 0; sh < 2; ++sh)
+                for (int dt = 0; dt < 2; ++dt)
+                    for (int lay = 0; lay < 3; ++lay)
+                        if ((rc = launch(dev->k[co][sh][dt][lay], dev->sms, P[co][sh][dt][lay], s))) return rc;
         if (n_out) {
             eq_outlier_scatter_kernel<<<(n_out + 127) / 128, 128, 0, s>>>(Q);
             if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;

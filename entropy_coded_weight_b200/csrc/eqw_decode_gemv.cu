@@ -495,7 +495,7 @@ int check_gemv_args(const eq_model *m, uint32_t first, uint32_t count, const voi
         if (reinterpret_cast<uintptr_t>(ys[i]) % 4) return EQ_ERR_INVALID_ARG;
         if (in.rows && in.cols) {
             if (!xs[i] || reinterpret_cast<uintptr_t>(xs[i]) % 16) return EQ_ERR_INVALID_ARG;
-            if (in.cols % kGroupSyms) return EQ_ERR_UNSUPPORTED;
+            if (in.cols % kGroupSyms || m->mats[first + i].codec != kCodecRans) return EQ_ERR_UNSUPPORTED;
         }
     }
     return EQ_OK;

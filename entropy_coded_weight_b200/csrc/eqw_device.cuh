@@ -335,6 +335,91 @@ __device__ __forceinline__ void rans_tail(uint32_t lut, uint32_t ring, uint32_t 
     }
 }
 
+// ---- the Huffman step (codec 1) --------------------------------------------------
+// Each lane holds its unread bits left-aligned in `buf` (nb of them).  A lane
+// with fewer than 12 takes the next word (positions by ballot + popcount, as
+// for rANS) into the bits just below its held ones; then the top 12 bits
+// index the slot table, whose entry gives the code length (bits 8..11) and
+// the symbol or its rank (low byte), and the code's bits are shifted out.
+__device__ __forceinline__ uint32_t shl_clamped(uint32_t v, uint32_t n) {  // v << n, 0 for n >= 32
+    uint32_t r;
+    asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(n));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t huff_step(uint32_t lut, uint32_t &rp, uint32_t &buf, uint32_t &nb,
+                                              uint32_t lt) {
+    const bool need = nb < kHuffMaxLen;
+    const uint32_t b = __ballot_sync(kFull, need);
+    const uint32_t w = lds_u16(mad_lo(__popc(b & lt), 2u, rp));
+    const uint32_t filled = buf | shl_clamped(w, 16u - nb);
+    buf = need ? filled : buf;
+    nb = need ? nb + 16u : nb;
+    rp = mad_lo(__popc(b), 2u, rp);
+    const uint32_t e = lds_u32(lut + 4u * (buf >> (32u - kHuffMaxLen)));
+    const uint32_t len = e >> 8;
+    buf = shl_clamped(buf, len);
+    nb -= len;
+    return e;
+}
+
+// Last, partial group (lane l active at step r while 8l + r < rem).
+__device__ __forceinline__ void huff_tail(uint32_t lut, uint32_t ring, uint32_t &buf, uint32_t &nb, uint32_t &pw,
+                                          uint32_t lt, uint32_t lane, uint32_t rem, uint32_t (&e8)[8]) {
+#pragma unroll
+    for (uint32_t r = 0; r < 8; ++r) {
+        const bool active = lane * kGroup + r < rem;
+        const bool need = active && nb < kHuffMaxLen;
+        const uint32_t b = __ballot_sync(kFull, need);
+        const uint32_t w = lds_u16(ring + ((pw + 2u * __popc(b & lt)) & (kRingBytes - 1)));
+        if (need) {
+            buf |= w << (16u - nb);
+            nb += 16u;
+        }
+        pw += 2u * __popc(b);
+        if (active) {
+            const uint32_t e = lds_u32(lut + 4u * (buf >> (32u - kHuffMaxLen)));
+            const uint32_t len = e >> 8;
+            buf = shl_clamped(buf, len);
+            nb -= len;
+            e8[r] = e;
+        }
+    }
+}
+
+// Per-lane decoder state of a codec, its step, tail, start and end checks.
+template <uint32_t CODEC> struct CodecState;
+template <> struct CodecState<kCodecRans> { uint32_t x; };
+template <> struct CodecState<kCodecHuffman> { uint32_t buf, nb; };
+
+template <uint32_t CODEC>
+__device__ __forceinline__ uint32_t codec_step(uint32_t lut, uint32_t &rp, CodecState<CODEC> &s, uint32_t lt) {
+    if constexpr (CODEC == kCodecHuffman) return huff_step(lut, rp, s.buf, s.nb, lt);
+    else return rans_step(lut, rp, s.x, lt);
+}
+
+template <uint32_t CODEC>
+__device__ __forceinline__ void codec_tail(uint32_t lut, uint32_t ring, CodecState<CODEC> &s, uint32_t &pw,
+                                           uint32_t lt, uint32_t lane, uint32_t rem, uint32_t (&e8)[8]) {
+    if constexpr (CODEC == kCodecHuffman) huff_tail(lut, ring, s.buf, s.nb, pw, lt, lane, rem, e8);
+    else rans_tail(lut, ring, s.x, pw, lt, lane, rem, e8);
+}
+
+// rANS: the state from the record; Huffman: no bits held.
+template <uint32_t CODEC>
+__device__ __forceinline__ CodecState<CODEC> codec_start(uint32_t x0) {
+    if constexpr (CODEC == kCodecHuffman) return CodecState<CODEC>{0u, 0u};
+    else return CodecState<CODEC>{x0};
+}
+
+// A valid stream ends with every rANS state back at 2^16 / every Huffman bit
+// still held being zero padding.
+template <uint32_t CODEC>
+__device__ __forceinline__ bool codec_done(const CodecState<CODEC> &s) {
+    if constexpr (CODEC == kCodecHuffman) return s.buf == 0;
+    else return s.x == kStateLow;
+}
+
 // Rank mode: with 2..32 distinct symbols and a warp-uniform row per group, the
 // slot table's low byte holds the symbol's rank (index in the ascending
 // frequency list) and lane r keeps fp32_rn(value(symbol of rank r) * row
@@ -381,10 +466,14 @@ __device__ __forceinline__ bool ring_start(RingCtl *ctl, const ChunkHead &h) {
     return true;
 }
 
-// Header of chunk k: checks it against the directory; on success fills the
-// record pointer, counts and this lane's initial state.
+// Bytes before a record's frequency list / code table: counts, plus the 32
+// lane states for rANS (Huffman records carry no states).
+template <uint32_t CODEC>
+constexpr uint32_t kHeadBytes = CODEC == kCodecHuffman ? kHuffRecordHeadBytes : kRecordHeadBytes;
 
-template <class Params, class Job>
+// Header of chunk k: checks it against the directory; on success fills the
+// record pointer, counts and (rANS) this lane's initial state.
+template <uint32_t CODEC = kCodecRans, class Params, class Job>
 __device__ __forceinline__ bool load_head(const Params &P, const Job &M, uint32_t k, uint32_t lane,
                                           ChunkHead &h) {
     const uint64_t first = (uint64_t)k * kChunkSyms;
@@ -392,7 +481,7 @@ __device__ __forceinline__ bool load_head(const Params &P, const Job &M, uint32_
     const uint32_t n_expect = rem < kChunkSyms ? (uint32_t)rem : kChunkSyms;
     const uint64_t off = M.chunk_index[k];
     const uint64_t end = M.chunk_index[k + 1];
-    if ((off & 15) || end > P.blob_len || end < off + kRecordHeadBytes + 16) {
+    if ((off & 15) || end > P.blob_len || end < off + kHeadBytes<CODEC> + 16) {
         flag(P.status, EQ_DEV_BAD_HEADER);
         return false;
     }
@@ -401,38 +490,69 @@ __device__ __forceinline__ bool load_head(const Params &P, const Job &M, uint32_
     h.n = head.x;
     h.n_words = head.y;
     h.n_present = head.z;
-    h.table_bytes = (kRecordHeadBytes + 4 * h.n_present + 15) & ~15u;
+    h.table_bytes = (kHeadBytes<CODEC> + 4 * h.n_present + 15) & ~15u;
     if (h.n != n_expect || h.n_present < 1 || h.n_present > 256 ||
         off + h.table_bytes + ((2ull * h.n_words + 15) & ~15ull) != end) {
         flag(P.status, EQ_DEV_BAD_HEADER);
         return false;
     }
-    h.x = reinterpret_cast<const uint32_t *>(h.rec + 16)[lane];
-    if (!__all_sync(kFull, h.x >= kStateLow)) {
-        flag(P.status, EQ_DEV_BAD_STATE);
-        return false;
+    if constexpr (CODEC == kCodecHuffman) {
+        h.x = 0;
+    } else {
+        h.x = reinterpret_cast<const uint32_t *>(h.rec + 16)[lane];
+        if (!__all_sync(kFull, h.x >= kStateLow)) {
+            flag(P.status, EQ_DEV_BAD_STATE);
+            return false;
+        }
     }
     return true;
 }
 
-// Check a frequency list (n_present entries at `tab`): ascending symbols,
-// reserved bits zero, f >= 1, sum 4096.  Optionally copies the entries and
-// their cumulative frequencies to shared memory, and/or expands the list into
-// a warp's slot table.  Returns validity (warp-uniform).
+// Slots a table entry covers: rANS its frequency f (entry = symbol | f << 16);
+// Huffman 2^(12 - length) (entry = symbol | length << 16; the empty code of a
+// single-symbol chunk, length 0, covers all 4096), 0 for a length over 12.
+template <uint32_t CODEC>
+__device__ __forceinline__ uint32_t entry_slots(uint32_t e) {
+    if constexpr (CODEC == kCodecHuffman) return (e >> 16) <= kHuffMaxLen ? 1u << (kHuffMaxLen - (e >> 16)) : 0u;
+    else return e >> 16;
+}
+
+// Order key of a table entry: rANS entries ascend by symbol, Huffman entries
+// by (length, symbol), which is the entry itself (bits 8..15 are zero).
+template <uint32_t CODEC>
+__device__ __forceinline__ int entry_key(uint32_t e) {
+    return CODEC == kCodecHuffman ? (int)e : (int)(e & 0xFFu);
+}
+
+// Slot-table entry for slot t of a list entry covering f slots: rANS
+// f << 20 | t << 8 | low; Huffman length << 8 | low.
+template <uint32_t CODEC>
+__device__ __forceinline__ uint32_t slot_entry(uint32_t e, uint32_t f, uint32_t t, uint32_t low) {
+    if constexpr (CODEC == kCodecHuffman) return ((e >> 16) << 8) | low;
+    else return (f << 20) | (t << 8) | low;
+}
+
+// Check a frequency list / code table (n_present entries at `tab`): keys
+// ascending, reserved bits zero, every entry covering >= 1 slot, all 4096
+// slots covered (rANS: sum of f; Huffman: Kraft equality).  Optionally copies
+// the entries and their cumulative slot counts to shared memory, and/or
+// expands the list into a warp's slot table.  Returns validity (warp-uniform).
+template <uint32_t CODEC = kCodecRans>
 __device__ __forceinline__ bool warp_table(const uint32_t *tab, uint32_t n_present, uint32_t lane,
                                            uint32_t *entries_out, uint32_t *cum_out, uint32_t *lut,
                                            bool by_rank) {
     uint32_t run = 0;
-    int prev_sym = -1;
+    int prev_key = -1;
     bool ok = true;
     for (uint32_t base = 0; base < n_present; base += 32) {
         const uint32_t i = base + lane;
         const bool have = i < n_present;
         const uint32_t e = have ? tab[i] : 0u;
-        const uint32_t f = e >> 16, sym = e & 0xFFu;
+        const uint32_t f = have ? entry_slots<CODEC>(e) : 0u, sym = e & 0xFFu;
         bool good = !have || ((e & 0xFF00u) == 0 && f >= 1 && f <= kProbTotal);
-        const int left = __shfl_up_sync(kFull, (int)sym, 1);
-        if (have && (int)sym <= (lane == 0 ? prev_sym : left)) good = false;
+        const int key = entry_key<CODEC>(e);
+        const int left = __shfl_up_sync(kFull, key, 1);
+        if (have && key <= (lane == 0 ? prev_key : left)) good = false;
         uint32_t inc = f;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
@@ -450,15 +570,15 @@ __device__ __forceinline__ bool warp_table(const uint32_t *tab, uint32_t n_prese
             for (uint32_t q = 0; q < cnt; ++q) {
                 const uint32_t fq = __shfl_sync(kFull, f, q);
                 const uint32_t cq = __shfl_sync(kFull, cum, q);
-                const uint32_t sq = __shfl_sync(kFull, sym, q);
+                const uint32_t eq = __shfl_sync(kFull, e, q);
+                const uint32_t low = by_rank ? base + q : (eq & 0xFFu);
                 for (uint32_t t = lane; t < fq; t += 32) {
                     const uint32_t slot = cq + t;
-                    if (slot < kProbTotal && fq < kProbTotal)
-                        lut[slot] = (fq << 20) | (t << 8) | (by_rank ? base + q : sq);
+                    if (slot < kProbTotal && fq < kProbTotal) lut[slot] = slot_entry<CODEC>(eq, fq, t, low);
                 }
             }
         }
-        prev_sym = __shfl_sync(kFull, (int)sym, cnt - 1);
+        prev_key = __shfl_sync(kFull, key, cnt - 1);
         run += __shfl_sync(kFull, inc, 31);
     }
     return ok && run == kProbTotal;
@@ -523,15 +643,15 @@ struct WarpSmem {
 // Shared-table kernels, on a change of matrix: rebuild the block's slot table
 // from the frequency list of chunk k0 (the first chunk of the block's tile),
 // after checking it.  All threads of the block take part.
-template <int WARPS, uint32_t LAYOUT, class Params, class Job, class WS>
+template <int WARPS, uint32_t LAYOUT, uint32_t CODEC = kCodecRans, class Params, class Job, class WS>
 __device__ __forceinline__ void shared_table_rebuild(const Params &P, const Job &M, uint32_t k0, uint32_t lane,
                                                      uint32_t warp, const WS &S) {
     __syncthreads();
     if (warp == 0) {
         ChunkHead h;
-        bool ok = load_head(P, M, k0, lane, h);
-        if (ok) ok = warp_table(reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes), h.n_present, lane,
-                                S.ref_entries, S.ref_cum, nullptr, false);
+        bool ok = load_head<CODEC>(P, M, k0, lane, h);
+        if (ok) ok = warp_table<CODEC>(reinterpret_cast<const uint32_t *>(h.rec + kHeadBytes<CODEC>), h.n_present,
+                                       lane, S.ref_entries, S.ref_cum, nullptr, false);
         if (lane == 0) {
             S.blk[0] = ok ? h.n_present : 0u;
             S.blk[1] = ok;
@@ -542,10 +662,10 @@ __device__ __forceinline__ void shared_table_rebuild(const Params &P, const Job 
     if (S.blk[1] && np > 1) {
         for (uint32_t i = 0; i < np; ++i) {
             const uint32_t e = S.ref_entries[i], c = S.ref_cum[i];
-            const uint32_t f = e >> 16, sy = e & 0xFFu;
+            const uint32_t f = entry_slots<CODEC>(e), sy = e & 0xFFu;
             const uint32_t low = table_low_byte<LAYOUT>(np, i, sy);
             for (uint32_t t = threadIdx.x; t < f; t += WARPS * 32)
-                if (c + t < kProbTotal && f < kProbTotal) S.lut[c + t] = (f << 20) | (t << 8) | low;
+                if (c + t < kProbTotal && f < kProbTotal) S.lut[c + t] = slot_entry<CODEC>(e, f, t, low);
         }
     }
     __syncthreads();
@@ -554,13 +674,13 @@ __device__ __forceinline__ void shared_table_rebuild(const Params &P, const Job 
 // Shared-table kernels: chunk k's header, checked, and its frequency list
 // compared with the block's (every chunk of a shared-table matrix must carry
 // the same list).  False (with a status flag) if either check fails.
-template <class Params, class Job, class WS>
+template <uint32_t CODEC = kCodecRans, class Params, class Job, class WS>
 __device__ __forceinline__ bool shared_chunk_head(const Params &P, const Job &M, uint32_t k, uint32_t lane,
                                                   uint32_t np, const WS &S, ChunkHead &h) {
-    if (!load_head(P, M, k, lane, h)) return false;
+    if (!load_head<CODEC>(P, M, k, lane, h)) return false;
     bool same = S.blk[1] && h.n_present == np;
     if (same) {
-        const uint32_t *tab = reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes);
+        const uint32_t *tab = reinterpret_cast<const uint32_t *>(h.rec + kHeadBytes<CODEC>);
         for (uint32_t i = lane; i < np; i += 32) same = same && tab[i] == S.ref_entries[i];
     }
     if (!__all_sync(kFull, same)) {
