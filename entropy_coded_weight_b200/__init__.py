@@ -249,6 +249,18 @@ class Model:
                                              _stream_handle(decode_stream), pfree, pready),
               "eq_decode_model_stream")
 
+    def decode_symbols(self, matrix: int, out, status, stream=None) -> None:
+        """eq_decode_symbols: the matrix's raw symbol bytes into ``out`` (uint8 CUDA tensor, >= rows*cols)."""
+        nbytes = out.numel() * out.element_size()
+        check(self._L.eq_decode_symbols(self._m, matrix, out.data_ptr(), nbytes, status.data_ptr(),
+                                        _stream_handle(stream)), "eq_decode_symbols")
+
+    def gemm_symbols(self, matrix: int, sym, x, y, status, stream=None) -> None:
+        """eq_gemm_symbols: y[t, r] = scale[r] * sum_c x[t, c] * value(sym[r, c]) (+ super weights), on the
+        tensor cores; x bf16 [tokens, cols], y fp32 [tokens, rows] (CUDA tensors)."""
+        check(self._L.eq_gemm_symbols(self._m, matrix, sym.data_ptr(), x.data_ptr(), x.shape[0], y.data_ptr(),
+                                      status.data_ptr(), _stream_handle(stream)), "eq_gemm_symbols")
+
     def decode_gemv_matrix(self, matrix: int, x, y, status, stream=None) -> None:
         """eq_decode_gemv_matrix: y = W x without materialising W (x bf16 [cols], y fp32 [rows], device)."""
         check(self._L.eq_decode_gemv_matrix(self._m, matrix, x.data_ptr(), y.data_ptr(), status.data_ptr(),

@@ -77,6 +77,8 @@ SIGNATURES = {
     "eq_encode_bound": (_i32, [_vp, _u32, _vp]),
     "eq_decode_gemv_matrix": (_i32, [_vp, _u32, _vp, _vp, _vp, _vp]),
     "eq_decode_gemv_block": (_i32, [_vp, _u32, _vp, _vp, _u32, _vp, _vp]),
+    "eq_decode_symbols": (_i32, [_vp, _u32, _vp, _sz, _vp, _vp]),
+    "eq_gemm_symbols": (_i32, [_vp, _u32, _vp, _vp, _u32, _vp, _vp, _vp]),
     "eq_selftest_wait_timeout": (_i32, [_vp, _vp]),
     "eq_status_string": (ctypes.c_char_p, [_i32]),
     "eq_format_version": (_i32, []),

@@ -117,6 +117,21 @@ __device__ __forceinline__ void store_elems(const OutCtx &O, uint64_t idx, uint3
     }
 }
 
+// Symbol bytes (layout kSymbolBytes): the low bytes of e8[0..count).
+__device__ __forceinline__ void store_symbol_bytes(const OutCtx &O, uint64_t idx, uint32_t count,
+                                                   const uint32_t (&e8)[8]) {
+    uint8_t *out = reinterpret_cast<uint8_t *>(O.out);
+    if (count == 8) {
+        const uint32_t lo = (e8[0] & 0xFFu) | (e8[1] & 0xFFu) << 8 | (e8[2] & 0xFFu) << 16 | e8[3] << 24;
+        const uint32_t hi = (e8[4] & 0xFFu) | (e8[5] & 0xFFu) << 8 | (e8[6] & 0xFFu) << 16 | e8[7] << 24;
+        asm volatile("st.global.v2.b32 [%0], {%1, %2};" ::"l"(out + idx), "r"(lo), "r"(hi) : "memory");
+        return;
+    }
+#pragma unroll
+    for (uint32_t r = 0; r < 8; ++r)
+        if (r < count) out[idx + r] = (uint8_t)e8[r];
+}
+
 // Output bookkeeping for one chunk.  kRowUniform (cols % 256 == 0) keeps the
 // warp-uniform row of the current 256-symbol group; kLaneRows keeps each
 // lane's own row and column.
@@ -134,7 +149,7 @@ __device__ __forceinline__ float row_scale(const OutCtx &O, uint32_t row) {
 
 template <int DT, uint32_t LAYOUT>
 __device__ __forceinline__ void cursor_init(const OutCtx &O, uint64_t first, uint32_t lane, Cursor &c) {
-    if constexpr (LAYOUT != kGeneric) {
+    if constexpr (LAYOUT == kRowUniform || LAYOUT == kLaneRows) {
         const uint64_t e0 = LAYOUT == kRowUniform ? first : first + kGroup * lane;
         c.row = (uint32_t)(e0 / O.cols);
         c.col = (uint32_t)(e0 - (uint64_t)c.row * O.cols);
@@ -170,6 +185,8 @@ __device__ __forceinline__ void group_store(const OutCtx &O, uint16_t *dst, uint
                                             const uint32_t (&e8)[8]) {
     if constexpr (LAYOUT == kGeneric) {
         store_elems<DT>(O, idx, 8, e8);
+    } else if constexpr (LAYOUT == kSymbolBytes) {
+        store_symbol_bytes(O, idx, 8, e8);
     } else {
         st_global_v4(dst, dequant8<DT>(e8, c.scale, O.small_scales));
         cursor_advance<DT, LAYOUT>(O, idx, c);
@@ -336,7 +353,10 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, ui
             group_store<DT, LAYOUT>(O, dst, first + (uint64_t)g * kGroupSyms + kGroup * lane, cur, e8);
         if (tail) {
             const uint32_t mine = tail > kGroup * lane ? min(8u, tail - kGroup * lane) : 0u;
-            store_elems<DT>(O, first + (uint64_t)n_full * kGroupSyms + kGroup * lane, mine, e8);
+            if constexpr (LAYOUT == kSymbolBytes)
+                store_symbol_bytes(O, first + (uint64_t)n_full * kGroupSyms + kGroup * lane, mine, e8);
+            else
+                store_elems<DT>(O, first + (uint64_t)n_full * kGroupSyms + kGroup * lane, mine, e8);
         }
         return true;
     }
@@ -445,11 +465,14 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, ui
         }
         const uint32_t rp0 = ring + (pw & (kRingBytes - 1));
         uint32_t rp = rp0;
-        if constexpr (LAYOUT == kGeneric) {
+        if constexpr (LAYOUT == kGeneric || LAYOUT == kSymbolBytes) {
             uint32_t e8[8];
 #pragma unroll
             for (int r = 0; r < 8; ++r) e8[r] = codec_step<CODEC>(lut, rp, x, lt);
-            store_elems<DT>(O, first + (uint64_t)g * kGroupSyms + kGroup * lane, 8, e8);
+            if constexpr (LAYOUT == kSymbolBytes)
+                store_symbol_bytes(O, first + (uint64_t)g * kGroupSyms + kGroup * lane, 8, e8);
+            else
+                store_elems<DT>(O, first + (uint64_t)g * kGroupSyms + kGroup * lane, 8, e8);
         } else {
             // dequantise pairs as they are decoded: 4 packed registers instead of 8 entries
             const float2 s2 = make_float2(cur.scale, cur.scale);
@@ -476,7 +499,10 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, ui
             uint32_t e8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
             codec_tail<CODEC>(lut, ring, x, pw, lt, lane, tail, e8);
             const uint32_t mine = tail > kGroup * lane ? min(8u, tail - kGroup * lane) : 0u;
-            store_elems<DT>(O, first + (uint64_t)n_full * kGroupSyms + kGroup * lane, mine, e8);
+            if constexpr (LAYOUT == kSymbolBytes)
+                store_symbol_bytes(O, first + (uint64_t)n_full * kGroupSyms + kGroup * lane, mine, e8);
+            else
+                store_elems<DT>(O, first + (uint64_t)n_full * kGroupSyms + kGroup * lane, mine, e8);
         }
     }
     if (!ring_drain(ctl, mbar)) {
@@ -611,7 +637,7 @@ __global__ void eq_wait_timeout_kernel(int32_t *status) {
 struct DeviceSetup {
     bool ready = false;
     int sms = 0;
-    KernelSetup<DecodeParams> k[2][2][2][3];
+    KernelSetup<DecodeParams> k[2][2][2][4];
 };
 std::mutex g_setup_mu;
 DeviceSetup g_setup[128];
@@ -640,8 +666,9 @@ int device_setup(DeviceSetup **out) {
         if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return EQ_ERR_CUDA;
         int rc;
         if ((rc = setup_pair<EQ_INT8, kRowUniform>(d)) || (rc = setup_pair<EQ_INT8, kLaneRows>(d)) ||
-            (rc = setup_pair<EQ_INT8, kGeneric>(d)) || (rc = setup_pair<EQ_E4M3, kRowUniform>(d)) ||
-            (rc = setup_pair<EQ_E4M3, kLaneRows>(d)) || (rc = setup_pair<EQ_E4M3, kGeneric>(d)))
+            (rc = setup_pair<EQ_INT8, kGeneric>(d)) || (rc = setup_pair<EQ_INT8, kSymbolBytes>(d)) ||
+            (rc = setup_pair<EQ_E4M3, kRowUniform>(d)) || (rc = setup_pair<EQ_E4M3, kLaneRows>(d)) ||
+            (rc = setup_pair<EQ_E4M3, kGeneric>(d)) || (rc = setup_pair<EQ_E4M3, kSymbolBytes>(d)))
             return rc;
         d.ready = true;
     }
@@ -660,13 +687,13 @@ uint32_t layout_of(const eq_matrix_info &in, const uint16_t *out) {
 // launch per kernel variant (codec x table scope x dtype x layout) present, then one
 // scatter launch for the super weights.
 int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *const *outs, int32_t *d_status,
-                  cudaStream_t s) {
+                  cudaStream_t s, bool symbols = false) {
     DeviceSetup *dev = nullptr;
     int rc = device_setup(&dev);
     if (rc) return rc;
     for (uint32_t base = 0; base < count; base += kMaxMatsPerLaunch) {
         const uint32_t cnt = std::min<uint32_t>(kMaxMatsPerLaunch, count - base);
-        DecodeParams P[2][2][2][3];
+        DecodeParams P[2][2][2][4];
         for (auto &a : P)
             for (auto &b : a)
                 for (auto &c : b)
@@ -683,7 +710,7 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
             const MatrixDesc &d = m->mats[first + base + i];
             if (d.info.n_chunks == 0) continue;
             const int sh = d.info.uniform_table ? 1 : 0;
-            const uint32_t lay = layout_of(d.info, outs[base + i]);
+            const uint32_t lay = symbols ? kSymbolBytes : layout_of(d.info, outs[base + i]);
             DecodeParams &Pv = P[d.codec][sh][d.info.dtype - 1][lay];
             MatJob &J = Pv.mats[Pv.n_mats++];
             J.chunk_index = reinterpret_cast<const uint64_t *>(m->d_blob + d.chunk_index_off);
@@ -698,7 +725,7 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
             J.small_scales = d.small_scales ? 1u : 0u;
             const uint32_t per_tile = kSharedWarps * EQ_CHAINS;
             Pv.total_units += sh ? (d.info.n_chunks + per_tile - 1) / per_tile : d.info.n_chunks;
-            if (d.info.n_outliers) {
+            if (d.info.n_outliers && !symbols) {
                 ScatterJob &O = Q.jobs[Q.n_jobs++];
                 O.rec = reinterpret_cast<const uint32_t *>(m->d_blob + d.outliers_off);
                 O.out = outs[base + i];
@@ -713,7 +740,7 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
         for (int co = 0; co < 2; ++co)
             for (int sh = 0; sh < 2; ++sh)
                 for (int dt = 0; dt < 2; ++dt)
-                    for (int lay = 0; lay < 3; ++lay)
+                    for (int lay = 0; lay < 4; ++lay)
                         if ((rc = launch(dev->k[co][sh][dt][lay], dev->sms, P[co][sh][dt][lay], s))) return rc;
         if (n_out) {
             eq_outlier_scatter_kernel<<<(n_out + 127) / 128, 128, 0, s>>>(Q);
@@ -734,6 +761,17 @@ extern "C" EQW_API int eq_decode_matrix(const eq_model *m, uint32_t matrix, void
     if (out_bytes < need) return EQ_ERR_NOSPACE;
     uint16_t *out = static_cast<uint16_t *>(d_out);
     return launch_decode(m, matrix, 1, &out, d_status, s);
+}
+
+extern "C" EQW_API int eq_decode_symbols(const eq_model *m, uint32_t matrix, void *d_out, size_t out_bytes,
+                                         int32_t *d_status, cudaStream_t s) {
+    if (!m || !d_status || matrix >= m->mats.size()) return EQ_ERR_INVALID_ARG;
+    const eq_matrix_info &in = m->mats[matrix].info;
+    const uint64_t need = (uint64_t)in.rows * in.cols;
+    if (need && (!d_out || reinterpret_cast<uintptr_t>(d_out) % 16)) return EQ_ERR_INVALID_ARG;
+    if (out_bytes < need) return EQ_ERR_NOSPACE;
+    uint16_t *out = static_cast<uint16_t *>(d_out);
+    return launch_decode(m, matrix, 1, &out, d_status, s, true);
 }
 
 extern "C" EQW_API int eq_decode_block(const eq_model *m, uint32_t layer, void *d_out, size_t out_bytes,

@@ -50,7 +50,10 @@ constexpr int kSharedWarps = EQ_SHARED_WARPS;      // warps per block, shared-ta
 constexpr int kSharedMinCtas = EQ_SHARED_MIN_CTAS; // register budget: blocks of kSharedWarps per SM
 constexpr int kPrivateWarps = 4;                   // warps per block, per-warp-table kernel
 
-enum : uint32_t { kRowUniform = 0, kLaneRows = 1, kGeneric = 2 };
+// Output layouts of the decode kernel: bf16 with warp-uniform rows per group
+// (cols % 256 == 0), bf16 with per-lane rows (cols % 8 == 0), bf16 element by
+// element, or the raw symbol bytes (no dequant, no super weights).
+enum : uint32_t { kRowUniform = 0, kLaneRows = 1, kGeneric = 2, kSymbolBytes = 3 };
 
 // ---- PTX helpers: mbarrier + bulk copy (TMA, 1-D, no multicast) ---------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

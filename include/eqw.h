@@ -313,6 +313,33 @@ EQW_API int eq_decode_gemv_matrix(const eq_model *m, uint32_t matrix, const void
 EQW_API int eq_decode_gemv_block(const eq_model *m, uint32_t layer, const void *const *d_x, float *const *d_y,
                                  uint32_t count, int32_t *d_status, cudaStream_t s);
 
+/* ---- prefill path: symbol bytes + tensor-core GEMM ------------------------------
+ * EntQuant section 4: the decode cost is amortised at long sequences, where a
+ * linear layer's forward pass is a GEMM over many tokens.
+ *
+ * eq_decode_symbols: decode one matrix's symbols, without dequantisation, into
+ * `d_out` (device, 16-byte aligned, >= rows * cols bytes, row-major): Int8 or
+ * E4M3 codes, half the bytes of bf16.  Super-weight positions hold the
+ * stream's placeholder symbol 0 (their values stay in the container).
+ */
+EQW_API int eq_decode_symbols(const eq_model *m, uint32_t matrix, void *d_out, size_t out_bytes, int32_t *d_status,
+                              cudaStream_t s);
+
+/*
+ * eq_gemm_symbols: Y = X W^T for a matrix whose symbols eq_decode_symbols
+ * wrote to `d_sym`, on the tensor cores (tcgen05.mma, bf16 inputs, fp32
+ * accumulation in tensor memory):
+ *   Y[t, r] = scale[r] * sum_c X[t, c] * value(sym[r, c])
+ *             + sum over super weights (r, c, v) of bf16(v) * X[t, c]
+ * value() is exact in bf16; the scale multiplies the fp32 sum once per output
+ * (round to nearest even).  X: device bf16 [tokens, cols] row-major, Y:
+ * device fp32 [tokens, rows] row-major, both 16-byte aligned.  Needs
+ * rows % 128 == 0 and cols % 64 == 0 (EQ_ERR_UNSUPPORTED otherwise).
+ * Enqueued on `s`.
+ */
+EQW_API int eq_gemm_symbols(const eq_model *m, uint32_t matrix, const void *d_sym, const void *d_x, uint32_t tokens,
+                            float *d_y, int32_t *d_status, cudaStream_t s);
+
 /* ---- failure detection ----------------------------------------------------------
  * Check of the decode kernels' timeout path: one warp runs the decoder's own
  * staging-ring drain on a ring slot marked as issued whose copy was never

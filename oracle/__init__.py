@@ -357,6 +357,45 @@ def gemv_exact(w_bits: np.ndarray, x_bits: np.ndarray) -> tuple[np.ndarray, np.n
     return w @ x, np.abs(w) @ np.abs(x)
 
 
+def symbol_values(dtype: int) -> np.ndarray:
+    """Exact value of every symbol byte (float64[256]; NaN codes of E4M3 are NaN)."""
+    f = int8_value if dtype == INT8 else e4m3_value
+    return np.array([f(b) for b in range(256)], np.float64)
+
+
+def stream_symbols(m) -> np.ndarray:
+    """The symbols a container stores for matrix ``m``: its symbols with the
+    placeholder 0 at every super-weight position."""
+    sym = np.ascontiguousarray(m.symbols, np.uint8).copy()
+    if len(m.out_row):
+        sym[np.asarray(m.out_row, np.int64), np.asarray(m.out_col, np.int64)] = 0
+    return sym
+
+
+def gemm_symbols_exact(m, x_bits: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Prefill forward of matrix ``m`` on tokens ``x`` (bf16 bits [tokens, cols]), in float64:
+    Y[t, r] = scale[r] * sum_c X[t, c] * value(sym[r, c]) + sum over super weights (r, c, v)
+    of bf16(v) * X[t, c]; and the matching sum of absolute terms (for error bounds).
+
+    EntQuant technical summary, section 4: at long sequences the decode cost is
+    amortised over a GEMM per linear layer.  The scale multiplies the row's sum
+    (it is the same real number as multiplying every product); super weights
+    enter with their bf16 value, as the decode path writes them.
+    """
+    vals = symbol_values(m.dtype)
+    w = vals[stream_symbols(m)]                       # [rows, cols], exact
+    x = bf16_to_f64(x_bits).reshape(np.shape(x_bits))  # [tokens, cols], exact
+    sc = np.asarray(m.scales, np.float64)
+    y = (x @ w.T) * sc[None, :]
+    mag = (np.abs(x) @ np.abs(w).T) * np.abs(sc)[None, :]
+    if len(m.out_row):
+        ov = bf16_to_f64(bf16_rne(np.asarray(m.out_val, np.float32)))
+        for r, c, v in zip(np.asarray(m.out_row, np.int64), np.asarray(m.out_col, np.int64), ov):
+            y[:, r] += v * x[:, c]
+            mag[:, r] += abs(v) * np.abs(x[:, c])
+    return y, mag
+
+
 # ---------------------------------------------------------------------------
 # container format v1 (writer)
 # ---------------------------------------------------------------------------

@@ -54,3 +54,32 @@ def test_against_exact_rationals(orc):
         absum = sum(abs(Fraction(float(wf[r, c])) * Fraction(float(xf[c]))) for c in range(13))
         assert abs(Fraction(float(y[r])) - exact) <= Fraction(13, 2 ** 53) * absum
         assert float(absum) == mag[r]
+
+
+# ---- prefill GEMM on symbols (oracle.gemm_symbols_exact) ----
+
+def test_gemm_symbols_orientation_and_scale(orc):
+    import workloads as W
+    m = W.random_int8_matrix(3, 2, 3)
+    m.symbols[:] = np.array([[1, 2, 3], [0xFF, 0, 5]], np.uint8)  # values 1 2 3 / -1 0 5
+    m.scales[:] = np.array([0.5, 2.0], np.float32)
+    x = _bits(torch.tensor([[1.0, 0.0, 0.0], [0.0, 1.0, 1.0]], dtype=torch.bfloat16))
+    y, mag = orc.gemm_symbols_exact(m, x)
+    # token 0 selects column 0: [0.5 * 1, 2 * -1]; token 1 sums columns 1, 2: [0.5 * 5, 2 * 5]
+    assert y.tolist() == [[0.5, -2.0], [2.5, 10.0]]
+    assert mag.tolist() == [[0.5, 2.0], [2.5, 10.0]]
+
+
+def test_gemm_symbols_e4m3_values_and_outliers(orc):
+    import workloads as W
+    m = W.random_e4m3_matrix(4, 2, 4)
+    m.symbols[:] = np.array([[0x38, 0xB8, 0x01, 0x7E], [0x00, 0x80, 0x40, 0x08]], np.uint8)
+    m.scales[:] = 1.0
+    m.out_row = np.array([1], np.uint32)
+    m.out_col = np.array([3], np.uint32)
+    m.out_val = np.array([100.0], np.float32)
+    x = _bits(torch.ones(1, 4, dtype=torch.bfloat16))
+    y, _ = orc.gemm_symbols_exact(m, x)
+    # 0x38 = 1, 0xB8 = -1, 0x01 = 2^-9, 0x7E = 448; row 1: 0, -0, 0x40 = 2, 0x08 = 2^-6 replaced by
+    # the placeholder 0 under the super weight, which adds 100
+    assert y.tolist() == [[1.0 - 1.0 + 2.0 ** -9 + 448.0, 2.0 + 100.0]]
