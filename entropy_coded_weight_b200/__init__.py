@@ -255,6 +255,13 @@ class Model:
         check(self._L.eq_decode_symbols(self._m, matrix, out.data_ptr(), nbytes, status.data_ptr(),
                                         _stream_handle(stream)), "eq_decode_symbols")
 
+    def decode_symbols_block(self, layer: int, outs, status, stream=None) -> None:
+        """eq_decode_symbols_block: raw symbol bytes of every matrix of ``layer`` into ``outs[i]``."""
+        n = len(outs)
+        po = (ctypes.c_void_p * max(1, n))(*(o.data_ptr() for o in outs))
+        check(self._L.eq_decode_symbols_block(self._m, layer, po, n, status.data_ptr(), _stream_handle(stream)),
+              "eq_decode_symbols_block")
+
     def gemm_symbols(self, matrix: int, sym, x, y, status, stream=None) -> None:
         """eq_gemm_symbols: y[t, r] = scale[r] * sum_c x[t, c] * value(sym[r, c]) (+ super weights), on the
         tensor cores; x bf16 [tokens, cols], y fp32 [tokens, rows] (CUDA tensors)."""

@@ -774,6 +774,21 @@ extern "C" EQW_API int eq_decode_symbols(const eq_model *m, uint32_t matrix, voi
     return launch_decode(m, matrix, 1, &out, d_status, s, true);
 }
 
+extern "C" EQW_API int eq_decode_symbols_block(const eq_model *m, uint32_t layer, void *const *d_outs,
+                                               uint32_t count, int32_t *d_status, cudaStream_t s) {
+    if (!m || !d_status || !d_outs || layer >= m->n_layers || count != m->layer_count[layer])
+        return EQ_ERR_INVALID_ARG;
+    const uint32_t first = m->layer_first[layer];
+    std::vector<uint16_t *> outs(count);
+    for (uint32_t i = 0; i < count; ++i) {
+        const eq_matrix_info &in = m->mats[first + i].info;
+        if ((uint64_t)in.rows * in.cols && (!d_outs[i] || reinterpret_cast<uintptr_t>(d_outs[i]) % 16))
+            return EQ_ERR_INVALID_ARG;
+        outs[i] = static_cast<uint16_t *>(d_outs[i]);
+    }
+    return launch_decode(m, first, count, outs.data(), d_status, s, true);
+}
+
 extern "C" EQW_API int eq_decode_block(const eq_model *m, uint32_t layer, void *d_out, size_t out_bytes,
                                        int32_t *d_status, cudaStream_t s) {
     if (!m || !d_status || layer >= m->n_layers) return EQ_ERR_INVALID_ARG;

@@ -551,7 +551,7 @@ __device__ __forceinline__ bool warp_table(const uint32_t *tab, uint32_t n_prese
         const uint32_t i = base + lane;
         const bool have = i < n_present;
         const uint32_t e = have ? tab[i] : 0u;
-        const uint32_t f = have ? entry_slots<CODEC>(e) : 0u, sym = e & 0xFFu;
+        const uint32_t f = have ? entry_slots<CODEC>(e) : 0u;
         bool good = !have || ((e & 0xFF00u) == 0 && f >= 1 && f <= kProbTotal);
         const int key = entry_key<CODEC>(e);
         const int left = __shfl_up_sync(kFull, key, 1);

@@ -36,15 +36,31 @@
 
 namespace {
 
-constexpr int kGemmThreads = 128;
-constexpr uint32_t kTileM = 128;   // tokens per tile (MMA M, accumulator lanes)
-constexpr uint32_t kTileN = 128;   // weight rows per tile (MMA N, accumulator columns)
-constexpr uint32_t kTileK = 64;    // K per stage
-constexpr uint32_t kMmaK = 16;     // K per tcgen05.mma (bf16)
-constexpr uint32_t kStageBytesA = kTileM * kTileK * 2;  // 16 KiB
+#ifndef EQ_GEMM_THREADS
+#define EQ_GEMM_THREADS 256
+#endif
+constexpr int kGemmThreads = EQ_GEMM_THREADS;  // 4 or 8 warps
+// One token tile of 128 per CTA and two stages is the configuration verified
+// on the GPU.  Two token halves per CTA (two accumulators fed by one widened
+// weight tile) raised an illegal-instruction error there, cause not found;
+// it is not used.
+#ifndef EQ_GEMM_HALVES
+#define EQ_GEMM_HALVES 1
+#endif
+#ifndef EQ_GEMM_STAGES
+#define EQ_GEMM_STAGES 2
+#endif
+static_assert(EQ_GEMM_HALVES == 1, "two token halves per CTA faulted on the GPU and are not used");
+constexpr uint32_t kMmaM = 128;                        // tokens per MMA (accumulator lanes)
+constexpr uint32_t kHalves = EQ_GEMM_HALVES;           // MMAs per widened weight tile
+constexpr uint32_t kTileM = kMmaM * kHalves;           // tokens per CTA tile
+constexpr uint32_t kTileN = 128;                       // weight rows per tile (MMA N, accumulator columns)
+constexpr uint32_t kTileK = 64;                        // K per stage
+constexpr uint32_t kMmaK = 16;                         // K per tcgen05.mma (bf16)
+constexpr uint32_t kStageBytesA = kTileM * kTileK * 2;  // 16 KiB per 128 tokens
 constexpr uint32_t kStageBytesB = kTileN * kTileK * 2;  // 16 KiB
-constexpr uint32_t kStages = 2;
-constexpr uint32_t kTmemCols = kTileN;  // fp32 accumulator columns
+constexpr uint32_t kStages = EQ_GEMM_STAGES;
+constexpr uint32_t kTmemCols = kTileN * kHalves;        // one fp32 accumulator per token half
 constexpr size_t kGemmSmem = kStages * (kStageBytesA + kStageBytesB) + 1024;
 
 struct GemmParams {
@@ -57,16 +73,21 @@ struct GemmParams {
     uint32_t dtype;
 };
 
-// Shared-memory matrix descriptor (tcgen05), K-major without swizzle: start
-// address, leading byte offset (between K-adjacent core matrices), stride
-// byte offset (between 8-row groups), all in 16-byte units; version 1.
+#ifndef EQ_GEMM_SWIZZLE
+#define EQ_GEMM_SWIZZLE 1
+#endif
+
+// Shared-memory matrix descriptor (tcgen05), K-major: start address, leading
+// byte offset, stride byte offset (between 8-row groups), all in 16-byte
+// units; version 1; layout type 2 = 128-byte swizzle, 0 = none.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
     uint64_t d = 0;
     d |= (uint64_t)((addr >> 4) & 0x3FFFu);
     d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
     d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-    d |= (uint64_t)1 << 46;  // descriptor version for tcgen05
-    return d;                // base offset 0, layout type 0 (no swizzle)
+    d |= (uint64_t)1 << 46;                        // descriptor version for tcgen05
+    if (EQ_GEMM_SWIZZLE) d |= (uint64_t)2 << 61;   // 128-byte swizzle (base offset 0: tiles 1024-aligned)
+    return d;
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
@@ -77,11 +98,23 @@ constexpr uint32_t kInstrDesc = (1u << 4)                 // D format fp32
                               | ((kTileN >> 3) << 17)     // N / 8
                               | ((kTileM >> 4) << 24);    // M / 16
 
-// Byte offset of element (row, k) of a [rows x 64] K-major tile in the
-// core-matrix layout: core (row / 8, k / 8) at ((row / 8) * 8 + k / 8) * 128,
-// row % 8 at 16-byte stride inside it, k % 8 at 2-byte stride.
+// Byte offset of the 16-byte chunk k8 (bf16 8 k8 .. 8 k8 + 7) of tile row `row`.
+// 128-byte swizzle: each 64-element row is one 128-byte line, 8-row groups are
+// 1024 bytes apart, and chunk k8 of row r sits at chunk position k8 ^ (r % 8).
+// Without swizzle: core matrices of 8 rows x 16 bytes, core (row / 8, k8) at
+// ((row / 8) * 8 + k8) * 128 with rows 16 bytes apart inside it.
 __device__ __forceinline__ uint32_t tile_offset(uint32_t row, uint32_t k8) {
+    if (EQ_GEMM_SWIZZLE) return (row >> 3) * 1024u + (row & 7u) * 128u + ((k8 ^ (row & 7u)) << 4);
     return ((row >> 3) * (kTileK / 8) + k8) * 128u + (row & 7u) * 16u;
+}
+
+// Descriptor of K step kk (16 bf16) of a tile at `buf`: 128-byte swizzle
+// advances the start by 32 bytes per step (the hardware applies the XOR),
+// LBO unused (1), SBO 1024; without swizzle two 128-byte cores per step,
+// LBO 128 (K-adjacent cores), SBO 1024 (8-row groups).
+__device__ __forceinline__ uint64_t tile_desc(uint32_t buf, uint32_t kk) {
+    if (EQ_GEMM_SWIZZLE) return smem_desc(buf + kk * 32u, 16u, 1024u);
+    return smem_desc(buf + kk * 256u, 128u, 1024u);
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
@@ -164,37 +197,53 @@ __global__ void __launch_bounds__(kGemmThreads) eq_gemm_symbols_kernel(const __g
     const uint32_t tmem = tmem_base_s;
 
     const uint32_t n_slabs = P.cols / kTileK;
+    // per thread: kXv 16-byte chunks of the X tile and kBv of the symbol tile
+    constexpr uint32_t kXv = kTileM * (kTileK / 8) / kGemmThreads;
+    constexpr uint32_t kBv = kTileN * (kTileK / 16) / kGemmThreads;
+    uint4 xr[kXv], br[kBv];
+    // global -> registers for slab `it` (issued one slab ahead of its use)
+    auto fetch = [&](uint32_t it) {
+        const uint32_t k0 = it * kTileK;
+#pragma unroll
+        for (uint32_t i = 0; i < kXv; ++i) {
+            const uint32_t e = tid + i * kGemmThreads, r = e >> 3, k8 = e & 7u;
+            xr[i] = m0 + r < P.tokens
+                        ? __ldg(reinterpret_cast<const uint4 *>(P.x + (size_t)(m0 + r) * P.cols + k0) + k8)
+                        : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (uint32_t i = 0; i < kBv; ++i) {
+            const uint32_t e = tid + i * kGemmThreads, r = e >> 2, c = e & 3u;
+            br[i] = __ldg(reinterpret_cast<const uint4 *>(P.sym + (size_t)(n0 + r) * P.cols + k0) + c);
+        }
+    };
+    if (n_slabs) fetch(0);
     bool ok = true;
     for (uint32_t it = 0; it < n_slabs && ok; ++it) {
-        const uint32_t s = it & 1u;
-        if (it >= kStages) {  // the MMAs that read this stage two slabs ago must be done
-            // commit number (it - 2) / 2 of stage s, i.e. its completion of parity ((it - 2) / 2) & 1
-            ok = mbar_wait_bounded(mbar0 + 8 * s, ((it - kStages) >> 1) & 1u);
+        const uint32_t s = it % kStages;
+        if (it >= kStages) {  // the MMAs that read this stage kStages slabs ago must be done
+            // commit number (it - kStages) / kStages of stage s, i.e. the completion of that parity
+            ok = mbar_wait_bounded(mbar0 + 8 * s, ((it - kStages) / kStages) & 1u);
             if (!__syncthreads_and(ok)) {
                 ok = false;
                 break;
             }
         }
-        const uint32_t k0 = it * kTileK;
-        // X tile: 128 rows x 8 chunks of 8 bf16
+        // registers -> stage s: the X tile as is, the symbol tile widened to bf16
 #pragma unroll
-        for (uint32_t i = 0; i < kTileM * (kTileK / 8) / kGemmThreads; ++i) {
-            const uint32_t e = tid + i * kGemmThreads, r = e >> 3, k8 = e & 7u;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (m0 + r < P.tokens)
-                v = __ldg(reinterpret_cast<const uint4 *>(P.x + (size_t)(m0 + r) * P.cols + k0) + k8);
-            st_shared_v4(bufA(s) + tile_offset(r, k8), v);
+        for (uint32_t i = 0; i < kXv; ++i) {
+            const uint32_t e = tid + i * kGemmThreads;
+            st_shared_v4(bufA(s) + tile_offset(e >> 3, e & 7u), xr[i]);
         }
-        // symbol tile: 128 rows x 4 chunks of 16 bytes, widened to bf16
 #pragma unroll
-        for (uint32_t i = 0; i < kTileN * (kTileK / 16) / kGemmThreads; ++i) {
+        for (uint32_t i = 0; i < kBv; ++i) {
             const uint32_t e = tid + i * kGemmThreads, r = e >> 2, c = e & 3u;
-            const uint4 b = __ldg(reinterpret_cast<const uint4 *>(P.sym + (size_t)(n0 + r) * P.cols + k0) + c);
             uint4 lo, hi;
-            widen16<DT>(b, lo, hi);
+            widen16<DT>(br[i], lo, hi);
             st_shared_v4(bufB(s) + tile_offset(r, 2 * c), lo);
             st_shared_v4(bufB(s) + tile_offset(r, 2 * c + 1), hi);
         }
+        if (it + 1 < n_slabs) fetch(it + 1);  // in flight during the barrier and the MMAs
         fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
         tc_fence_before();
         __syncthreads();
@@ -202,31 +251,39 @@ __global__ void __launch_bounds__(kGemmThreads) eq_gemm_symbols_kernel(const __g
             tc_fence_after();
 #pragma unroll
             for (uint32_t kk = 0; kk < kTileK / kMmaK; ++kk) {
-                // K step kk covers core columns 2kk, 2kk+1: 256 bytes further per step
-                const uint64_t da = smem_desc(bufA(s) + kk * 256u, 128u, 1024u);
-                const uint64_t db = smem_desc(bufB(s) + kk * 256u, 128u, 1024u);
-                tc_mma(tmem, da, db, (it | kk) != 0u);
+                const uint64_t db = tile_desc(bufB(s), kk);
+#pragma unroll
+                for (uint32_t h = 0; h < kHalves; ++h)  // token half h: A rows 128h.., accumulator columns 128h..
+                    tc_mma(tmem + h * kTileN, tile_desc(bufA(s) + h * (kMmaM * kTileK * 2), kk), db,
+                           (it | kk) != 0u);
             }
             tc_commit(mbar0 + 8 * s);
         }
     }
     // all MMAs done: the last commit of the last slab covers every earlier MMA of thread 0
     if (ok && n_slabs) {
-        const uint32_t last = n_slabs - 1;
-        ok = mbar_wait_bounded(mbar0 + 8 * (last & 1u), (last >> 1) & 1u);
-        if (ok && last) ok = mbar_wait_bounded(mbar0 + 8 * ((last - 1) & 1u), ((last - 1) >> 1) & 1u);
+        // the last commit of every stage (the very last one covers all MMAs of thread 0)
+        for (uint32_t j = 0; j < kStages && j < n_slabs && ok; ++j) {
+            const uint32_t it = n_slabs - 1 - j;
+            ok = mbar_wait_bounded(mbar0 + 8 * (it % kStages), (it / kStages) & 1u);
+        }
         ok = __syncthreads_and(ok);
     }
     tc_fence_after();
     if (ok) {
-        const uint32_t m = m0 + warp * 32u + lane;
+        // warp w may read accumulator lanes 32 (w % 4) .. + 31; the warps that
+        // share a lane quarter split the accumulator columns (kHalves x 128)
+        constexpr uint32_t kWarps = kGemmThreads / 32, kColsPerWarp = kTmemCols * 4 / kWarps;
+        const uint32_t quarter = warp & 3u, c_first = (warp >> 2) * (kColsPerWarp / 32);
 #pragma unroll 1
-        for (uint32_t c = 0; c < kTileN / 32; ++c) {
+        for (uint32_t c = c_first; c < c_first + kColsPerWarp / 32; ++c) {
+            const uint32_t h = c / (kTileN / 32), cn = c % (kTileN / 32);  // token half, column chunk
+            const uint32_t m = m0 + h * kMmaM + quarter * 32u + lane;
             uint32_t r[32];
-            tmem_ld32(tmem + ((warp * 32u) << 16) + c * 32u, r);
+            tmem_ld32(tmem + ((quarter * 32u) << 16) + c * 32u, r);
             if (m < P.tokens) {
-                float4 *dst = reinterpret_cast<float4 *>(P.y + (size_t)m * P.rows + n0 + c * 32u);
-                const float4 *sc = reinterpret_cast<const float4 *>(P.scales + n0 + c * 32u);
+                float4 *dst = reinterpret_cast<float4 *>(P.y + (size_t)m * P.rows + n0 + cn * 32u);
+                const float4 *sc = reinterpret_cast<const float4 *>(P.scales + n0 + cn * 32u);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const float4 s4 = __ldg(sc + q);

@@ -325,6 +325,12 @@ EQW_API int eq_decode_gemv_block(const eq_model *m, uint32_t layer, const void *
 EQW_API int eq_decode_symbols(const eq_model *m, uint32_t matrix, void *d_out, size_t out_bytes, int32_t *d_status,
                               cudaStream_t s);
 
+/* The same for every matrix of `layer` in one launch: d_outs[i] (host array of
+ * `count` device pointers, count = the layer's matrix count, each 16-byte
+ * aligned with rows * cols bytes) receives matrix i of the layer. */
+EQW_API int eq_decode_symbols_block(const eq_model *m, uint32_t layer, void *const *d_outs, uint32_t count,
+                                    int32_t *d_status, cudaStream_t s);
+
 /*
  * eq_gemm_symbols: Y = X W^T for a matrix whose symbols eq_decode_symbols
  * wrote to `d_sym`, on the tensor cores (tcgen05.mma, bf16 inputs, fp32

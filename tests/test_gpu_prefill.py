@@ -162,3 +162,16 @@ def test_unsupported_shapes(eqw):
                            torch.zeros(4, 100, dtype=torch.float32, device="cuda"), status)
     assert e.value.code == EQ_ERR_UNSUPPORTED
     model.close()
+
+
+def test_decode_symbols_block_bit_exact(eqw, orc):
+    mats = W.llama70b_int8_layer(0)
+    model = _open(eqw, mats)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    outs = [torch.empty(m.rows * m.cols, dtype=torch.uint8, device="cuda") for m in mats]
+    model.decode_symbols_block(0, outs, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for m, o in zip(mats, outs):
+        assert np.array_equal(o.cpu().numpy().reshape(m.rows, m.cols), orc.stream_symbols(m))
+    model.close()
