@@ -49,8 +49,8 @@ UNIT = "GB/s"
 # block, from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of
 # the same launch configuration, and the SHA-256 of the decode sources it was
 # taken on: the figure is reported only while the sources are unchanged.
-DECODE_TRAFFIC_BYTES = 1_897_507_936
-DECODE_TRAFFIC_SOURCES_SHA256 = "dd6fd885e04a84efc15272c5534d75a880bd670005d7c9fb030788120f21c1db"
+DECODE_TRAFFIC_BYTES = 1_899_555_600
+DECODE_TRAFFIC_SOURCES_SHA256 = "81d52fc7861db322b4dbc22c2df003f8f0b4437df08a4f9246e70d4251b28a0c"
 DECODE_SOURCES = ("entropy_coded_weight_b200/csrc/eqw_decode.cu", "entropy_coded_weight_b200/csrc/eqw_device.cuh")
 
 
@@ -190,6 +190,15 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
                 "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
+
+
+def measured_bf16_peak() -> float:
+    """Dense bf16 TFLOP/s: the measured burst figure, else the recipe's fallback (1590)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
 
 
 def measured_hbm_peak() -> tuple[float, str]:
@@ -454,6 +463,56 @@ def bench_eqw(args, d: Dist) -> dict | None:
         hstack.close()
         del hblob
 
+    # ---- E: prefill on tensor cores: symbols of layer 0 decoded once, 7 GEMMs over 1024 tokens ----
+    prefill = None
+    if d.rank == 0:
+        pstep = stack.steps[0]
+        pm = pstep.model
+        idx = list(pm.layer_matrices(pstep.layer))
+        infos = [pm.info(i) for i in idx]
+        tokens = 1024
+        syms = [torch.empty(inf.rows * inf.cols, dtype=torch.uint8, device=dev) for inf in infos]
+        xs_p = [W.gemv_activation(7, j, tokens * inf.cols).reshape(tokens, inf.cols).to(dev)
+                for j, inf in enumerate(infos)]
+        ys_p = [torch.empty(tokens, inf.rows, dtype=torch.float32, device=dev) for inf in infos]
+        pst = torch.zeros(1, dtype=torch.int32, device=dev)
+        ps = torch.cuda.Stream(device=dev)
+
+        def p_decode():
+            pm.decode_symbols_block(pstep.layer, syms, pst, ps)
+
+        def p_gemm():
+            for i, mi in enumerate(idx):
+                pm.gemm_symbols(mi, syms[i], xs_p[i], ys_p[i], pst, ps)
+
+        def p_time(fn, n=5):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(ps)
+            for _ in range(n):
+                fn()
+            b.record(ps)
+            torch.cuda.synchronize()
+            return a.elapsed_time(b) / n
+
+        dec_ms = p_time(p_decode)
+        gemm_ms = p_time(p_gemm)
+        if int(pst.item()) != 0:
+            raise RuntimeError(f"prefill status {int(pst.item())}")
+        flops = sum(2.0 * tokens * inf.rows * inf.cols for inf in infos)
+        bf16_peak = measured_bf16_peak()
+        tflops = flops / (gemm_ms / 1e3) / 1e12
+        prefill = {"tokens": tokens, "decode_symbols_ms": round(dec_ms, 4), "gemm_ms": round(gemm_ms, 4),
+                   "tflops": round(tflops, 1), "unit": "TFLOP/s", "bf16_peak": bf16_peak,
+                   "frac": round(tflops / bf16_peak, 4), "kernel": "eq_gemm_symbols_kernel (tcgen05)",
+                   "layer_ms": round(dec_ms + gemm_ms, 4),
+                   "note": "layer 0: the 7 matrices' symbols decoded to bytes in one launch, then one tcgen05 "
+                           "GEMM per matrix against 1024 bf16 tokens (fp32 out); frac of the measured cuBLAS "
+                           "bf16 burst peak"}
+        del syms, xs_p, ys_p
+
     # ---- C: fused decode + GEMV, no bf16 buffers; blocks in sequence on one stream ----
     fstream = torch.cuda.Stream(device=dev)
     fys = [torch.empty_like(y) for y in ys]
@@ -540,6 +599,7 @@ def bench_eqw(args, d: Dist) -> dict | None:
                             "note": "y = W x per matrix with W decoded in registers; value = bf16 weight bytes "
                                     "consumed per second (2 x symbols / time), one block after another"},
         "huffman": huff,
+        "prefill": prefill,
         "e2e": {"value": round(value_e, 2), "unit": UNIT, "h2d_bytes_per_step": int(blob.size * stack.copies),
                 "d2h_bytes_per_step": 4, "ms_per_step": round(ms_e_max / args.steps, 3)},
         "cpu_baseline": cpu,
