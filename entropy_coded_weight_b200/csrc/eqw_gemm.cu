@@ -14,17 +14,21 @@
 // is applied once per output in the epilogue and the (rare) super weights by
 // a small second kernel.
 //
-// Kernel eq_gemm_symbols_kernel, one CTA per 128 x 128 output tile, 4 warps:
-//   stage      K slab of 64: all threads copy the X tile (16-byte loads) and
-//              widen the symbol tile into shared memory in the canonical
-//              K-major layout without swizzle (8 x 16-byte core matrices,
-//              K-adjacent cores 128 B apart, 8-row groups 1024 B apart);
-//              two stages alternate so the copy of slab s+1 overlaps the
-//              tensor-core work on slab s
-//   MMA        one thread issues 4 x tcgen05.mma (M 128, N 128, K 16) per
-//              slab and tcgen05.commit to the stage's mbarrier
-//   epilogue   warp w reads accumulator lanes 32w..32w+31 with tcgen05.ld,
-//              multiplies by the row scales and stores fp32
+// Kernel eq_gemm_symbols_kernel, one CTA per 128 x 128 output tile, 8
+// producer warps and one MMA warp:
+//   producers  per K slab of 64: copy the token tile (16-byte loads,
+//              prefetched one slab ahead into registers) and widen the symbol
+//              tile into a shared-memory stage in the 128-byte-swizzled
+//              K-major layout (16-byte chunk c of row r at chunk position
+//              c ^ (r % 8), 8-row groups 1024 B apart); arrive on the stage's
+//              "full" mbarrier; refill a stage once its "empty" barrier says
+//              the tensor core is done with it (a ring of 3 stages)
+//   MMA warp   one lane waits for "full", issues 4 x tcgen05.mma (M 128,
+//              N 128, K 16, fp32 accumulator in 128 TMEM columns) and
+//              tcgen05.commit to the stage's "empty" barrier; a last commit
+//              to "done" releases the epilogue
+//   epilogue   producer warp w reads accumulator lanes 32 (w % 4) with
+//              tcgen05.ld, multiplies by the row scales and stores fp32
 // Every mbarrier wait is bounded; on expiry the CTA records EQ_DEV_TIMEOUT,
 // still releases its tensor memory and stops.
 #include <cuda_runtime.h>
@@ -48,7 +52,7 @@ constexpr int kGemmThreads = EQ_GEMM_THREADS;  // 4 or 8 warps
 #define EQ_GEMM_HALVES 1
 #endif
 #ifndef EQ_GEMM_STAGES
-#define EQ_GEMM_STAGES 2
+#define EQ_GEMM_STAGES 3
 #endif
 static_assert(EQ_GEMM_HALVES == 1, "two token halves per CTA faulted on the GPU and are not used");
 constexpr uint32_t kMmaM = 128;                        // tokens per MMA (accumulator lanes)
@@ -122,16 +126,47 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                  : "memory");
 }
 
-// 16 symbol bytes -> 16 bf16 (exact), as two 16-byte vectors.
+// 16 symbol bytes -> 16 bf16 (exact), as two 16-byte vectors, without the
+// conversion pipe.  Int8: with the sign bit flipped, byte u = v + 128 placed
+// under the exponent of 2^23 (bits 0x4B0000uu) is the float 2^23 + 128 + v,
+// so one exact fp32 subtraction gives v, whose bf16 is the float's upper
+// half (v has at most 8 significant bits).  E4M3: the 7 exponent/mantissa
+// bits at bit 20 and the sign at bit 31 are value * 2^-120 as an fp32
+// (subnormal codes included), and * 2^120 is exact; again the upper half is
+// the bf16 (3 mantissa bits).  Pairs are packed with one byte permute.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+template <int DT>
+__device__ __forceinline__ float byte_value(uint32_t w, uint32_t i) {
+    if constexpr (DT == EQ_INT8) {
+        // bytes of (w ^ 0x80808080) and 0x4B000000: byte i, then 0x00, 0x00, 0x4B
+        const uint32_t bits = prmt(w, 0x4B000000u, 0x7440u | i);
+        return __fadd_rn(__uint_as_float(bits), -8388736.0f);  // - (2^23 + 128)
+    } else {
+        const uint32_t b = (w >> (8 * i)) & 0xFFu;
+        return __fmul_rn(__uint_as_float(((b & 0x80u) << 24) | ((b & 0x7Fu) << 20)), 0x1p120f);
+    }
+}
+
 template <int DT>
 __device__ __forceinline__ void widen16(uint4 b, uint4 &lo, uint4 &hi) {
-    const uint32_t w[4] = {b.x, b.y, b.z, b.w};
+    uint32_t w[4] = {b.x, b.y, b.z, b.w};
+    if constexpr (DT == EQ_INT8) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] ^= 0x80808080u;
+    }
     uint32_t o[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const uint32_t src = w[i / 2] >> (16 * (i & 1));
-        const float f0 = symbol_value<DT>(src & 0xFFu), f1 = symbol_value<DT>((src >> 8) & 0xFFu);
-        o[i] = pack_bf16x2(make_float2(f0, f1));
+        const uint32_t src = w[i / 2];
+        const uint32_t j = 2 * (i & 1);  // bytes j, j + 1 of the word
+        const float f0 = byte_value<DT>(src, j), f1 = byte_value<DT>(src, j + 1);
+        // upper halves of f0 (low bf16) and f1 (high bf16)
+        o[i] = prmt(__float_as_uint(f0), __float_as_uint(f1), 0x7632u);
     }
     lo = make_uint4(o[0], o[1], o[2], o[3]);
     hi = make_uint4(o[4], o[5], o[6], o[7]);
@@ -168,19 +203,31 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Warp-specialised mainloop: kProducerWarps warps fill a ring of kStages
+// shared-memory stages (token tile copied, symbol tile widened) and arrive on
+// the stage's "full" barrier (one arrival per warp); the MMA warp's first lane
+// waits for "full", issues the slab's 4 MMAs and commits them to the stage's
+// "empty" barrier, which the producers wait on before refilling the stage; a
+// final commit to "done" releases the epilogue.  No block-wide barrier runs
+// inside the loop.
 template <int DT>
-__global__ void __launch_bounds__(kGemmThreads) eq_gemm_symbols_kernel(const __grid_constant__ GemmParams P) {
+__global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(const __grid_constant__ GemmParams P) {
+    constexpr uint32_t kProducerWarps = kGemmThreads / 32;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t mbar_s[kStages];
+    __shared__ __align__(8) uint64_t full_s[kStages], empty_s[kStages], done_s;
     __shared__ uint32_t tmem_base_s;
     const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
+    const bool mma_warp = warp == kProducerWarps;
     const uint32_t n0 = blockIdx.x * kTileN;   // weight rows (outputs)
     const uint32_t m0 = blockIdx.y * kTileM;   // tokens
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    // stage s: A tile at base + s * (A + B bytes), B tile right after it; its mbarrier at mbar0 + 8 s
     auto bufA = [&](uint32_t st) { return base + st * (kStageBytesA + kStageBytesB); };
     auto bufB = [&](uint32_t st) { return base + st * (kStageBytesA + kStageBytesB) + kStageBytesA; };
-    const uint32_t mbar0 = smem_u32(&mbar_s[0]);
+    const uint32_t full0 = smem_u32(&full_s[0]), empty0 = smem_u32(&empty_s[0]), done = smem_u32(&done_s);
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -188,115 +235,112 @@ __global__ void __launch_bounds__(kGemmThreads) eq_gemm_symbols_kernel(const __g
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
-        for (uint32_t st = 0; st < kStages; ++st) mbar_init(mbar0 + 8 * st, 1);
+        for (uint32_t st = 0; st < kStages; ++st) {
+            mbar_init(full0 + 8 * st, kProducerWarps);
+            mbar_init(empty0 + 8 * st, 1);
+        }
+        mbar_init(done, 1);
         fence_mbar_init();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_s;
-
     const uint32_t n_slabs = P.cols / kTileK;
-    // per thread: kXv 16-byte chunks of the X tile and kBv of the symbol tile
-    constexpr uint32_t kXv = kTileM * (kTileK / 8) / kGemmThreads;
-    constexpr uint32_t kBv = kTileN * (kTileK / 16) / kGemmThreads;
-    uint4 xr[kXv], br[kBv];
-    // global -> registers for slab `it` (issued one slab ahead of its use)
-    auto fetch = [&](uint32_t it) {
-        const uint32_t k0 = it * kTileK;
-#pragma unroll
-        for (uint32_t i = 0; i < kXv; ++i) {
-            const uint32_t e = tid + i * kGemmThreads, r = e >> 3, k8 = e & 7u;
-            xr[i] = m0 + r < P.tokens
-                        ? __ldg(reinterpret_cast<const uint4 *>(P.x + (size_t)(m0 + r) * P.cols + k0) + k8)
-                        : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (uint32_t i = 0; i < kBv; ++i) {
-            const uint32_t e = tid + i * kGemmThreads, r = e >> 2, c = e & 3u;
-            br[i] = __ldg(reinterpret_cast<const uint4 *>(P.sym + (size_t)(n0 + r) * P.cols + k0) + c);
-        }
-    };
-    if (n_slabs) fetch(0);
     bool ok = true;
-    for (uint32_t it = 0; it < n_slabs && ok; ++it) {
-        const uint32_t s = it % kStages;
-        if (it >= kStages) {  // the MMAs that read this stage kStages slabs ago must be done
-            // commit number (it - kStages) / kStages of stage s, i.e. the completion of that parity
-            ok = mbar_wait_bounded(mbar0 + 8 * s, ((it - kStages) / kStages) & 1u);
-            if (!__syncthreads_and(ok)) {
+
+    if (!mma_warp) {
+        // per thread: kXv 16-byte chunks of the token tile and kBv of the symbol tile
+        constexpr uint32_t kXv = kTileM * (kTileK / 8) / kGemmThreads;
+        constexpr uint32_t kBv = kTileN * (kTileK / 16) / kGemmThreads;
+        uint4 xr[kXv], br[kBv];
+        auto fetch = [&](uint32_t it) {
+            const uint32_t k0 = it * kTileK;
+#pragma unroll
+            for (uint32_t i = 0; i < kXv; ++i) {
+                const uint32_t e = tid + i * kGemmThreads, r = e >> 3, k8 = e & 7u;
+                xr[i] = m0 + r < P.tokens
+                            ? __ldg(reinterpret_cast<const uint4 *>(P.x + (size_t)(m0 + r) * P.cols + k0) + k8)
+                            : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (uint32_t i = 0; i < kBv; ++i) {
+                const uint32_t e = tid + i * kGemmThreads, r = e >> 2, c = e & 3u;
+                br[i] = __ldg(reinterpret_cast<const uint4 *>(P.sym + (size_t)(n0 + r) * P.cols + k0) + c);
+            }
+        };
+        if (n_slabs) fetch(0);
+        for (uint32_t it = 0; it < n_slabs; ++it) {
+            const uint32_t s = it % kStages;
+            // stage s was last filled kStages slabs ago: wait until its MMAs are done
+            // (the decision is warp-uniform: the __syncwarp below needs every lane)
+            if (it >= kStages &&
+                !__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty0 + 8 * s, ((it - kStages) / kStages) & 1u))) {
                 ok = false;
                 break;
             }
-        }
-        // registers -> stage s: the X tile as is, the symbol tile widened to bf16
 #pragma unroll
-        for (uint32_t i = 0; i < kXv; ++i) {
-            const uint32_t e = tid + i * kGemmThreads;
-            st_shared_v4(bufA(s) + tile_offset(e >> 3, e & 7u), xr[i]);
-        }
+            for (uint32_t i = 0; i < kXv; ++i) {
+                const uint32_t e = tid + i * kGemmThreads;
+                st_shared_v4(bufA(s) + tile_offset(e >> 3, e & 7u), xr[i]);
+            }
 #pragma unroll
-        for (uint32_t i = 0; i < kBv; ++i) {
-            const uint32_t e = tid + i * kGemmThreads, r = e >> 2, c = e & 3u;
-            uint4 lo, hi;
-            widen16<DT>(br[i], lo, hi);
-            st_shared_v4(bufB(s) + tile_offset(r, 2 * c), lo);
-            st_shared_v4(bufB(s) + tile_offset(r, 2 * c + 1), hi);
+            for (uint32_t i = 0; i < kBv; ++i) {
+                const uint32_t e = tid + i * kGemmThreads, r = e >> 2, c = e & 3u;
+                uint4 lo, hi;
+                widen16<DT>(br[i], lo, hi);
+                st_shared_v4(bufB(s) + tile_offset(r, 2 * c), lo);
+                st_shared_v4(bufB(s) + tile_offset(r, 2 * c + 1), hi);
+            }
+            if (it + 1 < n_slabs) fetch(it + 1);  // in flight while the stage is consumed
+            fence_proxy_async_smem();              // generic-proxy stores -> visible to the tensor core
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full0 + 8 * s);
         }
-        if (it + 1 < n_slabs) fetch(it + 1);  // in flight during the barrier and the MMAs
-        fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
+    } else if (lane == 0) {
+        for (uint32_t it = 0; it < n_slabs; ++it) {
+            const uint32_t s = it % kStages;
+            if (!mbar_wait_bounded(full0 + 8 * s, (it / kStages) & 1u)) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
 #pragma unroll
-            for (uint32_t kk = 0; kk < kTileK / kMmaK; ++kk) {
-                const uint64_t db = tile_desc(bufB(s), kk);
-#pragma unroll
-                for (uint32_t h = 0; h < kHalves; ++h)  // token half h: A rows 128h.., accumulator columns 128h..
-                    tc_mma(tmem + h * kTileN, tile_desc(bufA(s) + h * (kMmaM * kTileK * 2), kk), db,
-                           (it | kk) != 0u);
-            }
-            tc_commit(mbar0 + 8 * s);
+            for (uint32_t kk = 0; kk < kTileK / kMmaK; ++kk)
+                tc_mma(tmem, tile_desc(bufA(s), kk), tile_desc(bufB(s), kk), (it | kk) != 0u);
+            tc_commit(empty0 + 8 * s);
         }
+        tc_commit(done);  // completes when every MMA issued above has
     }
-    // all MMAs done: the last commit of the last slab covers every earlier MMA of thread 0
-    if (ok && n_slabs) {
-        // the last commit of every stage (the very last one covers all MMAs of thread 0)
-        for (uint32_t j = 0; j < kStages && j < n_slabs && ok; ++j) {
-            const uint32_t it = n_slabs - 1 - j;
-            ok = mbar_wait_bounded(mbar0 + 8 * (it % kStages), (it / kStages) & 1u);
-        }
-        ok = __syncthreads_and(ok);
-    }
-    tc_fence_after();
-    if (ok) {
-        // warp w may read accumulator lanes 32 (w % 4) .. + 31; the warps that
-        // share a lane quarter split the accumulator columns (kHalves x 128)
-        constexpr uint32_t kWarps = kGemmThreads / 32, kColsPerWarp = kTmemCols * 4 / kWarps;
-        const uint32_t quarter = warp & 3u, c_first = (warp >> 2) * (kColsPerWarp / 32);
+    if (!mma_warp) {
+        ok = mbar_wait_bounded(done, 0u) && ok;
+        tc_fence_after();
+        if (__all_sync(0xFFFFFFFFu, ok)) {
+            // warp w reads accumulator lanes 32 (w % 4) .. + 31; warps sharing a
+            // lane quarter split the 128 columns
+            constexpr uint32_t kColsPerWarp = kTmemCols * 4 / kProducerWarps;
+            const uint32_t quarter = warp & 3u, c_first = (warp >> 2) * (kColsPerWarp / 32);
+            const uint32_t m = m0 + quarter * 32u + lane;
 #pragma unroll 1
-        for (uint32_t c = c_first; c < c_first + kColsPerWarp / 32; ++c) {
-            const uint32_t h = c / (kTileN / 32), cn = c % (kTileN / 32);  // token half, column chunk
-            const uint32_t m = m0 + h * kMmaM + quarter * 32u + lane;
-            uint32_t r[32];
-            tmem_ld32(tmem + ((quarter * 32u) << 16) + c * 32u, r);
-            if (m < P.tokens) {
-                float4 *dst = reinterpret_cast<float4 *>(P.y + (size_t)m * P.rows + n0 + cn * 32u);
-                const float4 *sc = reinterpret_cast<const float4 *>(P.scales + n0 + cn * 32u);
+            for (uint32_t c = c_first; c < c_first + kColsPerWarp / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tmem + ((quarter * 32u) << 16) + c * 32u, r);
+                if (m < P.tokens) {
+                    float4 *dst = reinterpret_cast<float4 *>(P.y + (size_t)m * P.rows + n0 + c * 32u);
+                    const float4 *sc = reinterpret_cast<const float4 *>(P.scales + n0 + c * 32u);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 s4 = __ldg(sc + q);
-                    dst[q] = make_float4(__fmul_rn(__uint_as_float(r[4 * q]), s4.x),
-                                         __fmul_rn(__uint_as_float(r[4 * q + 1]), s4.y),
-                                         __fmul_rn(__uint_as_float(r[4 * q + 2]), s4.z),
-                                         __fmul_rn(__uint_as_float(r[4 * q + 3]), s4.w));
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 s4 = __ldg(sc + q);
+                        dst[q] = make_float4(__fmul_rn(__uint_as_float(r[4 * q]), s4.x),
+                                             __fmul_rn(__uint_as_float(r[4 * q + 1]), s4.y),
+                                             __fmul_rn(__uint_as_float(r[4 * q + 2]), s4.z),
+                                             __fmul_rn(__uint_as_float(r[4 * q + 3]), s4.w));
+                    }
                 }
             }
         }
-    } else if (tid == 0) {
-        atomicOr(P.status, EQ_DEV_TIMEOUT);
     }
+    if (!ok) atomicOr(P.status, EQ_DEV_TIMEOUT);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -358,7 +402,7 @@ extern "C" EQW_API int eq_gemm_symbols(const eq_model *m, uint32_t matrix, const
         attr = true;
     }
     const dim3 grid(in.rows / kTileN, (tokens + kTileM - 1) / kTileM);
-    fn<<<grid, kGemmThreads, kGemmSmem, s>>>(P);
+    fn<<<grid, kGemmThreads + 32, kGemmSmem, s>>>(P);
     if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
     if (in.n_outliers) {
         const uint64_t n = (uint64_t)in.n_outliers * tokens;
