@@ -16,13 +16,15 @@
 //
 // Kernel eq_gemm_symbols_kernel, one CTA per 128 x 128 output tile, 8
 // producer warps and one MMA warp:
-//   producers  per K slab of 64: copy the token tile (16-byte loads,
-//              prefetched one slab ahead into registers) and widen the symbol
-//              tile into a shared-memory stage in the 128-byte-swizzled
-//              K-major layout (16-byte chunk c of row r at chunk position
-//              c ^ (r % 8), 8-row groups 1024 B apart); arrive on the stage's
-//              "full" mbarrier; refill a stage once its "empty" barrier says
-//              the tensor core is done with it (a ring of 3 stages)
+//   producers  per K slab of 64: cp.async copies of the token tile straight
+//              into the 128-byte-swizzled K-major layout (16-byte chunk c of
+//              row r at chunk position c ^ (r % 8), 8-row groups 1024 B
+//              apart) and of the symbol bytes into a staging area, issued
+//              kAhead slabs ahead into a ring of kStages stages; once a
+//              thread's copies of a slab have landed it widens its own symbol
+//              chunks into the swizzled bf16 tile and its warp arrives on the
+//              stage's "full" mbarrier; a stage is refilled only after its
+//              "empty" barrier says the tensor core is done with it
 //   MMA warp   one lane waits for "full", issues 4 x tcgen05.mma (M 128,
 //              N 128, K 16, fp32 accumulator in 128 TMEM columns) and
 //              tcgen05.commit to the stage's "empty" barrier; a last commit
@@ -52,7 +54,7 @@ constexpr int kGemmThreads = EQ_GEMM_THREADS;  // 4 or 8 warps
 #define EQ_GEMM_HALVES 1
 #endif
 #ifndef EQ_GEMM_STAGES
-#define EQ_GEMM_STAGES 3
+#define EQ_GEMM_STAGES 4
 #endif
 static_assert(EQ_GEMM_HALVES == 1, "two token halves per CTA faulted on the GPU and are not used");
 constexpr uint32_t kMmaM = 128;                        // tokens per MMA (accumulator lanes)
@@ -64,8 +66,15 @@ constexpr uint32_t kMmaK = 16;                         // K per tcgen05.mma (bf1
 constexpr uint32_t kStageBytesA = kTileM * kTileK * 2;  // 16 KiB per 128 tokens
 constexpr uint32_t kStageBytesB = kTileN * kTileK * 2;  // 16 KiB
 constexpr uint32_t kStages = EQ_GEMM_STAGES;
+#ifndef EQ_GEMM_AHEAD
+#define EQ_GEMM_AHEAD 2
+#endif
+constexpr uint32_t kAhead = EQ_GEMM_AHEAD;              // slabs whose copies are in flight ahead of use
+static_assert(kAhead < kStages, "a stage is refilled only after its previous slab's MMAs");
+constexpr uint32_t kStageBytesS = kTileN * kTileK;      // 8 KiB of symbol bytes (staging)
+constexpr uint32_t kStageBytes = kStageBytesA + kStageBytesB + kStageBytesS;
 constexpr uint32_t kTmemCols = kTileN * kHalves;        // one fp32 accumulator per token half
-constexpr size_t kGemmSmem = kStages * (kStageBytesA + kStageBytesB) + 1024;
+constexpr size_t kGemmSmem = kStages * kStageBytes + 1024;
 
 struct GemmParams {
     const uint16_t *x;        // bf16 [tokens, cols]
@@ -203,6 +212,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 16-byte asynchronous copy global -> shared (src_bytes 0: zero fill).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -225,8 +248,10 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
     const uint32_t n0 = blockIdx.x * kTileN;   // weight rows (outputs)
     const uint32_t m0 = blockIdx.y * kTileM;   // tokens
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    auto bufA = [&](uint32_t st) { return base + st * (kStageBytesA + kStageBytesB); };
-    auto bufB = [&](uint32_t st) { return base + st * (kStageBytesA + kStageBytesB) + kStageBytesA; };
+    // stage st: token tile (swizzled bf16), widened symbol tile (swizzled bf16), symbol bytes (staging)
+    auto bufA = [&](uint32_t st) { return base + st * kStageBytes; };
+    auto bufB = [&](uint32_t st) { return base + st * kStageBytes + kStageBytesA; };
+    auto bufS = [&](uint32_t st) { return base + st * kStageBytes + kStageBytesA + kStageBytesB; };
     const uint32_t full0 = smem_u32(&full_s[0]), empty0 = smem_u32(&empty_s[0]), done = smem_u32(&done_s);
 
     if (warp == 0) {
@@ -253,50 +278,57 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
         // per thread: kXv 16-byte chunks of the token tile and kBv of the symbol tile
         constexpr uint32_t kXv = kTileM * (kTileK / 8) / kGemmThreads;
         constexpr uint32_t kBv = kTileN * (kTileK / 16) / kGemmThreads;
-        uint4 xr[kXv], br[kBv];
-        auto fetch = [&](uint32_t it) {
+        // this thread's copies of slab `it` into stage `st`
+        auto issue = [&](uint32_t it, uint32_t st) {
             const uint32_t k0 = it * kTileK;
 #pragma unroll
             for (uint32_t i = 0; i < kXv; ++i) {
                 const uint32_t e = tid + i * kGemmThreads, r = e >> 3, k8 = e & 7u;
-                xr[i] = m0 + r < P.tokens
-                            ? __ldg(reinterpret_cast<const uint4 *>(P.x + (size_t)(m0 + r) * P.cols + k0) + k8)
-                            : make_uint4(0, 0, 0, 0);
+                const bool in = m0 + r < P.tokens;
+                const uint16_t *src = in ? P.x + (size_t)(m0 + r) * P.cols + k0 + 8 * k8 : P.x;
+                cp_async16(bufA(st) + tile_offset(r, k8), src, in ? 16u : 0u);
             }
 #pragma unroll
             for (uint32_t i = 0; i < kBv; ++i) {
                 const uint32_t e = tid + i * kGemmThreads, r = e >> 2, c = e & 3u;
-                br[i] = __ldg(reinterpret_cast<const uint4 *>(P.sym + (size_t)(n0 + r) * P.cols + k0) + c);
+                cp_async16(bufS(st) + e * 16u, P.sym + (size_t)(n0 + r) * P.cols + k0 + 16 * c, 16u);
             }
         };
-        if (n_slabs) fetch(0);
+        // the first kAhead slabs go to stages that start out free
+        for (uint32_t it = 0; it < kAhead; ++it) {
+            if (it < n_slabs) issue(it, it % kStages);
+            cp_async_commit();
+        }
         for (uint32_t it = 0; it < n_slabs; ++it) {
             const uint32_t s = it % kStages;
-            // stage s was last filled kStages slabs ago: wait until its MMAs are done
-            // (the decision is warp-uniform: the __syncwarp below needs every lane)
-            if (it >= kStages &&
-                !__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty0 + 8 * s, ((it - kStages) / kStages) & 1u))) {
-                ok = false;
-                break;
+            const uint32_t ahead = it + kAhead;
+            if (ahead < n_slabs) {
+                const uint32_t sa = ahead % kStages;
+                // stage sa last held slab ahead - kStages: wait until its MMAs are done
+                // (the decision is warp-uniform: the __syncwarp below needs every lane)
+                if (ahead >= kStages &&
+                    !__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty0 + 8 * sa, ((ahead - kStages) / kStages) & 1u))) {
+                    ok = false;
+                    break;
+                }
+                issue(ahead, sa);
             }
-#pragma unroll
-            for (uint32_t i = 0; i < kXv; ++i) {
-                const uint32_t e = tid + i * kGemmThreads;
-                st_shared_v4(bufA(s) + tile_offset(e >> 3, e & 7u), xr[i]);
-            }
+            cp_async_commit();            // one group per slab, empty past the end
+            cp_async_wait<kAhead>();      // this thread's copies of slab `it` have landed
+            // widen this thread's own symbol chunks of slab `it`
 #pragma unroll
             for (uint32_t i = 0; i < kBv; ++i) {
                 const uint32_t e = tid + i * kGemmThreads, r = e >> 2, c = e & 3u;
                 uint4 lo, hi;
-                widen16<DT>(br[i], lo, hi);
+                widen16<DT>(ld_shared_v4(bufS(s) + e * 16u), lo, hi);
                 st_shared_v4(bufB(s) + tile_offset(r, 2 * c), lo);
                 st_shared_v4(bufB(s) + tile_offset(r, 2 * c + 1), hi);
             }
-            if (it + 1 < n_slabs) fetch(it + 1);  // in flight while the stage is consumed
-            fence_proxy_async_smem();              // generic-proxy stores -> visible to the tensor core
+            fence_proxy_async_smem();  // copies and stores -> visible to the tensor core
             __syncwarp();
             if (lane == 0) mbar_arrive(full0 + 8 * s);
         }
+        cp_async_wait<0>();
     } else if (lane == 0) {
         for (uint32_t it = 0; it < n_slabs; ++it) {
             const uint32_t s = it % kStages;
