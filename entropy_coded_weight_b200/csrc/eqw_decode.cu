@@ -245,83 +245,88 @@ struct Chain {
     uint16_t *dst;
 };
 
-// Two 256-symbol groups in rank mode, one per chain, interleaved step by step.
-template <uint32_t CODEC>
-__device__ __forceinline__ void group2_rank(uint32_t lut, uint32_t ringA, uint32_t ringB, Chain<CODEC> &A, Chain<CODEC> &B,
+// One 256-symbol group of each of the C chains in rank mode, interleaved
+// step by step (chain 0, 1, ..., C-1 for every step).
+template <uint32_t CODEC, uint32_t C>
+__device__ __forceinline__ void groupN_rank(uint32_t lut, const uint32_t (&ring)[C], Chain<CODEC> (&ch)[C],
                                             uint32_t lt) {
-    const uint32_t a0 = ringA + (A.pw & (kRingBytes - 1));
-    const uint32_t b0 = ringB + (B.pw & (kRingBytes - 1));
-    uint32_t ra = a0, rb = b0;
-    uint32_t oa[4], ob[4];
+    uint32_t r0[C], rp[C], o[C][4];
+#pragma unroll
+    for (uint32_t c = 0; c < C; ++c) rp[c] = r0[c] = ring[c] + (ch[c].pw & (kRingBytes - 1));
 #pragma unroll
     for (int r = 0; r < 8; r += 2) {
-        const uint32_t ea0 = codec_step<CODEC>(lut, ra, A.x, lt);
-        const uint32_t eb0 = codec_step<CODEC>(lut, rb, B.x, lt);
-        const uint32_t ea1 = codec_step<CODEC>(lut, ra, A.x, lt);
-        const uint32_t eb1 = codec_step<CODEC>(lut, rb, B.x, lt);
-        oa[r / 2] = pack_bf16x2(make_float2(__shfl_sync(kFull, A.vr, ea0), __shfl_sync(kFull, A.vr, ea1)));
-        ob[r / 2] = pack_bf16x2(make_float2(__shfl_sync(kFull, B.vr, eb0), __shfl_sync(kFull, B.vr, eb1)));
+        uint32_t e0[C], e1[C];
+#pragma unroll
+        for (uint32_t c = 0; c < C; ++c) e0[c] = codec_step<CODEC>(lut, rp[c], ch[c].x, lt);
+#pragma unroll
+        for (uint32_t c = 0; c < C; ++c) e1[c] = codec_step<CODEC>(lut, rp[c], ch[c].x, lt);
+#pragma unroll
+        for (uint32_t c = 0; c < C; ++c)
+            o[c][r / 2] = pack_bf16x2(make_float2(__shfl_sync(kFull, ch[c].vr, e0[c]),
+                                                  __shfl_sync(kFull, ch[c].vr, e1[c])));
     }
-    st_global_v4(A.dst, make_uint4(oa[0], oa[1], oa[2], oa[3]));
-    st_global_v4(B.dst, make_uint4(ob[0], ob[1], ob[2], ob[3]));
-    A.pw += ra - a0;
-    B.pw += rb - b0;
-    A.dst += kGroupSyms;
-    B.dst += kGroupSyms;
+#pragma unroll
+    for (uint32_t c = 0; c < C; ++c) {
+        st_global_v4(ch[c].dst, make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]));
+        ch[c].pw += rp[c] - r0[c];
+        ch[c].dst += kGroupSyms;
+    }
 }
 
-template <int DT, uint32_t CODEC>
-__device__ __forceinline__ bool decode_pair(int32_t *status, const OutCtx &O, const ChunkHead &hA,
-                                            const ChunkHead &hB, uint64_t firstA, uint64_t firstB, uint32_t lut,
-                                            uint32_t ringA, uint32_t ringB, uint32_t mbarA, uint32_t mbarB,
-                                            RingCtl *ctlA, RingCtl *ctlB, uint32_t lane, uint32_t lt,
-                                            uint32_t lane_sym) {
-    ring_start(ctlA, hA);
-    ring_start(ctlB, hB);
+// C full chunks per warp in lockstep (rank mode, row-uniform layout, every
+// chunk 65536 symbols, cols a multiple of 512): C independent state chains
+// whose latencies overlap.  Row changes fall between pairs of groups.
+template <int DT, uint32_t CODEC, uint32_t C>
+__device__ __forceinline__ bool decode_multi(int32_t *status, const OutCtx &O, const ChunkHead (&h)[C],
+                                             const uint64_t (&first)[C], uint32_t lut, const uint32_t (&ring)[C],
+                                             const uint32_t (&mbar)[C], RingCtl *ctl, uint32_t lane, uint32_t lt,
+                                             uint32_t lane_sym) {
+#pragma unroll
+    for (uint32_t c = 0; c < C; ++c) ring_start(ctl + c, h[c]);
     __syncwarp();
     const float vraw = symbol_value<DT>(lane_sym);
-    Chain<CODEC> A, B;
-    A.x = codec_start<CODEC>(hA.x);
-    B.x = codec_start<CODEC>(hB.x);
-    A.pw = B.pw = 0;
-    A.limit = hA.n_words ? 0u : kNoLimit;
-    B.limit = hB.n_words ? 0u : kNoLimit;
-    A.row = (uint32_t)(firstA / O.cols);
-    A.col = (uint32_t)(firstA - (uint64_t)A.row * O.cols);
-    B.row = (uint32_t)(firstB / O.cols);
-    B.col = (uint32_t)(firstB - (uint64_t)B.row * O.cols);
-    A.vr = __fmul_rn(vraw, __ldg(O.scales + A.row));
-    B.vr = __fmul_rn(vraw, __ldg(O.scales + B.row));
-    A.dst = O.out + firstA + kGroup * lane;
-    B.dst = O.out + firstB + kGroup * lane;
+    Chain<CODEC> ch[C];
+#pragma unroll
+    for (uint32_t c = 0; c < C; ++c) {
+        ch[c].x = codec_start<CODEC>(h[c].x);
+        ch[c].pw = 0;
+        ch[c].limit = h[c].n_words ? 0u : kNoLimit;
+        ch[c].row = (uint32_t)(first[c] / O.cols);
+        ch[c].col = (uint32_t)(first[c] - (uint64_t)ch[c].row * O.cols);
+        ch[c].vr = __fmul_rn(vraw, __ldg(O.scales + ch[c].row));
+        ch[c].dst = O.out + first[c] + kGroup * lane;
+    }
     constexpr uint32_t kPairs = kChunkSyms / (2 * kGroupSyms);
     for (uint32_t q = 0; q < kPairs; ++q) {
-        if (A.pw >= A.limit) A.limit = ring_service(ctlA, ringA, mbarA, A.pw);
-        if (B.pw >= B.limit) B.limit = ring_service(ctlB, ringB, mbarB, B.pw);
-        if (ctlA->dead || ctlB->dead) break;
-        group2_rank(lut, ringA, ringB, A, B, lt);
-        group2_rank(lut, ringA, ringB, A, B, lt);
-        A.col += 2 * kGroupSyms;
-        if (A.col == O.cols) {
-            A.col = 0;
-            ++A.row;
-            if (A.row < O.rows) A.vr = __fmul_rn(vraw, __ldg(O.scales + A.row));
+        bool dead = false;
+#pragma unroll
+        for (uint32_t c = 0; c < C; ++c) {
+            if (ch[c].pw >= ch[c].limit) ch[c].limit = ring_service(ctl + c, ring[c], mbar[c], ch[c].pw);
+            dead = dead || ctl[c].dead;
         }
-        B.col += 2 * kGroupSyms;
-        if (B.col == O.cols) {
-            B.col = 0;
-            ++B.row;
-            if (B.row < O.rows) B.vr = __fmul_rn(vraw, __ldg(O.scales + B.row));
+        if (dead) break;
+        groupN_rank<CODEC, C>(lut, ring, ch, lt);
+        groupN_rank<CODEC, C>(lut, ring, ch, lt);
+#pragma unroll
+        for (uint32_t c = 0; c < C; ++c) {
+            ch[c].col += 2 * kGroupSyms;
+            if (ch[c].col == O.cols) {
+                ch[c].col = 0;
+                ++ch[c].row;
+                if (ch[c].row < O.rows) ch[c].vr = __fmul_rn(vraw, __ldg(O.scales + ch[c].row));
+            }
         }
     }
-    const bool okA = ring_drain(ctlA, mbarA);
-    const bool okB = ring_drain(ctlB, mbarB);
-    if (!okA || !okB) {
+    bool drained = true;
+#pragma unroll
+    for (uint32_t c = 0; c < C; ++c) drained = ring_drain(ctl + c, mbar[c]) && drained;
+    if (!drained) {
         flag(status, EQ_DEV_TIMEOUT);
         return false;
     }
-    if (!__all_sync(kFull, codec_done(A.x)) || A.pw != 2u * hA.n_words) flag(status, EQ_DEV_BAD_END);
-    if (!__all_sync(kFull, codec_done(B.x)) || B.pw != 2u * hB.n_words) flag(status, EQ_DEV_BAD_END);
+#pragma unroll
+    for (uint32_t c = 0; c < C; ++c)
+        if (!__all_sync(kFull, codec_done(ch[c].x)) || ch[c].pw != 2u * h[c].n_words) flag(status, EQ_DEV_BAD_END);
     return true;
 }
 
@@ -546,13 +551,20 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
                 if (have[c]) have[c] = shared_chunk_head<CODEC>(P, M, k, lane, np, S, hc[c]);
             }
             const OutCtx O = out_ctx(M);
-            if constexpr (C == 2 && LAYOUT == kRowUniform) {
-                if (have[0] && have[1] && rank_mode<LAYOUT>(np) && hc[0].n == kChunkSyms &&
-                    hc[1].n == kChunkSyms && O.cols % (2 * kGroupSyms) == 0) {
-                    decode_pair<DT, CODEC>(P.status, O, hc[0], hc[1], (uint64_t)(k0 + warp) * kChunkSyms,
-                                    (uint64_t)(k0 + warp + WARPS) * kChunkSyms, S.lut_addr, S.ring,
-                                    S.ring + kRingStride, S.mbar, S.mbar + 8 * kRingSegs, ctl, ctl + 1, lane, lt,
-                                    lane_sym);
+            if constexpr (C >= 2 && LAYOUT == kRowUniform) {
+                bool all_full = rank_mode<LAYOUT>(np) && O.cols % (2 * kGroupSyms) == 0;
+                for (uint32_t c = 0; c < C; ++c) all_full = all_full && have[c] && hc[c].n == kChunkSyms;
+                if (all_full) {
+                    uint64_t first[C];
+                    uint32_t rings[C], mbars[C];
+#pragma unroll
+                    for (uint32_t c = 0; c < C; ++c) {
+                        first[c] = (uint64_t)(k0 + warp + c * WARPS) * kChunkSyms;
+                        rings[c] = S.ring + c * kRingStride;
+                        mbars[c] = S.mbar + 8 * kRingSegs * c;
+                    }
+                    decode_multi<DT, CODEC, C>(P.status, O, hc, first, S.lut_addr, rings, mbars, ctl, lane, lt,
+                                               lane_sym);
                     __syncwarp();
                     continue;
                 }
