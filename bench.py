@@ -344,34 +344,34 @@ def isolated_launches(stack, n: int, dev) -> list[float]:
     return [a.elapsed_time(b) for a, b in pairs]
 
 
-def cpu_oracle_sample(blob: np.ndarray, target_s: float = 12.0) -> dict:
-    """The CPU oracle (scalar rANS decode + dequant) on a bounded sample of chunks, all host cores."""
+def oracle_rate(blob: np.ndarray, threads: int, target_s: float, layer: int = 0) -> tuple[int, int, float, int]:
+    """The CPU oracle (scalar rANS or Huffman decode + dequant) on chunks of one
+    layer, in a seeded random order, ``threads`` at a time, until at least
+    ``target_s`` of wall time has passed.  Returns (symbols, chunks, seconds,
+    chunks in the layer)."""
     import oracle
     from concurrent.futures import ThreadPoolExecutor
-    cores = len(os.sched_getaffinity(0))
     parsed = oracle.parse_container(blob)
-    chunks = []
-    for mi, m in enumerate(parsed["matrices"]):
-        if m["layer"] != 0:
-            continue
-        for k in range(m["n_chunks"]):
-            chunks.append((mi, k))
+    chunks = [(mi, k) for mi, m in enumerate(parsed["matrices"]) if m["layer"] == layer
+              for k in range(m["n_chunks"])]
+    chunks = [chunks[i] for i in np.random.default_rng(0).permutation(len(chunks))]
 
     def one(job):
         mi, k = job
         m = parsed["matrices"][mi]
         n = m["rows"] * m["cols"]
         cnt = min(oracle.CHUNK_SYMS, n - k * oracle.CHUNK_SYMS)
-        sym = oracle._decode_record(parsed["blob"], int(m["chunk_offsets"][k]), int(m["chunk_offsets"][k + 1]), cnt)
+        sym = oracle._decode_record(parsed["blob"], int(m["chunk_offsets"][k]), int(m["chunk_offsets"][k + 1]), cnt,
+                                    m.get("codec", oracle.CODEC_RANS))
         first = k * oracle.CHUNK_SYMS
         rows = np.arange(first, first + cnt) // m["cols"]
         oracle.dequant_pairs(m["dtype"], sym, m["scales"][rows])
         return cnt
 
-    # batches of 4 chunks per core until at least target_s of wall time has passed
-    batch = 4 * cores
+    # batches of 4 chunks per thread until at least target_s of wall time has passed
+    batch = 4 * threads
     done, n_sample, pos = 0, 0, 0
-    with ThreadPoolExecutor(cores) as ex:
+    with ThreadPoolExecutor(threads) as ex:
         t0 = time.perf_counter()
         while True:
             sample = [chunks[(pos + i) % len(chunks)] for i in range(batch)]
@@ -381,11 +381,17 @@ def cpu_oracle_sample(blob: np.ndarray, target_s: float = 12.0) -> dict:
             dt = time.perf_counter() - t0
             if dt >= target_s:
                 break
-    sample = range(n_sample)
+    return done, n_sample, dt, len(chunks)
+
+
+def cpu_oracle_sample(blob: np.ndarray, target_s: float = 12.0) -> dict:
+    """The CPU oracle (scalar rANS decode + dequant) on a bounded sample of chunks, all host cores."""
+    cores = len(os.sched_getaffinity(0))
+    done, n_sample, dt, n_chunks = oracle_rate(blob, cores, target_s)
     return {"value": round(2.0 * done / dt / 1e9, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{len(sample)} chunks ({done} symbols, cycling over the {len(chunks)} chunks of layer 0), "
-                      f"scalar rANS decode + dequant, "
-                      f"{cores} threads, {dt:.1f}s", "gsym_s": round(done / dt / 1e9, 5)}
+            "sample": f"{n_sample} chunks ({done} symbols, cycling over the {n_chunks} chunks of layer 0 "
+                      f"in a seeded order), scalar rANS decode + dequant, {cores} threads, {dt:.1f}s",
+            "gsym_s": round(done / dt / 1e9, 5)}
 
 
 def bench_eqw(args, d: Dist) -> dict | None:
@@ -460,6 +466,11 @@ def bench_eqw(args, d: Dist) -> dict | None:
                 "rans_launch_ms": round(launch_ms, 4),
                 "note": "layer 0 Huffman-coded (canonical codes <= 12 bits) and decoded by eq_decode_kernel's "
                         "Huffman instance, launches timed alone; bits/sym incl. tables and chunk index"}
+        if not args.no_cpu_baseline and d.world == 1:
+            # the multi-threaded CPU decode of the same chunks (the oracle's bit-serial Huffman decoder)
+            hs, hn, ht, _ = oracle_rate(hblob, threads, 4.0)
+            huff["cpu_oracle"] = {"value": round(2.0 * hs / ht / 1e9, 4), "unit": UNIT, "cores": threads,
+                                  "sample": f"{hn} chunks of layer 0, {ht:.1f}s"}
         hstack.close()
         del hblob
 
@@ -609,6 +620,172 @@ def bench_eqw(args, d: Dist) -> dict | None:
     }
 
 
+# ---------------------------------------------------------------------------
+# per-workload table: workloads 1-4 one block at a time, workload 5's stream parity
+# ---------------------------------------------------------------------------
+
+def _config_rows():
+    import workloads as W
+    return (
+        ("1", "single 1024x1024 Int8 matrix, ~2.1 bits/sym", lambda t: W.single_matrix(2.1)),
+        ("2a", "Llama-7B-shape block, Int8 ~2.1 bits/sym", lambda t: W.llama7b_int8_block(2.1, threads=t)),
+        ("2b", "Llama-7B-shape block, Int8 ~3.0 bits/sym", lambda t: W.llama7b_int8_block(3.0, threads=t)),
+        ("3", "Llama-70B-shape block, E4M3 ~2.1 bits/sym", lambda t: W.llama70b_e4m3_block(2.1, threads=t)),
+        ("4", "Llama-7B-shape block, Int8 ~2.5 bits/sym, 16 outliers in down",
+         lambda t: W.llama7b_int8_block_with_outliers(threads=t)),
+    )
+
+
+def _block_launches(model, layer: int, n: int, dev, flush=None) -> list[float]:
+    """n decodes of one block, each bracketed by CUDA events on its stream; with
+    ``flush`` (a buffer larger than L2) rewritten before each, outside the bracket."""
+    import torch
+    s = torch.cuda.Stream(device=dev)
+    buf = torch.empty(model.block_bytes(layer), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    pairs = []
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        for i in range(n):
+            if flush is not None:
+                flush.fill_(i & 0xFF)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            model.decode_block(layer, buf, status, s)
+            b.record(s)
+            pairs.append((a, b))
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"decode status {int(status.item())}")
+    return [a.elapsed_time(b) for a, b in pairs]
+
+
+def _checksums_host(bits: np.ndarray) -> np.ndarray:
+    """(sum, row-weighted sum, column-weighted sum) of a uint16 [rows, cols] matrix, exact in int64."""
+    v = bits.astype(np.int64)
+    rows, cols = v.shape
+    return np.array([v.sum(), (v.sum(1) * np.arange(1, rows + 1)).sum(), (v.sum(0) * np.arange(1, cols + 1)).sum()],
+                    np.int64)
+
+
+def _checksums_device(w):
+    import torch
+    v = w.view(torch.int16).to(torch.int64) & 0xFFFF
+    rows, cols = v.shape
+    r = torch.arange(1, rows + 1, device=v.device, dtype=torch.int64)
+    c = torch.arange(1, cols + 1, device=v.device, dtype=torch.int64)
+    return torch.stack([v.sum(), (v.sum(1) * r).sum(), (v.sum(0) * c).sum()])
+
+
+def bench_configs(args) -> None:
+    """One JSON line per workload: decode throughput of one block per launch
+    (inputs in HBM, L2 rewritten between launches), compression, bit-exactness
+    of the whole block against the oracle, and the oracle's own rate on 1 and
+    on all host cores (bounded samples).  Then the streamed 80-layer model's
+    parity: every block that the ping-pong loop hands its consumer is
+    checksummed on the device and compared with the oracle's, and four layers
+    are compared element by element."""
+    import torch
+
+    import entropy_coded_weight_b200 as E
+    import oracle
+    from entropy_coded_weight_b200.streamer import PingPongStreamer
+    import workloads as W
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cores = len(os.sched_getaffinity(0))
+    peak, peak_kind = measured_hbm_peak()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 2 x L2
+    for key, name, make in _config_rows():
+        mats = make(cores)
+        n = sum(m.n for m in mats)
+        blob = E.encode_host(mats, n_threads=cores)
+        model = E.Model(E.upload(blob, dev), blob)
+        infos = [model.info(i) for i in model.layer_matrices(0)]
+        records = sum(i.compressed_bytes for i in infos)
+        read = records + sum(8 * (i.n_chunks + 1) + 4 * i.rows + 12 * i.n_outliers for i in infos)
+        write = 2 * n + sum(2 * i.n_outliers for i in infos)
+        # parity: the whole decoded block against the oracle's direct dequant + scatter
+        offs, total = model.block_layout(0)
+        out = torch.empty(total, dtype=torch.uint8, device=dev)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        model.decode_block(0, out, status)
+        torch.cuda.synchronize()
+        host = out.cpu().numpy()
+        exact = int(status.item()) == 0
+        for m, o in zip(mats, offs):
+            got = host[o:o + 2 * m.n].view(np.uint16).reshape(m.rows, m.cols)
+            exact = exact and bool(np.array_equal(got, oracle.dequant_direct(m, threads=cores)))
+        del host, out
+        lines = {}
+        flushed = _block_launches(model, 0, args.warmup + args.steps, dev, flush)[args.warmup:]
+        lines["l2_flushed"] = statistics.mean(flushed)
+        if key == "1":
+            hot = _block_launches(model, 0, args.warmup + 10 * args.steps, dev)[args.warmup:]
+            lines["hot"] = statistics.mean(hot)
+        s1, _, t1, _ = oracle_rate(blob, 1, 3.0)
+        sa, _, ta, _ = oracle_rate(blob, cores, 3.0)
+        row = {"config": key, "workload": name, "symbols": n, "matrices": len(mats),
+               "bits_per_sym_records": round(8.0 * records / n, 4),
+               "bits_per_sym_container": round(8.0 * blob.size / n, 4),
+               "empirical_entropy_bits": round(float(np.mean([W.empirical_entropy_bits(m.symbols) for m in mats])), 4),
+               "bit_exact": exact}
+        for kind, ms in lines.items():
+            row[kind] = {"launch_ms": round(ms, 5), "decoded_gb_s": round(2.0 * n / (ms / 1e3) / 1e9, 1),
+                         "gsym_s": round(n / (ms / 1e3) / 1e9, 2),
+                         "hbm_frac": round((read + write) / (ms / 1e3) / 1e9 / peak, 4)}
+        row["oracle"] = {"gsym_s_1core": round(s1 / t1 / 1e9, 5), "gsym_s_all": round(sa / ta / 1e9, 5),
+                         "cores": cores, "sample_s": [round(t1, 1), round(ta, 1)]}
+        row["peak"] = {"hbm_gbs": peak, "kind": peak_kind}
+        print(json.dumps(row), flush=True)
+        model.close()
+        del mats, blob, model
+
+    # workload 5: the streamed model; every block checksummed as the consumer sees it
+    distinct = args.distinct_layers
+    blob, _ = build_blob(distinct, cores, dev)
+    stack = ResidentStack(blob, distinct, dev, args.layers)
+    streamer = PingPongStreamer(stack.steps, dev)
+    sums = torch.zeros(len(stack.steps), 7, 3, dtype=torch.int64, device=dev)
+
+    def consumer(i, step, views, stream):
+        for j, w in enumerate(views):
+            sums[i, j] = _checksums_device(w)
+
+    run_pass(streamer, consumer)
+    streamer.join()
+    torch.cuda.synchronize()
+    ok_status = int(streamer.status.item()) == 0
+    got = sums.cpu().numpy()
+    want = np.zeros((distinct, 7, 3), np.int64)
+    full = []
+    for layer in range(distinct):
+        mats = W.llama70b_int8_layer(layer, 2.1, threads=cores)
+        direct = [oracle.dequant_direct(m, threads=cores) for m in mats]
+        for j, w in enumerate(direct):
+            want[layer, j] = _checksums_host(w)
+        if layer < 4:  # element by element: block decoded on its own, copied back
+            st = next(s for s in stack.steps if s.layer == layer)
+            offs, total = st.model.block_layout(layer)
+            out = torch.empty(total, dtype=torch.uint8, device=dev)
+            status = torch.zeros(1, dtype=torch.int32, device=dev)
+            st.model.decode_block(layer, out, status)
+            torch.cuda.synchronize()
+            host = out.cpu().numpy()
+            full.append(int(status.item()) == 0 and all(
+                np.array_equal(host[o:o + 2 * m.n].view(np.uint16).reshape(m.rows, m.cols), w)
+                for m, o, w in zip(mats, offs, direct)))
+            del out, host
+        del mats, direct
+    match = [bool(np.array_equal(got[i], want[i % distinct])) for i in range(len(stack.steps))]
+    print(json.dumps({"config": "5", "workload": f"streamed {args.layers}-layer Llama-70B-shape model, Int8 ~2.1 bits/sym "
+                                                  f"({distinct} distinct layers)",
+                      "stream_status_ok": ok_status, "blocks_checksum_equal": f"{sum(match)}/{len(match)}",
+                      "layers_compared_in_full": len(full), "full_compare_equal": all(full)}), flush=True)
+    stack.close()
+
+
 def bench_reference(args) -> dict:
     """The CPU oracle, as it stands, on host cores: same metric and unit, bounded samples."""
     import oracle
@@ -640,6 +817,8 @@ def main(argv=None):
     ap.add_argument("--distinct-layers", type=int, default=8)
     ap.add_argument("--layers", type=int, default=N_LAYERS, help="blocks per pass (80 = the 70B model)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--configs", action="store_true",
+                    help="per-workload table (workloads 1-4, stream parity of 5) instead of the bench line")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -653,6 +832,9 @@ def main(argv=None):
     import torch
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA GPU")
+    if args.configs:
+        bench_configs(args)
+        return 0
     d = Dist()
     if d.world == 1:
         torch.cuda.set_device(0)

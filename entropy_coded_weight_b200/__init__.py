@@ -113,7 +113,7 @@ def encode_host(matrices, n_threads: int = 0, table_scope: str = "matrix", codec
     return out
 
 
-def _device_matrix_in_array(matrices, table_scope: str):
+def _device_matrix_in_array(matrices, table_scope: str, codec: str = "rans"):
     """eq_matrix_in[] whose pointers are device addresses (CUDA tensors on one device)."""
     import torch
     keep = []
@@ -141,19 +141,19 @@ def _device_matrix_in_array(matrices, table_scope: str):
         e.out_row = orow.data_ptr() if n_out else None
         e.out_col = ocol.data_ptr() if n_out else None
         e.out_val = oval.data_ptr() if n_out else None
-        e.flags = _flags(m, table_scope, "rans")
+        e.flags = _flags(m, table_scope, codec)
     return arr, keep
 
 
-def encode_device(matrices, table_scope: str = "matrix", stream=None):
+def encode_device(matrices, table_scope: str = "matrix", stream=None, codec: str = "rans"):
     """eq_encode_device: encode matrices whose symbols, scales and super weights
     are CUDA tensors; returns the container as a uint8 CUDA tensor (the same
     bytes eq_encode_host writes).  Each matrix needs ``layer``, ``dtype``,
     ``symbols`` (uint8 [rows, cols]), ``scales`` (float32 [rows]) and optionally
-    ``out_row``, ``out_col`` (integer), ``out_val`` (float32).  Synchronises
-    the stream."""
+    ``out_row``, ``out_col`` (integer), ``out_val`` (float32).  ``table_scope``
+    and ``codec`` as for encode_host.  Synchronises the stream."""
     import torch
-    arr, keep = _device_matrix_in_array(matrices, table_scope)
+    arr, keep = _device_matrix_in_array(matrices, table_scope, codec)
     n = len(matrices)
     L = load()
     wb, ob, ln = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()

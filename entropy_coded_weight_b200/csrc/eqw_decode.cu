@@ -15,8 +15,9 @@
 //               every chunk of the matrix carries the same frequency table
 //               (checked by eq_model_open and again per chunk), so one table
 //               per thread block serves all its warps, which work on tiles of
-//               WARPS consecutive chunks; SHARED = false: one table per warp,
-//               rebuilt for every chunk.
+//               consecutive chunks (two per warp; as few warps per tile as
+//               keep a small launch on every SM, see assign_tiles);
+//               SHARED = false: one table per warp, rebuilt for every chunk.
 //   staging     each warp streams its chunk's 16-bit renormalisation words
 //               into a private 2 KB shared-memory ring in 512-byte segments
 //               with TMA bulk copies (cp.async.bulk, mbarrier completion, no
@@ -75,6 +76,7 @@ struct DecodeParams {
     int32_t *status;
     uint32_t n_mats;
     uint32_t total_units;
+    uint32_t tile_warps;          // shared-table kernels: warps that take chunks of a tile (assign_tiles)
     MatJob mats[kMaxMatsPerLaunch];
 };
 
@@ -535,19 +537,20 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
         for (uint32_t unit = blockIdx.x; unit < P.total_units; unit += gridDim.x) {
             const uint32_t mi = job_of(P, unit);
             const MatJob &M = P.mats[mi];
-            const uint32_t k0 = (unit - M.begin) * WARPS * C;
+            const uint32_t TW = P.tile_warps;
+            const uint32_t k0 = (unit - M.begin) * TW * C;
             if (mi != cur_mat) {
                 shared_table_rebuild<WARPS, LAYOUT, CODEC>(P, M, k0, lane, warp, S);
                 cur_mat = mi;
             }
             const uint32_t np = S.blk[0];
             const uint32_t lane_sym = S.ref_entries[lane < np ? lane : 0] & 0xFFu;
-            // this warp's chunks: k0 + warp (+ WARPS for the second chain)
+            // this warp's chunks: k0 + warp (+ TW for the second chain); warps >= TW sit the tile out
             ChunkHead hc[C];
             bool have[C];
             for (uint32_t c = 0; c < C; ++c) {
-                const uint32_t k = k0 + warp + c * WARPS;
-                have[c] = k < M.n_chunks && !ctl[0].dead && !ctl[C - 1].dead;
+                const uint32_t k = k0 + warp + c * TW;
+                have[c] = warp < TW && k < M.n_chunks && !ctl[0].dead && !ctl[C - 1].dead;
                 if (have[c]) have[c] = shared_chunk_head<CODEC>(P, M, k, lane, np, S, hc[c]);
             }
             const OutCtx O = out_ctx(M);
@@ -559,7 +562,7 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
                     uint32_t rings[C], mbars[C];
 #pragma unroll
                     for (uint32_t c = 0; c < C; ++c) {
-                        first[c] = (uint64_t)(k0 + warp + c * WARPS) * kChunkSyms;
+                        first[c] = (uint64_t)(k0 + warp + c * TW) * kChunkSyms;
                         rings[c] = S.ring + c * kRingStride;
                         mbars[c] = S.mbar + 8 * kRingSegs * c;
                     }
@@ -571,7 +574,7 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
             }
             for (uint32_t c = 0; c < C; ++c) {
                 if (!have[c] || ctl->dead) continue;
-                decode_body<DT, LAYOUT, CODEC>(P.status, O, (uint64_t)(k0 + warp + c * WARPS) * kChunkSyms, hc[c].n,
+                decode_body<DT, LAYOUT, CODEC>(P.status, O, (uint64_t)(k0 + warp + c * TW) * kChunkSyms, hc[c].n,
                                         hc[c].n_words, hc[c].rec + hc[c].table_bytes, np == 1,
                                         S.ref_entries[0] & 0xFFu, hc[c].x, S.lut_addr, S.ring, S.mbar, ctl, lane,
                                         lt, rank_mode<LAYOUT>(np), lane_sym);
@@ -735,8 +738,7 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
             J.dtype = d.info.dtype;
             J.layout = lay;
             J.small_scales = d.small_scales ? 1u : 0u;
-            const uint32_t per_tile = kSharedWarps * EQ_CHAINS;
-            Pv.total_units += sh ? (d.info.n_chunks + per_tile - 1) / per_tile : d.info.n_chunks;
+            Pv.total_units += d.info.n_chunks;  // per-chunk units; shared-table launches are re-tiled below
             if (d.info.n_outliers && !symbols) {
                 ScatterJob &O = Q.jobs[Q.n_jobs++];
                 O.rec = reinterpret_cast<const uint32_t *>(m->d_blob + d.outliers_off);
@@ -749,6 +751,12 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
             }
         }
         Q.total = n_out;
+        for (int co = 0; co < 2; ++co)
+            for (int dt = 0; dt < 2; ++dt)
+                for (int lay = 0; lay < 4; ++lay) {
+                    const auto &k = dev->k[co][1][dt][lay];
+                    assign_tiles(P[co][1][dt][lay], (uint32_t)(dev->sms * k.ctas_per_sm), kSharedWarps, EQ_CHAINS);
+                }
         for (int co = 0; co < 2; ++co)
             for (int sh = 0; sh < 2; ++sh)
                 for (int dt = 0; dt < 2; ++dt)

@@ -73,6 +73,7 @@ struct GemvParams {
     int32_t *status;
     uint32_t n_mats;
     uint32_t total_units;
+    uint32_t tile_warps;          // shared-table kernels: warps that take chunks of a tile (assign_tiles)
     GemvJob mats[kMaxMatsPerLaunch];
 };
 
@@ -141,16 +142,16 @@ __device__ __forceinline__ void flush_segment(int32_t *status, const GemvJob &M,
 // One 256-symbol group times x.  BY_RANK: the slot entry's low 5 bits name
 // the lane holding the weight (lane r holds bf16(value(rank r) * scale));
 // otherwise `w` is the row scale and the weight is formed from the symbol.
-template <int DT, bool BY_RANK>
-__device__ __forceinline__ void group_dot(uint32_t lut, uint32_t ring, uint32_t &pw, uint32_t &x, uint32_t lt,
-                                          float w, const uint4 *xp, float &a0, float &a1) {
+template <int DT, bool BY_RANK, uint32_t CODEC>
+__device__ __forceinline__ void group_dot(uint32_t lut, uint32_t ring, uint32_t &pw, CodecState<CODEC> &x,
+                                          uint32_t lt, float w, const uint4 *xp, float &a0, float &a1) {
     const uint4 xv = __ldg(xp);
     const uint32_t rp0 = ring + (pw & (kRingBytes - 1));
     uint32_t rp = rp0;
 #pragma unroll
     for (int r = 0; r < 8; r += 2) {
-        const uint32_t e0 = rans_step(lut, rp, x, lt);
-        const uint32_t e1 = rans_step(lut, rp, x, lt);
+        const uint32_t e0 = codec_step<CODEC>(lut, rp, x, lt);
+        const uint32_t e1 = codec_step<CODEC>(lut, rp, x, lt);
         float w0, w1;
         if constexpr (BY_RANK) {
             w0 = __shfl_sync(kFull, w, e0);
@@ -167,10 +168,10 @@ __device__ __forceinline__ void group_dot(uint32_t lut, uint32_t ring, uint32_t 
 
 // Runs of groups within one row, two groups per ring check (the ring keeps
 // two groups' worth of words resident past each check).
-template <int DT, bool BY_RANK>
+template <int DT, bool BY_RANK, uint32_t CODEC>
 __device__ __forceinline__ void run_dot(uint32_t lut, uint32_t ring, uint32_t mbar, RingCtl *ctl, uint32_t &pw,
-                                        uint32_t &limit, uint32_t &x, uint32_t lt, float w, const uint4 *xp,
-                                        uint32_t run, float &a0, float &a1) {
+                                        uint32_t &limit, CodecState<CODEC> &x, uint32_t lt, float w,
+                                        const uint4 *xp, uint32_t run, float &a0, float &a1) {
     uint32_t i = 0;
     while (i < run) {
         if (pw >= limit) {
@@ -179,13 +180,13 @@ __device__ __forceinline__ void run_dot(uint32_t lut, uint32_t ring, uint32_t mb
         }
         if (i + 1 < run) {
             do {
-                group_dot<DT, BY_RANK>(lut, ring, pw, x, lt, w, xp, a0, a1);
-                group_dot<DT, BY_RANK>(lut, ring, pw, x, lt, w, xp + kGroupSyms / 8, a0, a1);
+                group_dot<DT, BY_RANK, CODEC>(lut, ring, pw, x, lt, w, xp, a0, a1);
+                group_dot<DT, BY_RANK, CODEC>(lut, ring, pw, x, lt, w, xp + kGroupSyms / 8, a0, a1);
                 i += 2;
                 xp += 2 * kGroupSyms / 8;
             } while (i + 1 < run && pw < limit);
         } else {
-            group_dot<DT, BY_RANK>(lut, ring, pw, x, lt, w, xp, a0, a1);
+            group_dot<DT, BY_RANK, CODEC>(lut, ring, pw, x, lt, w, xp, a0, a1);
             i += 1;
             xp += kGroupSyms / 8;
         }
@@ -194,7 +195,7 @@ __device__ __forceinline__ void run_dot(uint32_t lut, uint32_t ring, uint32_t mb
 
 // One chunk (its slot table ready at `lut`, or a single symbol `single`).
 // Returns false if a bounded wait gave up (the warp must stop).
-template <int DT>
+template <int DT, uint32_t CODEC>
 __device__ __forceinline__ bool gemv_body(int32_t *status, const GemvJob &M, uint64_t first, const ChunkHead &h,
                                           bool single_sym, uint32_t single, uint32_t lut, uint32_t ring,
                                           uint32_t mbar, RingCtl *ctl, uint32_t lane, uint32_t lt, bool by_rank,
@@ -202,10 +203,10 @@ __device__ __forceinline__ bool gemv_body(int32_t *status, const GemvJob &M, uin
     const uint32_t n_groups = h.n / kGroupSyms;
     uint32_t row = (uint32_t)(first / M.cols);
     uint32_t col = (uint32_t)(first - (uint64_t)row * M.cols);
-    uint32_t x = h.x;
+    CodecState<CODEC> x = codec_start<CODEC>(h.x);
     if (single_sym) {
-        // f = 4096: the states never change and there are no words
-        if (h.n_words != 0 || !__all_sync(kFull, x == kStateLow)) {
+        // rANS f = 4096 / Huffman length 0: the states never change and there are no words
+        if (h.n_words != 0 || !__all_sync(kFull, CODEC == kCodecHuffman || h.x == kStateLow)) {
             flag(status, EQ_DEV_BAD_END);
             return true;
         }
@@ -244,9 +245,10 @@ __device__ __forceinline__ bool gemv_body(int32_t *status, const GemvJob &M, uin
         const uint4 *xp = M.x + col / 8 + lane;
         float a0 = 0.f, a1 = 0.f;
         if (by_rank)
-            run_dot<DT, true>(lut, ring, mbar, ctl, pw, limit, x, lt, bf16_round(__fmul_rn(vraw, s)), xp, run, a0, a1);
+            run_dot<DT, true, CODEC>(lut, ring, mbar, ctl, pw, limit, x, lt, bf16_round(__fmul_rn(vraw, s)), xp,
+                                     run, a0, a1);
         else
-            run_dot<DT, false>(lut, ring, mbar, ctl, pw, limit, x, lt, s, xp, run, a0, a1);
+            run_dot<DT, false, CODEC>(lut, ring, mbar, ctl, pw, limit, x, lt, s, xp, run, a0, a1);
         const uint64_t lo = (uint64_t)row * M.cols + col;
         flush_segment(status, M, row, lo, lo + (uint64_t)run * kGroupSyms, a0 + a1, lane);
         g += run;
@@ -260,30 +262,33 @@ __device__ __forceinline__ bool gemv_body(int32_t *status, const GemvJob &M, uin
         flag(status, EQ_DEV_TIMEOUT);
         return false;
     }
-    if (!__all_sync(kFull, x == kStateLow) || pw != 2u * h.n_words) flag(status, EQ_DEV_BAD_END);
+    if (!__all_sync(kFull, codec_done(x)) || pw != 2u * h.n_words) flag(status, EQ_DEV_BAD_END);
     return true;
 }
 
 // Two full chunks per warp in lockstep (rank mode, cols % 512 == 0), as in
 // the decode kernel; each chain keeps its own row, weights and accumulators.
+template <uint32_t CODEC>
 struct DotChain {
-    uint32_t x, pw, limit, row, col;
+    CodecState<CODEC> x;
+    uint32_t pw, limit, row, col;
     float w, a0, a1;
     const uint4 *xp;
 };
 
-__device__ __forceinline__ void group2_dot(uint32_t lut, uint32_t ringA, uint32_t ringB, DotChain &A, DotChain &B,
-                                           uint32_t lt) {
+template <uint32_t CODEC>
+__device__ __forceinline__ void group2_dot(uint32_t lut, uint32_t ringA, uint32_t ringB, DotChain<CODEC> &A,
+                                           DotChain<CODEC> &B, uint32_t lt) {
     const uint4 xa = __ldg(A.xp), xb = __ldg(B.xp);
     const uint32_t a0 = ringA + (A.pw & (kRingBytes - 1));
     const uint32_t b0 = ringB + (B.pw & (kRingBytes - 1));
     uint32_t ra = a0, rb = b0;
 #pragma unroll
     for (int r = 0; r < 8; r += 2) {
-        const uint32_t ea0 = rans_step(lut, ra, A.x, lt);
-        const uint32_t eb0 = rans_step(lut, rb, B.x, lt);
-        const uint32_t ea1 = rans_step(lut, ra, A.x, lt);
-        const uint32_t eb1 = rans_step(lut, rb, B.x, lt);
+        const uint32_t ea0 = codec_step<CODEC>(lut, ra, A.x, lt);
+        const uint32_t eb0 = codec_step<CODEC>(lut, rb, B.x, lt);
+        const uint32_t ea1 = codec_step<CODEC>(lut, ra, A.x, lt);
+        const uint32_t eb1 = codec_step<CODEC>(lut, rb, B.x, lt);
         const uint32_t ua = vec_word(xa, r / 2), ub = vec_word(xb, r / 2);
         fma_pair(A.a0, A.a1, __shfl_sync(kFull, A.w, ea0), __shfl_sync(kFull, A.w, ea1), bf_lo(ua), bf_hi(ua));
         fma_pair(B.a0, B.a1, __shfl_sync(kFull, B.w, eb0), __shfl_sync(kFull, B.w, eb1), bf_lo(ub), bf_hi(ub));
@@ -294,14 +299,16 @@ __device__ __forceinline__ void group2_dot(uint32_t lut, uint32_t ringA, uint32_
     B.xp += kGroupSyms / 8;
 }
 
-__device__ __forceinline__ void chain_row(const GemvJob &M, DotChain &C, float vraw, uint32_t lane) {
+template <uint32_t CODEC>
+__device__ __forceinline__ void chain_row(const GemvJob &M, DotChain<CODEC> &C, float vraw, uint32_t lane) {
     C.w = bf16_round(__fmul_rn(vraw, __ldg(M.scales + C.row)));
     C.xp = M.x + C.col / 8 + lane;
     C.a0 = C.a1 = 0.f;
 }
 
 // After a pair of groups: at the end of a row, flush the segment and move on.
-__device__ __forceinline__ void chain_advance(int32_t *status, const GemvJob &M, DotChain &C, uint64_t first,
+template <uint32_t CODEC>
+__device__ __forceinline__ void chain_advance(int32_t *status, const GemvJob &M, DotChain<CODEC> &C, uint64_t first,
                                               float vraw, uint32_t lane) {
     C.col += 2 * kGroupSyms;
     if (C.col == M.cols) {
@@ -313,7 +320,7 @@ __device__ __forceinline__ void chain_advance(int32_t *status, const GemvJob &M,
     }
 }
 
-template <int DT>
+template <int DT, uint32_t CODEC>
 __device__ __forceinline__ bool gemv_pair(int32_t *status, const GemvJob &M, const ChunkHead &hA, const ChunkHead &hB,
                                           uint64_t firstA, uint64_t firstB, uint32_t lut, uint32_t ringA,
                                           uint32_t ringB, uint32_t mbarA, uint32_t mbarB, RingCtl *ctlA,
@@ -322,9 +329,9 @@ __device__ __forceinline__ bool gemv_pair(int32_t *status, const GemvJob &M, con
     ring_start(ctlB, hB);
     __syncwarp();
     const float vraw = symbol_value<DT>(lane_sym);
-    DotChain A, B;
-    A.x = hA.x;
-    B.x = hB.x;
+    DotChain<CODEC> A, B;
+    A.x = codec_start<CODEC>(hA.x);
+    B.x = codec_start<CODEC>(hB.x);
     A.pw = B.pw = 0;
     A.limit = hA.n_words ? 0u : kNoLimit;
     B.limit = hB.n_words ? 0u : kNoLimit;
@@ -359,16 +366,17 @@ __device__ __forceinline__ bool gemv_pair(int32_t *status, const GemvJob &M, con
         flag(status, EQ_DEV_TIMEOUT);
         return false;
     }
-    if (!__all_sync(kFull, A.x == kStateLow) || A.pw != 2u * hA.n_words) flag(status, EQ_DEV_BAD_END);
-    if (!__all_sync(kFull, B.x == kStateLow) || B.pw != 2u * hB.n_words) flag(status, EQ_DEV_BAD_END);
+    if (!__all_sync(kFull, codec_done(A.x)) || A.pw != 2u * hA.n_words) flag(status, EQ_DEV_BAD_END);
+    if (!__all_sync(kFull, codec_done(B.x)) || B.pw != 2u * hB.n_words) flag(status, EQ_DEV_BAD_END);
     return true;
 }
 
 // Same work distribution as eq_decode_kernel (row-uniform layout only):
-// SHARED = one slot table per block over tiles of WARPS x chains chunks,
+// SHARED = one slot table per block over tiles of P.tile_warps x chains chunks,
 // otherwise one table per warp and chunk.
-template <int WARPS, bool SHARED, int DT>
-__global__ void __launch_bounds__(WARPS * 32, SHARED ? kGemvMinCtas : 1) eq_decode_gemv_kernel(const __grid_constant__ GemvParams P) {
+template <int WARPS, bool SHARED, int DT, uint32_t CODEC>
+__global__ void __launch_bounds__(WARPS * 32, SHARED ? kGemvMinCtas : 1)
+    eq_decode_gemv_kernel(const __grid_constant__ GemvParams P) {
     constexpr uint32_t LAYOUT = kRowUniform;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t lane = threadIdx.x & 31u;
@@ -383,9 +391,10 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kGemvMinCtas : 1) eq_deco
         for (uint32_t unit = blockIdx.x; unit < P.total_units; unit += gridDim.x) {
             const uint32_t mi = job_of(P, unit);
             const GemvJob &M = P.mats[mi];
-            const uint32_t k0 = (unit - M.begin) * WARPS * C;
+            const uint32_t TW = P.tile_warps;
+            const uint32_t k0 = (unit - M.begin) * TW * C;
             if (mi != cur_mat) {
-                shared_table_rebuild<WARPS, LAYOUT>(P, M, k0, lane, warp, S);
+                shared_table_rebuild<WARPS, LAYOUT, CODEC>(P, M, k0, lane, warp, S);
                 cur_mat = mi;
             }
             const uint32_t np = S.blk[0];
@@ -393,15 +402,15 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kGemvMinCtas : 1) eq_deco
             ChunkHead hc[C];
             bool have[C];
             for (uint32_t c = 0; c < C; ++c) {
-                const uint32_t k = k0 + warp + c * WARPS;
-                have[c] = k < M.n_chunks && !ctl[0].dead && !ctl[C - 1].dead;
-                if (have[c]) have[c] = shared_chunk_head(P, M, k, lane, np, S, hc[c]);
+                const uint32_t k = k0 + warp + c * TW;
+                have[c] = warp < TW && k < M.n_chunks && !ctl[0].dead && !ctl[C - 1].dead;
+                if (have[c]) have[c] = shared_chunk_head<CODEC>(P, M, k, lane, np, S, hc[c]);
             }
             if constexpr (C == 2) {
                 if (have[0] && have[1] && rank_mode<LAYOUT>(np) && hc[0].n == kChunkSyms &&
                     hc[1].n == kChunkSyms && M.cols % (2 * kGroupSyms) == 0) {
-                    gemv_pair<DT>(P.status, M, hc[0], hc[1], (uint64_t)(k0 + warp) * kChunkSyms,
-                                  (uint64_t)(k0 + warp + WARPS) * kChunkSyms, S.lut_addr, S.ring,
+                    gemv_pair<DT, CODEC>(P.status, M, hc[0], hc[1], (uint64_t)(k0 + warp) * kChunkSyms,
+                                  (uint64_t)(k0 + warp + TW) * kChunkSyms, S.lut_addr, S.ring,
                                   S.ring + kRingStride, S.mbar, S.mbar + 8 * kRingSegs, ctl, ctl + 1, lane, lt,
                                   lane_sym);
                     __syncwarp();
@@ -410,7 +419,7 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kGemvMinCtas : 1) eq_deco
             }
             for (uint32_t c = 0; c < C; ++c) {
                 if (!have[c] || ctl->dead) continue;
-                gemv_body<DT>(P.status, M, (uint64_t)(k0 + warp + c * WARPS) * kChunkSyms, hc[c], np == 1,
+                gemv_body<DT, CODEC>(P.status, M, (uint64_t)(k0 + warp + c * TW) * kChunkSyms, hc[c], np == 1,
                               S.ref_entries[0] & 0xFFu, S.lut_addr, S.ring, S.mbar, ctl, lane, lt,
                               rank_mode<LAYOUT>(np), lane_sym);
                 __syncwarp();
@@ -422,16 +431,16 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kGemvMinCtas : 1) eq_deco
             const GemvJob &M = P.mats[job_of(P, c)];
             const uint32_t k = c - M.begin;
             ChunkHead h;
-            if (!load_head(P, M, k, lane, h)) continue;
-            const uint32_t *tab = reinterpret_cast<const uint32_t *>(h.rec + kRecordHeadBytes);
+            if (!load_head<CODEC>(P, M, k, lane, h)) continue;
+            const uint32_t *tab = reinterpret_cast<const uint32_t *>(h.rec + kHeadBytes<CODEC>);
             __syncwarp();  // the previous chunk's reads of the slot table are done
             const bool by_rank = rank_mode<LAYOUT>(h.n_present);
-            if (!warp_table(tab, h.n_present, lane, nullptr, nullptr, S.lut, by_rank)) {
+            if (!warp_table<CODEC>(tab, h.n_present, lane, nullptr, nullptr, S.lut, by_rank)) {
                 flag(P.status, EQ_DEV_BAD_TABLE);
                 continue;
             }
             __syncwarp();
-            gemv_body<DT>(P.status, M, (uint64_t)k * kChunkSyms, h, h.n_present == 1, tab[0] & 0xFFu, S.lut_addr,
+            gemv_body<DT, CODEC>(P.status, M, (uint64_t)k * kChunkSyms, h, h.n_present == 1, tab[0] & 0xFFu, S.lut_addr,
                           S.ring, S.mbar, ctl, lane, lt, by_rank, tab[lane < h.n_present ? lane : 0] & 0xFFu);
             __syncwarp();
         }
@@ -453,22 +462,22 @@ __global__ void eq_zero_rows_kernel(const __grid_constant__ ZeroParams Z) {
 
 // ---- host side ---------------------------------------------------------------------
 
-// variants: [shared][dtype - 1]
+// variants: [codec][shared][dtype - 1]
 struct GemvSetup {
     bool ready = false;
     int sms = 0;
-    KernelSetup<GemvParams> k[2][2];
+    KernelSetup<GemvParams> k[2][2][2];
 };
 std::mutex g_gemv_mu;
 GemvSetup g_gemv_setup[128];
 
-template <int DT>
-int setup_dtype(GemvSetup &d) {
-    int rc = setup_kernel(d.k[1][DT - 1], eq_decode_gemv_kernel<kGemvWarps, true, DT>, kGemvWarps,
+template <int DT, uint32_t CODEC>
+int setup_variant(GemvSetup &d) {
+    int rc = setup_kernel(d.k[CODEC][1][DT - 1], eq_decode_gemv_kernel<kGemvWarps, true, DT, CODEC>, kGemvWarps,
                           Smem<kGemvWarps, true>::kBytes, 1);
     if (rc) return rc;
-    return setup_kernel(d.k[0][DT - 1], eq_decode_gemv_kernel<kPrivateWarps, false, DT>, kPrivateWarps,
-                        Smem<kPrivateWarps, false>::kBytes, kPrivateWarps);
+    return setup_kernel(d.k[CODEC][0][DT - 1], eq_decode_gemv_kernel<kPrivateWarps, false, DT, CODEC>,
+                        kPrivateWarps, Smem<kPrivateWarps, false>::kBytes, kPrivateWarps);
 }
 
 int gemv_setup(GemvSetup **out) {
@@ -479,7 +488,9 @@ int gemv_setup(GemvSetup **out) {
     if (!d.ready) {
         if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return EQ_ERR_CUDA;
         int rc;
-        if ((rc = setup_dtype<EQ_INT8>(d)) || (rc = setup_dtype<EQ_E4M3>(d))) return rc;
+        if ((rc = setup_variant<EQ_INT8, kCodecRans>(d)) || (rc = setup_variant<EQ_E4M3, kCodecRans>(d)) ||
+            (rc = setup_variant<EQ_INT8, kCodecHuffman>(d)) || (rc = setup_variant<EQ_E4M3, kCodecHuffman>(d)))
+            return rc;
         d.ready = true;
     }
     *out = &d;
@@ -495,7 +506,7 @@ int check_gemv_args(const eq_model *m, uint32_t first, uint32_t count, const voi
         if (reinterpret_cast<uintptr_t>(ys[i]) % 4) return EQ_ERR_INVALID_ARG;
         if (in.rows && in.cols) {
             if (!xs[i] || reinterpret_cast<uintptr_t>(xs[i]) % 16) return EQ_ERR_INVALID_ARG;
-            if (in.cols % kGroupSyms || m->mats[first + i].codec != kCodecRans) return EQ_ERR_UNSUPPORTED;
+            if (in.cols % kGroupSyms) return EQ_ERR_UNSUPPORTED;
         }
     }
     return EQ_OK;
@@ -525,19 +536,20 @@ int launch_gemv(const eq_model *m, uint32_t first, uint32_t count, const void *c
             eq_zero_rows_kernel<<<std::min<uint32_t>((max_rows + 255) / 256, 4u * dev->sms), 256, 0, s>>>(Z);
             if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
         }
-        GemvParams P[2][2];
+        GemvParams P[2][2][2];
         for (auto &a : P)
-            for (auto &c : a) {
-                c = GemvParams{};
-                c.blob = m->d_blob;
-                c.blob_len = m->len;
-                c.status = d_status;
-            }
+            for (auto &b : a)
+                for (auto &c : b) {
+                    c = GemvParams{};
+                    c.blob = m->d_blob;
+                    c.blob_len = m->len;
+                    c.status = d_status;
+                }
         for (uint32_t i = 0; i < cnt; ++i) {
             const MatrixDesc &d = m->mats[first + base + i];
             if (d.info.n_chunks == 0) continue;
             const int sh = d.info.uniform_table ? 1 : 0;
-            GemvParams &Pv = P[sh][d.info.dtype - 1];
+            GemvParams &Pv = P[d.codec][sh][d.info.dtype - 1];
             GemvJob &J = Pv.mats[Pv.n_mats++];
             J.chunk_index = reinterpret_cast<const uint64_t *>(m->d_blob + d.chunk_index_off);
             J.scales = reinterpret_cast<const float *>(m->d_blob + d.scales_off);
@@ -550,12 +562,16 @@ int launch_gemv(const eq_model *m, uint32_t first, uint32_t count, const void *c
             J.n_chunks = d.info.n_chunks;
             J.begin = Pv.total_units;
             J.n_out = d.info.n_outliers;
-            const uint32_t per_tile = kGemvWarps * EQ_CHAINS;
-            Pv.total_units += sh ? (d.info.n_chunks + per_tile - 1) / per_tile : d.info.n_chunks;
+            Pv.total_units += d.info.n_chunks;  // per-chunk units; shared-table launches are re-tiled below
         }
-        for (int sh = 0; sh < 2; ++sh)
+        for (int co = 0; co < 2; ++co)
             for (int dt = 0; dt < 2; ++dt)
-                if ((rc = launch(dev->k[sh][dt], dev->sms, P[sh][dt], s))) return rc;
+                assign_tiles(P[co][1][dt], (uint32_t)(dev->sms * dev->k[co][1][dt].ctas_per_sm), kGemvWarps,
+                             EQ_CHAINS);
+        for (int co = 0; co < 2; ++co)
+            for (int sh = 0; sh < 2; ++sh)
+                for (int dt = 0; dt < 2; ++dt)
+                    if ((rc = launch(dev->k[co][sh][dt], dev->sms, P[co][sh][dt], s))) return rc;
     }
     return EQ_OK;
 }

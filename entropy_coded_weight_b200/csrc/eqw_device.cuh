@@ -726,6 +726,32 @@ int setup_kernel(KernelSetup<Params> &k, void (*fn)(Params), int warps, size_t s
     return EQ_OK;
 }
 
+// Shared-table kernels take their chunks in tiles: tile t of a matrix holds
+// chunks [t * W * chains, (t + 1) * W * chains), warp w of the block decoding
+// chunks w, w + W, ... of it.  W (P.tile_warps) is the fewest warps per tile
+// that still fit the whole launch into one round of resident blocks, so that
+// a block of small matrices spreads over every SM instead of filling a few of
+// them with full tiles; when even full tiles (W = max_warps) need more than
+// one round, W = max_warps.  Sets every matrix's first unit and the total.
+template <class Params>
+void assign_tiles(Params &P, uint32_t resident, uint32_t max_warps, uint32_t chains) {
+    uint32_t tw = max_warps;
+    for (uint32_t w = 1; w < max_warps; ++w) {
+        uint64_t units = 0;
+        for (uint32_t i = 0; i < P.n_mats; ++i) units += (P.mats[i].n_chunks + w * chains - 1) / (w * chains);
+        if (units <= resident) {
+            tw = w;
+            break;
+        }
+    }
+    P.tile_warps = tw;
+    P.total_units = 0;
+    for (uint32_t i = 0; i < P.n_mats; ++i) {
+        P.mats[i].begin = P.total_units;
+        P.total_units += (P.mats[i].n_chunks + tw * chains - 1) / (tw * chains);
+    }
+}
+
 // Persistent grid: at most one round of resident blocks, fewer when there is
 // less work than that.
 template <class Params>

@@ -93,78 +93,6 @@ void encode_record(const uint8_t *sym, uint32_t n, const uint32_t *table, std::v
     std::memcpy(p + table_end, w, 2 * (size_t)n_words);
 }
 
-// ---- Huffman codec (EntroLLM technical overview, "Huffman weight encoding") -----
-// Code lengths: Huffman's construction (repeatedly merge the two lightest
-// nodes; ties by creation order, leaves in symbol order first), then, if a
-// code exceeds 12 bits, the length adjustment of the JPEG standard (ITU-T
-// T.81 Annex K.3, "Adjust_BITS"): two codes of the longest length i give way
-// to one code of length i-1, and one code of the deepest shorter length j
-// becomes two codes of length j+1, which keeps the Kraft sum at 1.  The
-// lengths are then handed out shortest first to the most frequent symbols.
-// One distinct symbol: the empty code (all lengths 0).
-void huffman_lengths(const uint64_t cnt[256], uint8_t len[256]) {
-    std::memset(len, 0, 256);
-    struct Node {
-        uint64_t w;
-        int left, right;
-    };
-    std::vector<Node> nodes;
-    std::vector<int> sym_node(256, -1);
-    for (int s = 0; s < 256; ++s)
-        if (cnt[s]) {
-            sym_node[s] = (int)nodes.size();
-            nodes.push_back({cnt[s], -1, -1});
-        }
-    const int n = (int)nodes.size();
-    if (n < 2) return;
-    // min-heap on (weight, node index)
-    auto heavier = [&](int a, int b) { return nodes[a].w != nodes[b].w ? nodes[a].w > nodes[b].w : a > b; };
-    std::vector<int> heap;
-    for (int i = 0; i < n; ++i) heap.push_back(i);
-    std::make_heap(heap.begin(), heap.end(), heavier);
-    while (heap.size() > 1) {
-        std::pop_heap(heap.begin(), heap.end(), heavier);
-        const int a = heap.back();
-        heap.pop_back();
-        std::pop_heap(heap.begin(), heap.end(), heavier);
-        const int b = heap.back();
-        heap.pop_back();
-        nodes.push_back({nodes[a].w + nodes[b].w, a, b});
-        heap.push_back((int)nodes.size() - 1);
-        std::push_heap(heap.begin(), heap.end(), heavier);
-    }
-    // depth of every leaf
-    std::vector<int> depth(nodes.size(), 0);
-    for (int i = (int)nodes.size() - 1; i >= n; --i) {
-        depth[nodes[i].left] = depth[i] + 1;
-        depth[nodes[i].right] = depth[i] + 1;
-    }
-    std::vector<uint32_t> bits(258, 0);  // bits[l] = number of codes of length l
-    int max_len = 0;
-    for (int i = 0; i < n; ++i) {
-        ++bits[depth[i]];
-        max_len = std::max(max_len, depth[i]);
-    }
-    for (int i = max_len; i > (int)kHuffMaxLen; --i) {
-        while (bits[i] > 0) {
-            int j = i - 2;
-            while (bits[j] == 0) --j;
-            bits[i] -= 2;
-            bits[i - 1] += 1;
-            bits[j + 1] += 2;
-            bits[j] -= 1;
-        }
-    }
-    // shortest codes to the most frequent symbols (ties: smaller symbol first)
-    std::vector<int> order;
-    for (int s = 0; s < 256; ++s)
-        if (cnt[s]) order.push_back(s);
-    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cnt[a] > cnt[b]; });
-    size_t k = 0;
-    for (uint32_t l = 1; l <= kHuffMaxLen; ++l)
-        for (uint32_t c = 0; c < bits[l]; ++c) len[order[k++]] = (uint8_t)l;
-}
-
 // One Huffman chunk record.  `table_len` holds the matrix-wide lengths, or
 // null to build this chunk's own code.  Lane l's bit stream is its symbols'
 // canonical codes in step order, most significant bit first, cut into 16-bit
@@ -180,18 +108,13 @@ void encode_record_huffman(const uint8_t *sym, uint32_t n, const uint32_t *table
     } else {
         huffman_lengths(cnt, len);
     }
-    // canonical codes in (length, symbol) order
+    // canonical codes; table entries in (length, symbol) order
+    uint16_t code[256];
+    huffman_codes(len, code);
     std::vector<uint32_t> entries;
-    uint16_t code[256] = {0};
-    uint32_t c = 0, prev_len = 0;
     for (uint32_t l = 1; l <= kHuffMaxLen; ++l)
-        for (int s = 0; s < 256; ++s) {
-            if (len[s] != l) continue;
-            c = prev_len ? (c + 1) << (l - prev_len) : 0u;
-            prev_len = l;
-            code[s] = (uint16_t)c;
-            entries.push_back((uint32_t)s | (l << 16));
-        }
+        for (int s = 0; s < 256; ++s)
+            if (len[s] == l) entries.push_back((uint32_t)s | (l << 16));
     const bool single = entries.empty();
     std::vector<uint16_t> out;
     if (single) {

@@ -23,6 +23,11 @@
 // (the decoder's lane mapping); within a step the renormalising lanes' words
 // are stored in ascending lane order just in front of the words of the
 // following steps, at positions given by a ballot and a population count.
+// Huffman matrices (EntroLLM technical overview, "Huffman weight encoding")
+// take K3 eq_enc_huff_kernel<0/1> in place of K2, with code lengths built on
+// the host from the K1 histograms by the host encoder's routine: the
+// decoder's refill schedule walked forwards, each lane cutting its own code
+// string into the 16-bit words it hands out at its refills.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -53,6 +58,7 @@ struct EncMat {
     uint32_t per_chunk;       // 1: each chunk has its own table
     uint32_t table0;          // table slot of chunk 0 (per_chunk: + k)
     uint32_t hist0;           // per_chunk: chunk-histogram slot of chunk 0
+    uint32_t codec;           // kCodecRans or kCodecHuffman
 };
 
 struct EncWork {
@@ -61,7 +67,7 @@ struct EncWork {
     uint32_t n_jobs;
     unsigned long long *mat_hist;  // [n_mats][256]
     uint32_t *chunk_hist;          // [per-chunk chunks][256]
-    const uint32_t *tables;        // [slots][256] frequencies
+    const uint32_t *tables;        // [slots][256] rANS frequencies, or Huffman codes (huff_slot)
     uint32_t *n_words;             // [n_jobs]
     uint32_t *status;              // bit 0: an E4M3 NaN code
     uint8_t *out;                  // container (pass 2)
@@ -167,6 +173,7 @@ __global__ void __launch_bounds__(kEncWarps * 32) eq_enc_rans_kernel(const __gri
     asm("mov.u32 %0, %%lanemask_ge;" : "=r"(lanemask_ge));
     for (uint32_t job = blockIdx.x * kEncWarps + warp; job < W.n_jobs; job += gridDim.x * kEncWarps) {
         const EncMat &M = W.mats[mat_of(W, job)];
+        if (M.codec != kCodecRans) continue;
         const uint32_t k = job - M.first_job;
         const uint64_t first = (uint64_t)k * kChunkSyms;
         const uint32_t n = (uint32_t)(M.n - first < kChunkSyms ? M.n - first : kChunkSyms);
@@ -261,6 +268,150 @@ __global__ void __launch_bounds__(kEncWarps * 32) eq_enc_rans_kernel(const __gri
     }
 }
 
+// The 8 symbols of load8 with the super weights among them replaced by the
+// placeholder symbol 0.
+__device__ __forceinline__ uint2 load8_patched(const EncMat &M, uint64_t first, uint32_t n, uint32_t g,
+                                               uint32_t lane) {
+    uint2 v = load8(M, first, n, g, lane);
+    if (M.n_out) {
+        const uint64_t lo = first + (uint64_t)g * kGroupSyms + kGroup * lane;
+        for (uint32_t o = out_lower_bound(M, lo); o < M.n_out && out_lin(M, o) < lo + kGroup; ++o) {
+            const uint32_t r = (uint32_t)(out_lin(M, o) - lo);
+            if (r < 4) v.x &= ~(0xFFu << (8 * r));
+            else v.y &= ~(0xFFu << (8 * (r - 4)));
+        }
+    }
+    return v;
+}
+
+// Huffman table slot entry: code length (0: no code), canonical code, and a
+// mark on the one symbol of a table without codes.
+__host__ __device__ constexpr uint32_t huff_slot(uint32_t len, uint32_t code, bool single) {
+    return len | code << 8 | (single ? 1u << 31 : 0u);
+}
+
+// One chunk's Huffman record.  Lane l's code string is the canonical codes
+// of its symbols in step order; before each of its symbols the decoder gives
+// a lane holding fewer than 12 unread bits its next 16-bit word, the words of
+// one step in ascending lane order.  This walks those steps forwards: every
+// lane counts the bits it holds and, at a refill, cuts the next 16 bits off
+// its string (a producer running ahead over its own symbols; zero padding
+// after the last code).  WRITE = 0: word count into n_words[job]; WRITE = 1:
+// the whole record at its offset.
+template <int WRITE>
+__global__ void __launch_bounds__(kEncWarps * 32) eq_enc_huff_kernel(const __grid_constant__ EncWork W) {
+    __shared__ uint32_t tab_s[kEncWarps][256];
+    const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
+    uint32_t *T = tab_s[warp];
+    const uint32_t lt = (1u << lane) - 1u;
+    for (uint32_t job = blockIdx.x * kEncWarps + warp; job < W.n_jobs; job += gridDim.x * kEncWarps) {
+        const EncMat &M = W.mats[mat_of(W, job)];
+        if (M.codec != kCodecHuffman) continue;
+        const uint32_t k = job - M.first_job;
+        const uint64_t first = (uint64_t)k * kChunkSyms;
+        const uint32_t n = (uint32_t)(M.n - first < kChunkSyms ? M.n - first : kChunkSyms);
+        const uint32_t *tab = W.tables + 256ull * (M.table0 + (M.per_chunk ? k : 0u));
+        uint32_t n_coded = 0, single = 0;
+        for (uint32_t base = 0; base < 256; base += 32) {
+            const uint32_t e = tab[base + lane];
+            T[base + lane] = e;
+            n_coded += __popc(__ballot_sync(kFullMask, (e & 0xFFu) != 0));
+            const uint32_t m = __ballot_sync(kFullMask, (e >> 31) != 0);
+            if (m) single = base + __ffs(m) - 1;
+        }
+        __syncwarp();
+        const uint32_t n_present = n_coded ? n_coded : 1u;
+
+        uint16_t *words = nullptr;
+        uint8_t *rec = nullptr;
+        if (WRITE) {
+            const uint64_t off = reinterpret_cast<const uint64_t *>(W.out + M.ci)[k];
+            rec = W.out + off;
+            words = reinterpret_cast<uint16_t *>(rec + ((kHuffRecordHeadBytes + 4u * n_present + 15u) & ~15u));
+        }
+        uint32_t count = 0;  // WRITE = 0: this lane's refills; WRITE = 1: the warp's words so far
+        if (n_coded) {
+            const uint32_t steps = kGroup * ((n + kGroupSyms - 1) / kGroupSyms);
+            uint32_t held = 0;
+            uint2 cv = make_uint2(0, 0), pv = make_uint2(0, 0);
+            uint32_t cg = ~0u, pg = ~0u;
+            uint32_t pt = 0, nacc = 0;  // producer: next step to append, bits pending in acc
+            uint64_t acc = 0;
+            for (uint32_t t = 0; t < steps; ++t) {
+                const uint32_t g = t / kGroup, r = t % kGroup;
+                const bool active = g * kGroupSyms + kGroup * lane + r < n;
+                if (g != cg) {
+                    cv = load8_patched(M, first, n, g, lane);
+                    cg = g;
+                }
+                const bool need = active && held < kHuffMaxLen;
+                if (WRITE) {
+                    const uint32_t b = __ballot_sync(kFullMask, need);
+                    if (need) {
+                        for (;;) {
+                            if (nacc >= 16) break;
+                            const uint32_t pgi = pt / kGroup;
+                            if (pgi * kGroupSyms + kGroup * lane + pt % kGroup >= n) break;  // string ends
+                            if (pgi != pg) {
+                                pv = load8_patched(M, first, n, pgi, lane);
+                                pg = pgi;
+                            }
+                            const uint32_t e = T[byte_of(pv, pt % kGroup)];
+                            const uint32_t L = e & 0xFFu;
+                            acc = (acc << L) | ((e >> 8) & 0xFFFu);
+                            nacc += L;
+                            ++pt;
+                        }
+                        uint32_t w;
+                        if (nacc >= 16) {
+                            nacc -= 16;
+                            w = (uint32_t)(acc >> nacc) & 0xFFFFu;
+                            acc &= (1ull << nacc) - 1ull;
+                        } else {
+                            w = (uint32_t)(acc << (16 - nacc)) & 0xFFFFu;
+                            nacc = 0;
+                            acc = 0;
+                        }
+                        words[count + __popc(b & lt)] = (uint16_t)w;
+                    }
+                    count += __popc(b);
+                } else if (need) {
+                    ++count;
+                }
+                if (need) held += 16;
+                if (active) held -= T[byte_of(cv, r)] & 0xFFu;
+            }
+        }
+        if (!WRITE) {
+            for (int d = 16; d > 0; d >>= 1) count += __shfl_xor_sync(kFullMask, count, d);
+            if (lane == 0) W.n_words[job] = count;
+        } else {
+            uint32_t *head = reinterpret_cast<uint32_t *>(rec);
+            if (lane == 0) {
+                head[0] = n;
+                head[1] = count;
+                head[2] = n_present;
+                head[3] = 0;
+            }
+            uint32_t *entries = head + kHuffRecordHeadBytes / 4;
+            if (!n_coded) {
+                if (lane == 0) entries[0] = single;
+            } else {
+                uint32_t at = 0;
+                for (uint32_t l = 1; l <= kHuffMaxLen; ++l)
+                    for (uint32_t base = 0; base < 256; base += 32) {
+                        const uint32_t s = base + lane;
+                        const bool has = (T[s] & 0xFFu) == l;
+                        const uint32_t b = __ballot_sync(kFullMask, has);
+                        if (has) entries[at + __popc(b & lt)] = s | (l << 16);
+                        at += __popc(b);
+                    }
+            }
+        }
+        __syncwarp();
+    }
+}
+
 struct WorkLayout {
     size_t mats, mat_hist, chunk_hist, tables, n_words, status, total;
     uint32_t n_pc_chunks;
@@ -333,7 +484,6 @@ int encode_device(const eq_matrix_in *mats, uint32_t n_mats, void *d_out, size_t
     if (rc) return rc;
     for (uint32_t i = 0; i < n_mats; ++i) {
         const eq_matrix_in &m = mats[i];
-        if (m.flags & EQ_CODEC_HUFFMAN) return EQ_ERR_UNSUPPORTED;
         if ((uint64_t)m.rows * m.cols && reinterpret_cast<uintptr_t>(m.symbols) % 8) return EQ_ERR_INVALID_ARG;
     }
     ContainerPlan P;
@@ -381,6 +531,7 @@ int encode_device(const eq_matrix_in *mats, uint32_t n_mats, void *d_out, size_t
         e.per_chunk = (m.flags & EQ_TABLE_PER_CHUNK) ? 1u : 0u;
         e.table0 = e.per_chunk ? n_mats + pc : d;
         e.hist0 = pc;
+        e.codec = (m.flags & EQ_CODEC_HUFFMAN) ? kCodecHuffman : kCodecRans;
         if (e.per_chunk) pc += P.n_chunks[d];
     }
     EncWork W{};
@@ -423,33 +574,57 @@ int encode_device(const eq_matrix_in *mats, uint32_t n_mats, void *d_out, size_t
         return rc;
     if (status) return EQ_ERR_INVALID_ARG;  // an E4M3 NaN code
 
-    // frequency tables: slot d for matrix-wide tables, n_mats + chunk for per-chunk ones
+    // tables: slot d for matrix-wide tables, n_mats + chunk for per-chunk
+    // ones; rANS: quantised frequencies; Huffman: lengths and canonical codes
+    // (huff_slot), both by the host encoder's routines
     std::vector<uint32_t> tables(256ull * (n_mats + pc + 1), 0);
     std::vector<uint32_t> n_present(P.n_jobs, 0);
     for (uint32_t d = 0; d < n_mats; ++d) {
         const EncMat &e = em[d];
         const uint64_t n = e.n;
+        uint32_t np_matrix = 0;
         for (uint32_t k = 0; k < e.n_chunks; ++k) {
             uint32_t *f = tables.data() + 256ull * (e.table0 + (e.per_chunk ? k : 0u));
-            if (e.per_chunk) {
+            if (e.per_chunk || k == 0) {
                 uint64_t cnt[256];
-                for (int t = 0; t < 256; ++t) cnt[t] = chunk_hist[256ull * (e.hist0 + k) + t];
-                quantize_table(cnt, std::min<uint64_t>(kChunkSyms, n - (uint64_t)k * kChunkSyms), f);
-            } else if (k == 0) {
-                quantize_table(reinterpret_cast<const uint64_t *>(mat_hist.data() + 256ull * d), n, f);
+                for (int t = 0; t < 256; ++t)
+                    cnt[t] = e.per_chunk ? chunk_hist[256ull * (e.hist0 + k) + t] : mat_hist[256ull * d + t];
+                uint32_t np = 0;
+                if (e.codec == kCodecHuffman) {
+                    uint8_t len[256];
+                    uint16_t code[256];
+                    huffman_lengths(cnt, len);
+                    huffman_codes(len, code);
+                    int first_sym = -1;
+                    for (int t = 0; t < 256; ++t) {
+                        np += len[t] != 0;
+                        if (cnt[t] && first_sym < 0) first_sym = t;
+                    }
+                    for (int t = 0; t < 256; ++t) f[t] = huff_slot(len[t], code[t], !np && t == first_sym);
+                    if (!np) np = 1;  // the empty code: one table entry, no words
+                } else {
+                    quantize_table(cnt, e.per_chunk ? std::min<uint64_t>(kChunkSyms, n - (uint64_t)k * kChunkSyms)
+                                                    : n, f);
+                    for (int t = 0; t < 256; ++t) np += f[t] != 0;
+                }
+                np_matrix = np;
             }
-            uint32_t np = 0;
-            for (int t = 0; t < 256; ++t) np += f[t] != 0;
-            n_present[e.first_job + k] = np;
+            n_present[e.first_job + k] = np_matrix;
         }
     }
     if ((rc = cuda_ok(cudaMemcpyAsync(wk + L.tables, tables.data(), 4 * tables.size(), cudaMemcpyHostToDevice, s))))
         return rc;
 
-    // K2, pass 1: word counts
+    // K2 / K3, pass 1: word counts
+    bool any_rans = false, any_huff = false;
+    for (const EncMat &e : em) {
+        any_rans |= e.n_chunks && e.codec == kCodecRans;
+        any_huff |= e.n_chunks && e.codec == kCodecHuffman;
+    }
     std::vector<uint32_t> n_words(P.n_jobs);
     if (P.n_jobs) {
-        eq_enc_rans_kernel<0><<<grid, kEncWarps * 32, 0, s>>>(W);
+        if (any_rans) eq_enc_rans_kernel<0><<<grid, kEncWarps * 32, 0, s>>>(W);
+        if (any_huff) eq_enc_huff_kernel<0><<<grid, kEncWarps * 32, 0, s>>>(W);
         if ((rc = cuda_ok(cudaGetLastError())) ||
             (rc = cuda_ok(cudaMemcpyAsync(n_words.data(), wk + L.n_words, 4ull * P.n_jobs, cudaMemcpyDeviceToHost,
                                           s))))
@@ -459,7 +634,11 @@ int encode_device(const eq_matrix_in *mats, uint32_t n_mats, void *d_out, size_t
 
     // the container plan, then everything but the records
     std::vector<uint64_t> rec_size(P.n_jobs);
-    for (uint32_t j = 0; j < P.n_jobs; ++j) rec_size[j] = record_bytes(n_present[j], n_words[j]);
+    for (uint32_t d = 0; d < n_mats; ++d)
+        for (uint32_t k = 0; k < em[d].n_chunks; ++k) {
+            const uint32_t j = em[d].first_job + k;
+            rec_size[j] = record_bytes(n_present[j], n_words[j], em[d].codec);
+        }
     plan_offsets(mats, rec_size, P);
     *out_len = P.total;
     if (out_cap < P.total) return EQ_ERR_NOSPACE;
@@ -495,9 +674,10 @@ int encode_device(const eq_matrix_in *mats, uint32_t n_mats, void *d_out, size_t
                                                 cudaMemcpyHostToDevice, s))))
         return rc;
 
-    // K2, pass 2: the records
+    // K2 / K3, pass 2: the records
     if (P.n_jobs) {
-        eq_enc_rans_kernel<1><<<grid, kEncWarps * 32, 0, s>>>(W);
+        if (any_rans) eq_enc_rans_kernel<1><<<grid, kEncWarps * 32, 0, s>>>(W);
+        if (any_huff) eq_enc_huff_kernel<1><<<grid, kEncWarps * 32, 0, s>>>(W);
         if ((rc = cuda_ok(cudaGetLastError()))) return rc;
     }
     return cuda_ok(cudaStreamSynchronize(s));

@@ -245,8 +245,10 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
     __shared__ uint32_t tmem_base_s;
     const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
     const bool mma_warp = warp == kProducerWarps;
-    const uint32_t n0 = blockIdx.x * kTileN;   // weight rows (outputs)
-    const uint32_t m0 = blockIdx.y * kTileM;   // tokens
+    // token tiles vary fastest, so the blocks that read one weight tile run
+    // together and it comes from DRAM once (the token matrix stays in L2)
+    const uint32_t n0 = blockIdx.y * kTileN;   // weight rows (outputs)
+    const uint32_t m0 = blockIdx.x * kTileM;   // tokens
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     // stage st: token tile (swizzled bf16), widened symbol tile (swizzled bf16), symbol bytes (staging)
     auto bufA = [&](uint32_t st) { return base + st * kStageBytes; };
@@ -408,7 +410,7 @@ extern "C" EQW_API int eq_gemm_symbols(const eq_model *m, uint32_t matrix, const
     const MatrixDesc &d = m->mats[matrix];
     const eq_matrix_info &in = d.info;
     if (!tokens || !in.rows || !in.cols) return EQ_OK;
-    if (in.rows % kTileN || in.cols % kTileK) return EQ_ERR_UNSUPPORTED;
+    if (in.rows % kTileN || in.cols % kTileK || in.rows / kTileN > 65535u) return EQ_ERR_UNSUPPORTED;
     if (!d_sym || !d_x || !d_y) return EQ_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(d_sym) % 16 || reinterpret_cast<uintptr_t>(d_x) % 16 ||
         reinterpret_cast<uintptr_t>(d_y) % 16 || d.scales_off % 16)
@@ -433,7 +435,7 @@ extern "C" EQW_API int eq_gemm_symbols(const eq_model *m, uint32_t matrix, const
             return EQ_ERR_CUDA;
         attr = true;
     }
-    const dim3 grid(in.rows / kTileN, (tokens + kTileM - 1) / kTileM);
+    const dim3 grid((tokens + kTileM - 1) / kTileM, in.rows / kTileN);
     fn<<<grid, kGemmThreads + 32, kGemmSmem, s>>>(P);
     if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
     if (in.n_outliers) {

@@ -133,8 +133,8 @@ typedef struct eq_matrix_in {
  * (words ordered by step, then lane); a chunk with one distinct symbol has
  * the empty code.  Huffman chunk record: u32 n_syms, n_words, n_present, 0;
  * u32 table[n_present] = symbol | length << 16 sorted by (length, symbol);
- * padding to 16 B; u16 words; padding to 16 B (no states).  Host encoder
- * only (eq_encode_device returns EQ_ERR_UNSUPPORTED).
+ * padding to 16 B; u16 words; padding to 16 B (no states).  Both encoders
+ * write it (the same bytes for the same inputs).
  */
 #define EQ_CODEC_HUFFMAN 2u
 
@@ -170,10 +170,10 @@ EQW_API int eq_encode_host(const eq_matrix_in *mats, uint32_t n_mats, int n_thre
  * pointer inside eq_matrix_in is a DEVICE address: symbols (8-byte aligned),
  * scales, out_row, out_col, out_val.  Steps, all on stream `s`: per-chunk
  * histograms on the GPU (super-weight positions count as symbol 0; an E4M3
- * NaN code is an error), frequency tables on the host with the host
- * encoder's routine, a GPU pass that counts each chunk's renormalisation
- * words, the container plan on the host, and a GPU pass that writes the
- * records.  Unlike every other entry point it synchronises `s` (the plan
+ * NaN code is an error), frequency tables (rANS) or code lengths and
+ * canonical codes (Huffman) on the host with the host encoder's routines, a
+ * GPU pass that counts each chunk's words, the container plan on the host,
+ * and a GPU pass that writes the records.  Unlike every other entry point it synchronises `s` (the plan
  * needs the counts on the host).
  *   d_out    device, out_cap bytes (eq_encode_bound gives a sufficient size);
  *            *out_len receives the exact container size; EQ_ERR_NOSPACE
@@ -300,7 +300,8 @@ EQW_API int eq_gemv_bf16(const void *d_w, const void *d_x, float *d_y, uint32_t 
  * Arguments: x (device, bf16 [cols], 16-byte aligned), y (device, fp32 [rows],
  * overwritten: zeroed on `s` first, then accumulated by the kernel), d_status
  * as for the decoders.  Every matrix with rows * cols > 0 needs
- * cols % 256 == 0 (EQ_ERR_UNSUPPORTED otherwise).  Enqueued on `s`.
+ * cols % 256 == 0 (EQ_ERR_UNSUPPORTED otherwise); rANS and Huffman matrices
+ * alike.  Enqueued on `s`.
  */
 EQW_API int eq_decode_gemv_matrix(const eq_model *m, uint32_t matrix, const void *d_x, float *d_y,
                                   int32_t *d_status, cudaStream_t s);
@@ -340,7 +341,8 @@ EQW_API int eq_decode_symbols_block(const eq_model *m, uint32_t layer, void *con
  * value() is exact in bf16; the scale multiplies the fp32 sum once per output
  * (round to nearest even).  X: device bf16 [tokens, cols] row-major, Y:
  * device fp32 [tokens, rows] row-major, both 16-byte aligned.  Needs
- * rows % 128 == 0 and cols % 64 == 0 (EQ_ERR_UNSUPPORTED otherwise).
+ * rows % 128 == 0, rows <= 128 * 65535 and cols % 64 == 0
+ * (EQ_ERR_UNSUPPORTED otherwise).
  * Enqueued on `s`.
  */
 EQW_API int eq_gemm_symbols(const eq_model *m, uint32_t matrix, const void *d_sym, const void *d_x, uint32_t tokens,

@@ -40,11 +40,14 @@ class DevMatrix:
 
 def _dev(m):
     has = len(m.out_row) > 0
-    return DevMatrix(m.layer, m.dtype, torch.from_numpy(np.ascontiguousarray(m.symbols)).cuda(),
-                     torch.from_numpy(np.ascontiguousarray(m.scales)).cuda(),
-                     torch.from_numpy(m.out_row.astype(np.int32)).cuda() if has else None,
-                     torch.from_numpy(m.out_col.astype(np.int32)).cuda() if has else None,
-                     torch.from_numpy(m.out_val.astype(np.float32)).cuda() if has else None)
+    d = DevMatrix(m.layer, m.dtype, torch.from_numpy(np.ascontiguousarray(m.symbols)).cuda(),
+                  torch.from_numpy(np.ascontiguousarray(m.scales)).cuda(),
+                  torch.from_numpy(m.out_row.astype(np.int32)).cuda() if has else None,
+                  torch.from_numpy(m.out_col.astype(np.int32)).cuda() if has else None,
+                  torch.from_numpy(m.out_val.astype(np.float32)).cuda() if has else None)
+    if hasattr(m, "codec"):
+        d.codec = m.codec  # a matrix's own codec wins over the call's
+    return d
 
 
 def _ragged():
@@ -64,20 +67,45 @@ def _ragged():
     return mats
 
 
+@pytest.mark.parametrize("codec", ["rans", "huffman"])
 @pytest.mark.parametrize("scope", ["matrix", "chunk"])
-def test_ragged_bytes_equal_host_encoder(eqw, scope):
+def test_ragged_bytes_equal_host_encoder(eqw, scope, codec):
     mats = _ragged()
-    host = eqw.encode_host(mats, table_scope=scope)
-    dev = eqw.encode_device([_dev(m) for m in mats], table_scope=scope).cpu().numpy()
+    host = eqw.encode_host(mats, table_scope=scope, codec=codec)
+    dev = eqw.encode_device([_dev(m) for m in mats], table_scope=scope, codec=codec).cpu().numpy()
     assert dev.size == host.size
     assert np.array_equal(dev, host)
 
 
-@pytest.mark.parametrize("which", ["llama70b_int8_layer", "llama70b_e4m3_block", "llama7b_int8_block_with_outliers"])
-def test_full_size_bytes_equal_host_encoder(eqw, which):
-    mats = W.llama70b_int8_layer(0) if which == "llama70b_int8_layer" else getattr(W, which)()
+def test_mixed_codecs_bytes_equal_host_encoder(eqw):
+    mats = _ragged()
+    for i, m in enumerate(mats):
+        m.codec = "huffman" if i % 2 else "rans"
     host = eqw.encode_host(mats)
     dev = eqw.encode_device([_dev(m) for m in mats]).cpu().numpy()
+    assert np.array_equal(dev, host)
+
+
+def test_huffman_long_codes_bytes_equal_host_encoder(eqw):
+    """Skewed counts over 254 E4M3 codes: many codes at the 12-bit limit, long refill look-ahead."""
+    rng = np.random.default_rng(5)
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    p = 0.5 ** np.arange(codes.size) + 1e-6
+    sym = rng.choice(codes, size=(64, 4096), p=p / p.sum()).astype(np.uint8)
+    sym[0, :len(codes)] = codes
+    m = W.Matrix(0, 0, "all", W.E4M3, sym, np.ones(64, np.float32))
+    for scope in ("matrix", "chunk"):
+        host = eqw.encode_host([m], table_scope=scope, codec="huffman")
+        dev = eqw.encode_device([_dev(m)], table_scope=scope, codec="huffman").cpu().numpy()
+        assert np.array_equal(dev, host), scope
+
+
+@pytest.mark.parametrize("codec", ["rans", "huffman"])
+@pytest.mark.parametrize("which", ["llama70b_int8_layer", "llama70b_e4m3_block", "llama7b_int8_block_with_outliers"])
+def test_full_size_bytes_equal_host_encoder(eqw, which, codec):
+    mats = W.llama70b_int8_layer(0) if which == "llama70b_int8_layer" else getattr(W, which)()
+    host = eqw.encode_host(mats, codec=codec)
+    dev = eqw.encode_device([_dev(m) for m in mats], codec=codec).cpu().numpy()
     assert np.array_equal(dev, host)
 
 

@@ -116,8 +116,29 @@ def test_device_detects_corruption(eqw, orc, scope):
     assert _corrupt_and_decode(eqw, blob, payload) & eqw.EQ_DEV_BAD_END
 
 
-def test_fused_gemv_refuses_huffman(eqw):
-    m = W.random_int8_matrix(300, 64, 512)
+@pytest.mark.parametrize("scope", ["matrix", "chunk"])
+def test_fused_gemv_within_bound(eqw, orc, scope):
+    """Fused decode + GEMV on Huffman matrices: the bound of test_gpu_fused_gemv."""
+    from test_gpu_fused_gemv import _bits, _bound_ok, _n_out_rows, _run_matrices, _x_for
+    mats = [W.random_int8_matrix(300, 64, 512, layer=0, index=0),
+            W.random_int8_matrix(301, 300, 1024, n_out=7, layer=0, index=1),
+            W.random_e4m3_matrix(302, 96, 4096, alpha=1.0, layer=0, index=2),
+            W.random_int8_matrix(303, 1024, 8192, layer=0, index=3)]
+    single = W.random_int8_matrix(304, 40, 2048, layer=0, index=4)
+    single.symbols[:] = 0x05
+    mats.append(single)
+    blob = eqw.encode_host(mats, table_scope=scope, codec="huffman")
+    for per_matrix in (True, False):
+        st, ys = _run_matrices(eqw, blob, mats, per_matrix=per_matrix)
+        assert st == 0
+        for m, y in zip(mats, ys):
+            ref, mag = orc.gemv_exact(orc.dequant_direct(m), _bits(_x_for(m)))
+            ok, info = _bound_ok(y, ref, mag, m.cols, _n_out_rows(m))
+            assert ok, (scope, per_matrix, m.index, info)
+
+
+def test_fused_gemv_needs_cols_multiple_of_256(eqw):
+    m = W.random_int8_matrix(305, 64, 500)
     blob = eqw.encode_host([m], codec="huffman")
     model = eqw.Model(eqw.upload(blob), blob)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
