@@ -14,8 +14,9 @@
 // is applied once per output in the epilogue and the (rare) super weights by
 // a small second kernel.
 //
-// Kernel eq_gemm_symbols_kernel, one CTA per 128 x 128 output tile, 8
-// producer warps and one MMA warp:
+// Kernel eq_gemm_symbols_kernel, one CTA per 256-token x 128-row output tile
+// (two token halves sharing each widened weight tile), 8 producer warps and
+// one MMA warp:
 //   producers  per K slab of 64: cp.async copies of the token tile straight
 //              into the 128-byte-swizzled K-major layout (16-byte chunk c of
 //              row r at chunk position c ^ (r % 8), 8-row groups 1024 B
@@ -25,10 +26,11 @@
 //              chunks into the swizzled bf16 tile and its warp arrives on the
 //              stage's "full" mbarrier; a stage is refilled only after its
 //              "empty" barrier says the tensor core is done with it
-//   MMA warp   one lane waits for "full", issues 4 x tcgen05.mma (M 128,
-//              N 128, K 16, fp32 accumulator in 128 TMEM columns) and
-//              tcgen05.commit to the stage's "empty" barrier; a last commit
-//              to "done" releases the epilogue
+//   MMA warp   one lane waits for "full", issues 4 x 2 tcgen05.mma (M 128,
+//              N 128, K 16; token half h into the fp32 accumulator in TMEM
+//              columns 128 h .. 128 h + 127) and tcgen05.commit to the
+//              stage's "empty" barrier; a last commit to "done" releases the
+//              epilogue
 //   epilogue   producer warp w reads accumulator lanes 32 (w % 4) with
 //              tcgen05.ld, multiplies by the row scales and stores fp32
 // Every mbarrier wait is bounded; on expiry the CTA records EQ_DEV_TIMEOUT,
@@ -46,17 +48,16 @@ namespace {
 #define EQ_GEMM_THREADS 256
 #endif
 constexpr int kGemmThreads = EQ_GEMM_THREADS;  // 4 or 8 warps
-// One token tile of 128 per CTA and two stages is the configuration verified
-// on the GPU.  Two token halves per CTA (two accumulators fed by one widened
-// weight tile) raised an illegal-instruction error there, cause not found;
-// it is not used.
+// Token halves per CTA: each widened weight tile feeds kHalves MMAs of 128
+// tokens into kHalves accumulators (one instruction shape, M = 128, whatever
+// the CTA's token tile).
 #ifndef EQ_GEMM_HALVES
-#define EQ_GEMM_HALVES 1
+#define EQ_GEMM_HALVES 2
 #endif
 #ifndef EQ_GEMM_STAGES
 #define EQ_GEMM_STAGES 4
 #endif
-static_assert(EQ_GEMM_HALVES == 1, "two token halves per CTA faulted on the GPU and are not used");
+static_assert(EQ_GEMM_HALVES == 1 || EQ_GEMM_HALVES == 2, "one or two token halves per CTA");
 constexpr uint32_t kMmaM = 128;                        // tokens per MMA (accumulator lanes)
 constexpr uint32_t kHalves = EQ_GEMM_HALVES;           // MMAs per widened weight tile
 constexpr uint32_t kTileM = kMmaM * kHalves;           // tokens per CTA tile
@@ -104,12 +105,15 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
-// K-major, N and M of the tile.
+// K-major, N and M of one MMA.  M is the instruction's 128, not the CTA's
+// token tile: cta_group::1 takes M = 64 or 128 only, and an M field of 256
+// here is an illegal instruction on the GPU.
+static_assert(kMmaM == 64 || kMmaM == 128, "cta_group::1 MMA shape");
 constexpr uint32_t kInstrDesc = (1u << 4)                 // D format fp32
                               | (1u << 7)                 // A format bf16
                               | (1u << 10)                // B format bf16
                               | ((kTileN >> 3) << 17)     // N / 8
-                              | ((kTileM >> 4) << 24);    // M / 16
+                              | ((kMmaM >> 4) << 24);     // M / 16
 
 // Byte offset of the 16-byte chunk k8 (bf16 8 k8 .. 8 k8 + 7) of tile row `row`.
 // 128-byte swizzle: each 64-element row is one 128-byte line, 8-row groups are
@@ -341,7 +345,10 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
             tc_fence_after();
 #pragma unroll
             for (uint32_t kk = 0; kk < kTileK / kMmaK; ++kk)
-                tc_mma(tmem, tile_desc(bufA(s), kk), tile_desc(bufB(s), kk), (it | kk) != 0u);
+#pragma unroll
+                for (uint32_t h = 0; h < kHalves; ++h)  // half h: tokens 128 h .., accumulator columns 128 h ..
+                    tc_mma(tmem + h * kTileN, tile_desc(bufA(s) + h * kMmaM * kTileK * 2u, kk),
+                           tile_desc(bufB(s), kk), (it | kk) != 0u);
             tc_commit(empty0 + 8 * s);
         }
         tc_commit(done);  // completes when every MMA issued above has
@@ -351,17 +358,18 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
         tc_fence_after();
         if (__all_sync(0xFFFFFFFFu, ok)) {
             // warp w reads accumulator lanes 32 (w % 4) .. + 31; warps sharing a
-            // lane quarter split the 128 columns
+            // lane quarter split the columns (half h = columns 128 h ..)
             constexpr uint32_t kColsPerWarp = kTmemCols * 4 / kProducerWarps;
             const uint32_t quarter = warp & 3u, c_first = (warp >> 2) * (kColsPerWarp / 32);
-            const uint32_t m = m0 + quarter * 32u + lane;
 #pragma unroll 1
             for (uint32_t c = c_first; c < c_first + kColsPerWarp / 32; ++c) {
                 uint32_t r[32];
                 tmem_ld32(tmem + ((quarter * 32u) << 16) + c * 32u, r);
+                const uint32_t half = c * 32u / kTileN, n_off = c * 32u % kTileN;
+                const uint32_t m = m0 + half * kMmaM + quarter * 32u + lane;
                 if (m < P.tokens) {
-                    float4 *dst = reinterpret_cast<float4 *>(P.y + (size_t)m * P.rows + n0 + c * 32u);
-                    const float4 *sc = reinterpret_cast<const float4 *>(P.scales + n0 + c * 32u);
+                    float4 *dst = reinterpret_cast<float4 *>(P.y + (size_t)m * P.rows + n0 + n_off);
+                    const float4 *sc = reinterpret_cast<const float4 *>(P.scales + n0 + n_off);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const float4 s4 = __ldg(sc + q);
