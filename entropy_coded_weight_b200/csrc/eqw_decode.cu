@@ -332,6 +332,85 @@ __device__ __forceinline__ bool decode_multi(int32_t *status, const OutCtx &O, c
     return true;
 }
 
+// Symbol bytes (layout kSymbolBytes) of C full chunks per warp in lockstep:
+// the same interleaved steps as decode_multi, each lane's 8 low bytes of a
+// group packed with byte permutes into one 8-byte store.  Any table (the
+// bytes are the stored symbols), any shape (the output is the flat symbol
+// array).
+__device__ __forceinline__ uint32_t bytes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    uint32_t ab, cd, r;
+    asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(ab) : "r"(a), "r"(b));  // a.b0, b.b0
+    asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(cd) : "r"(c), "r"(d));
+    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(ab), "r"(cd));  // ab.b0 ab.b1 cd.b0 cd.b1
+    return r;
+}
+
+template <uint32_t CODEC, uint32_t C>
+__device__ __forceinline__ void groupN_bytes(uint32_t lut, const uint32_t (&ring)[C], Chain<CODEC> (&ch)[C],
+                                             uint32_t lt) {
+    uint32_t r0[C], rp[C], o[C][2];
+#pragma unroll
+    for (uint32_t c = 0; c < C; ++c) rp[c] = r0[c] = ring[c] + (ch[c].pw & (kRingBytes - 1));
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t e[C][4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (uint32_t c = 0; c < C; ++c) e[c][r] = codec_step<CODEC>(lut, rp[c], ch[c].x, lt);
+#pragma unroll
+        for (uint32_t c = 0; c < C; ++c) o[c][h] = bytes4(e[c][0], e[c][1], e[c][2], e[c][3]);
+    }
+#pragma unroll
+    for (uint32_t c = 0; c < C; ++c) {
+        asm volatile("st.global.v2.b32 [%0], {%1, %2};" ::"l"(ch[c].dst), "r"(o[c][0]), "r"(o[c][1]) : "memory");
+        ch[c].pw += rp[c] - r0[c];
+        ch[c].dst += kGroupSyms / 2;  // 256 bytes, in bf16 units of the output pointer
+    }
+}
+
+template <uint32_t CODEC, uint32_t C>
+__device__ __forceinline__ bool decode_multi_bytes(int32_t *status, const OutCtx &O, const ChunkHead (&h)[C],
+                                                   const uint64_t (&first)[C], uint32_t lut,
+                                                   const uint32_t (&ring)[C], const uint32_t (&mbar)[C],
+                                                   RingCtl *ctl, uint32_t lane, uint32_t lt) {
+#pragma unroll
+    for (uint32_t c = 0; c < C; ++c) ring_start(ctl + c, h[c]);
+    __syncwarp();
+    Chain<CODEC> ch[C];
+#pragma unroll
+    for (uint32_t c = 0; c < C; ++c) {
+        ch[c].x = codec_start<CODEC>(h[c].x);
+        ch[c].pw = 0;
+        ch[c].limit = h[c].n_words ? 0u : kNoLimit;
+        // byte address first + 8 lane, carried in a bf16 pointer (always even)
+        ch[c].dst = reinterpret_cast<uint16_t *>(reinterpret_cast<uint8_t *>(O.out) + first[c] + kGroup * lane);
+    }
+    constexpr uint32_t kPairs = kChunkSyms / (2 * kGroupSyms);
+    for (uint32_t q = 0; q < kPairs; ++q) {
+        bool dead = false;
+#pragma unroll
+        for (uint32_t c = 0; c < C; ++c) {
+            if (ch[c].pw >= ch[c].limit) ch[c].limit = ring_service(ctl + c, ring[c], mbar[c], ch[c].pw);
+            dead = dead || ctl[c].dead;
+        }
+        if (dead) break;
+        groupN_bytes<CODEC, C>(lut, ring, ch, lt);
+        groupN_bytes<CODEC, C>(lut, ring, ch, lt);
+    }
+    bool drained = true;
+#pragma unroll
+    for (uint32_t c = 0; c < C; ++c) drained = ring_drain(ctl + c, mbar[c]) && drained;
+    if (!drained) {
+        flag(status, EQ_DEV_TIMEOUT);
+        return false;
+    }
+#pragma unroll
+    for (uint32_t c = 0; c < C; ++c)
+        if (!__all_sync(kFull, codec_done(ch[c].x)) || ch[c].pw != 2u * h[c].n_words) flag(status, EQ_DEV_BAD_END);
+    return true;
+}
+
 // Decode one chunk whose slot table is ready at `lut` (n_present >= 2) or
 // whose single symbol's stored byte is `single` (n_present == 1).  Returns
 // false if a bounded wait gave up (the warp must stop).
@@ -554,8 +633,9 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
                 if (have[c]) have[c] = shared_chunk_head<CODEC>(P, M, k, lane, np, S, hc[c]);
             }
             const OutCtx O = out_ctx(M);
-            if constexpr (C >= 2 && LAYOUT == kRowUniform) {
-                bool all_full = rank_mode<LAYOUT>(np) && O.cols % (2 * kGroupSyms) == 0;
+            if constexpr (C >= 2 && (LAYOUT == kRowUniform || LAYOUT == kSymbolBytes)) {
+                bool all_full = LAYOUT == kSymbolBytes ? np >= 2
+                                                       : rank_mode<LAYOUT>(np) && O.cols % (2 * kGroupSyms) == 0;
                 for (uint32_t c = 0; c < C; ++c) all_full = all_full && have[c] && hc[c].n == kChunkSyms;
                 if (all_full) {
                     uint64_t first[C];
@@ -566,8 +646,11 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
                         rings[c] = S.ring + c * kRingStride;
                         mbars[c] = S.mbar + 8 * kRingSegs * c;
                     }
-                    decode_multi<DT, CODEC, C>(P.status, O, hc, first, S.lut_addr, rings, mbars, ctl, lane, lt,
-                                               lane_sym);
+                    if constexpr (LAYOUT == kSymbolBytes)
+                        decode_multi_bytes<CODEC, C>(P.status, O, hc, first, S.lut_addr, rings, mbars, ctl, lane, lt);
+                    else
+                        decode_multi<DT, CODEC, C>(P.status, O, hc, first, S.lut_addr, rings, mbars, ctl, lane, lt,
+                                                   lane_sym);
                     __syncwarp();
                     continue;
                 }
