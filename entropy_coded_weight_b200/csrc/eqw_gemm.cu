@@ -17,15 +17,17 @@
 // Kernel eq_gemm_symbols_kernel, one CTA per 256-token x 128-row output tile
 // (two token halves sharing each widened weight tile), 8 producer warps and
 // one MMA warp:
-//   producers  per K slab of 64: cp.async copies of the token tile straight
-//              into the 128-byte-swizzled K-major layout (16-byte chunk c of
-//              row r at chunk position c ^ (r % 8), 8-row groups 1024 B
-//              apart) and of the symbol bytes into a staging area, issued
-//              kAhead slabs ahead into a ring of kStages stages; once a
-//              thread's copies of a slab have landed it widens its own symbol
-//              chunks into the swizzled bf16 tile and its warp arrives on the
-//              stage's "full" mbarrier; a stage is refilled only after its
-//              "empty" barrier says the tensor core is done with it
+//   producers  per K slab of 64: one TMA tensor copy of the token tile
+//              (issued by thread 0, 128-byte swizzle: the K-major layout the
+//              MMA reads, 16-byte chunk c of row r at chunk position
+//              c ^ (r % 8), 8-row groups 1024 B apart) and cp.async copies of
+//              the symbol bytes into a staging area, issued kAhead slabs
+//              ahead into a ring of kStages stages; once a thread's copies of
+//              a slab have landed it widens its own symbol chunks into the
+//              swizzled bf16 tile and its warp arrives on the stage's "full"
+//              mbarrier (which also waits for the tensor copy's bytes); a
+//              stage is refilled only after its "empty" barrier says the
+//              tensor core is done with it
 //   MMA warp   one lane waits for "full", issues 4 x 2 tcgen05.mma (M 128,
 //              N 128, K 16; token half h into the fp32 accumulator in TMEM
 //              columns 128 h .. 128 h + 127) and tcgen05.commit to the
@@ -35,10 +37,13 @@
 //              tcgen05.ld, multiplies by the row scales and stores fp32
 // Every mbarrier wait is bounded; on expiry the CTA records EQ_DEV_TIMEOUT,
 // still releases its tensor memory and stops.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "eqw_device.cuh"
 
@@ -78,6 +83,7 @@ constexpr uint32_t kTmemCols = kTileN * kHalves;        // one fp32 accumulator 
 constexpr size_t kGemmSmem = kStages * kStageBytes + 1024;
 
 struct GemmParams {
+    CUtensorMap tmap_x;       // bf16 [tokens, cols], box 64 x kTileM, 128-byte swizzle
     const uint16_t *x;        // bf16 [tokens, cols]
     const uint8_t *sym;       // [rows, cols]
     const float *scales;      // [rows]
@@ -267,7 +273,7 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
     }
     if (tid == 0) {
         for (uint32_t st = 0; st < kStages; ++st) {
-            mbar_init(full0 + 8 * st, kProducerWarps);
+            mbar_init(full0 + 8 * st, kProducerWarps + 1u);  // + the token tile's expect_tx arrival
             mbar_init(empty0 + 8 * st, 1);
         }
         mbar_init(done, 1);
@@ -281,18 +287,21 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
     bool ok = true;
 
     if (!mma_warp) {
-        // per thread: kXv 16-byte chunks of the token tile and kBv of the symbol tile
-        constexpr uint32_t kXv = kTileM * (kTileK / 8) / kGemmThreads;
+        // per thread: kBv 16-byte chunks of the symbol tile
         constexpr uint32_t kBv = kTileN * (kTileK / 16) / kGemmThreads;
         // this thread's copies of slab `it` into stage `st`
         auto issue = [&](uint32_t it, uint32_t st) {
             const uint32_t k0 = it * kTileK;
-#pragma unroll
-            for (uint32_t i = 0; i < kXv; ++i) {
-                const uint32_t e = tid + i * kGemmThreads, r = e >> 3, k8 = e & 7u;
-                const bool in = m0 + r < P.tokens;
-                const uint16_t *src = in ? P.x + (size_t)(m0 + r) * P.cols + k0 + 8 * k8 : P.x;
-                cp_async16(bufA(st) + tile_offset(r, k8), src, in ? 16u : 0u);
+            // token tile: one TMA tensor copy (x = k0 is a multiple of 64
+            // elements, 128 bytes; rows past the last token read as zeros),
+            // completing on the stage's "full" barrier
+            if (tid == 0) {
+                mbar_expect_tx(full0 + 8 * st, kStageBytesA);
+                asm volatile(
+                    "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                    " [%0], [%1, {%2, %3}], [%4];" ::"r"(bufA(st)),
+                    "l"(reinterpret_cast<uint64_t>(&P.tmap_x)), "r"(k0), "r"(m0), "r"(full0 + 8 * st)
+                    : "memory");
             }
 #pragma unroll
             for (uint32_t i = 0; i < kBv; ++i) {
@@ -410,6 +419,36 @@ __global__ void eq_gemm_outliers_kernel(const uint32_t *rec, uint32_t n_out, con
 
 bool g_gemm_attr_set[128][2];
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Tensor map of the token matrix: inner dimension cols (K), outer tokens;
+// box 64 x kTileM with the 128-byte swizzle the MMA descriptors expect.
+int encode_token_map(CUtensorMap *map, const void *x, uint32_t tokens, uint32_t cols) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return EQ_ERR_CUDA;
+    const cuuint64_t dims[2] = {cols, tokens};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2u};
+    const cuuint32_t box[2] = {kTileK, kTileM};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? EQ_OK : EQ_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" EQW_API int eq_gemm_symbols(const eq_model *m, uint32_t matrix, const void *d_sym, const void *d_x,
@@ -426,6 +465,7 @@ extern "C" EQW_API int eq_gemm_symbols(const eq_model *m, uint32_t matrix, const
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return EQ_ERR_CUDA;
     GemmParams P{};
+    if (const int rc = encode_token_map(&P.tmap_x, d_x, tokens, in.cols)) return rc;
     P.x = static_cast<const uint16_t *>(d_x);
     P.sym = static_cast<const uint8_t *>(d_sym);
     P.scales = reinterpret_cast<const float *>(m->d_blob + d.scales_off);
