@@ -558,13 +558,16 @@ def bench_eqw(args, d: Dist) -> dict | None:
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(copy_stream)
     for _ in range(args.steps):
+        # one copy per resident blob; the blocks of a blob decode as soon as it has landed
+        landed = []
         with torch.cuda.stream(copy_stream):
             for db in stack.d_blobs:
                 db.copy_(pinned, non_blocking=True)
-        ev = torch.cuda.Event()
-        ev.record(copy_stream)
-        streamer.begin(ev)
-        run_pass(streamer)
+                ev = torch.cuda.Event()
+                ev.record(copy_stream)
+                landed.append(ev)
+        streamer.begin(landed[0])
+        streamer.run(None, None, [landed[i // args.distinct_layers] for i in range(len(stack.steps))])
         streamer.join()
         with torch.cuda.stream(streamer.consumer_stream):
             status_host.copy_(streamer.status, non_blocking=True)

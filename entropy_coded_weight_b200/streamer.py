@@ -80,17 +80,23 @@ class PingPongStreamer:
         for ds in set(self.decode_streams):
             self.consumer_stream.wait_stream(ds)
 
-    def run(self, consumer=None, decode_events: list | None = None) -> None:
+    def run(self, consumer=None, decode_events: list | None = None, ready_events: list | None = None) -> None:
         """Enqueue one pass over all steps.
 
         ``consumer(i, step, views, stream)`` is called for step i after its
         buffer is ready, with bf16 matrix views, and must only enqueue work on
         ``stream``.  ``decode_events`` (optional) receives (start, end) CUDA
         events recorded on the decode stream around each block decode.
+        ``ready_events`` (optional, one per step, entries may be None): the
+        decode of step i waits for ``ready_events[i]`` first, e.g. the end of
+        the copy that brings its compressed block into device memory, so the
+        copies of later blocks overlap the decode of earlier ones.
         """
         for i, step in enumerate(self.steps):
             b = step.layer & 1
             ds = self.decode_streams[b]
+            if ready_events is not None and ready_events[i] is not None:
+                ds.wait_event(ready_events[i])
             ev0 = ev1 = None
             if decode_events is not None:
                 # start after the buffer is free so the pair brackets the kernels only

@@ -59,6 +59,47 @@ def test_ping_pong_every_block_bit_exact(eqw, orc):
     model.close()
 
 
+def test_blocks_decode_after_their_copy_lands(eqw, orc):
+    """ready_events: every block of two resident copies waits for the host-to-
+    device copy of its own container copy, issued on a side stream from pinned
+    memory into freshly zeroed device buffers; any decode that ran before its
+    copy landed would read zeros and fail the end check or the comparison."""
+    from entropy_coded_weight_b200.streamer import PingPongStreamer, Step
+    mats = []
+    for layer in range(4):
+        mats += [W.random_int8_matrix(600 + layer, 1024, 1024, layer=layer, index=0),
+                 W.random_int8_matrix(610 + layer, 256, 2048, layer=layer, index=1, n_out=3)]
+    blob = eqw.encode_host(mats)
+    pinned = torch.from_numpy(blob).pin_memory()
+    d_blobs = [torch.zeros(blob.size, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    torch.cuda.synchronize()
+    models = [eqw.Model(d, blob) for d in d_blobs]
+    steps = [Step(models[i // 4], i % 4) for i in range(8)]
+    streamer = PingPongStreamer(steps)
+    side = torch.cuda.Stream()
+    landed = []
+    with torch.cuda.stream(side):
+        for d in d_blobs:
+            torch.cuda._sleep(2_000_000)  # hold the copy back so an unordered decode would overtake it
+            d.copy_(pinned, non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(side)
+            landed.append(ev)
+    copies = {}
+
+    def consumer(i, step, views, stream):
+        copies[i] = [v.clone() for v in views]
+
+    streamer.run(consumer, None, [landed[i // 4] for i in range(8)])
+    torch.cuda.synchronize()
+    assert int(streamer.status.item()) == 0
+    for i in range(8):
+        for j, v in enumerate(copies[i]):
+            assert np.array_equal(_bits(v), orc.dequant_direct(mats[2 * (i % 4) + j])), (i, j)
+    for m in models:
+        m.close()
+
+
 def test_gemv_consumer_against_fp64(eqw):
     torch.manual_seed(0)
     for rows, cols in ((1024, 8192), (8192, 28672), (7, 16)):
