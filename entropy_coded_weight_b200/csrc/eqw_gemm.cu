@@ -67,7 +67,13 @@ constexpr uint32_t kMmaM = 128;                        // tokens per MMA (accumu
 constexpr uint32_t kHalves = EQ_GEMM_HALVES;           // MMAs per widened weight tile
 constexpr uint32_t kTileM = kMmaM * kHalves;           // tokens per CTA tile
 constexpr uint32_t kTileN = 128;                       // weight rows per tile (MMA N, accumulator columns)
-constexpr uint32_t kTileK = 64;                        // K per stage
+#ifndef EQ_GEMM_K
+#define EQ_GEMM_K 64
+#endif
+constexpr uint32_t kTileK = EQ_GEMM_K;                 // K per stage: 64 (128-byte rows) or 32 (64-byte rows)
+static_assert(kTileK == 64 || kTileK == 32, "K per stage");
+constexpr uint32_t kRowBytes = kTileK * 2;             // one bf16 tile row = one swizzle row
+constexpr uint32_t kAtomBytes = 8 * kRowBytes;         // 8-row swizzle atom (SBO)
 constexpr uint32_t kMmaK = 16;                         // K per tcgen05.mma (bf16)
 constexpr uint32_t kStageBytesA = kTileM * kTileK * 2;  // 16 KiB per 128 tokens
 constexpr uint32_t kStageBytesB = kTileN * kTileK * 2;  // 16 KiB
@@ -93,9 +99,6 @@ struct GemmParams {
     uint32_t dtype;
 };
 
-#ifndef EQ_GEMM_SWIZZLE
-#define EQ_GEMM_SWIZZLE 1
-#endif
 
 // Shared-memory matrix descriptor (tcgen05), K-major: start address, leading
 // byte offset, stride byte offset (between 8-row groups), all in 16-byte
@@ -106,7 +109,9 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
     d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
     d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
     d |= (uint64_t)1 << 46;                        // descriptor version for tcgen05
-    if (EQ_GEMM_SWIZZLE) d |= (uint64_t)2 << 61;   // 128-byte swizzle (base offset 0: tiles 1024-aligned)
+    // layout type: 2 = 128-byte swizzle (K 64), 4 = 64-byte swizzle (K 32); base
+    // offset 0: every tile starts on a 1024-byte boundary
+    d |= (uint64_t)(kTileK == 64 ? 2 : 4) << 61;
     return d;
 }
 
@@ -121,23 +126,22 @@ constexpr uint32_t kInstrDesc = (1u << 4)                 // D format fp32
                               | ((kTileN >> 3) << 17)     // N / 8
                               | ((kMmaM >> 4) << 24);     // M / 16
 
-// Byte offset of the 16-byte chunk k8 (bf16 8 k8 .. 8 k8 + 7) of tile row `row`.
-// 128-byte swizzle: each 64-element row is one 128-byte line, 8-row groups are
-// 1024 bytes apart, and chunk k8 of row r sits at chunk position k8 ^ (r % 8).
-// Without swizzle: core matrices of 8 rows x 16 bytes, core (row / 8, k8) at
-// ((row / 8) * 8 + k8) * 128 with rows 16 bytes apart inside it.
+// Byte offset of the 16-byte chunk k8 (bf16 8 k8 .. 8 k8 + 7) of tile row
+// `row` in the swizzled K-major layout: one tile row per swizzle row, 8-row
+// atoms kAtomBytes apart, and chunk k8 of row r at chunk position
+// k8 ^ (r % 8) (128-byte swizzle) or k8 ^ ((r / 2) % 4) (64-byte swizzle):
+// the XOR of the offset's bits 4.. with its bits 7.. that both the TMA copy
+// and the MMA's descriptors apply.
 __device__ __forceinline__ uint32_t tile_offset(uint32_t row, uint32_t k8) {
-    if (EQ_GEMM_SWIZZLE) return (row >> 3) * 1024u + (row & 7u) * 128u + ((k8 ^ (row & 7u)) << 4);
-    return ((row >> 3) * (kTileK / 8) + k8) * 128u + (row & 7u) * 16u;
+    const uint32_t sw = kTileK == 64 ? (row & 7u) : ((row >> 1) & 3u);
+    return (row >> 3) * kAtomBytes + (row & 7u) * kRowBytes + ((k8 ^ sw) << 4);
 }
 
-// Descriptor of K step kk (16 bf16) of a tile at `buf`: 128-byte swizzle
-// advances the start by 32 bytes per step (the hardware applies the XOR),
-// LBO unused (1), SBO 1024; without swizzle two 128-byte cores per step,
-// LBO 128 (K-adjacent cores), SBO 1024 (8-row groups).
+// Descriptor of K step kk (16 bf16) of a tile at `buf`: the start advances by
+// 32 bytes per step inside the swizzle row (the hardware applies the XOR),
+// LBO unused (16), SBO = one 8-row atom.
 __device__ __forceinline__ uint64_t tile_desc(uint32_t buf, uint32_t kk) {
-    if (EQ_GEMM_SWIZZLE) return smem_desc(buf + kk * 32u, 16u, 1024u);
-    return smem_desc(buf + kk * 256u, 128u, 1024u);
+    return smem_desc(buf + kk * 32u, 16u, kAtomBytes);
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
@@ -287,8 +291,9 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
     bool ok = true;
 
     if (!mma_warp) {
-        // per thread: kBv 16-byte chunks of the symbol tile
-        constexpr uint32_t kBv = kTileN * (kTileK / 16) / kGemmThreads;
+        // per thread: kBv 16-byte chunks of the symbol tile (kSymChunks per row)
+        constexpr uint32_t kSymChunks = kTileK / 16;
+        constexpr uint32_t kBv = kTileN * kSymChunks / kGemmThreads;
         // this thread's copies of slab `it` into stage `st`
         auto issue = [&](uint32_t it, uint32_t st) {
             const uint32_t k0 = it * kTileK;
@@ -305,7 +310,7 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
             }
 #pragma unroll
             for (uint32_t i = 0; i < kBv; ++i) {
-                const uint32_t e = tid + i * kGemmThreads, r = e >> 2, c = e & 3u;
+                const uint32_t e = tid + i * kGemmThreads, r = e / kSymChunks, c = e % kSymChunks;
                 cp_async16(bufS(st) + e * 16u, P.sym + (size_t)(n0 + r) * P.cols + k0 + 16 * c, 16u);
             }
         };
@@ -333,7 +338,7 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
             // widen this thread's own symbol chunks of slab `it`
 #pragma unroll
             for (uint32_t i = 0; i < kBv; ++i) {
-                const uint32_t e = tid + i * kGemmThreads, r = e >> 2, c = e & 3u;
+                const uint32_t e = tid + i * kGemmThreads, r = e / kSymChunks, c = e % kSymChunks;
                 uint4 lo, hi;
                 widen16<DT>(ld_shared_v4(bufS(s) + e * 16u), lo, hi);
                 st_shared_v4(bufB(s) + tile_offset(r, 2 * c), lo);
@@ -356,7 +361,7 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
             for (uint32_t kk = 0; kk < kTileK / kMmaK; ++kk)
 #pragma unroll
                 for (uint32_t h = 0; h < kHalves; ++h)  // half h: tokens 128 h .., accumulator columns 128 h ..
-                    tc_mma(tmem + h * kTileN, tile_desc(bufA(s) + h * kMmaM * kTileK * 2u, kk),
+                    tc_mma(tmem + h * kTileN, tile_desc(bufA(s) + h * kMmaM * kRowBytes, kk),
                            tile_desc(bufB(s), kk), (it | kk) != 0u);
             tc_commit(empty0 + 8 * s);
         }
@@ -435,7 +440,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // Tensor map of the token matrix: inner dimension cols (K), outer tokens;
-// box 64 x kTileM with the 128-byte swizzle the MMA descriptors expect.
+// box kTileK x kTileM with the swizzle the MMA descriptors expect.
 int encode_token_map(CUtensorMap *map, const void *x, uint32_t tokens, uint32_t cols) {
     auto enc = tensor_map_encoder();
     if (!enc) return EQ_ERR_CUDA;
@@ -444,7 +449,8 @@ int encode_token_map(CUtensorMap *map, const void *x, uint32_t tokens, uint32_t 
     const cuuint32_t box[2] = {kTileK, kTileM};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           kTileK == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? EQ_OK : EQ_ERR_CUDA;
 }
