@@ -16,7 +16,8 @@
  * Coding used here: rANS, 12-bit frequencies (M = 4096), 32-bit states in
  * [2^16, 2^32), 16-bit renormalisation words, 32 interleaved states per chunk
  * of up to 65536 symbols, per-chunk frequency tables, fp32 per-row scales,
- * fp32 COO outliers.  Byte layout ("container v1", little-endian, sections
+ * fp32 COO outliers; or, per matrix, canonical Huffman codes on the same
+ * chunk and lane layout (EQ_CODEC_HUFFMAN below).  Byte layout ("container v1", little-endian, sections
  * 256-byte aligned):
  *   header (64 B): "EQW1", version 1, format constants, counts, total length;
  *   directory (64 B per matrix): layer, index, dtype, rows, cols, chunk
@@ -35,8 +36,9 @@
  *   - Return value: EQ_OK (0) or one of the EQ_ERR_* codes; nothing throws.
  *   - The caller owns all memory, streams and events.  The library never
  *     allocates device memory, never frees caller memory and never
- *     synchronises a stream or the device, except eq_encode_device, which
- *     synchronises its stream.  The only allocations it makes are host-side
+ *     synchronises a stream or the device, except the device encoders
+ *     (eq_encode_device, eq_encode_device_noalloc), which synchronise their
+ *     stream.  The only allocations it makes are host-side
  *     descriptors and staging (eq_model, eq_encoded, encoder plans).
  *   - Device pointers are plain addresses in the current CUDA device's
  *     memory (from PyTorch: tensor.data_ptr()); streams/events are raw
@@ -244,17 +246,21 @@ EQW_API int eq_block_layout(const eq_model *m, uint32_t layer, size_t *offsets, 
                             size_t *total_bytes);
 
 /* ---- decode (hot path) ------------------------------------------------------
- * Decode one matrix into `d_out` (device, 16-byte aligned, >= 2*rows*cols
- * bytes, row-major bf16): rANS decode + dequant of every chunk (one warp per
- * chunk), then the outlier scatter, both enqueued on `s`.
+ * Decode one matrix into `d_out` (device, 2-byte aligned; 16-byte aligned and
+ * cols % 8 == 0 take the vectorised stores; >= 2*rows*cols bytes, row-major
+ * bf16): rANS or Huffman decode + dequant of every chunk (one warp per chunk,
+ * two chunks per warp in lockstep where they fill whole tiles), then the
+ * outlier scatter, both enqueued on `s`.
  */
 EQW_API int eq_decode_matrix(const eq_model *m, uint32_t matrix, void *d_out, size_t out_bytes,
                              int32_t *d_status, cudaStream_t s);
 
 /*
- * Decode every matrix of `layer` into `d_out` (device, 256-byte aligned,
- * >= eq_block_layout total) in one decode launch plus one scatter launch
- * when the layer has outliers.  EQ_ERR_NOSPACE if out_bytes is too small.
+ * Decode every matrix of `layer` into `d_out` (device, 16-byte aligned,
+ * >= eq_block_layout total): one decode launch per kernel variant the layer
+ * needs (codec x table scope x dtype x output layout; one for a uniform
+ * layer) plus one scatter launch when the layer has outliers.
+ * EQ_ERR_NOSPACE if out_bytes is too small.
  */
 EQW_API int eq_decode_block(const eq_model *m, uint32_t layer, void *d_out, size_t out_bytes,
                             int32_t *d_status, cudaStream_t s);
