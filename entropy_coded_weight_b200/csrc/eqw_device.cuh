@@ -339,52 +339,56 @@ __device__ __forceinline__ void rans_tail(uint32_t lut, uint32_t ring, uint32_t 
 }
 
 // ---- the Huffman step (codec 1) --------------------------------------------------
-// Each lane holds its unread bits left-aligned in `buf` (nb of them).  A lane
-// with fewer than 12 takes the next word (positions by ballot + popcount, as
-// for rANS) into the bits just below its held ones; then the top 12 bits
-// index the slot table, whose entry gives the code length (bits 8..11) and
-// the symbol or its rank (low byte), and the code's bits are shifted out.
+// Each lane holds its unread bits left-aligned in `buf`; `sh` = 16 - (bits
+// held), kept as a signed count so that it is directly the shift that places
+// a refill word just below the held bits.  A lane holding fewer than 12 bits
+// (sh > 4) takes the next word (positions by ballot + popcount, as for rANS);
+// then the top 12 bits index the slot table, whose entry gives the code
+// length (bits 8..11) and the symbol or its rank (low byte), and the code's
+// bits are shifted out.  Shifts by constants and the table address are
+// written as IMADs (FMA pipe), leaving the integer ALU pipe the variable
+// shifts, the merge and the selects.
 __device__ __forceinline__ uint32_t shl_clamped(uint32_t v, uint32_t n) {  // v << n, 0 for n >= 32
     uint32_t r;
     asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(n));
     return r;
 }
 
-__device__ __forceinline__ uint32_t huff_step(uint32_t lut, uint32_t &rp, uint32_t &buf, uint32_t &nb,
+__device__ __forceinline__ uint32_t huff_step(uint32_t lut, uint32_t &rp, uint32_t &buf, uint32_t &sh,
                                               uint32_t lt) {
-    const bool need = nb < kHuffMaxLen;
+    const bool need = static_cast<int32_t>(sh) > static_cast<int32_t>(16u - kHuffMaxLen);
     const uint32_t b = __ballot_sync(kFull, need);
     const uint32_t w = lds_u16(mad_lo(__popc(b & lt), 2u, rp));
-    const uint32_t filled = buf | shl_clamped(w, 16u - nb);
+    const uint32_t filled = buf | shl_clamped(w, sh);
     buf = need ? filled : buf;
-    nb = need ? nb + 16u : nb;
+    sh = need ? sh - 16u : sh;
     rp = mad_lo(__popc(b), 2u, rp);
-    const uint32_t e = lds_u32(lut + 4u * (buf >> (32u - kHuffMaxLen)));
-    const uint32_t len = e >> 8;
+    const uint32_t e = lds_u32(mad_lo(mad_hi(buf, 1u << kHuffMaxLen, 0u), 4u, lut));  // lut + 4 * (buf >> 20)
+    const uint32_t len = mad_hi(e, 1u << 24, 0u);                                      // e >> 8
     buf = shl_clamped(buf, len);
-    nb -= len;
+    sh += len;
     return e;
 }
 
 // Last, partial group (lane l active at step r while 8l + r < rem).
-__device__ __forceinline__ void huff_tail(uint32_t lut, uint32_t ring, uint32_t &buf, uint32_t &nb, uint32_t &pw,
+__device__ __forceinline__ void huff_tail(uint32_t lut, uint32_t ring, uint32_t &buf, uint32_t &sh, uint32_t &pw,
                                           uint32_t lt, uint32_t lane, uint32_t rem, uint32_t (&e8)[8]) {
 #pragma unroll
     for (uint32_t r = 0; r < 8; ++r) {
         const bool active = lane * kGroup + r < rem;
-        const bool need = active && nb < kHuffMaxLen;
+        const bool need = active && static_cast<int32_t>(sh) > static_cast<int32_t>(16u - kHuffMaxLen);
         const uint32_t b = __ballot_sync(kFull, need);
         const uint32_t w = lds_u16(ring + ((pw + 2u * __popc(b & lt)) & (kRingBytes - 1)));
         if (need) {
-            buf |= w << (16u - nb);
-            nb += 16u;
+            buf |= w << sh;
+            sh -= 16u;
         }
         pw += 2u * __popc(b);
         if (active) {
             const uint32_t e = lds_u32(lut + 4u * (buf >> (32u - kHuffMaxLen)));
             const uint32_t len = e >> 8;
             buf = shl_clamped(buf, len);
-            nb -= len;
+            sh += len;
             e8[r] = e;
         }
     }
@@ -393,25 +397,25 @@ __device__ __forceinline__ void huff_tail(uint32_t lut, uint32_t ring, uint32_t 
 // Per-lane decoder state of a codec, its step, tail, start and end checks.
 template <uint32_t CODEC> struct CodecState;
 template <> struct CodecState<kCodecRans> { uint32_t x; };
-template <> struct CodecState<kCodecHuffman> { uint32_t buf, nb; };
+template <> struct CodecState<kCodecHuffman> { uint32_t buf, sh; };
 
 template <uint32_t CODEC>
 __device__ __forceinline__ uint32_t codec_step(uint32_t lut, uint32_t &rp, CodecState<CODEC> &s, uint32_t lt) {
-    if constexpr (CODEC == kCodecHuffman) return huff_step(lut, rp, s.buf, s.nb, lt);
+    if constexpr (CODEC == kCodecHuffman) return huff_step(lut, rp, s.buf, s.sh, lt);
     else return rans_step(lut, rp, s.x, lt);
 }
 
 template <uint32_t CODEC>
 __device__ __forceinline__ void codec_tail(uint32_t lut, uint32_t ring, CodecState<CODEC> &s, uint32_t &pw,
                                            uint32_t lt, uint32_t lane, uint32_t rem, uint32_t (&e8)[8]) {
-    if constexpr (CODEC == kCodecHuffman) huff_tail(lut, ring, s.buf, s.nb, pw, lt, lane, rem, e8);
+    if constexpr (CODEC == kCodecHuffman) huff_tail(lut, ring, s.buf, s.sh, pw, lt, lane, rem, e8);
     else rans_tail(lut, ring, s.x, pw, lt, lane, rem, e8);
 }
 
 // rANS: the state from the record; Huffman: no bits held.
 template <uint32_t CODEC>
 __device__ __forceinline__ CodecState<CODEC> codec_start(uint32_t x0) {
-    if constexpr (CODEC == kCodecHuffman) return CodecState<CODEC>{0u, 0u};
+    if constexpr (CODEC == kCodecHuffman) return CodecState<CODEC>{0u, 16u};  // no bits held
     else return CodecState<CODEC>{x0};
 }
 
