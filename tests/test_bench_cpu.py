@@ -44,3 +44,10 @@ def test_oracle_rate_counts_whole_chunks():
     # 96 x 2048 = three full chunks of 64 Ki symbols
     assert done == n_sample * 65536
     assert dt >= 0.05
+
+
+def test_oracle_rate_decodes_huffman_containers():
+    m = W.random_int8_matrix(41, 64, 1024)  # one full chunk
+    blob = oracle.encode_container([m], codec="huffman")
+    done, n_sample, dt, n_chunks = bench.oracle_rate(blob, 1, 0.01)
+    assert n_chunks == 1 and done == n_sample * 65536
