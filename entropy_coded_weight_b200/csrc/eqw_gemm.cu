@@ -62,7 +62,7 @@ constexpr int kGemmThreads = EQ_GEMM_THREADS;  // 4 or 8 warps
 #ifndef EQ_GEMM_STAGES
 #define EQ_GEMM_STAGES 4
 #endif
-static_assert(EQ_GEMM_HALVES == 1 || EQ_GEMM_HALVES == 2, "one or two token halves per CTA");
+static_assert(EQ_GEMM_HALVES >= 1 && EQ_GEMM_HALVES <= 4, "one to four 128-token parts per CTA");
 constexpr uint32_t kMmaM = 128;                        // tokens per MMA (accumulator lanes)
 constexpr uint32_t kHalves = EQ_GEMM_HALVES;           // MMAs per widened weight tile
 constexpr uint32_t kTileM = kMmaM * kHalves;           // tokens per CTA tile
@@ -85,11 +85,15 @@ constexpr uint32_t kAhead = EQ_GEMM_AHEAD;              // slabs whose copies ar
 static_assert(kAhead < kStages, "a stage is refilled only after its previous slab's MMAs");
 constexpr uint32_t kStageBytesS = kTileN * kTileK;      // 8 KiB of symbol bytes (staging)
 constexpr uint32_t kStageBytes = kStageBytesA + kStageBytesB + kStageBytesS;
-constexpr uint32_t kTmemCols = kTileN * kHalves;        // one fp32 accumulator per token half
+constexpr uint32_t kTmemCols = kTileN * kHalves;        // one fp32 accumulator per token part
+// tcgen05.alloc takes a power of two of at least 32 columns
+constexpr uint32_t kTmemAlloc = kTmemCols <= 32 ? 32 : kTmemCols <= 64 ? 64 : kTmemCols <= 128 ? 128
+                              : kTmemCols <= 256 ? 256 : 512;
+static_assert(kTmemCols <= 512, "tensor memory has 512 columns");
 constexpr size_t kGemmSmem = kStages * kStageBytes + 1024;
 
 struct GemmParams {
-    CUtensorMap tmap_x;       // bf16 [tokens, cols], box 64 x kTileM, 128-byte swizzle
+    CUtensorMap tmap_x;       // bf16 [tokens, cols], box kTileK x 128 (one per token part), swizzled
     const uint16_t *x;        // bf16 [tokens, cols]
     const uint8_t *sym;       // [rows, cols]
     const float *scales;      // [rows]
@@ -272,7 +276,7 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32(&tmem_base_s)), "r"(kTmemCols) : "memory");
+                     ::"r"(smem_u32(&tmem_base_s)), "r"(kTmemAlloc) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
@@ -302,11 +306,14 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
             // completing on the stage's "full" barrier
             if (tid == 0) {
                 mbar_expect_tx(full0 + 8 * st, kStageBytesA);
-                asm volatile(
-                    "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-                    " [%0], [%1, {%2, %3}], [%4];" ::"r"(bufA(st)),
-                    "l"(reinterpret_cast<uint64_t>(&P.tmap_x)), "r"(k0), "r"(m0), "r"(full0 + 8 * st)
-                    : "memory");
+#pragma unroll
+                for (uint32_t h = 0; h < kHalves; ++h)  // one 128-token box per part
+                    asm volatile(
+                        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                        " [%0], [%1, {%2, %3}], [%4];" ::"r"(bufA(st) + h * kMmaM * kRowBytes),
+                        "l"(reinterpret_cast<uint64_t>(&P.tmap_x)), "r"(k0), "r"(m0 + h * kMmaM),
+                        "r"(full0 + 8 * st)
+                        : "memory");
             }
 #pragma unroll
             for (uint32_t i = 0; i < kBv; ++i) {
@@ -401,7 +408,7 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemAlloc)
                      : "memory");
     }
 }
@@ -446,7 +453,7 @@ int encode_token_map(CUtensorMap *map, const void *x, uint32_t tokens, uint32_t 
     if (!enc) return EQ_ERR_CUDA;
     const cuuint64_t dims[2] = {cols, tokens};
     const cuuint64_t strides[1] = {(cuuint64_t)cols * 2u};
-    const cuuint32_t box[2] = {kTileK, kTileM};
+    const cuuint32_t box[2] = {kTileK, kMmaM};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE,
