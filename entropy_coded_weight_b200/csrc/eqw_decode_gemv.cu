@@ -74,6 +74,7 @@ struct GemvParams {
     uint32_t n_mats;
     uint32_t total_units;
     uint32_t tile_warps;          // shared-table kernels: warps that take chunks of a tile (assign_tiles)
+    uint32_t tile_chains;         // shared-table kernels: chunks per warp in a tile, 1 or 2 (assign_tiles)
     GemvJob mats[kMaxMatsPerLaunch];
 };
 
@@ -391,8 +392,8 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kGemvMinCtas : 1)
         for (uint32_t unit = blockIdx.x; unit < P.total_units; unit += gridDim.x) {
             const uint32_t mi = job_of(P, unit);
             const GemvJob &M = P.mats[mi];
-            const uint32_t TW = P.tile_warps;
-            const uint32_t k0 = (unit - M.begin) * TW * C;
+            const uint32_t TW = P.tile_warps, TC = P.tile_chains;
+            const uint32_t k0 = (unit - M.begin) * TW * TC;
             if (mi != cur_mat) {
                 shared_table_rebuild<WARPS, LAYOUT, CODEC>(P, M, k0, lane, warp, S);
                 cur_mat = mi;
@@ -403,7 +404,7 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kGemvMinCtas : 1)
             bool have[C];
             for (uint32_t c = 0; c < C; ++c) {
                 const uint32_t k = k0 + warp + c * TW;
-                have[c] = warp < TW && k < M.n_chunks && !ctl[0].dead && !ctl[C - 1].dead;
+                have[c] = c < TC && warp < TW && k < M.n_chunks && !ctl[0].dead && !ctl[C - 1].dead;
                 if (have[c]) have[c] = shared_chunk_head<CODEC>(P, M, k, lane, np, S, hc[c]);
             }
             if constexpr (C == 2) {

@@ -731,24 +731,32 @@ int setup_kernel(KernelSetup<Params> &k, void (*fn)(Params), int warps, size_t s
 }
 
 // Shared-table kernels take their chunks in tiles: tile t of a matrix holds
-// chunks [t * W * chains, (t + 1) * W * chains), warp w of the block decoding
-// chunks w, w + W, ... of it.  W (P.tile_warps) is the fewest warps per tile
-// that still fit the whole launch into one round of resident blocks, so that
-// a block of small matrices spreads over every SM instead of filling a few of
-// them with full tiles; when even full tiles (W = max_warps) need more than
-// one round, W = max_warps.  Sets every matrix's first unit and the total.
+// chunks [t * W * C, (t + 1) * W * C), warp w of the block decoding chunks
+// w, w + W, ... (C of them, in lockstep when C = 2) of it.  A launch whose
+// tiles of max_warps single chunks fit one round of resident blocks runs one
+// chain per warp (C = 1: a small launch is bound by the latency of each
+// chunk's 2048 dependent steps, and a warp with one chain steps faster than
+// one with two); otherwise C = max_chains.  W (P.tile_warps) is the fewest
+// warps per tile that still fit the launch into one round, so that a block of
+// small matrices spreads over every SM instead of filling a few of them with
+// full tiles; when even full tiles need more than one round, W = max_warps.
+// Sets the tile shape, every matrix's first unit and the total.
 template <class Params>
-void assign_tiles(Params &P, uint32_t resident, uint32_t max_warps, uint32_t chains) {
-    uint32_t tw = max_warps;
-    for (uint32_t w = 1; w < max_warps; ++w) {
+void assign_tiles(Params &P, uint32_t resident, uint32_t max_warps, uint32_t max_chains) {
+    auto units_for = [&](uint32_t w, uint32_t c) {
         uint64_t units = 0;
-        for (uint32_t i = 0; i < P.n_mats; ++i) units += (P.mats[i].n_chunks + w * chains - 1) / (w * chains);
-        if (units <= resident) {
+        for (uint32_t i = 0; i < P.n_mats; ++i) units += (P.mats[i].n_chunks + w * c - 1) / (w * c);
+        return units;
+    };
+    const uint32_t chains = units_for(max_warps, 1) <= resident ? 1u : max_chains;
+    uint32_t tw = max_warps;
+    for (uint32_t w = 1; w < max_warps; ++w)
+        if (units_for(w, chains) <= resident) {
             tw = w;
             break;
         }
-    }
     P.tile_warps = tw;
+    P.tile_chains = chains;
     P.total_units = 0;
     for (uint32_t i = 0; i < P.n_mats; ++i) {
         P.mats[i].begin = P.total_units;

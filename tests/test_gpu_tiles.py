@@ -1,12 +1,14 @@
-"""Shared-table launches at every tile width.
+"""Shared-table launches at every tile shape.
 
 The shared-table kernels take a matrix's chunks in tiles of (warps per tile) x
-2 chunks, using as few warps per tile as keep the launch within one block per
-SM.  The cases below are sized so that the chosen width runs from 1 to the
-full block, with ragged last tiles, and decode and fused decode + GEMV are
-compared with the oracle: decode bit for bit, GEMV within the bound of
-test_gpu_fused_gemv.  `tile_warps` mirrors the host rule so each case states
-which width it exercises.
+(chunks per warp): one chunk per warp when tiles of 24 single chunks fit one
+round of resident blocks (one per SM), else two in lockstep; as few warps per
+tile as keep the launch within one round.  The cases below are sized so that
+the chosen shape runs from 1 warp to the full block with one and with two
+chains per warp, with ragged last tiles, and decode and fused decode + GEMV
+are compared with the oracle: decode bit for bit, GEMV within the bound of
+test_gpu_fused_gemv.  `tile_shape` mirrors the host rule so each case states
+which shape it exercises.
 """
 import numpy as np
 import pytest
@@ -31,11 +33,14 @@ def eqw():
     return E
 
 
-def tile_warps(n_chunks: list[int], resident: int) -> int:
+def tile_shape(n_chunks: list[int], resident: int) -> tuple[int, int]:
+    def units(w, c):
+        return sum(-(-n // (w * c)) for n in n_chunks)
+    chains = 1 if units(FULL_WARPS, 1) <= resident else CHAINS
     for w in range(1, FULL_WARPS):
-        if sum(-(-n // (w * CHAINS)) for n in n_chunks) <= resident:
-            return w
-    return FULL_WARPS
+        if units(w, chains) <= resident:
+            return w, chains
+    return FULL_WARPS, chains
 
 
 def _bits(t):
@@ -54,10 +59,11 @@ def _matrix(seed, n_chunks, cols=4096, layer=0, index=0, n_out=0):
 CASES = {
     "one_chunk": [1],
     "one_tile_ragged": [3],
-    "width_1_many_tiles": [290],
-    "width_2": [300],
-    "width_7_ragged": [2000],
+    "width_2_many_tiles": [290],
+    "width_3": [300],
+    "width_14_ragged": [2000],
     "block_mixed": [16, 64, 700, 700, 1100],
+    "two_chains_width_17": [5000],
 }
 
 
@@ -65,8 +71,8 @@ CASES = {
 def test_decode_block_bit_exact(eqw, orc, name):
     counts = CASES[name]
     mats = [_matrix(500 + i, n, index=i, n_out=4 if i == 0 else 0) for i, n in enumerate(counts)]
-    tw = tile_warps(counts, _sms())
-    assert 1 <= tw <= FULL_WARPS
+    tw, tc = tile_shape(counts, _sms())
+    assert 1 <= tw <= FULL_WARPS and tc in (1, 2)
     blob = eqw.encode_host(mats)
     model = eqw.Model(eqw.upload(blob), blob)
     offs, total = model.block_layout(0)
@@ -78,20 +84,25 @@ def test_decode_block_bit_exact(eqw, orc, name):
     host = out.cpu().numpy()
     for m, o in zip(mats, offs):
         got = host[o:o + 2 * m.n].view(np.uint16).reshape(m.rows, m.cols)
-        assert np.array_equal(got, orc.dequant_direct(m)), (name, tw, m.index)
+        assert np.array_equal(got, orc.dequant_direct(m)), (name, tw, tc, m.index)
     model.close()
 
 
-def test_width_range_is_covered():
-    """On a 148-SM B200 the cases above span widths 1, 2, 7 and a mixed block."""
-    widths = {name: tile_warps(c, 148) for name, c in CASES.items()}
-    assert widths["one_chunk"] == 1 and widths["width_1_many_tiles"] == 1
-    assert widths["width_2"] == 2
-    assert widths["width_7_ragged"] == 7
-    assert tile_warps([13056], 148) == FULL_WARPS  # a Llama-70B-shape block keeps full tiles
+def test_shape_range_is_covered():
+    """On a 148-SM B200 the cases above span one-chain widths 1 to 18 and a
+    two-chain width of 17; 7B- and 70B-shape blocks get (22, 1) and (24, 2)."""
+    shapes = {name: tile_shape(c, 148) for name, c in CASES.items()}
+    assert shapes["one_chunk"] == (1, 1) and shapes["one_tile_ragged"] == (1, 1)
+    assert shapes["width_2_many_tiles"] == (2, 1)
+    assert shapes["width_3"] == (3, 1)
+    assert shapes["width_14_ragged"] == (14, 1)
+    assert shapes["block_mixed"] == (18, 1)
+    assert shapes["two_chains_width_17"] == (17, 2)
+    assert tile_shape([256] * 4 + [688] * 3, 148) == (22, 1)     # Llama-7B-shape block
+    assert tile_shape([1024, 128, 128, 1024, 3584, 3584, 3584], 148) == (FULL_WARPS, 2)  # Llama-70B shape
 
 
-@pytest.mark.parametrize("name", ["one_tile_ragged", "width_2", "width_7_ragged", "block_mixed"])
+@pytest.mark.parametrize("name", ["one_tile_ragged", "width_3", "width_14_ragged", "block_mixed", "two_chains_width_17"])
 def test_fused_gemv_within_bound(eqw, orc, name):
     counts = CASES[name]
     mats = [_matrix(600 + i, n, cols=8192, index=i) for i, n in enumerate(counts)]
