@@ -197,6 +197,12 @@ class Model:
             self._L.eq_model_close(self._m)
             self._m = None
 
+    def set_sm_limit(self, max_sms: int) -> None:
+        """eq_model_set_sm_limit: decode launches of this model use at most
+        ``max_sms`` SMs (0: all), leaving the rest to a kernel that runs beside
+        them, e.g. the consumer of the previous block."""
+        check(self._L.eq_model_set_sm_limit(self._m, int(max_sms)), "eq_model_set_sm_limit")
+
     def __del__(self):
         try:
             self.close()

@@ -63,6 +63,7 @@ SIGNATURES = {
     "eq_encode_host": (_i32, [_P(eq_matrix_in), _u32, _i32, _vp, _sz, _P(_sz)]),
     "eq_model_open": (_i32, [_vp, _sz, _vp, _P(_vp)]),
     "eq_model_close": (None, [_vp]),
+    "eq_model_set_sm_limit": (_i32, [_vp, ctypes.c_uint32]),
     "eq_model_counts": (_i32, [_vp, _P(_u32), _P(_u32)]),
     "eq_matrix_get_info": (_i32, [_vp, _u32, _P(eq_matrix_info)]),
     "eq_layer_matrices": (_i32, [_vp, _u32, _P(_u32), _P(_u32)]),

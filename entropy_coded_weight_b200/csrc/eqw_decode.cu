@@ -790,6 +790,7 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
     DeviceSetup *dev = nullptr;
     int rc = device_setup(&dev);
     if (rc) return rc;
+    const int sms = m->sm_limit && m->sm_limit < (uint32_t)dev->sms ? (int)m->sm_limit : dev->sms;
     for (uint32_t base = 0; base < count; base += kMaxMatsPerLaunch) {
         const uint32_t cnt = std::min<uint32_t>(kMaxMatsPerLaunch, count - base);
         DecodeParams P[2][2][2][4];
@@ -839,13 +840,13 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
             for (int dt = 0; dt < 2; ++dt)
                 for (int lay = 0; lay < 4; ++lay) {
                     const auto &k = dev->k[co][1][dt][lay];
-                    assign_tiles(P[co][1][dt][lay], (uint32_t)(dev->sms * k.ctas_per_sm), kSharedWarps, EQ_CHAINS);
+                    assign_tiles(P[co][1][dt][lay], (uint32_t)(sms * k.ctas_per_sm), kSharedWarps, EQ_CHAINS);
                 }
         for (int co = 0; co < 2; ++co)
             for (int sh = 0; sh < 2; ++sh)
                 for (int dt = 0; dt < 2; ++dt)
                     for (int lay = 0; lay < 4; ++lay)
-                        if ((rc = launch(dev->k[co][sh][dt][lay], dev->sms, P[co][sh][dt][lay], s))) return rc;
+                        if ((rc = launch(dev->k[co][sh][dt][lay], sms, P[co][sh][dt][lay], s))) return rc;
         if (n_out) {
             eq_outlier_scatter_kernel<<<(n_out + 127) / 128, 128, 0, s>>>(Q);
             if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;

@@ -522,6 +522,7 @@ int launch_gemv(const eq_model *m, uint32_t first, uint32_t count, const void *c
     if (rc) return rc;
     GemvSetup *dev = nullptr;
     if ((rc = gemv_setup(&dev))) return rc;
+    const int sms = m->sm_limit && m->sm_limit < (uint32_t)dev->sms ? (int)m->sm_limit : dev->sms;
     for (uint32_t base = 0; base < count; base += kMaxMatsPerLaunch) {
         const uint32_t cnt = std::min<uint32_t>(kMaxMatsPerLaunch, count - base);
         ZeroParams Z{};
@@ -567,12 +568,12 @@ int launch_gemv(const eq_model *m, uint32_t first, uint32_t count, const void *c
         }
         for (int co = 0; co < 2; ++co)
             for (int dt = 0; dt < 2; ++dt)
-                assign_tiles(P[co][1][dt], (uint32_t)(dev->sms * dev->k[co][1][dt].ctas_per_sm), kGemvWarps,
+                assign_tiles(P[co][1][dt], (uint32_t)(sms * dev->k[co][1][dt].ctas_per_sm), kGemvWarps,
                              EQ_CHAINS);
         for (int co = 0; co < 2; ++co)
             for (int sh = 0; sh < 2; ++sh)
                 for (int dt = 0; dt < 2; ++dt)
-                    if ((rc = launch(dev->k[co][sh][dt], dev->sms, P[co][sh][dt], s))) return rc;
+                    if ((rc = launch(dev->k[co][sh][dt], sms, P[co][sh][dt], s))) return rc;
     }
     return EQ_OK;
 }

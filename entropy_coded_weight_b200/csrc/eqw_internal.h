@@ -51,6 +51,7 @@ struct eq_model {
     const uint8_t *d_blob;
     size_t len;
     uint32_t n_layers;
+    uint32_t sm_limit = 0;  // decode launches use at most this many SMs (0: all)
     std::vector<eqw::MatrixDesc> mats;
     std::vector<uint32_t> layer_first;
     std::vector<uint32_t> layer_count;

@@ -214,6 +214,12 @@ extern "C" EQW_API int eq_model_open(const void *d_blob, size_t len, const void 
 
 extern "C" EQW_API void eq_model_close(eq_model *m) { delete m; }
 
+extern "C" EQW_API int eq_model_set_sm_limit(eq_model *m, uint32_t max_sms) {
+    if (!m) return EQ_ERR_INVALID_ARG;
+    m->sm_limit = max_sms;
+    return EQ_OK;
+}
+
 extern "C" EQW_API int eq_model_counts(const eq_model *m, uint32_t *n_layers, uint32_t *n_matrices) {
     if (!m) return EQ_ERR_INVALID_ARG;
     if (n_layers) *n_layers = m->n_layers;

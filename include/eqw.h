@@ -230,6 +230,16 @@ EQW_API int eq_model_open(const void *d_blob, size_t len, const void *h_blob, eq
 /* Free the host descriptor (NULL is ignored).  Device memory is the caller's. */
 EQW_API void eq_model_close(eq_model *m);
 
+/*
+ * Let this model's decode launches (eq_decode_*, eq_decode_gemv_*) use at
+ * most `max_sms` SMs (0: all, the default).  The decode kernels keep one
+ * block per SM for the whole launch, so a kernel that must run beside them
+ * -- the consumer of the previous block in a streamed forward pass -- only
+ * gets SMs they leave free.  Host-side setting; takes effect for launches
+ * enqueued after the call.  Errors: EQ_ERR_INVALID_ARG (m NULL).
+ */
+EQW_API int eq_model_set_sm_limit(eq_model *m, uint32_t max_sms);
+
 EQW_API int eq_model_counts(const eq_model *m, uint32_t *n_layers, uint32_t *n_matrices);
 EQW_API int eq_matrix_get_info(const eq_model *m, uint32_t matrix, eq_matrix_info *info);
 

@@ -322,3 +322,14 @@ def test_huffman_size_near_entropy(eqw, orc):
         p = c[c > 0] / n_k
         shannon += n_k * float(-(p * np.log2(p)).sum()) / 8
     assert shannon <= payload <= shannon + flat.size / 8
+
+
+def test_sm_limit_is_a_host_setting(eqw, orc):
+    blob = orc.encode_container(_ragged(41))
+    rc, h = _open(eqw, blob)
+    assert rc == 0
+    L = eqw.load()
+    assert L.eq_model_set_sm_limit(h, 17) == 0
+    assert L.eq_model_set_sm_limit(h, 0) == 0
+    assert L.eq_model_set_sm_limit(None, 4) == 1  # EQ_ERR_INVALID_ARG
+    L.eq_model_close(h)

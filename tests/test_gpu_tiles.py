@@ -113,3 +113,31 @@ def test_fused_gemv_within_bound(eqw, orc, name):
         ref, mag = orc.gemv_exact(orc.dequant_direct(m), _bits(_x_for(m)))
         ok, info = _bound_ok(y, ref, mag, m.cols, _n_out_rows(m))
         assert ok, (name, m.index, info)
+
+
+@pytest.mark.parametrize("limit", [1, 7, 100])
+def test_sm_limit_keeps_results(eqw, orc, limit):
+    """eq_model_set_sm_limit: fewer resident blocks, more rounds per block; the
+    decoded block and the fused GEMV stay exact / within bound."""
+    counts = [700, 1100]
+    mats = [_matrix(700 + i, n, cols=8192, index=i) for i, n in enumerate(counts)]
+    blob = eqw.encode_host(mats)
+    model = eqw.Model(eqw.upload(blob), blob)
+    model.set_sm_limit(limit)
+    offs, total = model.block_layout(0)
+    out = torch.empty(total, dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    model.decode_block(0, out, status)
+    xs = [_x_for(m).cuda() for m in mats]
+    ys = [torch.empty(m.rows, dtype=torch.float32, device="cuda") for m in mats]
+    model.decode_gemv_block(0, xs, ys, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    host = out.cpu().numpy()
+    for m, o, y in zip(mats, offs, ys):
+        w = orc.dequant_direct(m)
+        assert np.array_equal(host[o:o + 2 * m.n].view(np.uint16).reshape(m.rows, m.cols), w)
+        ref, mag = orc.gemv_exact(w, _bits(_x_for(m)))
+        ok, info = _bound_ok(y.cpu().numpy(), ref, mag, m.cols, _n_out_rows(m))
+        assert ok, (limit, m.index, info)
+    model.close()
