@@ -66,7 +66,11 @@ static_assert(EQ_GEMM_HALVES >= 1 && EQ_GEMM_HALVES <= 4, "one to four 128-token
 constexpr uint32_t kMmaM = 128;                        // tokens per MMA (accumulator lanes)
 constexpr uint32_t kHalves = EQ_GEMM_HALVES;           // MMAs per widened weight tile
 constexpr uint32_t kTileM = kMmaM * kHalves;           // tokens per CTA tile
-constexpr uint32_t kTileN = 128;                       // weight rows per tile (MMA N, accumulator columns)
+#ifndef EQ_GEMM_TILE_N
+#define EQ_GEMM_TILE_N 128
+#endif
+constexpr uint32_t kTileN = EQ_GEMM_TILE_N;            // weight rows per tile (MMA N, accumulator columns)
+static_assert(kTileN % 16 == 0 && kTileN >= 16 && kTileN <= 256, "cta_group::1 MMA with M = 128: N in 16..256");
 #ifndef EQ_GEMM_K
 #define EQ_GEMM_K 64
 #endif
