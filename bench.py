@@ -687,6 +687,20 @@ def _checksums_device(w):
     return torch.stack([v.sum(), (v.sum(1) * r).sum(), (v.sum(0) * c).sum()])
 
 
+def configs_table_row(row: dict) -> str:
+    """One markdown row of the per-workload results table from a `--configs` JSON line."""
+    fl = row["l2_flushed"]
+    if "hot" in row:
+        gbs = f"{row['hot']['decoded_gb_s']:.1f} / {fl['decoded_gb_s']:.1f}"
+        gsym = f"{row['hot']['gsym_s']:.2f} / {fl['gsym_s']:.2f}"
+    else:
+        gbs, gsym = f"{fl['decoded_gb_s']:.0f}", f"{fl['gsym_s']:.0f}"
+    o = row["oracle"]
+    return (f"| {row['config']}: {row['workload']} | {row['symbols']:,} | {row['bits_per_sym_records']:.3f} / "
+            f"{row['bits_per_sym_container']:.3f} | {gbs} | {gsym} | {100 * fl['hbm_frac']:.1f} % | "
+            f"{'yes' if row['bit_exact'] else 'NO'} | {o['gsym_s_1core']:.3f} | {o['gsym_s_all']:.2f} |")
+
+
 def bench_configs(args) -> None:
     """One JSON line per workload: decode throughput of one block per launch
     (inputs in HBM, L2 rewritten between launches), compression, bit-exactness
@@ -748,6 +762,7 @@ def bench_configs(args) -> None:
                          "cores": cores, "sample_s": [round(t1, 1), round(ta, 1)]}
         row["peak"] = {"hbm_gbs": peak, "kind": peak_kind}
         print(json.dumps(row), flush=True)
+        print(configs_table_row(row), file=sys.stderr, flush=True)
         model.close()
         del mats, blob, model
 

@@ -51,3 +51,17 @@ def test_oracle_rate_decodes_huffman_containers():
     blob = oracle.encode_container([m], codec="huffman")
     done, n_sample, dt, n_chunks = bench.oracle_rate(blob, 1, 0.01)
     assert n_chunks == 1 and done == n_sample * 65536
+
+
+def test_configs_table_row_formats_a_result_line():
+    row = {"config": "2a", "workload": "Llama-7B-shape block, Int8 ~2.1 bits/sym", "symbols": 202375168,
+           "bits_per_sym_records": 2.1251, "bits_per_sym_container": 2.133, "bit_exact": True,
+           "l2_flushed": {"launch_ms": 0.231, "decoded_gb_s": 1751.8, "gsym_s": 875.92, "hbm_frac": 0.3078},
+           "oracle": {"gsym_s_1core": 0.04253, "gsym_s_all": 0.42649, "cores": 16}}
+    line = bench.configs_table_row(row)
+    assert line.startswith("| 2a: Llama-7B-shape block") and line.endswith("|")
+    cells = [c.strip() for c in line.strip("|").split("|")]
+    assert cells[1] == "202,375,168" and cells[2] == "2.125 / 2.133" and cells[3] == "1752"
+    assert cells[5] == "30.8 %" and cells[6] == "yes" and cells[8] == "0.43"
+    hot = dict(row, hot={"decoded_gb_s": 11.4, "gsym_s": 5.68, "hbm_frac": 0.002})
+    assert "11.4 / 1751.8" in bench.configs_table_row(hot)
