@@ -233,6 +233,14 @@ class Model:
     def block_bytes(self, layer: int) -> int:
         return self.block_layout(layer)[1]
 
+    def decode_plan(self, layer: int, sms: int) -> list[int]:
+        """eq_decode_plan: per matrix of ``layer``, the leading chunks the
+        two-chunks-per-warp kernel decodes on a GPU with ``sms`` SMs."""
+        n = len(self.layer_matrices(layer))
+        out = (ctypes.c_uint32 * max(1, n))()
+        check(self._L.eq_decode_plan(self._m, layer, sms, out, n), "eq_decode_plan")
+        return [out[i] for i in range(n)]
+
     def decode_matrix(self, matrix: int, out, status, stream=None) -> None:
         """eq_decode_matrix into ``out`` (device tensor, >= 2*rows*cols bytes)."""
         nbytes = out.numel() * out.element_size()

@@ -68,6 +68,7 @@ SIGNATURES = {
     "eq_matrix_get_info": (_i32, [_vp, _u32, _P(eq_matrix_info)]),
     "eq_layer_matrices": (_i32, [_vp, _u32, _P(_u32), _P(_u32)]),
     "eq_block_layout": (_i32, [_vp, _u32, _P(_sz), _u32, _P(_sz)]),
+    "eq_decode_plan": (_i32, [_vp, _u32, _u32, _P(_u32), _u32]),
     "eq_decode_matrix": (_i32, [_vp, _u32, _vp, _sz, _vp, _vp]),
     "eq_decode_block": (_i32, [_vp, _u32, _vp, _sz, _vp, _vp]),
     "eq_decode_model_stream": (_i32, [_vp, _u32, _P(_vp), _sz, _vp, _vp, _P(_vp), _P(_vp)]),

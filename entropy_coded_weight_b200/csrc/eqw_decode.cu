@@ -54,6 +54,11 @@
 #include <vector>
 
 #include "eqw_device.cuh"
+#include "eqw_pairs.h"
+
+#ifndef EQ_USE_PAIRS
+#define EQ_USE_PAIRS 1
+#endif
 
 namespace {
 
@@ -64,6 +69,7 @@ struct MatJob {
     uint64_t n_elems;
     uint32_t cols;
     uint32_t n_chunks;
+    uint32_t chunk0;              // first chunk decoded here (the pair kernel took the ones before)
     uint32_t begin;               // first launch-wide work unit (tile or chunk) of this matrix
     uint32_t dtype;
     uint32_t layout;              // kRowUniform: cols % 256 == 0; kLaneRows: cols % 8 == 0; else kGeneric
@@ -618,7 +624,7 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
             const uint32_t mi = job_of(P, unit);
             const MatJob &M = P.mats[mi];
             const uint32_t TW = P.tile_warps, TC = P.tile_chains;
-            const uint32_t k0 = (unit - M.begin) * TW * TC;
+            const uint32_t k0 = M.chunk0 + (unit - M.begin) * TW * TC;
             if (mi != cur_mat) {
                 shared_table_rebuild<WARPS, LAYOUT, CODEC>(P, M, k0, lane, warp, S);
                 cur_mat = mi;
@@ -669,7 +675,7 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
         const uint32_t stride = gridDim.x * WARPS;
         for (uint32_t c = blockIdx.x * WARPS + warp; c < P.total_units && !ctl->dead; c += stride) {
             const MatJob &M = P.mats[job_of(P, c)];
-            const uint32_t k = c - M.begin;
+            const uint32_t k = M.chunk0 + (c - M.begin);
             ChunkHead h;
             if (!load_head<CODEC>(P, M, k, lane, h)) continue;
             const uint32_t *tab = reinterpret_cast<const uint32_t *>(h.rec + kHeadBytes<CODEC>);
@@ -806,24 +812,37 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
         ScatterParams Q{};
         Q.status = d_status;
         uint32_t n_out = 0;
+        // leading pairs of full chunks of the common-case matrices: the pair kernel
+        uint32_t handled[kMaxMatsPerLaunch] = {};
+#if EQ_USE_PAIRS
+        if (!symbols) {
+            uint32_t ids[kMaxMatsPerLaunch];
+            for (uint32_t i = 0; i < cnt; ++i) ids[i] = first + base + i;
+            if ((rc = launch_decode_pairs(m, ids, outs + base, cnt, d_status, s, sms, handled))) return rc;
+        }
+#endif
         for (uint32_t i = 0; i < cnt; ++i) {
             const MatrixDesc &d = m->mats[first + base + i];
             if (d.info.n_chunks == 0) continue;
             const int sh = d.info.uniform_table ? 1 : 0;
             const uint32_t lay = symbols ? kSymbolBytes : layout_of(d.info, outs[base + i]);
-            DecodeParams &Pv = P[d.codec][sh][d.info.dtype - 1][lay];
-            MatJob &J = Pv.mats[Pv.n_mats++];
-            J.chunk_index = reinterpret_cast<const uint64_t *>(m->d_blob + d.chunk_index_off);
-            J.scales = reinterpret_cast<const float *>(m->d_blob + d.scales_off);
-            J.out = outs[base + i];
-            J.n_elems = (uint64_t)d.info.rows * d.info.cols;
-            J.cols = d.info.cols;
-            J.n_chunks = d.info.n_chunks;
-            J.begin = Pv.total_units;
-            J.dtype = d.info.dtype;
-            J.layout = lay;
-            J.small_scales = d.small_scales ? 1u : 0u;
-            Pv.total_units += d.info.n_chunks;  // per-chunk units; shared-table launches are re-tiled below
+            if (handled[i] < d.info.n_chunks) {
+                DecodeParams &Pv = P[d.codec][sh][d.info.dtype - 1][lay];
+                MatJob &J = Pv.mats[Pv.n_mats++];
+                J.chunk_index = reinterpret_cast<const uint64_t *>(m->d_blob + d.chunk_index_off);
+                J.scales = reinterpret_cast<const float *>(m->d_blob + d.scales_off);
+                J.out = outs[base + i];
+                J.n_elems = (uint64_t)d.info.rows * d.info.cols;
+                J.cols = d.info.cols;
+                J.n_chunks = d.info.n_chunks;
+                J.chunk0 = handled[i];
+                J.begin = Pv.total_units;
+                J.dtype = d.info.dtype;
+                J.layout = lay;
+                J.small_scales = d.small_scales ? 1u : 0u;
+                // per-chunk units; shared-table launches are re-tiled below
+                Pv.total_units += d.info.n_chunks - handled[i];
+            }
             if (d.info.n_outliers && !symbols) {
                 ScatterJob &O = Q.jobs[Q.n_jobs++];
                 O.rec = reinterpret_cast<const uint32_t *>(m->d_blob + d.outliers_off);
@@ -920,6 +939,23 @@ extern "C" EQW_API int eq_decode_model_stream(const eq_model *m, uint32_t layer,
     int rc = eq_decode_block(m, layer, d_buf[b], buf_bytes, d_status, decode_stream);
     if (rc) return rc;
     if (cudaEventRecord(ev_ready[b], decode_stream) != cudaSuccess) return EQ_ERR_CUDA;
+    return EQ_OK;
+}
+
+extern "C" EQW_API int eq_decode_plan(const eq_model *m, uint32_t layer, uint32_t sms, uint32_t *pair_chunks,
+                                      uint32_t cap) {
+    if (!m || !pair_chunks || !sms || layer >= m->n_layers || cap < m->layer_count[layer]) return EQ_ERR_INVALID_ARG;
+    const uint32_t first = m->layer_first[layer], count = m->layer_count[layer];
+    const uint32_t eff = m->sm_limit && m->sm_limit < sms ? m->sm_limit : sms;
+    for (uint32_t i = 0; i < count; ++i) pair_chunks[i] = 0;
+#if EQ_USE_PAIRS
+    for (uint32_t base = 0; base < count; base += kMaxMatsPerLaunch) {
+        const uint32_t cnt = std::min<uint32_t>(kMaxMatsPerLaunch, count - base);
+        uint32_t ids[kMaxMatsPerLaunch];
+        for (uint32_t i = 0; i < cnt; ++i) ids[i] = first + base + i;
+        plan_decode_pairs(m, ids, cnt, eff, pair_chunks + base);
+    }
+#endif
     return EQ_OK;
 }
 

@@ -63,6 +63,7 @@ struct GemvJob {
     uint32_t cols;
     uint32_t rows;
     uint32_t n_chunks;
+    uint32_t chunk0;              // always 0: every chunk of the matrix is decoded here
     uint32_t begin;               // first launch-wide work unit (tile or chunk) of this matrix
     uint32_t n_out;
 };
@@ -562,6 +563,7 @@ int launch_gemv(const eq_model *m, uint32_t first, uint32_t count, const void *c
             J.cols = d.info.cols;
             J.rows = d.info.rows;
             J.n_chunks = d.info.n_chunks;
+            J.chunk0 = 0;
             J.begin = Pv.total_units;
             J.n_out = d.info.n_outliers;
             Pv.total_units += d.info.n_chunks;  // per-chunk units; shared-table launches are re-tiled below

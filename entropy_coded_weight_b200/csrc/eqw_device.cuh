@@ -203,9 +203,13 @@ __device__ __forceinline__ uint32_t ring_limit(uint32_t n_segs, uint32_t issued,
     return lim;
 }
 
+#ifndef EQ_RING_INLINE
+#define EQ_RING_INLINE __forceinline__
+#endif
 // Refill free slots, then make payload bytes [pw, pw + kSpan) resident.  Returns
-// the new limit; on a wait that gave up sets ctl->dead and returns kNoLimit.
-__device__ __noinline__ uint32_t ring_service(RingCtl *ctl, uint32_t ring, uint32_t mbar, uint32_t pw) {
+// the new limit; on a wait that gave up sets ctl->dead and returns kNoLimit,
+// leaving that segment counted as not ready.
+__device__ EQ_RING_INLINE uint32_t ring_service(RingCtl *ctl, uint32_t ring, uint32_t mbar, uint32_t pw) {
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t n_segs = ctl->n_segs, pbytes = ctl->pbytes;
     uint32_t issued = ctl->issued, ready = ctl->ready, phase = ctl->phase;
@@ -230,13 +234,12 @@ __device__ __noinline__ uint32_t ring_service(RingCtl *ctl, uint32_t ring, uint3
     bool ok = true;
     while (ready <= need && ready < issued) {
         const uint32_t slot = ready % kRingSegs;
-        const bool got = mbar_wait_bounded(mbar + 8 * slot, (phase >> slot) & 1u);
-        phase ^= 1u << slot;
-        ++ready;
-        if (!__all_sync(kFull, got)) {
-            ok = false;
+        if (!__all_sync(kFull, mbar_wait_bounded(mbar + 8 * slot, (phase >> slot) & 1u))) {
+            ok = false;  // the segment stays not ready: ring_drain waits for its copy again
             break;
         }
+        phase ^= 1u << slot;
+        ++ready;
     }
     __syncwarp();
     if (lane == 0) {
@@ -745,7 +748,7 @@ template <class Params>
 void assign_tiles(Params &P, uint32_t resident, uint32_t max_warps, uint32_t max_chains) {
     auto units_for = [&](uint32_t w, uint32_t c) {
         uint64_t units = 0;
-        for (uint32_t i = 0; i < P.n_mats; ++i) units += (P.mats[i].n_chunks + w * c - 1) / (w * c);
+        for (uint32_t i = 0; i < P.n_mats; ++i) units += (P.mats[i].n_chunks - P.mats[i].chunk0 + w * c - 1) / (w * c);
         return units;
     };
     const uint32_t chains = units_for(max_warps, 1) <= resident ? 1u : max_chains;
@@ -760,7 +763,7 @@ void assign_tiles(Params &P, uint32_t resident, uint32_t max_warps, uint32_t max
     P.total_units = 0;
     for (uint32_t i = 0; i < P.n_mats; ++i) {
         P.mats[i].begin = P.total_units;
-        P.total_units += (P.mats[i].n_chunks + tw * chains - 1) / (tw * chains);
+        P.total_units += (P.mats[i].n_chunks - P.mats[i].chunk0 + tw * chains - 1) / (tw * chains);
     }
 }
 

@@ -43,6 +43,7 @@ struct MatrixDesc {
     uint64_t outliers_off;
     bool small_scales;    // every scale finite with |scale| < 2^8 (E4M3 single-multiply dequant is exact)
     uint32_t codec;       // kCodecRans or kCodecHuffman
+    uint32_t n_present0;  // distinct symbols in the first chunk's table (all chunks' when uniform_table)
 };
 
 }  // namespace eqw

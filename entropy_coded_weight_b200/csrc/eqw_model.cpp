@@ -167,6 +167,7 @@ int parse(const uint8_t *b, size_t len, eq_model *m) {
             const uint32_t np = rd<uint32_t>(b + off + 8);
             if (k == 0) {
                 np0 = np;
+                d.n_present0 = np;
             } else if (in.uniform_table) {
                 const uint64_t off0 = rd<uint64_t>(b + d.chunk_index_off);
                 const uint32_t hb = record_head_bytes(d.codec);

@@ -191,9 +191,15 @@ EQW_API int eq_encode_device(const eq_matrix_in *mats, uint32_t n_mats, void *d_
 
 /* eq_encode_device with a workspace the library keeps in a file-scope device
  * array (16 MiB per device, reserved when the library loads): no device
- * memory is allocated and no workspace is passed.  Calls are serialised by a
- * host lock.  EQ_ERR_NOSPACE if the matrices need more workspace than that
- * (eq_encode_device_workspace tells). */
+ * memory is allocated and no workspace is passed, for callers that cannot
+ * allocate device memory themselves.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  Every call shares the
+ * array: the library serialises its own callers with a host lock and
+ * synchronises `s` before returning (also on errors), so its calls never
+ * overlap on the GPU.  EQ_ERR_NOSPACE if the matrices need more workspace than
+ * the array holds (eq_encode_device_workspace tells).  The pages have no
+ * counterpart of this entry point. */
 EQW_API int eq_encode_device_noalloc(const eq_matrix_in *mats, uint32_t n_mats, void *d_out, size_t out_cap,
                                      size_t *out_len, cudaStream_t s);
 
@@ -254,6 +260,23 @@ EQW_API int eq_layer_matrices(const eq_model *m, uint32_t layer, uint32_t *first
  */
 EQW_API int eq_block_layout(const eq_model *m, uint32_t layer, size_t *offsets, uint32_t cap,
                             size_t *total_bytes);
+
+/*
+ * How a decode of `layer` (eq_decode_block, eq_decode_model_stream) divides
+ * the layer's chunks between the two decode kernels on a GPU with `sms` SMs
+ * (or the model's SM limit, if that is lower): pair_chunks[i] (host, `cap` >=
+ * the layer's matrix count) receives how many leading chunks of the layer's
+ * i-th matrix go to the kernel that decodes two full chunks per warp in
+ * lockstep; the general kernel takes the rest.  A matrix qualifies when all
+ * its chunks share one frequency table of 2..32 symbols and its rows are a
+ * multiple of 512 symbols; a launch qualifies when it gives every warp of every
+ * SM at least one pair.  Host only, no CUDA call: the decision is a pure
+ * function of the container and `sms`.  The pages describe no such split
+ * (EntroLLM technical overview, "parallel decoding strategy", only has chunks
+ * decode independently).  Errors: EQ_ERR_INVALID_ARG (m or pair_chunks NULL,
+ * layer out of range, cap too small, sms == 0).
+ */
+EQW_API int eq_decode_plan(const eq_model *m, uint32_t layer, uint32_t sms, uint32_t *pair_chunks, uint32_t cap);
 
 /* ---- decode (hot path) ------------------------------------------------------
  * Decode one matrix into `d_out` (device, 2-byte aligned; 16-byte aligned and
