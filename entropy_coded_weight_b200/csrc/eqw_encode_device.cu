@@ -694,10 +694,14 @@ namespace {
 
 // Workspace of eq_encode_device_noalloc: a file-scope device array (one per
 // device context, reserved when the library's module loads), so that entry
-// point allocates nothing; a host mutex serialises its users.
+// point allocates nothing; a host mutex serialises its users.  In host code
+// the array's name is only a host-side stand-in: its device address comes from
+// cudaGetSymbolAddress, looked up once per device (with that device current)
+// on the entry point's first call there.
 constexpr size_t kStaticScratchBytes = 16u << 20;
-__device__ __align__(256) uint8_t g_encode_scratch[kStaticScratchBytes];
+static __device__ __align__(256) uint8_t g_encode_scratch[kStaticScratchBytes];
 std::mutex g_encode_scratch_mu;
+void *g_encode_scratch_ptr[128];  // device address of the array on each device (null: not looked up yet)
 
 }  // namespace
 
@@ -708,8 +712,17 @@ extern "C" EQW_API int eq_encode_device_noalloc(const eq_matrix_in *mats, uint32
     int rc = eq_encode_device_workspace(mats, n_mats, &need);
     if (rc) return rc;
     if (need > kStaticScratchBytes) return EQ_ERR_NOSPACE;
-    void *scratch = nullptr;
-    if (cudaGetSymbolAddress(&scratch, g_encode_scratch) != cudaSuccess) return EQ_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return EQ_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_encode_scratch_mu);
-    return encode_device(mats, n_mats, d_out, out_cap, out_len, scratch, kStaticScratchBytes, s);
+    if (!g_encode_scratch_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_encode_scratch) != cudaSuccess || !p) return EQ_ERR_CUDA;
+        g_encode_scratch_ptr[dev] = p;
+    }
+    rc = encode_device(mats, n_mats, d_out, out_cap, out_len, g_encode_scratch_ptr[dev], kStaticScratchBytes, s);
+    // an error return may come after a kernel launch: let the stream drain before
+    // the next caller may reuse the array
+    if (rc) cudaStreamSynchronize(s);
+    return rc;
 }

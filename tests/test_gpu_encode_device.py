@@ -1,9 +1,13 @@
-"""GPU encoder (eq_encode_device) against the host encoder, byte for byte.
+"""GPU encoder (eq_encode_device): its containers decoded by the CPU oracle,
+and its bytes against the host encoder's.
 
-Both encoders quantise the same tables and lay out the same container, so for
-the same inputs the device encoder's bytes must equal eq_encode_host's, which
-the CPU tests already tie to the oracle (the oracle decodes them exactly:
-EntQuant technical summary, section 2 "weight encoding", lossless coding).
+The first check is independent of the product: the oracle's own scalar
+decoder (O-decode, which shares no code with either encoder) must turn every
+container the GPU wrote back into exactly the oracle's direct dequantisation
+of the input symbols (EntQuant technical summary, section 2 "weight
+encoding": the ANS coding is lossless).  The second pins the two product
+encoders to each other: they quantise the same tables and lay out the same
+container, so for the same inputs their bytes must be equal.
 """
 import ctypes
 from dataclasses import dataclass
@@ -50,6 +54,18 @@ def _dev(m):
     return d
 
 
+def _oracle_decodes(orc, blob, mats):
+    """The oracle decodes the container exactly to O-direct, matrix by matrix."""
+    got = orc.decode_container(blob)
+    assert len(got) == len(mats)
+    for g, m in zip(got, mats):
+        want = orc.dequant_direct(m)
+        assert g.shape == want.shape
+        if not np.array_equal(g, want):
+            raise AssertionError(f"matrix {m.layer}/{m.index}: {int(np.count_nonzero(g != want))} of {m.n} "
+                                 f"outputs differ after the oracle's decode")
+
+
 def _ragged():
     mats = [
         W.random_int8_matrix(1, 300, 229, layer=0, index=0),                 # tail chunk, cols % 8 != 0
@@ -69,24 +85,26 @@ def _ragged():
 
 @pytest.mark.parametrize("codec", ["rans", "huffman"])
 @pytest.mark.parametrize("scope", ["matrix", "chunk"])
-def test_ragged_bytes_equal_host_encoder(eqw, scope, codec):
+def test_ragged_bytes_equal_host_encoder(eqw, orc, scope, codec):
     mats = _ragged()
     host = eqw.encode_host(mats, table_scope=scope, codec=codec)
     dev = eqw.encode_device([_dev(m) for m in mats], table_scope=scope, codec=codec).cpu().numpy()
+    _oracle_decodes(orc, dev, mats)
     assert dev.size == host.size
     assert np.array_equal(dev, host)
 
 
-def test_mixed_codecs_bytes_equal_host_encoder(eqw):
+def test_mixed_codecs_bytes_equal_host_encoder(eqw, orc):
     mats = _ragged()
     for i, m in enumerate(mats):
         m.codec = "huffman" if i % 2 else "rans"
     host = eqw.encode_host(mats)
     dev = eqw.encode_device([_dev(m) for m in mats]).cpu().numpy()
+    _oracle_decodes(orc, dev, mats)
     assert np.array_equal(dev, host)
 
 
-def test_huffman_long_codes_bytes_equal_host_encoder(eqw):
+def test_huffman_long_codes_bytes_equal_host_encoder(eqw, orc):
     """Skewed counts over 254 E4M3 codes: many codes at the 12-bit limit, long refill look-ahead."""
     rng = np.random.default_rng(5)
     codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
@@ -97,15 +115,17 @@ def test_huffman_long_codes_bytes_equal_host_encoder(eqw):
     for scope in ("matrix", "chunk"):
         host = eqw.encode_host([m], table_scope=scope, codec="huffman")
         dev = eqw.encode_device([_dev(m)], table_scope=scope, codec="huffman").cpu().numpy()
+        _oracle_decodes(orc, dev, [m])
         assert np.array_equal(dev, host), scope
 
 
 @pytest.mark.parametrize("codec", ["rans", "huffman"])
 @pytest.mark.parametrize("which", ["llama70b_int8_layer", "llama70b_e4m3_block", "llama7b_int8_block_with_outliers"])
-def test_full_size_bytes_equal_host_encoder(eqw, which, codec):
+def test_full_size_bytes_equal_host_encoder(eqw, orc, which, codec):
     mats = W.llama70b_int8_layer(0) if which == "llama70b_int8_layer" else getattr(W, which)()
     host = eqw.encode_host(mats, codec=codec)
     dev = eqw.encode_device([_dev(m) for m in mats], codec=codec).cpu().numpy()
+    _oracle_decodes(orc, dev, mats)
     assert np.array_equal(dev, host)
 
 

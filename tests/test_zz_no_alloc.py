@@ -53,17 +53,24 @@ def _encode_noalloc(E, dev_mats, scope="matrix"):
 
 
 @pytest.mark.parametrize("scope", ["matrix", "chunk"])
-def test_bytes_equal_host_and_nothing_allocated(eqw, scope):
+def test_bytes_equal_host_and_nothing_allocated(eqw, orc, scope):
     mats = [W.random_int8_matrix(1, 300, 1229, n_out=6, layer=0, index=0),
             W.random_e4m3_matrix(2, 77, 1000, alpha=1.0, layer=0, index=1),
             W.random_int8_matrix(3, 512, 2048, h_bits=3.0, layer=1, index=0)]
     dev = [_Dev(m) for m in mats]
-    rc, _, _ = _encode_noalloc(eqw, dev, scope)    # loads the module and its scratch array
+    rc, first, _ = _encode_noalloc(eqw, dev, scope)    # loads the module and its scratch array
     assert rc == 0
     rc, got, allocated = _encode_noalloc(eqw, dev, scope)
     assert rc == 0
     assert allocated == 0
+    # two calls in a row give the same bytes as the entry point with a caller workspace ...
+    with_workspace = eqw.encode_device(dev, table_scope=scope).cpu().numpy()
+    assert np.array_equal(first, with_workspace)
+    assert np.array_equal(got, with_workspace)
     assert np.array_equal(got, eqw.encode_host(mats, table_scope=scope))
+    # ... and the CPU oracle decodes them exactly to its direct dequantisation
+    for g, m in zip(orc.decode_container(got), mats):
+        assert np.array_equal(g, orc.dequant_direct(m))
 
 
 def test_reports_nospace_beyond_static_workspace(eqw):
