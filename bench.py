@@ -51,7 +51,8 @@ UNIT = "GB/s"
 # taken on: the figure is reported only while the sources are unchanged.
 DECODE_TRAFFIC_BYTES = 1_898_072_576
 DECODE_TRAFFIC_SOURCES_SHA256 = "6fe9b580c68901f86f1e677d1dca88e0581f9147959e43257b7cfeaec6a04721"
-DECODE_SOURCES = ("entropy_coded_weight_b200/csrc/eqw_decode.cu", "entropy_coded_weight_b200/csrc/eqw_device.cuh")
+DECODE_SOURCES = ("entropy_coded_weight_b200/csrc/eqw_decode.cu", "entropy_coded_weight_b200/csrc/eqw_device.cuh",
+                  "entropy_coded_weight_b200/csrc/eqw_decode_pairs.cu")
 
 
 def decode_sources_sha256() -> str:
@@ -394,6 +395,18 @@ def cpu_oracle_sample(blob: np.ndarray, target_s: float = 12.0) -> dict:
             "gsym_s": round(done / dt / 1e9, 5)}
 
 
+def workload_config(layers: int, distinct: int, world: int) -> dict:
+    """The bench line's `config`: the streamed 70B-shape model as decoded here."""
+    import workloads as W
+    per_layer = sum(r * c for r, c in W.LLAMA70B_BLOCK)
+    return {"workload": f"streamed {layers}-layer Llama-70B-shape model, Int8 ~2.1 bits/sym, "
+                        f"{distinct} distinct layers x {(layers + distinct - 1) // distinct} HBM copies, "
+                        "ping-pong bf16 buffers, no-op consumer",
+            "layers": layers, "symbols_per_step": layers * per_layer,
+            "l2": "inputs larger than L2 (each layer ~0.23 GB compressed, 1.7 GB decoded)",
+            "parallelism": f"replicas x{world}"}
+
+
 def bench_eqw(args, d: Dist) -> dict | None:
     import torch
 
@@ -589,22 +602,23 @@ def bench_eqw(args, d: Dist) -> dict | None:
     stack.close()
     if d.rank != 0:
         return None
+    # workloads 1-4, one block per launch, each checked against the oracle outside its timing
+    per_config = None
+    if not args.no_per_config:
+        del streamer, pinned
+        torch.cuda.empty_cache()
+        per_config = per_config_summary(dev, threads, 3, 10, peak)
     launches = len(stack.steps) * args.steps  # one decode kernel per block (no outliers in this workload)
     return {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": d.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "u32 rANS state, f32 dequant -> bf16",
         "data": "synthetic (seeded Laplace Int8 symbols at 2.1 bits; no checkpoint)",
-        "config": {"workload": f"streamed {args.layers}-layer Llama-70B-shape model, Int8 ~2.1 bits/sym, "
-                               f"{args.distinct_layers} distinct layers x {stack.copies} HBM copies, "
-                               "ping-pong bf16 buffers, no-op consumer",
-                   "layers": args.layers, "symbols_per_step": n_syms_pass,
-                   "l2": "inputs larger than L2 (each layer ~0.23 GB compressed, 1.7 GB decoded)",
-                   "parallelism": f"replicas x{d.world}"},
+        "config": workload_config(args.layers, args.distinct_layers, d.world),
         "gsym_s": round(gsym, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": decode_traffic(),
-                     "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "eq_decode_kernel",
+                     "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "eq_decode_pairs_kernel",
                      "alg_bytes_per_launch": int(alg_per_launch), "launch_ms": round(launch_ms, 4)},
         "with_gemv_consumer": {"value": round(value_b, 2), "unit": UNIT, "ms_per_step": round(ms_b_max / args.steps, 3),
                                "decode_sm_limit": args.consumer_sm_limit,
@@ -623,6 +637,7 @@ def bench_eqw(args, d: Dist) -> dict | None:
         "e2e": {"value": round(value_e, 2), "unit": UNIT, "h2d_bytes_per_step": int(blob.size * stack.copies),
                 "d2h_bytes_per_step": 4, "ms_per_step": round(ms_e_max / args.steps, 3)},
         "cpu_baseline": cpu,
+        "per_config": per_config,
         "encode": enc,
         "clocks": clk,
         "gpu_launches": launches,
@@ -701,6 +716,73 @@ def configs_table_row(row: dict) -> str:
             f"{'yes' if row['bit_exact'] else 'NO'} | {o['gsym_s_1core']:.3f} | {o['gsym_s_all']:.2f} |")
 
 
+def measure_config(key: str, name: str, mats, blob: np.ndarray, dev, cores: int, flush, warmup: int, steps: int,
+                   peak: float) -> dict:
+    """One workload block: bit-exactness of the whole decoded block against the
+    oracle's direct dequantisation (outside any timed region), then `steps`
+    block decodes after `warmup`, each timed with CUDA events on its stream and
+    L2 rewritten before it (config 1, which fits in L2, is also timed hot)."""
+    import torch
+
+    import entropy_coded_weight_b200 as E
+    import oracle
+    import workloads as W
+    n = sum(m.n for m in mats)
+    model = E.Model(E.upload(blob, dev), blob)
+    infos = [model.info(i) for i in model.layer_matrices(0)]
+    records = sum(i.compressed_bytes for i in infos)
+    read = records + sum(8 * (i.n_chunks + 1) + 4 * i.rows + 12 * i.n_outliers for i in infos)
+    write = 2 * n + sum(2 * i.n_outliers for i in infos)
+    offs, total = model.block_layout(0)
+    out = torch.empty(total, dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    model.decode_block(0, out, status)
+    torch.cuda.synchronize()
+    host = out.cpu().numpy()
+    exact = int(status.item()) == 0
+    for m, o in zip(mats, offs):
+        got = host[o:o + 2 * m.n].view(np.uint16).reshape(m.rows, m.cols)
+        exact = exact and bool(np.array_equal(got, oracle.dequant_direct(m, threads=cores)))
+    del host, out
+    lines = {"l2_flushed": statistics.mean(_block_launches(model, 0, warmup + steps, dev, flush)[warmup:])}
+    if key == "1":
+        lines["hot"] = statistics.mean(_block_launches(model, 0, warmup + 10 * steps, dev)[warmup:])
+    row = {"config": key, "workload": name, "symbols": n, "matrices": len(mats),
+           "bits_per_sym_records": round(8.0 * records / n, 4),
+           "bits_per_sym_container": round(8.0 * blob.size / n, 4),
+           "empirical_entropy_bits": round(float(np.mean([W.empirical_entropy_bits(m.symbols) for m in mats])), 4),
+           "bit_exact": exact}
+    for kind, ms in lines.items():
+        row[kind] = {"launch_ms": round(ms, 5), "decoded_gb_s": round(2.0 * n / (ms / 1e3) / 1e9, 1),
+                     "gsym_s": round(n / (ms / 1e3) / 1e9, 2),
+                     "hbm_frac": round((read + write) / (ms / 1e3) / 1e9 / peak, 4)}
+    model.close()
+    return row
+
+
+def per_config_summary(dev, cores: int, warmup: int, steps: int, peak: float) -> dict:
+    """Workloads 1-4 one block per launch, compactly, for the bench line."""
+    import torch
+
+    import entropy_coded_weight_b200 as E
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 2 x L2
+    res = {}
+    for key, name, make in _config_rows():
+        mats = make(cores)
+        blob = E.encode_host(mats, n_threads=cores)
+        row = measure_config(key, name, mats, blob, dev, cores, flush, warmup, steps, peak)
+        ent = {"symbols": row["symbols"], "bit_exact": row["bit_exact"],
+               "bits_per_sym": row["bits_per_sym_records"]}
+        for kind in ("l2_flushed", "hot"):
+            if kind in row:
+                ent[kind] = {k: row[kind][k] for k in ("launch_ms", "decoded_gb_s", "gsym_s", "hbm_frac")}
+        res[key] = ent
+        del mats, blob
+    del flush
+    torch.cuda.empty_cache()
+    return res
+
+
 def bench_configs(args) -> None:
     """One JSON line per workload: decode throughput of one block per launch
     (inputs in HBM, L2 rewritten between launches), compression, bit-exactness
@@ -722,49 +804,16 @@ def bench_configs(args) -> None:
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 2 x L2
     for key, name, make in _config_rows():
         mats = make(cores)
-        n = sum(m.n for m in mats)
         blob = E.encode_host(mats, n_threads=cores)
-        model = E.Model(E.upload(blob, dev), blob)
-        infos = [model.info(i) for i in model.layer_matrices(0)]
-        records = sum(i.compressed_bytes for i in infos)
-        read = records + sum(8 * (i.n_chunks + 1) + 4 * i.rows + 12 * i.n_outliers for i in infos)
-        write = 2 * n + sum(2 * i.n_outliers for i in infos)
-        # parity: the whole decoded block against the oracle's direct dequant + scatter
-        offs, total = model.block_layout(0)
-        out = torch.empty(total, dtype=torch.uint8, device=dev)
-        status = torch.zeros(1, dtype=torch.int32, device=dev)
-        model.decode_block(0, out, status)
-        torch.cuda.synchronize()
-        host = out.cpu().numpy()
-        exact = int(status.item()) == 0
-        for m, o in zip(mats, offs):
-            got = host[o:o + 2 * m.n].view(np.uint16).reshape(m.rows, m.cols)
-            exact = exact and bool(np.array_equal(got, oracle.dequant_direct(m, threads=cores)))
-        del host, out
-        lines = {}
-        flushed = _block_launches(model, 0, args.warmup + args.steps, dev, flush)[args.warmup:]
-        lines["l2_flushed"] = statistics.mean(flushed)
-        if key == "1":
-            hot = _block_launches(model, 0, args.warmup + 10 * args.steps, dev)[args.warmup:]
-            lines["hot"] = statistics.mean(hot)
+        row = measure_config(key, name, mats, blob, dev, cores, flush, args.warmup, args.steps, peak)
         s1, _, t1, _ = oracle_rate(blob, 1, 3.0)
         sa, _, ta, _ = oracle_rate(blob, cores, 3.0)
-        row = {"config": key, "workload": name, "symbols": n, "matrices": len(mats),
-               "bits_per_sym_records": round(8.0 * records / n, 4),
-               "bits_per_sym_container": round(8.0 * blob.size / n, 4),
-               "empirical_entropy_bits": round(float(np.mean([W.empirical_entropy_bits(m.symbols) for m in mats])), 4),
-               "bit_exact": exact}
-        for kind, ms in lines.items():
-            row[kind] = {"launch_ms": round(ms, 5), "decoded_gb_s": round(2.0 * n / (ms / 1e3) / 1e9, 1),
-                         "gsym_s": round(n / (ms / 1e3) / 1e9, 2),
-                         "hbm_frac": round((read + write) / (ms / 1e3) / 1e9 / peak, 4)}
         row["oracle"] = {"gsym_s_1core": round(s1 / t1 / 1e9, 5), "gsym_s_all": round(sa / ta / 1e9, 5),
                          "cores": cores, "sample_s": [round(t1, 1), round(ta, 1)]}
         row["peak"] = {"hbm_gbs": peak, "kind": peak_kind}
         print(json.dumps(row), flush=True)
         print(configs_table_row(row), file=sys.stderr, flush=True)
-        model.close()
-        del mats, blob, model
+        del mats, blob
 
     # workload 5: the streamed model; every block checksummed as the consumer sees it
     distinct = args.distinct_layers
@@ -811,11 +860,16 @@ def bench_configs(args) -> None:
 
 
 def bench_reference(args) -> dict:
-    """The CPU oracle, as it stands, on host cores: same metric and unit, bounded samples."""
+    """The CPU oracle, as it stands, on host cores: the same metric, unit and
+    config as the GPU arm, each step a bounded sample of layer 0's 13,056 chunks
+    (the same seeded layer the GPU arm decodes, here encoded by the oracle's own
+    encoder)."""
     import oracle
     import workloads as W
-    mats = [W._int8_matrix(5, 0, 0, W.LLAMA70B_BLOCK[0], 2.1)]  # layer 0, q: 1024 chunks
-    blob = oracle.encode_container(mats)
+    cores = len(os.sched_getaffinity(0))
+    mats = W.llama70b_int8_layer(0, 2.1, threads=cores)
+    blob = oracle.encode_container(mats, threads=cores)
+    del mats
     res = []
     for _ in range(args.warmup + args.steps):
         res.append(cpu_oracle_sample(blob, target_s=max(2.0, 60.0 / max(1, args.warmup + args.steps))))
@@ -826,8 +880,8 @@ def bench_reference(args) -> dict:
     return {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": UNIT, "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "u32 rANS state, f32 dequant -> bf16",
-            "data": "synthetic (seeded Laplace Int8 symbols at 2.1 bits)",
-            "config": {"workload": "streamed 80-layer Llama-70B-shape model (sampled chunks of layer 0)"},
+            "data": "synthetic (seeded Laplace Int8 symbols at 2.1 bits; no checkpoint)",
+            "config": workload_config(args.layers, args.distinct_layers, 1),
             "cpu_baseline": cpu, "e2e": {"value": round(v, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                                          "d2h_bytes_per_step": 0}}
 
@@ -841,6 +895,8 @@ def main(argv=None):
     ap.add_argument("--distinct-layers", type=int, default=8)
     ap.add_argument("--layers", type=int, default=N_LAYERS, help="blocks per pass (80 = the 70B model)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the one-block-per-launch table of workloads 1-4 in the bench line")
     ap.add_argument("--consumer-sm-limit", type=int, default=112,
                     help="SMs the decode launches may use while the GEMV consumer runs beside them (0: all)")
     ap.add_argument("--configs", action="store_true",
