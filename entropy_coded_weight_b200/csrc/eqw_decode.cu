@@ -878,6 +878,7 @@ int launch_decode(const eq_model *m, uint32_t first, uint32_t count, uint16_t *c
 
 extern "C" EQW_API int eq_decode_matrix(const eq_model *m, uint32_t matrix, void *d_out, size_t out_bytes,
                                         int32_t *d_status, cudaStream_t s) {
+    const eqw::NvtxScope nvtx_range("eq_decode_matrix");
     if (!m || !d_status || matrix >= m->mats.size()) return EQ_ERR_INVALID_ARG;
     const eq_matrix_info &in = m->mats[matrix].info;
     const uint64_t need = 2ull * in.rows * in.cols;
@@ -889,6 +890,7 @@ extern "C" EQW_API int eq_decode_matrix(const eq_model *m, uint32_t matrix, void
 
 extern "C" EQW_API int eq_decode_symbols(const eq_model *m, uint32_t matrix, void *d_out, size_t out_bytes,
                                          int32_t *d_status, cudaStream_t s) {
+    const eqw::NvtxScope nvtx_range("eq_decode_symbols");
     if (!m || !d_status || matrix >= m->mats.size()) return EQ_ERR_INVALID_ARG;
     const eq_matrix_info &in = m->mats[matrix].info;
     const uint64_t need = (uint64_t)in.rows * in.cols;
@@ -900,6 +902,7 @@ extern "C" EQW_API int eq_decode_symbols(const eq_model *m, uint32_t matrix, voi
 
 extern "C" EQW_API int eq_decode_symbols_block(const eq_model *m, uint32_t layer, void *const *d_outs,
                                                uint32_t count, int32_t *d_status, cudaStream_t s) {
+    const eqw::NvtxScope nvtx_range("eq_decode_symbols_block");
     if (!m || !d_status || !d_outs || layer >= m->n_layers || count != m->layer_count[layer])
         return EQ_ERR_INVALID_ARG;
     const uint32_t first = m->layer_first[layer];
@@ -915,6 +918,7 @@ extern "C" EQW_API int eq_decode_symbols_block(const eq_model *m, uint32_t layer
 
 extern "C" EQW_API int eq_decode_block(const eq_model *m, uint32_t layer, void *d_out, size_t out_bytes,
                                        int32_t *d_status, cudaStream_t s) {
+    const eqw::NvtxScope nvtx_range("eq_decode_block");
     if (!m || !d_status || layer >= m->n_layers) return EQ_ERR_INVALID_ARG;
     const uint32_t first = m->layer_first[layer], count = m->layer_count[layer];
     std::vector<size_t> offs(count);
@@ -932,6 +936,7 @@ extern "C" EQW_API int eq_decode_block(const eq_model *m, uint32_t layer, void *
 extern "C" EQW_API int eq_decode_model_stream(const eq_model *m, uint32_t layer, void *const d_buf[2],
                                               size_t buf_bytes, int32_t *d_status, cudaStream_t decode_stream,
                                               cudaEvent_t const ev_free[2], cudaEvent_t const ev_ready[2]) {
+    const eqw::NvtxScope nvtx_range("eq_decode_model_stream");
     if (!m || !d_buf || !ev_free || !ev_ready || layer >= m->n_layers) return EQ_ERR_INVALID_ARG;
     const uint32_t b = layer & 1u;
     if (!ev_ready[b]) return EQ_ERR_INVALID_ARG;

@@ -584,12 +584,14 @@ int launch_gemv(const eq_model *m, uint32_t first, uint32_t count, const void *c
 
 extern "C" EQW_API int eq_decode_gemv_matrix(const eq_model *m, uint32_t matrix, const void *d_x, float *d_y,
                                              int32_t *d_status, cudaStream_t s) {
+    const eqw::NvtxScope nvtx_range("eq_decode_gemv_matrix");
     if (!m || !d_status || matrix >= m->mats.size()) return EQ_ERR_INVALID_ARG;
     return launch_gemv(m, matrix, 1, &d_x, &d_y, d_status, s);
 }
 
 extern "C" EQW_API int eq_decode_gemv_block(const eq_model *m, uint32_t layer, const void *const *d_x,
                                             float *const *d_y, uint32_t count, int32_t *d_status, cudaStream_t s) {
+    const eqw::NvtxScope nvtx_range("eq_decode_gemv_block");
     if (!m || !d_status || layer >= m->n_layers || !d_x || !d_y) return EQ_ERR_INVALID_ARG;
     if (count != m->layer_count[layer]) return EQ_ERR_INVALID_ARG;
     return launch_gemv(m, m->layer_first[layer], count, d_x, d_y, d_status, s);

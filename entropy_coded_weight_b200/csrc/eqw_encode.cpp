@@ -331,6 +331,7 @@ extern "C" EQW_API void eq_encoded_free(eq_encoded *h) { delete h; }
 
 extern "C" EQW_API int eq_encode_host(const eq_matrix_in *mats, uint32_t n_mats, int n_threads, void *out,
                                       size_t out_cap, size_t *out_len) {
+    const eqw::NvtxScope nvtx_range("eq_encode_host");
     if (!out_len) return EQ_ERR_INVALID_ARG;
     eq_encoded *h = nullptr;
     size_t size = 0;

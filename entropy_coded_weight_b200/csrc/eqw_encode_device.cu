@@ -687,6 +687,7 @@ int encode_device(const eq_matrix_in *mats, uint32_t n_mats, void *d_out, size_t
 
 extern "C" EQW_API int eq_encode_device(const eq_matrix_in *mats, uint32_t n_mats, void *d_out, size_t out_cap,
                                         size_t *out_len, void *d_work, size_t work_bytes, cudaStream_t s) {
+    const eqw::NvtxScope nvtx_range("eq_encode_device");
     return encode_device(mats, n_mats, d_out, out_cap, out_len, d_work, work_bytes, s);
 }
 
@@ -707,6 +708,7 @@ void *g_encode_scratch_ptr[128];  // device address of the array on each device 
 
 extern "C" EQW_API int eq_encode_device_noalloc(const eq_matrix_in *mats, uint32_t n_mats, void *d_out,
                                                 size_t out_cap, size_t *out_len, cudaStream_t s) {
+    const eqw::NvtxScope nvtx_range("eq_encode_device_noalloc");
     if (!out_len) return EQ_ERR_INVALID_ARG;
     size_t need = 0;
     int rc = eq_encode_device_workspace(mats, n_mats, &need);

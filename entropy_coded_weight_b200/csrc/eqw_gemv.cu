@@ -56,6 +56,7 @@ eq_gemv_bf16_kernel(const uint4 *__restrict__ w, const uint4 *__restrict__ x, fl
 
 extern "C" EQW_API int eq_gemv_bf16(const void *d_w, const void *d_x, float *d_y, uint32_t rows, uint32_t cols,
                                     cudaStream_t s) {
+    const eqw::NvtxScope nvtx_range("eq_gemv_bf16");
     if (!rows) return EQ_OK;
     if (!d_w || !d_x || !d_y || cols % 8) return EQ_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(d_w) % 16 || reinterpret_cast<uintptr_t>(d_x) % 16) return EQ_ERR_INVALID_ARG;

@@ -8,6 +8,8 @@
 #include <cstdint>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/eqw.h"
 
 namespace eqw {
@@ -35,6 +37,15 @@ inline uint32_t record_head_bytes(uint32_t codec) {
 }
 
 inline uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+// A named NVTX range over a host entry point: encode, decode and consumer
+// calls show up by name on a profiler's timeline (a no-op when none is attached).
+struct NvtxScope {
+    explicit NvtxScope(const char *name) { nvtxRangePushA(name); }
+    ~NvtxScope() { nvtxRangePop(); }
+    NvtxScope(const NvtxScope &) = delete;
+    NvtxScope &operator=(const NvtxScope &) = delete;
+};
 
 struct MatrixDesc {
     eq_matrix_info info;
