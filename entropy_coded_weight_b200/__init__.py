@@ -307,3 +307,11 @@ def selftest_wait_timeout(status, stream=None) -> None:
     """eq_selftest_wait_timeout: make one bounded staging wait run out (about a
     second); the kernel ORs EQ_DEV_TIMEOUT into ``status`` (device int32)."""
     check(load().eq_selftest_wait_timeout(status.data_ptr(), _stream_handle(stream)), "eq_selftest_wait_timeout")
+
+
+def selftest_gemm_wait_timeout(status, stream=None) -> None:
+    """eq_selftest_gemm_wait_timeout: the prefill GEMM's MMA lane waits on a
+    "full" barrier nothing arrives on until its bounded wait runs out (about a
+    second); the block ORs EQ_DEV_TIMEOUT into ``status`` and frees its TMEM."""
+    check(load().eq_selftest_gemm_wait_timeout(status.data_ptr(), _stream_handle(stream)),
+          "eq_selftest_gemm_wait_timeout")

@@ -1,7 +1,7 @@
 """ctypes binding of libeqw.so (include/eqw.h): argument marshalling only.
 
 Every entry point keeps its C name.  The library is loaded from this package's
-directory; if it is missing the import fails loudly (there is no CPU
+directory (or from the path in EQW_LIBRARY); if it is missing the import fails loudly (there is no CPU
 fallback: decoding only runs in the CUDA kernels of libeqw).
 """
 from __future__ import annotations
@@ -10,12 +10,13 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libeqw.so")
+# EQW_LIBRARY selects another build of the same library, e.g. libeqw_checked.so
+LIB_PATH = os.environ.get("EQW_LIBRARY") or os.path.join(HERE, "libeqw.so")
 
 EQ_OK, EQ_ERR_INVALID_ARG, EQ_ERR_CORRUPT, EQ_ERR_UNSUPPORTED = 0, 1, 2, 3
 EQ_ERR_CUDA, EQ_ERR_TIMEOUT, EQ_ERR_NOSPACE = 4, 5, 6
 EQ_DEV_BAD_HEADER, EQ_DEV_BAD_TABLE, EQ_DEV_BAD_STATE = 1, 2, 4
-EQ_DEV_BAD_END, EQ_DEV_TIMEOUT, EQ_DEV_BAD_OUTLIER = 8, 16, 32
+EQ_DEV_BAD_END, EQ_DEV_TIMEOUT, EQ_DEV_BAD_OUTLIER, EQ_DEV_CHECK = 8, 16, 32, 64
 EQ_INT8, EQ_E4M3 = 1, 2
 EQ_TABLE_PER_CHUNK = 1
 EQ_CODEC_HUFFMAN = 2
@@ -83,8 +84,10 @@ SIGNATURES = {
     "eq_decode_symbols_block": (_i32, [_vp, _u32, _vp, _u32, _vp, _vp]),
     "eq_gemm_symbols": (_i32, [_vp, _u32, _vp, _vp, _u32, _vp, _vp, _vp]),
     "eq_selftest_wait_timeout": (_i32, [_vp, _vp]),
+    "eq_selftest_gemm_wait_timeout": (_i32, [_vp, _vp]),
     "eq_status_string": (ctypes.c_char_p, [_i32]),
     "eq_format_version": (_i32, []),
+    "eq_build_checked": (_i32, []),
 }
 
 _lib = None

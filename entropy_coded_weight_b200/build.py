@@ -18,6 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libeqw.so")
+LIB_CHECKED = os.path.join(HERE, "libeqw_checked.so")  # EQ_CHECKED=1: run-time checks of the kernels' invariants
 GENCODE = "-gencode=arch=compute_100a,code=sm_100a"
 
 
@@ -32,18 +33,26 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
         glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False, defines: dict | None = None, out: str | None = None) -> str:
+def build(force: bool = False, verbose: bool = False, defines: dict | None = None, out: str | None = None,
+          checked: bool = False) -> str:
     """Compile and link libeqw.so.  ``defines`` (-D NAME=VALUE for the CUDA
-    sources, e.g. EQ_SHARED_WARPS) and ``out`` build a tuning variant elsewhere."""
+    sources, e.g. EQ_SHARED_WARPS) and ``out`` build a tuning variant
+    elsewhere; ``checked`` builds libeqw_checked.so (EQ_CHECKED=1), whose
+    kernels test their invariants at run time (EQ_DEV_CHECK)."""
+    if checked:
+        defines = dict(defines or {}, EQ_CHECKED=1)
+        if out is None and not force and not _stale(LIB_CHECKED):
+            return LIB_CHECKED
+        out = out or LIB_CHECKED
     target = out or LIB
     if not force and out is None and not _stale():
         return LIB
@@ -64,6 +73,7 @@ def build(force: bool = False, verbose: bool = False, defines: dict | None = Non
             cuda_inc = os.path.join(os.path.dirname(os.path.dirname(os.path.realpath(nvcc))), "include")
             cmd = [os.environ.get("CXX", "g++"), "-O3", "-std=c++17", "-fPIC", "-fvisibility=hidden", "-pthread",
                    "-Wall", "-Wextra", "-I", INCLUDE, "-I", cuda_inc, "-c", src, "-o", obj]
+            cmd += [f"-D{k}={v}" for k, v in (defines or {}).items()]
         subprocess.check_call(cmd)
         objs.append(obj)
     tmp = target + f".{os.getpid()}.tmp"
@@ -76,6 +86,7 @@ if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--checked", action="store_true", help="build libeqw_checked.so (EQ_CHECKED=1)")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose, checked=a.checked))
     sys.exit(0)

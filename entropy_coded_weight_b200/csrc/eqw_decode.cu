@@ -318,6 +318,7 @@ __device__ __forceinline__ bool decode_multi(int32_t *status, const OutCtx &O, c
         groupN_rank<CODEC, C>(lut, ring, ch, lt);
 #pragma unroll
         for (uint32_t c = 0; c < C; ++c) {
+            check_progress(status, ctl + c, ch[c].pw, ch[c].dst, O.out, O.n_elems, lane);
             ch[c].col += 2 * kGroupSyms;
             if (ch[c].col == O.cols) {
                 ch[c].col = 0;
@@ -489,11 +490,13 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, ui
                         group_rank(lut, ring, pw, x, lt, vr, dst + kGroupSyms);
                         i += 2;
                         dst += 2 * kGroupSyms;
+                        check_progress(status, ctl, pw, dst, O.out, O.n_elems, lane);
                     } while (i + 1 < run && pw < limit);
                 } else {
                     group_rank(lut, ring, pw, x, lt, vr, dst);
                     i += 1;
                     dst += kGroupSyms;
+                    check_progress(status, ctl, pw, dst, O.out, O.n_elems, lane);
                 }
             }
             g += run;
@@ -533,6 +536,7 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, ui
                 }
                 group_row<DT, CODEC>(lut, ring, pw, x, lt, s2, O.small_scales, dst);
                 group_row<DT, CODEC>(lut, ring, pw, x, lt, s2, O.small_scales, dst + kGroupSyms);
+                check_progress(status, ctl, pw, dst + 2 * kGroupSyms, O.out, O.n_elems, lane);
             }
             if (i < run && !ctl->dead) {
                 if (pw >= limit) limit = ring_service(ctl, ring, mbar, pw);
@@ -584,6 +588,7 @@ __device__ __forceinline__ bool decode_body(int32_t *status, const OutCtx &O, ui
             cursor_advance<DT, LAYOUT>(O, first + (uint64_t)g * kGroupSyms + kGroup * lane, cur);
         }
         pw += rp - rp0;
+        check_progress(status, ctl, pw, dst + kGroupSyms, O.out, O.n_elems, lane);
     }
     }
     if (tail && !tail_done && !ctl->dead) {
@@ -687,6 +692,7 @@ __global__ void __launch_bounds__(WARPS * 32, SHARED ? kSharedMinCtas : 1)
                 continue;
             }
             __syncwarp();
+            if (h.n_present > 1) check_table<CODEC>(P.status, S.lut, lane, 32);
             decode_body<DT, LAYOUT, CODEC>(P.status, out_ctx(M), (uint64_t)k * kChunkSyms, h.n, h.n_words,
                                     h.rec + h.table_bytes, h.n_present == 1, tab[0] & 0xFFu, h.x,
                                     S.lut_addr, S.ring, S.mbar, ctl, lane, lt, by_rank,
@@ -969,3 +975,5 @@ extern "C" EQW_API int eq_selftest_wait_timeout(int32_t *d_status, cudaStream_t 
     eq_wait_timeout_kernel<<<1, 32, 0, s>>>(d_status);
     return cudaGetLastError() == cudaSuccess ? EQ_OK : EQ_ERR_CUDA;
 }
+
+extern "C" EQW_API int eq_build_checked(void) { return EQ_CHECKED; }

@@ -76,12 +76,8 @@ struct PairSmem {
     static constexpr uint32_t kMetaOff = kRefOff + kPairTables * 64 * 4;      // per table: n_present (0: invalid)
     static constexpr uint32_t kBytes = kMetaOff + kPairTables * 4;
 };
-#ifndef EQ_TUPLE
-#define EQ_TUPLE 2
-#endif
-constexpr int kTuple = EQ_TUPLE;  // chunks decoded in lockstep per warp
-static_assert(PairSmem<kPairWarps, kTuple>::kBytes <= 227 * 1024, "pair kernel shared memory");
-static_assert(PairSmem<kPairWarps, kTuple>::kRingOff % 128 == 0, "ring alignment");
+static_assert(PairSmem<kPairWarps, 2>::kBytes <= 227 * 1024, "pair kernel shared memory");
+static_assert(PairSmem<kPairWarps, 2>::kRingOff % 128 == 0, "ring alignment");
 
 template <class Params>
 __device__ __forceinline__ uint32_t pair_job(const Params &P, uint32_t pair, uint32_t from) {
@@ -113,7 +109,7 @@ struct TupleSrc {
 // position at which the ring next needs service.  A wait that gives up sets
 // `dead` and leaves that segment not ready, so the drain waits for it again.
 __device__ __forceinline__ uint32_t tuple_service(RingRegs &R, uint32_t P, uint32_t gend, uint32_t ring,
-                                                  uint32_t mbar, const TupleSrc *src, bool &dead) {
+                                                  uint32_t mbar, const TupleSrc *src, bool &dead, int32_t *status) {
     const uint32_t horizon = min(gend, P / kSegBytes + kRingSegs);
     if (R.issued < horizon) {
         __syncwarp();
@@ -125,6 +121,7 @@ __device__ __forceinline__ uint32_t tuple_service(RingRegs &R, uint32_t P, uint3
                 const uint32_t off = (g - g0) * kSegBytes;
                 const uint32_t bytes = min(kSegBytes, pbytes - off);
                 const uint32_t slot = g % kRingSegs;
+                check(status, off < pbytes && off + bytes <= pbytes && bytes % 16 == 0);
                 mbar_expect_tx(mbar + 8 * slot, slot == 0 ? 2 * bytes : bytes);
                 bulk_load(ring + slot * kSegBytes, payload + off, bytes, mbar + 8 * slot);
                 if (slot == 0) bulk_load(ring + kRingBytes, payload + off, bytes, mbar);
@@ -214,7 +211,7 @@ struct TupleChain {
 // byte_off from the chain's current output position).
 template <uint32_t CODEC, int C>
 __device__ __forceinline__ void tuple_group(uint32_t lut, uint32_t ring0, TupleChain<CODEC> (&ch)[C], uint32_t lt,
-                                            uint32_t byte_off) {
+                                            uint32_t byte_off, int32_t *status) {
     uint32_t r0[C], rp[C], o[C][4];
 #pragma unroll
     for (int c = 0; c < C; ++c) rp[c] = r0[c] = ring0 + c * kRingStride + (ch[c].P & (kRingBytes - 1));
@@ -232,6 +229,8 @@ __device__ __forceinline__ void tuple_group(uint32_t lut, uint32_t ring0, TupleC
     }
 #pragma unroll
     for (int c = 0; c < C; ++c) {
+        // every word read lay in [r0, rp]: inside this chain's ring and its mirror
+        check(status, rp[c] + 2 <= ring0 + c * kRingStride + kRingStride);
         st_global_v4(reinterpret_cast<uint16_t *>(reinterpret_cast<uint8_t *>(ch[c].dst) + byte_off),
                      make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]));
         ch[c].P += rp[c] - r0[c];
@@ -286,13 +285,23 @@ __device__ __forceinline__ bool decode_tuple(int32_t *status, const PairJob &M, 
                 for (int c = 0; c < C; ++c)
                     if (ch[c].P >= ch[c].limit)
                         ch[c].limit = tuple_service(ch[c].R, ch[c].P, ch[c].gend, ring0 + c * kRingStride,
-                                                    mbar0 + 8 * kRingSegs * c, src + c, dead);
+                                                    mbar0 + 8 * kRingSegs * c, src + c, dead, status);
                 if (dead) break;
             }
-            tuple_group<CODEC, C>(lut, ring0, ch, lt, 0);
-            tuple_group<CODEC, C>(lut, ring0, ch, lt, 2 * kGroupSyms);
+            tuple_group<CODEC, C>(lut, ring0, ch, lt, 0, status);
+            tuple_group<CODEC, C>(lut, ring0, ch, lt, 2 * kGroupSyms, status);
 #pragma unroll
-            for (int c = 0; c < C; ++c) ch[c].dst += 2 * kGroupSyms;
+            for (int c = 0; c < C; ++c) {
+#if EQ_CHECKED
+                // the words consumed were waited for; the two stores lay inside the matrix
+                const uint32_t pb = (2u * h[c].n_words + 15u) & ~15u;
+                const uint32_t resident = ch[c].R.ready < ch[c].gend ? ch[c].R.ready * kSegBytes : g0[c] * kSegBytes + pb;
+                check(status, ch[c].P <= resident);
+                check(status, (uint64_t)(ch[c].dst - M.out) + 2 * kGroupSyms - kGroup * lane <=
+                                  (uint64_t)M.rows * M.cols);
+#endif
+                ch[c].dst += 2 * kGroupSyms;
+            }
         }
 #pragma unroll
         for (int c = 0; c < C; ++c)
@@ -373,6 +382,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) eq_decode_pairs_kernel(const __
         }
     }
     __syncthreads();
+    for (uint32_t j = 0; j < nt; ++j)
+        if (meta[j]) check_table<CODEC>(P.status, reinterpret_cast<uint32_t *>(smem) + j * kProbTotal, threadIdx.x,
+                                        WARPS * 32);
 
     const uint32_t lt = lanemask_lt();
     RingRegs R[C];  // ring counters and frame position carry over from tuple to tuple
@@ -402,15 +414,24 @@ __global__ void __launch_bounds__(WARPS * 32, 1) eq_decode_pairs_kernel(const __
 
 struct PairSetup {
     bool ready = false;
-    KernelSetup<PairParams> k[2][2];  // [codec][dtype - 1]
+    KernelSetup<PairParams> k[2][2][2];  // [chains per warp - 1][codec][dtype - 1]
 };
 std::mutex g_pair_mu;
 PairSetup g_pair[128];
 
-template <int DT, uint32_t CODEC>
+template <int C, int DT, uint32_t CODEC>
 int pair_setup_one(PairSetup &d) {
-    return setup_kernel(d.k[CODEC][DT - 1], eq_decode_pairs_kernel<kPairWarps, kTuple, DT, CODEC>, kPairWarps,
-                        PairSmem<kPairWarps, kTuple>::kBytes, 1);
+    return setup_kernel(d.k[C - 1][CODEC][DT - 1], eq_decode_pairs_kernel<kPairWarps, C, DT, CODEC>, kPairWarps,
+                        PairSmem<kPairWarps, C>::kBytes, 1);
+}
+
+template <int C>
+int pair_setup_chains(PairSetup &d) {
+    int rc;
+    if ((rc = pair_setup_one<C, EQ_INT8, kCodecRans>(d)) || (rc = pair_setup_one<C, EQ_E4M3, kCodecRans>(d)) ||
+        (rc = pair_setup_one<C, EQ_INT8, kCodecHuffman>(d)) || (rc = pair_setup_one<C, EQ_E4M3, kCodecHuffman>(d)))
+        return rc;
+    return EQ_OK;
 }
 
 int pair_setup(PairSetup **out) {
@@ -420,22 +441,20 @@ int pair_setup(PairSetup **out) {
     PairSetup &d = g_pair[dev];
     if (!d.ready) {
         int rc;
-        if ((rc = pair_setup_one<EQ_INT8, kCodecRans>(d)) || (rc = pair_setup_one<EQ_E4M3, kCodecRans>(d)) ||
-            (rc = pair_setup_one<EQ_INT8, kCodecHuffman>(d)) || (rc = pair_setup_one<EQ_E4M3, kCodecHuffman>(d)))
-            return rc;
+        if ((rc = pair_setup_chains<1>(d)) || (rc = pair_setup_chains<2>(d))) return rc;
         d.ready = true;
     }
     *out = &d;
     return EQ_OK;
 }
 
-// True if P can go to the pair kernel on `sms` SMs: the launch fills every warp
-// at least once (a launch with less than one round of pairs per warp is bound
-// by the latency of each chunk's dependent steps, and KB2 spreads it over more
-// warps, one chain each) and no block's range touches more than kPairTables
-// matrices.
-bool pairs_fit(const PairParams &P, uint32_t sms) {
-    if (!P.total_pairs || P.total_pairs < sms * (uint32_t)kPairWarps) return false;
+// True if P (tuples of `chains` chunks) can go to the kernel on `sms` SMs: with
+// two chains per warp the launch must give every warp a tuple at least once
+// (below that, each chunk's latency rules, and one chain per warp is faster);
+// and no block's range may touch more than kPairTables matrices.
+bool pairs_fit(const PairParams &P, uint32_t sms, uint32_t chains) {
+    if (!P.total_pairs) return false;
+    if (chains == 2 && P.total_pairs < sms * (uint32_t)kPairWarps) return false;
     const uint32_t grid = std::min<uint32_t>(sms, P.total_pairs);
     for (uint32_t b = 0; b < grid; ++b) {
         const uint32_t p0 = (uint32_t)((uint64_t)b * P.total_pairs / grid);
@@ -458,65 +477,84 @@ bool pair_eligible(const MatrixDesc &d, const void *out) {
     const eq_matrix_info &in = d.info;
     const uint64_t n = (uint64_t)in.rows * in.cols;
     return in.uniform_table && d.n_present0 >= 2 && d.n_present0 <= 32 && in.cols % (2 * kGroupSyms) == 0 &&
-           reinterpret_cast<uintptr_t>(out) % 16 == 0 && n / ((uint64_t)kTuple * kChunkSyms) >= 1;
+           reinterpret_cast<uintptr_t>(out) % 16 == 0 && n >= kChunkSyms;
 }
 
-// The pair-kernel launches for matrices mats[0..count) written to outs[]: one
-// per (codec, dtype) and up to kMaxMatsPerLaunch matrices, kept only where
-// pairs_fit; handled[i] = leading chunks of mats[i] they decode.  Host only.
+#ifndef EQ_SINGLES
+#define EQ_SINGLES 0
+#endif
+constexpr uint32_t kMinChains = EQ_SINGLES ? 1 : 2;
+
+// A launch of the tuple kernel: chains per warp, codec, dtype and its parameters.
+struct TupleLaunch {
+    uint32_t chains, codec, dtype;
+    PairParams P;
+};
+
+// The launches for matrices mats[0..count) written to outs[]: one per (codec,
+// dtype) and up to kMaxMatsPerLaunch matrices, each with two chains per warp
+// where that launch fills a round of warps, else one; handled[i] = leading
+// chunks of mats[i] they decode.  Host only.
 static void plan_pairs(const eq_model *m, const uint32_t *mats, uint16_t *const *outs, uint32_t count,
-                       int32_t *d_status, uint32_t sms, std::vector<std::pair<uint32_t, PairParams>> &launches,
-                       uint32_t *handled) {
+                       int32_t *d_status, uint32_t sms, std::vector<TupleLaunch> &launches, uint32_t *handled) {
     for (uint32_t i = 0; i < count; ++i) handled[i] = 0;
     for (uint32_t co = 0; co < 2; ++co)
         for (uint32_t dt = 0; dt < 2; ++dt) {
-            PairParams P{};
-            uint32_t idx[kMaxMatsPerLaunch];
-            auto reset = [&]() {
-                P = PairParams{};
-                P.blob = m->d_blob;
-                P.blob_len = m->len;
-                P.status = d_status;
-            };
-            auto flush = [&]() {
-                if (P.n_mats && pairs_fit(P, sms)) {
-                    for (uint32_t t = 0; t < P.n_mats; ++t) handled[idx[t]] = kTuple * P.mats[t].n_pairs;
-                    launches.emplace_back(2 * co + dt, P);
-                }
-                reset();
-            };
-            reset();
+            std::vector<uint32_t> ids;
             for (uint32_t i = 0; i < count; ++i) {
                 const MatrixDesc &d = m->mats[mats[i]];
-                if (d.codec != co || d.info.dtype != dt + 1 || !pair_eligible(d, outs[i])) continue;
-                if (P.n_mats == kMaxMatsPerLaunch) flush();
-                PairJob &J = P.mats[P.n_mats];
-                idx[P.n_mats++] = i;
-                J.chunk_index = reinterpret_cast<const uint64_t *>(m->d_blob + d.chunk_index_off);
-                J.scales = reinterpret_cast<const float *>(m->d_blob + d.scales_off);
-                J.out = outs[i];
-                J.cols = d.info.cols;
-                J.rows = d.info.rows;
-                J.first_pair = P.total_pairs;
-                J.n_pairs = (uint32_t)((uint64_t)d.info.rows * d.info.cols / ((uint64_t)kTuple * kChunkSyms));
-                P.total_pairs += J.n_pairs;
+                if (d.codec == co && d.info.dtype == dt + 1 && pair_eligible(d, outs[i])) ids.push_back(i);
             }
-            flush();
+            for (size_t base = 0; base < ids.size(); base += kMaxMatsPerLaunch) {
+                const size_t cnt = std::min<size_t>(kMaxMatsPerLaunch, ids.size() - base);
+                for (uint32_t chains = 2; chains >= kMinChains; --chains) {
+                    PairParams P{};
+                    P.blob = m->d_blob;
+                    P.blob_len = m->len;
+                    P.status = d_status;
+                    for (size_t t = 0; t < cnt; ++t) {
+                        const uint32_t i = ids[base + t];
+                        const MatrixDesc &d = m->mats[mats[i]];
+                        const uint32_t tuples =
+                            (uint32_t)((uint64_t)d.info.rows * d.info.cols / ((uint64_t)chains * kChunkSyms));
+                        if (!tuples) continue;
+                        PairJob &J = P.mats[P.n_mats++];
+                        J.chunk_index = reinterpret_cast<const uint64_t *>(m->d_blob + d.chunk_index_off);
+                        J.scales = reinterpret_cast<const float *>(m->d_blob + d.scales_off);
+                        J.out = outs[i];
+                        J.cols = d.info.cols;
+                        J.rows = d.info.rows;
+                        J.first_pair = P.total_pairs;
+                        J.n_pairs = tuples;
+                        P.total_pairs += tuples;
+                    }
+                    if (!pairs_fit(P, sms, chains)) continue;
+                    uint32_t j = 0;
+                    for (size_t t = 0; t < cnt; ++t) {
+                        const uint32_t i = ids[base + t];
+                        const MatrixDesc &d = m->mats[mats[i]];
+                        if ((uint64_t)d.info.rows * d.info.cols / ((uint64_t)chains * kChunkSyms))
+                            handled[i] = chains * P.mats[j++].n_pairs;
+                    }
+                    launches.push_back(TupleLaunch{chains, co, dt, P});
+                    break;
+                }
+            }
         }
 }
 
 int launch_decode_pairs(const eq_model *m, const uint32_t *mats, uint16_t *const *outs, uint32_t count,
                         int32_t *d_status, cudaStream_t s, int sms, uint32_t *handled) {
-    std::vector<std::pair<uint32_t, PairParams>> launches;
+    std::vector<TupleLaunch> launches;
     plan_pairs(m, mats, outs, count, d_status, (uint32_t)sms, launches, handled);
     if (launches.empty()) return EQ_OK;
     PairSetup *dev = nullptr;
     int rc = pair_setup(&dev);
     if (rc) return rc;
     for (auto &L : launches) {
-        const KernelSetup<PairParams> &k = dev->k[L.first / 2][L.first % 2];
-        const uint32_t grid = std::min<uint32_t>((uint32_t)sms, L.second.total_pairs);
-        k.fn<<<grid, k.warps * 32, k.smem, s>>>(L.second);
+        const KernelSetup<PairParams> &k = dev->k[L.chains - 1][L.codec][L.dtype];
+        const uint32_t grid = std::min<uint32_t>((uint32_t)sms, L.P.total_pairs);
+        k.fn<<<grid, k.warps * 32, k.smem, s>>>(L.P);
         if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
     }
     return EQ_OK;
@@ -525,7 +563,7 @@ int launch_decode_pairs(const eq_model *m, const uint32_t *mats, uint16_t *const
 int plan_decode_pairs(const eq_model *m, const uint32_t *mats, uint32_t count, uint32_t sms, uint32_t *handled) {
     // outputs as eq_decode_block places them: 256-byte aligned
     std::vector<uint16_t *> outs(count, reinterpret_cast<uint16_t *>(static_cast<uintptr_t>(256)));
-    std::vector<std::pair<uint32_t, PairParams>> launches;
+    std::vector<TupleLaunch> launches;
     plan_pairs(m, mats, outs.data(), count, nullptr, sms, launches, handled);
     return EQ_OK;
 }

@@ -178,6 +178,23 @@ __device__ __forceinline__ void flag(int32_t *status, int32_t bits) {
     if ((threadIdx.x & 31u) == 0) atomicOr(status, bits);
 }
 
+// Checked build (EQ_CHECKED=1): conditions the kernels guarantee by
+// construction are tested at run time, per lane; a failure ORs EQ_DEV_CHECK
+// into the status word and the kernel carries on.  Compiled out otherwise.
+#ifndef EQ_CHECKED
+#define EQ_CHECKED 0
+#endif
+constexpr int32_t kDevCheck = 64;  // EQ_DEV_CHECK
+
+__device__ __forceinline__ void check(int32_t *status, bool cond) {
+#if EQ_CHECKED
+    if (!cond) atomicOr(status, kDevCheck);
+#else
+    (void)status;
+    (void)cond;
+#endif
+}
+
 // ---- word staging ring ------------------------------------------------------------
 // Per-warp bookkeeping lives in shared memory so that the decode loop keeps a
 // single register for it: `limit`, the consumed-byte count at which the next
@@ -273,6 +290,25 @@ __device__ __noinline__ bool ring_drain(RingCtl *ctl, uint32_t mbar) {
     }
     __syncwarp();
     return all_ok && !ctl->dead;
+}
+
+// Checked build: after a run of groups, the payload bytes consumed so far
+// (pw) were all waited for, and the next output position of this lane (dst)
+// is still inside the matrix ([out, out + n)).
+__device__ __forceinline__ void check_progress(int32_t *status, const RingCtl *ctl, uint32_t pw, const uint16_t *dst,
+                                               const uint16_t *out, uint64_t n, uint32_t lane) {
+#if EQ_CHECKED
+    check(status, pw <= min(ctl->ready * kSegBytes, ctl->pbytes));
+    check(status, (uint64_t)(dst - out) <= n + kGroup * lane);
+#else
+    (void)status;
+    (void)ctl;
+    (void)pw;
+    (void)dst;
+    (void)out;
+    (void)n;
+    (void)lane;
+#endif
 }
 
 // ---- the rANS step ---------------------------------------------------------------
@@ -542,6 +578,29 @@ __device__ __forceinline__ uint32_t slot_entry(uint32_t e, uint32_t f, uint32_t 
     else return (f << 20) | (t << 8) | low;
 }
 
+// Checked build: every slot of a filled table holds a usable entry -- rANS:
+// f >= 1 and slot - cum < f; Huffman: a code length of 1..12.  Threads
+// `first`, `first + step`, ... check their slots.
+template <uint32_t CODEC>
+__device__ __forceinline__ void check_table(int32_t *status, const uint32_t *lut, uint32_t first, uint32_t step) {
+#if EQ_CHECKED
+    for (uint32_t t = first; t < kProbTotal; t += step) {
+        const uint32_t e = lut[t];
+        if constexpr (CODEC == kCodecHuffman) {
+            const uint32_t len = (e >> 8) & 0xFu;
+            check(status, len >= 1 && len <= kHuffMaxLen);
+        } else {
+            check(status, (e >> 20) >= 1 && ((e >> 8) & 0xFFFu) < (e >> 20));
+        }
+    }
+#else
+    (void)status;
+    (void)lut;
+    (void)first;
+    (void)step;
+#endif
+}
+
 // Check a frequency list / code table (n_present entries at `tab`): keys
 // ascending, reserved bits zero, every entry covering >= 1 slot, all 4096
 // slots covered (rANS: sum of f; Huffman: Kraft equality).  Optionally copies
@@ -679,6 +738,7 @@ __device__ __forceinline__ void shared_table_rebuild(const Params &P, const Job 
         }
     }
     __syncthreads();
+    if (S.blk[1] && np > 1) check_table<CODEC>(P.status, S.lut, threadIdx.x, WARPS * 32);
 }
 
 // Shared-table kernels: chunk k's header, checked, and its frequency list

@@ -52,6 +52,9 @@ namespace {
 #ifndef EQ_GEMM_THREADS
 #define EQ_GEMM_THREADS 256
 #endif
+#ifndef EQ_GEMM_TMEM_A
+#define EQ_GEMM_TMEM_A 1
+#endif
 constexpr int kGemmThreads = EQ_GEMM_THREADS;  // 4 or 8 warps
 // Token halves per CTA: each widened weight tile feeds kHalves MMAs of 128
 // tokens into kHalves accumulators (one instruction shape, M = 128, whatever
@@ -417,6 +420,250 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
     }
 }
 
+// ---- weights in tensor memory -------------------------------------------------------
+// eq_gemm_tm_kernel: the same product with the roles of the operands swapped
+// and the widened weights never in shared memory.  One CTA per 128-row x
+// 256-token output tile; the MMA is M = 128 weight rows (A, read from tensor
+// memory) x N = 256 tokens (B, the TMA-copied token tile in shared memory),
+// K 16, fp32 accumulator in tensor memory (128 lanes x 256 columns: lane =
+// weight row, column = token).  Per K slab of 64:
+//   producers  thread (w, l) of the 8 producer warps owns weight row
+//              32 (w % 4) + l and half w / 4 of the slab's 64 columns: it
+//              loads its 32 symbol bytes straight into registers (one slab
+//              ahead), widens them exactly to bf16 and stores them with
+//              tcgen05.st into its own tensor-memory lane, in the stage's 16
+//              columns of that half (two bf16 per 32-bit column, the lower K
+//              index in the low half); thread 0 also issues the token tile's
+//              two TMA tensor copies (128 tokens each)
+//   MMA warp   one lane waits for "full", issues the slab's 4 MMAs (A from
+//              tensor memory, B from the swizzled token tile) and commits them
+//              to the stage's "empty" barrier
+//   epilogue   thread (w, l) reads its weight row's 128 accumulator columns
+//              of half w / 4 (tcgen05.ld), multiplies by its row's scale and
+//              stores them, one token column at a time (a warp's 32 lanes
+//              write 32 consecutive outputs of one token)
+// Shared memory per slab: the token tile written once (32 KB) and read once by
+// the MMAs (32 KB), against 128 KB in eq_gemm_symbols_kernel.
+constexpr uint32_t kTmTileN = 128;                     // weight rows per CTA (MMA M)
+constexpr uint32_t kTmTileT = 256;                     // tokens per CTA (MMA N)
+constexpr uint32_t kTmK = 64;                          // K per slab
+constexpr uint32_t kTmStages = 4;
+constexpr uint32_t kTmBBytes = kTmTileT * kTmK * 2;    // 32 KB token tile per stage
+constexpr uint32_t kTmAccCols = kTmTileT;              // fp32 accumulator columns
+constexpr uint32_t kTmACols = kTmK / 2;                // tensor-memory columns of one stage's weights
+constexpr uint32_t kTmAlloc = 512;                     // accumulator + kTmStages weight stages, rounded up
+static_assert(kTmAccCols + kTmStages * kTmACols <= kTmAlloc, "tensor memory columns");
+static_assert(kTileK == kTmK, "token map box: 64 columns");
+constexpr size_t kTmSmem = kTmStages * kTmBBytes + 1024;
+constexpr uint32_t kTmInstrDesc = (1u << 4)                  // D format fp32
+                                | (1u << 7)                  // A format bf16
+                                | (1u << 10)                 // B format bf16
+                                | ((kTmTileT >> 3) << 17)    // N / 8
+                                | ((kTmTileN >> 4) << 24);   // M / 16
+
+__device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "r"(tmem_a), "l"(db), "r"(kTmInstrDesc), "r"(accumulate)
+        : "memory");
+}
+
+// 16 consecutive 32-bit columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_tm_kernel(const __grid_constant__ GemmParams P) {
+    constexpr uint32_t kProducerWarps = kGemmThreads / 32;
+    static_assert(kProducerWarps == 8, "two producer warps per tensor-memory lane quarter");
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t full_s[kTmStages], empty_s[kTmStages], done_s;
+    __shared__ uint32_t tmem_base_s;
+    const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
+    const bool mma_warp = warp == kProducerWarps;
+    // token tiles vary fastest, so the blocks that read one weight tile run together
+    const uint32_t n0 = blockIdx.y * kTmTileN;  // weight rows
+    const uint32_t m0 = blockIdx.x * kTmTileT;  // tokens
+    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    auto bufB = [&](uint32_t st) { return base + st * kTmBBytes; };
+    const uint32_t full0 = smem_u32(&full_s[0]), empty0 = smem_u32(&empty_s[0]), done = smem_u32(&done_s);
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(&tmem_base_s)), "r"(kTmAlloc) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        for (uint32_t st = 0; st < kTmStages; ++st) {
+            mbar_init(full0 + 8 * st, kProducerWarps + 1u);  // + the token tile's expect_tx arrival
+            mbar_init(empty0 + 8 * st, 1);
+        }
+        mbar_init(done, 1);
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_s;                 // lane 0, first allocated column
+    const uint32_t tmem_a = tmem + kTmAccCols;         // weight stages follow the accumulator
+    const uint32_t n_slabs = P.cols / kTmK;
+    bool ok = true;
+
+    if (!mma_warp) {
+        const uint32_t quarter = warp & 3u, half = warp >> 2;
+        const uint32_t lane_base = (quarter * 32u) << 16;
+        const uint8_t *src = P.sym + (size_t)(n0 + quarter * 32u + lane) * P.cols + half * 32u;
+        uint4 cur0 = ldg_nc_v4(src), cur1 = ldg_nc_v4(src + 16);
+        for (uint32_t it = 0; it < n_slabs; ++it) {
+            const uint32_t s = it % kTmStages;
+            uint4 nx0 = cur0, nx1 = cur1;
+            if (it + 1 < n_slabs) {  // next slab's symbols, one slab ahead
+                nx0 = ldg_nc_v4(src + (size_t)(it + 1) * kTmK);
+                nx1 = ldg_nc_v4(src + (size_t)(it + 1) * kTmK + 16);
+            }
+            // stage s last held slab it - kTmStages: wait until its MMAs are done
+            if (it >= kTmStages) {
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty0 + 8 * s, ((it - kTmStages) / kTmStages) & 1u))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+            }
+            if (tid == 0) {
+                // token tile: two TMA tensor copies of 128 tokens (x = k0, a multiple of
+                // 64 elements; rows past the last token read as zeros)
+                mbar_expect_tx(full0 + 8 * s, kTmBBytes);
+#pragma unroll
+                for (uint32_t h = 0; h < 2; ++h)
+                    asm volatile(
+                        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                        " [%0], [%1, {%2, %3}], [%4];" ::"r"(bufB(s) + h * kMmaM * kRowBytes),
+                        "l"(reinterpret_cast<uint64_t>(&P.tmap_x)), "r"(it * kTmK), "r"(m0 + h * kMmaM),
+                        "r"(full0 + 8 * s)
+                        : "memory");
+            }
+            // this row's 32 symbols of the slab, widened exactly, into its tensor-memory lane
+            uint4 lo0, hi0, lo1, hi1;
+            widen16<DT>(cur0, lo0, hi0);
+            widen16<DT>(cur1, lo1, hi1);
+            const uint32_t v[16] = {lo0.x, lo0.y, lo0.z, lo0.w, hi0.x, hi0.y, hi0.z, hi0.w,
+                                    lo1.x, lo1.y, lo1.z, lo1.w, hi1.x, hi1.y, hi1.z, hi1.w};
+            tmem_st16(tmem_a + lane_base + s * kTmACols + half * (kTmACols / 2), v);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full0 + 8 * s);
+            cur0 = nx0;
+            cur1 = nx1;
+        }
+    } else if (lane == 0) {
+        for (uint32_t it = 0; it < n_slabs; ++it) {
+            const uint32_t s = it % kTmStages;
+            if (!mbar_wait_bounded(full0 + 8 * s, (it / kTmStages) & 1u)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (uint32_t kk = 0; kk < kTmK / kMmaK; ++kk)
+                tc_mma_ts(tmem, tmem_a + s * kTmACols + kk * (kMmaK / 2), tile_desc(bufB(s), kk), (it | kk) != 0u);
+            tc_commit(empty0 + 8 * s);
+        }
+        tc_commit(done);  // completes when every MMA issued above has
+    }
+    if (!mma_warp) {
+        ok = mbar_wait_bounded(done, 0u) && ok;
+        tc_fence_after();
+        if (__all_sync(0xFFFFFFFFu, ok)) {
+            // thread (w, l): weight row 32 (w % 4) + l, tokens 128 (w / 4) ..
+            const uint32_t quarter = warp & 3u, half = warp >> 2;
+            const uint32_t r = n0 + quarter * 32u + lane;
+            const float sc = __ldg(P.scales + r);
+#pragma unroll 1
+            for (uint32_t c = 0; c < kTmAccCols / 2; c += 32) {
+                uint32_t acc[32];
+                tmem_ld32(tmem + ((quarter * 32u) << 16) + half * (kTmAccCols / 2) + c, acc);
+                const uint32_t t0 = m0 + half * (kTmAccCols / 2) + c;
+#pragma unroll
+                for (uint32_t j = 0; j < 32; ++j)
+                    if (t0 + j < P.tokens) P.y[(size_t)(t0 + j) * P.rows + r] = __fmul_rn(__uint_as_float(acc[j]), sc);
+            }
+        }
+    }
+    if (!ok) atomicOr(P.status, EQ_DEV_TIMEOUT);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmAlloc)
+                     : "memory");
+    }
+}
+
+// Failure-path check of the GEMM's waits: the GEMM's own set-up (TMEM
+// allocation, "full" / "empty" / "done" barriers with its arrival counts) and
+// exit path (status flag, TMEM release), but no producer ever arrives on
+// "full", so the MMA lane's bounded wait must give up; it then arrives on
+// "done" itself, the producers pass it (or give up on it) and the block
+// returns with EQ_DEV_TIMEOUT set and its TMEM freed.
+__global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_wait_timeout_kernel(int32_t *status) {
+    constexpr uint32_t kProducerWarps = kGemmThreads / 32;
+    __shared__ __align__(8) uint64_t full_s[kStages], empty_s[kStages], done_s;
+    __shared__ uint32_t tmem_base_s;
+    const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
+    const uint32_t full0 = smem_u32(&full_s[0]), empty0 = smem_u32(&empty_s[0]), done = smem_u32(&done_s);
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(&tmem_base_s)), "r"(kTmemAlloc) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        for (uint32_t st = 0; st < kStages; ++st) {
+            mbar_init(full0 + 8 * st, kProducerWarps + 1u);
+            mbar_init(empty0 + 8 * st, 1);
+        }
+        mbar_init(done, 1);
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_s;
+    bool ok = true;
+    if (warp == kProducerWarps) {
+        if (lane == 0) {
+            ok = mbar_wait_bounded(full0, 0u);  // nothing arrives: gives up after the limit
+            mbar_arrive(done);                  // releases the producers (synchronous: nothing left in flight)
+        }
+    } else {
+        ok = mbar_wait_bounded(done, 0u);
+    }
+    if (!ok) atomicOr(status, EQ_DEV_TIMEOUT);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemAlloc)
+                     : "memory");
+    }
+}
+
 // Super weights: Y[t, r] += bf16(v) * X[t, c], one thread per (super weight, token).
 __global__ void eq_gemm_outliers_kernel(const uint32_t *rec, uint32_t n_out, const uint16_t *x, uint32_t tokens,
                                         uint32_t rows, uint32_t cols, float *y, int32_t *status) {
@@ -470,6 +717,7 @@ int encode_token_map(CUtensorMap *map, const void *x, uint32_t tokens, uint32_t 
 
 extern "C" EQW_API int eq_gemm_symbols(const eq_model *m, uint32_t matrix, const void *d_sym, const void *d_x,
                                        uint32_t tokens, float *d_y, int32_t *d_status, cudaStream_t s) {
+    const eqw::NvtxScope nvtx_range("eq_gemm_symbols");
     if (!m || !d_status || matrix >= m->mats.size()) return EQ_ERR_INVALID_ARG;
     const MatrixDesc &d = m->mats[matrix];
     const eq_matrix_info &in = d.info;
@@ -492,16 +740,23 @@ extern "C" EQW_API int eq_gemm_symbols(const eq_model *m, uint32_t matrix, const
     P.rows = in.rows;
     P.cols = in.cols;
     P.dtype = in.dtype;
+#if EQ_GEMM_TMEM_A
+    auto fn = in.dtype == EQ_INT8 ? eq_gemm_tm_kernel<EQ_INT8> : eq_gemm_tm_kernel<EQ_E4M3>;
+    const size_t smem = kTmSmem;
+    const dim3 grid((tokens + kTmTileT - 1) / kTmTileT, in.rows / kTmTileN);
+#else
     auto fn = in.dtype == EQ_INT8 ? eq_gemm_symbols_kernel<EQ_INT8> : eq_gemm_symbols_kernel<EQ_E4M3>;
+    const size_t smem = kGemmSmem;
+    const dim3 grid((tokens + kTileM - 1) / kTileM, in.rows / kTileN);
+#endif
     bool &attr = g_gemm_attr_set[dev][in.dtype - 1];
     if (!attr) {
         if (cudaFuncSetAttribute(reinterpret_cast<const void *>(fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kGemmSmem) != cudaSuccess)
+                                 (int)smem) != cudaSuccess)
             return EQ_ERR_CUDA;
         attr = true;
     }
-    const dim3 grid((tokens + kTileM - 1) / kTileM, in.rows / kTileN);
-    fn<<<grid, kGemmThreads + 32, kGemmSmem, s>>>(P);
+    fn<<<grid, kGemmThreads + 32, smem, s>>>(P);
     if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
     if (in.n_outliers) {
         const uint64_t n = (uint64_t)in.n_outliers * tokens;
@@ -511,4 +766,10 @@ extern "C" EQW_API int eq_gemm_symbols(const eq_model *m, uint32_t matrix, const
         if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
     }
     return EQ_OK;
+}
+
+extern "C" EQW_API int eq_selftest_gemm_wait_timeout(int32_t *d_status, cudaStream_t s) {
+    if (!d_status) return EQ_ERR_INVALID_ARG;
+    eq_gemm_wait_timeout_kernel<<<1, kGemmThreads + 32, 0, s>>>(d_status);
+    return cudaGetLastError() == cudaSuccess ? EQ_OK : EQ_ERR_CUDA;
 }

@@ -84,7 +84,11 @@ enum {
     EQ_DEV_BAD_STATE = 4,    /* an initial state outside [2^16, 2^32) */
     EQ_DEV_BAD_END = 8,      /* final states != 2^16 or words consumed != n_words */
     EQ_DEV_TIMEOUT = 16,     /* a bounded wait for a staged copy gave up */
-    EQ_DEV_BAD_OUTLIER = 32  /* outlier position outside its matrix, or a non-zero stream value under it */
+    EQ_DEV_BAD_OUTLIER = 32, /* outlier position outside its matrix, or a non-zero stream value under it */
+    EQ_DEV_CHECK = 64        /* checked build only (EQ_CHECKED=1): an invariant the kernels rely on failed --
+                                a staging-ring word read outside the ring or before its copy was waited for,
+                                an unfilled slot-table entry, a store outside the matrix, or a bulk copy
+                                outside the chunk's payload; never set by a release build */
 };
 
 /* symbol formats */
@@ -396,6 +400,20 @@ EQW_API int eq_gemm_symbols(const eq_model *m, uint32_t matrix, const void *d_sy
  * the context stays usable.  Enqueued on `s`; d_status as for the decoders.
  */
 EQW_API int eq_selftest_wait_timeout(int32_t *d_status, cudaStream_t s);
+
+/* 1 if this library was built with EQ_CHECKED=1 (libeqw_checked.so: the decode
+ * kernels test their invariants at run time and report EQ_DEV_CHECK), else 0.
+ * The checked build's outputs are those of the release build, bit for bit. */
+EQW_API int eq_build_checked(void);
+
+/*
+ * The same check for the prefill GEMM's waits (eq_gemm_symbols): one block
+ * with the GEMM's TMEM allocation and mbarrier ring, whose MMA lane waits on a
+ * "full" barrier no producer arrives on; after the bounded wait gives up (~1
+ * s) the block ORs EQ_DEV_TIMEOUT into *d_status, frees its TMEM and returns.
+ * No fault, trap or hang.  Errors: EQ_ERR_INVALID_ARG, EQ_ERR_CUDA.
+ */
+EQW_API int eq_selftest_gemm_wait_timeout(int32_t *d_status, cudaStream_t s);
 
 /* ---- misc ----------------------------------------------------------------------- */
 EQW_API const char *eq_status_string(int status);
