@@ -76,8 +76,9 @@ struct PairSmem {
     static constexpr uint32_t kMetaOff = kRefOff + kPairTables * 64 * 4;      // per table: n_present (0: invalid)
     static constexpr uint32_t kBytes = kMetaOff + kPairTables * 4;
 };
-static_assert(PairSmem<kPairWarps, 2>::kBytes <= 227 * 1024, "pair kernel shared memory");
-static_assert(PairSmem<kPairWarps, 2>::kRingOff % 128 == 0, "ring alignment");
+constexpr int kTuple = 2;  // chunks decoded in lockstep per warp
+static_assert(PairSmem<kPairWarps, kTuple>::kBytes <= 227 * 1024, "pair kernel shared memory");
+static_assert(PairSmem<kPairWarps, kTuple>::kRingOff % 128 == 0, "ring alignment");
 
 template <class Params>
 __device__ __forceinline__ uint32_t pair_job(const Params &P, uint32_t pair, uint32_t from) {
@@ -414,24 +415,15 @@ __global__ void __launch_bounds__(WARPS * 32, 1) eq_decode_pairs_kernel(const __
 
 struct PairSetup {
     bool ready = false;
-    KernelSetup<PairParams> k[2][2][2];  // [chains per warp - 1][codec][dtype - 1]
+    KernelSetup<PairParams> k[2][2];  // [codec][dtype - 1]
 };
 std::mutex g_pair_mu;
 PairSetup g_pair[128];
 
-template <int C, int DT, uint32_t CODEC>
+template <int DT, uint32_t CODEC>
 int pair_setup_one(PairSetup &d) {
-    return setup_kernel(d.k[C - 1][CODEC][DT - 1], eq_decode_pairs_kernel<kPairWarps, C, DT, CODEC>, kPairWarps,
-                        PairSmem<kPairWarps, C>::kBytes, 1);
-}
-
-template <int C>
-int pair_setup_chains(PairSetup &d) {
-    int rc;
-    if ((rc = pair_setup_one<C, EQ_INT8, kCodecRans>(d)) || (rc = pair_setup_one<C, EQ_E4M3, kCodecRans>(d)) ||
-        (rc = pair_setup_one<C, EQ_INT8, kCodecHuffman>(d)) || (rc = pair_setup_one<C, EQ_E4M3, kCodecHuffman>(d)))
-        return rc;
-    return EQ_OK;
+    return setup_kernel(d.k[CODEC][DT - 1], eq_decode_pairs_kernel<kPairWarps, kTuple, DT, CODEC>, kPairWarps,
+                        PairSmem<kPairWarps, kTuple>::kBytes, 1);
 }
 
 int pair_setup(PairSetup **out) {
@@ -441,20 +433,22 @@ int pair_setup(PairSetup **out) {
     PairSetup &d = g_pair[dev];
     if (!d.ready) {
         int rc;
-        if ((rc = pair_setup_chains<1>(d)) || (rc = pair_setup_chains<2>(d))) return rc;
+        if ((rc = pair_setup_one<EQ_INT8, kCodecRans>(d)) || (rc = pair_setup_one<EQ_E4M3, kCodecRans>(d)) ||
+            (rc = pair_setup_one<EQ_INT8, kCodecHuffman>(d)) || (rc = pair_setup_one<EQ_E4M3, kCodecHuffman>(d)))
+            return rc;
         d.ready = true;
     }
     *out = &d;
     return EQ_OK;
 }
 
-// True if P (tuples of `chains` chunks) can go to the kernel on `sms` SMs: with
-// two chains per warp the launch must give every warp a tuple at least once
-// (below that, each chunk's latency rules, and one chain per warp is faster);
-// and no block's range may touch more than kPairTables matrices.
-bool pairs_fit(const PairParams &P, uint32_t sms, uint32_t chains) {
-    if (!P.total_pairs) return false;
-    if (chains == 2 && P.total_pairs < sms * (uint32_t)kPairWarps) return false;
+// True if P can go to the pair kernel on `sms` SMs: the launch gives every
+// warp a pair at least once (a launch with less than one round of pairs per
+// warp is bound by the latency of each chunk's dependent steps; KB2 spreads it
+// over more warps, one chain each, and takes the whole call in one launch) and
+// no block's range touches more than kPairTables matrices.
+bool pairs_fit(const PairParams &P, uint32_t sms) {
+    if (!P.total_pairs || P.total_pairs < sms * (uint32_t)kPairWarps) return false;
     const uint32_t grid = std::min<uint32_t>(sms, P.total_pairs);
     for (uint32_t b = 0; b < grid; ++b) {
         const uint32_t p0 = (uint32_t)((uint64_t)b * P.total_pairs / grid);
@@ -477,26 +471,20 @@ bool pair_eligible(const MatrixDesc &d, const void *out) {
     const eq_matrix_info &in = d.info;
     const uint64_t n = (uint64_t)in.rows * in.cols;
     return in.uniform_table && d.n_present0 >= 2 && d.n_present0 <= 32 && in.cols % (2 * kGroupSyms) == 0 &&
-           reinterpret_cast<uintptr_t>(out) % 16 == 0 && n >= kChunkSyms;
+           reinterpret_cast<uintptr_t>(out) % 16 == 0 && n >= (uint64_t)kTuple * kChunkSyms;
 }
 
-#ifndef EQ_SINGLES
-#define EQ_SINGLES 0
-#endif
-constexpr uint32_t kMinChains = EQ_SINGLES ? 1 : 2;
-
-// A launch of the tuple kernel: chains per warp, codec, dtype and its parameters.
-struct TupleLaunch {
-    uint32_t chains, codec, dtype;
+// A launch of the pair kernel: codec, dtype and its parameters.
+struct PairLaunch {
+    uint32_t codec, dtype;
     PairParams P;
 };
 
 // The launches for matrices mats[0..count) written to outs[]: one per (codec,
-// dtype) and up to kMaxMatsPerLaunch matrices, each with two chains per warp
-// where that launch fills a round of warps, else one; handled[i] = leading
-// chunks of mats[i] they decode.  Host only.
+// dtype) and up to kMaxMatsPerLaunch matrices, each kept only where pairs_fit;
+// handled[i] = leading chunks of mats[i] they decode.  Host only.
 static void plan_pairs(const eq_model *m, const uint32_t *mats, uint16_t *const *outs, uint32_t count,
-                       int32_t *d_status, uint32_t sms, std::vector<TupleLaunch> &launches, uint32_t *handled) {
+                       int32_t *d_status, uint32_t sms, std::vector<PairLaunch> &launches, uint32_t *handled) {
     for (uint32_t i = 0; i < count; ++i) handled[i] = 0;
     for (uint32_t co = 0; co < 2; ++co)
         for (uint32_t dt = 0; dt < 2; ++dt) {
@@ -507,52 +495,39 @@ static void plan_pairs(const eq_model *m, const uint32_t *mats, uint16_t *const 
             }
             for (size_t base = 0; base < ids.size(); base += kMaxMatsPerLaunch) {
                 const size_t cnt = std::min<size_t>(kMaxMatsPerLaunch, ids.size() - base);
-                for (uint32_t chains = 2; chains >= kMinChains; --chains) {
-                    PairParams P{};
-                    P.blob = m->d_blob;
-                    P.blob_len = m->len;
-                    P.status = d_status;
-                    for (size_t t = 0; t < cnt; ++t) {
-                        const uint32_t i = ids[base + t];
-                        const MatrixDesc &d = m->mats[mats[i]];
-                        const uint32_t tuples =
-                            (uint32_t)((uint64_t)d.info.rows * d.info.cols / ((uint64_t)chains * kChunkSyms));
-                        if (!tuples) continue;
-                        PairJob &J = P.mats[P.n_mats++];
-                        J.chunk_index = reinterpret_cast<const uint64_t *>(m->d_blob + d.chunk_index_off);
-                        J.scales = reinterpret_cast<const float *>(m->d_blob + d.scales_off);
-                        J.out = outs[i];
-                        J.cols = d.info.cols;
-                        J.rows = d.info.rows;
-                        J.first_pair = P.total_pairs;
-                        J.n_pairs = tuples;
-                        P.total_pairs += tuples;
-                    }
-                    if (!pairs_fit(P, sms, chains)) continue;
-                    uint32_t j = 0;
-                    for (size_t t = 0; t < cnt; ++t) {
-                        const uint32_t i = ids[base + t];
-                        const MatrixDesc &d = m->mats[mats[i]];
-                        if ((uint64_t)d.info.rows * d.info.cols / ((uint64_t)chains * kChunkSyms))
-                            handled[i] = chains * P.mats[j++].n_pairs;
-                    }
-                    launches.push_back(TupleLaunch{chains, co, dt, P});
-                    break;
+                PairParams P{};
+                P.blob = m->d_blob;
+                P.blob_len = m->len;
+                P.status = d_status;
+                for (size_t t = 0; t < cnt; ++t) {
+                    const MatrixDesc &d = m->mats[mats[ids[base + t]]];
+                    PairJob &J = P.mats[P.n_mats++];
+                    J.chunk_index = reinterpret_cast<const uint64_t *>(m->d_blob + d.chunk_index_off);
+                    J.scales = reinterpret_cast<const float *>(m->d_blob + d.scales_off);
+                    J.out = outs[ids[base + t]];
+                    J.cols = d.info.cols;
+                    J.rows = d.info.rows;
+                    J.first_pair = P.total_pairs;
+                    J.n_pairs = (uint32_t)((uint64_t)d.info.rows * d.info.cols / ((uint64_t)kTuple * kChunkSyms));
+                    P.total_pairs += J.n_pairs;
                 }
+                if (!pairs_fit(P, sms)) continue;
+                for (size_t t = 0; t < cnt; ++t) handled[ids[base + t]] = kTuple * P.mats[t].n_pairs;
+                launches.push_back(PairLaunch{co, dt, P});
             }
         }
 }
 
 int launch_decode_pairs(const eq_model *m, const uint32_t *mats, uint16_t *const *outs, uint32_t count,
                         int32_t *d_status, cudaStream_t s, int sms, uint32_t *handled) {
-    std::vector<TupleLaunch> launches;
+    std::vector<PairLaunch> launches;
     plan_pairs(m, mats, outs, count, d_status, (uint32_t)sms, launches, handled);
     if (launches.empty()) return EQ_OK;
     PairSetup *dev = nullptr;
     int rc = pair_setup(&dev);
     if (rc) return rc;
     for (auto &L : launches) {
-        const KernelSetup<PairParams> &k = dev->k[L.chains - 1][L.codec][L.dtype];
+        const KernelSetup<PairParams> &k = dev->k[L.codec][L.dtype];
         const uint32_t grid = std::min<uint32_t>((uint32_t)sms, L.P.total_pairs);
         k.fn<<<grid, k.warps * 32, k.smem, s>>>(L.P);
         if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
@@ -563,7 +538,7 @@ int launch_decode_pairs(const eq_model *m, const uint32_t *mats, uint16_t *const
 int plan_decode_pairs(const eq_model *m, const uint32_t *mats, uint32_t count, uint32_t sms, uint32_t *handled) {
     // outputs as eq_decode_block places them: 256-byte aligned
     std::vector<uint16_t *> outs(count, reinterpret_cast<uint16_t *>(static_cast<uintptr_t>(256)));
-    std::vector<TupleLaunch> launches;
+    std::vector<PairLaunch> launches;
     plan_pairs(m, mats, outs.data(), count, nullptr, sms, launches, handled);
     return EQ_OK;
 }
