@@ -493,27 +493,18 @@ def bench_eqw(args, d: Dist) -> dict | None:
         hstack.close()
         del hblob
 
-    # ---- E: prefill on tensor cores: symbols of layer 0 decoded once, 7 GEMMs over 1024 tokens ----
+    # ---- E: prefill on tensor cores: symbols of layer 0 decoded once, the layer's 7 GEMMs in one ----
+    # ---- persistent launch over 1024 (and 4096) tokens                                          ----
     prefill = None
     if d.rank == 0:
         pstep = stack.steps[0]
         pm = pstep.model
         idx = list(pm.layer_matrices(pstep.layer))
         infos = [pm.info(i) for i in idx]
-        tokens = 1024
         syms = [torch.empty(inf.rows * inf.cols, dtype=torch.uint8, device=dev) for inf in infos]
-        xs_p = [W.gemv_activation(7, j, tokens * inf.cols).reshape(tokens, inf.cols).to(dev)
-                for j, inf in enumerate(infos)]
-        ys_p = [torch.empty(tokens, inf.rows, dtype=torch.float32, device=dev) for inf in infos]
         pst = torch.zeros(1, dtype=torch.int32, device=dev)
         ps = torch.cuda.Stream(device=dev)
-
-        def p_decode():
-            pm.decode_symbols_block(pstep.layer, syms, pst, ps)
-
-        def p_gemm():
-            for i, mi in enumerate(idx):
-                pm.gemm_symbols(mi, syms[i], xs_p[i], ys_p[i], pst, ps)
+        bf16_peak = measured_bf16_peak()
 
         def p_time(fn, n=5):
             for _ in range(3):
@@ -527,21 +518,27 @@ def bench_eqw(args, d: Dist) -> dict | None:
             torch.cuda.synchronize()
             return a.elapsed_time(b) / n
 
-        dec_ms = p_time(p_decode)
-        gemm_ms = p_time(p_gemm)
+        dec_ms = p_time(lambda: pm.decode_symbols_block(pstep.layer, syms, pst, ps))
+        by_tokens = {}
+        for tokens in (1024, 4096):
+            xs_p = [W.gemv_activation(7, j, tokens * inf.cols).reshape(tokens, inf.cols).to(dev)
+                    for j, inf in enumerate(infos)]
+            ys_p = [torch.empty(tokens, inf.rows, dtype=torch.float32, device=dev) for inf in infos]
+            gemm_ms = p_time(lambda: pm.gemm_symbols_block(pstep.layer, syms, xs_p, ys_p, pst, ps))
+            flops = sum(2.0 * tokens * inf.rows * inf.cols for inf in infos)
+            tflops = flops / (gemm_ms / 1e3) / 1e12
+            by_tokens[tokens] = {"gemm_ms": round(gemm_ms, 4), "tflops": round(tflops, 1),
+                                 "frac": round(tflops / bf16_peak, 4), "layer_ms": round(dec_ms + gemm_ms, 4)}
+            del xs_p, ys_p
         if int(pst.item()) != 0:
             raise RuntimeError(f"prefill status {int(pst.item())}")
-        flops = sum(2.0 * tokens * inf.rows * inf.cols for inf in infos)
-        bf16_peak = measured_bf16_peak()
-        tflops = flops / (gemm_ms / 1e3) / 1e12
-        prefill = {"tokens": tokens, "decode_symbols_ms": round(dec_ms, 4), "gemm_ms": round(gemm_ms, 4),
-                   "tflops": round(tflops, 1), "unit": "TFLOP/s", "bf16_peak": bf16_peak,
-                   "frac": round(tflops / bf16_peak, 4), "kernel": "eq_gemm_symbols_kernel (tcgen05)",
-                   "layer_ms": round(dec_ms + gemm_ms, 4),
-                   "note": "layer 0: the 7 matrices' symbols decoded to bytes in one launch, then one tcgen05 "
-                           "GEMM per matrix against 1024 bf16 tokens (fp32 out); frac of the measured cuBLAS "
-                           "bf16 burst peak"}
-        del syms, xs_p, ys_p
+        prefill = {"tokens": 1024, "decode_symbols_ms": round(dec_ms, 4), **by_tokens[1024],
+                   "unit": "TFLOP/s", "bf16_peak": bf16_peak, "tokens_4096": by_tokens[4096],
+                   "kernel": "eq_gemm_symbols_kernel (tcgen05)",
+                   "note": "layer 0: the 7 matrices' symbols decoded to bytes in one launch, then the 7 "
+                           "tcgen05 GEMMs in one persistent launch (eq_gemm_symbols_block) against 1024 "
+                           "bf16 tokens (fp32 out); frac of the measured cuBLAS bf16 burst peak"}
+        del syms
 
     # ---- C: fused decode + GEMV, no bf16 buffers; blocks in sequence on one stream ----
     fstream = torch.cuda.Stream(device=dev)

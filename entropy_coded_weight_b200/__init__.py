@@ -282,6 +282,21 @@ class Model:
         check(self._L.eq_gemm_symbols(self._m, matrix, sym.data_ptr(), x.data_ptr(), x.shape[0], y.data_ptr(),
                                       status.data_ptr(), _stream_handle(stream)), "eq_gemm_symbols")
 
+    def gemm_symbols_block(self, layer: int, syms, xs, ys, status, stream=None) -> None:
+        """eq_gemm_symbols_block: ``gemm_symbols`` for every matrix of ``layer`` (``syms[i]``, ``xs[i]``,
+        ``ys[i]`` belong to matrix i of the layer), one persistent tensor-core launch per weight type."""
+        n = len(syms)
+        if len(xs) != n or len(ys) != n:
+            raise ValueError("syms, xs and ys must have one entry per matrix of the layer")
+        tokens = xs[0].shape[0] if n else 0
+        if any(x.shape[0] != tokens for x in xs):
+            raise ValueError("every input of a block GEMM takes the same number of tokens")
+        ps = (ctypes.c_void_p * max(1, n))(*(t.data_ptr() for t in syms))
+        px = (ctypes.c_void_p * max(1, n))(*(t.data_ptr() for t in xs))
+        py = (ctypes.c_void_p * max(1, n))(*(t.data_ptr() for t in ys))
+        check(self._L.eq_gemm_symbols_block(self._m, layer, ps, px, tokens, py, n, status.data_ptr(),
+                                            _stream_handle(stream)), "eq_gemm_symbols_block")
+
     def decode_gemv_matrix(self, matrix: int, x, y, status, stream=None) -> None:
         """eq_decode_gemv_matrix: y = W x without materialising W (x bf16 [cols], y fp32 [rows], device)."""
         check(self._L.eq_decode_gemv_matrix(self._m, matrix, x.data_ptr(), y.data_ptr(), status.data_ptr(),

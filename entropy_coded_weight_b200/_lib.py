@@ -83,6 +83,7 @@ SIGNATURES = {
     "eq_decode_symbols": (_i32, [_vp, _u32, _vp, _sz, _vp, _vp]),
     "eq_decode_symbols_block": (_i32, [_vp, _u32, _vp, _u32, _vp, _vp]),
     "eq_gemm_symbols": (_i32, [_vp, _u32, _vp, _vp, _u32, _vp, _vp, _vp]),
+    "eq_gemm_symbols_block": (_i32, [_vp, _u32, _vp, _vp, _u32, _vp, _u32, _vp, _vp]),
     "eq_selftest_wait_timeout": (_i32, [_vp, _vp]),
     "eq_selftest_gemm_wait_timeout": (_i32, [_vp, _vp]),
     "eq_status_string": (ctypes.c_char_p, [_i32]),

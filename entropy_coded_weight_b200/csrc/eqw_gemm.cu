@@ -8,33 +8,45 @@
 //   Y[t, r] = scale[r] * sum_c X[t, c] * value(sym[r, c])
 //             + sum over super weights (r, c, v) of bf16(v) * X[t, c]
 // X is bf16 [tokens, cols], Y fp32 [tokens, rows], both row-major.  Every
-// Int8 / E4M3 value is exact in bf16, so each tile of symbols is widened
-// exactly to bf16 in shared memory and multiplied with tcgen05.mma
-// (kind::f16, bf16 x bf16, fp32 accumulator in tensor memory); the row scale
-// is applied once per output in the epilogue and the (rare) super weights by
-// a small second kernel.
+// Int8 / E4M3 value is exact in bf16, so each slab of symbols is widened
+// exactly to bf16 and multiplied with tcgen05.mma (kind::f16, bf16 x bf16,
+// fp32 accumulator in tensor memory); the row scale is applied once per
+// output in the epilogue and the (rare) super weights by a small second
+// kernel.
 //
-// Kernel eq_gemm_symbols_kernel, one CTA per 256-token x 128-row output tile
-// (two token halves sharing each widened weight tile), 8 producer warps and
-// one MMA warp:
-//   producers  per K slab of 64: one TMA tensor copy of the token tile
-//              (issued by thread 0, 128-byte swizzle: the K-major layout the
-//              MMA reads, 16-byte chunk c of row r at chunk position
-//              c ^ (r % 8), 8-row groups 1024 B apart) and cp.async copies of
-//              the symbol bytes into a staging area, issued kAhead slabs
-//              ahead into a ring of kStages stages; once a thread's copies of
-//              a slab have landed it widens its own symbol chunks into the
-//              swizzled bf16 tile and its warp arrives on the stage's "full"
+// Kernel eq_gemm_symbols_kernel: a persistent launch (one CTA per SM) over the
+// 128-row x 256-token output tiles of up to 8 matrices of one weight type (a
+// transformer block's projections in one launch; the matrix with the longest
+// K first, CTA b taking tiles b, b + grid, ...), 8 producer warps and one MMA
+// warp per CTA.  The MMA is M = 128 weight rows (A, read
+// from tensor memory) x N = 256 tokens (B, in shared memory) x K 16, with the
+// fp32 accumulator in tensor memory (128 lanes x 256 columns: lane = weight
+// row, column = token).  Per K slab of 64:
+//   producers  thread (w, l) owns weight row 32 (w % 4) + l and half w / 4 of
+//              the slab's 64 columns: it loads its 32 symbol bytes straight
+//              into registers (one slab ahead), widens them exactly to bf16
+//              and stores them with tcgen05.st into its own tensor-memory lane,
+//              in the stage's 16 columns of that half (two bf16 per 32-bit
+//              column, the lower K index in the low half); thread 0 also issues
+//              the token tile's two TMA tensor copies (128 tokens each, 128-byte
+//              swizzle: the K-major layout the MMA's B descriptor reads, 16-byte
+//              chunk c of row r at chunk position c ^ (r % 8), 8-row groups
+//              1024 B apart); each warp then arrives on the stage's "full"
 //              mbarrier (which also waits for the tensor copy's bytes); a
-//              stage is refilled only after its "empty" barrier says the
-//              tensor core is done with it
-//   MMA warp   one lane waits for "full", issues 4 x 2 tcgen05.mma (M 128,
-//              N 128, K 16; token half h into the fp32 accumulator in TMEM
-//              columns 128 h .. 128 h + 127) and tcgen05.commit to the
-//              stage's "empty" barrier; a last commit to "done" releases the
-//              epilogue
-//   epilogue   producer warp w reads accumulator lanes 32 (w % 4) with
-//              tcgen05.ld, multiplies by the row scales and stores fp32
+//              stage is refilled only after its "empty" barrier says the tensor
+//              core is done with it
+//   MMA warp   one lane waits for "full", issues the slab's 4 MMAs and
+//              tcgen05.commits them to the stage's "empty" barrier; a last
+//              commit to "done" releases the epilogue
+//   epilogue   thread (w, l) reads its weight row's 128 accumulator columns of
+//              half w / 4 (tcgen05.ld), multiplies by the row's scale and stores
+//              them one token column at a time (a warp's 32 lanes write 32
+//              consecutive outputs of one token)
+// Between tiles the MMA warp waits on "acc_free" (every producer warp has read
+// its part of the accumulator) before the next tile's first MMA; the stage
+// ring and its barrier phases run on across tiles.
+// Shared memory per slab: the token tile written once and read once by the
+// MMAs, 32 KB; the widened weights never touch it.
 // Every mbarrier wait is bounded; on expiry the CTA records EQ_DEV_TIMEOUT,
 // still releases its tensor memory and stops.
 #include <cuda.h>
@@ -44,72 +56,51 @@
 
 #include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "eqw_device.cuh"
 
 namespace {
 
-#ifndef EQ_GEMM_THREADS
-#define EQ_GEMM_THREADS 256
-#endif
-#ifndef EQ_GEMM_TMEM_A
-#define EQ_GEMM_TMEM_A 1
-#endif
-constexpr int kGemmThreads = EQ_GEMM_THREADS;  // 4 or 8 warps
-// Token halves per CTA: each widened weight tile feeds kHalves MMAs of 128
-// tokens into kHalves accumulators (one instruction shape, M = 128, whatever
-// the CTA's token tile).
-#ifndef EQ_GEMM_HALVES
-#define EQ_GEMM_HALVES 2
-#endif
-#ifndef EQ_GEMM_STAGES
-#define EQ_GEMM_STAGES 4
-#endif
-static_assert(EQ_GEMM_HALVES >= 1 && EQ_GEMM_HALVES <= 4, "one to four 128-token parts per CTA");
-constexpr uint32_t kMmaM = 128;                        // tokens per MMA (accumulator lanes)
-constexpr uint32_t kHalves = EQ_GEMM_HALVES;           // MMAs per widened weight tile
-constexpr uint32_t kTileM = kMmaM * kHalves;           // tokens per CTA tile
-#ifndef EQ_GEMM_TILE_N
-#define EQ_GEMM_TILE_N 128
-#endif
-constexpr uint32_t kTileN = EQ_GEMM_TILE_N;            // weight rows per tile (MMA N, accumulator columns)
-static_assert(kTileN % 16 == 0 && kTileN >= 16 && kTileN <= 256, "cta_group::1 MMA with M = 128: N in 16..256");
-#ifndef EQ_GEMM_K
-#define EQ_GEMM_K 64
-#endif
-constexpr uint32_t kTileK = EQ_GEMM_K;                 // K per stage: 64 (128-byte rows) or 32 (64-byte rows)
-static_assert(kTileK == 64 || kTileK == 32, "K per stage");
-constexpr uint32_t kRowBytes = kTileK * 2;             // one bf16 tile row = one swizzle row
+constexpr int kGemmThreads = 256;                      // 8 producer warps (two per tensor-memory lane quarter)
+constexpr uint32_t kTileN = 128;                       // weight rows per CTA (MMA M, accumulator lanes)
+constexpr uint32_t kTileT = 256;                       // tokens per CTA (MMA N, accumulator columns)
+constexpr uint32_t kTileK = 64;                        // K per slab (128-byte rows: the 128-byte swizzle)
+constexpr uint32_t kBoxT = 128;                        // tokens per TMA box
+constexpr uint32_t kRowBytes = kTileK * 2;             // one bf16 token row of a slab = one swizzle row
 constexpr uint32_t kAtomBytes = 8 * kRowBytes;         // 8-row swizzle atom (SBO)
 constexpr uint32_t kMmaK = 16;                         // K per tcgen05.mma (bf16)
-constexpr uint32_t kStageBytesA = kTileM * kTileK * 2;  // 16 KiB per 128 tokens
-constexpr uint32_t kStageBytesB = kTileN * kTileK * 2;  // 16 KiB
-constexpr uint32_t kStages = EQ_GEMM_STAGES;
-#ifndef EQ_GEMM_AHEAD
-#define EQ_GEMM_AHEAD 2
-#endif
-constexpr uint32_t kAhead = EQ_GEMM_AHEAD;              // slabs whose copies are in flight ahead of use
-static_assert(kAhead < kStages, "a stage is refilled only after its previous slab's MMAs");
-constexpr uint32_t kStageBytesS = kTileN * kTileK;      // 8 KiB of symbol bytes (staging)
-constexpr uint32_t kStageBytes = kStageBytesA + kStageBytesB + kStageBytesS;
-constexpr uint32_t kTmemCols = kTileN * kHalves;        // one fp32 accumulator per token part
-// tcgen05.alloc takes a power of two of at least 32 columns
-constexpr uint32_t kTmemAlloc = kTmemCols <= 32 ? 32 : kTmemCols <= 64 ? 64 : kTmemCols <= 128 ? 128
-                              : kTmemCols <= 256 ? 256 : 512;
-static_assert(kTmemCols <= 512, "tensor memory has 512 columns");
+constexpr uint32_t kStages = 4;
+constexpr uint32_t kStageBytes = kTileT * kTileK * 2;  // 32 KB token tile per stage
+constexpr uint32_t kAccCols = kTileT;                  // fp32 accumulator columns
+constexpr uint32_t kACols = kTileK / 2;                // tensor-memory columns of one stage's weights
+constexpr uint32_t kTmemAlloc = 512;                   // accumulator + kStages weight stages, rounded up
+static_assert(kAccCols + kStages * kACols <= kTmemAlloc, "tensor memory columns");
 constexpr size_t kGemmSmem = kStages * kStageBytes + 1024;
 
-struct GemmParams {
-    CUtensorMap tmap_x;       // bf16 [tokens, cols], box kTileK x 128 (one per token part), swizzled
-    const uint16_t *x;        // bf16 [tokens, cols]
+constexpr uint32_t kMaxGemmJobs = 8;  // matrices per launch (a transformer block has 7)
+
+// One matrix of a launch: its tiles are [first_tile, first_tile + rows / 128 *
+// token tiles), weight-row tile major, token tile fastest.
+struct GemmJob {
+    CUtensorMap tmap_x;       // bf16 [tokens, cols] input of this matrix, box kTileK x kBoxT, 128-byte swizzle
     const uint8_t *sym;       // [rows, cols]
     const float *scales;      // [rows]
     float *y;                 // [tokens, rows]
-    int32_t *status;
-    uint32_t tokens, rows, cols;
-    uint32_t dtype;
+    uint32_t rows, cols;
+    uint32_t first_tile;
+    uint32_t pad;
 };
 
+struct GemmParams {
+    int32_t *status;
+    uint32_t tokens;
+    uint32_t t_tiles;         // token tiles per weight-row tile
+    uint32_t n_jobs;
+    uint32_t total_tiles;
+    GemmJob jobs[kMaxGemmJobs];
+};
+static_assert(sizeof(GemmParams) <= 4096, "kernel parameter space");
 
 // Shared-memory matrix descriptor (tcgen05), K-major: start address, leading
 // byte offset, stride byte offset (between 8-row groups), all in 16-byte
@@ -120,44 +111,27 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
     d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
     d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
     d |= (uint64_t)1 << 46;                        // descriptor version for tcgen05
-    // layout type: 2 = 128-byte swizzle (K 64), 4 = 64-byte swizzle (K 32); base
-    // offset 0: every tile starts on a 1024-byte boundary
-    d |= (uint64_t)(kTileK == 64 ? 2 : 4) << 61;
+    // layout type 2 = 128-byte swizzle; base offset 0: every tile starts on a
+    // 1024-byte boundary
+    d |= (uint64_t)2 << 61;
     return d;
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
-// K-major, N and M of one MMA.  M is the instruction's 128, not the CTA's
-// token tile: cta_group::1 takes M = 64 or 128 only, and an M field of 256
-// here is an illegal instruction on the GPU.
-static_assert(kMmaM == 64 || kMmaM == 128, "cta_group::1 MMA shape");
+// K-major, N = 256 tokens, M = 128 weight rows (cta_group::1 takes M = 64 or
+// 128 only).
 constexpr uint32_t kInstrDesc = (1u << 4)                 // D format fp32
                               | (1u << 7)                 // A format bf16
                               | (1u << 10)                // B format bf16
-                              | ((kTileN >> 3) << 17)     // N / 8
-                              | ((kMmaM >> 4) << 24);     // M / 16
-
-// Byte offset of the 16-byte chunk k8 (bf16 8 k8 .. 8 k8 + 7) of tile row
-// `row` in the swizzled K-major layout: one tile row per swizzle row, 8-row
-// atoms kAtomBytes apart, and chunk k8 of row r at chunk position
-// k8 ^ (r % 8) (128-byte swizzle) or k8 ^ ((r / 2) % 4) (64-byte swizzle):
-// the XOR of the offset's bits 4.. with its bits 7.. that both the TMA copy
-// and the MMA's descriptors apply.
-__device__ __forceinline__ uint32_t tile_offset(uint32_t row, uint32_t k8) {
-    const uint32_t sw = kTileK == 64 ? (row & 7u) : ((row >> 1) & 3u);
-    return (row >> 3) * kAtomBytes + (row & 7u) * kRowBytes + ((k8 ^ sw) << 4);
-}
+                              | ((kTileT >> 3) << 17)     // N / 8
+                              | ((kTileN >> 4) << 24);    // M / 16
+static_assert(kTileN == 128 && kTileT % 16 == 0 && kTileT <= 256, "cta_group::1 MMA shape");
 
 // Descriptor of K step kk (16 bf16) of a tile at `buf`: the start advances by
 // 32 bytes per step inside the swizzle row (the hardware applies the XOR),
 // LBO unused (16), SBO = one 8-row atom.
 __device__ __forceinline__ uint64_t tile_desc(uint32_t buf, uint32_t kk) {
     return smem_desc(buf + kk * 32u, 16u, kAtomBytes);
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                 : "memory");
 }
 
 // 16 symbol bytes -> 16 bf16 (exact), as two 16-byte vectors, without the
@@ -209,15 +183,6 @@ __device__ __forceinline__ void widen16(uint4 b, uint4 &lo, uint4 &hi) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(tmem_d), "l"(da), "l"(db), "r"(kInstrDesc), "r"(accumulate)
-        : "memory");
-}
-
 __device__ __forceinline__ void tc_commit(uint32_t mbar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
                  : "memory");
@@ -237,236 +202,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// 16-byte asynchronous copy global -> shared (src_bytes 0: zero fill).
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-    return v;
-}
-
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-
-// Warp-specialised mainloop: kProducerWarps warps fill a ring of kStages
-// shared-memory stages (token tile copied, symbol tile widened) and arrive on
-// the stage's "full" barrier (one arrival per warp); the MMA warp's first lane
-// waits for "full", issues the slab's 4 MMAs and commits them to the stage's
-// "empty" barrier, which the producers wait on before refilling the stage; a
-// final commit to "done" releases the epilogue.  No block-wide barrier runs
-// inside the loop.
-template <int DT>
-__global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(const __grid_constant__ GemmParams P) {
-    constexpr uint32_t kProducerWarps = kGemmThreads / 32;
-    extern __shared__ __align__(1024) unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t full_s[kStages], empty_s[kStages], done_s;
-    __shared__ uint32_t tmem_base_s;
-    const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
-    const bool mma_warp = warp == kProducerWarps;
-    // token tiles vary fastest, so the blocks that read one weight tile run
-    // together and it comes from DRAM once (the token matrix stays in L2)
-    const uint32_t n0 = blockIdx.y * kTileN;   // weight rows (outputs)
-    const uint32_t m0 = blockIdx.x * kTileM;   // tokens
-    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    // stage st: token tile (swizzled bf16), widened symbol tile (swizzled bf16), symbol bytes (staging)
-    auto bufA = [&](uint32_t st) { return base + st * kStageBytes; };
-    auto bufB = [&](uint32_t st) { return base + st * kStageBytes + kStageBytesA; };
-    auto bufS = [&](uint32_t st) { return base + st * kStageBytes + kStageBytesA + kStageBytesB; };
-    const uint32_t full0 = smem_u32(&full_s[0]), empty0 = smem_u32(&empty_s[0]), done = smem_u32(&done_s);
-
-    if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32(&tmem_base_s)), "r"(kTmemAlloc) : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    if (tid == 0) {
-        for (uint32_t st = 0; st < kStages; ++st) {
-            mbar_init(full0 + 8 * st, kProducerWarps + 1u);  // + the token tile's expect_tx arrival
-            mbar_init(empty0 + 8 * st, 1);
-        }
-        mbar_init(done, 1);
-        fence_mbar_init();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = tmem_base_s;
-    const uint32_t n_slabs = P.cols / kTileK;
-    bool ok = true;
-
-    if (!mma_warp) {
-        // per thread: kBv 16-byte chunks of the symbol tile (kSymChunks per row)
-        constexpr uint32_t kSymChunks = kTileK / 16;
-        constexpr uint32_t kBv = kTileN * kSymChunks / kGemmThreads;
-        // this thread's copies of slab `it` into stage `st`
-        auto issue = [&](uint32_t it, uint32_t st) {
-            const uint32_t k0 = it * kTileK;
-            // token tile: one TMA tensor copy (x = k0 is a multiple of 64
-            // elements, 128 bytes; rows past the last token read as zeros),
-            // completing on the stage's "full" barrier
-            if (tid == 0) {
-                mbar_expect_tx(full0 + 8 * st, kStageBytesA);
-#pragma unroll
-                for (uint32_t h = 0; h < kHalves; ++h)  // one 128-token box per part
-                    asm volatile(
-                        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-                        " [%0], [%1, {%2, %3}], [%4];" ::"r"(bufA(st) + h * kMmaM * kRowBytes),
-                        "l"(reinterpret_cast<uint64_t>(&P.tmap_x)), "r"(k0), "r"(m0 + h * kMmaM),
-                        "r"(full0 + 8 * st)
-                        : "memory");
-            }
-#pragma unroll
-            for (uint32_t i = 0; i < kBv; ++i) {
-                const uint32_t e = tid + i * kGemmThreads, r = e / kSymChunks, c = e % kSymChunks;
-                cp_async16(bufS(st) + e * 16u, P.sym + (size_t)(n0 + r) * P.cols + k0 + 16 * c, 16u);
-            }
-        };
-        // the first kAhead slabs go to stages that start out free
-        for (uint32_t it = 0; it < kAhead; ++it) {
-            if (it < n_slabs) issue(it, it % kStages);
-            cp_async_commit();
-        }
-        for (uint32_t it = 0; it < n_slabs; ++it) {
-            const uint32_t s = it % kStages;
-            const uint32_t ahead = it + kAhead;
-            if (ahead < n_slabs) {
-                const uint32_t sa = ahead % kStages;
-                // stage sa last held slab ahead - kStages: wait until its MMAs are done
-                // (the decision is warp-uniform: the __syncwarp below needs every lane)
-                if (ahead >= kStages &&
-                    !__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty0 + 8 * sa, ((ahead - kStages) / kStages) & 1u))) {
-                    ok = false;
-                    break;
-                }
-                issue(ahead, sa);
-            }
-            cp_async_commit();            // one group per slab, empty past the end
-            cp_async_wait<kAhead>();      // this thread's copies of slab `it` have landed
-            // widen this thread's own symbol chunks of slab `it`
-#pragma unroll
-            for (uint32_t i = 0; i < kBv; ++i) {
-                const uint32_t e = tid + i * kGemmThreads, r = e / kSymChunks, c = e % kSymChunks;
-                uint4 lo, hi;
-                widen16<DT>(ld_shared_v4(bufS(s) + e * 16u), lo, hi);
-                st_shared_v4(bufB(s) + tile_offset(r, 2 * c), lo);
-                st_shared_v4(bufB(s) + tile_offset(r, 2 * c + 1), hi);
-            }
-            fence_proxy_async_smem();  // copies and stores -> visible to the tensor core
-            __syncwarp();
-            if (lane == 0) mbar_arrive(full0 + 8 * s);
-        }
-        cp_async_wait<0>();
-    } else if (lane == 0) {
-        for (uint32_t it = 0; it < n_slabs; ++it) {
-            const uint32_t s = it % kStages;
-            if (!mbar_wait_bounded(full0 + 8 * s, (it / kStages) & 1u)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-#pragma unroll
-            for (uint32_t kk = 0; kk < kTileK / kMmaK; ++kk)
-#pragma unroll
-                for (uint32_t h = 0; h < kHalves; ++h)  // half h: tokens 128 h .., accumulator columns 128 h ..
-                    tc_mma(tmem + h * kTileN, tile_desc(bufA(s) + h * kMmaM * kRowBytes, kk),
-                           tile_desc(bufB(s), kk), (it | kk) != 0u);
-            tc_commit(empty0 + 8 * s);
-        }
-        tc_commit(done);  // completes when every MMA issued above has
-    }
-    if (!mma_warp) {
-        ok = mbar_wait_bounded(done, 0u) && ok;
-        tc_fence_after();
-        if (__all_sync(0xFFFFFFFFu, ok)) {
-            // warp w reads accumulator lanes 32 (w % 4) .. + 31; warps sharing a
-            // lane quarter split the columns (half h = columns 128 h ..)
-            constexpr uint32_t kColsPerWarp = kTmemCols * 4 / kProducerWarps;
-            const uint32_t quarter = warp & 3u, c_first = (warp >> 2) * (kColsPerWarp / 32);
-#pragma unroll 1
-            for (uint32_t c = c_first; c < c_first + kColsPerWarp / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tmem + ((quarter * 32u) << 16) + c * 32u, r);
-                const uint32_t half = c * 32u / kTileN, n_off = c * 32u % kTileN;
-                const uint32_t m = m0 + half * kMmaM + quarter * 32u + lane;
-                if (m < P.tokens) {
-                    float4 *dst = reinterpret_cast<float4 *>(P.y + (size_t)m * P.rows + n0 + n_off);
-                    const float4 *sc = reinterpret_cast<const float4 *>(P.scales + n0 + n_off);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 s4 = __ldg(sc + q);
-                        dst[q] = make_float4(__fmul_rn(__uint_as_float(r[4 * q]), s4.x),
-                                             __fmul_rn(__uint_as_float(r[4 * q + 1]), s4.y),
-                                             __fmul_rn(__uint_as_float(r[4 * q + 2]), s4.z),
-                                             __fmul_rn(__uint_as_float(r[4 * q + 3]), s4.w));
-                    }
-                }
-            }
-        }
-    }
-    if (!ok) atomicOr(P.status, EQ_DEV_TIMEOUT);
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemAlloc)
-                     : "memory");
-    }
-}
-
-// ---- weights in tensor memory -------------------------------------------------------
-// eq_gemm_tm_kernel: the same product with the roles of the operands swapped
-// and the widened weights never in shared memory.  One CTA per 128-row x
-// 256-token output tile; the MMA is M = 128 weight rows (A, read from tensor
-// memory) x N = 256 tokens (B, the TMA-copied token tile in shared memory),
-// K 16, fp32 accumulator in tensor memory (128 lanes x 256 columns: lane =
-// weight row, column = token).  Per K slab of 64:
-//   producers  thread (w, l) of the 8 producer warps owns weight row
-//              32 (w % 4) + l and half w / 4 of the slab's 64 columns: it
-//              loads its 32 symbol bytes straight into registers (one slab
-//              ahead), widens them exactly to bf16 and stores them with
-//              tcgen05.st into its own tensor-memory lane, in the stage's 16
-//              columns of that half (two bf16 per 32-bit column, the lower K
-//              index in the low half); thread 0 also issues the token tile's
-//              two TMA tensor copies (128 tokens each)
-//   MMA warp   one lane waits for "full", issues the slab's 4 MMAs (A from
-//              tensor memory, B from the swizzled token tile) and commits them
-//              to the stage's "empty" barrier
-//   epilogue   thread (w, l) reads its weight row's 128 accumulator columns
-//              of half w / 4 (tcgen05.ld), multiplies by its row's scale and
-//              stores them, one token column at a time (a warp's 32 lanes
-//              write 32 consecutive outputs of one token)
-// Shared memory per slab: the token tile written once (32 KB) and read once by
-// the MMAs (32 KB), against 128 KB in eq_gemm_symbols_kernel.
-constexpr uint32_t kTmTileN = 128;                     // weight rows per CTA (MMA M)
-constexpr uint32_t kTmTileT = 256;                     // tokens per CTA (MMA N)
-constexpr uint32_t kTmK = 64;                          // K per slab
-constexpr uint32_t kTmStages = 4;
-constexpr uint32_t kTmBBytes = kTmTileT * kTmK * 2;    // 32 KB token tile per stage
-constexpr uint32_t kTmAccCols = kTmTileT;              // fp32 accumulator columns
-constexpr uint32_t kTmACols = kTmK / 2;                // tensor-memory columns of one stage's weights
-constexpr uint32_t kTmAlloc = 512;                     // accumulator + kTmStages weight stages, rounded up
-static_assert(kTmAccCols + kTmStages * kTmACols <= kTmAlloc, "tensor memory columns");
-static_assert(kTileK == kTmK, "token map box: 64 columns");
-constexpr size_t kTmSmem = kTmStages * kTmBBytes + 1024;
-constexpr uint32_t kTmInstrDesc = (1u << 4)                  // D format fp32
-                                | (1u << 7)                  // A format bf16
-                                | (1u << 10)                 // B format bf16
-                                | ((kTmTileT >> 3) << 17)    // N / 8
-                                | ((kTmTileN >> 4) << 24);   // M / 16
 
 __device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(tmem_d), "r"(tmem_a), "l"(db), "r"(kTmInstrDesc), "r"(accumulate)
+        ::"r"(tmem_d), "r"(tmem_a), "l"(db), "r"(kInstrDesc), "r"(accumulate)
         : "memory");
 }
 
@@ -489,121 +234,150 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
 }
 
 template <int DT>
-__global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_tm_kernel(const __grid_constant__ GemmParams P) {
+__global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(const __grid_constant__ GemmParams P) {
     constexpr uint32_t kProducerWarps = kGemmThreads / 32;
     static_assert(kProducerWarps == 8, "two producer warps per tensor-memory lane quarter");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t full_s[kTmStages], empty_s[kTmStages], done_s;
+    __shared__ __align__(8) uint64_t full_s[kStages], empty_s[kStages], done_s, acc_free_s;
     __shared__ uint32_t tmem_base_s;
+    __shared__ volatile uint32_t abort_s;  // a bounded wait gave up: every loop stops
     const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
     const bool mma_warp = warp == kProducerWarps;
-    // token tiles vary fastest, so the blocks that read one weight tile run together
-    const uint32_t n0 = blockIdx.y * kTmTileN;  // weight rows
-    const uint32_t m0 = blockIdx.x * kTmTileT;  // tokens
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    auto bufB = [&](uint32_t st) { return base + st * kTmBBytes; };
-    const uint32_t full0 = smem_u32(&full_s[0]), empty0 = smem_u32(&empty_s[0]), done = smem_u32(&done_s);
+    auto bufB = [&](uint32_t st) { return base + st * kStageBytes; };
+    const uint32_t full0 = smem_u32(&full_s[0]), empty0 = smem_u32(&empty_s[0]);
+    const uint32_t done = smem_u32(&done_s), acc_free = smem_u32(&acc_free_s);
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32(&tmem_base_s)), "r"(kTmAlloc) : "memory");
+                     ::"r"(smem_u32(&tmem_base_s)), "r"(kTmemAlloc) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
-        for (uint32_t st = 0; st < kTmStages; ++st) {
+        for (uint32_t st = 0; st < kStages; ++st) {
             mbar_init(full0 + 8 * st, kProducerWarps + 1u);  // + the token tile's expect_tx arrival
             mbar_init(empty0 + 8 * st, 1);
         }
         mbar_init(done, 1);
+        mbar_init(acc_free, kProducerWarps);  // every producer warp has read its accumulator part
         fence_mbar_init();
+        abort_s = 0;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_s;                 // lane 0, first allocated column
-    const uint32_t tmem_a = tmem + kTmAccCols;         // weight stages follow the accumulator
-    const uint32_t n_slabs = P.cols / kTmK;
+    const uint32_t tmem_a = tmem + kAccCols;           // weight stages follow the accumulator
+    const uint32_t quarter = warp & 3u, half = warp >> 2;
+    const uint32_t lane_base = (quarter * 32u) << 16;
     bool ok = true;
+    uint32_t g = 0;  // slabs so far in this CTA: stage g % kStages, phase g / kStages
 
-    if (!mma_warp) {
-        const uint32_t quarter = warp & 3u, half = warp >> 2;
-        const uint32_t lane_base = (quarter * 32u) << 16;
-        const uint8_t *src = P.sym + (size_t)(n0 + quarter * 32u + lane) * P.cols + half * 32u;
-        uint4 cur0 = ldg_nc_v4(src), cur1 = ldg_nc_v4(src + 16);
-        for (uint32_t it = 0; it < n_slabs; ++it) {
-            const uint32_t s = it % kTmStages;
-            uint4 nx0 = cur0, nx1 = cur1;
-            if (it + 1 < n_slabs) {  // next slab's symbols, one slab ahead
-                nx0 = ldg_nc_v4(src + (size_t)(it + 1) * kTmK);
-                nx1 = ldg_nc_v4(src + (size_t)(it + 1) * kTmK + 16);
-            }
-            // stage s last held slab it - kTmStages: wait until its MMAs are done
-            if (it >= kTmStages) {
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty0 + 8 * s, ((it - kTmStages) / kTmStages) & 1u))) {
-                    ok = false;
-                    break;
+    // persistent loop over the launch's tiles, longest matrices (most slabs) first
+    uint32_t ti = 0;
+    uint32_t jb = 0;
+    for (uint32_t tile = blockIdx.x; tile < P.total_tiles; tile += gridDim.x, ++ti) {
+        while (jb + 1 < P.n_jobs && tile >= P.jobs[jb + 1].first_tile) ++jb;
+        const GemmJob &J = P.jobs[jb];
+        const uint32_t local = tile - J.first_tile;
+        const uint32_t n0 = (local / P.t_tiles) * kTileN;  // weight rows
+        const uint32_t m0 = (local % P.t_tiles) * kTileT;  // tokens
+        const uint32_t n_slabs = J.cols / kTileK;
+
+        if (!mma_warp) {
+            if (__any_sync(0xFFFFFFFFu, abort_s != 0u)) break;  // another warp's wait gave up
+            const uint8_t *src = J.sym + (size_t)(n0 + quarter * 32u + lane) * J.cols + half * 32u;
+            uint4 cur0 = ldg_nc_v4(src), cur1 = ldg_nc_v4(src + 16);
+            for (uint32_t it = 0; it < n_slabs; ++it, ++g) {
+                const uint32_t s = g % kStages;
+                uint4 nx0 = cur0, nx1 = cur1;
+                if (it + 1 < n_slabs) {  // next slab's symbols, one slab ahead
+                    nx0 = ldg_nc_v4(src + (size_t)(it + 1) * kTileK);
+                    nx1 = ldg_nc_v4(src + (size_t)(it + 1) * kTileK + 16);
                 }
-                tc_fence_after();
-            }
-            if (tid == 0) {
-                // token tile: two TMA tensor copies of 128 tokens (x = k0, a multiple of
-                // 64 elements; rows past the last token read as zeros)
-                mbar_expect_tx(full0 + 8 * s, kTmBBytes);
+                // stage s last held slab g - kStages: wait until its MMAs are done
+                if (g >= kStages) {
+                    if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty0 + 8 * s, ((g - kStages) / kStages) & 1u))) {
+                        ok = false;
+                        abort_s = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                }
+                if (tid == 0) {
+                    // token tile: two TMA tensor copies of 128 tokens (x = k0, a multiple of
+                    // 64 elements; rows past the last token read as zeros)
+                    mbar_expect_tx(full0 + 8 * s, kStageBytes);
 #pragma unroll
-                for (uint32_t h = 0; h < 2; ++h)
-                    asm volatile(
-                        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-                        " [%0], [%1, {%2, %3}], [%4];" ::"r"(bufB(s) + h * kMmaM * kRowBytes),
-                        "l"(reinterpret_cast<uint64_t>(&P.tmap_x)), "r"(it * kTmK), "r"(m0 + h * kMmaM),
-                        "r"(full0 + 8 * s)
-                        : "memory");
+                    for (uint32_t h = 0; h < 2; ++h)
+                        asm volatile(
+                            "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                            " [%0], [%1, {%2, %3}], [%4];" ::"r"(bufB(s) + h * kBoxT * kRowBytes),
+                            "l"(reinterpret_cast<uint64_t>(&J.tmap_x)), "r"(it * kTileK), "r"(m0 + h * kBoxT),
+                            "r"(full0 + 8 * s)
+                            : "memory");
+                }
+                // this row's 32 symbols of the slab, widened exactly, into its tensor-memory lane
+                uint4 lo0, hi0, lo1, hi1;
+                widen16<DT>(cur0, lo0, hi0);
+                widen16<DT>(cur1, lo1, hi1);
+                const uint32_t v[16] = {lo0.x, lo0.y, lo0.z, lo0.w, hi0.x, hi0.y, hi0.z, hi0.w,
+                                        lo1.x, lo1.y, lo1.z, lo1.w, hi1.x, hi1.y, hi1.z, hi1.w};
+                tmem_st16(tmem_a + lane_base + s * kACols + half * (kACols / 2), v);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(full0 + 8 * s);
+                cur0 = nx0;
+                cur1 = nx1;
             }
-            // this row's 32 symbols of the slab, widened exactly, into its tensor-memory lane
-            uint4 lo0, hi0, lo1, hi1;
-            widen16<DT>(cur0, lo0, hi0);
-            widen16<DT>(cur1, lo1, hi1);
-            const uint32_t v[16] = {lo0.x, lo0.y, lo0.z, lo0.w, hi0.x, hi0.y, hi0.z, hi0.w,
-                                    lo1.x, lo1.y, lo1.z, lo1.w, hi1.x, hi1.y, hi1.z, hi1.w};
-            tmem_st16(tmem_a + lane_base + s * kTmACols + half * (kTmACols / 2), v);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(full0 + 8 * s);
-            cur0 = nx0;
-            cur1 = nx1;
-        }
-    } else if (lane == 0) {
-        for (uint32_t it = 0; it < n_slabs; ++it) {
-            const uint32_t s = it % kTmStages;
-            if (!mbar_wait_bounded(full0 + 8 * s, (it / kTmStages) & 1u)) {
+            if (!ok) break;
+            // epilogue of this tile: thread (w, l) holds weight row 32 (w % 4) + l, tokens 128 (w / 4) ..
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(done, ti & 1u))) {
                 ok = false;
+                abort_s = 1;
                 break;
             }
             tc_fence_after();
-#pragma unroll
-            for (uint32_t kk = 0; kk < kTmK / kMmaK; ++kk)
-                tc_mma_ts(tmem, tmem_a + s * kTmACols + kk * (kMmaK / 2), tile_desc(bufB(s), kk), (it | kk) != 0u);
-            tc_commit(empty0 + 8 * s);
-        }
-        tc_commit(done);  // completes when every MMA issued above has
-    }
-    if (!mma_warp) {
-        ok = mbar_wait_bounded(done, 0u) && ok;
-        tc_fence_after();
-        if (__all_sync(0xFFFFFFFFu, ok)) {
-            // thread (w, l): weight row 32 (w % 4) + l, tokens 128 (w / 4) ..
-            const uint32_t quarter = warp & 3u, half = warp >> 2;
             const uint32_t r = n0 + quarter * 32u + lane;
-            const float sc = __ldg(P.scales + r);
+            const float sc = __ldg(J.scales + r);
 #pragma unroll 1
-            for (uint32_t c = 0; c < kTmAccCols / 2; c += 32) {
+            for (uint32_t c = 0; c < kAccCols / 2; c += 32) {
                 uint32_t acc[32];
-                tmem_ld32(tmem + ((quarter * 32u) << 16) + half * (kTmAccCols / 2) + c, acc);
-                const uint32_t t0 = m0 + half * (kTmAccCols / 2) + c;
+                tmem_ld32(tmem + lane_base + half * (kAccCols / 2) + c, acc);
+                const uint32_t t0 = m0 + half * (kAccCols / 2) + c;
 #pragma unroll
                 for (uint32_t j = 0; j < 32; ++j)
-                    if (t0 + j < P.tokens) P.y[(size_t)(t0 + j) * P.rows + r] = __fmul_rn(__uint_as_float(acc[j]), sc);
+                    if (t0 + j < P.tokens) J.y[(size_t)(t0 + j) * J.rows + r] = __fmul_rn(__uint_as_float(acc[j]), sc);
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_free);  // the MMA warp may overwrite the accumulator
+        } else if (lane == 0) {
+            // the previous tile's epilogue must have read the accumulator
+            if (abort_s || (ti > 0 && !mbar_wait_bounded(acc_free, (ti - 1) & 1u))) {
+                ok = false;
+                abort_s = 1;
+                break;
+            }
+            tc_fence_after();
+            for (uint32_t it = 0; it < n_slabs; ++it, ++g) {
+                const uint32_t s = g % kStages;
+                if (abort_s || !mbar_wait_bounded(full0 + 8 * s, (g / kStages) & 1u)) {
+                    ok = false;
+                    abort_s = 1;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (uint32_t kk = 0; kk < kTileK / kMmaK; ++kk)
+                    tc_mma_ts(tmem, tmem_a + s * kACols + kk * (kMmaK / 2), tile_desc(bufB(s), kk), (it | kk) != 0u);
+                tc_commit(empty0 + 8 * s);
+            }
+            tc_commit(done);  // completes when every MMA issued above has
+            if (!ok) break;
+        } else {
+            g += n_slabs;  // lanes 1..31 of the MMA warp only keep count
         }
     }
     if (!ok) atomicOr(P.status, EQ_DEV_TIMEOUT);
@@ -611,7 +385,7 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_tm_kernel(const 
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmAlloc)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemAlloc)
                      : "memory");
     }
 }
@@ -698,19 +472,114 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // Tensor map of the token matrix: inner dimension cols (K), outer tokens;
-// box kTileK x kTileM with the swizzle the MMA descriptors expect.
+// box kTileK x kBoxT with the swizzle the MMA descriptors expect.
 int encode_token_map(CUtensorMap *map, const void *x, uint32_t tokens, uint32_t cols) {
     auto enc = tensor_map_encoder();
     if (!enc) return EQ_ERR_CUDA;
     const cuuint64_t dims[2] = {cols, tokens};
     const cuuint64_t strides[1] = {(cuuint64_t)cols * 2u};
-    const cuuint32_t box[2] = {kTileK, kMmaM};
+    const cuuint32_t box[2] = {kTileK, kBoxT};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           kTileK == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                           CU_TENSOR_MAP_SWIZZLE_128B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? EQ_OK : EQ_ERR_CUDA;
+}
+
+}  // namespace
+
+namespace {
+
+struct GemmRequest {
+    uint32_t matrix;
+    const void *sym, *x;
+    float *y;
+};
+
+// Checks one request against its matrix; EQ_OK, or the error the entry point returns.
+int check_request(const eq_model *m, const GemmRequest &q) {
+    if (q.matrix >= m->mats.size()) return EQ_ERR_INVALID_ARG;
+    const MatrixDesc &d = m->mats[q.matrix];
+    const eq_matrix_info &in = d.info;
+    if (!in.rows || !in.cols) return EQ_OK;
+    if (in.rows % kTileN || in.cols % kTileK || in.rows / kTileN > 65535u) return EQ_ERR_UNSUPPORTED;
+    if (!q.sym || !q.x || !q.y) return EQ_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(q.sym) % 16 || reinterpret_cast<uintptr_t>(q.x) % 16 ||
+        reinterpret_cast<uintptr_t>(q.y) % 16 || d.scales_off % 16)
+        return EQ_ERR_INVALID_ARG;
+    return EQ_OK;
+}
+
+// One persistent launch per weight type over the tiles of all requests of that
+// type (at most kMaxGemmJobs per launch), longest K first so that the static
+// round-robin tile order ends with the short tiles; then the super weights.
+int gemm_launch(const eq_model *m, const GemmRequest *req, uint32_t n, uint32_t tokens, int32_t *d_status,
+                cudaStream_t s) {
+    if (!m || !d_status || (n && !req)) return EQ_ERR_INVALID_ARG;
+    for (uint32_t i = 0; i < n; ++i)
+        if (const int rc = check_request(m, req[i])) return rc;
+    if (!tokens) return EQ_OK;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return EQ_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return EQ_ERR_CUDA;
+    if (m->sm_limit && m->sm_limit < (uint32_t)sms) sms = (int)m->sm_limit;
+    const uint32_t t_tiles = (tokens + kTileT - 1) / kTileT;
+    for (int dt = EQ_INT8; dt <= EQ_E4M3; ++dt) {
+        std::vector<uint32_t> order;
+        for (uint32_t i = 0; i < n; ++i) {
+            const eq_matrix_info &in = m->mats[req[i].matrix].info;
+            if (in.dtype == dt && in.rows && in.cols) order.push_back(i);
+        }
+        std::stable_sort(order.begin(), order.end(), [&](uint32_t a, uint32_t b) {
+            return m->mats[req[a].matrix].info.cols > m->mats[req[b].matrix].info.cols;
+        });
+        auto fn = dt == EQ_INT8 ? eq_gemm_symbols_kernel<EQ_INT8> : eq_gemm_symbols_kernel<EQ_E4M3>;
+        for (size_t at = 0; at < order.size(); at += kMaxGemmJobs) {
+            GemmParams P{};
+            P.status = d_status;
+            P.tokens = tokens;
+            P.t_tiles = t_tiles;
+            uint64_t tiles = 0;
+            for (size_t k = at; k < order.size() && k < at + kMaxGemmJobs; ++k) {
+                const GemmRequest &q = req[order[k]];
+                const MatrixDesc &d = m->mats[q.matrix];
+                GemmJob &J = P.jobs[P.n_jobs++];
+                if (const int rc = encode_token_map(&J.tmap_x, q.x, tokens, d.info.cols)) return rc;
+                J.sym = static_cast<const uint8_t *>(q.sym);
+                J.scales = reinterpret_cast<const float *>(m->d_blob + d.scales_off);
+                J.y = q.y;
+                J.rows = d.info.rows;
+                J.cols = d.info.cols;
+                J.first_tile = (uint32_t)tiles;
+                tiles += (uint64_t)(d.info.rows / kTileN) * t_tiles;
+            }
+            if (tiles > 0xFFFFFFFFull - (uint64_t)sms) return EQ_ERR_UNSUPPORTED;
+            P.total_tiles = (uint32_t)tiles;
+            bool &attr = g_gemm_attr_set[dev][dt - 1];
+            if (!attr) {
+                if (cudaFuncSetAttribute(reinterpret_cast<const void *>(fn),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem) != cudaSuccess)
+                    return EQ_ERR_CUDA;
+                attr = true;
+            }
+            const uint32_t grid = std::min<uint64_t>(tiles, (uint64_t)sms);
+            fn<<<grid, kGemmThreads + 32, kGemmSmem, s>>>(P);
+            if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
+        }
+    }
+    for (uint32_t i = 0; i < n; ++i) {
+        const MatrixDesc &d = m->mats[req[i].matrix];
+        const eq_matrix_info &in = d.info;
+        if (!in.n_outliers || !in.rows || !in.cols) continue;
+        const uint64_t cnt = (uint64_t)in.n_outliers * tokens;
+        eq_gemm_outliers_kernel<<<(unsigned)((cnt + 255) / 256), 256, 0, s>>>(
+            reinterpret_cast<const uint32_t *>(m->d_blob + d.outliers_off), in.n_outliers,
+            static_cast<const uint16_t *>(req[i].x), tokens, in.rows, in.cols, req[i].y, d_status);
+        if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
+    }
+    return EQ_OK;
 }
 
 }  // namespace
@@ -718,54 +587,20 @@ int encode_token_map(CUtensorMap *map, const void *x, uint32_t tokens, uint32_t 
 extern "C" EQW_API int eq_gemm_symbols(const eq_model *m, uint32_t matrix, const void *d_sym, const void *d_x,
                                        uint32_t tokens, float *d_y, int32_t *d_status, cudaStream_t s) {
     const eqw::NvtxScope nvtx_range("eq_gemm_symbols");
-    if (!m || !d_status || matrix >= m->mats.size()) return EQ_ERR_INVALID_ARG;
-    const MatrixDesc &d = m->mats[matrix];
-    const eq_matrix_info &in = d.info;
-    if (!tokens || !in.rows || !in.cols) return EQ_OK;
-    if (in.rows % kTileN || in.cols % kTileK || in.rows / kTileN > 65535u) return EQ_ERR_UNSUPPORTED;
-    if (!d_sym || !d_x || !d_y) return EQ_ERR_INVALID_ARG;
-    if (reinterpret_cast<uintptr_t>(d_sym) % 16 || reinterpret_cast<uintptr_t>(d_x) % 16 ||
-        reinterpret_cast<uintptr_t>(d_y) % 16 || d.scales_off % 16)
-        return EQ_ERR_INVALID_ARG;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return EQ_ERR_CUDA;
-    GemmParams P{};
-    if (const int rc = encode_token_map(&P.tmap_x, d_x, tokens, in.cols)) return rc;
-    P.x = static_cast<const uint16_t *>(d_x);
-    P.sym = static_cast<const uint8_t *>(d_sym);
-    P.scales = reinterpret_cast<const float *>(m->d_blob + d.scales_off);
-    P.y = d_y;
-    P.status = d_status;
-    P.tokens = tokens;
-    P.rows = in.rows;
-    P.cols = in.cols;
-    P.dtype = in.dtype;
-#if EQ_GEMM_TMEM_A
-    auto fn = in.dtype == EQ_INT8 ? eq_gemm_tm_kernel<EQ_INT8> : eq_gemm_tm_kernel<EQ_E4M3>;
-    const size_t smem = kTmSmem;
-    const dim3 grid((tokens + kTmTileT - 1) / kTmTileT, in.rows / kTmTileN);
-#else
-    auto fn = in.dtype == EQ_INT8 ? eq_gemm_symbols_kernel<EQ_INT8> : eq_gemm_symbols_kernel<EQ_E4M3>;
-    const size_t smem = kGemmSmem;
-    const dim3 grid((tokens + kTileM - 1) / kTileM, in.rows / kTileN);
-#endif
-    bool &attr = g_gemm_attr_set[dev][in.dtype - 1];
-    if (!attr) {
-        if (cudaFuncSetAttribute(reinterpret_cast<const void *>(fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem) != cudaSuccess)
-            return EQ_ERR_CUDA;
-        attr = true;
-    }
-    fn<<<grid, kGemmThreads + 32, smem, s>>>(P);
-    if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
-    if (in.n_outliers) {
-        const uint64_t n = (uint64_t)in.n_outliers * tokens;
-        eq_gemm_outliers_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
-            reinterpret_cast<const uint32_t *>(m->d_blob + d.outliers_off), in.n_outliers,
-            static_cast<const uint16_t *>(d_x), tokens, in.rows, in.cols, d_y, d_status);
-        if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
-    }
-    return EQ_OK;
+    const GemmRequest q{matrix, d_sym, d_x, d_y};
+    return gemm_launch(m, &q, 1, tokens, d_status, s);
+}
+
+extern "C" EQW_API int eq_gemm_symbols_block(const eq_model *m, uint32_t layer, const void *const *d_syms,
+                                             const void *const *d_xs, uint32_t tokens, float *const *d_ys,
+                                             uint32_t count, int32_t *d_status, cudaStream_t s) {
+    const eqw::NvtxScope nvtx_range("eq_gemm_symbols_block");
+    if (!m || layer >= m->n_layers) return EQ_ERR_INVALID_ARG;
+    const uint32_t first = m->layer_first[layer], n = m->layer_count[layer];
+    if (count != n || (n && (!d_syms || !d_xs || !d_ys))) return EQ_ERR_INVALID_ARG;
+    std::vector<GemmRequest> req(n);
+    for (uint32_t i = 0; i < n; ++i) req[i] = GemmRequest{first + i, d_syms[i], d_xs[i], d_ys[i]};
+    return gemm_launch(m, req.data(), n, tokens, d_status, s);
 }
 
 extern "C" EQW_API int eq_selftest_gemm_wait_timeout(int32_t *d_status, cudaStream_t s) {

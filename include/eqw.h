@@ -241,8 +241,9 @@ EQW_API int eq_model_open(const void *d_blob, size_t len, const void *h_blob, eq
 EQW_API void eq_model_close(eq_model *m);
 
 /*
- * Let this model's decode launches (eq_decode_*, eq_decode_gemv_*) use at
- * most `max_sms` SMs (0: all, the default).  The decode kernels keep one
+ * Let this model's decode launches (eq_decode_*, eq_decode_gemv_*) and its
+ * prefill GEMMs (eq_gemm_symbols*) use at most `max_sms` SMs (0: all, the
+ * default).  The decode kernels keep one
  * block per SM for the whole launch, so a kernel that must run beside them
  * -- the consumer of the previous block in a streamed forward pass -- only
  * gets SMs they leave free.  Host-side setting; takes effect for launches
@@ -390,6 +391,17 @@ EQW_API int eq_decode_symbols_block(const eq_model *m, uint32_t layer, void *con
  */
 EQW_API int eq_gemm_symbols(const eq_model *m, uint32_t matrix, const void *d_sym, const void *d_x, uint32_t tokens,
                             float *d_y, int32_t *d_status, cudaStream_t s);
+
+/* The same for every matrix of `layer`, one persistent launch per weight type
+ * (the tiles of all the layer's matrices shared out over the SMs, so that a
+ * small matrix does not leave SMs idle): d_syms[i], d_xs[i], d_ys[i] (host
+ * arrays of `count` device pointers, count = the layer's matrix count) belong
+ * to matrix i of the layer in directory order; all take `tokens` tokens.  Each
+ * matrix has the requirements of eq_gemm_symbols; nothing is launched when one
+ * fails them (EQ_ERR_UNSUPPORTED / EQ_ERR_INVALID_ARG). */
+EQW_API int eq_gemm_symbols_block(const eq_model *m, uint32_t layer, const void *const *d_syms,
+                                  const void *const *d_xs, uint32_t tokens, float *const *d_ys, uint32_t count,
+                                  int32_t *d_status, cudaStream_t s);
 
 /* ---- failure detection ----------------------------------------------------------
  * Check of the decode kernels' timeout path: one warp runs the decoder's own

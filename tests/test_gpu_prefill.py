@@ -175,3 +175,111 @@ def test_decode_symbols_block_bit_exact(eqw, orc):
     for m, o in zip(mats, outs):
         assert np.array_equal(o.cpu().numpy().reshape(m.rows, m.cols), orc.stream_symbols(m))
     model.close()
+
+
+def _one_hot(seed, tokens, cols):
+    rng = np.random.default_rng(seed)
+    x = torch.zeros(tokens, cols, dtype=torch.bfloat16)
+    x[torch.arange(tokens), torch.from_numpy(rng.integers(0, cols, size=tokens))] = torch.from_numpy(
+        rng.choice([-2.0, -0.5, 1.0, 3.0], size=tokens).astype(np.float32)).to(torch.bfloat16)
+    return x
+
+
+def _block_mats():
+    """Both weight types, K from 64 to 1024, super weights, in one layer."""
+    return [W.random_int8_matrix(30, 256, 512, n_out=8, layer=0, index=0),
+            W.random_e4m3_matrix(31, 128, 192, alpha=1.0, layer=0, index=1),
+            W.random_int8_matrix(32, 384, 64, layer=0, index=2),
+            W.random_int8_matrix(33, 128, 1024, h_bits=4.0, layer=0, index=3),
+            W.random_e4m3_matrix(34, 256, 256, alpha=1.0, layer=0, index=4)]
+
+
+@pytest.mark.parametrize("sms", [0, 1, 3])
+def test_gemm_block_one_hot_bit_exact(eqw, orc, sms):
+    """One persistent launch per weight type over every tile of the layer; sms = 1 or 3 makes each
+    CTA run many tiles of different matrices (stage ring and barrier phases carried across tiles)."""
+    mats = _block_mats()
+    tokens = 700                                     # 3 token tiles, the last one ragged
+    model = _open(eqw, mats)
+    model.set_sm_limit(sms)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    syms = [torch.empty(m.rows * m.cols, dtype=torch.uint8, device="cuda") for m in mats]
+    model.decode_symbols_block(0, syms, status)
+    xs = [_one_hot(40 + i, tokens, m.cols) for i, m in enumerate(mats)]
+    ys = [torch.full((tokens, m.rows), float("nan"), dtype=torch.float32, device="cuda") for m in mats]
+    model.gemm_symbols_block(0, syms, [x.cuda() for x in xs], ys, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for i, (m, x, y) in enumerate(zip(mats, xs, ys)):
+        ref, _ = orc.gemm_symbols_exact(m, _bits(x))
+        assert np.array_equal(y.cpu().numpy().view(np.uint32), ref.astype(np.float32).view(np.uint32)), i
+    model.close()
+
+
+def test_gemm_block_random_tokens_within_bound(eqw, orc):
+    mats = _block_mats()
+    tokens = 300
+    model = _open(eqw, mats)
+    model.set_sm_limit(2)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    syms = [torch.empty(m.rows * m.cols, dtype=torch.uint8, device="cuda") for m in mats]
+    model.decode_symbols_block(0, syms, status)
+    xs = [W.gemv_activation(9, i, tokens * m.cols).reshape(tokens, m.cols) for i, m in enumerate(mats)]
+    ys = [torch.empty(tokens, m.rows, dtype=torch.float32, device="cuda") for m in mats]
+    model.gemm_symbols_block(0, syms, [x.cuda() for x in xs], ys, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for m, x, y in zip(mats, xs, ys):
+        ref, mag = orc.gemm_symbols_exact(m, _bits(x))
+        _check_bound(y.cpu().numpy(), ref, mag, m.cols)
+    model.close()
+
+
+def test_gemm_block_llama70b_layer_sampled_rows(eqw, orc):
+    """A full 70B-shape layer (7 matrices, 1312 tiles at 512 tokens) in one launch: every output equals
+    the single-matrix launch's bit for bit (same tile arithmetic), and sampled weight rows of every
+    matrix are within the fp32 bound of the oracle."""
+    mats = W.llama70b_int8_layer(0)
+    tokens = 512
+    model = _open(eqw, mats)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    syms = [torch.empty(m.rows * m.cols, dtype=torch.uint8, device="cuda") for m in mats]
+    model.decode_symbols_block(0, syms, status)
+    xs = [W.gemv_activation(11, i, tokens * m.cols).reshape(tokens, m.cols) for i, m in enumerate(mats)]
+    xd = [x.cuda() for x in xs]
+    ys = [torch.empty(tokens, m.rows, dtype=torch.float32, device="cuda") for m in mats]
+    model.gemm_symbols_block(0, syms, xd, ys, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rng = np.random.default_rng(12)
+    for i, (m, x, y) in enumerate(zip(mats, xs, ys)):
+        y1 = torch.empty_like(y)
+        model.gemm_symbols(i, syms[i], xd[i], y1, status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert torch.equal(y.view(torch.int32), y1.view(torch.int32)), i
+        rows = np.sort(rng.choice(m.rows, size=64, replace=False))
+        sub = W.Matrix(m.layer, m.index, m.name, m.dtype, m.symbols[rows], m.scales[rows])
+        ref, mag = orc.gemm_symbols_exact(sub, _bits(x))
+        _check_bound(y.cpu().numpy()[:, rows], ref, mag, m.cols)
+    model.close()
+
+
+def test_gemm_block_argument_errors(eqw):
+    mats = _block_mats()
+    model = _open(eqw, mats)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    syms = [torch.empty(m.rows * m.cols, dtype=torch.uint8, device="cuda") for m in mats]
+    xs = [torch.zeros(4, m.cols, dtype=torch.bfloat16, device="cuda") for m in mats]
+    ys = [torch.zeros(4, m.rows, dtype=torch.float32, device="cuda") for m in mats]
+    with pytest.raises(ValueError):
+        model.gemm_symbols_block(0, syms[:-1], xs, ys, status)
+    with pytest.raises(eqw.EqError):                 # count != the layer's matrix count
+        model.gemm_symbols_block(0, syms[:-1], xs[:-1], ys[:-1], status)
+    bad = list(ys)
+    bad[2] = torch.zeros(4 * mats[2].rows + 1, dtype=torch.float32, device="cuda")[1:].view(4, mats[2].rows)
+    with pytest.raises(eqw.EqError):                 # y not 16-byte aligned: nothing launched
+        model.gemm_symbols_block(0, syms, xs, bad, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    model.close()
