@@ -17,36 +17,39 @@
 // Kernel eq_gemm_symbols_kernel: a persistent launch (one CTA per SM) over the
 // 128-row x 256-token output tiles of up to 8 matrices of one weight type (a
 // transformer block's projections in one launch; the matrix with the longest
-// K first, CTA b taking tiles b, b + grid, ...), 8 producer warps and one MMA
-// warp per CTA.  The MMA is M = 128 weight rows (A, read
-// from tensor memory) x N = 256 tokens (B, in shared memory) x K 16, with the
-// fp32 accumulator in tensor memory (128 lanes x 256 columns: lane = weight
-// row, column = token).  Per K slab of 64:
-//   producers  thread (w, l) owns weight row 32 (w % 4) + l and half w / 4 of
-//              the slab's 64 columns: it loads its 32 symbol bytes straight
-//              into registers (one slab ahead), widens them exactly to bf16
-//              and stores them with tcgen05.st into its own tensor-memory lane,
-//              in the stage's 16 columns of that half (two bf16 per 32-bit
-//              column, the lower K index in the low half); thread 0 also issues
-//              the token tile's two TMA tensor copies (128 tokens each, 128-byte
-//              swizzle: the K-major layout the MMA's B descriptor reads, 16-byte
-//              chunk c of row r at chunk position c ^ (r % 8), 8-row groups
-//              1024 B apart); each warp then arrives on the stage's "full"
-//              mbarrier (which also waits for the tensor copy's bytes); a
-//              stage is refilled only after its "empty" barrier says the tensor
-//              core is done with it
-//   MMA warp   one lane waits for "full", issues the slab's 4 MMAs and
-//              tcgen05.commits them to the stage's "empty" barrier; a last
-//              commit to "done" releases the epilogue
-//   epilogue   thread (w, l) reads its weight row's 128 accumulator columns of
-//              half w / 4 (tcgen05.ld), multiplies by the row's scale and stores
-//              them one token column at a time (a warp's 32 lanes write 32
-//              consecutive outputs of one token)
-// Between tiles the MMA warp waits on "acc_free" (every producer warp has read
-// its part of the accumulator) before the next tile's first MMA; the stage
-// ring and its barrier phases run on across tiles.
-// Shared memory per slab: the token tile written once and read once by the
-// MMAs, 32 KB; the widened weights never touch it.
+// K first, CTA b taking tiles b, b + grid, ...).  The MMA is M = 128 weight
+// rows (A, read from tensor memory) x N = 256 tokens (B, in shared memory) x
+// K 16, with the fp32 accumulator in tensor memory (128 lanes x 256 columns:
+// lane = weight row, column = token).  Three roles per CTA, over a ring of 5
+// stages (one K slab of 64 each):
+//   loader     one lane of warp 9: for each slab, once the stage's "empty"
+//              barrier says the tensor core is done with it, arms the stage's
+//              "load" barrier and issues three TMA tensor copies: the token
+//              tile (two boxes of 128 tokens x 64 bf16, 128-byte swizzle: the
+//              K-major layout the MMA's B descriptor reads, 16-byte chunk c of
+//              row r at chunk c ^ (r % 8), 8-row groups 1024 B apart) and the
+//              symbol tile (128 rows x 64 bytes, 64-byte swizzle)
+//   producers  warps 0-7; thread (w, l) owns weight row 32 (w % 4) + l and
+//              half w / 4 of the slab's 64 columns: after "load" it reads its
+//              32 symbol bytes from the symbol tile (conflict-free thanks to
+//              the swizzle), widens them exactly to bf16 and stores them with
+//              tcgen05.st into its own tensor-memory lane, in the stage's 16
+//              columns of that half (two bf16 per 32-bit column, the lower K
+//              index in the low half); the warp arrives on the stage's "full"
+//              barrier once the store has completed (checked one slab later,
+//              so that the store's latency overlaps the next slab's work)
+//   MMA warp   one lane waits for "full" (and "load"), issues the slab's 4
+//              MMAs and tcgen05.commits them to the stage's "empty" barrier; a
+//              commit to "done" after a tile's last slab releases the epilogue
+//   epilogue   the producers: thread (w, l) reads its weight row's 128
+//              accumulator columns of half w / 4 (tcgen05.ld), multiplies by
+//              the row's scale and stores them one token column at a time (a
+//              warp's 32 lanes write 32 consecutive outputs of one token), then
+//              arrives on "acc_free", which the MMA lane waits for before the
+//              next tile's first MMA; the stage ring runs on across tiles, so
+//              the loader fetches the next tile's first slabs meanwhile
+// Shared memory per stage: 32 KB token tile + 8 KB symbol tile; the widened
+// weights never touch it.
 // Every mbarrier wait is bounded; on expiry the CTA records EQ_DEV_TIMEOUT,
 // still releases its tensor memory and stops.
 #include <cuda.h>
@@ -62,7 +65,8 @@
 
 namespace {
 
-constexpr int kGemmThreads = 256;                      // 8 producer warps (two per tensor-memory lane quarter)
+constexpr uint32_t kProducerWarps = 8;                 // two per tensor-memory lane quarter
+constexpr int kGemmThreads = (kProducerWarps + 2) * 32; // + the MMA warp and the loader warp
 constexpr uint32_t kTileN = 128;                       // weight rows per CTA (MMA M, accumulator lanes)
 constexpr uint32_t kTileT = 256;                       // tokens per CTA (MMA N, accumulator columns)
 constexpr uint32_t kTileK = 64;                        // K per slab (128-byte rows: the 128-byte swizzle)
@@ -70,13 +74,16 @@ constexpr uint32_t kBoxT = 128;                        // tokens per TMA box
 constexpr uint32_t kRowBytes = kTileK * 2;             // one bf16 token row of a slab = one swizzle row
 constexpr uint32_t kAtomBytes = 8 * kRowBytes;         // 8-row swizzle atom (SBO)
 constexpr uint32_t kMmaK = 16;                         // K per tcgen05.mma (bf16)
-constexpr uint32_t kStages = 4;
-constexpr uint32_t kStageBytes = kTileT * kTileK * 2;  // 32 KB token tile per stage
+constexpr uint32_t kStages = 5;
+constexpr uint32_t kXBytes = kTileT * kTileK * 2;      // token tile of a stage, 32 KB
+constexpr uint32_t kWBytes = kTileN * kTileK;          // symbol tile of a stage, 8 KB
+constexpr uint32_t kStageBytes = kXBytes + kWBytes;    // both land on the stage's "load" barrier
 constexpr uint32_t kAccCols = kTileT;                  // fp32 accumulator columns
 constexpr uint32_t kACols = kTileK / 2;                // tensor-memory columns of one stage's weights
 constexpr uint32_t kTmemAlloc = 512;                   // accumulator + kStages weight stages, rounded up
 static_assert(kAccCols + kStages * kACols <= kTmemAlloc, "tensor memory columns");
 constexpr size_t kGemmSmem = kStages * kStageBytes + 1024;
+static_assert(kGemmSmem <= 227u * 1024u, "shared memory per block");
 
 constexpr uint32_t kMaxGemmJobs = 8;  // matrices per launch (a transformer block has 7)
 
@@ -84,6 +91,7 @@ constexpr uint32_t kMaxGemmJobs = 8;  // matrices per launch (a transformer bloc
 // token tiles), weight-row tile major, token tile fastest.
 struct GemmJob {
     CUtensorMap tmap_x;       // bf16 [tokens, cols] input of this matrix, box kTileK x kBoxT, 128-byte swizzle
+    CUtensorMap tmap_w;       // uint8 [rows, cols] symbols, box kTileK x kTileN, 64-byte swizzle
     const uint8_t *sym;       // [rows, cols]
     const float *scales;      // [rows]
     float *y;                 // [tokens, rows]
@@ -227,25 +235,30 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
-    uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-    return v;
+// 32 symbol bytes of weight row `row`, half `half` of a slab, from the slab's
+// 64-byte-swizzled symbol tile (16-byte chunk c of row r stored at chunk
+// c ^ ((r >> 1) & 3) of the row): the 32 lanes of a warp (32 consecutive rows)
+// then read 8 distinct 16-byte bank groups per 128 bytes, no conflicts.
+__device__ __forceinline__ void lds_sym32(uint32_t tile, uint32_t row, uint32_t half, uint4 &a, uint4 &b) {
+    const uint32_t base = tile + row * kTileK, x = (row >> 1) & 3u;
+    const uint32_t pa = base + (((2u * half) ^ x) << 4), pb = base + (((2u * half + 1u) ^ x) << 4);
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w) : "r"(pa)
+                 : "memory");
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w) : "r"(pb)
+                 : "memory");
 }
 
 template <int DT>
-__global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(const __grid_constant__ GemmParams P) {
-    constexpr uint32_t kProducerWarps = kGemmThreads / 32;
-    static_assert(kProducerWarps == 8, "two producer warps per tensor-memory lane quarter");
+__global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const __grid_constant__ GemmParams P) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t full_s[kStages], empty_s[kStages], done_s, acc_free_s;
+    __shared__ __align__(8) uint64_t load_s[kStages], full_s[kStages], empty_s[kStages], done_s, acc_free_s;
     __shared__ uint32_t tmem_base_s;
-    __shared__ volatile uint32_t abort_s;  // a bounded wait gave up: every loop stops
+    __shared__ volatile uint32_t abort_s;  // a bounded wait gave up: every role stops
     const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
-    const bool mma_warp = warp == kProducerWarps;
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    auto bufB = [&](uint32_t st) { return base + st * kStageBytes; };
-    const uint32_t full0 = smem_u32(&full_s[0]), empty0 = smem_u32(&empty_s[0]);
+    auto bufB = [&](uint32_t st) { return base + st * kStageBytes; };            // token tile
+    auto bufW = [&](uint32_t st) { return base + st * kStageBytes + kXBytes; };  // symbol tile
+    const uint32_t load0 = smem_u32(&load_s[0]), full0 = smem_u32(&full_s[0]), empty0 = smem_u32(&empty_s[0]);
     const uint32_t done = smem_u32(&done_s), acc_free = smem_u32(&acc_free_s);
 
     if (warp == 0) {
@@ -255,8 +268,9 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
     }
     if (tid == 0) {
         for (uint32_t st = 0; st < kStages; ++st) {
-            mbar_init(full0 + 8 * st, kProducerWarps + 1u);  // + the token tile's expect_tx arrival
-            mbar_init(empty0 + 8 * st, 1);
+            mbar_init(load0 + 8 * st, 1);              // the loader's expect_tx arrival + the copies' bytes
+            mbar_init(full0 + 8 * st, kProducerWarps);  // every producer warp has stored its weights
+            mbar_init(empty0 + 8 * st, 1);             // tcgen05.commit of the stage's MMAs
         }
         mbar_init(done, 1);
         mbar_init(acc_free, kProducerWarps);  // every producer warp has read its accumulator part
@@ -266,80 +280,58 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = tmem_base_s;                 // lane 0, first allocated column
-    const uint32_t tmem_a = tmem + kAccCols;           // weight stages follow the accumulator
-    const uint32_t quarter = warp & 3u, half = warp >> 2;
-    const uint32_t lane_base = (quarter * 32u) << 16;
+    const uint32_t tmem = tmem_base_s;        // lane 0, first allocated column
+    const uint32_t tmem_a = tmem + kAccCols;  // weight stages follow the accumulator
     bool ok = true;
     uint32_t g = 0;  // slabs so far in this CTA: stage g % kStages, phase g / kStages
 
-    // persistent loop over the launch's tiles, longest matrices (most slabs) first
-    uint32_t ti = 0;
-    uint32_t jb = 0;
-    for (uint32_t tile = blockIdx.x; tile < P.total_tiles; tile += gridDim.x, ++ti) {
-        while (jb + 1 < P.n_jobs && tile >= P.jobs[jb + 1].first_tile) ++jb;
-        const GemmJob &J = P.jobs[jb];
-        const uint32_t local = tile - J.first_tile;
-        const uint32_t n0 = (local / P.t_tiles) * kTileN;  // weight rows
-        const uint32_t m0 = (local % P.t_tiles) * kTileT;  // tokens
-        const uint32_t n_slabs = J.cols / kTileK;
-
-        if (!mma_warp) {
-            if (__any_sync(0xFFFFFFFFu, abort_s != 0u)) break;  // another warp's wait gave up
-            const uint8_t *src = J.sym + (size_t)(n0 + quarter * 32u + lane) * J.cols + half * 32u;
-            uint4 cur0 = ldg_nc_v4(src), cur1 = ldg_nc_v4(src + 16);
+    if (warp < kProducerWarps) {
+        // ---- producers: symbols (shared) -> bf16 -> tensor memory; the tile's epilogue ----
+        const uint32_t quarter = warp & 3u, half = warp >> 2;
+        const uint32_t row = quarter * 32u + lane;  // weight row within the tile = tensor-memory lane
+        const uint32_t lane_base = (quarter * 32u) << 16;
+        uint32_t ti = 0, jb = 0;
+        for (uint32_t tile = blockIdx.x; tile < P.total_tiles; tile += gridDim.x, ++ti) {
+            if (__any_sync(0xFFFFFFFFu, abort_s != 0u)) break;
+            while (jb + 1 < P.n_jobs && tile >= P.jobs[jb + 1].first_tile) ++jb;
+            const GemmJob &J = P.jobs[jb];
+            const uint32_t local = tile - J.first_tile;
+            const uint32_t n0 = (local / P.t_tiles) * kTileN, m0 = (local % P.t_tiles) * kTileT;
+            const uint32_t n_slabs = J.cols / kTileK;
             for (uint32_t it = 0; it < n_slabs; ++it, ++g) {
                 const uint32_t s = g % kStages;
-                uint4 nx0 = cur0, nx1 = cur1;
-                if (it + 1 < n_slabs) {  // next slab's symbols, one slab ahead
-                    nx0 = ldg_nc_v4(src + (size_t)(it + 1) * kTileK);
-                    nx1 = ldg_nc_v4(src + (size_t)(it + 1) * kTileK + 16);
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(load0 + 8 * s, (g / kStages) & 1u))) {
+                    ok = false;
+                    break;
                 }
-                // stage s last held slab g - kStages: wait until its MMAs are done
-                if (g >= kStages) {
-                    if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(empty0 + 8 * s, ((g - kStages) / kStages) & 1u))) {
-                        ok = false;
-                        abort_s = 1;
-                        break;
-                    }
-                    tc_fence_after();
-                }
-                if (tid == 0) {
-                    // token tile: two TMA tensor copies of 128 tokens (x = k0, a multiple of
-                    // 64 elements; rows past the last token read as zeros)
-                    mbar_expect_tx(full0 + 8 * s, kStageBytes);
-#pragma unroll
-                    for (uint32_t h = 0; h < 2; ++h)
-                        asm volatile(
-                            "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-                            " [%0], [%1, {%2, %3}], [%4];" ::"r"(bufB(s) + h * kBoxT * kRowBytes),
-                            "l"(reinterpret_cast<uint64_t>(&J.tmap_x)), "r"(it * kTileK), "r"(m0 + h * kBoxT),
-                            "r"(full0 + 8 * s)
-                            : "memory");
-                }
-                // this row's 32 symbols of the slab, widened exactly, into its tensor-memory lane
-                uint4 lo0, hi0, lo1, hi1;
-                widen16<DT>(cur0, lo0, hi0);
-                widen16<DT>(cur1, lo1, hi1);
+                tc_fence_after();
+                uint4 a, b, lo0, hi0, lo1, hi1;
+                lds_sym32(bufW(s), row, half, a, b);
+                widen16<DT>(a, lo0, hi0);
+                widen16<DT>(b, lo1, hi1);
                 const uint32_t v[16] = {lo0.x, lo0.y, lo0.z, lo0.w, hi0.x, hi0.y, hi0.z, hi0.w,
                                         lo1.x, lo1.y, lo1.z, lo1.w, hi1.x, hi1.y, hi1.z, hi1.w};
+                // the previous slab's tensor-memory store has had this slab's work to complete
+                if (it > 0) {
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(full0 + 8 * ((g - 1) % kStages));
+                }
                 tmem_st16(tmem_a + lane_base + s * kACols + half * (kACols / 2), v);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(full0 + 8 * s);
-                cur0 = nx0;
-                cur1 = nx1;
             }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
             if (!ok) break;
-            // epilogue of this tile: thread (w, l) holds weight row 32 (w % 4) + l, tokens 128 (w / 4) ..
+            if (lane == 0) mbar_arrive(full0 + 8 * ((g - 1) % kStages));
+            // epilogue: thread (w, l) holds weight row 32 (w % 4) + l, tokens 128 (w / 4) .. + 127
             if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(done, ti & 1u))) {
                 ok = false;
-                abort_s = 1;
                 break;
             }
             tc_fence_after();
-            const uint32_t r = n0 + quarter * 32u + lane;
+            const uint32_t r = n0 + row;
             const float sc = __ldg(J.scales + r);
 #pragma unroll 1
             for (uint32_t c = 0; c < kAccCols / 2; c += 32) {
@@ -353,19 +345,25 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(acc_free);  // the MMA warp may overwrite the accumulator
-        } else if (lane == 0) {
+        }
+    } else if (warp == kProducerWarps && lane == 0) {
+        // ---- MMA issuer ----
+        uint32_t ti = 0, n_done = 0;
+        for (uint32_t tile = blockIdx.x, jb = 0; tile < P.total_tiles; tile += gridDim.x, ++ti) {
+            while (jb + 1 < P.n_jobs && tile >= P.jobs[jb + 1].first_tile) ++jb;
+            const uint32_t n_slabs = P.jobs[jb].cols / kTileK;
             // the previous tile's epilogue must have read the accumulator
             if (abort_s || (ti > 0 && !mbar_wait_bounded(acc_free, (ti - 1) & 1u))) {
                 ok = false;
-                abort_s = 1;
                 break;
             }
             tc_fence_after();
             for (uint32_t it = 0; it < n_slabs; ++it, ++g) {
                 const uint32_t s = g % kStages;
-                if (abort_s || !mbar_wait_bounded(full0 + 8 * s, (g / kStages) & 1u)) {
+                // the producers' weights, and the token tile the loader's copy brought in
+                if (abort_s || !mbar_wait_bounded(full0 + 8 * s, (g / kStages) & 1u) ||
+                    !mbar_wait_bounded(load0 + 8 * s, (g / kStages) & 1u)) {
                     ok = false;
-                    abort_s = 1;
                     break;
                 }
                 tc_fence_after();
@@ -375,12 +373,54 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
                 tc_commit(empty0 + 8 * s);
             }
             tc_commit(done);  // completes when every MMA issued above has
+            ++n_done;
             if (!ok) break;
-        } else {
-            g += n_slabs;  // lanes 1..31 of the MMA warp only keep count
         }
+        // no MMA may still be running when the tensor memory is released
+        if (n_done > 0 && !mbar_wait_bounded(done, (n_done - 1) & 1u)) ok = false;
+    } else if (warp == kProducerWarps + 1 && lane == 0) {
+        // ---- loader: the token tile and the symbol tile of every slab, kStages ahead ----
+        for (uint32_t tile = blockIdx.x, jb = 0; tile < P.total_tiles && ok; tile += gridDim.x) {
+            while (jb + 1 < P.n_jobs && tile >= P.jobs[jb + 1].first_tile) ++jb;
+            const GemmJob &J = P.jobs[jb];
+            const uint32_t local = tile - J.first_tile;
+            const uint32_t n0 = (local / P.t_tiles) * kTileN, m0 = (local % P.t_tiles) * kTileT;
+            const uint32_t n_slabs = J.cols / kTileK;
+            const uint64_t map_x = reinterpret_cast<uint64_t>(&J.tmap_x);
+            const uint64_t map_w = reinterpret_cast<uint64_t>(&J.tmap_w);
+            for (uint32_t it = 0; it < n_slabs; ++it, ++g) {
+                const uint32_t s = g % kStages;
+                // stage s last held slab g - kStages: its MMAs (and so its producers) are done
+                if (g >= kStages && (abort_s || !mbar_wait_bounded(empty0 + 8 * s, ((g - kStages) / kStages) & 1u))) {
+                    ok = false;
+                    break;
+                }
+                mbar_expect_tx(load0 + 8 * s, kStageBytes);
+                // token tile: two boxes of 128 tokens (x = k0, a multiple of 64 elements; rows past
+                // the last token read as zeros); symbol tile: 128 rows x 64 bytes (x = k0 bytes)
+#pragma unroll
+                for (uint32_t h = 0; h < 2; ++h)
+                    asm volatile(
+                        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                        " [%0], [%1, {%2, %3}], [%4];" ::"r"(bufB(s) + h * kBoxT * kRowBytes),
+                        "l"(map_x), "r"(it * kTileK), "r"(m0 + h * kBoxT), "r"(load0 + 8 * s)
+                        : "memory");
+                asm volatile(
+                    "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                    " [%0], [%1, {%2, %3}], [%4];" ::"r"(bufW(s)), "l"(map_w), "r"(it * kTileK), "r"(n0),
+                    "r"(load0 + 8 * s)
+                    : "memory");
+            }
+        }
+        // no copy may still be writing shared memory when the block exits: wait (bounded) for
+        // the last copy issued to each stage; at normal exit they have all been consumed already
+        for (uint32_t k = g > kStages ? g - kStages : 0; k < g; ++k)
+            if (!mbar_wait_bounded(load0 + 8 * (k % kStages), (k / kStages) & 1u)) ok = false;
     }
-    if (!ok) atomicOr(P.status, EQ_DEV_TIMEOUT);
+    if (!ok) {
+        abort_s = 1;
+        atomicOr(P.status, EQ_DEV_TIMEOUT);
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -391,17 +431,17 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_symbols_kernel(c
 }
 
 // Failure-path check of the GEMM's waits: the GEMM's own set-up (TMEM
-// allocation, "full" / "empty" / "done" barriers with its arrival counts) and
-// exit path (status flag, TMEM release), but no producer ever arrives on
-// "full", so the MMA lane's bounded wait must give up; it then arrives on
-// "done" itself, the producers pass it (or give up on it) and the block
-// returns with EQ_DEV_TIMEOUT set and its TMEM freed.
-__global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_wait_timeout_kernel(int32_t *status) {
-    constexpr uint32_t kProducerWarps = kGemmThreads / 32;
-    __shared__ __align__(8) uint64_t full_s[kStages], empty_s[kStages], done_s;
+// allocation, "load" / "full" / "empty" / "done" barriers with their arrival
+// counts, the GEMM's block size) and exit path (status flag, TMEM release),
+// but no producer ever arrives on "full", so the MMA lane's bounded wait must
+// give up; it then arrives on "done" itself, the producers pass it (or give up
+// on it) and the block returns with EQ_DEV_TIMEOUT set and its TMEM freed.
+__global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_wait_timeout_kernel(int32_t *status) {
+    __shared__ __align__(8) uint64_t load_s[kStages], full_s[kStages], empty_s[kStages], done_s;
     __shared__ uint32_t tmem_base_s;
     const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
-    const uint32_t full0 = smem_u32(&full_s[0]), empty0 = smem_u32(&empty_s[0]), done = smem_u32(&done_s);
+    const uint32_t load0 = smem_u32(&load_s[0]), full0 = smem_u32(&full_s[0]), empty0 = smem_u32(&empty_s[0]);
+    const uint32_t done = smem_u32(&done_s);
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(smem_u32(&tmem_base_s)), "r"(kTmemAlloc) : "memory");
@@ -409,7 +449,8 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_wait_timeout_ker
     }
     if (tid == 0) {
         for (uint32_t st = 0; st < kStages; ++st) {
-            mbar_init(full0 + 8 * st, kProducerWarps + 1u);
+            mbar_init(load0 + 8 * st, 1);
+            mbar_init(full0 + 8 * st, kProducerWarps);
             mbar_init(empty0 + 8 * st, 1);
         }
         mbar_init(done, 1);
@@ -425,7 +466,7 @@ __global__ void __launch_bounds__(kGemmThreads + 32, 1) eq_gemm_wait_timeout_ker
             ok = mbar_wait_bounded(full0, 0u);  // nothing arrives: gives up after the limit
             mbar_arrive(done);                  // releases the producers (synchronous: nothing left in flight)
         }
-    } else {
+    } else if (warp < kProducerWarps) {
         ok = mbar_wait_bounded(done, 0u);
     }
     if (!ok) atomicOr(status, EQ_DEV_TIMEOUT);
@@ -483,6 +524,21 @@ int encode_token_map(CUtensorMap *map, const void *x, uint32_t tokens, uint32_t 
     const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? EQ_OK : EQ_ERR_CUDA;
+}
+
+// Tensor map of a matrix's symbols: inner dimension cols, outer rows; box
+// kTileK bytes x kTileN rows with the 64-byte swizzle the producers read.
+int encode_symbol_map(CUtensorMap *map, const void *sym, uint32_t rows, uint32_t cols) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return EQ_ERR_CUDA;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols};
+    const cuuint32_t box[2] = {kTileK, kTileN};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(sym), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? EQ_OK : EQ_ERR_CUDA;
 }
@@ -547,6 +603,7 @@ int gemm_launch(const eq_model *m, const GemmRequest *req, uint32_t n, uint32_t 
                 const MatrixDesc &d = m->mats[q.matrix];
                 GemmJob &J = P.jobs[P.n_jobs++];
                 if (const int rc = encode_token_map(&J.tmap_x, q.x, tokens, d.info.cols)) return rc;
+                if (const int rc = encode_symbol_map(&J.tmap_w, q.sym, d.info.rows, d.info.cols)) return rc;
                 J.sym = static_cast<const uint8_t *>(q.sym);
                 J.scales = reinterpret_cast<const float *>(m->d_blob + d.scales_off);
                 J.y = q.y;
@@ -565,7 +622,7 @@ int gemm_launch(const eq_model *m, const GemmRequest *req, uint32_t n, uint32_t 
                 attr = true;
             }
             const uint32_t grid = std::min<uint64_t>(tiles, (uint64_t)sms);
-            fn<<<grid, kGemmThreads + 32, kGemmSmem, s>>>(P);
+            fn<<<grid, kGemmThreads, kGemmSmem, s>>>(P);
             if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
         }
     }
@@ -605,6 +662,6 @@ extern "C" EQW_API int eq_gemm_symbols_block(const eq_model *m, uint32_t layer, 
 
 extern "C" EQW_API int eq_selftest_gemm_wait_timeout(int32_t *d_status, cudaStream_t s) {
     if (!d_status) return EQ_ERR_INVALID_ARG;
-    eq_gemm_wait_timeout_kernel<<<1, kGemmThreads + 32, 0, s>>>(d_status);
+    eq_gemm_wait_timeout_kernel<<<1, kGemmThreads, 0, s>>>(d_status);
     return cudaGetLastError() == cudaSuccess ? EQ_OK : EQ_ERR_CUDA;
 }
