@@ -494,7 +494,7 @@ def bench_eqw(args, d: Dist) -> dict | None:
         del hblob
 
     # ---- E: prefill on tensor cores: symbols of layer 0 decoded once, the layer's 7 GEMMs in one ----
-    # ---- persistent launch over 1024 (and 4096) tokens                                          ----
+    # ---- persistent launch over 128, 1024 and 4096 tokens                                        ----
     prefill = None
     if d.rank == 0:
         pstep = stack.steps[0]
@@ -519,26 +519,44 @@ def bench_eqw(args, d: Dist) -> dict | None:
             return a.elapsed_time(b) / n
 
         dec_ms = p_time(lambda: pm.decode_symbols_block(pstep.layer, syms, pst, ps))
+        # comparison path: the same layer decoded to bf16 by eq_decode_block, then one library
+        # (torch / cuBLAS) bf16 matmul per matrix; context for the symbol-buffer path, not the product
+        offs, total = pm.block_layout(pstep.layer)
+        wbuf = torch.empty(total, dtype=torch.uint8, device=dev)
+        dec_bf16_ms = p_time(lambda: pm.decode_block(pstep.layer, wbuf, pst, ps))
+        wmats = [wbuf[o:o + 2 * inf.rows * inf.cols].view(torch.bfloat16).view(inf.rows, inf.cols)
+                 for o, inf in zip(offs, infos)]
         by_tokens = {}
-        for tokens in (1024, 4096):
+        for tokens in (128, 1024, 4096):
             xs_p = [W.gemv_activation(7, j, tokens * inf.cols).reshape(tokens, inf.cols).to(dev)
                     for j, inf in enumerate(infos)]
             ys_p = [torch.empty(tokens, inf.rows, dtype=torch.float32, device=dev) for inf in infos]
             gemm_ms = p_time(lambda: pm.gemm_symbols_block(pstep.layer, syms, xs_p, ys_p, pst, ps))
             flops = sum(2.0 * tokens * inf.rows * inf.cols for inf in infos)
             tflops = flops / (gemm_ms / 1e3) / 1e12
-            by_tokens[tokens] = {"gemm_ms": round(gemm_ms, 4), "tflops": round(tflops, 1),
-                                 "frac": round(tflops / bf16_peak, 4), "layer_ms": round(dec_ms + gemm_ms, 4)}
+            row = {"gemm_ms": round(gemm_ms, 4), "tflops": round(tflops, 1), "frac": round(tflops / bf16_peak, 4),
+                   "layer_ms": round(dec_ms + gemm_ms, 4)}
+            if tokens <= 1024:
+                def lib_gemm():
+                    with torch.cuda.stream(ps):
+                        for x, w in zip(xs_p, wmats):
+                            torch.matmul(x, w.t())
+                lib_ms = p_time(lib_gemm)
+                row["bf16_path"] = {"decode_ms": round(dec_bf16_ms, 4), "library_gemm_ms": round(lib_ms, 4),
+                                    "layer_ms": round(dec_bf16_ms + lib_ms, 4)}
+            by_tokens[tokens] = row
             del xs_p, ys_p
         if int(pst.item()) != 0:
             raise RuntimeError(f"prefill status {int(pst.item())}")
         prefill = {"tokens": 1024, "decode_symbols_ms": round(dec_ms, 4), **by_tokens[1024],
-                   "unit": "TFLOP/s", "bf16_peak": bf16_peak, "tokens_4096": by_tokens[4096],
-                   "kernel": "eq_gemm_symbols_kernel (tcgen05)",
+                   "unit": "TFLOP/s", "bf16_peak": bf16_peak, "tokens_128": by_tokens[128],
+                   "tokens_4096": by_tokens[4096], "kernel": "eq_gemm_symbols_kernel (tcgen05)",
                    "note": "layer 0: the 7 matrices' symbols decoded to bytes in one launch, then the 7 "
-                           "tcgen05 GEMMs in one persistent launch (eq_gemm_symbols_block) against 1024 "
-                           "bf16 tokens (fp32 out); frac of the measured cuBLAS bf16 burst peak"}
-        del syms
+                           "tcgen05 GEMMs in one persistent launch (eq_gemm_symbols_block; 256-token tiles, "
+                           "128-token tiles up to 128 tokens), bf16 tokens, fp32 out; frac of the measured "
+                           "cuBLAS bf16 burst peak.  bf16_path: the same layer decoded to bf16 by "
+                           "eq_decode_block, then one torch (cuBLAS) bf16 matmul per matrix, for comparison"}
+        del syms, wbuf, wmats
 
     # ---- C: fused decode + GEMV, no bf16 buffers; blocks in sequence on one stream ----
     fstream = torch.cuda.Stream(device=dev)

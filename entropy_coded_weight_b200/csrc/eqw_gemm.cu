@@ -66,26 +66,48 @@
 namespace {
 
 constexpr uint32_t kProducerWarps = 8;                 // two per tensor-memory lane quarter
+constexpr uint32_t kParts = kProducerWarps / 4;        // producer warps sharing a lane quarter's slab
 constexpr int kGemmThreads = (kProducerWarps + 2) * 32; // + the MMA warp and the loader warp
 constexpr uint32_t kTileN = 128;                       // weight rows per CTA (MMA M, accumulator lanes)
-constexpr uint32_t kTileT = 256;                       // tokens per CTA (MMA N, accumulator columns)
 constexpr uint32_t kTileK = 64;                        // K per slab (128-byte rows: the 128-byte swizzle)
 constexpr uint32_t kBoxT = 128;                        // tokens per TMA box
 constexpr uint32_t kRowBytes = kTileK * 2;             // one bf16 token row of a slab = one swizzle row
 constexpr uint32_t kAtomBytes = 8 * kRowBytes;         // 8-row swizzle atom (SBO)
 constexpr uint32_t kMmaK = 16;                         // K per tcgen05.mma (bf16)
-constexpr uint32_t kStages = 5;
-constexpr uint32_t kXBytes = kTileT * kTileK * 2;      // token tile of a stage, 32 KB
 constexpr uint32_t kWBytes = kTileN * kTileK;          // symbol tile of a stage, 8 KB
-constexpr uint32_t kStageBytes = kXBytes + kWBytes;    // both land on the stage's "load" barrier
-constexpr uint32_t kAccCols = kTileT;                  // fp32 accumulator columns
 constexpr uint32_t kACols = kTileK / 2;                // tensor-memory columns of one stage's weights
-constexpr uint32_t kTmemAlloc = 512;                   // accumulator + kStages weight stages, rounded up
-static_assert(kAccCols + kStages * kACols <= kTmemAlloc, "tensor memory columns");
-constexpr size_t kGemmSmem = kStages * kStageBytes + 1024;
-static_assert(kGemmSmem <= 227u * 1024u, "shared memory per block");
+constexpr uint32_t kPartBytes = kTileK / kParts;       // symbol bytes one producer thread widens per slab
+constexpr uint32_t kPartCols = kACols / kParts;        // tensor-memory columns it stores them in
+static_assert(kParts == 2 || kParts == 4, "a producer thread takes 32 or 16 bytes of its row's slab");
+constexpr uint32_t kTmemAlloc = 512;                   // accumulator + the weight stages, rounded up
 
-constexpr uint32_t kMaxGemmJobs = 8;  // matrices per launch (a transformer block has 7)
+// The token-tile width TT (MMA N) fixes the rest: 256 tokens for long inputs
+// (5 stages of 32 + 8 KB), 128 for short ones (8 stages of 16 + 8 KB: the
+// weights are then read once, and the MMA does no work on absent tokens).
+template <uint32_t TT>
+struct GemmShape {
+    static_assert(TT == 128 || TT == 256, "token tile");
+    static constexpr uint32_t kTileT = TT;                       // tokens per tile (MMA N, accumulator columns)
+    static constexpr uint32_t kStages = TT == 256 ? 5 : 8;
+    static constexpr uint32_t kXBytes = TT * kTileK * 2;         // token tile of a stage
+    static constexpr uint32_t kStageBytes = kXBytes + kWBytes;   // both land on the stage's "load" barrier
+    static constexpr uint32_t kAccCols = TT;                     // fp32 accumulator columns
+    static constexpr size_t kSmem = kStages * kStageBytes + 1024;
+    // instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
+    // K-major, N = TT tokens, M = 128 weight rows (cta_group::1 takes M = 64
+    // or 128 only)
+    static constexpr uint32_t kInstrDesc = (1u << 4)             // D format fp32
+                                         | (1u << 7)             // A format bf16
+                                         | (1u << 10)            // B format bf16
+                                         | ((TT >> 3) << 17)     // N / 8
+                                         | ((kTileN >> 4) << 24);  // M / 16
+    static_assert(kAccCols + kStages * kACols <= kTmemAlloc, "tensor memory columns");
+    static_assert(kSmem <= 227u * 1024u, "shared memory per block");
+    static_assert(kTileN == 128 && TT % 16 == 0 && TT <= 256, "cta_group::1 MMA shape");
+};
+
+constexpr uint32_t kMaxGemmJobs = 8;
+constexpr uint32_t kNarrowTokens = 128;  // inputs up to this many tokens take the 128-token tile  // matrices per launch (a transformer block has 7)
 
 // One matrix of a launch: its tiles are [first_tile, first_tile + rows / 128 *
 // token tiles), weight-row tile major, token tile fastest.
@@ -125,15 +147,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
     return d;
 }
 
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
-// K-major, N = 256 tokens, M = 128 weight rows (cta_group::1 takes M = 64 or
-// 128 only).
-constexpr uint32_t kInstrDesc = (1u << 4)                 // D format fp32
-                              | (1u << 7)                 // A format bf16
-                              | (1u << 10)                // B format bf16
-                              | ((kTileT >> 3) << 17)     // N / 8
-                              | ((kTileN >> 4) << 24);    // M / 16
-static_assert(kTileN == 128 && kTileT % 16 == 0 && kTileT <= 256, "cta_group::1 MMA shape");
 
 // Descriptor of K step kk (16 bf16) of a tile at `buf`: the start advances by
 // 32 bytes per step inside the swizzle row (the hardware applies the XOR),
@@ -214,17 +227,18 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-__device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t accumulate) {
+__device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc,
+                                          uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(tmem_d), "r"(tmem_a), "l"(db), "r"(kInstrDesc), "r"(accumulate)
+        ::"r"(tmem_d), "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
 // 16 consecutive 32-bit columns of this thread's tensor-memory lane.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *v) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
         "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
@@ -233,23 +247,33 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// 32 symbol bytes of weight row `row`, half `half` of a slab, from the slab's
-// 64-byte-swizzled symbol tile (16-byte chunk c of row r stored at chunk
-// c ^ ((r >> 1) & 3) of the row): the 32 lanes of a warp (32 consecutive rows)
-// then read 8 distinct 16-byte bank groups per 128 bytes, no conflicts.
-__device__ __forceinline__ void lds_sym32(uint32_t tile, uint32_t row, uint32_t half, uint4 &a, uint4 &b) {
-    const uint32_t base = tile + row * kTileK, x = (row >> 1) & 3u;
-    const uint32_t pa = base + (((2u * half) ^ x) << 4), pb = base + (((2u * half + 1u) ^ x) << 4);
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w) : "r"(pa)
-                 : "memory");
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w) : "r"(pb)
+// 8 consecutive 32-bit columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t *v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                 ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+                   "r"(v[7])
                  : "memory");
 }
 
-template <int DT>
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 16-byte chunk c (0..3) of weight row `row` in a slab's 64-byte-swizzled
+// symbol tile (chunk c of row r is stored at chunk c ^ ((r >> 1) & 3) of the
+// row): the 32 lanes of a warp (32 consecutive rows) reading the same c hit 8
+// distinct 16-byte bank groups per 128 bytes, no conflicts.
+__device__ __forceinline__ uint4 lds_sym16(uint32_t tile, uint32_t row, uint32_t c) {
+    const uint32_t addr = tile + row * kTileK + ((c ^ ((row >> 1) & 3u)) << 4);
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+template <int DT, uint32_t TT>
 __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const __grid_constant__ GemmParams P) {
+    using S = GemmShape<TT>;
+    constexpr uint32_t kStages = S::kStages, kStageBytes = S::kStageBytes, kXBytes = S::kXBytes;
+    constexpr uint32_t kTileT = S::kTileT, kAccCols = S::kAccCols;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t load_s[kStages], full_s[kStages], empty_s[kStages], done_s, acc_free_s;
     __shared__ uint32_t tmem_base_s;
@@ -287,7 +311,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
 
     if (warp < kProducerWarps) {
         // ---- producers: symbols (shared) -> bf16 -> tensor memory; the tile's epilogue ----
-        const uint32_t quarter = warp & 3u, half = warp >> 2;
+        const uint32_t quarter = warp & 3u, part = warp >> 2;
         const uint32_t row = quarter * 32u + lane;  // weight row within the tile = tensor-memory lane
         const uint32_t lane_base = (quarter * 32u) << 16;
         uint32_t ti = 0, jb = 0;
@@ -305,12 +329,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
                     break;
                 }
                 tc_fence_after();
-                uint4 a, b, lo0, hi0, lo1, hi1;
-                lds_sym32(bufW(s), row, half, a, b);
-                widen16<DT>(a, lo0, hi0);
-                widen16<DT>(b, lo1, hi1);
-                const uint32_t v[16] = {lo0.x, lo0.y, lo0.z, lo0.w, hi0.x, hi0.y, hi0.z, hi0.w,
-                                        lo1.x, lo1.y, lo1.z, lo1.w, hi1.x, hi1.y, hi1.z, hi1.w};
+                // this thread's kPartBytes symbols of the slab, widened exactly
+                uint32_t v[kPartCols];
+#pragma unroll
+                for (uint32_t j = 0; j < kPartBytes / 16; ++j) {
+                    uint4 lo, hi;
+                    widen16<DT>(lds_sym16(bufW(s), row, part * (kPartBytes / 16) + j), lo, hi);
+                    v[8 * j + 0] = lo.x, v[8 * j + 1] = lo.y, v[8 * j + 2] = lo.z, v[8 * j + 3] = lo.w;
+                    v[8 * j + 4] = hi.x, v[8 * j + 5] = hi.y, v[8 * j + 6] = hi.z, v[8 * j + 7] = hi.w;
+                }
                 // the previous slab's tensor-memory store has had this slab's work to complete
                 if (it > 0) {
                     tmem_st_wait();
@@ -318,14 +345,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
                     __syncwarp();
                     if (lane == 0) mbar_arrive(full0 + 8 * ((g - 1) % kStages));
                 }
-                tmem_st16(tmem_a + lane_base + s * kACols + half * (kACols / 2), v);
+                const uint32_t ta = tmem_a + lane_base + s * kACols + part * kPartCols;
+                if constexpr (kPartCols == 16) {
+                    tmem_st16(ta, v);
+                } else {
+                    tmem_st8(ta, v);
+                }
             }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (!ok) break;
             if (lane == 0) mbar_arrive(full0 + 8 * ((g - 1) % kStages));
-            // epilogue: thread (w, l) holds weight row 32 (w % 4) + l, tokens 128 (w / 4) .. + 127
+            // epilogue: thread (w, l) holds weight row 32 (w % 4) + l and part w / 4 of the tile's tokens
             if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(done, ti & 1u))) {
                 ok = false;
                 break;
@@ -334,10 +366,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
             const uint32_t r = n0 + row;
             const float sc = __ldg(J.scales + r);
 #pragma unroll 1
-            for (uint32_t c = 0; c < kAccCols / 2; c += 32) {
+            for (uint32_t c = 0; c < kAccCols / kParts; c += 32) {
                 uint32_t acc[32];
-                tmem_ld32(tmem + lane_base + half * (kAccCols / 2) + c, acc);
-                const uint32_t t0 = m0 + half * (kAccCols / 2) + c;
+                tmem_ld32(tmem + lane_base + part * (kAccCols / kParts) + c, acc);
+                const uint32_t t0 = m0 + part * (kAccCols / kParts) + c;
 #pragma unroll
                 for (uint32_t j = 0; j < 32; ++j)
                     if (t0 + j < P.tokens) J.y[(size_t)(t0 + j) * J.rows + r] = __fmul_rn(__uint_as_float(acc[j]), sc);
@@ -369,7 +401,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
                 tc_fence_after();
 #pragma unroll
                 for (uint32_t kk = 0; kk < kTileK / kMmaK; ++kk)
-                    tc_mma_ts(tmem, tmem_a + s * kACols + kk * (kMmaK / 2), tile_desc(bufB(s), kk), (it | kk) != 0u);
+                    tc_mma_ts(tmem, tmem_a + s * kACols + kk * (kMmaK / 2), tile_desc(bufB(s), kk), S::kInstrDesc,
+                              (it | kk) != 0u);
                 tc_commit(empty0 + 8 * s);
             }
             tc_commit(done);  // completes when every MMA issued above has
@@ -399,7 +432,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
                 // token tile: two boxes of 128 tokens (x = k0, a multiple of 64 elements; rows past
                 // the last token read as zeros); symbol tile: 128 rows x 64 bytes (x = k0 bytes)
 #pragma unroll
-                for (uint32_t h = 0; h < 2; ++h)
+                for (uint32_t h = 0; h < kTileT / kBoxT; ++h)
                     asm volatile(
                         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
                         " [%0], [%1, {%2, %3}], [%4];" ::"r"(bufB(s) + h * kBoxT * kRowBytes),
@@ -437,6 +470,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
 // give up; it then arrives on "done" itself, the producers pass it (or give up
 // on it) and the block returns with EQ_DEV_TIMEOUT set and its TMEM freed.
 __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_wait_timeout_kernel(int32_t *status) {
+    constexpr uint32_t kStages = GemmShape<256>::kStages;
     __shared__ __align__(8) uint64_t load_s[kStages], full_s[kStages], empty_s[kStages], done_s;
     __shared__ uint32_t tmem_base_s;
     const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
@@ -495,7 +529,7 @@ __global__ void eq_gemm_outliers_kernel(const uint32_t *rec, uint32_t n_out, con
     atomicAdd(y + (size_t)tok * rows + r, __fmul_rn(w, xv));
 }
 
-bool g_gemm_attr_set[128][2];
+bool g_gemm_attr_set[128][2][2];  // device, weight type, token-tile width
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against the driver library).
@@ -581,7 +615,12 @@ int gemm_launch(const eq_model *m, const GemmRequest *req, uint32_t n, uint32_t 
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
         return EQ_ERR_CUDA;
     if (m->sm_limit && m->sm_limit < (uint32_t)sms) sms = (int)m->sm_limit;
-    const uint32_t t_tiles = (tokens + kTileT - 1) / kTileT;
+    // short inputs (<= 128 tokens) take the 128-token tile: each weight tile is read once and the
+    // MMA does no work on absent tokens
+    const bool narrow = tokens <= kNarrowTokens;
+    const uint32_t tile_t = narrow ? 128u : 256u;
+    const size_t smem = narrow ? GemmShape<128>::kSmem : GemmShape<256>::kSmem;
+    const uint32_t t_tiles = (tokens + tile_t - 1) / tile_t;
     for (int dt = EQ_INT8; dt <= EQ_E4M3; ++dt) {
         std::vector<uint32_t> order;
         for (uint32_t i = 0; i < n; ++i) {
@@ -591,7 +630,8 @@ int gemm_launch(const eq_model *m, const GemmRequest *req, uint32_t n, uint32_t 
         std::stable_sort(order.begin(), order.end(), [&](uint32_t a, uint32_t b) {
             return m->mats[req[a].matrix].info.cols > m->mats[req[b].matrix].info.cols;
         });
-        auto fn = dt == EQ_INT8 ? eq_gemm_symbols_kernel<EQ_INT8> : eq_gemm_symbols_kernel<EQ_E4M3>;
+        auto fn = dt == EQ_INT8 ? (narrow ? eq_gemm_symbols_kernel<EQ_INT8, 128> : eq_gemm_symbols_kernel<EQ_INT8, 256>)
+                                : (narrow ? eq_gemm_symbols_kernel<EQ_E4M3, 128> : eq_gemm_symbols_kernel<EQ_E4M3, 256>);
         for (size_t at = 0; at < order.size(); at += kMaxGemmJobs) {
             GemmParams P{};
             P.status = d_status;
@@ -614,15 +654,15 @@ int gemm_launch(const eq_model *m, const GemmRequest *req, uint32_t n, uint32_t 
             }
             if (tiles > 0xFFFFFFFFull - (uint64_t)sms) return EQ_ERR_UNSUPPORTED;
             P.total_tiles = (uint32_t)tiles;
-            bool &attr = g_gemm_attr_set[dev][dt - 1];
+            bool &attr = g_gemm_attr_set[dev][dt - 1][narrow ? 0 : 1];
             if (!attr) {
                 if (cudaFuncSetAttribute(reinterpret_cast<const void *>(fn),
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem) != cudaSuccess)
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
                     return EQ_ERR_CUDA;
                 attr = true;
             }
             const uint32_t grid = std::min<uint64_t>(tiles, (uint64_t)sms);
-            fn<<<grid, kGemmThreads, kGemmSmem, s>>>(P);
+            fn<<<grid, kGemmThreads, smem, s>>>(P);
             if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
         }
     }

@@ -194,12 +194,13 @@ def _block_mats():
             W.random_e4m3_matrix(34, 256, 256, alpha=1.0, layer=0, index=4)]
 
 
+@pytest.mark.parametrize("tokens", [700, 100])
 @pytest.mark.parametrize("sms", [0, 1, 3])
-def test_gemm_block_one_hot_bit_exact(eqw, orc, sms):
+def test_gemm_block_one_hot_bit_exact(eqw, orc, sms, tokens):
     """One persistent launch per weight type over every tile of the layer; sms = 1 or 3 makes each
-    CTA run many tiles of different matrices (stage ring and barrier phases carried across tiles)."""
+    CTA run many tiles of different matrices (stage ring and barrier phases carried across tiles).
+    700 tokens: three 256-token tiles, the last one ragged; 100: one ragged 128-token tile."""
     mats = _block_mats()
-    tokens = 700                                     # 3 token tiles, the last one ragged
     model = _open(eqw, mats)
     model.set_sm_limit(sms)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -216,9 +217,9 @@ def test_gemm_block_one_hot_bit_exact(eqw, orc, sms):
     model.close()
 
 
-def test_gemm_block_random_tokens_within_bound(eqw, orc):
+@pytest.mark.parametrize("tokens", [300, 128])
+def test_gemm_block_random_tokens_within_bound(eqw, orc, tokens):
     mats = _block_mats()
-    tokens = 300
     model = _open(eqw, mats)
     model.set_sm_limit(2)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -235,12 +236,12 @@ def test_gemm_block_random_tokens_within_bound(eqw, orc):
     model.close()
 
 
-def test_gemm_block_llama70b_layer_sampled_rows(eqw, orc):
-    """A full 70B-shape layer (7 matrices, 1312 tiles at 512 tokens) in one launch: every output equals
-    the single-matrix launch's bit for bit (same tile arithmetic), and sampled weight rows of every
-    matrix are within the fp32 bound of the oracle."""
+@pytest.mark.parametrize("tokens", [512, 96])
+def test_gemm_block_llama70b_layer_sampled_rows(eqw, orc, tokens):
+    """A full 70B-shape layer (7 matrices: 1312 tiles of 256 tokens at 512 tokens, 448 tiles of 128
+    tokens at 96) in one launch: every output equals the single-matrix launch's bit for bit (same tile
+    arithmetic), and sampled weight rows of every matrix are within the fp32 bound of the oracle."""
     mats = W.llama70b_int8_layer(0)
-    tokens = 512
     model = _open(eqw, mats)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     syms = [torch.empty(m.rows * m.cols, dtype=torch.uint8, device="cuda") for m in mats]
