@@ -230,6 +230,40 @@ class DeviceMatrix:
         self.out_row = self.out_col = self.out_val = None
 
 
+def oracle_check_sampled_chunks(blob: np.ndarray, mats, threads: int) -> int:
+    """Check of the device-encoded container, outside any timed region: the
+    oracle decodes the first, the last and one seeded random chunk of every
+    matrix of every layer, and each must give the generated symbols back.
+    Returns the number of chunks checked; raises on any mismatch."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    parsed = oracle.parse_container(blob)
+    if len(parsed["matrices"]) != len(mats):
+        raise RuntimeError("device-encoded container: wrong matrix count")
+    rng = np.random.default_rng(11)
+    jobs = []
+    for mi, pm in enumerate(parsed["matrices"]):
+        nc = int(pm["n_chunks"])
+        for k in sorted({0, nc - 1, int(rng.integers(nc))}):
+            jobs.append((mi, k))
+
+    def one(job):
+        mi, k = job
+        pm, m = parsed["matrices"][mi], mats[mi]
+        first = k * oracle.CHUNK_SYMS
+        cnt = min(oracle.CHUNK_SYMS, m.n - first)
+        sym = oracle._decode_record(parsed["blob"], int(pm["chunk_offsets"][k]), int(pm["chunk_offsets"][k + 1]),
+                                    cnt, pm.get("codec", oracle.CODEC_RANS))
+        return bool(np.array_equal(sym, np.ascontiguousarray(m.symbols).reshape(-1)[first:first + cnt]))
+
+    with ThreadPoolExecutor(threads) as ex:
+        ok = list(ex.map(one, jobs))
+    if not all(ok):
+        bad = [jobs[i] for i, v in enumerate(ok) if not v][:4]
+        raise RuntimeError(f"device-encoded container: the oracle's decode differs at (matrix, chunk) {bad}")
+    return len(jobs)
+
+
 def build_blob(distinct: int, threads: int, device) -> tuple[np.ndarray, dict]:
     """Generate `distinct` seeded 70B-shape Int8 layers (host) and encode them on
     the GPU with eq_encode_device; layer 0 is also encoded on the host, timed,
@@ -250,6 +284,7 @@ def build_blob(distinct: int, threads: int, device) -> tuple[np.ndarray, dict]:
     t3 = time.time()
     blob = d_blob.cpu().numpy()
     del d_blob, dmats
+    n_checked = oracle_check_sampled_chunks(blob, mats, threads)
     n_syms = sum(m.n for m in mats)
     layer0 = [m for m in mats if m.layer == 0]
     t4 = time.time()
@@ -264,9 +299,10 @@ def build_blob(distinct: int, threads: int, device) -> tuple[np.ndarray, dict]:
           file=sys.stderr, flush=True)
     enc = {"device_gsym_s": round(n_syms / (t3 - t2) / 1e9, 3), "device_s": round(t3 - t2, 2),
            "symbols": n_syms, "host_gsym_s": round(n0 / (t5 - t4) / 1e9, 3), "host_threads": threads,
-           "bytes_equal_host": same,
+           "bytes_equal_host": same, "oracle_checked_chunks": n_checked,
            "note": "eq_encode_device on symbols already in HBM (wall clock, it synchronises); host = eq_encode_host "
-                   "of layer 0 on all cores"}
+                   "of layer 0 on all cores; oracle_checked_chunks: first, last and one random chunk of every "
+                   "matrix of every layer decoded by the oracle and equal to the generated symbols"}
     if not same:
         raise RuntimeError("device and host encoders disagree")
     return blob, enc
