@@ -380,7 +380,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
         }
     } else if (warp == kProducerWarps && lane == 0) {
         // ---- MMA issuer ----
-        uint32_t ti = 0, n_done = 0;
+        // One lane issues every MMA, so its loop is kept short: one wait per slab ("full": the
+        // producers arrive only after they have seen the slab's copies land on "load"), the stage
+        // and phase kept incrementally, and the descriptors advanced by adding to their address
+        // field (16-byte units, well below its 14-bit limit for any shared-memory address).
+        const uint64_t desc0 = tile_desc(bufB(0), 0);
+        uint32_t ti = 0, n_done = 0, s = 0, ph = 0;  // stage and phase of the next slab
         for (uint32_t tile = blockIdx.x, jb = 0; tile < P.total_tiles; tile += gridDim.x, ++ti) {
             while (jb + 1 < P.n_jobs && tile >= P.jobs[jb + 1].first_tile) ++jb;
             const uint32_t n_slabs = P.jobs[jb].cols / kTileK;
@@ -390,20 +395,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
                 break;
             }
             tc_fence_after();
-            for (uint32_t it = 0; it < n_slabs; ++it, ++g) {
-                const uint32_t s = g % kStages;
-                // the producers' weights, and the token tile the loader's copy brought in
-                if (abort_s || !mbar_wait_bounded(full0 + 8 * s, (g / kStages) & 1u) ||
-                    !mbar_wait_bounded(load0 + 8 * s, (g / kStages) & 1u)) {
+            for (uint32_t it = 0; it < n_slabs; ++it) {
+                if (!mbar_wait_bounded(full0 + 8 * s, ph)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint64_t db = desc0 + ((s * kStageBytes) >> 4);
+                const uint32_t ta = tmem_a + s * kACols;
 #pragma unroll
-                for (uint32_t kk = 0; kk < kTileK / kMmaK; ++kk)
-                    tc_mma_ts(tmem, tmem_a + s * kACols + kk * (kMmaK / 2), tile_desc(bufB(s), kk), S::kInstrDesc,
-                              (it | kk) != 0u);
+                for (uint32_t kk = 0; kk < kTileK / kMmaK; ++kk)  // K step kk: +32 bytes, 2 descriptor units
+                    tc_mma_ts(tmem, ta + kk * (kMmaK / 2), db + 2u * kk, S::kInstrDesc, (it | kk) != 0u);
                 tc_commit(empty0 + 8 * s);
+                if (++s == kStages) {
+                    s = 0;
+                    ph ^= 1u;
+                }
             }
             tc_commit(done);  // completes when every MMA issued above has
             ++n_done;
