@@ -201,6 +201,19 @@ __device__ __forceinline__ void widen16(uint4 b, uint4 &lo, uint4 &hi) {
     hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
+// Non-blocking check that the phase with parity `parity` has completed (acquire).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -386,6 +399,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
         // field (16-byte units, well below its 14-bit limit for any shared-memory address).
         const uint64_t desc0 = tile_desc(bufB(0), 0);
         uint32_t ti = 0, n_done = 0, s = 0, ph = 0;  // stage and phase of the next slab
+        bool ready = false;  // the next slab's "full" phase was already seen complete
         for (uint32_t tile = blockIdx.x, jb = 0; tile < P.total_tiles; tile += gridDim.x, ++ti) {
             while (jb + 1 < P.n_jobs && tile >= P.jobs[jb + 1].first_tile) ++jb;
             const uint32_t n_slabs = P.jobs[jb].cols / kTileK;
@@ -396,7 +410,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
             }
             tc_fence_after();
             for (uint32_t it = 0; it < n_slabs; ++it) {
-                if (!mbar_wait_bounded(full0 + 8 * s, ph)) {
+                if (!ready && !mbar_wait_bounded(full0 + 8 * s, ph)) {
                     ok = false;
                     break;
                 }
@@ -406,11 +420,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
 #pragma unroll
                 for (uint32_t kk = 0; kk < kTileK / kMmaK; ++kk)  // K step kk: +32 bytes, 2 descriptor units
                     tc_mma_ts(tmem, ta + kk * (kMmaK / 2), db + 2u * kk, S::kInstrDesc, (it | kk) != 0u);
+                const uint32_t s_next = s + 1 == kStages ? 0u : s + 1, ph_next = s + 1 == kStages ? ph ^ 1u : ph;
+                // peek (non-blocking) at the next slab's barrier while this slab's commit goes out
+                ready = mbar_test(full0 + 8 * s_next, ph_next);
                 tc_commit(empty0 + 8 * s);
-                if (++s == kStages) {
-                    s = 0;
-                    ph ^= 1u;
-                }
+                s = s_next;
+                ph = ph_next;
             }
             tc_commit(done);  // completes when every MMA issued above has
             ++n_done;
