@@ -321,6 +321,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
     const uint32_t tmem_a = tmem + kAccCols;  // weight stages follow the accumulator
     bool ok = true;
     uint32_t g = 0;  // slabs so far in this CTA: stage g % kStages, phase g / kStages
+    uint32_t st = 0, sph = 0, st_prev = 0;  // g % kStages, (g / kStages) & 1 and the previous slab's stage
 
     if (warp < kProducerWarps) {
         // ---- producers: symbols (shared) -> bf16 -> tensor memory; the tile's epilogue ----
@@ -336,8 +337,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
             const uint32_t n0 = (local / P.t_tiles) * kTileN, m0 = (local % P.t_tiles) * kTileT;
             const uint32_t n_slabs = J.cols / kTileK;
             for (uint32_t it = 0; it < n_slabs; ++it, ++g) {
-                const uint32_t s = g % kStages;
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(load0 + 8 * s, (g / kStages) & 1u))) {
+                const uint32_t s = st;
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(load0 + 8 * s, sph))) {
                     ok = false;
                     break;
                 }
@@ -356,7 +357,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(full0 + 8 * ((g - 1) % kStages));
+                    if (lane == 0) mbar_arrive(full0 + 8 * st_prev);
                 }
                 const uint32_t ta = tmem_a + lane_base + s * kACols + part * kPartCols;
                 if constexpr (kPartCols == 16) {
@@ -364,12 +365,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
                 } else {
                     tmem_st8(ta, v);
                 }
+                st_prev = st;
+                if (++st == kStages) {
+                    st = 0;
+                    sph ^= 1u;
+                }
             }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (!ok) break;
-            if (lane == 0) mbar_arrive(full0 + 8 * ((g - 1) % kStages));
+            if (lane == 0) mbar_arrive(full0 + 8 * st_prev);
             // epilogue: thread (w, l) holds weight row 32 (w % 4) + l and part w / 4 of the tile's tokens
             if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(done, ti & 1u))) {
                 ok = false;
@@ -444,9 +450,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
             const uint64_t map_x = reinterpret_cast<uint64_t>(&J.tmap_x);
             const uint64_t map_w = reinterpret_cast<uint64_t>(&J.tmap_w);
             for (uint32_t it = 0; it < n_slabs; ++it, ++g) {
-                const uint32_t s = g % kStages;
-                // stage s last held slab g - kStages: its MMAs (and so its producers) are done
-                if (g >= kStages && (abort_s || !mbar_wait_bounded(empty0 + 8 * s, ((g - kStages) / kStages) & 1u))) {
+                const uint32_t s = st;
+                // stage s last held slab g - kStages (phase sph ^ 1): its MMAs (and so its producers) are done
+                if (g >= kStages && (abort_s || !mbar_wait_bounded(empty0 + 8 * s, sph ^ 1u))) {
                     ok = false;
                     break;
                 }
@@ -465,6 +471,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
                     " [%0], [%1, {%2, %3}], [%4];" ::"r"(bufW(s)), "l"(map_w), "r"(it * kTileK), "r"(n0),
                     "r"(load0 + 8 * s)
                     : "memory");
+                if (++st == kStages) {
+                    st = 0;
+                    sph ^= 1u;
+                }
             }
         }
         // no copy may still be writing shared memory when the block exits: wait (bounded) for
