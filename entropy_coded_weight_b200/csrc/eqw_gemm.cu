@@ -495,6 +495,316 @@ __global__ void __launch_bounds__(kGemmThreads, 1) eq_gemm_symbols_kernel(const 
     }
 }
 
+// ---- 2-SM variant (cta_group::2) -----------------------------------------------------
+// For 256-token tiles over matrices whose rows are a multiple of 256, a
+// cluster of two CTAs (one per SM of a pair) computes 256 weight rows x 256
+// tokens with tcgen05.mma.cta_group::2 (M = 256): CTA r of the pair holds
+// weight rows 128 r .. + 127 of the tile in its tensor memory (A, widened by
+// its own producers), tokens 128 r .. + 127 of the tile in its shared memory
+// (half of B), and the accumulator of its 128 weight rows for all 256 tokens.
+// Each SM thus keeps half the token tile of the one-SM kernel per slab (16
+// KB): 8 stages fit where 5 did, and the one lane that issues the MMAs (in CTA
+// 0) issues half as many per FLOP.
+//   loader     (each CTA) after its own "empty" (arrived by CTA 0's commit,
+//              multicast to both CTAs), its token half (one 128-token box) and
+//              its 128-row symbol tile, on its own "load" barrier
+//   producers  (each CTA) widen as in the one-SM kernel, then arrive on CTA
+//              0's "full" barrier (16 arrivals: 8 warps in each CTA)
+//   MMA lane   (CTA 0) waits for "full", issues the slab's 4 MMAs and commits
+//              them to "empty" in both CTAs; after a tile, to "done" in both
+//   epilogue   (each CTA) its 128 rows x 256 tokens, then arrives on CTA 0's
+//              "acc_free" (16 arrivals)
+// Both CTAs take part in the same two cluster barriers (after set-up, before
+// releasing the tensor memory); every other wait is bounded.
+constexpr uint32_t kPairStages = 8;
+constexpr uint32_t kPairXBytes = kBoxT * kTileK * 2;          // this CTA's 128 tokens of a slab, 16 KB
+constexpr uint32_t kPairStageBytes = kPairXBytes + kWBytes;    // + its 128-row symbol tile
+constexpr uint32_t kPairAcc = 256;                             // accumulator columns (tokens)
+constexpr size_t kPairSmem = kPairStages * kPairStageBytes + 1024;
+constexpr uint32_t kPairInstrDesc = (1u << 4) | (1u << 7) | (1u << 10)  // fp32 D, bf16 A and B, K-major
+                                  | ((kPairAcc >> 3) << 17)              // N / 8
+                                  | ((2 * kTileN >> 4) << 24);           // M / 16, M = 256 over the pair
+static_assert(kPairAcc + kPairStages * kACols <= kTmemAlloc, "tensor memory columns");
+static_assert(kPairSmem + 1024 <= 227u * 1024u, "shared memory per block");
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Every thread of both CTAs.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// The shared::cluster address of the variable at `local` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+
+// Arrive on a barrier given by its shared::cluster address (possibly the other
+// CTA's), with the default semantics.  What it publishes is the arriving
+// warp's tensor-memory stores (ordered by tcgen05.wait::st and
+// tcgen05.fence::before_thread_sync) and reads of the accumulator, not data
+// in memory, so no cluster-wide release is needed.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_poll_cluster(uint32_t bar, uint32_t parity, bool blocking) {
+    uint32_t ok;
+    if (blocking)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on a local barrier that threads of the other CTA (or CTA 0's
+// commits) arrive on.
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity) {
+    if (mbar_poll_cluster(bar, parity, true)) return true;
+    const long long t0 = clock64();
+    for (;;) {
+        if (mbar_poll_cluster(bar, parity, true)) return true;
+        if (clock64() - t0 > kWaitCycles) return false;
+    }
+}
+
+__device__ __forceinline__ void tc_mma_ts_pair(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "r"(tmem_a), "l"(db), "r"(kPairInstrDesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrives (when every MMA issued so far by this thread has completed) on the
+// barrier at shared-memory offset `bar` in both CTAs of the pair.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .b16 m;\n\t"
+        "mov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}"
+        ::"r"(bar)
+        : "memory");
+}
+
+template <int DT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    eq_gemm_symbols_pair_kernel(const __grid_constant__ GemmParams P) {
+    constexpr uint32_t kStages = kPairStages, kStageBytes = kPairStageBytes;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t load_s[kStages], full_s[kStages], empty_s[kStages], done_s, acc_free_s;
+    __shared__ uint32_t tmem_base_s;
+    __shared__ volatile uint32_t abort_s;
+    const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
+    const uint32_t rank = cluster_rank();
+    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    auto bufB = [&](uint32_t st) { return base + st * kStageBytes; };                // this CTA's token half
+    auto bufW = [&](uint32_t st) { return base + st * kStageBytes + kPairXBytes; };  // its symbol tile
+    const uint32_t load0 = smem_u32(&load_s[0]), full0 = smem_u32(&full_s[0]), empty0 = smem_u32(&empty_s[0]);
+    const uint32_t done = smem_u32(&done_s), acc_free = smem_u32(&acc_free_s);
+
+    if (warp == 0) {  // the same warp in both CTAs allocates, collectively
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(&tmem_base_s)), "r"(kTmemAlloc) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        for (uint32_t st = 0; st < kStages; ++st) {
+            mbar_init(load0 + 8 * st, 1);                   // this CTA's expect_tx arrival + its copies
+            mbar_init(full0 + 8 * st, 2 * kProducerWarps);  // (CTA 0) the producer warps of both CTAs
+            mbar_init(empty0 + 8 * st, 1);                  // CTA 0's commit
+        }
+        mbar_init(done, 1);
+        mbar_init(acc_free, 2 * kProducerWarps);
+        fence_mbar_init();
+        abort_s = 0;
+    }
+    tc_fence_before();
+    cluster_sync_all();  // both CTAs' barriers initialised and tensor memory allocated
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_s;
+    const uint32_t tmem_a = tmem + kPairAcc;
+    const uint32_t n_clusters = gridDim.x / 2, cl = blockIdx.x / 2;
+    bool ok = true;
+
+    if (warp < kProducerWarps) {
+        // ---- producers (both CTAs) ----
+        const uint32_t quarter = warp & 3u, part = warp >> 2;
+        const uint32_t row = quarter * 32u + lane;
+        const uint32_t lane_base = (quarter * 32u) << 16;
+        const uint32_t full_c0 = cluster_addr(full0, 0), acc_free_c0 = cluster_addr(acc_free, 0);
+        uint32_t st = 0, sph = 0, st_prev = 0, ti = 0, jb = 0;
+        for (uint32_t tile = cl; tile < P.total_tiles; tile += n_clusters, ++ti) {
+            if (__any_sync(0xFFFFFFFFu, abort_s != 0u)) break;
+            while (jb + 1 < P.n_jobs && tile >= P.jobs[jb + 1].first_tile) ++jb;
+            const GemmJob &J = P.jobs[jb];
+            const uint32_t local = tile - J.first_tile;
+            const uint32_t n0 = (local / P.t_tiles) * (2 * kTileN) + rank * kTileN, m0 = (local % P.t_tiles) * kPairAcc;
+            const uint32_t n_slabs = J.cols / kTileK;
+            for (uint32_t it = 0; it < n_slabs; ++it) {
+                const uint32_t s = st;
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(load0 + 8 * s, sph))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t v[kPartCols];
+#pragma unroll
+                for (uint32_t j = 0; j < kPartBytes / 16; ++j) {
+                    uint4 lo, hi;
+                    widen16<DT>(lds_sym16(bufW(s), row, part * (kPartBytes / 16) + j), lo, hi);
+                    v[8 * j + 0] = lo.x, v[8 * j + 1] = lo.y, v[8 * j + 2] = lo.z, v[8 * j + 3] = lo.w;
+                    v[8 * j + 4] = hi.x, v[8 * j + 5] = hi.y, v[8 * j + 6] = hi.z, v[8 * j + 7] = hi.w;
+                }
+                if (it > 0) {  // the previous slab's store has completed: tell CTA 0's MMA lane
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(full_c0 + 8 * st_prev);
+                }
+                const uint32_t ta = tmem_a + lane_base + s * kACols + part * kPartCols;
+                if constexpr (kPartCols == 16) {
+                    tmem_st16(ta, v);
+                } else {
+                    tmem_st8(ta, v);
+                }
+                st_prev = st;
+                if (++st == kStages) {
+                    st = 0;
+                    sph ^= 1u;
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (!ok) break;
+            if (lane == 0) mbar_arrive_cluster(full_c0 + 8 * st_prev);
+            // epilogue: this CTA's 128 weight rows, part w / 4 of the tile's 256 tokens
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_cluster(done, ti & 1u))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t r = n0 + row;
+            const float sc = __ldg(J.scales + r);
+#pragma unroll 1
+            for (uint32_t c = 0; c < kPairAcc / kParts; c += 32) {
+                uint32_t acc[32];
+                tmem_ld32(tmem + lane_base + part * (kPairAcc / kParts) + c, acc);
+                const uint32_t t0 = m0 + part * (kPairAcc / kParts) + c;
+#pragma unroll
+                for (uint32_t j = 0; j < 32; ++j)
+                    if (t0 + j < P.tokens) J.y[(size_t)(t0 + j) * J.rows + r] = __fmul_rn(__uint_as_float(acc[j]), sc);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_free_c0);
+        }
+    } else if (warp == kProducerWarps && lane == 0 && rank == 0) {
+        // ---- MMA lane (CTA 0) ----
+        const uint64_t desc0 = tile_desc(bufB(0), 0);
+        uint32_t ti = 0, n_done = 0, s = 0, ph = 0;
+        bool ready = false;
+        for (uint32_t tile = cl, jb = 0; tile < P.total_tiles; tile += n_clusters, ++ti) {
+            while (jb + 1 < P.n_jobs && tile >= P.jobs[jb + 1].first_tile) ++jb;
+            const uint32_t n_slabs = P.jobs[jb].cols / kTileK;
+            if (abort_s || (ti > 0 && !mbar_wait_cluster(acc_free, (ti - 1) & 1u))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            for (uint32_t it = 0; it < n_slabs; ++it) {
+                if (!ready && !mbar_wait_cluster(full0 + 8 * s, ph)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t db = desc0 + ((s * kStageBytes) >> 4);
+                const uint32_t ta = tmem_a + s * kACols;
+#pragma unroll
+                for (uint32_t kk = 0; kk < kTileK / kMmaK; ++kk)
+                    tc_mma_ts_pair(tmem, ta + kk * (kMmaK / 2), db + 2u * kk, (it | kk) != 0u);
+                const uint32_t s_next = s + 1 == kStages ? 0u : s + 1, ph_next = s + 1 == kStages ? ph ^ 1u : ph;
+                ready = mbar_poll_cluster(full0 + 8 * s_next, ph_next, false);
+                tc_commit_pair(empty0 + 8 * s);
+                s = s_next;
+                ph = ph_next;
+            }
+            tc_commit_pair(done);
+            ++n_done;
+            if (!ok) break;
+        }
+        if (n_done > 0 && !mbar_wait_cluster(done, (n_done - 1) & 1u)) ok = false;
+    } else if (warp == kProducerWarps + 1 && lane == 0) {
+        // ---- loader (both CTAs) ----
+        uint32_t st = 0, sph = 0, g = 0;
+        for (uint32_t tile = cl, jb = 0; tile < P.total_tiles && ok; tile += n_clusters) {
+            while (jb + 1 < P.n_jobs && tile >= P.jobs[jb + 1].first_tile) ++jb;
+            const GemmJob &J = P.jobs[jb];
+            const uint32_t local = tile - J.first_tile;
+            const uint32_t n0 = (local / P.t_tiles) * (2 * kTileN) + rank * kTileN;
+            const uint32_t m0 = (local % P.t_tiles) * kPairAcc + rank * kBoxT;  // this CTA's token half
+            const uint32_t n_slabs = J.cols / kTileK;
+            const uint64_t map_x = reinterpret_cast<uint64_t>(&J.tmap_x);
+            const uint64_t map_w = reinterpret_cast<uint64_t>(&J.tmap_w);
+            for (uint32_t it = 0; it < n_slabs; ++it, ++g) {
+                const uint32_t s = st;
+                if (g >= kStages && (abort_s || !mbar_wait_cluster(empty0 + 8 * s, sph ^ 1u))) {
+                    ok = false;
+                    break;
+                }
+                mbar_expect_tx(load0 + 8 * s, kStageBytes);
+                asm volatile(
+                    "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                    " [%0], [%1, {%2, %3}], [%4];" ::"r"(bufB(s)), "l"(map_x), "r"(it * kTileK), "r"(m0),
+                    "r"(load0 + 8 * s)
+                    : "memory");
+                asm volatile(
+                    "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                    " [%0], [%1, {%2, %3}], [%4];" ::"r"(bufW(s)), "l"(map_w), "r"(it * kTileK), "r"(n0),
+                    "r"(load0 + 8 * s)
+                    : "memory");
+                if (++st == kStages) {
+                    st = 0;
+                    sph ^= 1u;
+                }
+            }
+        }
+        for (uint32_t k = g > kStages ? g - kStages : 0; k < g; ++k)
+            if (!mbar_wait_bounded(load0 + 8 * (k % kStages), (k / kStages) & 1u)) ok = false;
+    }
+    if (!ok) {
+        abort_s = 1;
+        atomicOr(P.status, EQ_DEV_TIMEOUT);
+    }
+    tc_fence_before();
+    cluster_sync_all();  // no MMA of CTA 0 reads this CTA's memory any more
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemAlloc)
+                     : "memory");
+    }
+}
+
 // Failure-path check of the GEMM's waits: the GEMM's own set-up (TMEM
 // allocation, "load" / "full" / "empty" / "done" barriers with their arrival
 // counts, the GEMM's block size) and exit path (status flag, TMEM release),
@@ -561,7 +871,7 @@ __global__ void eq_gemm_outliers_kernel(const uint32_t *rec, uint32_t n_out, con
     atomicAdd(y + (size_t)tok * rows + r, __fmul_rn(w, xv));
 }
 
-bool g_gemm_attr_set[128][2][2];  // device, weight type, token-tile width
+bool g_gemm_attr_set[128][2][3];  // device, weight type, kernel (128-token, 256-token, 2-SM)
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against the driver library).
@@ -665,12 +975,17 @@ int gemm_launch(const eq_model *m, const GemmRequest *req, uint32_t n, uint32_t 
         auto fn = dt == EQ_INT8 ? (narrow ? eq_gemm_symbols_kernel<EQ_INT8, 128> : eq_gemm_symbols_kernel<EQ_INT8, 256>)
                                 : (narrow ? eq_gemm_symbols_kernel<EQ_E4M3, 128> : eq_gemm_symbols_kernel<EQ_E4M3, 256>);
         for (size_t at = 0; at < order.size(); at += kMaxGemmJobs) {
+            const size_t end = std::min(order.size(), at + kMaxGemmJobs);
+            // the 2-SM kernel: 256-token tiles, every matrix a whole number of 256-row tiles
+            bool pair = !narrow && sms >= 2;
+            for (size_t k = at; k < end && pair; ++k) pair = m->mats[req[order[k]].matrix].info.rows % (2 * kTileN) == 0;
+            const uint32_t tile_rows = pair ? 2 * kTileN : kTileN;
             GemmParams P{};
             P.status = d_status;
             P.tokens = tokens;
             P.t_tiles = t_tiles;
             uint64_t tiles = 0;
-            for (size_t k = at; k < order.size() && k < at + kMaxGemmJobs; ++k) {
+            for (size_t k = at; k < end; ++k) {
                 const GemmRequest &q = req[order[k]];
                 const MatrixDesc &d = m->mats[q.matrix];
                 GemmJob &J = P.jobs[P.n_jobs++];
@@ -682,19 +997,29 @@ int gemm_launch(const eq_model *m, const GemmRequest *req, uint32_t n, uint32_t 
                 J.rows = d.info.rows;
                 J.cols = d.info.cols;
                 J.first_tile = (uint32_t)tiles;
-                tiles += (uint64_t)(d.info.rows / kTileN) * t_tiles;
+                tiles += (uint64_t)(d.info.rows / tile_rows) * t_tiles;
             }
             if (tiles > 0xFFFFFFFFull - (uint64_t)sms) return EQ_ERR_UNSUPPORTED;
             P.total_tiles = (uint32_t)tiles;
-            bool &attr = g_gemm_attr_set[dev][dt - 1][narrow ? 0 : 1];
+            const int variant = pair ? 2 : narrow ? 0 : 1;
+            const void *kfn = pair ? reinterpret_cast<const void *>(dt == EQ_INT8 ? eq_gemm_symbols_pair_kernel<EQ_INT8>
+                                                                                  : eq_gemm_symbols_pair_kernel<EQ_E4M3>)
+                                   : reinterpret_cast<const void *>(fn);
+            const size_t ksmem = pair ? kPairSmem : smem;
+            bool &attr = g_gemm_attr_set[dev][dt - 1][variant];
             if (!attr) {
-                if (cudaFuncSetAttribute(reinterpret_cast<const void *>(fn),
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+                if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ksmem) != cudaSuccess)
                     return EQ_ERR_CUDA;
                 attr = true;
             }
-            const uint32_t grid = std::min<uint64_t>(tiles, (uint64_t)sms);
-            fn<<<grid, kGemmThreads, smem, s>>>(P);
+            if (pair) {
+                const uint32_t clusters = (uint32_t)std::min<uint64_t>(tiles, (uint64_t)(sms / 2));
+                auto pfn = dt == EQ_INT8 ? eq_gemm_symbols_pair_kernel<EQ_INT8> : eq_gemm_symbols_pair_kernel<EQ_E4M3>;
+                pfn<<<2 * clusters, kGemmThreads, ksmem, s>>>(P);
+            } else {
+                const uint32_t grid = std::min<uint64_t>(tiles, (uint64_t)sms);
+                fn<<<grid, kGemmThreads, smem, s>>>(P);
+            }
             if (cudaGetLastError() != cudaSuccess) return EQ_ERR_CUDA;
         }
     }
