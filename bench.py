@@ -519,7 +519,7 @@ def bench_eqw(args, d: Dist) -> dict | None:
         huff = {"value": round(2.0 * n0 / (h_ms / 1e3) / 1e9, 2), "unit": UNIT, "launch_ms": round(h_ms, 4),
                 "bits_per_sym": round(8.0 * hb["read"] / n0, 4), "rans_bits_per_sym": round(8.0 * r_read / n0, 4),
                 "rans_launch_ms": round(launch_ms, 4),
-                "note": "layer 0 Huffman-coded (canonical codes <= 12 bits) and decoded by eq_decode_kernel's "
+                "note": "layer 0 Huffman-coded (canonical codes <= 12 bits) and decoded by the pair kernel's "
                         "Huffman instance, launches timed alone; bits/sym incl. tables and chunk index"}
         if not args.no_cpu_baseline and d.world == 1:
             # the multi-threaded CPU decode of the same chunks (the oracle's bit-serial Huffman decoder)
@@ -586,10 +586,13 @@ def bench_eqw(args, d: Dist) -> dict | None:
             raise RuntimeError(f"prefill status {int(pst.item())}")
         prefill = {"tokens": 1024, "decode_symbols_ms": round(dec_ms, 4), **by_tokens[1024],
                    "unit": "TFLOP/s", "bf16_peak": bf16_peak, "tokens_128": by_tokens[128],
-                   "tokens_4096": by_tokens[4096], "kernel": "eq_gemm_symbols_kernel (tcgen05)",
+                   "tokens_4096": by_tokens[4096],
+                   "kernel": "eq_gemm_symbols_pair_kernel (tcgen05.mma.cta_group::2) at 1024 and 4096 tokens, "
+                             "eq_gemm_symbols_kernel (cta_group::1, 128-token tiles) at 128",
                    "note": "layer 0: the 7 matrices' symbols decoded to bytes in one launch, then the 7 "
-                           "tcgen05 GEMMs in one persistent launch (eq_gemm_symbols_block; 256-token tiles, "
-                           "128-token tiles up to 128 tokens), bf16 tokens, fp32 out; frac of the measured "
+                           "tcgen05 GEMMs in one persistent launch (eq_gemm_symbols_block; 256-row x 256-token "
+                           "tiles over CTA pairs, 128-token tiles up to 128 tokens), bf16 tokens, fp32 out; "
+                           "frac of the measured "
                            "cuBLAS bf16 burst peak.  bf16_path: the same layer decoded to bf16 by "
                            "eq_decode_block, then one torch (cuBLAS) bf16 matmul per matrix, for comparison"}
         del syms, wbuf, wmats
