@@ -284,3 +284,52 @@ def test_gemm_block_argument_errors(eqw):
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     model.close()
+
+
+def _pair_mats():
+    """Every matrix a whole number of 256-row tiles: the layer takes the 2-SM (cta_group::2) kernel."""
+    return [W.random_int8_matrix(50, 256, 512, n_out=6, layer=0, index=0),
+            W.random_int8_matrix(51, 512, 64, layer=0, index=1),
+            W.random_int8_matrix(52, 256, 1024, h_bits=4.0, layer=0, index=2),
+            W.random_e4m3_matrix(53, 256, 192, alpha=1.0, layer=0, index=3),
+            W.random_e4m3_matrix(54, 512, 256, alpha=1.0, layer=0, index=4)]
+
+
+@pytest.mark.parametrize("sms", [0, 2, 5])
+def test_gemm_block_pair_kernel_one_hot_bit_exact(eqw, orc, sms):
+    """The 2-SM kernel: 700 tokens (three 256-token tiles, the last ragged), both weight types, K from 64
+    to 1024, super weights; sms = 2 or 5 leaves one or two CTA pairs, each running many tiles."""
+    mats = _pair_mats()
+    tokens = 700
+    model = _open(eqw, mats)
+    model.set_sm_limit(sms)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    syms = [torch.empty(m.rows * m.cols, dtype=torch.uint8, device="cuda") for m in mats]
+    model.decode_symbols_block(0, syms, status)
+    xs = [_one_hot(60 + i, tokens, m.cols) for i, m in enumerate(mats)]
+    ys = [torch.full((tokens, m.rows), float("nan"), dtype=torch.float32, device="cuda") for m in mats]
+    model.gemm_symbols_block(0, syms, [x.cuda() for x in xs], ys, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for i, (m, x, y) in enumerate(zip(mats, xs, ys)):
+        ref, _ = orc.gemm_symbols_exact(m, _bits(x))
+        assert np.array_equal(y.cpu().numpy().view(np.uint32), ref.astype(np.float32).view(np.uint32)), i
+    model.close()
+
+
+def test_gemm_block_pair_kernel_random_tokens_within_bound(eqw, orc):
+    mats = _pair_mats()
+    tokens = 300
+    model = _open(eqw, mats)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    syms = [torch.empty(m.rows * m.cols, dtype=torch.uint8, device="cuda") for m in mats]
+    model.decode_symbols_block(0, syms, status)
+    xs = [W.gemv_activation(13, i, tokens * m.cols).reshape(tokens, m.cols) for i, m in enumerate(mats)]
+    ys = [torch.empty(tokens, m.rows, dtype=torch.float32, device="cuda") for m in mats]
+    model.gemm_symbols_block(0, syms, [x.cuda() for x in xs], ys, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for m, x, y in zip(mats, xs, ys):
+        ref, mag = orc.gemm_symbols_exact(m, _bits(x))
+        _check_bound(y.cpu().numpy(), ref, mag, m.cols)
+    model.close()
