@@ -14,6 +14,14 @@
 // output in the epilogue and the (rare) super weights by a small second
 // kernel.
 //
+// Two kernels, chosen per launch by the host:
+//   eq_gemm_symbols_pair_kernel  (tcgen05.mma.cta_group::2, M = 256 over a pair
+//                                of CTAs on two SMs) for 256-token tiles when
+//                                every matrix has a multiple of 256 rows; it is
+//                                described where it is defined, below;
+//   eq_gemm_symbols_kernel       (cta_group::1, M = 128) otherwise, and with
+//                                128-token tiles for inputs of <= 128 tokens.
+//
 // Kernel eq_gemm_symbols_kernel: a persistent launch (one CTA per SM) over the
 // 128-row x 256-token output tiles of up to 8 matrices of one weight type (a
 // transformer block's projections in one launch; the matrix with the longest

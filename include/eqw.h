@@ -394,7 +394,9 @@ EQW_API int eq_gemm_symbols(const eq_model *m, uint32_t matrix, const void *d_sy
 
 /* The same for every matrix of `layer`, one persistent launch per weight type
  * (the tiles of all the layer's matrices shared out over the SMs, so that a
- * small matrix does not leave SMs idle): d_syms[i], d_xs[i], d_ys[i] (host
+ * small matrix does not leave SMs idle; 256-token tiles of matrices with a
+ * multiple of 256 rows run on pairs of SMs with tcgen05.mma.cta_group::2, and
+ * inputs of at most 128 tokens take 128-token tiles): d_syms[i], d_xs[i], d_ys[i] (host
  * arrays of `count` device pointers, count = the layer's matrix count) belong
  * to matrix i of the layer in directory order; all take `tokens` tokens.  Each
  * matrix has the requirements of eq_gemm_symbols; nothing is launched when one
