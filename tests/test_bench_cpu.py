@@ -65,3 +65,25 @@ def test_configs_table_row_formats_a_result_line():
     assert cells[5] == "30.8 %" and cells[6] == "yes" and cells[8] == "0.43"
     hot = dict(row, hot={"decoded_gb_s": 11.4, "gsym_s": 5.68, "hbm_frac": 0.002})
     assert "11.4 / 1751.8" in bench.configs_table_row(hot)
+
+
+def test_device_encoder_check_accepts_matching_container_and_catches_a_wrong_one():
+    """The bench's gate on the device-encoded model (run before any timing): the oracle decodes the
+    first, last and one random chunk of every matrix and compares them with the generated symbols."""
+    import entropy_coded_weight_b200 as E
+    from entropy_coded_weight_b200 import build
+    build.build()
+    mats = [W.random_int8_matrix(1, 300, 700, layer=0, index=0),
+            W.random_int8_matrix(2, 64, 64, layer=0, index=1),
+            W.random_e4m3_matrix(3, 200, 1000, alpha=1.0, layer=1, index=0)]
+    blob = E.encode_host(mats)
+    # first, last and one seeded random chunk of the 4-chunk matrix (3 distinct here), 1 of each other
+    assert bench.oracle_check_sampled_chunks(blob, mats, 2) == 3 + 1 + 1
+    wrong = list(mats)
+    wrong[1] = W.random_int8_matrix(9, 64, 64, layer=0, index=1)  # other symbols, same shape
+    try:
+        bench.oracle_check_sampled_chunks(blob, wrong, 2)
+    except RuntimeError as e:
+        assert "(1, 0)" in str(e)
+    else:
+        raise AssertionError("a container that does not decode to the generated symbols was accepted")
